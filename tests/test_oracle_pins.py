@@ -1,0 +1,335 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a different
+algorithm (brute force over all N joint scores), a closed form derived by
+hand, a special case that reduces to a library routine (numpy/scipy), or an
+invariant of the method.  The cases are chosen so that a plausible mistake
+(a dropped log-softmax, a transposed router matrix, a swapped (i, j) -> id
+mapping, a wrong SiLU sign, a V row mix-up, an unsorted schedule) fails one.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit, logsumexp, softmax
+
+import oracle as O
+import workloads as WL
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f64(a, cfg):
+    return WL.bf16_bits_to_f32(a).astype(np.float64) if cfg.dtype == WL.BF16 else \
+        np.asarray(a, np.float64)
+
+
+def _small(**kw):
+    base = dict(name="pin", L=24, d=16, Nr=6, Nc=9, k=4, K=4, B=3, dtype=WL.F32, seed=7)
+    base.update(kw)
+    return WL.Config(**base)
+
+
+# --------------------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("name", ["tiny-fp32", "bf16-N16K", "bf16-skewed-N256K",
+                                  "bf16-prefill-N1M", "bf16-decode-N1M"])
+def test_kxk_path_equals_bruteforce(name, inputs_cache):
+    """Top-K over the k x k candidates equals top-K over all N joint scores when
+    k >= K (per-axis dominance), index for index and gate for gate."""
+    cfg = WL.CONFIGS[name]
+    inp = inputs_cache(cfg, experts=False)
+    tok = WL.sample_tokens(cfg, 512 if cfg.N <= 16384 else 128)
+    lr, lc = O.axis_logprobs(cfg, inp, tok)
+    idx, gate, score = O.select(cfg, lr, lc)
+    bi, bg, bs, nxt = O.select_bruteforce(cfg, lr, lc)
+    np.testing.assert_array_equal(idx, bi)
+    np.testing.assert_allclose(gate, bg, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(score, bs, rtol=0, atol=0)
+    # the K-th score beats the (K+1)-th (strict order by (S desc, e asc))
+    assert np.all(bs[:, -1] >= nxt)
+
+
+@pytest.mark.parametrize("name", ["tiny-fp32", "bf16-N16K", "bf16-skewed-N256K",
+                                  "bf16-decode-N1M"])
+def test_gates_sum_to_one_and_are_ordered(name, inputs_cache):
+    cfg = WL.CONFIGS[name]
+    inp = inputs_cache(cfg, experts=False)
+    tok = WL.sample_tokens(cfg, 256)
+    idx, gate, score = O.route(cfg, inp, tok)
+    np.testing.assert_allclose(gate.sum(1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(gate > 0)
+    # outputs ordered by (score desc, id asc); gates follow the scores
+    assert np.all(np.diff(score, axis=1) <= 0)
+    tie = np.diff(score, axis=1) == 0
+    assert np.all(np.diff(idx, axis=1)[tie] > 0)
+    assert np.all(np.diff(gate, axis=1) <= 1e-15)
+    # gate ratio equals exp of score difference (softmax of the joint scores)
+    np.testing.assert_allclose(gate / gate[:, :1], np.exp(score - score[:, :1]), rtol=1e-12)
+
+
+def test_K1_is_argmax_of_each_axis():
+    """k = K = 1: the expert is (argmax row logit, argmax column logit), gate 1.
+    Reference: numpy matmul + argmax on the raw logits; Nr != Nc so a swapped
+    (i, j) -> id mapping or a transposed router matrix fails."""
+    cfg = _small(k=1, K=1, L=64)
+    inp = WL.make_inputs(cfg, experts=False)
+    x, Wr, Wc = (_f64(inp[n], cfg) for n in ("x", "Wr", "Wc"))
+    idx, gate, _ = O.route(cfg, inp)
+    i_ref = np.argmax(x @ Wr.T, axis=1)
+    j_ref = np.argmax(x @ Wc.T, axis=1)
+    np.testing.assert_array_equal(idx[:, 0], i_ref * cfg.Nc + j_ref)
+    np.testing.assert_array_equal(gate, 1.0)
+
+
+def test_select_all_is_the_product_distribution():
+    """Brute force with K = N selects every expert; its scores are log(pr_i pc_j)
+    and its gates pr_i * pc_j, with pr, pc the per-axis softmax (scipy)."""
+    cfg = _small(L=8)
+    inp = WL.make_inputs(cfg, experts=False)
+    x, Wr, Wc = (_f64(inp[n], cfg) for n in ("x", "Wr", "Wc"))
+    lr, lc = O.axis_logprobs(cfg, inp)
+    full = cfg.with_(K=cfg.N, k=min(cfg.Nr, cfg.Nc))
+    idx, gate, score, nxt = O.select_bruteforce(full, lr, lc)
+    pr = softmax(x @ Wr.T, axis=1)
+    pc = softmax(x @ Wc.T, axis=1)
+    prod = (pr[:, :, None] * pc[:, None, :]).reshape(cfg.L, cfg.N)
+    for t in range(cfg.L):
+        np.testing.assert_allclose(gate[t], prod[t, idx[t]], rtol=1e-12)
+        np.testing.assert_allclose(score[t], np.log(prod[t, idx[t]]), rtol=0, atol=1e-12)
+        assert sorted(idx[t].tolist()) == list(range(cfg.N))
+    assert np.all(np.isinf(nxt))
+    np.testing.assert_allclose(logsumexp(score, axis=1), 0.0, atol=1e-12)
+
+
+def test_hand_worked_example():
+    """A 2 x 2 grid worked by hand (d = 2, fp32 storage).
+
+    x = (1, 0).  Row keys give row logits (ln 3, 0): pr = (3/4, 1/4).
+    Column keys give column logits (0, ln 2): pc = (1/3, 2/3).
+    Joint probabilities (e = i*Nc + j): e0 = 1/4, e1 = 1/2, e2 = 1/12, e3 = 1/6.
+    With k = K = 2: rows {0, 1}, columns {1, 0}; the best two are e1, e0,
+    scores log(1/2), log(1/4), gates (1/2)/(3/4) = 2/3 and 1/3.
+    Experts: W[1] = (a, 0), W[0] = (b, 0) with a = ln 3, b = -2, so
+    h1 = SiLU(ln 3) = ln3 / (1 + 1/3) = (3/4) ln 3, h0 = -2 / (1 + e^2).
+    V[1] = (1, 0), V[0] = (0, 1):  y = (2/3 * (3/4) ln 3, 1/3 * (-2/(1+e^2))).
+    """
+    ln3, ln2 = math.log(3.0), math.log(2.0)
+    cfg = WL.Config("hand", L=1, d=2, Nr=2, Nc=2, k=2, K=2, B=2, dtype=WL.F32)
+    f = lambda a: np.ascontiguousarray(a, np.float32)
+    inp = {
+        "x": f([[1.0, 0.0]]),
+        "Wr": f([[ln3, 0.0], [0.0, 0.0]]),
+        "Wc": f([[0.0, 0.0], [ln2, 0.0]]),
+        "W": f([[-2.0, 0.0], [ln3, 0.0], [0.0, 0.0], [0.0, 0.0]]),
+        "V": f([[0.0, 1.0], [1.0, 0.0], [0.0, 0.0], [0.0, 0.0]]),
+        "bias_r": None, "bias_c": None,
+    }
+    # the fp32-stored values of ln 3 and ln 2 (what the oracle reads)
+    l3, l2 = float(np.float32(ln3)), float(np.float32(ln2))
+    pr = np.exp([l3, 0.0]) / (math.exp(l3) + 1.0)
+    pc = np.exp([0.0, l2]) / (1.0 + math.exp(l2))
+    idx, gate, score = O.route(cfg, inp)
+    assert idx.tolist() == [[1, 0]]
+    np.testing.assert_allclose(score[0], [math.log(pr[0] * pc[1]), math.log(pr[0] * pc[0])],
+                               atol=1e-14)
+    np.testing.assert_allclose(gate[0], [2 / 3, 1 / 3], atol=1e-7)   # fp32-stored ln's
+    np.testing.assert_allclose(gate[0], [pc[1], pc[0]], atol=1e-14)  # exact for stored ln 2
+    sched = O.schedule(cfg, idx, gate)
+    y, rows = O.forward_expert(cfg, inp, sched)
+    h1 = l3 / (1 + math.exp(-l3))
+    h0 = -2.0 / (1 + math.exp(2.0))
+    np.testing.assert_allclose(y[0], [gate[0, 0] * h1, gate[0, 1] * h0], atol=1e-15)
+    np.testing.assert_allclose(y[0], [2 / 3 * 0.75 * ln3, 1 / 3 * (-2 / (1 + math.e ** 2))],
+                               atol=1e-7)
+    assert rows == (2, 2)
+
+
+def test_equal_logits_break_ties_by_smaller_id():
+    """x = 0 makes every logit equal: all joint scores tie, the K smallest ids
+    of the k x k candidate grid win (rows 0.., columns 0..), gates are 1/K."""
+    cfg = _small(k=3, K=5, L=4)
+    inp = WL.make_inputs(cfg, experts=False)
+    inp["x"] = np.zeros_like(inp["x"])
+    idx, gate, score = O.route(cfg, inp)
+    want = sorted(i * cfg.Nc + j for i in range(cfg.k) for j in range(cfg.k))[: cfg.K]
+    for t in range(cfg.L):
+        assert idx[t].tolist() == want
+    np.testing.assert_allclose(gate, 1.0 / cfg.K, atol=1e-15)
+    np.testing.assert_allclose(score, -math.log(cfg.Nr) - math.log(cfg.Nc), atol=1e-14)
+
+
+def test_bias_shift_invariance_and_bias_sign():
+    """A constant added to every row bias (or column bias) cancels in the
+    per-axis log-softmax; a large bias on row a / column b forces expert
+    a*Nc + b to the top with gate near 1."""
+    cfg = _small(L=32)
+    inp = WL.make_inputs(cfg, experts=False)
+    z = dict(inp)
+    z["bias_r"] = np.zeros(cfg.Nr, np.float32)
+    z["bias_c"] = np.zeros(cfg.Nc, np.float32)
+    i0, g0, s0 = O.route(cfg, z)
+    z["bias_r"] = np.full(cfg.Nr, 3.25, np.float32)
+    z["bias_c"] = np.full(cfg.Nc, -7.5, np.float32)
+    i1, g1, s1 = O.route(cfg, z)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_allclose(g0, g1, atol=1e-13)
+    np.testing.assert_allclose(s0, s1, atol=1e-12)
+    z["bias_r"] = np.zeros(cfg.Nr, np.float32)
+    z["bias_c"] = np.zeros(cfg.Nc, np.float32)
+    z["bias_r"][4] = 60.0
+    z["bias_c"][7] = 60.0
+    i2, g2, s2 = O.route(cfg, z)
+    assert np.all(i2[:, 0] == 4 * cfg.Nc + 7)
+    assert np.all(g2[:, 0] > 1 - 1e-12)
+
+
+def test_router_cost_ratio_golden():
+    """(Nr + Nc) / N at N = 16K with a square grid is the printed 1.56%."""
+    vals = {}
+    with open(os.path.join(GOLDEN, "router_cost.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()
+                vals[k] = float(v)
+    cfg = WL.BF16_16K
+    assert (cfg.N, cfg.Nr, cfg.Nc) == (vals["N"], vals["Nr"], vals["Nc"])
+    ratio = 100.0 * (cfg.Nr + cfg.Nc) / cfg.N
+    assert ratio == 1.5625
+    assert round(ratio, 2) == vals["ratio_percent_printed"]
+    assert cfg.Nr == math.isqrt(cfg.N)
+
+
+# --------------------------------------------------------------------------- schedule
+
+
+def _reference_order(idx, gate, tok, B):
+    """The schedule's definition written with library primitives:
+    np.unique (sorted unique ids), searchsorted (rank), np.lexsort."""
+    K = idx.shape[1]
+    t = np.repeat(tok, K)
+    e = idx.reshape(-1).astype(np.int64)
+    g = gate.reshape(-1)
+    U = np.unique(e)
+    grp = np.searchsorted(U, e) // B
+    order = np.lexsort((e, t, grp))
+    go = np.searchsorted(grp[order], np.arange((len(U) + B - 1) // B + 1), side="left")
+    go[-1] = len(e)
+    return t[order], e[order], g[order], U, go
+
+
+@pytest.mark.parametrize("name,B", [("tiny-fp32", None), ("bf16-N16K", None),
+                                    ("tiny-fp32", 1), ("tiny-fp32", 10 ** 6),
+                                    ("bf16-skewed-N256K", None), ("bf16-decode-N1M", None)])
+def test_schedule_matches_library_definition(name, B, inputs_cache):
+    cfg = WL.CONFIGS[name]
+    if B is not None:
+        cfg = cfg.with_(B=B)
+    inp = inputs_cache(cfg.with_(B=WL.CONFIGS[name].B), experts=False)
+    tok = WL.sample_tokens(cfg, 1024)
+    idx, gate, _ = O.route(cfg, inp, tok)
+    s = O.schedule(cfg, idx, gate, tok)
+    tt, te, tg, U, go = _reference_order(idx, gate, tok, cfg.B)
+    np.testing.assert_array_equal(s["task_token"], tt)
+    np.testing.assert_array_equal(s["task_expert"], te)
+    np.testing.assert_array_equal(s["task_gate"], tg)
+    np.testing.assert_array_equal(s["uniq"], U)
+    np.testing.assert_array_equal(s["group_off"], go)
+    assert s["n_active"] == len(U)
+    assert s["n_groups"] == (len(U) + cfg.B - 1) // cfg.B
+    # structural invariants
+    assert np.all(np.diff(s["uniq"]) > 0)
+    assert np.all(np.diff(s["group_off"]) > 0)  # no empty group
+    for g in range(s["n_groups"]):
+        seg = s["task_expert"][s["group_off"][g]:s["group_off"][g + 1]]
+        assert len(np.unique(seg)) <= cfg.B
+        assert set(np.unique(seg)) == set(s["uniq"][g * cfg.B:(g + 1) * cfg.B])
+    if cfg.B == 1:
+        assert s["n_groups"] == s["n_active"]
+    if cfg.B >= s["n_active"]:
+        assert s["n_groups"] == 1
+
+
+# --------------------------------------------------------------------------- execution
+
+
+@pytest.mark.parametrize("name", ["tiny-fp32", "bf16-N16K", "bf16-skewed-N256K"])
+def test_expert_centric_equals_token_centric(name, inputs_cache):
+    """Both execution orders compute the same layer output (the scheduling is a
+    pure reordering); row counters equal the traffic model 2d*|E| vs 2d*L*K."""
+    cfg = WL.CONFIGS[name]
+    inp = inputs_cache(cfg, experts=True)
+    tok = WL.sample_tokens(cfg, 512)
+    idx, gate, _ = O.route(cfg, inp, tok)
+    s = O.schedule(cfg, idx, gate, tok)
+    ye, re = O.forward_expert(cfg, inp, s, tok)
+    yt, rt = O.forward_token(cfg, inp, idx, gate, tok)
+    scale = np.abs(yt).max()
+    assert scale > 0
+    assert np.abs(ye - yt).max() <= 1e-12 * scale
+    M = len(tok) * cfg.K
+    assert re == (s["n_active"], s["n_active"])
+    assert rt == (M, M)
+    d_tok = cfg.d * (rt[0] + rt[1])
+    d_exp = cfg.d * (re[0] + re[1])
+    assert d_tok == 2 * cfg.d * len(tok) * cfg.K
+    assert d_exp == 2 * cfg.d * s["n_active"]
+    assert d_exp <= d_tok
+
+
+def _manual_schedule(cfg, idx, gate):
+    tok = np.arange(idx.shape[0], dtype=np.int64)
+    return O.schedule(cfg, idx, gate, tok)
+
+
+def test_one_hot_value_rows_recover_gate_times_silu():
+    """V[e] = one-hot at column (e mod d): y[t, c] = sum over t's experts with
+    e mod d = c of gate * SiLU(x[t] . W[e]); h from numpy dot + scipy expit."""
+    cfg = WL.Config("probe", L=16, d=32, Nr=8, Nc=8, k=4, K=5, B=4, dtype=WL.F32, seed=3)
+    inp = WL.make_inputs(cfg)
+    V = np.zeros((cfg.N, cfg.d), np.float32)
+    V[np.arange(cfg.N), np.arange(cfg.N) % cfg.d] = 1.0
+    inp = dict(inp, V=V)
+    idx, gate, _ = O.route(cfg, inp)
+    y, _ = O.forward_expert(cfg, inp, _manual_schedule(cfg, idx, gate))
+    x, W = inp["x"].astype(np.float64), inp["W"].astype(np.float64)
+    ref = np.zeros((cfg.L, cfg.d))
+    for t in range(cfg.L):
+        for q in range(cfg.K):
+            e = idx[t, q]
+            z = float(np.dot(x[t], W[e]))
+            ref[t, e % cfg.d] += gate[t, q] * z * expit(z)
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-14)
+
+
+def test_execution_closed_forms():
+    """Hand-made tasks: x[t] = s_t * e_0 and W[e] = a_e * e_0 give
+    x . W[e] = s_t a_e exactly; SiLU(z) = z / (1 + e^-z) with its sign;
+    x = 0 gives y = 0; scaling V scales y (linearity, sign of V)."""
+    cfg = WL.Config("closed", L=3, d=8, Nr=2, Nc=3, k=2, K=2, B=2, dtype=WL.F32)
+    x = np.zeros((3, 8), np.float32)
+    x[:, 0] = [1.0, -1.5, 0.0]
+    W = np.zeros((6, 8), np.float32)
+    W[:, 0] = [2.0, -2.0, 0.5, 1.0, -0.25, 3.0]
+    V = np.zeros((6, 8), np.float32)
+    V[np.arange(6), [1, 2, 3, 4, 5, 6]] = [1.0, 2.0, -1.0, 0.5, 4.0, -3.0]
+    inp = {"x": x, "W": W, "V": V}
+    idx = np.array([[1, 5], [0, 4], [2, 3]], np.int32)
+    gate = np.array([[0.75, 0.25], [0.5, 0.5], [0.9, 0.1]])
+    sched = _manual_schedule(cfg, idx, gate)
+    y, _ = O.forward_expert(cfg, inp, sched)
+    silu = lambda z: z / (1.0 + math.exp(-z))
+    ref = np.zeros((3, 8))
+    ref[0, 2] = 0.75 * silu(1.0 * -2.0) * 2.0
+    ref[0, 6] = 0.25 * silu(1.0 * 3.0) * -3.0
+    ref[1, 1] = 0.5 * silu(-1.5 * 2.0) * 1.0
+    ref[1, 5] = 0.5 * silu(-1.5 * -0.25) * 4.0
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-15)
+    assert silu(-2.0) < 0 < silu(3.0)
+    assert np.all(y[2] == 0.0)  # x = 0 -> SiLU(0) = 0
+    y2, _ = O.forward_expert(cfg, dict(inp, V=-2 * V), sched)
+    np.testing.assert_allclose(y2, -2 * y, rtol=0, atol=1e-15)
+    yt, _ = O.forward_token(cfg, inp, idx, gate)
+    np.testing.assert_allclose(yt, ref, rtol=0, atol=1e-15)
