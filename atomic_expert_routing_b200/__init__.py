@@ -1,0 +1,221 @@
+"""Routed atomic-expert branch of an OmniMoE layer on B200 (sm_100a).
+
+Thin binding over the C ABI of ``libomnimoe.so`` (include/omnimoe.h).  Every
+step of the layer runs in the library's CUDA kernels; this module only checks
+tensor placement, allocates outputs and workspace with PyTorch, and passes raw
+pointers and the current CUDA stream.  There is no CPU path: calls need a CUDA
+device and the built library and raise otherwise.
+
+Names follow the layer: ``route`` (Cartesian Product Router), ``schedule``
+(Expert-Centric Scheduling), ``expert_forward`` (grouped execution),
+``moe_forward`` (all three), ``token_centric_forward`` (the ablation).
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_WS_EXPERT, OMNI_WS_FUSED,
+                   OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
+
+__all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",
+           "token_centric_forward", "new_counts", "OmniError", "workspace_size"]
+
+
+@dataclass(frozen=True)
+class LayerDims:
+    L: int
+    d: int
+    Nr: int
+    Nc: int
+    k: int
+    K: int
+    B: int
+    dtype: int = OMNI_BF16
+    flags: int = 0
+
+    @property
+    def N(self) -> int:
+        return self.Nr * self.Nc
+
+    @property
+    def M(self) -> int:
+        return self.L * self.K
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == OMNI_F32 else torch.bfloat16
+
+    def c(self) -> _lib.Dims:
+        return _lib.Dims(self.L, self.d, self.Nr, self.Nc, self.k, self.K, self.B, self.dtype,
+                         self.flags)
+
+    @classmethod
+    def of(cls, cfg, L=None, flags: int = 0) -> "LayerDims":
+        """From any object with L, d, Nr, Nc, k, K, B, dtype attributes."""
+        return cls(cfg.L if L is None else L, cfg.d, cfg.Nr, cfg.Nc, cfg.k, cfg.K, cfg.B,
+                   cfg.dtype, flags)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the CUDA library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the CUDA library must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _device(*ts):
+    for t in ts:
+        if t is not None:
+            return t.device
+    raise ValueError("no tensor given")
+
+
+def workspace_size(D: LayerDims, which: int) -> int:
+    n = C.c_size_t(0)
+    dd = D.c()
+    _lib.check("omni_workspace_size", _lib.load().omni_workspace_size(C.byref(dd), which,
+                                                                       C.byref(n)))
+    return int(n.value)
+
+
+class Workspace:
+    """Reusable device workspace (grows on demand)."""
+
+    def __init__(self):
+        self.buf = None
+
+    def get(self, nbytes: int, device) -> torch.Tensor | None:
+        if nbytes == 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return self.buf
+
+
+def _ws(D, which, device, ws):
+    n = workspace_size(D, which)
+    if ws is None:
+        ws = Workspace()
+    buf = ws.get(n, device)
+    return (_ptr(buf) if buf is not None else None), n
+
+
+def new_counts(device) -> torch.Tensor:
+    """Zeroed int32[4] device counters: n_active, n_groups, status bits, reserved."""
+    return torch.zeros(4, dtype=torch.int32, device=device)
+
+
+def route(D: LayerDims, x, Wr, Wc, bias_r=None, bias_c=None, *, counts=None, ws=None,
+          stream=None, with_score=True):
+    """Cartesian Product Router: (idx int32 [L,K], gate f32 [L,K], score f32 [L,K] or None)."""
+    dev = _device(x)
+    idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
+    gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
+    score = torch.empty((D.L, D.K), dtype=torch.float32, device=dev) if with_score else None
+    wsp, n = _ws(D, OMNI_WS_ROUTE, dev, ws)
+    dd = D.c()
+    _lib.check("omni_route", _lib.load().omni_route(
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c), _ptr(idx),
+        _ptr(gate), _ptr(score), _ptr(counts), wsp, n, _stream(stream)))
+    return idx, gate, score
+
+
+def router_logits(D: LayerDims, x, Wr, Wc, *, counts=None, stream=None):
+    """Router projections: float32 [L, Nr + Nc] (row logits, then column logits)."""
+    dev = _device(x)
+    z = torch.empty((D.L, D.Nr + D.Nc), dtype=torch.float32, device=dev)
+    dd = D.c()
+    _lib.check("omni_router_logits", _lib.load().omni_router_logits(
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(z), _ptr(counts), _stream(stream)))
+    return z
+
+
+def route_select(D: LayerDims, logits, bias_r=None, bias_c=None, *, counts=None, stream=None):
+    """Selection from axis logits [L, Nr + Nc] (float32)."""
+    dev = _device(logits)
+    idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
+    gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
+    score = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
+    dd = D.c()
+    _lib.check("omni_route_select", _lib.load().omni_route_select(
+        C.byref(dd), _ptr(logits), _ptr(bias_r), _ptr(bias_c), _ptr(idx), _ptr(gate),
+        _ptr(score), _ptr(counts), None, 0, _stream(stream)))
+    return idx, gate, score
+
+
+def schedule(D: LayerDims, idx, gate, *, counts=None, ws=None, stream=None) -> dict:
+    """Expert-Centric Scheduling of the L*K routing decisions (device tensors)."""
+    dev = _device(idx)
+    M = D.M
+    ucap = max(1, min(D.N, M))
+    gmax = (ucap + D.B - 1) // D.B
+    out = {
+        "task_token": torch.empty(M, dtype=torch.int32, device=dev),
+        "task_expert": torch.empty(M, dtype=torch.int32, device=dev),
+        "task_gate": torch.empty(M, dtype=torch.float32, device=dev),
+        "uniq": torch.empty(ucap, dtype=torch.int32, device=dev),
+        "group_off": torch.empty(gmax + 1, dtype=torch.int32, device=dev),
+        "counts": new_counts(dev) if counts is None else counts,
+    }
+    wsp, n = _ws(D, OMNI_WS_SCHEDULE, dev, ws)
+    dd = D.c()
+    _lib.check("omni_schedule", _lib.load().omni_schedule(
+        C.byref(dd), _ptr(idx), _ptr(gate), _ptr(out["task_token"]), _ptr(out["task_expert"]),
+        _ptr(out["task_gate"]), _ptr(out["uniq"]), _ptr(out["group_off"]), _ptr(out["counts"]),
+        wsp, n, _stream(stream)))
+    return out
+
+
+def expert_forward(D: LayerDims, x, W, V, sched: dict, *, y=None, ws=None, stream=None):
+    """Grouped (expert-centric) execution of a schedule; returns y [L, d]."""
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    wsp, n = _ws(D, OMNI_WS_EXPERT, dev, ws)
+    dd = D.c()
+    _lib.check("omni_expert_forward", _lib.load().omni_expert_forward(
+        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(sched["task_token"]),
+        _ptr(sched["task_expert"]), _ptr(sched["task_gate"]), _ptr(sched["uniq"]),
+        _ptr(sched["group_off"]), _ptr(sched["counts"]), _ptr(y), wsp, n, _stream(stream)))
+    return y
+
+
+def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=None,
+                counts=None, idx=None, gate=None, ws=None, stream=None):
+    """Route -> schedule -> grouped execution in one call; returns y [L, d]."""
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    if counts is None:
+        counts = new_counts(dev)
+    wsp, n = _ws(D, OMNI_WS_FUSED, dev, ws)
+    dd = D.c()
+    _lib.check("omni_moe_forward", _lib.load().omni_moe_forward(
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c), _ptr(W), _ptr(V),
+        _ptr(y), _ptr(idx), _ptr(gate), _ptr(counts), wsp, n, _stream(stream)))
+    return y
+
+
+def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, y=None, counts=None,
+                          stream=None):
+    """Token-centric execution (ablation): every token gathers its own experts."""
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    dd = D.c()
+    _lib.check("omni_token_centric_forward", _lib.load().omni_token_centric_forward(
+        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(idx), _ptr(gate), _ptr(y), _ptr(counts),
+        None, 0, _stream(stream)))
+    return y

@@ -1,0 +1,254 @@
+// C ABI of the routed atomic-expert layer: argument checks, workspace
+// carving and the launch sequence of every entry point (declared and
+// documented in include/omnimoe.h).  No call allocates memory, synchronises
+// the host or keeps state.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+using omni::Carver;
+using omni::Dims;
+
+namespace {
+
+bool al(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_dims(const omni_dims* in, Dims* D) {
+  if (in == nullptr) return OMNI_ERR_INVALID_ARG;
+  D->L = in->L; D->d = in->d; D->Nr = in->Nr; D->Nc = in->Nc;
+  D->k = in->k; D->K = in->K; D->B = in->B; D->dtype = in->dtype; D->flags = in->flags;
+  if (D->L < 0 || D->d < 1 || D->Nr < 1 || D->Nc < 1 || D->k < 1 || D->K < 1 || D->B < 1)
+    return OMNI_ERR_INVALID_ARG;
+  if (D->dtype != OMNI_F32 && D->dtype != OMNI_BF16) return OMNI_ERR_INVALID_ARG;
+  if ((D->flags & ~OMNI_FLAG_ROUTER_SIMT) != 0) return OMNI_ERR_INVALID_ARG;
+  if (D->k > D->Nr || D->k > D->Nc || D->K > D->k * D->k) return OMNI_ERR_INVALID_ARG;
+  if (D->Nr > OMNI_MAX_AXIS || D->Nc > OMNI_MAX_AXIS) return OMNI_ERR_UNSUPPORTED;
+  if (D->k > OMNI_MAX_TOPK || D->K > OMNI_MAX_TOPK) return OMNI_ERR_UNSUPPORTED;
+  if (D->N() >= (int64_t(1) << 31) || D->M() >= (int64_t(1) << 31)) return OMNI_ERR_UNSUPPORTED;
+  if (D->d % 8 != 0 || D->d > (int64_t(1) << 16)) return OMNI_ERR_UNSUPPORTED;
+  return OMNI_OK;
+}
+
+// workspace layouts
+struct RouteWs {
+  float* Z;
+};
+RouteWs carve_route(const Dims& D, Carver& c) {
+  RouteWs w;
+  w.Z = c.take<float>(static_cast<size_t>(D.L) * (D.Nr + D.Nc));
+  return w;
+}
+
+struct FusedWs {
+  RouteWs route;
+  int32_t *idx, *task_token, *task_expert, *uniq, *group_off;
+  float *gate, *task_gate;
+  void* sched;
+  void* expert;
+};
+FusedWs carve_fused(const Dims& D, Carver& c) {
+  FusedWs w;
+  w.route = carve_route(D, c);
+  const size_t M = static_cast<size_t>(D.M());
+  w.idx = c.take<int32_t>(M);
+  w.gate = c.take<float>(M);
+  w.task_token = c.take<int32_t>(M);
+  w.task_expert = c.take<int32_t>(M);
+  w.task_gate = c.take<float>(M);
+  w.uniq = c.take<int32_t>(static_cast<size_t>(D.ucap() > 0 ? D.ucap() : 1));
+  w.group_off = c.take<int32_t>(static_cast<size_t>(D.gmax()) + 1);
+  w.sched = c.take<char>(omni::schedule_ws_bytes(D));
+  w.expert = c.take<char>(omni::expert_ws_bytes(D));
+  return w;
+}
+
+size_t ws_size(const Dims& D, int which) {
+  Carver c(nullptr);
+  switch (which) {
+    case OMNI_WS_ROUTE: carve_route(D, c); break;
+    case OMNI_WS_SCHEDULE: c.take<char>(omni::schedule_ws_bytes(D)); break;
+    case OMNI_WS_EXPERT: c.take<char>(omni::expert_ws_bytes(D)); break;
+    case OMNI_WS_FUSED: carve_fused(D, c); break;
+    default: break;
+  }
+  return c.off;
+}
+
+int ws_ok(const Dims& D, int which, const void* ws, size_t ws_bytes) {
+  const size_t need = ws_size(D, which);
+  if (need == 0) return OMNI_OK;
+  if (ws == nullptr || !al(ws, 256) || ws_bytes < need) return OMNI_ERR_WORKSPACE;
+  return OMNI_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA; }
+
+int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, const float* br,
+               const float* bc, int32_t* idx, float* gate, float* score, int32_t* status,
+               float* Z, cudaStream_t s) {
+  cudaError_t e;
+  if (omni::router_tc_supported(D, x, Wr, Wc))
+    e = omni::launch_router_tc(D, x, Wr, Wc, Z, status, s);
+  else
+    e = omni::launch_router_simt(D, x, Wr, Wc, Z, s);
+  if (e != cudaSuccess) return OMNI_ERR_CUDA;
+  return cuda_status(omni::launch_select(D, Z, br, bc, idx, gate, score, s));
+}
+
+bool tensors_ok(const void* const* p16, int n16) {
+  for (int i = 0; i < n16; ++i)
+    if (p16[i] == nullptr || !al(p16[i], 16)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int omni_abi_version(void) { return OMNI_ABI_VERSION; }
+
+const char* omni_status_string(int status) {
+  switch (status) {
+    case OMNI_OK: return "ok";
+    case OMNI_ERR_INVALID_ARG: return "invalid argument";
+    case OMNI_ERR_UNSUPPORTED: return "unsupported by this build";
+    case OMNI_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case OMNI_ERR_CUDA: return "CUDA call failed";
+    default: return "unknown status";
+  }
+}
+
+int omni_workspace_size(const omni_dims* dims, int which, size_t* bytes) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (bytes == nullptr || which < OMNI_WS_ROUTE || which > OMNI_WS_SELECT) return OMNI_ERR_INVALID_ARG;
+  *bytes = ws_size(D, which);
+  return OMNI_OK;
+}
+
+int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+               const float* bias_r, const float* bias_c, int32_t* idx, float* gate, float* score,
+               int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc};
+  if (!tensors_ok(t16, 3) || idx == nullptr || gate == nullptr) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_ROUTE, ws, ws_bytes)) != OMNI_OK) return rc;
+  Carver c(ws);
+  RouteWs w = carve_route(D, c);
+  return route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, score,
+                    counts ? counts + 2 : nullptr, w.Z, static_cast<cudaStream_t>(stream));
+}
+
+int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                       float* logits, int32_t* counts, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, logits};
+  if (!tensors_ok(t16, 4)) return OMNI_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = omni::router_tc_supported(D, x, Wr, Wc)
+                      ? omni::launch_router_tc(D, x, Wr, Wc, logits, counts ? counts + 2 : nullptr, s)
+                      : omni::launch_router_simt(D, x, Wr, Wc, logits, s);
+  return cuda_status(e);
+}
+
+int omni_route_select(const omni_dims* dims, const float* logits, const float* bias_r,
+                      const float* bias_c, int32_t* idx, float* gate, float* score,
+                      int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  (void)counts;
+  (void)ws;
+  (void)ws_bytes;
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  if (logits == nullptr || !al(logits, 16) || idx == nullptr || gate == nullptr)
+    return OMNI_ERR_INVALID_ARG;
+  return cuda_status(omni::launch_select(D, logits, bias_r, bias_c, idx, gate, score,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int omni_schedule(const omni_dims* dims, const int32_t* idx, const float* gate,
+                  int32_t* task_token, int32_t* task_expert, float* task_gate, int32_t* uniq,
+                  int32_t* group_off, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (counts == nullptr || group_off == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L > 0 && (idx == nullptr || gate == nullptr || task_token == nullptr ||
+                  task_expert == nullptr || task_gate == nullptr || uniq == nullptr))
+    return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_SCHEDULE, ws, ws_bytes)) != OMNI_OK) return rc;
+  return cuda_status(omni::launch_schedule(D, idx, gate, task_token, task_expert, task_gate, uniq,
+                                           group_off, counts, ws,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, const void* V,
+                        const int32_t* task_token, const int32_t* task_expert,
+                        const float* task_gate, const int32_t* uniq, const int32_t* group_off,
+                        int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream) {
+  (void)uniq;
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W, V, y};
+  if (!tensors_ok(t16, 4) || task_token == nullptr || task_expert == nullptr ||
+      task_gate == nullptr || group_off == nullptr || counts == nullptr)
+    return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_EXPERT, ws, ws_bytes)) != OMNI_OK) return rc;
+  return cuda_status(omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate,
+                                         group_off, counts, y, ws,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                     const float* bias_r, const float* bias_c, const void* W, const void* V,
+                     void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
+                     size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, W, V, y};
+  if (!tensors_ok(t16, 6)) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carver c(ws);
+  FusedWs w = carve_fused(D, c);
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  float* gate = gate_out ? gate_out : w.gate;
+  rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s);
+  if (rc != OMNI_OK) return rc;
+  if (omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate, w.uniq,
+                            w.group_off, counts, w.sched, s) != cudaSuccess)
+    return OMNI_ERR_CUDA;
+  return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
+                                         w.group_off, counts, y, w.expert, s));
+}
+
+int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,
+                               const void* V, const int32_t* idx, const float* gate, void* y,
+                               int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W, V, y};
+  if (!tensors_ok(t16, 4) || idx == nullptr || gate == nullptr) return OMNI_ERR_INVALID_ARG;
+  return cuda_status(omni::launch_token(D, x, W, V, idx, gate, y, counts ? counts + 2 : nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace omni {
+
+struct Dims {
+  int64_t L, d, Nr, Nc, k, K, B;
+  int dtype;
+  int flags;
+  int64_t N() const { return Nr * Nc; }
+  int64_t M() const { return L * K; }
+  int64_t ucap() const { return N() < M() ? N() : M(); }       // bound on |U|
+  int64_t gmax() const { return (ucap() + B - 1) / B; }        // bound on #groups
+};
+
+// ---- router logits: Z [L x (Nr + Nc)] fp32 -------------------------------
+cudaError_t launch_router_simt(const Dims& D, const void* x, const void* Wr, const void* Wc,
+                               float* Z, cudaStream_t s);
+bool router_tc_supported(const Dims& D, const void* x, const void* Wr, const void* Wc);
+cudaError_t launch_router_tc(const Dims& D, const void* x, const void* Wr, const void* Wc,
+                             float* Z, int32_t* status, cudaStream_t s);
+
+// ---- selection: per-axis top-k, k x k merge, top-K, gate ----------------
+cudaError_t launch_select(const Dims& D, const float* Z, const float* br, const float* bc,
+                          int32_t* idx, float* gate, float* score, cudaStream_t s);
+
+// ---- scheduling ----------------------------------------------------------
+size_t schedule_ws_bytes(const Dims& D);
+cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate,
+                            int32_t* task_token, int32_t* task_expert, float* task_gate,
+                            int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
+                            cudaStream_t s);
+
+// ---- execution -----------------------------------------------------------
+size_t expert_ws_bytes(const Dims& D);
+cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
+                          const int32_t* task_token, const int32_t* task_expert,
+                          const float* task_gate, const int32_t* group_off,
+                          const int32_t* counts, void* y, void* ws, cudaStream_t s);
+cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
+                         const int32_t* idx, const float* gate, void* y, int32_t* status,
+                         cudaStream_t s);
+
+// 256-byte aligned carving of a workspace (base == nullptr: size only)
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+inline int64_t next_pow2(int64_t v) {
+  int64_t p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+}  // namespace omni

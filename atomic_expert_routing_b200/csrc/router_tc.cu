@@ -1,0 +1,278 @@
+// Router logits on the 5th-generation tensor cores (bf16 in, fp32 out):
+// Z[t, :Nr] = x[t] Wr^T and Z[t, Nr:] = x[t] Wc^T, the two projections of the
+// Cartesian Product Router ("OmniMoE: An Efficient MoE by Orchestrating
+// Atomic Experts at Scale" (gist.science), Technisch Overzicht section 2.2).
+// This is the one dense contraction of the routed layer: 2*d*(Nr+Nc) flops
+// per token.
+//
+// One CTA computes a 128 x BN tile of Z.  Warp 4 (one elected lane) streams
+// 128 x 64 tiles of x and BN x 64 tiles of the axis keys into shared memory
+// with TMA (128-byte swizzle, no multicast), warp 5 (one lane) issues
+// tcgen05.mma (M=128, N=BN, K=16, bf16 -> fp32) into a TMEM accumulator and
+// releases each stage with tcgen05.commit; warps 0-3 drain TMEM with
+// tcgen05.ld (one accumulator row per thread) and store fp32 logits.
+// Every mbarrier wait is bounded; a time-out sets OMNI_DEV_TIMEOUT.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace omni {
+namespace {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;  // 64 bf16 = 128 bytes = one swizzle atom row
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 192;
+
+// UMMA shared-memory descriptor for a K-major operand tile written by TMA
+// with 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu)  // start address
+         | (static_cast<uint64_t>(1) << 16)               // leading byte offset (unused)
+         | (static_cast<uint64_t>(1024 >> 4) << 32)       // stride byte offset
+         | (static_cast<uint64_t>(1) << 46)               // descriptor version
+         | (static_cast<uint64_t>(2) << 61);              // 128-byte swizzle
+}
+
+// instruction descriptor: D fp32, A and B bf16, both K-major, M x N
+template <int BN>
+__host__ __device__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>(TC_BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int BN>
+constexpr size_t tc_smem_bytes() {
+  return 1024 /* alignment slack */ +
+         static_cast<size_t>(TC_STAGES) * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) +
+         (2 * TC_STAGES + 1) * 8 + 16;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
+                const __grid_constant__ CUtensorMap tmBc, float* __restrict__ Z, int L, int Nr,
+                int Nc, int d, int tiles_r, int32_t* status) {
+  constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
+  constexpr uint32_t B_BYTES = BN * TC_BK * 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + TC_STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 1);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + TC_STAGES);
+  const uint32_t accum = smem_u32(bars + 2 * TC_STAGES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * TC_BM;
+  const bool colax = static_cast<int>(blockIdx.y) >= tiles_r;
+  const CUtensorMap* tmB = colax ? &tmBc : &tmBr;
+  const int n0 = (colax ? static_cast<int>(blockIdx.y) - tiles_r : static_cast<int>(blockIdx.y)) * BN;
+  const int naxis = colax ? Nc : Nr;
+  const int64_t ld = static_cast<int64_t>(Nr) + Nc;
+  const int zc0 = (colax ? Nr : 0) + n0;
+  const int nk = (d + TC_BK - 1) / TC_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accum, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4 && lane == 0) {
+    // producer: TMA loads of stage s
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % TC_STAGES;
+      const uint32_t ph = (kb / TC_STAGES) & 1;
+      if (!mbar_wait(empty0 + 8 * s, ph ^ 1, status)) break;
+      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES);
+      tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, full0 + 8 * s, kb * TC_BK, m0);
+      tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, kb * TC_BK, n0);
+    }
+  } else if (warp == 5 && lane == 0) {
+    // MMA issuer
+    constexpr uint32_t idesc = idesc_bf16<BN>();
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % TC_STAGES;
+      const uint32_t ph = (kb / TC_STAGES) & 1;
+      if (!mbar_wait(full0 + 8 * s, ph, status)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a0 = smem_u32(sA + s * A_BYTES);
+      const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk)
+        umma_bf16(tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                  (kb | kk) != 0 ? 1u : 0u);
+      umma_commit(empty0 + 8 * s);
+    }
+    umma_commit(accum);
+  } else if (warp < 4) {
+    // epilogue: TMEM lane (32*warp + lane) holds row m0 + 32*warp + lane
+    if (mbar_wait(accum, 0, status)) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const int64_t grow = static_cast<int64_t>(m0) + warp * 32 + lane;
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
+        if (grow < L) {
+          float* zp = Z + grow * ld + zc0 + c;
+          if (n0 + c + 32 <= naxis) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(zp + j) =
+                  make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                              __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (n0 + c + j < naxis) zp[j] = __uint_as_float(r[j]);
+          }
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN)
+                 : "memory");
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows x cols] matrix, box [box_rows x 64]
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(TC_BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int pick_bn(const Dims& D) {
+  const int64_t m = D.Nr < D.Nc ? D.Nr : D.Nc;
+  return m >= 256 ? 256 : (m >= 128 ? 128 : 64);
+}
+
+template <int BN>
+cudaError_t launch_bn(const Dims& D, const CUtensorMap& a, const CUtensorMap& br,
+                      const CUtensorMap& bc, float* Z, int32_t* status, cudaStream_t s) {
+  const size_t smem = tc_smem_bytes<BN>();
+  cudaError_t err = cudaFuncSetAttribute(k_router_tc<BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int tiles_r = static_cast<int>((D.Nr + BN - 1) / BN);
+  const int tiles_c = static_cast<int>((D.Nc + BN - 1) / BN);
+  dim3 grid(static_cast<unsigned>((D.L + TC_BM - 1) / TC_BM), tiles_r + tiles_c);
+  k_router_tc<BN><<<grid, TC_THREADS, smem, s>>>(a, br, bc, Z, static_cast<int>(D.L),
+                                                 static_cast<int>(D.Nr), static_cast<int>(D.Nc),
+                                                 static_cast<int>(D.d), tiles_r, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool router_tc_supported(const Dims& D, const void* x, const void* Wr, const void* Wc) {
+  if (D.dtype != OMNI_BF16 || (D.flags & OMNI_FLAG_ROUTER_SIMT)) return false;
+  if (D.d % 8 != 0 || D.L > (1ll << 30)) return false;  // TMA row pitch: multiple of 16 bytes
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return al16(x) && al16(Wr) && al16(Wc) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_router_tc(const Dims& D, const void* x, const void* Wr, const void* Wc,
+                             float* Z, int32_t* status, cudaStream_t s) {
+  if (D.L == 0) return cudaSuccess;
+  const int bn = pick_bn(D);
+  CUtensorMap a, br, bc;
+  if (!make_map(&a, x, D.L, D.d, TC_BM) || !make_map(&br, Wr, D.Nr, D.d, bn) ||
+      !make_map(&bc, Wc, D.Nc, D.d, bn))
+    return cudaErrorInvalidValue;
+  switch (bn) {
+    case 256: return launch_bn<256>(D, a, br, bc, Z, status, s);
+    case 128: return launch_bn<128>(D, a, br, bc, Z, status, s);
+    default: return launch_bn<64>(D, a, br, bc, Z, status, s);
+  }
+}
+
+}  // namespace omni

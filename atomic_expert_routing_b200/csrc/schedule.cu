@@ -1,0 +1,386 @@
+// Expert-Centric Scheduling on the device.
+//
+// "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at Scale"
+// (gist.science), Technisch Overzicht section 2.2 (task collection; grouping
+// and sorting; grouped execution) and the OmniMoE explainer (manus.space),
+// Expert-Centric Scheduling steps: flatten the L*K (token, expert, weight)
+// triples into tasks; collect the unique active experts, sort them by id and
+// cut every B into a group; sort tasks by group id, then token id.
+//
+// Steps (all on `stream`, data-dependent counts stay on the device):
+//  1. prep    one warp per token sorts its K (expert, gate) pairs by expert
+//             id, so the task list is in (token, expert) order, and flags
+//             every active expert in an N-long array;
+//  2. scan    exclusive prefix sum of the flags gives each active expert its
+//             rank in U (sorted unique ids), U itself, |U| and the group
+//             count ceil(|U| / B);
+//  3. sort    stable LSD radix sort of the tasks by group = rank / B with
+//             8-bit digits (as many passes as the group-count bound needs);
+//             stability keeps (token, expert) order inside each group;
+//  4. emit    gather the sorted tasks and mark each group's first task.
+#include "common.cuh"
+#include "internal.h"
+
+namespace omni {
+namespace {
+
+constexpr int kPrepWarps = 8;
+constexpr int kScanThreads = 1024;
+constexpr int kScanItems = 4;
+constexpr int kScanTile = kScanThreads * kScanItems;
+constexpr int kRsThreads = 256;
+constexpr int kRsWarps = kRsThreads / 32;
+constexpr int kRsPerWarp = 512;  // consecutive tasks per warp in a tile
+constexpr int kRsTile = kRsWarps * kRsPerWarp;
+
+// ---- 1. per-token sort by expert id + active flags -----------------------
+__global__ void __launch_bounds__(kPrepWarps * 32)
+    k_prep(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L, int K,
+           int Kp, int64_t N, int32_t* __restrict__ flags, int32_t* __restrict__ tmp_e,
+           float* __restrict__ tmp_g, int32_t* status) {
+  extern __shared__ uint64_t sbuf[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp;
+  if (t >= L) return;
+  uint64_t* s = sbuf + static_cast<size_t>(warp) * Kp;
+  for (int q = lane; q < Kp; q += 32) {
+    uint64_t key = ~0ull;
+    if (q < K) {
+      int64_t e = idx[t * K + q];
+      if (e < 0 || e >= N) {
+        raise_status(status, OMNI_DEV_BAD_INDEX);
+        e = 0;
+      }
+      flags[e] = 1;
+      key = (static_cast<uint64_t>(e) << 32) | static_cast<uint32_t>(q);
+    }
+    s[q] = key;
+  }
+  __syncwarp();
+  // bitonic sort, ascending
+  for (int size = 2; size <= Kp; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = lane; i < Kp / 2; i += 32) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool asc = (lo & size) == 0;
+        const uint64_t a = s[lo], b = s[hi];
+        if ((a > b) == asc) {
+          s[lo] = b;
+          s[hi] = a;
+        }
+      }
+      __syncwarp();
+    }
+  for (int j = lane; j < K; j += 32) {
+    const uint64_t key = s[j];
+    tmp_e[t * K + j] = static_cast<int32_t>(key >> 32);
+    tmp_g[t * K + j] = gate[t * K + static_cast<uint32_t>(key)];
+  }
+}
+
+// ---- 2. scan of the active flags ------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int w = lane < nw ? warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < nw) warp_tot[lane] = wi - w;
+    if (lane == nw - 1) *total = wi;
+  }
+  __syncthreads();
+  return incl - v + warp_tot[warp];
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_reduce(const int32_t* __restrict__ flags, int64_t N, int32_t* __restrict__ tile_sum) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
+  int v = 0;
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j)
+    if (base + j < N) v += flags[base + j];
+  block_exclusive_scan(v, warp_tot, &total);
+  if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
+}
+
+// single block: exclusive scan of the tile sums; counts[0] = |U|, counts[1] = groups
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_tiles(int32_t* __restrict__ tile_sum, int ntiles, int64_t B, int32_t* counts) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < ntiles; c0 += kScanThreads) {
+    const int i = c0 + threadIdx.x;
+    const int v = i < ntiles ? tile_sum[i] : 0;
+    const int ex = block_exclusive_scan(v, warp_tot, &total);
+    if (i < ntiles) tile_sum[i] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    counts[0] = carry;
+    counts[1] = static_cast<int32_t>((carry + B - 1) / B);
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_scan_finish(const int32_t* __restrict__ flags, int64_t N,
+                  const int32_t* __restrict__ tile_off, int32_t* __restrict__ rank,
+                  int32_t* __restrict__ uniq) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
+  int f[kScanItems];
+  int v = 0;
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    f[j] = (base + j < N) ? flags[base + j] : 0;
+    v += f[j];
+  }
+  int r = block_exclusive_scan(v, warp_tot, &total) + tile_off[blockIdx.x];
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    if (base + j < N) {
+      rank[base + j] = r;
+      if (f[j]) uniq[r] = static_cast<int32_t>(base + j);
+    }
+    r += f[j];
+  }
+}
+
+// ---- 3. stable radix sort by group id ---------------------------------------
+struct KeySrc {
+  const uint32_t* keys;    // previous pass output (nullptr on the first pass)
+  const int32_t* tmp_e;    // first pass: key = rank[tmp_e[i]] / B
+  const int32_t* rank;
+  int64_t B;
+  __device__ __forceinline__ uint32_t operator()(int64_t i) const {
+    if (keys != nullptr) return keys[i];
+    return static_cast<uint32_t>(rank[tmp_e[i]] / B);
+  }
+};
+
+__global__ void __launch_bounds__(kRsThreads)
+    k_rs_hist(KeySrc src, int64_t M, int shift, int ntiles, uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[256];
+  h[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRsTile;
+  for (int j = threadIdx.x; j < kRsTile; j += kRsThreads) {
+    const int64_t i = t0 + j;
+    if (i < M) atomicAdd(&h[(src(i) >> shift) & 255u], 1u);
+  }
+  __syncthreads();
+  hist[static_cast<int64_t>(threadIdx.x) * ntiles + blockIdx.x] = h[threadIdx.x];
+}
+
+// single block exclusive scan over n = 256 * ntiles words (digit-major)
+__global__ void __launch_bounds__(kScanThreads) k_rs_scan(uint32_t* __restrict__ hist, int64_t n) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int64_t chunk = static_cast<int64_t>(kScanThreads) * kScanItems;
+  for (int64_t c0 = 0; c0 < n; c0 += chunk) {
+    const int64_t base = c0 + static_cast<int64_t>(threadIdx.x) * kScanItems;
+    uint32_t v[kScanItems];
+    int s = 0;
+#pragma unroll
+    for (int j = 0; j < kScanItems; ++j) {
+      v[j] = (base + j < n) ? hist[base + j] : 0u;
+      s += static_cast<int>(v[j]);
+    }
+    int ex = block_exclusive_scan(s, warp_tot, &total) + carry;
+#pragma unroll
+    for (int j = 0; j < kScanItems; ++j) {
+      if (base + j < n) hist[base + j] = static_cast<uint32_t>(ex);
+      ex += static_cast<int>(v[j]);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kRsThreads)
+    k_rs_scatter(KeySrc src, const uint32_t* __restrict__ vals_in, int64_t M, int shift,
+                 int ntiles, const uint32_t* __restrict__ hist, uint32_t* __restrict__ keys_out,
+                 uint32_t* __restrict__ vals_out) {
+  __shared__ uint32_t wcount[kRsWarps][256];
+  __shared__ uint32_t dbase[256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = threadIdx.x; j < kRsWarps * 256; j += kRsThreads) (&wcount[0][0])[j] = 0;
+  dbase[threadIdx.x] = hist[static_cast<int64_t>(threadIdx.x) * ntiles + blockIdx.x];
+  __syncthreads();
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kRsTile + warp * kRsPerWarp;
+  constexpr int R = kRsPerWarp / 32;
+  uint32_t key[R], rnk[R];
+  // per-warp stable ranks, in element order
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = w0 + r * 32 + lane;
+    const bool valid = i < M;
+    key[r] = valid ? src(i) : 0u;
+    const uint32_t dig = valid ? ((key[r] >> shift) & 255u) : 0xffffffffu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+    const int leader = __ffs(peers) - 1;
+    uint32_t old = 0;
+    if (valid && lane == leader) {
+      old = wcount[warp][dig];
+      wcount[warp][dig] = old + __popc(peers);
+    }
+    old = __shfl_sync(0xffffffffu, old, leader);
+    rnk[r] = old + __popc(peers & lanemask_lt());
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive prefix of the per-warp counts, per digit
+  {
+    const int dgt = threadIdx.x;
+    uint32_t run = 0;
+    for (int w = 0; w < kRsWarps; ++w) {
+      const uint32_t c = wcount[w][dgt];
+      wcount[w][dgt] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = w0 + r * 32 + lane;
+    if (i < M) {
+      const uint32_t dig = (key[r] >> shift) & 255u;
+      const uint32_t pos = dbase[dig] + wcount[warp][dig] + rnk[r];
+      keys_out[pos] = key[r];
+      vals_out[pos] = vals_in ? vals_in[i] : static_cast<uint32_t>(i);
+    }
+  }
+}
+
+// ---- 4. emit ---------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_emit(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, int64_t M, int K,
+           const int32_t* __restrict__ tmp_e, const float* __restrict__ tmp_g,
+           int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
+           float* __restrict__ task_gate, int32_t* __restrict__ group_off,
+           const int32_t* __restrict__ counts) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M) return;
+  const uint32_t pos = vals ? vals[i] : static_cast<uint32_t>(i);
+  const uint32_t g = keys ? keys[i] : 0u;
+  task_token[i] = static_cast<int32_t>(pos / static_cast<uint32_t>(K));
+  task_expert[i] = tmp_e[pos];
+  task_gate[i] = tmp_g[pos];
+  if (i == 0 || (keys ? keys[i - 1] : 0u) != g) group_off[g] = static_cast<int32_t>(i);
+  if (i == M - 1) group_off[counts[1]] = static_cast<int32_t>(M);
+}
+
+struct SchedWs {
+  int32_t *flags, *rank, *tile_sum, *tmp_e;
+  float* tmp_g;
+  uint32_t *ka, *va, *kb, *vb, *hist;
+  int64_t nscan, ntiles;
+  int passes;
+};
+
+SchedWs carve(const Dims& D, void* base, size_t* bytes) {
+  Carver c(base);
+  SchedWs w{};
+  const int64_t N = D.N(), M = D.M();
+  w.nscan = (N + kScanTile - 1) / kScanTile;
+  w.ntiles = (M + kRsTile - 1) / kRsTile;
+  int bits = 0;
+  while ((int64_t(1) << bits) < D.gmax()) ++bits;
+  w.passes = (bits + 7) / 8;
+  w.flags = c.take<int32_t>(N);
+  w.rank = c.take<int32_t>(N);
+  w.tile_sum = c.take<int32_t>(w.nscan + 1);
+  w.tmp_e = c.take<int32_t>(M);
+  w.tmp_g = c.take<float>(M);
+  if (w.passes > 0) {
+    w.ka = c.take<uint32_t>(M);
+    w.va = c.take<uint32_t>(M);
+    w.kb = c.take<uint32_t>(M);
+    w.vb = c.take<uint32_t>(M);
+    w.hist = c.take<uint32_t>(256 * w.ntiles);
+  }
+  if (bytes) *bytes = c.off;
+  return w;
+}
+
+}  // namespace
+
+size_t schedule_ws_bytes(const Dims& D) {
+  size_t b = 0;
+  carve(D, nullptr, &b);
+  return b;
+}
+
+cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate,
+                            int32_t* task_token, int32_t* task_expert, float* task_gate,
+                            int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
+                            cudaStream_t s) {
+  const int64_t N = D.N(), M = D.M();
+  int32_t* status = counts + 2;
+  if (M == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, 2 * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(group_off, 0, sizeof(int32_t), s);
+    return e;
+  }
+  SchedWs w = carve(D, ws, nullptr);
+  cudaError_t err = cudaMemsetAsync(w.flags, 0, static_cast<size_t>(N) * sizeof(int32_t), s);
+  if (err != cudaSuccess) return err;
+  const int Kp = static_cast<int>(next_pow2(D.K));
+  const size_t prep_smem = static_cast<size_t>(kPrepWarps) * Kp * sizeof(uint64_t);
+  k_prep<<<static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps), kPrepWarps * 32,
+           prep_smem, s>>>(idx, gate, D.L, static_cast<int>(D.K), Kp, N, w.flags, w.tmp_e,
+                           w.tmp_g, status);
+  k_scan_reduce<<<static_cast<unsigned>(w.nscan), kScanThreads, 0, s>>>(w.flags, N, w.tile_sum);
+  k_scan_tiles<<<1, kScanThreads, 0, s>>>(w.tile_sum, static_cast<int>(w.nscan), D.B, counts);
+  k_scan_finish<<<static_cast<unsigned>(w.nscan), kScanThreads, 0, s>>>(w.flags, N, w.tile_sum,
+                                                                       w.rank, uniq);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const uint32_t* keys = nullptr;
+  const uint32_t* vals = nullptr;
+  uint32_t *ko = w.ka, *vo = w.va;
+  for (int p = 0; p < w.passes; ++p) {
+    KeySrc src{keys, w.tmp_e, w.rank, D.B};
+    k_rs_hist<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(src, M, 8 * p,
+                                                                      static_cast<int>(w.ntiles),
+                                                                      w.hist);
+    k_rs_scan<<<1, kScanThreads, 0, s>>>(w.hist, 256 * w.ntiles);
+    k_rs_scatter<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(
+        src, vals, M, 8 * p, static_cast<int>(w.ntiles), w.hist, ko, vo);
+    keys = ko;
+    vals = vo;
+    ko = (ko == w.ka) ? w.kb : w.ka;
+    vo = (vo == w.va) ? w.vb : w.va;
+  }
+  k_emit<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(
+      keys, vals, M, static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate,
+      group_off, counts);
+  return cudaGetLastError();
+}
+
+}  // namespace omni

@@ -1,0 +1,444 @@
+"""Benchmark of the routed atomic-expert layer (Cartesian router -> expert-centric
+schedule -> grouped execution) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload bf16-prefill-N1M|bf16-decode-N1M|...]
+
+One step = one omni_moe_forward over a batch of L tokens of synthetic inputs
+already resident in HBM.  L2 is flushed (a write larger than L2) before every
+timed step, outside the step's CUDA events.  Prints one JSON line on rank 0.
+
+Multi-GPU (torchrun): tokens are independent, so every rank runs its own
+batch (its own x, replicated router and expert weights) with no collective on
+the data path; value = all ranks' tokens / the slowest rank's time
+(weak scaling).  --impl reference times the fp64 CPU oracle instead (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as WL  # noqa: E402
+
+METRIC = "routed-layer tokens/s at N=1M,d=2048 (L=16K & L=64); % of TC/HBM roofline"
+PRIMARY = WL.PREFILL
+SECONDARY = WL.DECODE
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(
+            j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def layer_work(cfg, n_active):
+    """Algorithmic flops and bytes of one layer pass (the method's own work)."""
+    e = cfg.esize
+    flops = 2 * cfg.d * (cfg.Nr + cfg.Nc) * cfg.L + 4 * cfg.d * cfg.L * cfg.K
+    bytes_ = (cfg.L * cfg.d * e + (cfg.Nr + cfg.Nc) * cfg.d * e + 2 * cfg.d * n_active * e
+              + cfg.L * cfg.d * e)
+    return flops, bytes_
+
+
+def expert_stage_bytes(cfg, n_active):
+    """Algorithmic bytes of the grouped execution: active rows of W and V once,
+    x read, y written."""
+    e = cfg.esize
+    return 2 * cfg.d * n_active * e + 2 * cfg.L * cfg.d * e
+
+
+def kernel_launches(cfg):
+    """Kernels of this library launched by one omni_moe_forward (memsets excluded)."""
+    ucap = min(cfg.N, cfg.L * cfg.K)
+    gmax = (ucap + cfg.B - 1) // cfg.B
+    bits = max(0, int(np.ceil(np.log2(gmax)))) if gmax > 1 else 0
+    passes = (bits + 7) // 8
+    route = 2
+    sched = 1 + 3 + 3 * passes + 1
+    expert = 1 + (1 if cfg.dtype == WL.BF16 else 0)
+    return route + sched + expert
+
+
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle arm
+
+
+def oracle_timing(cfg, target_s=10.0, max_tokens=None):
+    """Time the fp64 oracle (route -> schedule -> expert-centric execution) on a
+    bounded token sample sized for about target_s of CPU work.  Returns
+    (tokens/s, sample tokens, seconds, threads)."""
+    import oracle as O
+
+    h = WL.make_inputs(cfg)
+    n = 64
+    while True:
+        tok = WL.sample_tokens(cfg, n)
+        cs = cfg.with_(L=len(tok))
+        hs = dict(h, x=np.ascontiguousarray(h["x"][tok]))
+        t0 = time.perf_counter()
+        O.moe_forward(cs, hs)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= cfg.L or (max_tokens and n >= max_tokens):
+            return len(tok) / dt, len(tok), dt, O.num_threads(), h
+        n = min(cfg.L, max(n * 2, int(n * target_s / max(dt, 1e-3) * 1.1)))
+        if max_tokens:
+            n = min(n, max_tokens)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = WL.CONFIGS[args.workload]
+    rate, n, dt, threads, _ = oracle_timing(cfg, target_s=max(2.0, 60.0 / max(1, args.steps)))
+    # steps: repeat the bounded sample K times after W warm-ups (each a full pass)
+    import oracle as O
+    h = WL.make_inputs(cfg)
+    tok = WL.sample_tokens(cfg, n)
+    cs = cfg.with_(L=len(tok))
+    hs = dict(h, x=np.ascontiguousarray(h["x"][tok]))
+    for _ in range(args.warmup):
+        O.moe_forward(cs, hs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.moe_forward(cs, hs)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = len(tok) / dt
+    cpu = {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{len(tok)} of {cfg.L} tokens of {cfg.name} per step (route+schedule+"
+                     "expert-centric execution, fp64)"}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "L": cfg.L, "d": cfg.d, "Nr": cfg.Nr, "Nc": cfg.Nc,
+                       "k": cfg.k, "K": cfg.K, "B": cfg.B, "sample_tokens": len(tok)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import atomic_expert_routing_b200 as omni
+    from atomic_expert_routing_b200 import build as libbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    libbuild.build()
+    hbm, tc, tc_sus, peak_src = measured_peaks()
+
+    def to_dev(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    cfg = WL.CONFIGS[args.workload]
+    # every rank draws its own token batch (seed + rank); weights are shared
+    rcfg = cfg.with_(seed=cfg.seed)
+    host = WL.make_inputs(rcfg, experts=False)
+    if rank > 0:
+        host["x"] = WL.make_inputs(cfg.with_(seed=cfg.seed + 1000 * rank), experts=False)["x"]
+    experts = WL.make_experts(cfg)
+    d = {k: to_dev(v) for k, v in host.items()}
+    d.update({k: to_dev(v) for k, v in experts.items()})
+    del experts
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def measure(c, dd, steps, warmup, graph=True):
+        D = omni.LayerDims.of(c)
+        ws = omni.Workspace()
+        counts = omni.new_counts(device)
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        stream = torch.cuda.Stream(device)
+
+        def fwd():
+            omni.moe_forward(D, dd["x"], dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                             dd["bias_c"], y=y, counts=counts, ws=ws, stream=stream)
+
+        with torch.cuda.stream(stream):
+            fwd()  # sizes the workspace
+        torch.cuda.synchronize()
+        g = None
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fwd()
+        run = g.replay if g is not None else fwd
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                flush.zero_()
+                run()
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with Clocks(local) as clk:
+            barrier()
+            with torch.cuda.stream(stream):
+                for a, b in ev:
+                    flush.zero_()
+                    a.record(stream)
+                    run()
+                    b.record(stream)
+            barrier()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        torch.cuda.synchronize()
+        n_active = int(counts[0].item())
+        status = int(counts[2].item())
+        return ms, n_active, status, clk.summary(), y
+
+    def measure_expert_stage(c, dd, steps):
+        """Grouped execution alone (its own events), for the kernel roofline."""
+        D = omni.LayerDims.of(c)
+        idx, gate, _ = omni.route(D, dd["x"], dd["Wr"], dd["Wc"], dd["bias_r"], dd["bias_c"])
+        s = omni.schedule(D, idx, gate)
+        ws = omni.Workspace()
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        stream = torch.cuda.current_stream(device)
+        omni.expert_forward(D, dd["x"], dd["W"], dd["V"], s, y=y, ws=ws)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            omni.expert_forward(D, dd["x"], dd["W"], dd["V"], s, y=y, ws=ws)
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / steps, int(s["counts"][0].item())
+
+    def measure_e2e(c, dd, steps, warmup):
+        """The public call with host buffers: pinned x -> device, forward, y -> pinned host."""
+        D = omni.LayerDims.of(c)
+        xh = torch.empty((c.L, c.d), dtype=D.torch_dtype).pin_memory()
+        xh.copy_(dd["x"].cpu())
+        yh = torch.empty((c.L, c.d), dtype=D.torch_dtype).pin_memory()
+        xd = torch.empty_like(dd["x"])
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        counts = omni.new_counts(device)
+        ws = omni.Workspace()
+        stream = torch.cuda.Stream(device)
+
+        def step():
+            xd.copy_(xh, non_blocking=True)
+            omni.moe_forward(D, xd, dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                             dd["bias_c"], y=y, counts=counts, ws=ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                flush.zero_()
+                step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        return ms, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+
+    ms, n_active, status, clocks, _ = measure(cfg, d, args.steps, args.warmup)
+    ms_all = ms
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_all = float(t.item())
+    e2e_ms, h2d, d2h = measure_e2e(cfg, d, max(3, args.steps // 2), args.warmup)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
+
+    extra = {}
+    if args.workload == PRIMARY.name and not args.no_secondary:
+        sc = SECONDARY
+        host2 = WL.make_inputs(sc.with_(seed=sc.seed + 1000 * rank), experts=False)
+        d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
+        ms2, na2, st2, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
+        if world > 1:
+            t = torch.tensor([ms2], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms2 = float(t.item())
+        f2, b2 = layer_work(sc, na2)
+        extra[sc.name] = {
+            "value": world * sc.L / (ms2 * 1e-3), "unit": "tokens/s", "ms_per_step": ms2,
+            "n_active": na2, "device_status": st2,
+            "layer_roofline": {"bound": "hbm" if b2 / (hbm * 1e9) > f2 / (tc * 1e12) else "tensor",
+                               "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
+                               "bytes": b2, "flops": f2}}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    flops, bytes_ = layer_work(cfg, n_active)
+    t_f = flops / (tc * 1e12)
+    t_b = bytes_ / (hbm * 1e9)
+    eb = expert_stage_bytes(cfg, n_act2)
+    achieved = eb / (st_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, n, dt, threads, _ = oracle_timing(cfg, target_s=args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} of {cfg.L} tokens of {cfg.name} (route+schedule+expert-centric "
+                         f"execution, fp64), {dt:.1f} s"}
+    line = {
+        "metric": METRIC,
+        "value": world * cfg.L / (ms_all * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_all,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == WL.BF16 else "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "L": cfg.L, "d": cfg.d, "Nr": cfg.Nr, "Nc": cfg.Nc,
+                   "N": cfg.N, "k": cfg.k, "K": cfg.K, "B": cfg.B, "l2": "flushed before each step",
+                   "graph": True, "parallelism": f"dp{world} (independent token batches)"},
+        "n_active": n_active,
+        "device_status": status,
+        "layer_roofline": {"bound": "hbm" if t_b >= t_f else "tensor",
+                           "frac": max(t_f, t_b) / (ms_all * 1e-3), "bytes": bytes_,
+                           "flops": flops, "peak_src": peak_src},
+        "roofline": {"kernel": "grouped expert-centric execution (omni_expert_forward)",
+                     "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": eb,
+                     "ms": st_ms, "peak_src": peak_src},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * cfg.L / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": kernel_launches(cfg) * args.steps,
+        "clocks": clocks,
+    }
+    if extra:
+        line["also"] = extra
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=PRIMARY.name, choices=sorted(WL.CONFIGS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

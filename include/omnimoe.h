@@ -1,0 +1,197 @@
+/*
+ * omnimoe.h -- C ABI of the routed atomic-expert branch of an OmniMoE layer,
+ * B200 (sm_100a) implementation.
+ *
+ * The layer (sources are web pages about OmniMoE, cited by title/section):
+ *   [NL 2.1]  "OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at
+ *             Scale" (gist.science, Dutch), Technisch Overzicht section 2.1:
+ *             atomic expert i is a vector pair (w_in, w_out) computing
+ *             E_i(x) = sigma(x w_in^T) w_out; all N experts are the rows of
+ *             two global matrices W, V (N x d).
+ *   [NL 2.2]  same page, section 2.2: the Cartesian Product Router (row and
+ *             column logits over an Nr x Nc grid of experts) and
+ *             Expert-Centric Scheduling (task collection, grouping and
+ *             sorting, grouped execution).
+ *   [MS router] OmniMoE explainer (omnimoeexpl, manus.space), Cartesian
+ *             product router section: S_ij = pr[i] + pc[j] in log space,
+ *             no N-wide score vector.
+ *   [MS sched]  same page, Expert-Centric Scheduling steps and the traffic
+ *             model D = 2d*L*K (token-centric) vs 2d*|E_active|.
+ *
+ * Conventions for every call
+ *   - All pointers are DEVICE pointers owned by the caller (except `dims`,
+ *     `bytes` and the returned strings, which are host memory).  The library
+ *     allocates no memory and keeps no state between calls; scratch space is
+ *     the caller's workspace `ws` of `ws_bytes` bytes (size from
+ *     omni_workspace_size, 256-byte aligned pointer).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Nothing synchronises the host;
+ *     data-dependent sizes (number of active experts, of groups) stay on the
+ *     device in `counts`.
+ *   - Row-major layouts.  x [L x d], W, V [N x d], y [L x d] in the storage
+ *     type `dims->dtype` (OMNI_F32: float, OMNI_BF16: bfloat16).  The router
+ *     keys Wr [Nr x d] and Wc [Nc x d] hold one d-vector per grid row/column
+ *     (the d x Nr projection of the pages, stored transposed), so row logit i
+ *     of token t is x[t] . Wr[i].  Optional biases are float [Nr], [Nc].
+ *     Expert id of grid cell (i, j) is e = i*Nc + j.
+ *   - Pointers to x, Wr, Wc, W, V, y and the logits must be 16-byte aligned,
+ *     all others 4-byte aligned; `ws` 256-byte aligned.
+ *   - Return value: OMNI_OK when the work was enqueued; an error code when
+ *     the host-side checks failed (nothing was enqueued) or a CUDA launch
+ *     failed.  No exception or exit crosses the ABI.
+ *   - counts (int32[4], device): [0] number of active experts, [1] number of
+ *     groups (both written by the scheduling step), [2] device status bits,
+ *     OR-ed by kernels and never cleared by the library (the caller zeroes
+ *     it; see OMNI_DEV_*), [3] reserved.
+ */
+#ifndef OMNIMOE_H
+#define OMNIMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OMNI_ABI_VERSION 1
+
+/* host-side status codes (return values) */
+#define OMNI_OK 0
+#define OMNI_ERR_INVALID_ARG 1  /* null/misaligned pointer, inconsistent sizes */
+#define OMNI_ERR_UNSUPPORTED 2  /* valid but outside this build's limits */
+#define OMNI_ERR_WORKSPACE 3    /* ws too small or misaligned */
+#define OMNI_ERR_CUDA 4         /* a CUDA runtime/driver call failed */
+
+/* device status bits, OR-ed into counts[2] */
+#define OMNI_DEV_TIMEOUT 1      /* a bounded device wait gave up (kernel returned early) */
+#define OMNI_DEV_BAD_INDEX 2    /* an expert id outside [0, N) was read and ignored */
+
+/* storage types */
+#define OMNI_F32 0
+#define OMNI_BF16 1
+
+/* dims.flags bits */
+#define OMNI_FLAG_ROUTER_SIMT 1 /* diagnostic: router logits on CUDA cores for bf16 too */
+
+/* Limits of this build (host checks return OMNI_ERR_UNSUPPORTED beyond them). */
+#define OMNI_MAX_AXIS 4096      /* Nr, Nc */
+#define OMNI_MAX_TOPK 256       /* k, K */
+
+typedef struct omni_dims {
+  int64_t L;     /* tokens in the batch (>= 0) */
+  int64_t d;     /* model width (multiple of 8; of 4 for OMNI_F32) */
+  int64_t Nr;    /* grid rows */
+  int64_t Nc;    /* grid columns; N = Nr*Nc atomic experts (< 2^31) */
+  int64_t k;     /* per-axis top-k, 1 <= k <= min(Nr, Nc) */
+  int64_t K;     /* experts per token, 1 <= K <= k*k */
+  int64_t B;     /* active experts per scheduling group, >= 1 */
+  int32_t dtype; /* OMNI_F32 or OMNI_BF16 */
+  int32_t flags; /* OMNI_FLAG_* */
+} omni_dims;
+
+/* workspace kinds for omni_workspace_size */
+#define OMNI_WS_ROUTE 0
+#define OMNI_WS_SCHEDULE 1
+#define OMNI_WS_EXPERT 2
+#define OMNI_WS_FUSED 3
+#define OMNI_WS_TOKEN 4
+#define OMNI_WS_SELECT 5
+
+/* Bytes of workspace the call `which` needs for `dims` (0 is possible). */
+int omni_workspace_size(const omni_dims* dims, int which, size_t* bytes);
+
+/*
+ * Cartesian Product Router [NL 2.2], [MS router].
+ * For every token t: row logits z_r = x[t] Wr^T + bias_r, column logits
+ * z_c = x[t] Wc^T + bias_c (fp32 accumulation); per-axis log-softmax
+ * lr, lc; top-k rows R and top-k columns C (value desc, index asc); joint
+ * scores S = lr[i] + lc[j] over R x C only; the K best by (S desc, e asc).
+ * Outputs, K per token in that order:
+ *   idx   int32 [L x K]  expert ids e = i*Nc + j
+ *   gate  float [L x K]  softmax of the K selected joint scores
+ *   score float [L x K]  the joint log-probabilities S (nullable)
+ * bias_r / bias_c may be NULL (no bias).
+ */
+int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+               const float* bias_r, const float* bias_c, int32_t* idx, float* gate,
+               float* score, int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The projection half of omni_route [NL 2.2]: logits float [L x (Nr + Nc)],
+ * row t = (x[t] Wr^T, x[t] Wc^T), fp32 accumulation, no bias.  bf16 storage
+ * runs on the tensor cores (tcgen05), fp32 storage on CUDA cores.  Needs no
+ * workspace.
+ */
+int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                       float* logits, int32_t* counts, void* stream);
+
+/*
+ * The selection half of omni_route, from axis logits the caller computed:
+ * logits float [L x (Nr + Nc)] holds z_r then z_c of each token (biases are
+ * added here when given).  Same outputs as omni_route.
+ */
+int omni_route_select(const omni_dims* dims, const float* logits, const float* bias_r,
+                      const float* bias_c, int32_t* idx, float* gate, float* score,
+                      int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Expert-Centric Scheduling [NL 2.2], [MS sched].
+ * Tasks are the M = L*K triples (t, idx[t,k], gate[t,k]).  U = the sorted
+ * unique active expert ids; the group of expert e is (rank of e in U) / B;
+ * tasks are sorted by (group, token, expert).  Outputs:
+ *   task_token, task_expert int32 [M], task_gate float [M]  sorted tasks
+ *   uniq      int32 [min(N, M)]        U (first counts[0] entries valid)
+ *   group_off int32 [G_max + 1]        group g = tasks [group_off[g], group_off[g+1]);
+ *                                      G_max = ceil(min(N, M) / B); first
+ *                                      counts[1] + 1 entries valid
+ *   counts    [0] = |U|, [1] = ceil(|U| / B)
+ * An id outside [0, N) sets OMNI_DEV_BAD_INDEX and is treated as expert 0.
+ */
+int omni_schedule(const omni_dims* dims, const int32_t* idx, const float* gate,
+                  int32_t* task_token, int32_t* task_expert, float* task_gate, int32_t* uniq,
+                  int32_t* group_off, int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Grouped (expert-centric) execution [NL 2.1], [NL 2.2], [MS sched]: group
+ * by group, every task (t, e, g) adds g * SiLU(x[t] . W[e]) * V[e] to y[t]
+ * (sigma = scalar SiLU).  Inputs are omni_schedule's outputs (counts read on
+ * the device).  y [L x d] is overwritten (tokens without tasks get 0);
+ * accumulation is fp32, the bf16 result rounded to nearest even.
+ */
+int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, const void* V,
+                        const int32_t* task_token, const int32_t* task_expert,
+                        const float* task_gate, const int32_t* uniq, const int32_t* group_off,
+                        int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole routed branch: omni_route -> omni_schedule -> omni_expert_forward
+ * on one stream, intermediates in ws.  idx_out / gate_out (nullable, [L x K])
+ * receive the routing decisions.  y as in omni_expert_forward.
+ */
+int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                     const float* bias_r, const float* bias_c, const void* W, const void* V,
+                     void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * Token-centric execution, the order Expert-Centric Scheduling replaces
+ * [NL 2.2], [MS sched]: every token gathers the rows of its own K experts,
+ * y[t] = sum_k gate[t,k] * SiLU(x[t] . W[idx[t,k]]) * V[idx[t,k]].
+ * Kept as the in-library ablation.  idx/gate as produced by omni_route.
+ */
+int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,
+                               const void* V, const int32_t* idx, const float* gate, void* y,
+                               int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* omni_status_string(int status);
+
+/* OMNI_ABI_VERSION of the loaded library. */
+int omni_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OMNIMOE_H */

@@ -60,6 +60,20 @@ def _tokens(cfg, tokens):
     return np.ascontiguousarray(tokens, dtype=np.int64)
 
 
+def axis_logits(cfg, inp, tokens=None):
+    """Raw router logits (zr [nt, Nr], zc [nt, Nc]) including the optional biases."""
+    tok = _tokens(cfg, tokens)
+    zr = np.empty((len(tok), cfg.Nr), np.float64)
+    zc = np.empty((len(tok), cfg.Nc), np.float64)
+    br = None if inp.get("bias_r") is None else np.ascontiguousarray(inp["bias_r"], np.float32)
+    bc = None if inp.get("bias_c") is None else np.ascontiguousarray(inp["bias_c"], np.float32)
+    D = dims(cfg)
+    _check(lib().oracle_axis_logits(C.byref(D), _p(inp["x"]), _p(inp["Wr"]), _p(inp["Wc"]),
+                                    _p(br), _p(bc), _p(tok), C.c_int64(len(tok)), _p(zr),
+                                    _p(zc)), "axis_logits")
+    return zr, zc
+
+
 def axis_logprobs(cfg, inp, tokens=None):
     """Per-axis log-softmax of the router logits: (lr [nt, Nr], lc [nt, Nc])."""
     tok = _tokens(cfg, tokens)

@@ -143,6 +143,26 @@ static void axis_topk(const double* lz, int64_t n, int64_t k, scored* tmp, int64
   }
 }
 
+/* Raw axis logits of the listed tokens: zr [nt x Nr], zc [nt x Nc]  [NL 2.2] */
+int oracle_axis_logits(const or_dims* D, const void* x, const void* Wr, const void* Wc,
+                       const float* bias_r, const float* bias_c, const int64_t* tok, int64_t nt,
+                       double* zr, double* zc) {
+  const int64_t d = D->d, Nr = D->Nr, Nc = D->Nc;
+#pragma omp parallel
+  {
+    double* xrow = (double*)malloc(sizeof(double) * d);
+    double* wrow = (double*)malloc(sizeof(double) * d);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nt; ++r) {
+      axis_logits(x, Wr, bias_r, D->dtype, tok[r], d, Nr, xrow, wrow, zr + r * Nr);
+      axis_logits(x, Wc, bias_c, D->dtype, tok[r], d, Nc, xrow, wrow, zc + r * Nc);
+    }
+    free(xrow);
+    free(wrow);
+  }
+  return 0;
+}
+
 /* Per-axis log-softmax logits of the listed tokens: lr [nt x Nr], lc [nt x Nc]. */
 int oracle_axis_logprobs(const or_dims* D, const void* x, const void* Wr, const void* Wc,
                          const float* bias_r, const float* bias_c, const int64_t* tok,

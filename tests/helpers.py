@@ -1,0 +1,58 @@
+"""Shared helpers of the GPU parity tests (data movement and comparisons only)."""
+import numpy as np
+import torch
+
+import workloads as WL
+
+
+def dev(a, device="cuda"):
+    """numpy array (bf16 as uint16 bits, or float32/int32) -> torch CUDA tensor."""
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def host_f64(t):
+    """torch tensor (bf16/f32/int) -> numpy float64 (bf16 widened exactly)."""
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.float().numpy().astype(np.float64)
+    return t.numpy().astype(np.float64)
+
+
+def rel_err(y, ref):
+    """max |y - ref| / max |ref|  (the layer-output parity metric)."""
+    scale = float(np.abs(ref).max())
+    return float(np.abs(y - ref).max()) / (scale if scale > 0 else 1.0)
+
+
+def tol_y(cfg):
+    return 1e-4 if cfg.dtype == WL.F32 else 2e-2
+
+
+def check_selection(cfg, gpu_idx, gpu_gate, gpu_score, ora_idx, ora_gate, ora_score, nxt, lr, lc,
+                    rel=1e-4):
+    """Per token: bit-exact ids unless the oracle's K-th and (K+1)-th scores are a
+    near-tie; near-tie tokens must still hold a valid top-K within the tie band.
+    Returns (number of exact tokens, number of near-tie tokens)."""
+    near = np.abs(ora_score[:, -1] - nxt) < rel * np.abs(ora_score[:, -1])
+    exact = ~near
+    bad = np.nonzero(exact & np.any(gpu_idx != ora_idx, axis=1))[0]
+    assert len(bad) == 0, f"{len(bad)} tokens differ in their selected experts, e.g. {bad[:5]}"
+    # gates and scores where the ids match
+    np.testing.assert_allclose(gpu_gate[exact], ora_gate[exact], rtol=2e-4, atol=2e-6)
+    if gpu_score is not None:
+        np.testing.assert_allclose(gpu_score[exact], ora_score[exact], rtol=0, atol=2e-4)
+    # near-tie tokens: the GPU set is a valid top-K of the oracle scores within the band
+    for r in np.nonzero(near)[0]:
+        e = gpu_idx[r].astype(np.int64)
+        assert len(np.unique(e)) == cfg.K and e.min() >= 0 and e.max() < cfg.N
+        s = lr[r, e // cfg.Nc] + lc[r, e % cfg.Nc]
+        band = rel * abs(ora_score[r, -1])
+        assert np.all(s >= ora_score[r, -1] - 2 * band)
+        must = ora_idx[r][ora_score[r] > ora_score[r, -1] + 2 * band]
+        assert set(must.tolist()) <= set(e.tolist())
+        np.testing.assert_allclose(gpu_gate[r].sum(), 1.0, atol=1e-5)
+    return int(exact.sum()), int(near.sum())

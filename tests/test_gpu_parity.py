@@ -1,0 +1,361 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle.
+
+Each stage is fed the oracle's own inputs (logits, routing, schedule) so errors
+do not compound; the fused call is then compared end to end.  Large
+configurations run the oracle on a seeded sub-batch of tokens (rows of x; the
+layer is row-independent) and, at full size, check sampled rows plus
+properties that hold at any size.
+
+Bars: integer outputs bit-exact (selected ids except reported near-ties, the
+task permutation, unique ids, group boundaries); y within
+max|dy| / max|y| <= 1e-4 (fp32 storage) or 2e-2 (bf16 storage, fp32
+accumulation); gates/scores within fp32 rounding of the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import atomic_expert_routing_b200 as omni
+import oracle as O
+import workloads as WL
+from helpers import check_selection, dev, host_f64, rel_err, tol_y
+
+pytestmark = pytest.mark.gpu
+
+ALL = [WL.TINY, WL.BF16_16K, WL.SKEWED, WL.PREFILL, WL.DECODE]
+IDS = [c.name for c in ALL]
+SUB = {WL.TINY.name: 128, WL.BF16_16K.name: 4096, WL.SKEWED.name: 1024,
+       WL.PREFILL.name: 512, WL.DECODE.name: 64}
+
+_HOST_R, _HOST_E, _DEV_R, _DEV_E = {}, {}, {}, {}
+
+
+def _keys(cfg):
+    return ((cfg.seed, cfg.L, cfg.d, cfg.Nr, cfg.Nc, cfg.dtype, cfg.zipf_s),
+            (cfg.seed, cfg.Nr, cfg.Nc, cfg.d, cfg.dtype))
+
+
+def host_inputs(cfg):
+    """Seeded inputs, cached for the session (experts shared by configs with equal N, d)."""
+    kr, ke = _keys(cfg)
+    if kr not in _HOST_R:
+        _HOST_R[kr] = WL.make_inputs(cfg, experts=False)
+    if ke not in _HOST_E:
+        _HOST_E[ke] = WL.make_experts(cfg)
+    return dict(_HOST_R[kr], **_HOST_E[ke])
+
+
+def dev_inputs(cfg):
+    kr, ke = _keys(cfg)
+    h = host_inputs(cfg)
+    if kr not in _DEV_R:
+        _DEV_R[kr] = {k: dev(h[k]) for k in ("x", "Wr", "Wc", "bias_r", "bias_c")}
+    if ke not in _DEV_E:
+        _DEV_E[ke] = {k: dev(h[k]) for k in ("W", "V")}
+    return dict(_DEV_R[kr], **_DEV_E[ke])
+
+
+def sub_batch(cfg, n=None):
+    """A seeded sub-batch of tokens as its own batch: (cfg_s, host inputs, device inputs)."""
+    n = SUB[cfg.name] if n is None else n
+    h = host_inputs(cfg)
+    d = dev_inputs(cfg)
+    if n >= cfg.L:
+        return cfg, h, d
+    tok = WL.sample_tokens(cfg, n)
+    hs = dict(h, x=np.ascontiguousarray(h["x"][tok]))
+    ds = dict(d, x=d["x"][torch.from_numpy(tok).to(d["x"].device)].contiguous())
+    return cfg.with_(L=n), hs, ds
+
+
+def oracle_route_full(cfg, h):
+    lr, lc = O.axis_logprobs(cfg, h)
+    idx, gate, score = O.select(cfg, lr, lc)
+    bi, bg, bs, nxt = O.select_bruteforce(cfg, lr, lc)
+    assert np.array_equal(idx, bi)
+    return idx, gate, score, nxt, lr, lc
+
+
+# --------------------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_router_logits(cfg):
+    """Router projections (tcgen05 for bf16, CUDA cores for fp32) vs the oracle's
+    fp64 logits; error bound: fp32 accumulation of d exact products,
+    |dz| <= 2 d 2^-24 sum|x_m w_m|."""
+    cs, h, d = sub_batch(cfg, min(SUB[cfg.name], 512))
+    D = omni.LayerDims.of(cs)
+    z = omni.router_logits(D, d["x"], d["Wr"], d["Wc"]).cpu().numpy().astype(np.float64)
+    hb = dict(h, bias_r=None, bias_c=None)
+    zr, zc = O.axis_logits(cs, hb)
+    ref = np.concatenate([zr, zc], axis=1)
+    f = (lambda a: WL.bf16_bits_to_f32(a)) if cs.dtype == WL.BF16 else (lambda a: a)
+    xa = np.abs(f(h["x"]).astype(np.float64))
+    wa = np.abs(np.concatenate([f(h["Wr"]), f(h["Wc"])]).astype(np.float64))
+    bound = 2 * cs.d * 2.0 ** -24 * (xa @ wa.T) + 1e-30
+    err = np.abs(z - ref)
+    assert np.all(err <= bound), f"max err/bound {np.max(err / bound):.3g}"
+    assert np.median(err / bound) < 0.05
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_route_select_from_oracle_logits(cfg):
+    """Selection kernel alone: fed the oracle's logits rounded to fp32; compared
+    with the oracle's selection from the same fp32 logits."""
+    cs, h, _ = sub_batch(cfg)
+    zr, zc = O.axis_logits(cs, h)  # biases included
+    z32 = np.concatenate([zr, zc], axis=1).astype(np.float32)
+    D = omni.LayerDims.of(cs)
+    idx, gate, score = omni.route_select(D, dev(z32))
+    lr = O.log_softmax(z32[:, :cs.Nr].astype(np.float64))
+    lc = O.log_softmax(z32[:, cs.Nr:].astype(np.float64))
+    oi, og, os_ = O.select(cs, lr, lc)
+    _, _, bs, nxt = O.select_bruteforce(cs, lr, lc)
+    ne, nn = check_selection(cs, idx.cpu().numpy(), gate.cpu().numpy(), score.cpu().numpy(),
+                             oi, og, os_, nxt, lr, lc)
+    assert ne > 0.7 * cs.L
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_route_end_to_end(cfg):
+    cs, h, d = sub_batch(cfg)
+    D = omni.LayerDims.of(cs)
+    idx, gate, score = omni.route(D, d["x"], d["Wr"], d["Wc"], d["bias_r"], d["bias_c"])
+    oi, og, os_, nxt, lr, lc = oracle_route_full(cs, h)
+    ne, nn = check_selection(cs, idx.cpu().numpy(), gate.cpu().numpy(), score.cpu().numpy(),
+                             oi, og, os_, nxt, lr, lc)
+    assert ne > 0.7 * cs.L
+
+
+def test_route_simt_diagnostic_path_matches_tensor_cores():
+    cfg = WL.BF16_16K
+    cs, h, d = sub_batch(cfg, 1024)
+    D = omni.LayerDims.of(cs)
+    Ds = omni.LayerDims.of(cs, flags=omni.OMNI_FLAG_ROUTER_SIMT)
+    z_tc = omni.router_logits(D, d["x"], d["Wr"], d["Wc"])
+    z_simt = omni.router_logits(Ds, d["x"], d["Wr"], d["Wc"])
+    assert torch.allclose(z_tc, z_simt, rtol=0, atol=1e-4)
+    oi, og, os_, nxt, lr, lc = oracle_route_full(cs, h)
+    idx, gate, score = omni.route(Ds, d["x"], d["Wr"], d["Wc"])
+    check_selection(cs, idx.cpu().numpy(), gate.cpu().numpy(), score.cpu().numpy(), oi, og, os_,
+                    nxt, lr, lc)
+
+
+# --------------------------------------------------------------------------- schedule
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_schedule_from_oracle_routing(cfg):
+    """Scheduler fed the oracle's routing: bit-exact task order, unique ids,
+    group boundaries and counts."""
+    cs, h, _ = sub_batch(cfg, min(cfg.L, 2048))
+    oi, og, _ = O.route(cs, h)
+    g32 = og.astype(np.float32)
+    ref = O.schedule(cs, oi, g32.astype(np.float64))
+    D = omni.LayerDims.of(cs)
+    s = omni.schedule(D, dev(oi), dev(g32))
+    cnt = s["counts"].cpu().numpy()
+    assert cnt[0] == ref["n_active"] and cnt[1] == ref["n_groups"] and cnt[2] == 0
+    np.testing.assert_array_equal(s["task_token"].cpu().numpy(), ref["task_token"])
+    np.testing.assert_array_equal(s["task_expert"].cpu().numpy(), ref["task_expert"])
+    np.testing.assert_array_equal(s["task_gate"].cpu().numpy(), ref["task_gate"].astype(np.float32))
+    np.testing.assert_array_equal(s["uniq"].cpu().numpy()[:cnt[0]], ref["uniq"])
+    np.testing.assert_array_equal(s["group_off"].cpu().numpy()[:cnt[1] + 1], ref["group_off"])
+
+
+@pytest.mark.parametrize("B", [1, 3, 10 ** 6])
+def test_schedule_group_size_extremes(B):
+    cfg = WL.TINY.with_(B=B)
+    h = host_inputs(WL.TINY)
+    oi, og, _ = O.route(cfg, h)
+    g32 = og.astype(np.float32)
+    ref = O.schedule(cfg, oi, g32.astype(np.float64))
+    s = omni.schedule(omni.LayerDims.of(cfg), dev(oi), dev(g32))
+    cnt = s["counts"].cpu().numpy()
+    assert cnt[1] == ref["n_groups"]
+    np.testing.assert_array_equal(s["task_expert"].cpu().numpy(), ref["task_expert"])
+    np.testing.assert_array_equal(s["task_token"].cpu().numpy(), ref["task_token"])
+    np.testing.assert_array_equal(s["group_off"].cpu().numpy()[:cnt[1] + 1], ref["group_off"])
+
+
+def test_schedule_bad_index_sets_status():
+    cfg = WL.TINY
+    h = host_inputs(cfg)
+    oi, og, _ = O.route(cfg, h)
+    oi = oi.copy()
+    oi[3, 2] = cfg.N + 5
+    s = omni.schedule(omni.LayerDims.of(cfg), dev(oi), dev(og.astype(np.float32)))
+    torch.cuda.synchronize()
+    assert int(s["counts"][2].item()) & omni._lib.OMNI_DEV_BAD_INDEX
+
+
+# --------------------------------------------------------------------------- execution
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_expert_forward_from_oracle_schedule(cfg):
+    cs, h, d = sub_batch(cfg)
+    oi, og, _ = O.route(cs, h)
+    g32 = og.astype(np.float32)
+    ref_s = O.schedule(cs, oi, g32.astype(np.float64))
+    y_ref, rows = O.forward_expert(cs, h, ref_s)
+    D = omni.LayerDims.of(cs)
+    M = cs.L * cs.K
+    counts = torch.tensor([ref_s["n_active"], ref_s["n_groups"], 0, 0], dtype=torch.int32,
+                          device="cuda")
+    sched = {"task_token": dev(ref_s["task_token"]), "task_expert": dev(ref_s["task_expert"]),
+             "task_gate": dev(ref_s["task_gate"].astype(np.float32)),
+             "uniq": dev(ref_s["uniq"]), "group_off": dev(ref_s["group_off"]), "counts": counts}
+    assert sched["task_token"].numel() == M
+    y = omni.expert_forward(D, d["x"], d["W"], d["V"], sched)
+    err = rel_err(host_f64(y), y_ref)
+    assert err <= tol_y(cs), err
+    assert int(counts[2].item()) == 0
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_token_centric_from_oracle_routing(cfg):
+    cs, h, d = sub_batch(cfg)
+    oi, og, _ = O.route(cs, h)
+    g32 = og.astype(np.float32)
+    y_ref, _ = O.forward_token(cs, h, oi, g32.astype(np.float64))
+    y = omni.token_centric_forward(omni.LayerDims.of(cs), d["x"], d["W"], d["V"], dev(oi),
+                                   dev(g32))
+    err = rel_err(host_f64(y), y_ref)
+    assert err <= tol_y(cs), err
+
+
+@pytest.mark.parametrize("cfg", ALL, ids=IDS)
+def test_moe_forward_end_to_end(cfg):
+    """The fused call on a sub-batch: routing ids as in test_route_end_to_end and
+    y of every token whose ids match the oracle's."""
+    cs, h, d = sub_batch(cfg)
+    D = omni.LayerDims.of(cs)
+    idx = torch.empty((cs.L, cs.K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cs.L, cs.K), dtype=torch.float32, device="cuda")
+    counts = omni.new_counts("cuda")
+    y = omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"],
+                         counts=counts, idx=idx, gate=gate)
+    res = O.moe_forward(cs, h)
+    _, _, bs, nxt = O.select_bruteforce(cs, *O.axis_logprobs(cs, h))
+    gi = idx.cpu().numpy()
+    lr, lc = O.axis_logprobs(cs, h)
+    check_selection(cs, gi, gate.cpu().numpy(), None, res["idx"], res["gate"], res["score"], nxt,
+                    lr, lc)
+    same = np.all(gi == res["idx"], axis=1)
+    yg = host_f64(y)
+    assert rel_err(yg[same], res["y"][same]) <= tol_y(cs)
+    c = counts.cpu().numpy()
+    assert c[2] == 0
+    if same.all():
+        assert c[0] == res["sched"]["n_active"] and c[1] == res["sched"]["n_groups"]
+
+
+# ------------------------------------------------------------- full size (bench configuration)
+
+
+@pytest.mark.parametrize("cfg", [WL.SKEWED, WL.PREFILL, WL.DECODE], ids=lambda c: c.name)
+def test_full_size_fused_and_staged(cfg):
+    """The whole batch as the benchmark runs it: the fused call against the staged
+    calls, sampled rows against the oracle, and the schedule's defining
+    properties checked on its own input at full size."""
+    h = host_inputs(cfg)
+    d = dev_inputs(cfg)
+    D = omni.LayerDims.of(cfg)
+    idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
+    counts = omni.new_counts("cuda")
+    y = omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"],
+                         counts=counts, idx=idx, gate=gate)
+    # staged
+    i2, g2, _ = omni.route(D, d["x"], d["Wr"], d["Wc"], d["bias_r"], d["bias_c"])
+    assert torch.equal(i2, idx) and torch.equal(g2, gate)
+    s = omni.schedule(D, i2, g2)
+    y2 = omni.expert_forward(D, d["x"], d["W"], d["V"], s)
+    assert rel_err(host_f64(y2), host_f64(y)) <= 1e-2
+    # schedule properties at full size, from its input: sorted by (group, token, expert)
+    gi = i2.cpu().numpy().astype(np.int64)
+    U = np.unique(gi)
+    c = s["counts"].cpu().numpy()
+    assert c[0] == len(U) and c[1] == (len(U) + cfg.B - 1) // cfg.B and c[2] == 0
+    np.testing.assert_array_equal(s["uniq"].cpu().numpy()[:c[0]], U)
+    t = np.repeat(np.arange(cfg.L), cfg.K)
+    e = gi.reshape(-1)
+    grp = np.searchsorted(U, e) // cfg.B
+    order = np.lexsort((e, t, grp))
+    np.testing.assert_array_equal(s["task_token"].cpu().numpy(), t[order])
+    np.testing.assert_array_equal(s["task_expert"].cpu().numpy(), e[order])
+    go = np.searchsorted(grp[order], np.arange(c[1] + 1))
+    go[-1] = len(e)
+    np.testing.assert_array_equal(s["group_off"].cpu().numpy()[:c[1] + 1], go)
+    # sampled rows against the oracle
+    tok = WL.sample_tokens(cfg, 128)
+    cs = cfg.with_(L=len(tok))
+    hs = dict(h, x=np.ascontiguousarray(h["x"][tok]))
+    res = O.moe_forward(cs, hs)
+    lr, lc = O.axis_logprobs(cs, hs)
+    _, _, _, nxt = O.select_bruteforce(cs, lr, lc)
+    gsub = gi[tok]
+    check_selection(cs, gsub, gate.cpu().numpy()[tok], None, res["idx"], res["gate"],
+                    res["score"], nxt, lr, lc)
+    same = np.all(gsub == res["idx"], axis=1)
+    assert same.mean() > 0.5
+    assert rel_err(host_f64(y)[tok][same], res["y"][same]) <= tol_y(cfg)
+
+
+# --------------------------------------------------------------------------- edge cases
+
+EDGE = [
+    WL.Config("ragged-bf16", L=130, d=72, Nr=48, Nc=80, k=5, K=7, B=4, dtype=WL.BF16, seed=11),
+    WL.Config("ragged-f32", L=37, d=40, Nr=12, Nc=20, k=3, K=9, B=2, dtype=WL.F32, seed=12),
+    WL.Config("single-token", L=1, d=64, Nr=16, Nc=16, k=4, K=4, B=3, dtype=WL.BF16, seed=13),
+    WL.Config("k1", L=200, d=128, Nr=32, Nc=64, k=1, K=1, B=5, dtype=WL.BF16, seed=14),
+    WL.Config("max-topk", L=64, d=64, Nr=4096, Nc=16, k=16, K=256, B=64, dtype=WL.BF16, seed=15),
+    WL.Config("wide-k", L=96, d=256, Nr=256, Nc=256, k=128, K=100, B=128, dtype=WL.BF16, seed=16),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=[c.name for c in EDGE])
+def test_edge_shapes(cfg):
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    D = omni.LayerDims.of(cfg)
+    idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
+    counts = omni.new_counts("cuda")
+    y = omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], counts=counts, idx=idx,
+                         gate=gate)
+    res = O.moe_forward(cfg, h)
+    lr, lc = O.axis_logprobs(cfg, h)
+    _, _, _, nxt = O.select_bruteforce(cfg, lr, lc)
+    gi = idx.cpu().numpy()
+    check_selection(cfg, gi, gate.cpu().numpy(), None, res["idx"], res["gate"], res["score"], nxt,
+                    lr, lc)
+    same = np.all(gi == res["idx"], axis=1)
+    assert rel_err(host_f64(y)[same], res["y"][same]) <= tol_y(cfg)
+    yt = omni.token_centric_forward(D, d["x"], d["W"], d["V"], idx, gate)
+    assert rel_err(host_f64(yt), host_f64(y)) <= tol_y(cfg)
+
+
+def test_equal_logits_pick_smallest_ids():
+    """x = 0: every joint score ties; the K smallest ids of the k x k grid win."""
+    cfg = WL.Config("ties", L=8, d=64, Nr=16, Nc=24, k=4, K=6, B=4, dtype=WL.BF16, seed=3)
+    h = WL.make_inputs(cfg)
+    h["x"] = np.zeros_like(h["x"])
+    d = {k: dev(v) for k, v in h.items()}
+    idx, gate, _ = omni.route(omni.LayerDims.of(cfg), d["x"], d["Wr"], d["Wc"])
+    want = sorted(i * cfg.Nc + j for i in range(cfg.k) for j in range(cfg.k))[:cfg.K]
+    assert np.all(idx.cpu().numpy() == np.array(want)[None, :])
+    np.testing.assert_allclose(gate.cpu().numpy(), 1.0 / cfg.K, rtol=1e-6)
+
+
+def test_empty_batch():
+    cfg = WL.TINY.with_(L=0)
+    D = omni.LayerDims.of(cfg)
+    x = torch.empty((0, cfg.d), device="cuda")
+    W = torch.zeros((cfg.N, cfg.d), device="cuda")
+    y = omni.moe_forward(D, x, torch.zeros((cfg.Nr, cfg.d), device="cuda"),
+                         torch.zeros((cfg.Nc, cfg.d), device="cuda"), W, W,
+                         y=torch.empty((0, cfg.d), device="cuda"))
+    assert y.shape == (0, cfg.d)

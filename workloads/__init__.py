@@ -137,9 +137,15 @@ def make_inputs(cfg: Config, experts: bool = True) -> dict:
         out["bias_r"] = zipf_bias(cfg.seed, _T_PERM_R, cfg.Nr, cfg.zipf_s)
         out["bias_c"] = zipf_bias(cfg.seed, _T_PERM_C, cfg.Nc, cfg.zipf_s)
     if experts:
-        out["W"] = _normal(cfg.seed, _T_W, (cfg.N, cfg.d), sc, cfg.dtype)
-        out["V"] = _normal(cfg.seed, _T_V, (cfg.N, cfg.d), sc, cfg.dtype)
+        out.update(make_experts(cfg))
     return out
+
+
+def make_experts(cfg: Config) -> dict:
+    """The expert matrices W, V [N x d] of ``cfg`` (they depend on seed, N, d, dtype only)."""
+    sc = 1.0 / np.sqrt(cfg.d)
+    return {"W": _normal(cfg.seed, _T_W, (cfg.N, cfg.d), sc, cfg.dtype),
+            "V": _normal(cfg.seed, _T_V, (cfg.N, cfg.d), sc, cfg.dtype)}
 
 
 def sample_tokens(cfg: Config, n: int, seed: int = 1234) -> np.ndarray:
