@@ -33,6 +33,7 @@ _I64 = C.c_int64
 SIGNATURES = {
     "omni_abi_version": ([], C.c_int),
     "omni_status_string": ([C.c_int], C.c_char_p),
+    "omni_last_cuda_error_name": ([], C.c_char_p),
     "omni_workspace_size": ([_P, C.c_int, C.POINTER(C.c_size_t)], C.c_int),
     "omni_route": ([_P] * 11 + [C.c_size_t, _P], C.c_int),
     "omni_route_select": ([_P] * 9 + [C.c_size_t, _P], C.c_int),
@@ -73,6 +74,8 @@ def load(path: str = LIB_PATH):
 class OmniError(RuntimeError):
     def __init__(self, fn: str, code: int):
         msg = load().omni_status_string(code).decode()
+        if code == OMNI_ERR_CUDA:
+            msg += f" [{load().omni_last_cuda_error_name().decode()}]"
         super().__init__(f"{fn} failed: {msg} (code {code})")
         self.code = code
 

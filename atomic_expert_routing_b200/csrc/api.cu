@@ -82,7 +82,14 @@ int ws_ok(const Dims& D, int which, const void* ws, size_t ws_bytes) {
   return OMNI_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA; }
+// last failing CUDA call of this host thread (diagnostics only)
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return OMNI_OK;
+  g_last_cuda = e;
+  return OMNI_ERR_CUDA;
+}
 
 int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, const float* br,
                const float* bc, int32_t* idx, float* gate, float* score, int32_t* status,
@@ -92,7 +99,7 @@ int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, con
     e = omni::launch_router_tc(D, x, Wr, Wc, Z, status, s);
   else
     e = omni::launch_router_simt(D, x, Wr, Wc, Z, s);
-  if (e != cudaSuccess) return OMNI_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(omni::launch_select(D, Z, br, bc, idx, gate, score, s));
 }
 
@@ -107,6 +114,8 @@ bool tensors_ok(const void* const* p16, int n16) {
 extern "C" {
 
 int omni_abi_version(void) { return OMNI_ABI_VERSION; }
+
+const char* omni_last_cuda_error_name(void) { return cudaGetErrorName(g_last_cuda); }
 
 const char* omni_status_string(int status) {
   switch (status) {
@@ -229,9 +238,9 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   float* gate = gate_out ? gate_out : w.gate;
   rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s);
   if (rc != OMNI_OK) return rc;
-  if (omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate, w.uniq,
-                            w.group_off, counts, w.sched, s) != cudaSuccess)
-    return OMNI_ERR_CUDA;
+  rc = cuda_status(omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate,
+                                         w.uniq, w.group_off, counts, w.sched, s));
+  if (rc != OMNI_OK) return rc;
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
                                          w.group_off, counts, y, w.expert, s));
 }

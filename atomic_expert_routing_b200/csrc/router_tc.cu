@@ -169,12 +169,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (mbar_wait(accum, 0, status)) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int64_t grow = static_cast<int64_t>(m0) + warp * 32 + lane;
+      const bool vec_ok = (ld % 4 == 0) && (zc0 % 4 == 0);  // 16-byte aligned rows
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
         if (grow < L) {
           float* zp = Z + grow * ld + zc0 + c;
-          if (n0 + c + 32 <= naxis) {
+          if (n0 + c + 32 <= naxis && vec_ok) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
               *reinterpret_cast<float4*>(zp + j) =

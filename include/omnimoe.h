@@ -187,6 +187,10 @@ int omni_token_centric_forward(const omni_dims* dims, const void* x, const void*
 /* Static description of a status code (never NULL). */
 const char* omni_status_string(int status);
 
+/* Name of the CUDA error behind the last OMNI_ERR_CUDA returned on this host
+ * thread ("cudaSuccess" if none); a static string. */
+const char* omni_last_cuda_error_name(void);
+
 /* OMNI_ABI_VERSION of the loaded library. */
 int omni_abi_version(void);
 

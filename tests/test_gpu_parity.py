@@ -243,7 +243,7 @@ def test_moe_forward_end_to_end(cfg):
     lr, lc = O.axis_logprobs(cs, h)
     check_selection(cs, gi, gate.cpu().numpy(), None, res["idx"], res["gate"], res["score"], nxt,
                     lr, lc)
-    same = np.all(gi == res["idx"], axis=1)
+    same = np.all(np.sort(gi, 1) == np.sort(res["idx"], 1), axis=1)
     yg = host_f64(y)
     assert rel_err(yg[same], res["y"][same]) <= tol_y(cs)
     c = counts.cpu().numpy()
@@ -299,7 +299,7 @@ def test_full_size_fused_and_staged(cfg):
     gsub = gi[tok]
     check_selection(cs, gsub, gate.cpu().numpy()[tok], None, res["idx"], res["gate"],
                     res["score"], nxt, lr, lc)
-    same = np.all(gsub == res["idx"], axis=1)
+    same = np.all(np.sort(gsub, 1) == np.sort(res["idx"], 1), axis=1)
     assert same.mean() > 0.5
     assert rel_err(host_f64(y)[tok][same], res["y"][same]) <= tol_y(cfg)
 
@@ -332,7 +332,7 @@ def test_edge_shapes(cfg):
     gi = idx.cpu().numpy()
     check_selection(cfg, gi, gate.cpu().numpy(), None, res["idx"], res["gate"], res["score"], nxt,
                     lr, lc)
-    same = np.all(gi == res["idx"], axis=1)
+    same = np.all(np.sort(gi, 1) == np.sort(res["idx"], 1), axis=1)
     assert rel_err(host_f64(y)[same], res["y"][same]) <= tol_y(cfg)
     yt = omni.token_centric_forward(D, d["x"], d["W"], d["V"], idx, gate)
     assert rel_err(host_f64(yt), host_f64(y)) <= tol_y(cfg)
