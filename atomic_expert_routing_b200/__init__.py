@@ -132,13 +132,15 @@ def route(D: LayerDims, x, Wr, Wc, bias_r=None, bias_c=None, *, counts=None, ws=
     return idx, gate, score
 
 
-def router_logits(D: LayerDims, x, Wr, Wc, *, counts=None, stream=None):
+def router_logits(D: LayerDims, x, Wr, Wc, *, counts=None, ws=None, stream=None):
     """Router projections: float32 [L, Nr + Nc] (row logits, then column logits)."""
     dev = _device(x)
     z = torch.empty((D.L, D.Nr + D.Nc), dtype=torch.float32, device=dev)
+    wsp, n = _ws(D, OMNI_WS_ROUTE, dev, ws)
     dd = D.c()
     _lib.check("omni_router_logits", _lib.load().omni_router_logits(
-        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(z), _ptr(counts), _stream(stream)))
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(z), _ptr(counts), wsp, n,
+        _stream(stream)))
     return z
 
 

@@ -37,7 +37,7 @@ SIGNATURES = {
     "omni_workspace_size": ([_P, C.c_int, C.POINTER(C.c_size_t)], C.c_int),
     "omni_route": ([_P] * 11 + [C.c_size_t, _P], C.c_int),
     "omni_route_select": ([_P] * 9 + [C.c_size_t, _P], C.c_int),
-    "omni_router_logits": ([_P] * 7, C.c_int),
+    "omni_router_logits": ([_P] * 7 + [C.c_size_t, _P], C.c_int),
     "omni_schedule": ([_P] * 10 + [C.c_size_t, _P], C.c_int),
     "omni_expert_forward": ([_P] * 12 + [C.c_size_t, _P], C.c_int),
     "omni_moe_forward": ([_P] * 13 + [C.c_size_t, _P], C.c_int),

@@ -36,7 +36,7 @@ struct RouteWs {
 };
 RouteWs carve_route(const Dims& D, Carver& c) {
   RouteWs w;
-  w.Z = c.take<float>(static_cast<size_t>(D.L) * (D.Nr + D.Nc));
+  w.Z = c.take<float>(static_cast<size_t>(omni::router_splits(D)) * D.L * (D.Nr + D.Nc));
   return w;
 }
 
@@ -95,12 +95,15 @@ int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, con
                const float* bc, int32_t* idx, float* gate, float* score, int32_t* status,
                float* Z, cudaStream_t s) {
   cudaError_t e;
-  if (omni::router_tc_supported(D, x, Wr, Wc))
+  int parts = 1;
+  if (omni::router_tc_supported(D, x, Wr, Wc)) {
     e = omni::launch_router_tc(D, x, Wr, Wc, Z, status, s);
-  else
+    parts = omni::router_splits(D);
+  } else {
     e = omni::launch_router_simt(D, x, Wr, Wc, Z, s);
+  }
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(omni::launch_select(D, Z, br, bc, idx, gate, score, s));
+  return cuda_status(omni::launch_select(D, Z, parts, br, bc, idx, gate, score, s));
 }
 
 bool tensors_ok(const void* const* p16, int n16) {
@@ -154,7 +157,7 @@ int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void*
 }
 
 int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
-                       float* logits, int32_t* counts, void* stream) {
+                       float* logits, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -162,9 +165,20 @@ int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, con
   const void* t16[] = {x, Wr, Wc, logits};
   if (!tensors_ok(t16, 4)) return OMNI_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = omni::router_tc_supported(D, x, Wr, Wc)
-                      ? omni::launch_router_tc(D, x, Wr, Wc, logits, counts ? counts + 2 : nullptr, s)
-                      : omni::launch_router_simt(D, x, Wr, Wc, logits, s);
+  if (!omni::router_tc_supported(D, x, Wr, Wc))
+    return cuda_status(omni::launch_router_simt(D, x, Wr, Wc, logits, s));
+  const int parts = omni::router_splits(D);
+  if (parts > 1 && (ws == nullptr || !al(ws, 256) ||
+                    ws_bytes < static_cast<size_t>(parts) * D.L * (D.Nr + D.Nc) * sizeof(float)))
+    return OMNI_ERR_WORKSPACE;
+  float* Z = parts > 1 ? static_cast<float*>(ws) : logits;
+  cudaError_t e = omni::launch_router_tc(D, x, Wr, Wc, Z, counts ? counts + 2 : nullptr, s);
+  if (e == cudaSuccess && parts > 1) {
+    e = omni::launch_sum_partials(Z, parts, D.L * (D.Nr + D.Nc), s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(logits, Z, static_cast<size_t>(D.L) * (D.Nr + D.Nc) * sizeof(float),
+                          cudaMemcpyDeviceToDevice, s);
+  }
   return cuda_status(e);
 }
 
@@ -180,7 +194,7 @@ int omni_route_select(const omni_dims* dims, const float* logits, const float* b
   if (D.L == 0) return OMNI_OK;
   if (logits == nullptr || !al(logits, 16) || idx == nullptr || gate == nullptr)
     return OMNI_ERR_INVALID_ARG;
-  return cuda_status(omni::launch_select(D, logits, bias_r, bias_c, idx, gate, score,
+  return cuda_status(omni::launch_select(D, logits, 1, bias_r, bias_c, idx, gate, score,
                                          static_cast<cudaStream_t>(stream)));
 }
 

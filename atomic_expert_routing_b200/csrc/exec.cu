@@ -30,9 +30,7 @@
 namespace omni {
 namespace {
 
-constexpr int kExpWarps = 8;
-constexpr int kExpChunk = kExpWarps * 32;  // tasks scanned for pieces per step
-constexpr int kPieceMax = 16;              // tasks of one token per piece (one reduction)
+constexpr int kExpThreads = 128;  // 4 warps per CTA, each executing its own task slice
 
 // Elements per 16-byte vector.
 template <typename T> constexpr int kEpv = 16 / sizeof(T);
@@ -74,165 +72,279 @@ __device__ __forceinline__ uint4 pack_vec(const float* a, float*) {
 }
 
 // Grouped execution over the schedule, taken as one task list in schedule
-// order (group after group; inside a group by token, then expert).  A CTA
-// scans chunks of kExpChunk consecutive tasks; a piece is a maximal stretch of
-// one token's tasks inside a chunk, at most kPieceMax long; each warp executes
-// pieces: x[t] is read once, every task reads W[e] and V[e] (a group's rows
-// come from HBM once and are re-read by its other pieces from L2), and the
-// piece adds its sum g*SiLU(x[t].W[e])*V[e] to the fp32 row y[t] with 16-byte
-// vector reductions.  NV > 0: d = NV * 32 * (16 / sizeof(T)), x[t] lives in
-// registers; NV == 0: any d that is a multiple of 16 bytes, x[t] in shared
-// memory.  Every index read from memory is range-checked before it is used
-// (a bad one sets OMNI_DEV_BAD_INDEX and the task is skipped).
+// order (group after group; inside a group by token, then expert).  Warp w
+// owns the slice of S consecutive tasks [w*S, (w+1)*S); inside its slice a
+// piece is a maximal stretch of one token's tasks.  For every piece the warp
+// reads x[t] once, and for every task of the piece the rows W[e] and V[e]
+// (issued together; a group's rows come from HBM once and are re-read by its
+// other pieces from L2 while the group is in flight), computes
+// c = g * SiLU(x[t] . W[e]) and accumulates c * V[e] in registers; the piece
+// then adds its d-vector to the fp32 row y[t] with 16-byte vector reductions.
+// NV > 0: d = NV * 32 * (16 / sizeof(T)), x[t] held in registers; NV == 0: any
+// d that is a multiple of 16 bytes (x[t] streamed from L2 per task).  Every
+// index read from memory is range-checked before use (a bad one sets
+// OMNI_DEV_BAD_INDEX and the task is skipped).  All warp shuffles sit at
+// warp-uniform points.
 template <typename T, int NV>
-__global__ void __launch_bounds__(kExpWarps * 32)
-    k_expert_pieces(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
+__global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
+    k_expert_slices(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
                     const int32_t* __restrict__ task_token,
                     const int32_t* __restrict__ task_expert,
                     const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
-                    float* __restrict__ yacc, int32_t* status) {
+                    int S, float* __restrict__ yacc, int32_t* status) {
   constexpr int EPV = kEpv<T>;
-  extern __shared__ __align__(16) uint8_t smem[];  // NV == 0: kExpWarps rows of x
-  __shared__ int pstart[kExpChunk + 1];
-  __shared__ int wcnt[kExpWarps];
-  __shared__ int npieces;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nvec = d / EPV;  // 16-byte vectors per row
-  uint4* xs = reinterpret_cast<uint4*>(smem) + static_cast<size_t>(warp) * nvec;
-  const int64_t nchunks = (M + kExpChunk - 1) / kExpChunk;
-  for (int64_t ch = blockIdx.x; ch < nchunks; ch += gridDim.x) {
-    const int64_t c0 = ch * kExpChunk;
-    const int64_t c1 = (M - c0 < kExpChunk) ? M : c0 + kExpChunk;
-    {
-      const int64_t i = c0 + threadIdx.x;
-      bool st = false;
-      if (i < c1) {
-        const int64_t off = i - c0;
-        st = (off == 0) || task_token[i] != task_token[i - 1];
-        if (!st) {
-          // cut a long run every kPieceMax tasks (counted from the run start)
-          int64_t k0 = i - 1;
-          while (k0 > c0 && task_token[k0 - 1] == task_token[i]) --k0;
-          st = ((i - k0) % kPieceMax) == 0;
-        }
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t a0 = wid * S;
+  if (a0 >= M) return;  // whole warp
+  const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
+  const int nvec = d / EPV;
+  // one task per lane (S <= 32): token, expert, gate
+  int64_t my_t = -1, my_e = -1;
+  float my_g = 0.0f;
+  if (lane < n) {
+    my_t = task_token[a0 + lane];
+    my_e = task_expert[a0 + lane];
+    my_g = task_gate[a0 + lane];
+    if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
+      raise_status(status, OMNI_DEV_BAD_INDEX);
+      my_e = -1;
+    }
+  }
+  const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
+  const bool start = lane < n && (lane == 0 || prev_t != my_t);
+  uint32_t starts = __ballot_sync(0xffffffffu, start);
+  while (starts) {
+    const int p = __ffs(starts) - 1;
+    starts &= starts - 1;
+    const int q = starts ? __ffs(starts) - 1 : n;  // piece = lanes [p, q)
+    const int64_t t = __shfl_sync(0xffffffffu, my_t, p);
+    if (t < 0 || t >= L) continue;  // warp-uniform
+    float* yr = yacc + t * d;
+    if constexpr (NV > 0) {
+      const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+      uint4 xv[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) xv[v] = xr[v * 32 + lane];
+      float acc[NV * EPV];
+#pragma unroll
+      for (int u = 0; u < NV * EPV; ++u) acc[u] = 0.0f;
+      for (int j = p; j < q; ++j) {
+        const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+        const float gj = __shfl_sync(0xffffffffu, my_g, j);
+        if (e < 0) continue;  // warp-uniform
+        const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
+        const uint4* vr = reinterpret_cast<const uint4*>(V + e * d);
+        uint4 wv[NV], vv[NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) wv[v] = wr[v * 32 + lane];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) vv[v] = vr[v * 32 + lane];
+        float s = 0.0f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) s += dot_vec(xv[v], wv[v], static_cast<T*>(nullptr));
+        s = warp_sum(s);
+        const float c = gj * silu(s);
+#pragma unroll
+        for (int v = 0; v < NV; ++v) axpy_vec(c, vv[v], acc + v * EPV, static_cast<T*>(nullptr));
       }
-      const uint32_t m = __ballot_sync(0xffffffffu, st);
-      if (lane == 0) wcnt[warp] = __popc(m);
-      __syncthreads();
-      int wbase = 0;
-      for (int w = 0; w < warp; ++w) wbase += wcnt[w];
-      const int pos = wbase + __popc(m & lanemask_lt());
-      if (st && pos < kExpChunk) pstart[pos] = static_cast<int>(i - c0);
-      if (threadIdx.x == kExpChunk - 1) {
-        const int n = wbase + __popc(m);
-        npieces = n;
-        pstart[n < kExpChunk ? n : kExpChunk] = static_cast<int>(c1 - c0);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        float* o = yr + static_cast<int64_t>(v * 32 + lane) * EPV;
+#pragma unroll
+        for (int u = 0; u < EPV; u += 4)
+          red_add_v4(o + u, acc[v * EPV + u], acc[v * EPV + u + 1], acc[v * EPV + u + 2],
+                     acc[v * EPV + u + 3]);
+      }
+    } else {
+      // generic d: activations first (x re-read from L2 per task), then the
+      // value rows vector block by vector block; trip counts are warp-uniform
+      const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+      float my_c = 0.0f;
+      for (int j = p; j < q; ++j) {
+        const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+        float sacc = 0.0f;
+        if (e >= 0) {  // warp-uniform; no shuffle inside
+          const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
+          for (int v = lane; v < nvec; v += 32) sacc += dot_vec(xr[v], wr[v], static_cast<T*>(nullptr));
+        }
+        sacc = warp_sum(sacc);
+        const float gj = __shfl_sync(0xffffffffu, my_g, j);
+        if (lane == j) my_c = (e >= 0) ? gj * silu(sacc) : 0.0f;
+      }
+      for (int v0 = 0; v0 < nvec; v0 += 32) {
+        const int v = v0 + lane;
+        const bool act = v < nvec;
+        float acc[EPV];
+#pragma unroll
+        for (int u = 0; u < EPV; ++u) acc[u] = 0.0f;
+        for (int j = p; j < q; ++j) {
+          const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+          const float c = __shfl_sync(0xffffffffu, my_c, j);
+          if (!act || e < 0) continue;
+          axpy_vec(c, reinterpret_cast<const uint4*>(V + e * d)[v], acc, static_cast<T*>(nullptr));
+        }
+        if (act) {
+#pragma unroll
+          for (int u = 0; u < EPV; u += 4)
+            red_add_v4(yr + static_cast<int64_t>(v) * EPV + u, acc[u], acc[u + 1], acc[u + 2],
+                       acc[u + 3]);
+        }
       }
     }
-    __syncthreads();
-    const int np = npieces;
-    for (int p = warp; p < np; p += kExpWarps) {
-      const int pa = pstart[p], pb = pstart[p + 1];
-      if (pa < 0 || pb > kExpChunk || pa >= pb) {
-        if (lane == 0) raise_status(status, OMNI_DEV_BAD_INDEX);
-        continue;
+  }
+}
+
+// L2 eviction policies (createpolicy): rows of W and V are streamed once
+// (evict first), the fp32 accumulator y is re-used by many pieces (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void red_add_v4_keep(float* addr, float a, float b, float c, float d,
+                                                uint64_t pol) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "l"(pol)
+               : "memory");
+}
+
+constexpr int kAsyncWarps = 8;
+
+// The same grouped execution as k_expert_slices for d = NV * 32 * (16 /
+// sizeof(T)), with the row traffic decoupled from the arithmetic: every warp
+// streams the W and V rows of its next R-1 tasks into its own shared-memory
+// ring with cp.async (each lane copies, and later reads, only its own 16-byte
+// vectors, so no cross-lane synchronisation is needed), prefetches x of the
+// next piece into registers one task ahead, and computes the current task
+// from shared memory.  Warps run a grid-stride loop over task slices; the
+// pipeline restarts at every slice.
+template <typename T, int NV, int R>
+__global__ void __launch_bounds__(kAsyncWarps * 32, 1)
+    k_expert_async(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
+                   const int32_t* __restrict__ task_token,
+                   const int32_t* __restrict__ task_expert,
+                   const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
+                   int S, int64_t nslices, float* __restrict__ yacc, int32_t* status) {
+  constexpr int EPV = kEpv<T>;
+  constexpr int SLOT = 2 * NV * 32;  // uint4 per ring slot: W vectors, then V vectors
+  extern __shared__ __align__(16) uint4 ring[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4* wring = ring + static_cast<size_t>(warp) * R * SLOT;
+  const uint32_t wring_s = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
+  const uint64_t pol_stream = policy_evict_first();
+  const uint64_t pol_keep = policy_evict_last();
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * kAsyncWarps;
+  for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kAsyncWarps + warp; sl < nslices; sl += nw) {
+    const int64_t a0 = sl * S;
+    const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
+    int64_t my_t = -1, my_e = -1;
+    float my_g = 0.0f;
+    if (lane < n) {
+      my_t = task_token[a0 + lane];
+      my_e = task_expert[a0 + lane];
+      my_g = task_gate[a0 + lane];
+      if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
+        raise_status(status, OMNI_DEV_BAD_INDEX);
+        my_e = -1;
+        my_t = -1;
       }
-      const int64_t a = c0 + pa, b = c0 + pb;
-      const int64_t t = task_token[a];
-      if (t < 0 || t >= L) {
-        if (lane == 0) raise_status(status, OMNI_DEV_BAD_INDEX);
-        continue;
-      }
-      const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
-      // this lane's task of the piece (pieces are <= kPieceMax <= 32 long)
-      int64_t my_e = -1;
-      float my_g = 0.0f;
-      if (lane < b - a) {
-        my_e = task_expert[a + lane];
-        my_g = task_gate[a + lane];
-        if (my_e < 0 || my_e >= N) {
-          raise_status(status, OMNI_DEV_BAD_INDEX);
-          my_e = -1;
-        }
-      }
-      const int nt = static_cast<int>(b - a);
-      if constexpr (NV > 0) {
-        uint4 xv[NV];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) xv[v] = xr[v * 32 + lane];
-        float acc[NV * EPV];
-#pragma unroll
-        for (int u = 0; u < NV * EPV; ++u) acc[u] = 0.0f;
-        for (int j = 0; j < nt; ++j) {
-          const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
-          const float gj = __shfl_sync(0xffffffffu, my_g, j);
-          if (e < 0 || e >= N) continue;  // warp-uniform
+    }
+    const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
+    const int64_t next_t = __shfl_down_sync(0xffffffffu, my_t, 1);
+    const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
+    const uint32_t ends = __ballot_sync(0xffffffffu, lane < n && (lane == n - 1 || next_t != my_t));
+
+    // issue the row copies of task j into slot j % R (one commit group per task)
+    auto issue = [&](int j) {
+      if (j < n) {
+        const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+        if (e >= 0) {
           const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
           const uint4* vr = reinterpret_cast<const uint4*>(V + e * d);
-          uint4 wv[NV], vv[NV];
+          const uint32_t base = wring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
 #pragma unroll
-          for (int v = 0; v < NV; ++v) wv[v] = wr[v * 32 + lane];
-#pragma unroll
-          for (int v = 0; v < NV; ++v) vv[v] = vr[v * 32 + lane];
-          float s = 0.0f;
-#pragma unroll
-          for (int v = 0; v < NV; ++v) s += dot_vec(xv[v], wv[v], static_cast<T*>(nullptr));
-          s = warp_sum(s);
-          const float c = gj * silu(s);
-#pragma unroll
-          for (int v = 0; v < NV; ++v) axpy_vec(c, vv[v], acc + v * EPV, static_cast<T*>(nullptr));
+          for (int v = 0; v < NV; ++v) {
+            cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, wr + v * 32 + lane, pol_stream);
+            cp_async16(base + static_cast<uint32_t>((NV + v) * 32 + lane) * 16u, vr + v * 32 + lane,
+                       pol_stream);
+          }
         }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int j = 0; j < R - 1; ++j) issue(j);
+
+    uint4 xc[NV], xn[NV];
+    {
+      const int64_t t0 = __shfl_sync(0xffffffffu, my_t, 0);
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (t0 < 0 ? 0 : t0) * d);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
+    }
+    float acc[NV * EPV];
+    for (int j = 0; j < n; ++j) {
+      issue(j + R - 1);
+      const bool st = (starts >> j) & 1u;
+      if (st) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) xc[v] = xn[v];
+#pragma unroll
+        for (int u = 0; u < NV * EPV; ++u) acc[u] = 0.0f;
+        // x of the next piece, one task ahead
+        const uint32_t later = starts & ~((2u << j) - 1u);
+        if (later) {
+          const int jn = __ffs(later) - 1;
+          const int64_t tn = __shfl_sync(0xffffffffu, my_t, jn);
+          const uint4* xr = reinterpret_cast<const uint4*>(x + (tn < 0 ? 0 : tn) * d);
+#pragma unroll
+          for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
+        }
+      }
+      cp_async_wait<R - 1>();
+      const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+      const float gj = __shfl_sync(0xffffffffu, my_g, j);
+      const int64_t t = __shfl_sync(0xffffffffu, my_t, j);
+      if (e >= 0) {  // warp-uniform
+        const uint4* slot = wring + (j % R) * SLOT;
+        float sdot = 0.0f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
+        sdot = warp_sum(sdot);
+        const float c = gj * silu(sdot);
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+          axpy_vec(c, slot[(NV + v) * 32 + lane], acc + v * EPV, static_cast<T*>(nullptr));
+      }
+      if (((ends >> j) & 1u) && t >= 0) {
         float* yr = yacc + t * d;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          float* q = yr + static_cast<int64_t>(v * 32 + lane) * EPV;
+          float* o = yr + static_cast<int64_t>(v * 32 + lane) * EPV;
 #pragma unroll
           for (int u = 0; u < EPV; u += 4)
-            red_add_v4(q + u, acc[v * EPV + u], acc[v * EPV + u + 1], acc[v * EPV + u + 2],
-                       acc[v * EPV + u + 3]);
+            red_add_v4_keep(o + u, acc[v * EPV + u], acc[v * EPV + u + 1], acc[v * EPV + u + 2],
+                            acc[v * EPV + u + 3], pol_keep);
         }
-      } else {
-        // generic d: x[t] in this warp's shared-memory row
-        for (int v = lane; v < nvec; v += 32) xs[v] = xr[v];
-        __syncwarp();
-        float my_c = 0.0f;
-        for (int j = 0; j < nt; ++j) {
-          const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
-          float s = 0.0f;
-          if (e >= 0 && e < N) {  // warp-uniform; the loop below holds no shuffle
-            const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
-            for (int v = lane; v < nvec; v += 32) s += dot_vec(xs[v], wr[v], static_cast<T*>(nullptr));
-          }
-          s = warp_sum(s);
-          if (lane == j) my_c = (e >= 0) ? my_g * silu(s) : 0.0f;
-        }
-        float* yr = yacc + t * d;
-        // the trip count is the same for every lane: the shuffles below need
-        // all 32 lanes; only the memory accesses are predicated
-        for (int v0 = 0; v0 < nvec; v0 += 32) {
-          const int v = v0 + lane;
-          const bool act = v < nvec;
-          float acc[EPV];
-#pragma unroll
-          for (int u = 0; u < EPV; ++u) acc[u] = 0.0f;
-          for (int j = 0; j < nt; ++j) {
-            const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
-            const float c = __shfl_sync(0xffffffffu, my_c, j);
-            if (!act || e < 0 || e >= N) continue;
-            const uint4* vr = reinterpret_cast<const uint4*>(V + e * d);
-            axpy_vec(c, vr[v], acc, static_cast<T*>(nullptr));
-          }
-          if (act) {
-#pragma unroll
-            for (int u = 0; u < EPV; u += 4)
-              red_add_v4(yr + static_cast<int64_t>(v) * EPV + u, acc[u], acc[u + 1], acc[u + 2],
-                         acc[u + 3]);
-          }
-        }
-        __syncwarp();
       }
     }
-    __syncthreads();
+    cp_async_wait<0>();
   }
 }
 
@@ -313,37 +425,61 @@ size_t expert_ws_bytes(const Dims& D) {
 }
 
 template <typename T, int NV>
-cudaError_t launch_pieces(const Dims& D, const void* x, const void* W, const void* V,
+cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* tt, const int32_t* te, const float* tg, float* acc,
                           int32_t* status, cudaStream_t s) {
-  const size_t smem = NV > 0 ? 0 : static_cast<size_t>(kExpWarps) * D.d * sizeof(T);
-  cudaError_t err = cudaFuncSetAttribute(k_expert_pieces<T, NV>,
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // slice length: about 16 warps per SM, at most 32 tasks (one per lane)
+  const int64_t M = D.M();
+  const int64_t want_warps = static_cast<int64_t>(sms) * 16;
+  int S = static_cast<int>((M + want_warps - 1) / want_warps);
+  S = S < 1 ? 1 : (S > 32 ? 32 : S);
+  const int64_t warps = (M + S - 1) / S;
+  const int64_t blocks = (warps + kExpThreads / 32 - 1) / (kExpThreads / 32);
+  k_expert_slices<T, NV><<<static_cast<unsigned>(blocks), kExpThreads, 0, s>>>(
+      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
+      M, D.L, D.N(), static_cast<int>(D.d), S, acc, status);
+  return cudaGetLastError();
+}
+
+template <typename T, int NV, int R>
+cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void* V,
+                         const int32_t* tt, const int32_t* te, const float* tg, float* acc,
+                         int32_t* status, cudaStream_t s) {
+  constexpr size_t smem = static_cast<size_t>(kAsyncWarps) * R * 2 * NV * 32 * 16;
+  cudaError_t err = cudaFuncSetAttribute(k_expert_async<T, NV, R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t nchunks = (D.M() + kExpChunk - 1) / kExpChunk;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
-  const unsigned grid = static_cast<unsigned>(nchunks < cap ? nchunks : cap);
-  k_expert_pieces<T, NV><<<grid, kExpWarps * 32, smem, s>>>(
-      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
-      D.M(), D.L, D.N(), static_cast<int>(D.d), acc, status);
+  const int64_t M = D.M();
+  const int64_t warps_all = static_cast<int64_t>(sms) * kAsyncWarps;
+  int S = static_cast<int>((M + warps_all - 1) / warps_all);
+  S = S < 1 ? 1 : (S > 32 ? 32 : S);
+  const int64_t nslices = (M + S - 1) / S;
+  int64_t blocks = (nslices + kAsyncWarps - 1) / kAsyncWarps;
+  if (blocks > sms) blocks = sms;  // persistent: one CTA per SM (shared-memory bound)
+  k_expert_async<T, NV, R><<<static_cast<unsigned>(blocks), kAsyncWarps * 32, smem, s>>>(
+      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg, M,
+      D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status);
   return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t dispatch_pieces(const Dims& D, const void* x, const void* W, const void* V,
+cudaError_t dispatch_slices(const Dims& D, const void* x, const void* W, const void* V,
                             const int32_t* tt, const int32_t* te, const float* tg, float* acc,
                             int32_t* status, cudaStream_t s) {
   constexpr int row = 32 * kEpv<T>;  // elements covered by one vector per lane
   switch (D.d == row * 8 ? 8 : D.d == row * 4 ? 4 : D.d == row * 2 ? 2 : D.d == row ? 1 : 0) {
-    case 8: return launch_pieces<T, 8>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 4: return launch_pieces<T, 4>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 2: return launch_pieces<T, 2>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 1: return launch_pieces<T, 1>(D, x, W, V, tt, te, tg, acc, status, s);
-    default: return launch_pieces<T, 0>(D, x, W, V, tt, te, tg, acc, status, s);
+    case 8: return launch_async<T, 8, 3>(D, x, W, V, tt, te, tg, acc, status, s);
+    case 4: return launch_async<T, 4, 4>(D, x, W, V, tt, te, tg, acc, status, s);
+    case 2: return launch_async<T, 2, 4>(D, x, W, V, tt, te, tg, acc, status, s);
+    case 1: return launch_async<T, 1, 4>(D, x, W, V, tt, te, tg, acc, status, s);
+    default: return launch_slices<T, 0>(D, x, W, V, tt, te, tg, acc, status, s);
   }
 }
 
@@ -359,8 +495,8 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   cudaError_t err = cudaMemsetAsync(acc, 0, ybytes, s);
   if (err != cudaSuccess) return err;
   int32_t* status = const_cast<int32_t*>(counts) + 2;
-  err = f32 ? dispatch_pieces<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
-            : dispatch_pieces<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
+  err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
+            : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
                                              status, s);
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;

@@ -21,12 +21,19 @@ struct Dims {
 cudaError_t launch_router_simt(const Dims& D, const void* x, const void* Wr, const void* Wc,
                                float* Z, cudaStream_t s);
 bool router_tc_supported(const Dims& D, const void* x, const void* Wr, const void* Wc);
+// Number of K-splits of the tensor-core router for these dims (1: no split).
+// Split partial logits are written to Z + s * L * (Nr + Nc), s < splits.
+int router_splits(const Dims& D);
 cudaError_t launch_router_tc(const Dims& D, const void* x, const void* Wr, const void* Wc,
                              float* Z, int32_t* status, cudaStream_t s);
+// Z[i] = sum over s < splits of Z[s * n + i] (fixed order), written in place.
+cudaError_t launch_sum_partials(float* Z, int splits, int64_t n, cudaStream_t s);
 
 // ---- selection: per-axis top-k, k x k merge, top-K, gate ----------------
-cudaError_t launch_select(const Dims& D, const float* Z, const float* br, const float* bc,
-                          int32_t* idx, float* gate, float* score, cudaStream_t s);
+// Z holds `parts` consecutive partial logit arrays, summed in order on load.
+cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
+                          const float* bc, int32_t* idx, float* gate, float* score,
+                          cudaStream_t s);
 
 // ---- scheduling ----------------------------------------------------------
 size_t schedule_ws_bytes(const Dims& D);

@@ -92,7 +92,7 @@ template <int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
                 const __grid_constant__ CUtensorMap tmBc, float* __restrict__ Z, int L, int Nr,
-                int Nc, int d, int tiles_r, int32_t* status) {
+                int Nc, int d, int tiles_r, int kper, int32_t* status) {
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
   constexpr uint32_t B_BYTES = BN * TC_BK * 2;
   extern __shared__ uint8_t smem_raw[];
@@ -114,7 +114,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int naxis = colax ? Nc : Nr;
   const int64_t ld = static_cast<int64_t>(Nr) + Nc;
   const int zc0 = (colax ? Nr : 0) + n0;
-  const int nk = (d + TC_BK - 1) / TC_BK;
+  // K range of this CTA; with a split K loop (gridDim.z > 1) every split
+  // writes its own partial logits, Z + blockIdx.z * L * (Nr + Nc)
+  const int nk_all = (d + TC_BK - 1) / TC_BK;
+  const int kb0 = static_cast<int>(blockIdx.z) * kper;
+  const int nk = (nk_all - kb0 < kper ? nk_all - kb0 : kper);
+  Z += static_cast<int64_t>(blockIdx.z) * L * (static_cast<int64_t>(Nr) + Nc);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
@@ -144,8 +149,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t ph = (kb / TC_STAGES) & 1;
       if (!mbar_wait(empty0 + 8 * s, ph ^ 1, status)) break;
       mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES);
-      tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, full0 + 8 * s, kb * TC_BK, m0);
-      tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, kb * TC_BK, n0);
+      tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, full0 + 8 * s, (kb0 + kb) * TC_BK, m0);
+      tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, (kb0 + kb) * TC_BK, n0);
     }
   } else if (warp == 5 && lane == 0) {
     // MMA issuer
@@ -166,7 +171,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     umma_commit(accum);
   } else if (warp < 4) {
     // epilogue: TMEM lane (32*warp + lane) holds row m0 + 32*warp + lane
-    if (mbar_wait(accum, 0, status)) {
+    // the wait's outcome is made warp-uniform: tcgen05.ld below is .sync.aligned
+    if (__all_sync(0xffffffffu, mbar_wait(accum, 0, status))) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int64_t grow = static_cast<int64_t>(m0) + warp * 32 + lane;
       const bool vec_ok = (ld % 4 == 0) && (zc0 % 4 == 0);  // 16-byte aligned rows
@@ -245,14 +251,49 @@ cudaError_t launch_bn(const Dims& D, const CUtensorMap& a, const CUtensorMap& br
   if (err != cudaSuccess) return err;
   const int tiles_r = static_cast<int>((D.Nr + BN - 1) / BN);
   const int tiles_c = static_cast<int>((D.Nc + BN - 1) / BN);
-  dim3 grid(static_cast<unsigned>((D.L + TC_BM - 1) / TC_BM), tiles_r + tiles_c);
+  const int64_t mt = (D.L + TC_BM - 1) / TC_BM;
+  const int nk = static_cast<int>((D.d + TC_BK - 1) / TC_BK);
+  const int ks = router_splits(D);
+  const int kper = (nk + ks - 1) / ks;
+  dim3 grid(static_cast<unsigned>(mt), tiles_r + tiles_c, ks);
   k_router_tc<BN><<<grid, TC_THREADS, smem, s>>>(a, br, bc, Z, static_cast<int>(D.L),
                                                  static_cast<int>(D.Nr), static_cast<int>(D.Nc),
-                                                 static_cast<int>(D.d), tiles_r, status);
+                                                 static_cast<int>(D.d), tiles_r, kper, status);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// K-splits from the dims alone (so workspace sizes are known on the host):
+// enough CTAs for about one per SM of a 148-SM B200, at most 16 partials.
+int router_splits(const Dims& D) {
+  if (D.dtype != OMNI_BF16 || (D.flags & OMNI_FLAG_ROUTER_SIMT)) return 1;
+  const int bn = pick_bn(D);
+  const int64_t tiles = ((D.L + TC_BM - 1) / TC_BM) *
+                        ((D.Nr + bn - 1) / bn + (D.Nc + bn - 1) / bn);
+  const int nk = static_cast<int>((D.d + TC_BK - 1) / TC_BK);
+  int ks = tiles >= 148 ? 1 : static_cast<int>(148 / tiles);
+  ks = ks < 1 ? 1 : (ks > 16 ? 16 : ks);
+  ks = ks > nk ? nk : ks;
+  const int kper = (nk + ks - 1) / ks;
+  return (nk + kper - 1) / kper;
+}
+
+namespace {
+__global__ void __launch_bounds__(256) k_sum_partials(float* __restrict__ Z, int splits, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = Z[i];
+  for (int s = 1; s < splits; ++s) acc += Z[s * n + i];
+  Z[i] = acc;
+}
+}  // namespace
+
+cudaError_t launch_sum_partials(float* Z, int splits, int64_t n, cudaStream_t s) {
+  if (splits <= 1 || n == 0) return cudaSuccess;
+  k_sum_partials<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(Z, splits, n);
+  return cudaGetLastError();
+}
 
 bool router_tc_supported(const Dims& D, const void* x, const void* Wr, const void* Wc) {
   if (D.dtype != OMNI_BF16 || (D.flags & OMNI_FLAG_ROUTER_SIMT)) return false;

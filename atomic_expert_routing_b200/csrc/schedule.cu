@@ -193,32 +193,56 @@ __global__ void __launch_bounds__(kRsThreads)
   hist[static_cast<int64_t>(threadIdx.x) * ntiles + blockIdx.x] = h[threadIdx.x];
 }
 
-// single block exclusive scan over n = 256 * ntiles words (digit-major)
-__global__ void __launch_bounds__(kScanThreads) k_rs_scan(uint32_t* __restrict__ hist, int64_t n) {
+// Device-wide exclusive scan of n words in place (digit-major radix table):
+// per-tile sums, one block scanning the tile sums, then each tile finishes.
+__global__ void __launch_bounds__(kScanThreads)
+    k_gscan_reduce(const uint32_t* __restrict__ v, int64_t n, int32_t* __restrict__ tile_sum) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
+  int acc = 0;
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j)
+    if (base + j < n) acc += static_cast<int>(v[base + j]);
+  block_exclusive_scan(acc, warp_tot, &total);
+  if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_gscan_tiles(int32_t* __restrict__ tile_sum, int ntiles) {
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  const int64_t chunk = static_cast<int64_t>(kScanThreads) * kScanItems;
-  for (int64_t c0 = 0; c0 < n; c0 += chunk) {
-    const int64_t base = c0 + static_cast<int64_t>(threadIdx.x) * kScanItems;
-    uint32_t v[kScanItems];
-    int s = 0;
-#pragma unroll
-    for (int j = 0; j < kScanItems; ++j) {
-      v[j] = (base + j < n) ? hist[base + j] : 0u;
-      s += static_cast<int>(v[j]);
-    }
-    int ex = block_exclusive_scan(s, warp_tot, &total) + carry;
-#pragma unroll
-    for (int j = 0; j < kScanItems; ++j) {
-      if (base + j < n) hist[base + j] = static_cast<uint32_t>(ex);
-      ex += static_cast<int>(v[j]);
-    }
+  for (int c0 = 0; c0 < ntiles; c0 += kScanThreads) {
+    const int i = c0 + threadIdx.x;
+    const int v = i < ntiles ? tile_sum[i] : 0;
+    const int ex = block_exclusive_scan(v, warp_tot, &total);
+    if (i < ntiles) tile_sum[i] = carry + ex;
     __syncthreads();
     if (threadIdx.x == 0) carry += total;
     __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    k_gscan_finish(uint32_t* __restrict__ v, int64_t n, const int32_t* __restrict__ tile_off) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
+  uint32_t f[kScanItems];
+  int acc = 0;
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    f[j] = (base + j < n) ? v[base + j] : 0u;
+    acc += static_cast<int>(f[j]);
+  }
+  int r = block_exclusive_scan(acc, warp_tot, &total) + tile_off[blockIdx.x];
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    if (base + j < n) v[base + j] = static_cast<uint32_t>(r);
+    r += static_cast<int>(f[j]);
   }
 }
 
@@ -295,11 +319,174 @@ __global__ void __launch_bounds__(256)
   if (i == M - 1) group_off[counts[1]] = static_cast<int32_t>(M);
 }
 
+// ---- small batches (M <= kSmallMax): the whole schedule in one CTA ----------
+constexpr int kSmallMax = 8192;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+constexpr int kSmallRounds = kSmallMax / kSmallThreads;  // rounds of 32 keys per warp
+
+// One stable LSD radix pass (8-bit digit at `shift`) of n <= kSmallMax keys
+// with 16-bit payloads, in shared memory, by the whole CTA.  Warp w ranks
+// keys [w*256, w*256+256) in order (match_any groups equal digits), then the
+// per-warp digit counts are scanned (warp-major inside each digit, then over
+// digits) and every key is scattered to its final slot.
+__device__ void block_radix_pass(const uint32_t* kin, const uint16_t* vin, uint32_t* kout,
+                                 uint16_t* vout, int n, int shift, uint32_t* wcount,
+                                 uint32_t* dbase, int* warp_tot, int* total) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int j = tid; j < kSmallWarps * 256; j += kSmallThreads) wcount[j] = 0u;
+  __syncthreads();
+  uint32_t dig[kSmallRounds], rnk[kSmallRounds];
+#pragma unroll
+  for (int r = 0; r < kSmallRounds; ++r) {
+    const int i = warp * (kSmallRounds * 32) + r * 32 + lane;
+    const bool valid = i < n;
+    dig[r] = valid ? ((kin[i] >> shift) & 255u) : 0xffffffffu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, dig[r]);
+    const int leader = __ffs(peers) - 1;
+    uint32_t old = 0;
+    if (valid && lane == leader) {
+      old = wcount[warp * 256 + dig[r]];
+      wcount[warp * 256 + dig[r]] = old + __popc(peers);
+    }
+    old = __shfl_sync(0xffffffffu, old, leader);
+    rnk[r] = old + __popc(peers & lanemask_lt());
+    __syncwarp();
+  }
+  __syncthreads();
+  if (tid < 256) {
+    uint32_t acc = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const uint32_t c = wcount[w * 256 + tid];
+      wcount[w * 256 + tid] = acc;
+      acc += c;
+    }
+    dbase[tid] = acc;
+  }
+  __syncthreads();
+  {
+    const int v = tid < 256 ? static_cast<int>(dbase[tid]) : 0;
+    const int ex = block_exclusive_scan(v, warp_tot, total);
+    if (tid < 256) dbase[tid] = static_cast<uint32_t>(ex);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kSmallRounds; ++r) {
+    const int i = warp * (kSmallRounds * 32) + r * 32 + lane;
+    if (i < n) {
+      const uint32_t pos = dbase[dig[r]] + wcount[warp * 256 + dig[r]] + rnk[r];
+      kout[pos] = kin[i];
+      vout[pos] = vin[i];
+    }
+  }
+  __syncthreads();
+}
+
+// Same outputs as the multi-kernel path.  (1) Radix-sort the tasks' expert
+// ids; a scan of the "new id" flags gives U and the rank of every task's
+// expert.  (2) Radix-sort the composite keys (group, token, rank inside the
+// group) -- unique, and ordered exactly like (group, token, expert).  (3) Emit.
+__global__ void __launch_bounds__(kSmallThreads)
+    k_sched_small(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L,
+                  int K, int64_t N, int64_t B, int epasses, int kpasses,
+                  int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
+                  float* __restrict__ task_gate, int32_t* __restrict__ uniq,
+                  int32_t* __restrict__ group_off, int32_t* counts) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* keyA = sm;
+  uint32_t* keyB = keyA + kSmallMax;
+  uint16_t* valA = reinterpret_cast<uint16_t*>(keyB + kSmallMax);
+  uint16_t* valB = valA + kSmallMax;
+  uint16_t* rk = valB + kSmallMax;  // rank of each task's expert
+  uint32_t* wcount = reinterpret_cast<uint32_t*>(rk + kSmallMax);  // [kSmallWarps][256]
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ uint32_t dbase[256];
+  const int tid = threadIdx.x;
+  const int M = static_cast<int>(L * K);
+  int32_t* status = counts + 2;
+  // (1) sort by expert id
+  for (int i = tid; i < M; i += kSmallThreads) {
+    int64_t e = idx[i];
+    if (e < 0 || e >= N) {
+      raise_status(status, OMNI_DEV_BAD_INDEX);
+      e = 0;
+    }
+    keyA[i] = static_cast<uint32_t>(e);
+    valA[i] = static_cast<uint16_t>(i);
+  }
+  __syncthreads();
+  uint32_t *kin = keyA, *kout = keyB;
+  uint16_t *vin = valA, *vout = valB;
+  for (int p = 0; p < epasses; ++p) {
+    block_radix_pass(kin, vin, kout, vout, M, 8 * p, wcount, dbase, warp_tot, &total);
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
+  // ranks: each thread takes kSmallRounds consecutive sorted positions
+  const int b0 = tid * kSmallRounds;
+  int nnew = 0;
+#pragma unroll
+  for (int j = 0; j < kSmallRounds; ++j) {
+    const int q = b0 + j;
+    if (q < M && (q == 0 || kin[q] != kin[q - 1])) ++nnew;
+  }
+  int r = block_exclusive_scan(nnew, warp_tot, &total) - 1;
+  const int n_active = total;
+#pragma unroll
+  for (int j = 0; j < kSmallRounds; ++j) {
+    const int q = b0 + j;
+    if (q < M) {
+      if (q == 0 || kin[q] != kin[q - 1]) {
+        ++r;
+        uniq[r] = static_cast<int32_t>(kin[q]);
+      }
+      rk[vin[q]] = static_cast<uint16_t>(r);
+    }
+  }
+  const int64_t G = (n_active + B - 1) / B;
+  if (tid == 0) {
+    counts[0] = n_active;
+    counts[1] = static_cast<int32_t>(G);
+  }
+  __syncthreads();
+  // (2) composite keys
+  const uint32_t Wl = static_cast<uint32_t>(B < M ? B : M);
+  for (int i = tid; i < M; i += kSmallThreads) {
+    const uint32_t rr = rk[i];
+    const uint32_t g = static_cast<uint32_t>(rr / static_cast<uint64_t>(B));
+    const uint32_t t = static_cast<uint32_t>(i / K);
+    keyA[i] = (g * static_cast<uint32_t>(L) + t) * Wl + (rr - g * static_cast<uint32_t>(B));
+    valA[i] = static_cast<uint16_t>(i);
+  }
+  __syncthreads();
+  kin = keyA; kout = keyB; vin = valA; vout = valB;
+  for (int p = 0; p < kpasses; ++p) {
+    block_radix_pass(kin, vin, kout, vout, M, 8 * p, wcount, dbase, warp_tot, &total);
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
+  // (3) emit
+  const uint32_t per_group = static_cast<uint32_t>(L) * Wl;
+  for (int p = tid; p < M; p += kSmallThreads) {
+    const int i = vin[p];
+    const uint32_t g = kin[p] / per_group;
+    task_token[p] = i / K;
+    int32_t e = idx[i];
+    if (e < 0 || e >= N) e = 0;
+    task_expert[p] = e;
+    task_gate[p] = gate[i];
+    if (p == 0 || kin[p - 1] / per_group != g) group_off[g] = p;
+    if (p == M - 1) group_off[G] = M;
+  }
+}
+
 struct SchedWs {
   int32_t *flags, *rank, *tile_sum, *tmp_e;
   float* tmp_g;
-  uint32_t *ka, *va, *kb, *vb, *hist;
-  int64_t nscan, ntiles;
+  uint32_t *ka, *va, *kb, *vb, *hist, *bits;
+  int32_t *hist_tiles, *wpre;
+  int64_t nscan, ntiles, nhscan;
   int passes;
 };
 
@@ -307,6 +494,10 @@ SchedWs carve(const Dims& D, void* base, size_t* bytes) {
   Carver c(base);
   SchedWs w{};
   const int64_t N = D.N(), M = D.M();
+  if (M <= kSmallMax) {  // the single-CTA path works in shared memory only
+    if (bytes) *bytes = 0;
+    return w;
+  }
   w.nscan = (N + kScanTile - 1) / kScanTile;
   w.ntiles = (M + kRsTile - 1) / kRsTile;
   int bits = 0;
@@ -323,6 +514,8 @@ SchedWs carve(const Dims& D, void* base, size_t* bytes) {
     w.kb = c.take<uint32_t>(M);
     w.vb = c.take<uint32_t>(M);
     w.hist = c.take<uint32_t>(256 * w.ntiles);
+    w.nhscan = (256 * w.ntiles + kScanTile - 1) / kScanTile;
+    w.hist_tiles = c.take<int32_t>(w.nhscan + 1);
   }
   if (bytes) *bytes = c.off;
   return w;
@@ -347,6 +540,26 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     if (e == cudaSuccess) e = cudaMemsetAsync(group_off, 0, sizeof(int32_t), s);
     return e;
   }
+  if (M <= kSmallMax) {
+    auto nbits = [](uint64_t v) {
+      int b = 0;
+      while ((uint64_t(1) << b) < v) ++b;
+      return b;
+    };
+    const int epasses = (nbits(static_cast<uint64_t>(N)) + 7) / 8;
+    // composite key < gmax * L * min(B, M)
+    const int kpasses = (nbits(static_cast<uint64_t>(D.gmax()) * static_cast<uint64_t>(D.L) *
+                               static_cast<uint64_t>(D.B < M ? D.B : M)) + 7) / 8;
+    const size_t smem = static_cast<size_t>(kSmallMax) * (2 * sizeof(uint32_t) + 3 * sizeof(uint16_t)) +
+                        static_cast<size_t>(kSmallWarps) * 256 * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(k_sched_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    k_sched_small<<<1, kSmallThreads, smem, s>>>(idx, gate, D.L, static_cast<int>(D.K), N, D.B,
+                                                  epasses, kpasses, task_token, task_expert,
+                                                  task_gate, uniq, group_off, counts);
+    return cudaGetLastError();
+  }
   SchedWs w = carve(D, ws, nullptr);
   cudaError_t err = cudaMemsetAsync(w.flags, 0, static_cast<size_t>(N) * sizeof(int32_t), s);
   if (err != cudaSuccess) return err;
@@ -369,7 +582,11 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     k_rs_hist<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(src, M, 8 * p,
                                                                       static_cast<int>(w.ntiles),
                                                                       w.hist);
-    k_rs_scan<<<1, kScanThreads, 0, s>>>(w.hist, 256 * w.ntiles);
+    k_gscan_reduce<<<static_cast<unsigned>(w.nhscan), kScanThreads, 0, s>>>(
+        w.hist, 256 * w.ntiles, w.hist_tiles);
+    k_gscan_tiles<<<1, kScanThreads, 0, s>>>(w.hist_tiles, static_cast<int>(w.nhscan));
+    k_gscan_finish<<<static_cast<unsigned>(w.nhscan), kScanThreads, 0, s>>>(
+        w.hist, 256 * w.ntiles, w.hist_tiles);
     k_rs_scatter<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(
         src, vals, M, 8 * p, static_cast<int>(w.ntiles), w.hist, ko, vo);
     keys = ko;

@@ -57,10 +57,22 @@ __device__ void warp_select_top(KeyFn key, int n, int want, uint64_t* out, uint3
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-      const uint64_t kk = key(i);
-      if (shift == 56 || (kk >> (shift + 8)) == (prefix >> (shift + 8)))
-        atomicAdd(&hist[(kk >> shift) & 255u], 1u);
+    // histogram of the next digit; lanes holding the same digit add once
+    // (one shared-memory atomic per distinct digit and step, not per key)
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      bool part = false;
+      uint32_t dig = 0;
+      if (i < n) {
+        const uint64_t kk = key(i);
+        part = shift == 56 || (kk >> (shift + 8)) == (prefix >> (shift + 8));
+        dig = static_cast<uint32_t>(kk >> shift) & 255u;
+      }
+      const uint32_t pm = __ballot_sync(0xffffffffu, part);
+      if (part) {
+        const uint32_t peers = __match_any_sync(pm, dig);
+        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(peers)));
+      }
     }
     __syncwarp();
     // bins in descending order: lane l owns bins 255-8l ... 248-8l
@@ -140,9 +152,219 @@ __device__ void warp_sort_desc(uint64_t* s, int P) {
     }
 }
 
+constexpr int kCandMax = 64;  // keys of the threshold bin resolved by sorting
+
+// Top `want` of n keys by (value desc, id asc), one warp, written sorted
+// (descending composite key) to out[0..P) (P = next power of two >= want,
+// padded with 0).  Value-range binning: with lo/hi the smallest/largest value,
+// bin(v) = floor((v - lo) * 256 / (hi - lo)) is monotone in v, so every key in
+// a bin above the threshold bin is selected and equal values share a bin; the
+// keys of the threshold bin (at most kCandMax) are ordered exactly by their
+// 64-bit keys.  Otherwise (threshold bin too full, non-finite scale) the radix
+// select decides.  hist: 256 words; cand: kCandMax keys.
+template <typename ValFn, typename IdFn>
+__device__ void warp_topk_sorted(ValFn val, IdFn id, int n, int want, int P, float lo, float hi,
+                                 uint64_t* out, uint32_t* hist, uint64_t* cand) {
+  const int lane = threadIdx.x & 31;
+  auto key = [&](int i) { return make_key(val(i), id(i)); };
+  const float range = hi - lo;
+  const float scale = 256.0f / range;
+  bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
+  if (fast) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    auto bin = [&](float v) {
+      const float f = (v - lo) * scale;
+      return f >= 255.0f ? 255u : (f > 0.0f ? static_cast<uint32_t>(f) : 0u);
+    };
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const bool part = i < n;
+      const uint32_t dig = part ? bin(val(i)) : 0u;
+      const uint32_t pm = __ballot_sync(0xffffffffu, part);
+      if (part) {
+        const uint32_t peers = __match_any_sync(pm, dig);
+        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(peers)));
+      }
+    }
+    __syncwarp();
+    uint32_t c[8];
+    uint32_t tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[j] = hist[255 - 8 * lane - j];
+      tot += c[j];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - tot;
+    int tb = -1;
+    uint32_t above = 0;
+    if (excl < static_cast<uint32_t>(want) && static_cast<uint32_t>(want) <= incl) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (tb < 0 && run + c[j] >= static_cast<uint32_t>(want)) {
+          tb = 255 - 8 * lane - j;
+          above = run;
+        }
+        run += c[j];
+      }
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, tb >= 0);
+    const int src = __ffs(who) - 1;
+    tb = __shfl_sync(0xffffffffu, tb, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    const uint32_t at = hist[tb];
+    __syncwarp();
+    fast = at <= kCandMax;
+    if (fast) {
+      // keys above the threshold bin -> out[0..above), the threshold bin -> cand
+      int nb = 0, nc = 0;
+      for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        uint32_t b = 0;
+        uint64_t kk = 0;
+        if (i < n) {
+          const float v = val(i);
+          b = bin(v);
+          kk = make_key(v, id(i));
+        }
+        const bool up = i < n && static_cast<int>(b) > tb;
+        const bool eq = i < n && static_cast<int>(b) == tb;
+        const uint32_t mu = __ballot_sync(0xffffffffu, up);
+        const uint32_t me = __ballot_sync(0xffffffffu, eq);
+        if (up) out[nb + __popc(mu & lanemask_lt())] = kk;
+        if (eq) cand[nc + __popc(me & lanemask_lt())] = kk;
+        nb += __popc(mu);
+        nc += __popc(me);
+      }
+      // order the threshold bin and take what is still needed
+      int cp = 1;
+      while (cp < nc) cp <<= 1;
+      for (int i = nc + lane; i < cp; i += 32) cand[i] = 0;
+      __syncwarp();
+      warp_sort_desc(cand, cp);
+      const int need = want - nb;
+      for (int i = lane; i < need; i += 32) out[nb + i] = cand[i];
+      __syncwarp();
+    }
+  }
+  if (!fast) warp_select_top(key, n, want, out, hist);
+  for (int i = want + lane; i < P; i += 32) out[i] = 0;
+  __syncwarp();
+  warp_sort_desc(out, P);
+}
+
+// The same selection as warp_topk_sorted for values held in registers: lane l
+// holds values v[j] of indices j*32 + l (indices >= n are absent).  The rare
+// fallback copies the values to `spill` (n floats) and runs the radix select.
+template <int NPL>
+__device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, float lo, float hi,
+                               uint64_t* out, uint32_t* hist, uint64_t* cand, float* spill) {
+  const int lane = threadIdx.x & 31;
+  const float range = hi - lo;
+  const float scale = 256.0f / range;
+  bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
+  if (fast) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    auto bin = [&](float x) {
+      const float f = (x - lo) * scale;
+      return f >= 255.0f ? 255u : (f > 0.0f ? static_cast<uint32_t>(f) : 0u);
+    };
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const bool part = j * 32 + lane < n;
+      const uint32_t dig = part ? bin(v[j]) : 0u;
+      const uint32_t pm = __ballot_sync(0xffffffffu, part);
+      if (part) {
+        const uint32_t peers = __match_any_sync(pm, dig);
+        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(peers)));
+      }
+    }
+    __syncwarp();
+    uint32_t c[8];
+    uint32_t tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[j] = hist[255 - 8 * lane - j];
+      tot += c[j];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const uint32_t excl = incl - tot;
+    int tb = -1;
+    uint32_t above = 0;
+    if (excl < static_cast<uint32_t>(want) && static_cast<uint32_t>(want) <= incl) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (tb < 0 && run + c[j] >= static_cast<uint32_t>(want)) {
+          tb = 255 - 8 * lane - j;
+          above = run;
+        }
+        run += c[j];
+      }
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, tb >= 0);
+    const int src = __ffs(who) - 1;
+    tb = __shfl_sync(0xffffffffu, tb, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    const uint32_t at = hist[tb];
+    __syncwarp();
+    fast = at <= kCandMax;
+    if (fast) {
+      int nb = 0, nc = 0;
+#pragma unroll
+      for (int j = 0; j < NPL; ++j) {
+        const int i = j * 32 + lane;
+        const bool valid = i < n;
+        const uint32_t b = valid ? bin(v[j]) : 0u;
+        const bool up = valid && static_cast<int>(b) > tb;
+        const bool eq = valid && static_cast<int>(b) == tb;
+        const uint64_t kk = make_key(v[j], static_cast<uint32_t>(i));
+        const uint32_t mu = __ballot_sync(0xffffffffu, up);
+        const uint32_t me = __ballot_sync(0xffffffffu, eq);
+        if (up) out[nb + __popc(mu & lanemask_lt())] = kk;
+        if (eq) cand[nc + __popc(me & lanemask_lt())] = kk;
+        nb += __popc(mu);
+        nc += __popc(me);
+      }
+      int cp = 1;
+      while (cp < nc) cp <<= 1;
+      for (int i = nc + lane; i < cp; i += 32) cand[i] = 0;
+      __syncwarp();
+      warp_sort_desc(cand, cp);
+      const int need = want - nb;
+      for (int i = lane; i < need; i += 32) out[nb + i] = cand[i];
+      __syncwarp();
+    }
+  }
+  if (!fast) {
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+      if (j * 32 + lane < n) spill[j * 32 + lane] = v[j];
+    __syncwarp();
+    warp_select_top([&](int i) { return make_key(spill[i], static_cast<uint32_t>(i)); }, n, want,
+                    out, hist);
+  }
+  for (int i = want + lane; i < P; i += 32) out[i] = 0;
+  __syncwarp();
+  warp_sort_desc(out, P);
+}
+
 struct SelPlan {
   int nr_pad, nc_pad, kp, Kp, cand;  // sizes (elements)
-  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc;
+  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc;
   int pair_bytes;
 };
 
@@ -170,10 +392,13 @@ SelPlan make_plan(const Dims& D) {
   p.off_cand = off; off = al(off + 8 * cand);
   p.off_out = off; off = al(off + 8 * p.Kp);
   p.off_misc = off; off = al(off + 16);
+  p.off_tr = off; off = al(off + 8 * kCandMax);
+  p.off_tc = off; off = al(off + 8 * kCandMax);
   p.pair_bytes = off;
   return p;
 }
 
+template <int NPL>
 __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int64_t L, int Nr,
                                                 int Nc, int k, int K,
                                                 const float* __restrict__ br,
@@ -199,25 +424,31 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
     float* vals = reinterpret_cast<float*>(base + (role ? P.off_vc : P.off_vr));
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + (role ? P.off_hc : P.off_hr));
     uint64_t* sel = reinterpret_cast<uint64_t*>(base + (role ? P.off_sc : P.off_sr));
-    float mx = -INFINITY;
-    for (int i = lane; i < n; i += 32) {
-      float v = z[i];
-      if (bias != nullptr) v += bias[i];
-      v = (v == 0.0f) ? 0.0f : v;  // one zero (no -0) so equal logits tie
-      vals[i] = v;
-      mx = fmaxf(mx, v);
+    uint64_t* tbin = reinterpret_cast<uint64_t*>(base + (role ? P.off_tc : P.off_tr));
+    float v[NPL];
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const int i = j * 32 + lane;
+      float x = 0.0f;
+      if (i < n) {
+        x = z[i];
+        if (bias != nullptr) x += bias[i];
+        x = (x == 0.0f) ? 0.0f : x;  // one zero (no -0) so equal logits tie
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+      }
+      v[j] = x;
     }
     mx = warp_max(mx);
+    mn = -warp_max(-mn);
     float s = 0.0f;
-    for (int i = lane; i < n; i += 32) s += expf(vals[i] - mx);
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+      if (j * 32 + lane < n) s += expf(v[j] - mx);
     s = warp_sum(s);
-    __syncwarp();
     if (lane == 0) misc[role] = mx + logf(s);
-    auto key = [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); };
-    warp_select_top(key, n, k, sel, hist);
-    for (int i = k + lane; i < P.kp; i += 32) sel[i] = 0;
-    __syncwarp();
-    warp_sort_desc(sel, P.kp);
+    warp_topk_regs<NPL>(v, n, k, P.kp, mn, mx, sel, hist, tbin, vals);
   }
   asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
   if (role != 0) return;
@@ -228,7 +459,9 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   uint64_t* cand = reinterpret_cast<uint64_t*>(base + P.off_cand);
   uint64_t* out = reinterpret_cast<uint64_t*>(base + P.off_out);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + P.off_hr);
+  uint64_t* tbin = reinterpret_cast<uint64_t*>(base + P.off_tr);
   int nc = 0;
+  float cmx = -INFINITY, cmn = INFINITY;
   for (int a = 0; a < k; ++a) {
     int nb = K / (a + 1);
     if (nb > k) nb = k;
@@ -241,15 +474,16 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
       const float sv = za + key_val(cb);
       const uint32_t e = ia * static_cast<uint32_t>(Nc) + key_id(cb);
       cand[nc + b] = make_key(sv, e);
+      cmx = fmaxf(cmx, sv);
+      cmn = fminf(cmn, sv);
     }
     nc += nb;
   }
+  cmx = warp_max(cmx);
+  cmn = -warp_max(-cmn);
   __syncwarp();
-  auto ckey = [&](int i) { return cand[i]; };
-  warp_select_top(ckey, nc, K, out, hist);
-  for (int i = K + lane; i < P.Kp; i += 32) out[i] = 0;
-  __syncwarp();
-  warp_sort_desc(out, P.Kp);
+  warp_topk_sorted([&](int i) { return key_val(cand[i]); }, [&](int i) { return key_id(cand[i]); },
+                   nc, K, P.Kp, cmn, cmx, out, hist, tbin);
 
   // ---- gate = softmax of the K selected joint scores ----
   const float s0 = key_val(out[0]);
@@ -268,22 +502,37 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
 
 }  // namespace
 
-cudaError_t launch_select(const Dims& D, const float* Z, const float* br, const float* bc,
-                          int32_t* idx, float* gate, float* score, cudaStream_t s) {
-  if (D.L == 0) return cudaSuccess;
+template <int NPL>
+cudaError_t launch_select_npl(const Dims& D, const float* Z, const float* br, const float* bc,
+                              int32_t* idx, float* gate, float* score, cudaStream_t s) {
   SelPlan P = make_plan(D);
   int pairs = 4;
   while (pairs > 1 && pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
   const size_t smem = static_cast<size_t>(pairs) * P.pair_bytes;
   cudaError_t err =
-      cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(k_select<NPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int64_t grid = (D.L + pairs - 1) / pairs;
-  k_select<<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
+  k_select<NPL><<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
       Z, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
       static_cast<int>(D.K), br, bc, idx, gate, score, P);
   return cudaGetLastError();
+}
+
+cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
+                          const float* bc, int32_t* idx, float* gate, float* score,
+                          cudaStream_t s) {
+  if (D.L == 0) return cudaSuccess;
+  if (parts > 1) {  // split-K partial logits: sum them first, in a fixed order
+    cudaError_t e = launch_sum_partials(const_cast<float*>(Z), parts, D.L * (D.Nr + D.Nc), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t n = D.Nr > D.Nc ? D.Nr : D.Nc;
+  if (n <= 256) return launch_select_npl<8>(D, Z, br, bc, idx, gate, score, s);
+  if (n <= 1024) return launch_select_npl<32>(D, Z, br, bc, idx, gate, score, s);
+  if (n <= 2048) return launch_select_npl<64>(D, Z, br, bc, idx, gate, score, s);
+  return launch_select_npl<128>(D, Z, br, bc, idx, gate, score, s);
 }
 
 }  // namespace omni

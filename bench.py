@@ -69,7 +69,10 @@ def kernel_launches(cfg):
     bits = max(0, int(np.ceil(np.log2(gmax)))) if gmax > 1 else 0
     passes = (bits + 7) // 8
     route = 2
-    sched = 1 + 3 + 3 * passes + 1
+    if cfg.L * cfg.K <= 8192:
+        sched = 1  # single-CTA schedule of small batches
+    else:
+        sched = 1 + 3 + 5 * passes + 1  # prep, flag scan, radix passes (hist, 3 scans, scatter), emit
     expert = 1 + (1 if cfg.dtype == WL.BF16 else 0)
     return route + sched + expert
 
@@ -90,7 +93,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -160,7 +163,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg = WL.CONFIGS[args.workload]
+    cfg = {**WL.CONFIGS, **WL.EXTRA}[args.workload]
     rate, n, dt, threads, _ = oracle_timing(cfg, target_s=max(2.0, 60.0 / max(1, args.steps)))
     # steps: repeat the bounded sample K times after W warm-ups (each a full pass)
     import oracle as O
@@ -219,7 +222,7 @@ def run_ours(args):
             return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
         return torch.from_numpy(a).to(device)
 
-    cfg = WL.CONFIGS[args.workload]
+    cfg = {**WL.CONFIGS, **WL.EXTRA}[args.workload]
     # every rank draws its own token batch (seed + rank); weights are shared
     rcfg = cfg.with_(seed=cfg.seed)
     host = WL.make_inputs(rcfg, experts=False)
@@ -265,6 +268,9 @@ def run_ours(args):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
         with Clocks(local) as clk:
+            t_wait = time.time()
+            while not clk.lines and time.time() - t_wait < 3.0:
+                time.sleep(0.01)
             barrier()
             with torch.cuda.stream(stream):
                 for a, b in ev:
@@ -298,6 +304,41 @@ def run_ours(args):
             b.record(stream)
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in ev) / steps, int(s["counts"][0].item())
+
+    def measure_stages(c, dd, steps):
+        """The three stages as separate calls with events between them (same
+        kernels as the fused call), L2 flushed before each pass."""
+        D = omni.LayerDims.of(c)
+        stream = torch.cuda.current_stream(device)
+        wr, wsd, we = omni.Workspace(), omni.Workspace(), omni.Workspace()
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        counts = omni.new_counts(device)
+
+        def one(evs=None):
+            if evs:
+                evs[0].record(stream)
+            idx, gate, _ = omni.route(D, dd["x"], dd["Wr"], dd["Wc"], dd["bias_r"], dd["bias_c"],
+                                      ws=wr, with_score=False, counts=counts)
+            if evs:
+                evs[1].record(stream)
+            s = omni.schedule(D, idx, gate, ws=wsd, counts=counts)
+            if evs:
+                evs[2].record(stream)
+            omni.expert_forward(D, dd["x"], dd["W"], dd["V"], s, y=y, ws=we)
+            if evs:
+                evs[3].record(stream)
+
+        one()
+        torch.cuda.synchronize()
+        tot = [0.0, 0.0, 0.0]
+        for _ in range(steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.zero_()
+            one(evs)
+            torch.cuda.synchronize()
+            for i in range(3):
+                tot[i] += evs[i].elapsed_time(evs[i + 1])
+        return {"route": tot[0] / steps, "schedule": tot[1] / steps, "expert": tot[2] / steps}
 
     def measure_e2e(c, dd, steps, warmup):
         """The public call with host buffers: pinned x -> device, forward, y -> pinned host."""
@@ -346,6 +387,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
+    stages = measure_stages(cfg, d, max(3, args.steps // 2))
 
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
@@ -353,6 +395,7 @@ def run_ours(args):
         host2 = WL.make_inputs(sc.with_(seed=sc.seed + 1000 * rank), experts=False)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
         ms2, na2, st2, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
+        stages2 = measure_stages(sc, d2, 10)
         if world > 1:
             t = torch.tensor([ms2], device=device)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -360,7 +403,7 @@ def run_ours(args):
         f2, b2 = layer_work(sc, na2)
         extra[sc.name] = {
             "value": world * sc.L / (ms2 * 1e-3), "unit": "tokens/s", "ms_per_step": ms2,
-            "n_active": na2, "device_status": st2,
+            "n_active": na2, "device_status": st2, "stages_ms": stages2,
             "layer_roofline": {"bound": "hbm" if b2 / (hbm * 1e9) > f2 / (tc * 1e12) else "tensor",
                                "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
                                "bytes": b2, "flops": f2}}
@@ -400,6 +443,7 @@ def run_ours(args):
                    "graph": True, "parallelism": f"dp{world} (independent token batches)"},
         "n_active": n_active,
         "device_status": status,
+        "stages_ms": stages,
         "layer_roofline": {"bound": "hbm" if t_b >= t_f else "tensor",
                            "frac": max(t_f, t_b) / (ms_all * 1e-3), "bytes": bytes_,
                            "flops": flops, "peak_src": peak_src},
@@ -428,7 +472,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=PRIMARY.name, choices=sorted(WL.CONFIGS))
+    ap.add_argument("--workload", default=PRIMARY.name, choices=sorted(WL.CONFIGS) + sorted(WL.EXTRA))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")

@@ -120,11 +120,13 @@ int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void*
 /*
  * The projection half of omni_route [NL 2.2]: logits float [L x (Nr + Nc)],
  * row t = (x[t] Wr^T, x[t] Wc^T), fp32 accumulation, no bias.  bf16 storage
- * runs on the tensor cores (tcgen05), fp32 storage on CUDA cores.  Needs no
- * workspace.
+ * runs on the tensor cores (tcgen05), fp32 storage on CUDA cores.  Small
+ * batches split the reduction over d into partial sums that are added in a
+ * fixed order (the result does not depend on timing); ws needs the
+ * OMNI_WS_ROUTE size for these dims.
  */
 int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
-                       float* logits, int32_t* counts, void* stream);
+                       float* logits, int32_t* counts, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * The selection half of omni_route, from axis logits the caller computed:
