@@ -194,6 +194,22 @@ def expert_forward(D: LayerDims, x, W, V, sched: dict, *, y=None, ws=None, strea
     return y
 
 
+def expert_forward_noalloc(D: LayerDims, x, W, V, sched: dict, *, y=None, stream=None):
+    """Grouped execution without a workspace, for callers that cannot allocate
+    device memory when the layer runs (the accumulator is a fixed array inside
+    the library; L*d <= 4194304; calls must not overlap on the GPU).  Pass y to
+    keep the call itself free of allocations."""
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    dd = D.c()
+    _lib.check("omni_expert_forward_noalloc", _lib.load().omni_expert_forward_noalloc(
+        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(sched["task_token"]),
+        _ptr(sched["task_expert"]), _ptr(sched["task_gate"]), _ptr(sched["uniq"]),
+        _ptr(sched["group_off"]), _ptr(sched["counts"]), _ptr(y), _stream(stream)))
+    return y
+
+
 def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=None,
                 counts=None, idx=None, gate=None, ws=None, stream=None):
     """Route -> schedule -> grouped execution in one call; returns y [L, d]."""

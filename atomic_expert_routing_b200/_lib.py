@@ -40,6 +40,7 @@ SIGNATURES = {
     "omni_router_logits": ([_P] * 7 + [C.c_size_t, _P], C.c_int),
     "omni_schedule": ([_P] * 10 + [C.c_size_t, _P], C.c_int),
     "omni_expert_forward": ([_P] * 12 + [C.c_size_t, _P], C.c_int),
+    "omni_expert_forward_noalloc": ([_P] * 12, C.c_int),
     "omni_moe_forward": ([_P] * 13 + [C.c_size_t, _P], C.c_int),
     "omni_token_centric_forward": ([_P] * 9 + [C.c_size_t, _P], C.c_int),
 }

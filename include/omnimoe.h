@@ -167,6 +167,28 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
                         int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * omni_expert_forward for callers that cannot allocate device memory when the
+ * layer runs: code running while a CUDA graph is being captured, runtimes that
+ * plan every device buffer ahead of time, plugin hosts that own all device
+ * memory and pass an operator only its inputs and outputs.  The pages have no
+ * counterpart of this call; it is a packaging of the same computation.
+ * Arguments and results are those of omni_expert_forward, without ws.  The
+ * fp32 accumulator it needs lives in a fixed device array inside the library
+ * (16 MiB, held by every GPU that loads the library until the process exits),
+ * so L*d must not exceed 4194304 (OMNI_ERR_UNSUPPORTED otherwise).  The array
+ * is shared by every call and zeroed by each call before use: calls that can
+ * overlap on the GPU (different streams, or several host threads) race on it
+ * and must be serialised by the caller.  The first call on a device looks up
+ * the array's device address; make that first call before any stream capture.
+ * Allocates nothing.
+ */
+int omni_expert_forward_noalloc(const omni_dims* dims, const void* x, const void* W,
+                                const void* V, const int32_t* task_token,
+                                const int32_t* task_expert, const float* task_gate,
+                                const int32_t* uniq, const int32_t* group_off, int32_t* counts,
+                                void* y, void* stream);
+
+/*
  * The whole routed branch: omni_route -> omni_schedule -> omni_expert_forward
  * on one stream, intermediates in ws.  idx_out / gate_out (nullable, [L x K])
  * receive the routing decisions.  y as in omni_expert_forward.
