@@ -348,6 +348,182 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
   }
 }
 
+// ---- large batches: activations, then accumulation sweeps over slices of d ----
+//
+// When the fp32 accumulator y (L x d) is larger than about a third of L2, the
+// scatter-adds of the grouped execution miss L2 and every reduction turns
+// into DRAM traffic.  The grouped execution is then split: k_act computes the
+// scalar c = gate * SiLU(x[t] . W[e]) of every task (W rows streamed group by
+// group, as in k_expert_async), and Q sweeps of k_acc each add c * V[e] for
+// one slice of Q columns of d -- only that slice of y is live, and it stays in
+// L2 while the V rows stream past it.  Every task still reads its rows of W
+// and V once, in schedule order, and the group's tokens still get their
+// contributions by scatter-add.
+
+constexpr int kActWarps = 8;
+
+template <typename T, int NV, int R>
+__global__ void __launch_bounds__(kActWarps * 32, 1)
+    k_act(const T* __restrict__ x, const T* __restrict__ W, const int32_t* __restrict__ task_token,
+          const int32_t* __restrict__ task_expert, const float* __restrict__ task_gate,
+          int64_t M, int64_t L, int64_t N, int d, int S, int64_t nslices, float* __restrict__ cbuf,
+          int32_t* status) {
+  constexpr int SLOT = NV * 32;  // uint4 per ring slot: one W row
+  extern __shared__ __align__(16) uint4 ring[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4* wring = ring + static_cast<size_t>(warp) * R * SLOT;
+  const uint32_t wring_s = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
+  const uint64_t pol_stream = policy_evict_first();
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * kActWarps;
+  for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kActWarps + warp; sl < nslices; sl += nw) {
+    const int64_t a0 = sl * S;
+    const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
+    int64_t my_t = -1, my_e = -1;
+    float my_g = 0.0f, my_c = 0.0f;
+    if (lane < n) {
+      my_t = task_token[a0 + lane];
+      my_e = task_expert[a0 + lane];
+      my_g = task_gate[a0 + lane];
+      if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
+        raise_status(status, OMNI_DEV_BAD_INDEX);
+        my_e = -1;
+        my_t = -1;
+      }
+    }
+    const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
+    const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
+    auto issue = [&](int j) {
+      if (j < n) {
+        const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+        if (e >= 0) {
+          const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
+          const uint32_t base = wring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
+#pragma unroll
+          for (int v = 0; v < NV; ++v)
+            cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, wr + v * 32 + lane, pol_stream);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int j = 0; j < R - 1; ++j) issue(j);
+    uint4 xc[NV], xn[NV];
+    {
+      const int64_t t0 = __shfl_sync(0xffffffffu, my_t, 0);
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (t0 < 0 ? 0 : t0) * d);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
+    }
+    for (int j = 0; j < n; ++j) {
+      issue(j + R - 1);
+      if ((starts >> j) & 1u) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) xc[v] = xn[v];
+        const uint32_t later = starts & ~((2u << j) - 1u);
+        if (later) {
+          const int jn = __ffs(later) - 1;
+          const int64_t tn = __shfl_sync(0xffffffffu, my_t, jn);
+          const uint4* xr = reinterpret_cast<const uint4*>(x + (tn < 0 ? 0 : tn) * d);
+#pragma unroll
+          for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
+        }
+      }
+      cp_async_wait<R - 1>();
+      const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+      const float gj = __shfl_sync(0xffffffffu, my_g, j);
+      if (e >= 0) {  // warp-uniform
+        const uint4* slot = wring + (j % R) * SLOT;
+        float sdot = 0.0f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
+        sdot = warp_sum(sdot);
+        if (lane == j) my_c = gj * silu(sdot);
+      }
+    }
+    cp_async_wait<0>();
+    if (lane < n) cbuf[a0 + lane] = my_c;
+  }
+}
+
+constexpr int kAccThreads = 128;
+constexpr int kAccUnroll = 4;  // value-row loads in flight per warp
+
+// One sweep: y[t, col0 : col0 + 32*NVQ*EPV] += sum over the piece of c * V[e, same columns].
+template <typename T, int NVQ>
+__global__ void __launch_bounds__(kAccThreads)
+    k_acc(const T* __restrict__ V, const int32_t* __restrict__ task_token,
+          const int32_t* __restrict__ task_expert, const float* __restrict__ cbuf, int64_t M,
+          int64_t L, int64_t N, int d, int col0, int S, float* __restrict__ yacc) {
+  constexpr int EPV = kEpv<T>;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kAccThreads + threadIdx.x) >> 5;
+  const int64_t a0 = wid * S;
+  if (a0 >= M) return;
+  const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
+  const uint64_t pol_stream = policy_evict_first();
+  const uint64_t pol_keep = policy_evict_last();
+  int64_t my_t = -1, my_e = -1;
+  float my_c = 0.0f;
+  if (lane < n) {
+    my_t = task_token[a0 + lane];
+    my_e = task_expert[a0 + lane];
+    my_c = cbuf[a0 + lane];
+    if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
+      my_e = -1;
+      my_t = -1;
+    }
+  }
+  const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
+  uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
+  while (starts) {
+    const int p = __ffs(starts) - 1;
+    starts &= starts - 1;
+    const int q = starts ? __ffs(starts) - 1 : n;
+    const int64_t t = __shfl_sync(0xffffffffu, my_t, p);
+    float acc[NVQ * EPV];
+#pragma unroll
+    for (int u = 0; u < NVQ * EPV; ++u) acc[u] = 0.0f;
+    for (int j0 = p; j0 < q; j0 += kAccUnroll) {
+      uint4 vv[kAccUnroll][NVQ];
+      float cc[kAccUnroll];
+#pragma unroll
+      for (int u = 0; u < kAccUnroll; ++u) {
+        const int j = j0 + u;
+        const int64_t e = __shfl_sync(0xffffffffu, my_e, j < q ? j : p);
+        cc[u] = __shfl_sync(0xffffffffu, my_c, j < q ? j : p);
+        const bool ok = j < q && e >= 0;
+        if (!ok) cc[u] = 0.0f;
+        const uint4* vr = reinterpret_cast<const uint4*>(V + (ok ? e : 0) * d + col0);
+#pragma unroll
+        for (int v = 0; v < NVQ; ++v) {
+          if (ok) {
+            asm volatile("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                         : "=r"(vv[u][v].x), "=r"(vv[u][v].y), "=r"(vv[u][v].z), "=r"(vv[u][v].w)
+                         : "l"(vr + v * 32 + lane), "l"(pol_stream));
+          } else {
+            vv[u][v] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kAccUnroll; ++u)
+#pragma unroll
+        for (int v = 0; v < NVQ; ++v) axpy_vec(cc[u], vv[u][v], acc + v * EPV, static_cast<T*>(nullptr));
+    }
+    if (t >= 0) {
+      float* yr = yacc + t * d + col0;
+#pragma unroll
+      for (int v = 0; v < NVQ; ++v) {
+        float* o = yr + static_cast<int64_t>(v * 32 + lane) * EPV;
+#pragma unroll
+        for (int u = 0; u < EPV; u += 4)
+          red_add_v4_keep(o + u, acc[v * EPV + u], acc[v * EPV + u + 1], acc[v * EPV + u + 2],
+                          acc[v * EPV + u + 3], pol_keep);
+      }
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src, T* __restrict__ dst,
                                               int64_t n) {
@@ -419,9 +595,30 @@ __global__ void __launch_bounds__(kTokThreads)
 
 }  // namespace
 
+// Number of accumulation sweeps: 1 keeps the fused kernel; Q > 1 splits the
+// columns of d so that each live slice of the fp32 accumulator is <= ~40 MiB.
+int expert_sweeps(const Dims& D) {
+  const int epv = D.dtype == OMNI_F32 ? 4 : 8;
+  const int64_t ybytes = D.L * D.d * 4;
+  const int64_t limit = int64_t(40) << 20;
+  if (ybytes <= limit) return 1;
+  const int64_t nv = D.d % (32 * epv) == 0 ? D.d / (32 * epv) : 0;
+  if (nv != 2 && nv != 4 && nv != 8) return 1;  // row shapes the sweep kernels are built for
+  for (int Q = 2; Q <= 16; Q *= 2) {
+    if (D.d % Q != 0) break;
+    const int64_t cols = D.d / Q;
+    if (cols % (32 * epv) != 0) break;
+    const int64_t nvq = cols / (32 * epv);
+    if (nvq > 4) continue;
+    if (ybytes / Q <= limit) return (nvq == 1 || nvq == 2 || nvq == 4) ? Q : 1;
+  }
+  return 1;
+}
+
 size_t expert_ws_bytes(const Dims& D) {
-  if (D.dtype == OMNI_F32) return 0;
-  return static_cast<size_t>(D.L) * D.d * sizeof(float);
+  size_t b = D.dtype == OMNI_F32 ? 0 : static_cast<size_t>(D.L) * D.d * sizeof(float);
+  if (expert_sweeps(D) > 1) b = ((b + 255) & ~size_t(255)) + static_cast<size_t>(D.M()) * sizeof(float);
+  return b;
 }
 
 template <typename T, int NV>
@@ -483,6 +680,57 @@ cudaError_t dispatch_slices(const Dims& D, const void* x, const void* W, const v
   }
 }
 
+template <typename T, int NV, int NVQ>
+cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const void* V,
+                      const int32_t* tt, const int32_t* te, const float* tg, float* cbuf,
+                      float* acc, int32_t* status, cudaStream_t s) {
+  constexpr int R = 6;
+  constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
+  cudaError_t err = cudaFuncSetAttribute(k_act<T, NV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t M = D.M();
+  const int S = 32;
+  const int64_t nslices = (M + S - 1) / S;
+  int64_t blocks = (nslices + kActWarps - 1) / kActWarps;
+  if (blocks > sms) blocks = sms;
+  k_act<T, NV, R><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
+      static_cast<const T*>(x), static_cast<const T*>(W), tt, te, tg, M, D.L, D.N(),
+      static_cast<int>(D.d), S, nslices, cbuf, status);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t ablocks = (nslices + kAccThreads / 32 - 1) / (kAccThreads / 32);
+  const int cols = static_cast<int>(D.d / Q);
+  for (int q = 0; q < Q; ++q) {
+    k_acc<T, NVQ><<<static_cast<unsigned>(ablocks), kAccThreads, 0, s>>>(
+        static_cast<const T*>(V), tt, te, cbuf, M, D.L, D.N(), static_cast<int>(D.d), q * cols, S,
+        acc);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, const void* V,
+                          const int32_t* tt, const int32_t* te, const float* tg, float* cbuf,
+                          float* acc, int32_t* status, cudaStream_t s) {
+  constexpr int row = 32 * kEpv<T>;
+  const int64_t nv = D.d / row;             // vectors per lane for a whole row
+  const int64_t nvq = (D.d / Q) / row;      // ... for one slice
+  if (D.d % row != 0) return cudaErrorInvalidValue;
+#define OMNI_SWEEP(NV_, NVQ_)                                                               \
+  if (nv == NV_ && nvq == NVQ_)                                                             \
+    return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, cbuf, acc, status, s);
+  OMNI_SWEEP(8, 4) OMNI_SWEEP(8, 2) OMNI_SWEEP(8, 1) OMNI_SWEEP(4, 2) OMNI_SWEEP(4, 1)
+  OMNI_SWEEP(2, 1)
+#undef OMNI_SWEEP
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* group_off,
@@ -495,9 +743,19 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   cudaError_t err = cudaMemsetAsync(acc, 0, ybytes, s);
   if (err != cudaSuccess) return err;
   int32_t* status = const_cast<int32_t*>(counts) + 2;
-  err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
-            : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
-                                             status, s);
+  const int Q = expert_sweeps(D);
+  if (Q > 1) {
+    size_t off = f32 ? 0 : ((ybytes + 255) & ~size_t(255));
+    float* cbuf = reinterpret_cast<float*>(static_cast<char*>(ws) + off);
+    err = f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate, cbuf, acc,
+                                     status, s)
+              : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
+                                             cbuf, acc, status, s);
+  } else {
+    err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
+              : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
+                                               status, s);
+  }
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;
   k_cast<__nv_bfloat16><<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(

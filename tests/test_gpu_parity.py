@@ -359,3 +359,31 @@ def test_empty_batch():
                          torch.zeros((cfg.Nc, cfg.d), device="cuda"), W, W,
                          y=torch.empty((0, cfg.d), device="cuda"))
     assert y.shape == (0, cfg.d)
+
+
+SWEEP = [
+    WL.Config("sweeps-bf16", L=8192, d=2048, Nr=64, Nc=64, k=8, K=8, B=32, dtype=WL.BF16, seed=31),
+    WL.Config("sweeps-f32", L=12288, d=1024, Nr=48, Nc=40, k=6, K=5, B=16, dtype=WL.F32, seed=32),
+]
+
+
+@pytest.mark.parametrize("cfg", SWEEP, ids=[c.name for c in SWEEP])
+def test_expert_sweeps_path(cfg):
+    """Batches whose fp32 accumulator exceeds ~40 MiB run as an activation pass
+    plus accumulation sweeps over column slices: same y as the oracle."""
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    oi, og, _ = O.route(cfg, h)
+    g32 = og.astype(np.float32)
+    ref_s = O.schedule(cfg, oi, g32.astype(np.float64))
+    y_ref, _ = O.forward_expert(cfg, h, ref_s)
+    counts = torch.tensor([ref_s["n_active"], ref_s["n_groups"], 0, 0], dtype=torch.int32,
+                          device="cuda")
+    sched = {"task_token": dev(ref_s["task_token"]), "task_expert": dev(ref_s["task_expert"]),
+             "task_gate": dev(ref_s["task_gate"].astype(np.float32)),
+             "uniq": dev(ref_s["uniq"]), "group_off": dev(ref_s["group_off"]), "counts": counts}
+    D = omni.LayerDims.of(cfg)
+    assert cfg.L * cfg.d * 4 > (40 << 20)
+    y = omni.expert_forward(D, d["x"], d["W"], d["V"], sched)
+    assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
+    assert int(counts[2].item()) == 0

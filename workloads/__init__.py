@@ -75,9 +75,10 @@ DECODE = Config("bf16-decode-N1M", L=64, d=2048, Nr=1024, Nc=1024, k=64, K=64, B
 
 CONFIGS = {c.name: c for c in (TINY, BF16_16K, SKEWED, PREFILL, DECODE)}
 
-# A reduced prefill of the same shape for counter captures (W, V 1 GiB each, still
-# far larger than L2; the same tasks per active expert as the prefill workload).
-PREFILL_PROXY = Config("bf16-prefill-proxy-N256K", L=4096, d=2048, Nr=512, Nc=512, k=64, K=64,
+# A reduced prefill for counter captures: W, V 1 GiB each (far larger than L2),
+# L*K = N (the same tasks per active expert as the prefill workload), and an
+# fp32 accumulator above 40 MiB (the same execution path).
+PREFILL_PROXY = Config("bf16-prefill-proxy-N256K", L=8192, d=2048, Nr=512, Nc=512, k=32, K=32,
                        B=128, dtype=BF16)
 DECODE_PROXY = Config("bf16-decode-proxy-N256K", L=64, d=2048, Nr=512, Nc=512, k=64, K=64,
                       B=128, dtype=BF16)
