@@ -364,7 +364,8 @@ __device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, fl
 
 struct SelPlan {
   int nr_pad, nc_pad, kp, Kp, cand;  // sizes (elements)
-  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc;
+  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc,
+      off_roff;
   int pair_bytes;
 };
 
@@ -394,6 +395,7 @@ SelPlan make_plan(const Dims& D) {
   p.off_misc = off; off = al(off + 16);
   p.off_tr = off; off = al(off + 8 * kCandMax);
   p.off_tc = off; off = al(off + 8 * kCandMax);
+  p.off_roff = off; off = al(off + 4 * static_cast<int>(D.k));
   p.pair_bytes = off;
   return p;
 }
@@ -460,24 +462,42 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   uint64_t* out = reinterpret_cast<uint64_t*>(base + P.off_out);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + P.off_hr);
   uint64_t* tbin = reinterpret_cast<uint64_t*>(base + P.off_tr);
-  int nc = 0;
-  float cmx = -INFINITY, cmn = INFINITY;
-  for (int a = 0; a < k; ++a) {
-    int nb = K / (a + 1);
-    if (nb > k) nb = k;
-    if (nb <= 0) break;
-    const uint64_t ra = sr[a];
-    const float za = key_val(ra);
-    const uint32_t ia = key_id(ra);
-    for (int b = lane; b < nb; b += 32) {
-      const uint64_t cb = sc[b];
-      const float sv = za + key_val(cb);
-      const uint32_t e = ia * static_cast<uint32_t>(Nc) + key_id(cb);
-      cand[nc + b] = make_key(sv, e);
-      cmx = fmaxf(cmx, sv);
-      cmn = fminf(cmn, sv);
+  // candidate (a, b) pairs with (a+1)(b+1) <= K, one per lane: row a's pairs
+  // start at roff[a] (prefix of min(k, K/(a+1)) over the rows)
+  int32_t* roff = reinterpret_cast<int32_t*>(base + P.off_roff);
+  int na = 0;
+  for (int a0 = 0; a0 < k; a0 += 32) {
+    const int a = a0 + lane;
+    int nb = 0;
+    if (a < k) {
+      nb = K / (a + 1);
+      if (nb > k) nb = k;
     }
-    nc += nb;
+    int incl = nb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t2;
+    }
+    if (a < k) roff[a] = na + incl - nb;
+    na += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  const int nc = na;
+  float cmx = -INFINITY, cmn = INFINITY;
+  for (int c = lane; c < nc; c += 32) {
+    int lo = 0, hi = k - 1;  // last row a with roff[a] <= c
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (roff[mid] <= c) lo = mid; else hi = mid - 1;
+    }
+    const int a = lo, b = c - roff[a];
+    const uint64_t ra = sr[a], cb = sc[b];
+    const float sv = key_val(ra) + key_val(cb);
+    const uint32_t e = key_id(ra) * static_cast<uint32_t>(Nc) + key_id(cb);
+    cand[c] = make_key(sv, e);
+    cmx = fmaxf(cmx, sv);
+    cmn = fminf(cmn, sv);
   }
   cmx = warp_max(cmx);
   cmn = -warp_max(-cmn);
