@@ -24,6 +24,7 @@
 //
 // Token-centric order (the ablation the scheduling replaces, section 2.2):
 // CTA t gathers the rows of its own K experts; no reductions across CTAs.
+#include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -352,12 +353,13 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
 //
 // When the fp32 accumulator y (L x d) is larger than about a third of L2, the
 // scatter-adds of the grouped execution miss L2 and every reduction turns
-// into DRAM traffic.  The grouped execution is then split: k_act computes the
-// scalar c = gate * SiLU(x[t] . W[e]) of every task (W rows streamed group by
-// group, as in k_expert_async), and Q sweeps of k_acc each add c * V[e] for
-// one slice of Q columns of d -- only that slice of y is live, and it stays in
-// L2 while the V rows stream past it.  Every task still reads its rows of W
-// and V once, in schedule order, and the group's tokens still get their
+// into DRAM traffic.  The grouped execution is then split: k_wsort merges
+// consecutive groups into windows ordered by token, k_act computes the scalar
+// c = gate * SiLU(x[t] . W[e]) of every task (W rows streamed window by
+// window, as in k_expert_async), and Q sweeps of k_acc each add
+// c * V[e] for one slice of Q columns of d -- only that slice of y is live,
+// and it stays in L2 while the V rows stream past it.  Every task still
+// reads its rows of W and V once, and the tokens of a window still get their
 // contributions by scatter-add.
 
 constexpr int kActWarps = 8;
@@ -445,82 +447,229 @@ __global__ void __launch_bounds__(kActWarps * 32, 1)
   }
 }
 
-constexpr int kAccThreads = 128;
-constexpr int kAccUnroll = 4;  // value-row loads in flight per warp
+// ---- windows: consecutive groups merged per token --------------------------
+//
+// A token's K experts lie in few rows of the Nr x Nc grid, so they fall into
+// far fewer windows of consecutive groups than groups.  Inside a window of
+// whole groups (about kWinTasks tasks) k_wsort orders the tasks by token
+// (stable: a token's tasks keep their group and expert order), so the sweeps
+// below can add a token's contributions from the whole window with one
+// scatter-add instead of one per group.  Every group is still executed as a
+// unit -- its rows are read while its window is in flight -- and every task
+// exactly once.
+constexpr int kWinTasks = 7168;
 
-// One sweep: y[t, col0 : col0 + 32*NVQ*EPV] += sum over the piece of c * V[e, same columns].
-template <typename T, int NVQ>
-__global__ void __launch_bounds__(kAccThreads)
+// Window w takes the groups whose first task lies in [w*T, (w+1)*T).  Windows
+// larger than the CTA sort (a single very large group) and the whole batch
+// when the group count on the device is out of range are copied in schedule
+// order (the latter with OMNI_DEV_BAD_INDEX raised).
+__global__ void __launch_bounds__(kBlockSortThreads)
+    k_wsort(const int32_t* __restrict__ tt, const int32_t* __restrict__ te,
+            const float* __restrict__ tg, const int32_t* __restrict__ group_off,
+            const int32_t* __restrict__ counts, int64_t M, int64_t gmax, int T, int passes,
+            int32_t* __restrict__ wt, int32_t* __restrict__ we, float* __restrict__ wg,
+            int32_t* status) {
+  extern __shared__ __align__(16) uint8_t wsm[];
+  uint32_t* kA = reinterpret_cast<uint32_t*>(wsm);
+  uint32_t* kB = kA + kBlockSortMax;
+  uint16_t* vA = reinterpret_cast<uint16_t*>(kB + kBlockSortMax);
+  uint16_t* vB = vA + kBlockSortMax;
+  uint32_t* wcount = reinterpret_cast<uint32_t*>(vB + kBlockSortMax);
+  __shared__ uint32_t dbase[256];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int64_t rng[2];
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * T;
+  const int64_t hi = M - lo < T ? M : lo + T;
+  if (threadIdx.x == 0) {
+    const int64_t G = counts[1];
+    int64_t a0 = lo, a1 = hi;
+    if (G < 1 || G > gmax) {
+      raise_status(status, OMNI_DEV_BAD_INDEX);
+    } else {
+      // first group starting at or after v (group_off[G] == M closes the list)
+      auto first_at = [&](int64_t v) {
+        int64_t l = 0, h = G;
+        while (l < h) {
+          const int64_t m = (l + h) >> 1;
+          if (group_off[m] >= v) h = m; else l = m + 1;
+        }
+        return l;
+      };
+      const int64_t g0 = first_at(lo), g1 = first_at(hi);
+      const int64_t b0 = g0 >= G ? M : group_off[g0];
+      const int64_t b1 = g1 >= G ? M : group_off[g1];
+      if (b0 < 0 || b1 > M || b0 > b1) {
+        raise_status(status, OMNI_DEV_BAD_INDEX);
+      } else {
+        a0 = b0;
+        a1 = b1;
+      }
+    }
+    rng[0] = a0;
+    rng[1] = a1;
+  }
+  __syncthreads();
+  const int64_t a0 = rng[0];
+  const int64_t n = rng[1] - a0;
+  if (n <= 0) return;
+  if (n > kBlockSortMax) {
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+      wt[a0 + i] = tt[a0 + i];
+      we[a0 + i] = te[a0 + i];
+      wg[a0 + i] = tg[a0 + i];
+    }
+    return;
+  }
+  const int nn = static_cast<int>(n);
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    kA[i] = static_cast<uint32_t>(tt[a0 + i]);
+    vA[i] = static_cast<uint16_t>(i);
+  }
+  __syncthreads();
+  uint32_t* kin = kA; uint32_t* kout = kB;
+  uint16_t* vin = vA; uint16_t* vout = vB;
+  for (int p = 0; p < passes; ++p) {
+    block_radix_pass(kin, vin, kout, vout, nn, 8 * p, wcount, dbase, warp_tot, &total);
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const int src = vin[i];
+    wt[a0 + i] = tt[a0 + src];
+    we[a0 + i] = te[a0 + src];
+    wg[a0 + i] = tg[a0 + src];
+  }
+}
+
+constexpr int kAccWarps = 4;
+
+// Four consecutive elements of T as one load: bf16 -> 8 bytes, fp32 -> 16 bytes.
+template <typename T> struct Quad;
+template <> struct Quad<__nv_bfloat16> { using type = uint2; };
+template <> struct Quad<float> { using type = uint4; };
+
+__device__ __forceinline__ uint2 ld_quad(const __nv_bfloat16* p, uint64_t pol) {
+  uint2 r;
+  asm volatile("ld.global.nc.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+               : "=r"(r.x), "=r"(r.y) : "l"(p), "l"(pol));
+  return r;
+}
+__device__ __forceinline__ uint4 ld_quad(const float* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "l"(pol));
+  return r;
+}
+__device__ __forceinline__ void fma_quad(float c, uint2 v, float* a) {
+  a[0] = fmaf(c, bf16lo(v.x), a[0]); a[1] = fmaf(c, bf16hi(v.x), a[1]);
+  a[2] = fmaf(c, bf16lo(v.y), a[2]); a[3] = fmaf(c, bf16hi(v.y), a[3]);
+}
+__device__ __forceinline__ void fma_quad(float c, uint4 v, float* a) {
+  a[0] = fmaf(c, __uint_as_float(v.x), a[0]); a[1] = fmaf(c, __uint_as_float(v.y), a[1]);
+  a[2] = fmaf(c, __uint_as_float(v.z), a[2]); a[3] = fmaf(c, __uint_as_float(v.w), a[3]);
+}
+
+// One sweep over the window-ordered tasks: y[t, col0 : col0 + 128*NB] +=
+// c * V[e, same columns], summed over each run of one token's tasks in a
+// 32-task slice and added with one vector reduction per run and 128 columns.
+// Lane l owns columns col0 + 128*b + 4*l .. +3 of every block b, so each
+// reduction instruction covers 512 contiguous bytes of y (whole sectors).
+// Warps take slices round-robin (the whole grid moves through the task list
+// together, so a window's re-used V rows are still in L2); the V loads run D
+// tasks ahead in registers, across run and slice boundaries.
+template <typename T, int NB, int D>
+__global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
     k_acc(const T* __restrict__ V, const int32_t* __restrict__ task_token,
           const int32_t* __restrict__ task_expert, const float* __restrict__ cbuf, int64_t M,
-          int64_t L, int64_t N, int d, int col0, int S, float* __restrict__ yacc) {
-  constexpr int EPV = kEpv<T>;
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kAccThreads + threadIdx.x) >> 5;
-  const int64_t a0 = wid * S;
-  if (a0 >= M) return;
-  const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
+          int64_t L, int64_t N, int d, int col0, int64_t nslices, float* __restrict__ yacc) {
+  static_assert(32 % D == 0, "the prefetch distance divides the slice");
+  using QT = typename Quad<T>::type;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t pol_stream = policy_evict_first();
   const uint64_t pol_keep = policy_evict_last();
-  int64_t my_t = -1, my_e = -1;
-  float my_c = 0.0f;
-  if (lane < n) {
-    my_t = task_token[a0 + lane];
-    my_e = task_expert[a0 + lane];
-    my_c = cbuf[a0 + lane];
-    if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
-      my_e = -1;
-      my_t = -1;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * kAccWarps;
+  int64_t sl = static_cast<int64_t>(blockIdx.x) * kAccWarps + warp;
+  if (sl >= nslices) return;
+  struct Meta {
+    int n, t, e;
+    float c;
+  };
+  auto load_meta = [&](int64_t s) {
+    Meta m{0, -1, -1, 0.0f};
+    if (s < nslices) {
+      const int64_t a0 = s * 32;
+      m.n = static_cast<int>(M - a0 < 32 ? M - a0 : 32);
+      if (lane < m.n) {
+        const int64_t t = task_token[a0 + lane];
+        const int64_t e = task_expert[a0 + lane];
+        if (t >= 0 && t < L && e >= 0 && e < N) {
+          m.t = static_cast<int>(t);
+          m.e = static_cast<int>(e);
+          m.c = cbuf[a0 + lane];
+        }
+      }
     }
-  }
-  const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
-  uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
-  while (starts) {
-    const int p = __ffs(starts) - 1;
-    starts &= starts - 1;
-    const int q = starts ? __ffs(starts) - 1 : n;
-    const int64_t t = __shfl_sync(0xffffffffu, my_t, p);
-    float acc[NVQ * EPV];
+    return m;
+  };
+  Meta cur = load_meta(sl);
+  Meta nxt = load_meta(sl + nw);
+  // position p counts from the current slice's first task; p >= 32 lies in
+  // the warp's next slice (only a full slice is followed by another)
+  auto issue = [&](int p, QT (&b)[NB]) {
+    int e = -1;
+    if (p < cur.n) {
+      e = __shfl_sync(0xffffffffu, cur.e, p);
+    } else if (cur.n == 32 && p - 32 < nxt.n) {
+      e = __shfl_sync(0xffffffffu, nxt.e, p - 32);
+    }
+    if (e >= 0) {  // warp-uniform
+      const T* row = V + static_cast<int64_t>(e) * d + col0 + 4 * lane;
 #pragma unroll
-    for (int u = 0; u < NVQ * EPV; ++u) acc[u] = 0.0f;
-    for (int j0 = p; j0 < q; j0 += kAccUnroll) {
-      uint4 vv[kAccUnroll][NVQ];
-      float cc[kAccUnroll];
+      for (int bb = 0; bb < NB; ++bb) b[bb] = ld_quad(row + 128 * bb, pol_stream);
+    }
+  };
+  QT buf[D][NB];
 #pragma unroll
-      for (int u = 0; u < kAccUnroll; ++u) {
-        const int j = j0 + u;
-        const int64_t e = __shfl_sync(0xffffffffu, my_e, j < q ? j : p);
-        cc[u] = __shfl_sync(0xffffffffu, my_c, j < q ? j : p);
-        const bool ok = j < q && e >= 0;
-        if (!ok) cc[u] = 0.0f;
-        const uint4* vr = reinterpret_cast<const uint4*>(V + (ok ? e : 0) * d + col0);
+  for (int q = 0; q < D; ++q) issue(q, buf[q]);
+  float acc[NB][4];
 #pragma unroll
-        for (int v = 0; v < NVQ; ++v) {
-          if (ok) {
-            asm volatile("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-                         : "=r"(vv[u][v].x), "=r"(vv[u][v].y), "=r"(vv[u][v].z), "=r"(vv[u][v].w)
-                         : "l"(vr + v * 32 + lane), "l"(pol_stream));
-          } else {
-            vv[u][v] = make_uint4(0u, 0u, 0u, 0u);
+  for (int bb = 0; bb < NB; ++bb) acc[bb][0] = acc[bb][1] = acc[bb][2] = acc[bb][3] = 0.0f;
+  while (true) {
+    const int next_t = __shfl_down_sync(0xffffffffu, cur.t, 1);
+    const uint32_t ends =
+        __ballot_sync(0xffffffffu, lane < cur.n && (lane == cur.n - 1 || next_t != cur.t));
+    for (int j0 = 0; j0 < 32; j0 += D) {
+#pragma unroll
+      for (int q = 0; q < D; ++q) {
+        const int j = j0 + q;
+        if (j < cur.n) {  // warp-uniform
+          const int e = __shfl_sync(0xffffffffu, cur.e, j);
+          const float c = __shfl_sync(0xffffffffu, cur.c, j);
+          if (e >= 0) {
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) fma_quad(c, buf[q][bb], acc[bb]);
+          }
+          issue(j + D, buf[q]);
+          if ((ends >> j) & 1u) {
+            const int t = __shfl_sync(0xffffffffu, cur.t, j);
+            if (t >= 0) {
+              float* yr = yacc + static_cast<int64_t>(t) * d + col0 + 4 * lane;
+#pragma unroll
+              for (int bb = 0; bb < NB; ++bb)
+                red_add_v4_keep(yr + 128 * bb, acc[bb][0], acc[bb][1], acc[bb][2], acc[bb][3],
+                                pol_keep);
+            }
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) acc[bb][0] = acc[bb][1] = acc[bb][2] = acc[bb][3] = 0.0f;
           }
         }
       }
-#pragma unroll
-      for (int u = 0; u < kAccUnroll; ++u)
-#pragma unroll
-        for (int v = 0; v < NVQ; ++v) axpy_vec(cc[u], vv[u][v], acc + v * EPV, static_cast<T*>(nullptr));
     }
-    if (t >= 0) {
-      float* yr = yacc + t * d + col0;
-#pragma unroll
-      for (int v = 0; v < NVQ; ++v) {
-        float* o = yr + static_cast<int64_t>(v * 32 + lane) * EPV;
-#pragma unroll
-        for (int u = 0; u < EPV; u += 4)
-          red_add_v4_keep(o + u, acc[v * EPV + u], acc[v * EPV + u + 1], acc[v * EPV + u + 2],
-                          acc[v * EPV + u + 3], pol_keep);
-      }
-    }
+    sl += nw;
+    if (sl >= nslices) break;
+    cur = nxt;
+    nxt = load_meta(sl + nw);
   }
 }
 
@@ -615,9 +764,36 @@ int expert_sweeps(const Dims& D) {
   return 1;
 }
 
+// Workspace of the sweeps path, after the fp32 accumulator: the activations
+// c and the window-ordered copy of the task list.
+struct SweepWs {
+  float* cbuf;
+  int32_t* wt;
+  int32_t* we;
+  float* wg;
+};
+
+size_t acc_bytes(const Dims& D) {
+  return D.dtype == OMNI_F32 ? 0 : static_cast<size_t>(D.L) * D.d * sizeof(float);
+}
+
+SweepWs carve_sweeps(const Dims& D, void* ws, size_t* bytes) {
+  Carver c(ws);
+  c.take<char>(acc_bytes(D));
+  SweepWs w;
+  const size_t M = static_cast<size_t>(D.M());
+  w.cbuf = c.take<float>(M);
+  w.wt = c.take<int32_t>(M);
+  w.we = c.take<int32_t>(M);
+  w.wg = c.take<float>(M);
+  if (bytes) *bytes = c.off;
+  return w;
+}
+
 size_t expert_ws_bytes(const Dims& D) {
-  size_t b = D.dtype == OMNI_F32 ? 0 : static_cast<size_t>(D.L) * D.d * sizeof(float);
-  if (expert_sweeps(D) > 1) b = ((b + 255) & ~size_t(255)) + static_cast<size_t>(D.M()) * sizeof(float);
+  if (expert_sweeps(D) <= 1) return acc_bytes(D);
+  size_t b = 0;
+  carve_sweeps(D, nullptr, &b);
   return b;
 }
 
@@ -680,35 +856,83 @@ cudaError_t dispatch_slices(const Dims& D, const void* x, const void* W, const v
   }
 }
 
-template <typename T, int NV, int NVQ>
-cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const void* V,
-                      const int32_t* tt, const int32_t* te, const float* tg, float* cbuf,
-                      float* acc, int32_t* status, cudaStream_t s) {
-  constexpr int R = 6;
-  constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
-  cudaError_t err = cudaFuncSetAttribute(k_act<T, NV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
+int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, const float* tg,
+                         const int32_t* group_off, const int32_t* counts, const SweepWs& w,
+                         int32_t* status, cudaStream_t s) {
+  constexpr size_t smem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 2 * 2) +
+                          static_cast<size_t>(kBlockSortWarps) * 256 * 4;
+  cudaError_t err = cudaFuncSetAttribute(k_wsort, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int64_t M = D.M();
+  // about one window per SM, within what one CTA sorts
+  int64_t T = (M + sm_count() - 1) / sm_count();
+  T = T < 1024 ? 1024 : (T > kWinTasks ? kWinTasks : T);
+  const int64_t nwin = (M + T - 1) / T;
+  int bits = 0;
+  while ((int64_t(1) << bits) < D.L) ++bits;
+  const int passes = (bits + 7) / 8;
+  k_wsort<<<static_cast<unsigned>(nwin), kBlockSortThreads, smem, s>>>(
+      tt, te, tg, group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.wt, w.we, w.wg,
+      status);
+  return cudaGetLastError();
+}
+
+template <typename T, int NB, int D>
+cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w, float* acc,
+                       cudaStream_t s) {
+  int per_sm = 1;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_acc<T, NB, D>,
+                                                                  kAccWarps * 32, 0);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t M = D_.M();
+  const int64_t nslices = (M + 31) / 32;
+  int64_t blocks = (nslices + kAccWarps - 1) / kAccWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  if (blocks > cap) blocks = cap;
+  k_acc<T, NB, D><<<static_cast<unsigned>(blocks), kAccWarps * 32, 0, s>>>(
+      static_cast<const T*>(V), w.wt, w.we, w.cbuf, M, D_.L, D_.N(), static_cast<int>(D_.d), col0,
+      nslices, acc);
+  return cudaGetLastError();
+}
+
+template <typename T, int NV, int NVQ>
+cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const void* V,
+                      const int32_t* tt, const int32_t* te, const float* tg,
+                      const int32_t* group_off, const int32_t* counts, const SweepWs& w,
+                      float* acc, int32_t* status, cudaStream_t s) {
+  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, status, s);
+  if (err != cudaSuccess) return err;
+  constexpr int R = 6;
+  constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
+  err = cudaFuncSetAttribute(k_act<T, NV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
   const int64_t M = D.M();
   const int S = 32;
   const int64_t nslices = (M + S - 1) / S;
   int64_t blocks = (nslices + kActWarps - 1) / kActWarps;
-  if (blocks > sms) blocks = sms;
+  if (blocks > sm_count()) blocks = sm_count();
   k_act<T, NV, R><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
-      static_cast<const T*>(x), static_cast<const T*>(W), tt, te, tg, M, D.L, D.N(),
-      static_cast<int>(D.d), S, nslices, cbuf, status);
+      static_cast<const T*>(x), static_cast<const T*>(W), w.wt, w.we, w.wg, M, D.L, D.N(),
+      static_cast<int>(D.d), S, nslices, w.cbuf, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int64_t ablocks = (nslices + kAccThreads / 32 - 1) / (kAccThreads / 32);
   const int cols = static_cast<int>(D.d / Q);
+  // 128-column blocks per slice and the prefetch distance (about 16 vectors
+  // of loads in flight per lane)
+  constexpr int NB = NVQ * 32 * kEpv<T> / 128;
+  constexpr int PD = 8 / NVQ;
   for (int q = 0; q < Q; ++q) {
-    k_acc<T, NVQ><<<static_cast<unsigned>(ablocks), kAccThreads, 0, s>>>(
-        static_cast<const T*>(V), tt, te, cbuf, M, D.L, D.N(), static_cast<int>(D.d), q * cols, S,
-        acc);
-    err = cudaGetLastError();
+    err = launch_acc<T, NB, PD>(D, q * cols, V, w, acc, s);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
@@ -716,7 +940,8 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
 
 template <typename T>
 cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, const void* V,
-                          const int32_t* tt, const int32_t* te, const float* tg, float* cbuf,
+                          const int32_t* tt, const int32_t* te, const float* tg,
+                          const int32_t* group_off, const int32_t* counts, const SweepWs& w,
                           float* acc, int32_t* status, cudaStream_t s) {
   constexpr int row = 32 * kEpv<T>;
   const int64_t nv = D.d / row;             // vectors per lane for a whole row
@@ -724,7 +949,8 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
   if (D.d % row != 0) return cudaErrorInvalidValue;
 #define OMNI_SWEEP(NV_, NVQ_)                                                               \
   if (nv == NV_ && nvq == NVQ_)                                                             \
-    return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, cbuf, acc, status, s);
+    return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, group_off, counts, w, acc,    \
+                                   status, s);
   OMNI_SWEEP(8, 4) OMNI_SWEEP(8, 2) OMNI_SWEEP(8, 1) OMNI_SWEEP(4, 2) OMNI_SWEEP(4, 1)
   OMNI_SWEEP(2, 1)
 #undef OMNI_SWEEP
@@ -735,7 +961,6 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* group_off,
                           const int32_t* counts, void* y, void* ws, cudaStream_t s) {
-  (void)group_off;
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
   float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
@@ -745,12 +970,11 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   int32_t* status = const_cast<int32_t*>(counts) + 2;
   const int Q = expert_sweeps(D);
   if (Q > 1) {
-    size_t off = f32 ? 0 : ((ybytes + 255) & ~size_t(255));
-    float* cbuf = reinterpret_cast<float*>(static_cast<char*>(ws) + off);
-    err = f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate, cbuf, acc,
-                                     status, s)
+    const SweepWs w = carve_sweeps(D, ws, nullptr);
+    err = f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate, group_off,
+                                     counts, w, acc, status, s)
               : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
-                                             cbuf, acc, status, s);
+                                             group_off, counts, w, acc, status, s);
   } else {
     err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
               : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,

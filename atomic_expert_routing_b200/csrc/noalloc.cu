@@ -55,8 +55,9 @@ extern "C" int omni_expert_forward_noalloc(const omni_dims* dims, const void* x,
   int rc = omni_workspace_size(dims, OMNI_WS_EXPERT, &need);  // also validates dims
   if (rc != OMNI_OK) return rc;
   if (dims->L == 0) return OMNI_OK;
-  if (static_cast<size_t>(dims->L) * static_cast<size_t>(dims->d) > kNoAllocMaxElems)
-    return OMNI_ERR_UNSUPPORTED;  // batch too large for the fixed accumulator
+  if (static_cast<size_t>(dims->L) * static_cast<size_t>(dims->d) > kNoAllocMaxElems ||
+      need > sizeof(g_noalloc_acc))
+    return OMNI_ERR_UNSUPPORTED;  // batch too large for the fixed scratch
   auto al16 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(x) || !al16(W) || !al16(V) || !al16(y) || task_token == nullptr ||
       task_expert == nullptr || task_gate == nullptr || group_off == nullptr || counts == nullptr)

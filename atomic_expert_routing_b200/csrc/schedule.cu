@@ -18,6 +18,7 @@
 //             8-bit digits (as many passes as the group-count bound needs);
 //             stability keeps (token, expert) order inside each group;
 //  4. emit    gather the sorted tasks and mark each group's first task.
+#include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -80,32 +81,6 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
 }
 
 // ---- 2. scan of the active flags ------------------------------------------
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    int w = lane < nw ? warp_tot[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
-    }
-    if (lane < nw) warp_tot[lane] = wi - w;
-    if (lane == nw - 1) *total = wi;
-  }
-  __syncthreads();
-  return incl - v + warp_tot[warp];
-}
-
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_reduce(const int32_t* __restrict__ flags, int64_t N, int32_t* __restrict__ tile_sum) {
   __shared__ int warp_tot[32];
@@ -320,67 +295,10 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---- small batches (M <= kSmallMax): the whole schedule in one CTA ----------
-constexpr int kSmallMax = 8192;
-constexpr int kSmallThreads = 1024;
+constexpr int kSmallMax = kBlockSortMax;
+constexpr int kSmallThreads = kBlockSortThreads;
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallRounds = kSmallMax / kSmallThreads;  // rounds of 32 keys per warp
-
-// One stable LSD radix pass (8-bit digit at `shift`) of n <= kSmallMax keys
-// with 16-bit payloads, in shared memory, by the whole CTA.  Warp w ranks
-// keys [w*256, w*256+256) in order (match_any groups equal digits), then the
-// per-warp digit counts are scanned (warp-major inside each digit, then over
-// digits) and every key is scattered to its final slot.
-__device__ void block_radix_pass(const uint32_t* kin, const uint16_t* vin, uint32_t* kout,
-                                 uint16_t* vout, int n, int shift, uint32_t* wcount,
-                                 uint32_t* dbase, int* warp_tot, int* total) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int j = tid; j < kSmallWarps * 256; j += kSmallThreads) wcount[j] = 0u;
-  __syncthreads();
-  uint32_t dig[kSmallRounds], rnk[kSmallRounds];
-#pragma unroll
-  for (int r = 0; r < kSmallRounds; ++r) {
-    const int i = warp * (kSmallRounds * 32) + r * 32 + lane;
-    const bool valid = i < n;
-    dig[r] = valid ? ((kin[i] >> shift) & 255u) : 0xffffffffu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, dig[r]);
-    const int leader = __ffs(peers) - 1;
-    uint32_t old = 0;
-    if (valid && lane == leader) {
-      old = wcount[warp * 256 + dig[r]];
-      wcount[warp * 256 + dig[r]] = old + __popc(peers);
-    }
-    old = __shfl_sync(0xffffffffu, old, leader);
-    rnk[r] = old + __popc(peers & lanemask_lt());
-    __syncwarp();
-  }
-  __syncthreads();
-  if (tid < 256) {
-    uint32_t acc = 0;
-    for (int w = 0; w < kSmallWarps; ++w) {
-      const uint32_t c = wcount[w * 256 + tid];
-      wcount[w * 256 + tid] = acc;
-      acc += c;
-    }
-    dbase[tid] = acc;
-  }
-  __syncthreads();
-  {
-    const int v = tid < 256 ? static_cast<int>(dbase[tid]) : 0;
-    const int ex = block_exclusive_scan(v, warp_tot, total);
-    if (tid < 256) dbase[tid] = static_cast<uint32_t>(ex);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kSmallRounds; ++r) {
-    const int i = warp * (kSmallRounds * 32) + r * 32 + lane;
-    if (i < n) {
-      const uint32_t pos = dbase[dig[r]] + wcount[warp * 256 + dig[r]] + rnk[r];
-      kout[pos] = kin[i];
-      vout[pos] = vin[i];
-    }
-  }
-  __syncthreads();
-}
 
 // Same outputs as the multi-kernel path.  (1) Radix-sort the tasks' expert
 // ids; a scan of the "new id" flags gives U and the rank of every task's

@@ -364,6 +364,9 @@ def test_empty_batch():
 SWEEP = [
     WL.Config("sweeps-bf16", L=8192, d=2048, Nr=64, Nc=64, k=8, K=8, B=32, dtype=WL.BF16, seed=31),
     WL.Config("sweeps-f32", L=12288, d=1024, Nr=48, Nc=40, k=6, K=5, B=16, dtype=WL.F32, seed=32),
+    # one group of all 49152 tasks: its window is larger than one CTA sorts
+    WL.Config("sweeps-one-group", L=12288, d=1024, Nr=8, Nc=8, k=4, K=4, B=64, dtype=WL.BF16,
+              seed=33),
 ]
 
 
@@ -387,3 +390,23 @@ def test_expert_sweeps_path(cfg):
     y = omni.expert_forward(D, d["x"], d["W"], d["V"], sched)
     assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
     assert int(counts[2].item()) == 0
+
+
+def test_expert_sweeps_bad_group_count():
+    """A group count on the device above its bound: the executor flags it
+    (OMNI_DEV_BAD_INDEX) and still executes every task once, in schedule order."""
+    cfg = SWEEP[0]
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    oi, og, _ = O.route(cfg, h)
+    ref_s = O.schedule(cfg, oi, og.astype(np.float32).astype(np.float64))
+    y_ref, _ = O.forward_expert(cfg, h, ref_s)
+    D = omni.LayerDims.of(cfg)
+    gmax = (min(cfg.N, cfg.L * cfg.K) + cfg.B - 1) // cfg.B
+    counts = torch.tensor([ref_s["n_active"], gmax + 7, 0, 0], dtype=torch.int32, device="cuda")
+    sched = {"task_token": dev(ref_s["task_token"]), "task_expert": dev(ref_s["task_expert"]),
+             "task_gate": dev(ref_s["task_gate"].astype(np.float32)),
+             "uniq": dev(ref_s["uniq"]), "group_off": dev(ref_s["group_off"]), "counts": counts}
+    y = omni.expert_forward(D, d["x"], d["W"], d["V"], sched)
+    assert int(counts[2].item()) & omni._lib.OMNI_DEV_BAD_INDEX
+    assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
