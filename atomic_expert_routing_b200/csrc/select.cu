@@ -9,14 +9,17 @@
 //
 // Per token, two warps work side by side: warp 0 takes the Nr row logits,
 // warp 1 the Nc column logits.  Each computes its axis' log-sum-exp and its
-// top-k entries by a warp radix select over 64-bit keys
-// (order-preserving bits of the logit << 32 | ~index), so ties fall to the
-// smaller index.  Warp 0 then forms the joint scores of the k x k candidate
-// pairs that can reach the top-K -- pair (a, b) of the sorted axis lists has
-// (a+1)(b+1) - 1 pairs that score at least as high, so only pairs with
-// (a+1)(b+1) <= K are needed -- and selects the K best by (S desc, e asc),
-// again by radix select over (bits of S << 32 | ~e).  The gate is the
-// softmax of the K selected joint scores.
+// top-k entries over 64-bit keys (order-preserving bits of the logit << 32 |
+// ~index, so ties fall to the smaller index): a 256-bin histogram over the
+// value range finds the bin that holds the k-th key, the keys above it are
+// compacted, the bin itself is sorted for the rest, and the k keys are sorted
+// by a register bitonic network.  Warp 0 then forms the joint scores of the
+// k x k candidate pairs that can reach the top-K -- pair (a, b) of the sorted
+// axis lists has (a+1)(b+1) - 1 pairs that score at least as high, so only
+// pairs with (a+1)(b+1) <= K are needed -- and selects the K best by
+// (S desc, e asc) the same way.  The gate is the softmax of the K selected
+// joint scores.  A radix select over the keys takes over when the value
+// range is degenerate or the threshold bin holds too many keys.
 //
 // Ordering uses the raw fp32 logit sums z_r[i] + z_c[j] (the per-token
 // log-sum-exp terms are constants and only enter the reported score), so no
@@ -133,161 +136,102 @@ __device__ void warp_select_top(KeyFn key, int n, int want, uint64_t* out, uint3
   __syncwarp();
 }
 
-// Bitonic sort of s[0..P) (P a power of two) into descending order, one warp.
-__device__ void warp_sort_desc(uint64_t* s, int P) {
-  const int lane = threadIdx.x & 31;
-  for (int size = 2; size <= P; size <<= 1)
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < P / 2; i += 32) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t a = s[lo], b = s[hi];
-        if ((a < b) == desc) {
-          s[lo] = b;
-          s[hi] = a;
-        }
-      }
-      __syncwarp();
-    }
-}
-
 constexpr int kCandMax = 64;  // keys of the threshold bin resolved by sorting
 
-// Top `want` of n keys by (value desc, id asc), one warp, written sorted
-// (descending composite key) to out[0..P) (P = next power of two >= want,
-// padded with 0).  Value-range binning: with lo/hi the smallest/largest value,
-// bin(v) = floor((v - lo) * 256 / (hi - lo)) is monotone in v, so every key in
-// a bin above the threshold bin is selected and equal values share a bin; the
-// keys of the threshold bin (at most kCandMax) are ordered exactly by their
-// 64-bit keys.  Otherwise (threshold bin too full, non-finite scale) the radix
-// select decides.  hist: 256 words; cand: kCandMax keys.
-template <typename ValFn, typename IdFn>
-__device__ void warp_topk_sorted(ValFn val, IdFn id, int n, int want, int P, float lo, float hi,
-                                 uint64_t* out, uint32_t* hist, uint64_t* cand) {
-  const int lane = threadIdx.x & 31;
-  auto key = [&](int i) { return make_key(val(i), id(i)); };
-  const float range = hi - lo;
-  const float scale = 256.0f / range;
-  bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
-  if (fast) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    auto bin = [&](float v) {
-      const float f = (v - lo) * scale;
-      return f >= 255.0f ? 255u : (f > 0.0f ? static_cast<uint32_t>(f) : 0u);
-    };
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const bool part = i < n;
-      const uint32_t dig = part ? bin(val(i)) : 0u;
-      const uint32_t pm = __ballot_sync(0xffffffffu, part);
-      if (part) {
-        const uint32_t peers = __match_any_sync(pm, dig);
-        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(peers)));
-      }
-    }
-    __syncwarp();
-    uint32_t c[8];
-    uint32_t tot = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      c[j] = hist[255 - 8 * lane - j];
-      tot += c[j];
-    }
-    uint32_t incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const uint32_t excl = incl - tot;
-    int tb = -1;
-    uint32_t above = 0;
-    if (excl < static_cast<uint32_t>(want) && static_cast<uint32_t>(want) <= incl) {
-      uint32_t run = excl;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (tb < 0 && run + c[j] >= static_cast<uint32_t>(want)) {
-          tb = 255 - 8 * lane - j;
-          above = run;
-        }
-        run += c[j];
-      }
-    }
-    const uint32_t who = __ballot_sync(0xffffffffu, tb >= 0);
-    const int src = __ffs(who) - 1;
-    tb = __shfl_sync(0xffffffffu, tb, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    const uint32_t at = hist[tb];
-    __syncwarp();
-    fast = at <= kCandMax;
-    if (fast) {
-      // keys above the threshold bin -> out[0..above), the threshold bin -> cand
-      int nb = 0, nc = 0;
-      for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        uint32_t b = 0;
-        uint64_t kk = 0;
-        if (i < n) {
-          const float v = val(i);
-          b = bin(v);
-          kk = make_key(v, id(i));
-        }
-        const bool up = i < n && static_cast<int>(b) > tb;
-        const bool eq = i < n && static_cast<int>(b) == tb;
-        const uint32_t mu = __ballot_sync(0xffffffffu, up);
-        const uint32_t me = __ballot_sync(0xffffffffu, eq);
-        if (up) out[nb + __popc(mu & lanemask_lt())] = kk;
-        if (eq) cand[nc + __popc(me & lanemask_lt())] = kk;
-        nb += __popc(mu);
-        nc += __popc(me);
-      }
-      // order the threshold bin and take what is still needed
-      int cp = 1;
-      while (cp < nc) cp <<= 1;
-      for (int i = nc + lane; i < cp; i += 32) cand[i] = 0;
-      __syncwarp();
-      warp_sort_desc(cand, cp);
-      const int need = want - nb;
-      for (int i = lane; i < need; i += 32) out[nb + i] = cand[i];
-      __syncwarp();
-    }
-  }
-  if (!fast) warp_select_top(key, n, want, out, hist);
-  for (int i = want + lane; i < P; i += 32) out[i] = 0;
-  __syncwarp();
-  warp_sort_desc(out, P);
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v), m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), m);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// The same selection as warp_topk_sorted for values held in registers: lane l
-// holds values v[j] of indices j*32 + l (indices >= n are absent).  The rare
-// fallback copies the values to `spill` (n floats) and runs the radix select.
-template <int NPL>
-__device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, float lo, float hi,
-                               uint64_t* out, uint32_t* hist, uint64_t* cand, float* spill) {
+// Bitonic sort into descending order of the 32*W keys a warp holds W per lane
+// (element i = w*32 + lane in key[w]); partners closer than 32 are exchanged
+// with shuffles, farther ones sit in the same lane.
+template <int W>
+__device__ __forceinline__ void reg_sort_desc(uint64_t (&key)[W]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 2; s <= 32 * W; s <<= 1) {
+#pragma unroll
+    for (int j = s >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const int wj = w ^ (j >> 5);
+          if (wj > w) {
+            const bool desc = ((w * 32) & s) == 0;
+            const uint64_t a = key[w], b = key[wj];
+            const bool sw = desc ? (a < b) : (a > b);
+            key[w] = sw ? b : a;
+            key[wj] = sw ? a : b;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const uint64_t o = shfl_xor64(key[w], j);
+          const bool desc = ((w * 32 + lane) & s) == 0;
+          const bool lower = (lane & j) == 0;
+          const bool mine_max = key[w] > o;
+          key[w] = (lower == desc) == mine_max ? key[w] : o;
+        }
+      }
+    }
+  }
+}
+
+// out[0 .. 32*W) := the first `m` keys of out sorted descending, then zeros.
+template <int W>
+__device__ __forceinline__ void sort_out(uint64_t* out, int m) {
+  const int lane = threadIdx.x & 31;
+  uint64_t key[W];
+#pragma unroll
+  for (int w = 0; w < W; ++w) key[w] = w * 32 + lane < m ? out[w * 32 + lane] : 0ull;
+  __syncwarp();
+  reg_sort_desc<W>(key);
+#pragma unroll
+  for (int w = 0; w < W; ++w) out[w * 32 + lane] = key[w];
+  __syncwarp();
+}
+
+// Top `want` (<= 32*W) of the n keys make_key(value, id) a warp holds, by
+// (value desc, id asc), written sorted to out[0 .. 32*W) (padded with 0).
+//
+// for_each(f) calls f(value, id) for every element of the calling lane (in
+// any order; elements are split over the lanes), key_at(i) gives the key of
+// element i < n (used only by the fallback, after the whole warp has called
+// prepare()).  Value-range binning with lo/hi
+// the smallest/largest value: bin(v) = floor((v - lo) * 256 / (hi - lo)) is
+// monotone in v, so every key in a bin above the threshold bin is selected
+// and equal values share a bin.  A 256-bin histogram (shared-memory atomics)
+// finds the threshold bin; keys above it are compacted through an atomic
+// counter (about want of n), the threshold bin's keys (at most kCandMax) are
+// sorted in registers for the remainder, and the want keys are sorted in
+// registers.  A threshold bin that is too full, or a non-finite range, falls
+// back to the radix select.  hist: 256 words; tbk: kCandMax keys; cnt: 2 words.
+template <int W, typename ForEach, typename Prepare, typename KeyAt>
+__device__ void warp_topk(ForEach for_each, Prepare prepare, KeyAt key_at, int n, int want,
+                          float lo, float hi, uint64_t* out, uint32_t* hist, uint64_t* tbk,
+                          uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
   const float range = hi - lo;
   const float scale = 256.0f / range;
   bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
   if (fast) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    auto bin = [&](float x) {
-      const float f = (x - lo) * scale;
-      return f >= 255.0f ? 255u : (f > 0.0f ? static_cast<uint32_t>(f) : 0u);
+    auto bin = [&](float v) -> int {
+      const float f = (v - lo) * scale;
+      return f >= 255.0f ? 255 : (f > 0.0f ? static_cast<int>(f) : 0);
     };
 #pragma unroll
-    for (int j = 0; j < NPL; ++j) {
-      const bool part = j * 32 + lane < n;
-      const uint32_t dig = part ? bin(v[j]) : 0u;
-      const uint32_t pm = __ballot_sync(0xffffffffu, part);
-      if (part) {
-        const uint32_t peers = __match_any_sync(pm, dig);
-        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(peers)));
-      }
+    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
+    if (lane == 0) {
+      cnt[0] = 0u;
+      cnt[1] = 0u;
     }
     __syncwarp();
+    for_each([&](float v, uint32_t) { atomicAdd(&hist[bin(v)], 1u); });
+    __syncwarp();
+    // bins in descending order: lane l owns bins 255-8l ... 248-8l
     uint32_t c[8];
     uint32_t tot = 0;
 #pragma unroll
@@ -303,7 +247,7 @@ __device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, fl
     }
     const uint32_t excl = incl - tot;
     int tb = -1;
-    uint32_t above = 0;
+    uint32_t above = 0, at = 0;
     if (excl < static_cast<uint32_t>(want) && static_cast<uint32_t>(want) <= incl) {
       uint32_t run = excl;
 #pragma unroll
@@ -311,6 +255,7 @@ __device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, fl
         if (tb < 0 && run + c[j] >= static_cast<uint32_t>(want)) {
           tb = 255 - 8 * lane - j;
           above = run;
+          at = c[j];
         }
         run += c[j];
       }
@@ -319,62 +264,49 @@ __device__ void warp_topk_regs(const float (&v)[NPL], int n, int want, int P, fl
     const int src = __ffs(who) - 1;
     tb = __shfl_sync(0xffffffffu, tb, src);
     above = __shfl_sync(0xffffffffu, above, src);
-    const uint32_t at = hist[tb];
-    __syncwarp();
-    fast = at <= kCandMax;
+    at = __shfl_sync(0xffffffffu, at, src);
+    fast = at <= static_cast<uint32_t>(kCandMax);
     if (fast) {
-      int nb = 0, nc = 0;
-#pragma unroll
-      for (int j = 0; j < NPL; ++j) {
-        const int i = j * 32 + lane;
-        const bool valid = i < n;
-        const uint32_t b = valid ? bin(v[j]) : 0u;
-        const bool up = valid && static_cast<int>(b) > tb;
-        const bool eq = valid && static_cast<int>(b) == tb;
-        const uint64_t kk = make_key(v[j], static_cast<uint32_t>(i));
-        const uint32_t mu = __ballot_sync(0xffffffffu, up);
-        const uint32_t me = __ballot_sync(0xffffffffu, eq);
-        if (up) out[nb + __popc(mu & lanemask_lt())] = kk;
-        if (eq) cand[nc + __popc(me & lanemask_lt())] = kk;
-        nb += __popc(mu);
-        nc += __popc(me);
-      }
-      int cp = 1;
-      while (cp < nc) cp <<= 1;
-      for (int i = nc + lane; i < cp; i += 32) cand[i] = 0;
+      // keys above the threshold bin -> out (unordered), its own keys -> tbk
+      for_each([&](float v, uint32_t id) {
+        const int b = bin(v);
+        if (b > tb) out[atomicAdd(&cnt[0], 1u)] = make_key(v, id);
+        else if (b == tb) tbk[atomicAdd(&cnt[1], 1u)] = make_key(v, id);
+      });
       __syncwarp();
-      warp_sort_desc(cand, cp);
-      const int need = want - nb;
-      for (int i = lane; i < need; i += 32) out[nb + i] = cand[i];
+      const int need = want - static_cast<int>(above);
+      if (at <= 32u) {
+        uint64_t key[1];
+        key[0] = lane < static_cast<int>(at) ? tbk[lane] : 0ull;
+        reg_sort_desc<1>(key);
+        if (lane < need) out[above + lane] = key[0];
+      } else {
+        uint64_t key[2];
+        key[0] = tbk[lane];
+        key[1] = 32 + lane < static_cast<int>(at) ? tbk[32 + lane] : 0ull;
+        reg_sort_desc<2>(key);
+        if (lane < need) out[above + lane] = key[0];
+        if (32 + lane < need) out[above + 32 + lane] = key[1];
+      }
       __syncwarp();
     }
   }
   if (!fast) {
-#pragma unroll
-    for (int j = 0; j < NPL; ++j)
-      if (j * 32 + lane < n) spill[j * 32 + lane] = v[j];
-    __syncwarp();
-    warp_select_top([&](int i) { return make_key(spill[i], static_cast<uint32_t>(i)); }, n, want,
-                    out, hist);
+    prepare();
+    warp_select_top(key_at, n, want, out, hist);
   }
-  for (int i = want + lane; i < P; i += 32) out[i] = 0;
-  __syncwarp();
-  warp_sort_desc(out, P);
+  sort_out<W>(out, want < n ? want : n);
 }
 
 struct SelPlan {
-  int nr_pad, nc_pad, kp, Kp, cand;  // sizes (elements)
+  int cand;                           // (a, b) candidate pairs of the k x k merge
   int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc,
-      off_roff;
+      off_cnt;
   int pair_bytes;
+  int table_bytes;                    // per CTA: the (a, b) pair table
 };
 
-// bytes per token pair, each array 16-byte aligned
-SelPlan make_plan(const Dims& D) {
-  SelPlan p{};
-  auto al = [](int v) { return (v + 15) & ~15; };
-  p.kp = static_cast<int>(next_pow2(D.k));
-  p.Kp = static_cast<int>(next_pow2(D.K));
+int merge_candidates(const Dims& D) {
   int cand = 0;
   for (int64_t a = 0; a < D.k; ++a) {
     int64_t nb = D.K / (a + 1);
@@ -382,25 +314,35 @@ SelPlan make_plan(const Dims& D) {
     if (nb <= 0) break;
     cand += static_cast<int>(nb);
   }
-  p.cand = cand;
+  return cand;
+}
+
+// bytes per token pair, each array 16-byte aligned
+SelPlan make_plan(const Dims& D, int W, int WK) {
+  SelPlan p{};
+  auto al = [](int v) { return (v + 15) & ~15; };
+  p.cand = merge_candidates(D);
   int off = 0;
   p.off_vr = off; off = al(off + 4 * static_cast<int>(D.Nr));
   p.off_vc = off; off = al(off + 4 * static_cast<int>(D.Nc));
   p.off_hr = off; off = al(off + 4 * 256);
   p.off_hc = off; off = al(off + 4 * 256);
-  p.off_sr = off; off = al(off + 8 * p.kp);
-  p.off_sc = off; off = al(off + 8 * p.kp);
-  p.off_cand = off; off = al(off + 8 * cand);
-  p.off_out = off; off = al(off + 8 * p.Kp);
+  p.off_sr = off; off = al(off + 8 * 32 * W);
+  p.off_sc = off; off = al(off + 8 * 32 * W);
+  p.off_cand = off; off = al(off + 8 * p.cand);
+  p.off_out = off; off = al(off + 8 * 32 * WK);
   p.off_misc = off; off = al(off + 16);
   p.off_tr = off; off = al(off + 8 * kCandMax);
   p.off_tc = off; off = al(off + 8 * kCandMax);
-  p.off_roff = off; off = al(off + 4 * static_cast<int>(D.k));
+  p.off_cnt = off; off = al(off + 16);
   p.pair_bytes = off;
+  p.table_bytes = al(4 * p.cand);
   return p;
 }
 
-template <int NPL>
+// NPL: logits per lane and axis (n <= 32*NPL); W, WK: sorted lengths 32*W >=
+// k and 32*WK >= K.
+template <int NPL, int W, int WK>
 __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int64_t L, int Nr,
                                                 int Nc, int k, int K,
                                                 const float* __restrict__ br,
@@ -413,9 +355,35 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   const int pair = threadIdx.x >> 6;
   const int role = (threadIdx.x >> 5) & 1;  // 0: rows, 1: columns
   const int pairs = blockDim.x >> 6;
+
+  // (a, b) pairs with (a+1)(b+1) <= K, row by row: pair c of row a sits at
+  // roff(a) + b, roff the prefix sum of min(k, K/(a+1)); built once per CTA
+  uint32_t* cab = reinterpret_cast<uint32_t*>(smem);
+  if (threadIdx.x < 32) {
+    int base = 0;
+    for (int a0 = 0; a0 < k; a0 += 32) {
+      const int a = a0 + lane;
+      int nb = 0;
+      if (a < k) {
+        nb = K / (a + 1);
+        if (nb > k) nb = k;
+      }
+      int incl = nb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t2;
+      }
+      const int off = base + incl - nb;
+      for (int b = 0; b < nb; ++b) cab[off + b] = (static_cast<uint32_t>(a) << 16) | b;
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  __syncthreads();
+
   const int64_t t = static_cast<int64_t>(blockIdx.x) * pairs + pair;
   if (t >= L) return;  // both warps of the pair leave together
-  uint8_t* base = smem + static_cast<size_t>(pair) * P.pair_bytes;
+  uint8_t* base = smem + P.table_bytes + static_cast<size_t>(pair) * P.pair_bytes;
   float* misc = reinterpret_cast<float*>(base + P.off_misc);
 
   // ---- per-axis: log-sum-exp and top-k ----
@@ -427,6 +395,7 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + (role ? P.off_hc : P.off_hr));
     uint64_t* sel = reinterpret_cast<uint64_t*>(base + (role ? P.off_sc : P.off_sr));
     uint64_t* tbin = reinterpret_cast<uint64_t*>(base + (role ? P.off_tc : P.off_tr));
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt) + 2 * role;
     float v[NPL];
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
@@ -450,7 +419,20 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
       if (j * 32 + lane < n) s += expf(v[j] - mx);
     s = warp_sum(s);
     if (lane == 0) misc[role] = mx + logf(s);
-    warp_topk_regs<NPL>(v, n, k, P.kp, mn, mx, sel, hist, tbin, vals);
+    warp_topk<W>(
+        [&](auto f) {
+#pragma unroll
+          for (int j = 0; j < NPL; ++j)
+            if (j * 32 + lane < n) f(v[j], static_cast<uint32_t>(j * 32 + lane));
+        },
+        [&]() {  // the radix fallback reads values by index
+#pragma unroll
+          for (int j = 0; j < NPL; ++j)
+            if (j * 32 + lane < n) vals[j * 32 + lane] = v[j];
+          __syncwarp();
+        },
+        [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
+        hist, tbin, cnt);
   }
   asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
   if (role != 0) return;
@@ -462,37 +444,12 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   uint64_t* out = reinterpret_cast<uint64_t*>(base + P.off_out);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + P.off_hr);
   uint64_t* tbin = reinterpret_cast<uint64_t*>(base + P.off_tr);
-  // candidate (a, b) pairs with (a+1)(b+1) <= K, one per lane: row a's pairs
-  // start at roff[a] (prefix of min(k, K/(a+1)) over the rows)
-  int32_t* roff = reinterpret_cast<int32_t*>(base + P.off_roff);
-  int na = 0;
-  for (int a0 = 0; a0 < k; a0 += 32) {
-    const int a = a0 + lane;
-    int nb = 0;
-    if (a < k) {
-      nb = K / (a + 1);
-      if (nb > k) nb = k;
-    }
-    int incl = nb;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t2;
-    }
-    if (a < k) roff[a] = na + incl - nb;
-    na += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  __syncwarp();
-  const int nc = na;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt);
+  const int nc = P.cand;
   float cmx = -INFINITY, cmn = INFINITY;
   for (int c = lane; c < nc; c += 32) {
-    int lo = 0, hi = k - 1;  // last row a with roff[a] <= c
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (roff[mid] <= c) lo = mid; else hi = mid - 1;
-    }
-    const int a = lo, b = c - roff[a];
-    const uint64_t ra = sr[a], cb = sc[b];
+    const uint32_t ab = cab[c];
+    const uint64_t ra = sr[ab >> 16], cb = sc[ab & 0xffffu];
     const float sv = key_val(ra) + key_val(cb);
     const uint32_t e = key_id(ra) * static_cast<uint32_t>(Nc) + key_id(cb);
     cand[c] = make_key(sv, e);
@@ -502,8 +459,14 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   cmx = warp_max(cmx);
   cmn = -warp_max(-cmn);
   __syncwarp();
-  warp_topk_sorted([&](int i) { return key_val(cand[i]); }, [&](int i) { return key_id(cand[i]); },
-                   nc, K, P.Kp, cmn, cmx, out, hist, tbin);
+  warp_topk<WK>(
+      [&](auto f) {
+        for (int c = lane; c < nc; c += 32) {
+          const uint64_t kk = cand[c];
+          f(key_val(kk), key_id(kk));
+        }
+      },
+      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbin, cnt);
 
   // ---- gate = softmax of the K selected joint scores ----
   const float s0 = key_val(out[0]);
@@ -520,25 +483,43 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   }
 }
 
-}  // namespace
+int sort_width(int64_t m) {
+  int w = 1;
+  while (32 * w < m) w <<= 1;
+  return w;
+}
 
-template <int NPL>
-cudaError_t launch_select_npl(const Dims& D, const float* Z, const float* br, const float* bc,
-                              int32_t* idx, float* gate, float* score, cudaStream_t s) {
-  SelPlan P = make_plan(D);
+template <int NPL, int W, int WK>
+cudaError_t launch_select_t(const Dims& D, const float* Z, const float* br, const float* bc,
+                            int32_t* idx, float* gate, float* score, cudaStream_t s) {
+  SelPlan P = make_plan(D, W, WK);
   int pairs = 4;
-  while (pairs > 1 && pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
-  const size_t smem = static_cast<size_t>(pairs) * P.pair_bytes;
+  while (pairs > 1 && P.table_bytes + pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
+  const size_t smem = static_cast<size_t>(P.table_bytes) + static_cast<size_t>(pairs) * P.pair_bytes;
   cudaError_t err =
-      cudaFuncSetAttribute(k_select<NPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(k_select<NPL, W, WK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int64_t grid = (D.L + pairs - 1) / pairs;
-  k_select<NPL><<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
+  k_select<NPL, W, WK><<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
       Z, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
       static_cast<int>(D.K), br, bc, idx, gate, score, P);
   return cudaGetLastError();
 }
+
+template <int NPL>
+cudaError_t launch_select_npl(const Dims& D, const float* Z, const float* br, const float* bc,
+                              int32_t* idx, float* gate, float* score, cudaStream_t s) {
+  // one sort width for both lists (32*W >= max(k, K))
+  switch (sort_width(D.k > D.K ? D.k : D.K)) {
+    case 1: return launch_select_t<NPL, 1, 1>(D, Z, br, bc, idx, gate, score, s);
+    case 2: return launch_select_t<NPL, 2, 2>(D, Z, br, bc, idx, gate, score, s);
+    case 4: return launch_select_t<NPL, 4, 4>(D, Z, br, bc, idx, gate, score, s);
+    default: return launch_select_t<NPL, 8, 8>(D, Z, br, bc, idx, gate, score, s);
+  }
+}
+
+}  // namespace
 
 cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
                           const float* bc, int32_t* idx, float* gate, float* score,
