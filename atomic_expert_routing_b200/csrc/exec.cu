@@ -208,6 +208,15 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+__device__ __forceinline__ void cp_async16_plain(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ uint4 ld_v4_hint(const void* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "l"(pol));
+  return r;
+}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "l"(pol)
@@ -364,86 +373,90 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
 
 constexpr int kActWarps = 8;
 
-template <typename T, int NV, int R>
-__global__ void __launch_bounds__(kActWarps * 32, 1)
-    k_act(const T* __restrict__ x, const T* __restrict__ W, const int32_t* __restrict__ task_token,
-          const int32_t* __restrict__ task_expert, const float* __restrict__ task_gate,
-          int64_t M, int64_t L, int64_t N, int d, int S, int64_t nslices, float* __restrict__ cbuf,
-          int32_t* status) {
-  constexpr int SLOT = NV * 32;  // uint4 per ring slot: one W row
+// c[dst[a]] = g[a] * SiLU(H[hidx[a]] . F[fidx[a]]) over a task list in which
+// tasks that share a held row H[h] are adjacent (a run).  Warp w takes slices
+// of S consecutive tasks; the run's held row sits in registers (the next
+// run's row is fetched while the current one is used; evict-first when
+// HOLD_ONCE), and every task's row of F streams through a ring of R
+// shared-memory slots per warp (cp.async, R - 1 rows in flight).  dst ==
+// nullptr writes c[a].  Indices are range-checked (OMNI_DEV_BAD_INDEX; the
+// task gets c = 0).
+template <typename T, int NV, int R, bool HOLD_ONCE>
+__global__ void __launch_bounds__(kActWarps * 32, 2)
+    k_act(const T* __restrict__ H, const int32_t* __restrict__ hidx, int64_t nh,
+          const T* __restrict__ F, const int32_t* __restrict__ fidx, int64_t nf,
+          const float* __restrict__ task_gate, const int32_t* __restrict__ dst, int64_t M, int d,
+          int S, int64_t nslices, float* __restrict__ cbuf, int32_t* status) {
+  constexpr int SLOT = NV * 32;  // uint4 per ring slot: one row of F
   extern __shared__ __align__(16) uint4 ring[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint4* wring = ring + static_cast<size_t>(warp) * R * SLOT;
-  const uint32_t wring_s = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
-  const uint64_t pol_stream = policy_evict_first();
+  uint4* fring = ring + static_cast<size_t>(warp) * R * SLOT;
+  const uint32_t fring_s = static_cast<uint32_t>(__cvta_generic_to_shared(fring));
+  const uint64_t pol_once = policy_evict_first();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kActWarps;
   for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kActWarps + warp; sl < nslices; sl += nw) {
     const int64_t a0 = sl * S;
     const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
-    int64_t my_t = -1, my_e = -1;
+    int64_t my_h = -1, my_f = -1, my_d = -1;
     float my_g = 0.0f, my_c = 0.0f;
     if (lane < n) {
-      my_t = task_token[a0 + lane];
-      my_e = task_expert[a0 + lane];
+      my_h = hidx[a0 + lane];
+      my_f = fidx[a0 + lane];
       my_g = task_gate[a0 + lane];
-      if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
+      my_d = dst != nullptr ? dst[a0 + lane] : a0 + lane;
+      if (my_h < 0 || my_h >= nh || my_f < 0 || my_f >= nf || my_d < 0 || my_d >= M) {
         raise_status(status, OMNI_DEV_BAD_INDEX);
-        my_e = -1;
-        my_t = -1;
+        my_h = -1;
+        my_f = -1;
+        if (my_d < 0 || my_d >= M) my_d = -1;
       }
     }
-    const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
-    const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
+    const int64_t prev_h = __shfl_up_sync(0xffffffffu, my_h, 1);
+    const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_h != my_h));
     auto issue = [&](int j) {
       if (j < n) {
-        const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
-        if (e >= 0) {
-          const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
-          const uint32_t base = wring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
+        const int64_t f = __shfl_sync(0xffffffffu, my_f, j);
+        if (f >= 0) {
+          const uint4* fr = reinterpret_cast<const uint4*>(F + f * d);
+          const uint32_t base = fring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
 #pragma unroll
           for (int v = 0; v < NV; ++v)
-            cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, wr + v * 32 + lane, pol_stream);
+            cp_async16_plain(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane);
         }
       }
       cp_async_commit();
     };
 #pragma unroll
     for (int j = 0; j < R - 1; ++j) issue(j);
-    uint4 xc[NV], xn[NV];
-    {
-      const int64_t t0 = __shfl_sync(0xffffffffu, my_t, 0);
-      const uint4* xr = reinterpret_cast<const uint4*>(x + (t0 < 0 ? 0 : t0) * d);
+    uint4 hc[NV], hn[NV];
+    auto load_held = [&](int64_t h) {
+      const uint4* hr = reinterpret_cast<const uint4*>(H + (h < 0 ? 0 : h) * d);
 #pragma unroll
-      for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
-    }
+      for (int v = 0; v < NV; ++v) hn[v] = HOLD_ONCE ? ld_v4_hint(hr + v * 32 + lane, pol_once) : hr[v * 32 + lane];
+    };
+    load_held(__shfl_sync(0xffffffffu, my_h, 0));
     for (int j = 0; j < n; ++j) {
       issue(j + R - 1);
       if ((starts >> j) & 1u) {
 #pragma unroll
-        for (int v = 0; v < NV; ++v) xc[v] = xn[v];
+        for (int v = 0; v < NV; ++v) hc[v] = hn[v];
         const uint32_t later = starts & ~((2u << j) - 1u);
-        if (later) {
-          const int jn = __ffs(later) - 1;
-          const int64_t tn = __shfl_sync(0xffffffffu, my_t, jn);
-          const uint4* xr = reinterpret_cast<const uint4*>(x + (tn < 0 ? 0 : tn) * d);
-#pragma unroll
-          for (int v = 0; v < NV; ++v) xn[v] = xr[v * 32 + lane];
-        }
+        if (later) load_held(__shfl_sync(0xffffffffu, my_h, __ffs(later) - 1));
       }
       cp_async_wait<R - 1>();
-      const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
+      const int64_t h = __shfl_sync(0xffffffffu, my_h, j);
       const float gj = __shfl_sync(0xffffffffu, my_g, j);
-      if (e >= 0) {  // warp-uniform
-        const uint4* slot = wring + (j % R) * SLOT;
+      if (h >= 0) {  // warp-uniform
+        const uint4* slot = fring + (j % R) * SLOT;
         float sdot = 0.0f;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
+        for (int v = 0; v < NV; ++v) sdot += dot_vec(hc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
         sdot = warp_sum(sdot);
         if (lane == j) my_c = gj * silu(sdot);
       }
     }
     cp_async_wait<0>();
-    if (lane < n) cbuf[a0 + lane] = my_c;
+    if (lane < n && my_d >= 0) cbuf[my_d] = my_c;
   }
 }
 
@@ -459,26 +472,40 @@ __global__ void __launch_bounds__(kActWarps * 32, 1)
 // exactly once.
 constexpr int kWinTasks = 7168;
 
-// Window w takes the groups whose first task lies in [w*T, (w+1)*T).  Windows
-// larger than the CTA sort (a single very large group) and the whole batch
-// when the group count on the device is out of range are copied in schedule
+// Window w takes the groups whose first task lies in [w*T, (w+1)*T).  Two
+// orders of its tasks are written: by token (wt/we/wg, for the accumulation
+// sweeps) and by expert (xt/xe/xg, for the activations, so that the tasks of
+// one expert are adjacent and its W row leaves HBM once), with xdst the
+// token-order position of each expert-order task.  Both sorts are stable
+// (a window arrives in (group, token, expert) order).  Windows larger than
+// the CTA sort (a single very large group) and the whole batch when the
+// group count on the device is out of range are passed through in schedule
 // order (the latter with OMNI_DEV_BAD_INDEX raised).
+struct WinOut {
+  int32_t *wt, *we;
+  float* wg;
+  int32_t *xt, *xe;
+  float* xg;
+  int32_t* xdst;
+};
+
 __global__ void __launch_bounds__(kBlockSortThreads)
     k_wsort(const int32_t* __restrict__ tt, const int32_t* __restrict__ te,
             const float* __restrict__ tg, const int32_t* __restrict__ group_off,
             const int32_t* __restrict__ counts, int64_t M, int64_t gmax, int T, int passes,
-            int32_t* __restrict__ wt, int32_t* __restrict__ we, float* __restrict__ wg,
-            int32_t* status) {
+            WinOut o, int32_t* status) {
   extern __shared__ __align__(16) uint8_t wsm[];
   uint32_t* kA = reinterpret_cast<uint32_t*>(wsm);
   uint32_t* kB = kA + kBlockSortMax;
   uint16_t* vA = reinterpret_cast<uint16_t*>(kB + kBlockSortMax);
   uint16_t* vB = vA + kBlockSortMax;
-  uint32_t* wcount = reinterpret_cast<uint32_t*>(vB + kBlockSortMax);
+  uint16_t* inv = vB + kBlockSortMax;  // token-order position of each task
+  uint32_t* wcount = reinterpret_cast<uint32_t*>(inv + kBlockSortMax);
   __shared__ uint32_t dbase[256];
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ int64_t rng[2];
+  __shared__ int emin, emax;
   const int64_t lo = static_cast<int64_t>(blockIdx.x) * T;
   const int64_t hi = M - lo < T ? M : lo + T;
   if (threadIdx.x == 0) {
@@ -508,6 +535,8 @@ __global__ void __launch_bounds__(kBlockSortThreads)
     }
     rng[0] = a0;
     rng[1] = a1;
+    emin = INT_MAX;
+    emax = INT_MIN;
   }
   __syncthreads();
   const int64_t a0 = rng[0];
@@ -515,18 +544,27 @@ __global__ void __launch_bounds__(kBlockSortThreads)
   if (n <= 0) return;
   if (n > kBlockSortMax) {
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-      wt[a0 + i] = tt[a0 + i];
-      we[a0 + i] = te[a0 + i];
-      wg[a0 + i] = tg[a0 + i];
+      const int32_t t = tt[a0 + i], e = te[a0 + i];
+      const float g = tg[a0 + i];
+      o.wt[a0 + i] = t; o.we[a0 + i] = e; o.wg[a0 + i] = g;
+      o.xt[a0 + i] = t; o.xe[a0 + i] = e; o.xg[a0 + i] = g;
+      o.xdst[a0 + i] = static_cast<int32_t>(a0 + i);
     }
     return;
   }
   const int nn = static_cast<int>(n);
+  int lmin = INT_MAX, lmax = INT_MIN;
   for (int i = threadIdx.x; i < nn; i += blockDim.x) {
     kA[i] = static_cast<uint32_t>(tt[a0 + i]);
     vA[i] = static_cast<uint16_t>(i);
+    const int e = te[a0 + i];
+    lmin = e < lmin ? e : lmin;
+    lmax = e > lmax ? e : lmax;
   }
+  atomicMin(&emin, lmin);
+  atomicMax(&emax, lmax);
   __syncthreads();
+  // by token
   uint32_t* kin = kA; uint32_t* kout = kB;
   uint16_t* vin = vA; uint16_t* vout = vB;
   for (int p = 0; p < passes; ++p) {
@@ -536,9 +574,34 @@ __global__ void __launch_bounds__(kBlockSortThreads)
   }
   for (int i = threadIdx.x; i < nn; i += blockDim.x) {
     const int src = vin[i];
-    wt[a0 + i] = tt[a0 + src];
-    we[a0 + i] = te[a0 + src];
-    wg[a0 + i] = tg[a0 + src];
+    inv[src] = static_cast<uint16_t>(i);
+    o.wt[a0 + i] = tt[a0 + src];
+    o.we[a0 + i] = te[a0 + src];
+    o.wg[a0 + i] = tg[a0 + src];
+  }
+  __syncthreads();  // the key/value buffers are reused below
+  // by expert (ids relative to the window's smallest)
+  const int64_t span = static_cast<int64_t>(emax) - emin;
+  int ebits = 0;
+  while (ebits < 32 && (int64_t(1) << ebits) <= span) ++ebits;
+  const int epasses = (ebits + 7) / 8;
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    kA[i] = static_cast<uint32_t>(te[a0 + i] - emin);
+    vA[i] = static_cast<uint16_t>(i);
+  }
+  __syncthreads();
+  kin = kA; kout = kB; vin = vA; vout = vB;
+  for (int p = 0; p < epasses; ++p) {
+    block_radix_pass(kin, vin, kout, vout, nn, 8 * p, wcount, dbase, warp_tot, &total);
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const int src = vin[i];
+    o.xt[a0 + i] = tt[a0 + src];
+    o.xe[a0 + i] = te[a0 + src];
+    o.xg[a0 + i] = tg[a0 + src];
+    o.xdst[a0 + i] = static_cast<int32_t>(a0 + inv[src]);
   }
 }
 
@@ -673,16 +736,49 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src, T* __restrict__ dst,
-                                              int64_t n) {
+// fp32 accumulator -> bf16 output (round to nearest even), 8 values per thread.
+__global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src,
+                                              __nv_bfloat16* __restrict__ dst, int64_t n) {
   const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (i >= n) return;
   const float4 a = *reinterpret_cast<const float4*>(src + i);
   const float4 b = *reinterpret_cast<const float4*>(src + i + 4);
   const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int u = 0; u < 8; ++u) dst[i + u] = from_float<T>(f[u]);
+  *reinterpret_cast<uint4*>(dst + i) = pack_vec(f, static_cast<__nv_bfloat16*>(nullptr));
+}
+
+// Bookkeeping between accumulation sweeps, on column slices of the fp32
+// accumulator (L rows of d floats), 8 columns per thread:
+//  - cast0 >= 0: columns [cast0, cast0 + cols) are final -- round them to
+//    bf16 into y and, the accumulator being scratch, drop its 128-byte lines
+//    from L2 without writing them back (discard.global.L2);
+//  - zero0 >= 0: zero columns [zero0, zero0 + cols) for the next sweep (the
+//    stores leave the slice in L2 for it).
+__global__ void __launch_bounds__(256)
+    k_slice_finish(float* __restrict__ acc, __nv_bfloat16* __restrict__ y, int64_t L, int d,
+                   int cast0, int zero0, int cols) {
+  const int per_row = cols / 8;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = i / per_row;
+  const int c8 = static_cast<int>(i % per_row) * 8;
+  const bool active = row < L;
+  if (cast0 >= 0) {
+    float* src = acc + row * d + cast0 + c8;
+    if (active) {
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      *reinterpret_cast<uint4*>(y + row * d + cast0 + c8) =
+          pack_vec(f, static_cast<__nv_bfloat16*>(nullptr));
+    }
+    __syncwarp();  // the four threads of a line have read it
+    if (active && (c8 & 31) == 0) asm volatile("discard.global.L2 [%0], 128;" ::"l"(src) : "memory");
+  }
+  if (zero0 >= 0 && active) {
+    float4* dst = reinterpret_cast<float4*>(acc + row * d + zero0 + c8);
+    dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 constexpr int kTokThreads = 128;
@@ -768,9 +864,7 @@ int expert_sweeps(const Dims& D) {
 // c and the window-ordered copy of the task list.
 struct SweepWs {
   float* cbuf;
-  int32_t* wt;
-  int32_t* we;
-  float* wg;
+  WinOut win;
 };
 
 size_t acc_bytes(const Dims& D) {
@@ -783,9 +877,13 @@ SweepWs carve_sweeps(const Dims& D, void* ws, size_t* bytes) {
   SweepWs w;
   const size_t M = static_cast<size_t>(D.M());
   w.cbuf = c.take<float>(M);
-  w.wt = c.take<int32_t>(M);
-  w.we = c.take<int32_t>(M);
-  w.wg = c.take<float>(M);
+  w.win.wt = c.take<int32_t>(M);
+  w.win.we = c.take<int32_t>(M);
+  w.win.wg = c.take<float>(M);
+  w.win.xt = c.take<int32_t>(M);
+  w.win.xe = c.take<int32_t>(M);
+  w.win.xg = c.take<float>(M);
+  w.win.xdst = c.take<int32_t>(M);
   if (bytes) *bytes = c.off;
   return w;
 }
@@ -866,7 +964,7 @@ int sm_count() {
 cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, const float* tg,
                          const int32_t* group_off, const int32_t* counts, const SweepWs& w,
                          int32_t* status, cudaStream_t s) {
-  constexpr size_t smem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 2 * 2) +
+  constexpr size_t smem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 3 * 2) +
                           static_cast<size_t>(kBlockSortWarps) * 256 * 4;
   cudaError_t err = cudaFuncSetAttribute(k_wsort, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -880,8 +978,7 @@ cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, co
   while ((int64_t(1) << bits) < D.L) ++bits;
   const int passes = (bits + 7) / 8;
   k_wsort<<<static_cast<unsigned>(nwin), kBlockSortThreads, smem, s>>>(
-      tt, te, tg, group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.wt, w.we, w.wg,
-      status);
+      tt, te, tg, group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.win, status);
   return cudaGetLastError();
 }
 
@@ -899,31 +996,44 @@ cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   if (blocks > cap) blocks = cap;
   k_acc<T, NB, D><<<static_cast<unsigned>(blocks), kAccWarps * 32, 0, s>>>(
-      static_cast<const T*>(V), w.wt, w.we, w.cbuf, M, D_.L, D_.N(), static_cast<int>(D_.d), col0,
-      nslices, acc);
+      static_cast<const T*>(V), w.win.wt, w.win.we, w.cbuf, M, D_.L, D_.N(),
+      static_cast<int>(D_.d), col0, nslices, acc);
   return cudaGetLastError();
 }
 
+cudaError_t launch_finish(const Dims& D, float* acc, __nv_bfloat16* y, int cast0, int zero0,
+                          int cols, cudaStream_t s) {
+  if (cast0 < 0 && zero0 < 0) return cudaSuccess;
+  const int64_t threads = D.L * (cols / 8);
+  k_slice_finish<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
+      acc, y, D.L, static_cast<int>(D.d), cast0, zero0, cols);
+  return cudaGetLastError();
+}
+
+// ycast: the bf16 output (nullptr for fp32, whose accumulator is y itself).
 template <typename T, int NV, int NVQ>
 cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const void* V,
                       const int32_t* tt, const int32_t* te, const float* tg,
                       const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                      float* acc, int32_t* status, cudaStream_t s) {
+                      float* acc, __nv_bfloat16* ycast, int32_t* status, cudaStream_t s) {
   cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, status, s);
   if (err != cudaSuccess) return err;
-  constexpr int R = 6;
+  // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
+  constexpr int R = 3;
   constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
-  err = cudaFuncSetAttribute(k_act<T, NV, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  err = cudaFuncSetAttribute(k_act<T, NV, R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int64_t M = D.M();
   const int S = 32;
   const int64_t nslices = (M + S - 1) / S;
   int64_t blocks = (nslices + kActWarps - 1) / kActWarps;
-  if (blocks > sm_count()) blocks = sm_count();
-  k_act<T, NV, R><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
-      static_cast<const T*>(x), static_cast<const T*>(W), w.wt, w.we, w.wg, M, D.L, D.N(),
-      static_cast<int>(D.d), S, nslices, w.cbuf, status);
+  if (blocks > 2 * sm_count()) blocks = 2 * sm_count();
+  // tasks by expert: x[t] held per run of one token, the W rows through the
+  // ring (an expert's repeated row comes from L2 right after its first read)
+  k_act<T, NV, R, false><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
+      static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W), w.win.xe, D.N(),
+      w.win.xg, w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int cols = static_cast<int>(D.d / Q);
@@ -931,18 +1041,22 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   // of loads in flight per lane)
   constexpr int NB = NVQ * 32 * kEpv<T> / 128;
   constexpr int PD = 8 / NVQ;
-  for (int q = 0; q < Q; ++q) {
+  // each sweep's slice is zeroed just before it and cast just after it
+  err = launch_finish(D, acc, ycast, -1, 0, cols, s);
+  for (int q = 0; q < Q && err == cudaSuccess; ++q) {
     err = launch_acc<T, NB, PD>(D, q * cols, V, w, acc, s);
-    if (err != cudaSuccess) return err;
+    if (err == cudaSuccess)
+      err = launch_finish(D, acc, ycast, ycast ? q * cols : -1, q + 1 < Q ? (q + 1) * cols : -1,
+                          cols, s);
   }
-  return cudaSuccess;
+  return err;
 }
 
 template <typename T>
 cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, const void* V,
                           const int32_t* tt, const int32_t* te, const float* tg,
                           const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                          float* acc, int32_t* status, cudaStream_t s) {
+                          float* acc, __nv_bfloat16* ycast, int32_t* status, cudaStream_t s) {
   constexpr int row = 32 * kEpv<T>;
   const int64_t nv = D.d / row;             // vectors per lane for a whole row
   const int64_t nvq = (D.d / Q) / row;      // ... for one slice
@@ -950,7 +1064,7 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
 #define OMNI_SWEEP(NV_, NVQ_)                                                               \
   if (nv == NV_ && nvq == NVQ_)                                                             \
     return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, group_off, counts, w, acc,    \
-                                   status, s);
+                                   ycast, status, s);
   OMNI_SWEEP(8, 4) OMNI_SWEEP(8, 2) OMNI_SWEEP(8, 1) OMNI_SWEEP(4, 2) OMNI_SWEEP(4, 1)
   OMNI_SWEEP(2, 1)
 #undef OMNI_SWEEP
@@ -964,25 +1078,25 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
   float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
+  int32_t* status = const_cast<int32_t*>(counts) + 2;
+  const int Q = expert_sweeps(D);
+  if (Q > 1) {  // the sweeps zero, accumulate and cast slice by slice
+    const SweepWs w = carve_sweeps(D, ws, nullptr);
+    __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
+    return f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate,
+                                      group_off, counts, w, acc, ycast, status, s)
+               : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
+                                              group_off, counts, w, acc, ycast, status, s);
+  }
   const size_t ybytes = static_cast<size_t>(D.L) * D.d * sizeof(float);
   cudaError_t err = cudaMemsetAsync(acc, 0, ybytes, s);
   if (err != cudaSuccess) return err;
-  int32_t* status = const_cast<int32_t*>(counts) + 2;
-  const int Q = expert_sweeps(D);
-  if (Q > 1) {
-    const SweepWs w = carve_sweeps(D, ws, nullptr);
-    err = f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate, group_off,
-                                     counts, w, acc, status, s)
-              : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
-                                             group_off, counts, w, acc, status, s);
-  } else {
-    err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
-              : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
-                                               status, s);
-  }
+  err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
+            : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
+                                             status, s);
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;
-  k_cast<__nv_bfloat16><<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(
+  k_cast<<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(
       acc, static_cast<__nv_bfloat16*>(y), n);
   return cudaGetLastError();
 }

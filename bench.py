@@ -62,19 +62,26 @@ def expert_stage_bytes(cfg, n_active):
     return 2 * cfg.d * n_active * e + 2 * cfg.L * cfg.d * e
 
 
-def kernel_launches(cfg):
-    """Kernels of this library launched by one omni_moe_forward (memsets excluded)."""
-    ucap = min(cfg.N, cfg.L * cfg.K)
-    gmax = (ucap + cfg.B - 1) // cfg.B
-    bits = max(0, int(np.ceil(np.log2(gmax)))) if gmax > 1 else 0
-    passes = (bits + 7) // 8
-    route = 2
-    if cfg.L * cfg.K <= 8192:
-        sched = 1  # single-CTA schedule of small batches
-    else:
-        sched = 1 + 3 + 5 * passes + 1  # prep, flag scan, radix passes (hist, 3 scans, scatter), emit
-    expert = 1 + (1 if cfg.dtype == WL.BF16 else 0)
-    return route + sched + expert
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (the forward's own launches; memset
+    nodes excluded), or None when the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kernels = 0
+        for node in nodes[:n]:
+            err, kind = rt.cudaGraphNodeGetType(node)
+            if err == rt.cudaError_t.cudaSuccess and kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kernels += 1
+        return kernels
+    except Exception:  # noqa: BLE001 -- introspection is best effort
+        return None
 
 
 class Clocks:
@@ -255,10 +262,13 @@ def run_ours(args):
             fwd()  # sizes the workspace
         torch.cuda.synchronize()
         g = None
+        kernels = None
         if graph:
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g, stream=stream):
                 fwd()
+            kernels = graph_kernel_nodes(g)
+            g.instantiate()
         run = g.replay if g is not None else fwd
         with torch.cuda.stream(stream):
             for _ in range(warmup):
@@ -283,7 +293,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         n_active = int(counts[0].item())
         status = int(counts[2].item())
-        return ms, n_active, status, clk.summary(), y
+        return ms, n_active, status, clk.summary(), y, kernels
 
     def measure_expert_stage(c, dd, steps):
         """Grouped execution alone (its own events), for the kernel roofline."""
@@ -375,7 +385,7 @@ def run_ours(args):
         ms = sum(a.elapsed_time(b) for a, b in ev) / steps
         return ms, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
 
-    ms, n_active, status, clocks, _ = measure(cfg, d, args.steps, args.warmup)
+    ms, n_active, status, clocks, _, kernels = measure(cfg, d, args.steps, args.warmup)
     ms_all = ms
     if world > 1:
         t = torch.tensor([ms], device=device)
@@ -394,7 +404,7 @@ def run_ours(args):
         sc = SECONDARY
         host2 = WL.make_inputs(sc.with_(seed=sc.seed + 1000 * rank), experts=False)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
-        ms2, na2, st2, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
+        ms2, na2, st2, _, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
         stages2 = measure_stages(sc, d2, 10)
         if world > 1:
             t = torch.tensor([ms2], device=device)
@@ -454,7 +464,10 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": world * cfg.L / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": kernel_launches(cfg) * args.steps,
+        # the library's kernels in the timed region: kernel nodes of the
+        # captured forward (one replay per step)
+        "gpu_launches": kernels * args.steps if kernels is not None else None,
+        "kernels_per_step": kernels,
         "clocks": clocks,
     }
     if extra:
