@@ -236,9 +236,14 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
          CUDA_SUCCESS;
 }
 
+// N tile: the widest the axes allow, narrowed while a few row tiles (small L)
+// would leave most SMs to split-K partials instead of output tiles.
 int pick_bn(const Dims& D) {
   const int64_t m = D.Nr < D.Nc ? D.Nr : D.Nc;
-  return m >= 256 ? 256 : (m >= 128 ? 128 : 64);
+  int bn = m >= 256 ? 256 : (m >= 128 ? 128 : 64);
+  const int64_t mt = (D.L + TC_BM - 1) / TC_BM;
+  while (bn > 64 && mt * ((D.Nr + bn - 1) / bn + (D.Nc + bn - 1) / bn) < 74) bn >>= 1;
+  return bn;
 }
 
 template <int BN>

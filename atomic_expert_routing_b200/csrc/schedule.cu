@@ -302,8 +302,9 @@ constexpr int kSmallRounds = kSmallMax / kSmallThreads;  // rounds of 32 keys pe
 
 // Same outputs as the multi-kernel path.  (1) Radix-sort the tasks' expert
 // ids; a scan of the "new id" flags gives U and the rank of every task's
-// expert.  (2) Radix-sort the composite keys (group, token, rank inside the
-// group) -- unique, and ordered exactly like (group, token, expert).  (3) Emit.
+// expert.  (2) Stable radix sort of the expert-ordered tasks by group * L +
+// token: equal keys keep their expert order, so the tasks end up ordered by
+// (group, token, expert).  (3) Emit.
 __global__ void __launch_bounds__(kSmallThreads)
     k_sched_small(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L,
                   int K, int64_t N, int64_t B, int epasses, int kpasses,
@@ -368,24 +369,26 @@ __global__ void __launch_bounds__(kSmallThreads)
     counts[1] = static_cast<int32_t>(G);
   }
   __syncthreads();
-  // (2) composite keys
-  const uint32_t Wl = static_cast<uint32_t>(B < M ? B : M);
-  for (int i = tid; i < M; i += kSmallThreads) {
-    const uint32_t rr = rk[i];
-    const uint32_t g = static_cast<uint32_t>(rr / static_cast<uint64_t>(B));
-    const uint32_t t = static_cast<uint32_t>(i / K);
-    keyA[i] = (g * static_cast<uint32_t>(L) + t) * Wl + (rr - g * static_cast<uint32_t>(B));
-    valA[i] = static_cast<uint16_t>(i);
+  // (2) key g * L + t over the expert-sorted tasks; the stable passes keep
+  // expert order among equal keys, so the result is ordered by (g, t, e)
+  for (int q = tid; q < M; q += kSmallThreads) {
+    const int i = vin[q];
+    const uint32_t g = static_cast<uint32_t>(rk[i] / static_cast<uint64_t>(B));
+    kout[q] = g * static_cast<uint32_t>(L) + static_cast<uint32_t>(i / K);
+    vout[q] = static_cast<uint16_t>(i);
   }
   __syncthreads();
-  kin = keyA; kout = keyB; vin = valA; vout = valB;
+  {
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
   for (int p = 0; p < kpasses; ++p) {
     block_radix_pass(kin, vin, kout, vout, M, 8 * p, wcount, dbase, warp_tot, &total);
     uint32_t* tk = kin; kin = kout; kout = tk;
     uint16_t* tv = vin; vin = vout; vout = tv;
   }
   // (3) emit
-  const uint32_t per_group = static_cast<uint32_t>(L) * Wl;
+  const uint32_t per_group = static_cast<uint32_t>(L);
   for (int p = tid; p < M; p += kSmallThreads) {
     const int i = vin[p];
     const uint32_t g = kin[p] / per_group;
@@ -465,9 +468,9 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
       return b;
     };
     const int epasses = (nbits(static_cast<uint64_t>(N)) + 7) / 8;
-    // composite key < gmax * L * min(B, M)
-    const int kpasses = (nbits(static_cast<uint64_t>(D.gmax()) * static_cast<uint64_t>(D.L) *
-                               static_cast<uint64_t>(D.B < M ? D.B : M)) + 7) / 8;
+    // key g * L + t < gmax * L
+    const int kpasses =
+        (nbits(static_cast<uint64_t>(D.gmax()) * static_cast<uint64_t>(D.L)) + 7) / 8;
     const size_t smem = static_cast<size_t>(kSmallMax) * (2 * sizeof(uint32_t) + 3 * sizeof(uint16_t)) +
                         static_cast<size_t>(kSmallWarps) * 256 * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(k_sched_small, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -194,26 +194,39 @@ __device__ __forceinline__ void sort_out(uint64_t* out, int m) {
   __syncwarp();
 }
 
-// Top `want` (<= 32*W) of the n keys make_key(value, id) a warp holds, by
-// (value desc, id asc), written sorted to out[0 .. 32*W) (padded with 0).
+template <int NW>
+__device__ __forceinline__ void group_sync(int bar_id) {
+  if (NW == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(NW * 32) : "memory");
+  }
+}
+
+// Top `want` (<= 32*W) of the n keys make_key(value, id) held by a group of
+// NW warps (gw: this warp's index in the group, bar_id: the group's named
+// barrier), by (value desc, id asc), written sorted to out[0 .. 32*W)
+// (padded with 0) by the group's warp 0 -- the other warps must synchronise
+// with it before reading out.
 //
-// for_each(f) calls f(value, id) for every element of the calling lane (in
-// any order; elements are split over the lanes), key_at(i) gives the key of
-// element i < n (used only by the fallback, after the whole warp has called
-// prepare()).  Value-range binning with lo/hi
-// the smallest/largest value: bin(v) = floor((v - lo) * 256 / (hi - lo)) is
-// monotone in v, so every key in a bin above the threshold bin is selected
-// and equal values share a bin.  A 256-bin histogram (shared-memory atomics)
-// finds the threshold bin; keys above it are compacted through an atomic
-// counter (about want of n), the threshold bin's keys (at most kCandMax) are
-// sorted in registers for the remainder, and the want keys are sorted in
-// registers.  A threshold bin that is too full, or a non-finite range, falls
-// back to the radix select.  hist: 256 words; tbk: kCandMax keys; cnt: 2 words.
-template <int W, typename ForEach, typename Prepare, typename KeyAt>
-__device__ void warp_topk(ForEach for_each, Prepare prepare, KeyAt key_at, int n, int want,
-                          float lo, float hi, uint64_t* out, uint32_t* hist, uint64_t* tbk,
-                          uint32_t* cnt) {
+// for_each(f) calls f(value, id) for every element of the calling thread (in
+// any order; elements are split over the group's threads), key_at(i) gives
+// the key of element i < n (used only by the fallback, after every thread
+// has called prepare()).  Value-range binning with lo/hi the smallest/largest
+// value: bin(v) = floor((v - lo) * 256 / (hi - lo)) is monotone in v, so
+// every key in a bin above the threshold bin is selected and equal values
+// share a bin.  A 256-bin histogram (shared-memory atomics) finds the
+// threshold bin; keys above it are compacted through an atomic counter
+// (about want of n), the threshold bin's keys (at most kCandMax) are sorted
+// in registers for the remainder, and the want keys are sorted in registers.
+// A threshold bin that is too full, or a non-finite range, falls back to the
+// radix select.  hist: 256 words; tbk: kCandMax keys; cnt: 2 words.
+template <int W, int NW, typename ForEach, typename Prepare, typename KeyAt>
+__device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare, KeyAt key_at,
+                           int n, int want, float lo, float hi, uint64_t* out, uint32_t* hist,
+                           uint64_t* tbk, uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
+  const int gt = gw * 32 + lane;
   const float range = hi - lo;
   const float scale = 256.0f / range;
   bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
@@ -222,16 +235,16 @@ __device__ void warp_topk(ForEach for_each, Prepare prepare, KeyAt key_at, int n
       const float f = (v - lo) * scale;
       return f >= 255.0f ? 255 : (f > 0.0f ? static_cast<int>(f) : 0);
     };
-#pragma unroll
-    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
-    if (lane == 0) {
+    for (int b = gt; b < 256; b += NW * 32) hist[b] = 0u;
+    if (gt == 0) {
       cnt[0] = 0u;
       cnt[1] = 0u;
     }
-    __syncwarp();
+    group_sync<NW>(bar_id);
     for_each([&](float v, uint32_t) { atomicAdd(&hist[bin(v)], 1u); });
-    __syncwarp();
-    // bins in descending order: lane l owns bins 255-8l ... 248-8l
+    group_sync<NW>(bar_id);
+    // every warp scans the bins in descending order: lane l owns bins
+    // 255-8l ... 248-8l
     uint32_t c[8];
     uint32_t tot = 0;
 #pragma unroll
@@ -273,29 +286,32 @@ __device__ void warp_topk(ForEach for_each, Prepare prepare, KeyAt key_at, int n
         if (b > tb) out[atomicAdd(&cnt[0], 1u)] = make_key(v, id);
         else if (b == tb) tbk[atomicAdd(&cnt[1], 1u)] = make_key(v, id);
       });
-      __syncwarp();
-      const int need = want - static_cast<int>(above);
-      if (at <= 32u) {
-        uint64_t key[1];
-        key[0] = lane < static_cast<int>(at) ? tbk[lane] : 0ull;
-        reg_sort_desc<1>(key);
-        if (lane < need) out[above + lane] = key[0];
-      } else {
-        uint64_t key[2];
-        key[0] = tbk[lane];
-        key[1] = 32 + lane < static_cast<int>(at) ? tbk[32 + lane] : 0ull;
-        reg_sort_desc<2>(key);
-        if (lane < need) out[above + lane] = key[0];
-        if (32 + lane < need) out[above + 32 + lane] = key[1];
+      group_sync<NW>(bar_id);
+      if (gw == 0) {
+        const int need = want - static_cast<int>(above);
+        if (at <= 32u) {
+          uint64_t key[1];
+          key[0] = lane < static_cast<int>(at) ? tbk[lane] : 0ull;
+          reg_sort_desc<1>(key);
+          if (lane < need) out[above + lane] = key[0];
+        } else {
+          uint64_t key[2];
+          key[0] = tbk[lane];
+          key[1] = 32 + lane < static_cast<int>(at) ? tbk[32 + lane] : 0ull;
+          reg_sort_desc<2>(key);
+          if (lane < need) out[above + lane] = key[0];
+          if (32 + lane < need) out[above + 32 + lane] = key[1];
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
   }
   if (!fast) {
     prepare();
-    warp_select_top(key_at, n, want, out, hist);
+    group_sync<NW>(bar_id);
+    if (gw == 0) warp_select_top(key_at, n, want, out, hist);
   }
-  sort_out<W>(out, want < n ? want : n);
+  if (gw == 0) sort_out<W>(out, want < n ? want : n);
 }
 
 struct SelPlan {
@@ -419,7 +435,8 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
       if (j * 32 + lane < n) s += expf(v[j] - mx);
     s = warp_sum(s);
     if (lane == 0) misc[role] = mx + logf(s);
-    warp_topk<W>(
+    group_topk<W, 1>(
+        0, 0,
         [&](auto f) {
 #pragma unroll
           for (int j = 0; j < NPL; ++j)
@@ -429,7 +446,6 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
 #pragma unroll
           for (int j = 0; j < NPL; ++j)
             if (j * 32 + lane < n) vals[j * 32 + lane] = v[j];
-          __syncwarp();
         },
         [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
         hist, tbin, cnt);
@@ -459,7 +475,8 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   cmx = warp_max(cmx);
   cmn = -warp_max(-cmn);
   __syncwarp();
-  warp_topk<WK>(
+  group_topk<WK, 1>(
+      0, 0,
       [&](auto f) {
         for (int c = lane; c < nc; c += 32) {
           const uint64_t kk = cand[c];
@@ -483,6 +500,244 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   }
 }
 
+// ---- small batches: one CTA of 8 warps per token ---------------------------
+//
+// The same selection with more warps per token, for batches too small to
+// fill the GPU with two warps per token: warps 0-3 take the row logits and
+// warps 4-7 the column logits (each warp NPW values per lane; named barriers
+// 1 and 2), and all eight warps form the merge candidates and their
+// histogram.  The sorted lists, the threshold bins and the gate are the work
+// of one warp, as in k_select.
+struct WidePlan {
+  int cand;
+  int off_vals, off_hist, off_sel, off_tbk, off_cnt, off_red, off_roff, off_cand, off_out, off_misc;
+  int bytes;
+};
+
+WidePlan make_wide_plan(const Dims& D, int W, int WK) {
+  WidePlan p{};
+  auto al = [](int v) { return (v + 15) & ~15; };
+  p.cand = merge_candidates(D);
+  const int nmax = static_cast<int>(D.Nr > D.Nc ? D.Nr : D.Nc);
+  int off = 0;
+  p.off_vals = off; off = al(off + 2 * 4 * nmax);
+  p.off_hist = off; off = al(off + 2 * 4 * 256);
+  p.off_sel = off; off = al(off + 2 * 8 * 32 * W);
+  p.off_tbk = off; off = al(off + 2 * 8 * kCandMax);
+  p.off_cnt = off; off = al(off + 16);
+  p.off_red = off; off = al(off + 4 * 3 * 8);
+  p.off_roff = off; off = al(off + 4 * static_cast<int>(D.k));
+  p.off_cand = off; off = al(off + 8 * p.cand);
+  p.off_out = off; off = al(off + 8 * 32 * WK);
+  p.off_misc = off; off = al(off + 16);
+  p.bytes = off;
+  return p;
+}
+
+template <int NPW, int W, int WK>
+__global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z, int parts,
+                                                     int64_t L, int Nr, int Nc, int k, int K,
+                                                     const float* __restrict__ br,
+                                                     const float* __restrict__ bc,
+                                                     int32_t* __restrict__ idx,
+                                                     float* __restrict__ gate,
+                                                     float* __restrict__ score, WidePlan P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int axis = warp >> 2, gw = warp & 3;
+  const int64_t t = blockIdx.x;
+  if (t >= L) return;  // the whole CTA leaves
+  const int nmax = Nr > Nc ? Nr : Nc;
+  float* red = reinterpret_cast<float*>(smem + P.off_red);   // [3][8]: max, min, sum
+  float* misc = reinterpret_cast<float*>(smem + P.off_misc);
+
+  // ---- per-axis: log-sum-exp and top-k, four warps per axis ----
+  {
+    const int n = axis ? Nc : Nr;
+    const float* z = Z + t * static_cast<int64_t>(Nr + Nc) + (axis ? Nr : 0);
+    const float* bias = axis ? bc : br;
+    float* vals = reinterpret_cast<float*>(smem + P.off_vals) + axis * nmax;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + P.off_hist) + axis * 256;
+    uint64_t* sel = reinterpret_cast<uint64_t*>(smem + P.off_sel) + axis * 32 * W;
+    uint64_t* tbk = reinterpret_cast<uint64_t*>(smem + P.off_tbk) + axis * kCandMax;
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + P.off_cnt) + 2 * axis;
+    const int bar = 1 + axis;
+    // split-K partial logits (parts > 1) are summed here, in order
+    const int64_t zs = L * static_cast<int64_t>(Nr + Nc);
+    float v[NPW];
+#pragma unroll
+    for (int j = 0; j < NPW; ++j) {
+      const int i = (j * 4 + gw) * 32 + lane;
+      v[j] = i < n ? z[i] : 0.0f;
+    }
+#pragma unroll 4
+    for (int p = 1; p < parts; ++p) {
+#pragma unroll
+      for (int j = 0; j < NPW; ++j) {
+        const int i = (j * 4 + gw) * 32 + lane;
+        if (i < n) v[j] += z[p * zs + i];
+      }
+    }
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int j = 0; j < NPW; ++j) {
+      const int i = (j * 4 + gw) * 32 + lane;
+      float x = 0.0f;
+      if (i < n) {
+        x = v[j];
+        if (bias != nullptr) x += bias[i];
+        x = (x == 0.0f) ? 0.0f : x;  // one zero (no -0) so equal logits tie
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+      }
+      v[j] = x;
+    }
+    mx = warp_max(mx);
+    mn = -warp_max(-mn);
+    if (lane == 0) {
+      red[warp] = mx;
+      red[8 + warp] = mn;
+    }
+    group_sync<4>(bar);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      mx = fmaxf(mx, red[axis * 4 + q]);
+      mn = fminf(mn, red[8 + axis * 4 + q]);
+    }
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPW; ++j)
+      if ((j * 4 + gw) * 32 + lane < n) s += expf(v[j] - mx);
+    s = warp_sum(s);
+    if (lane == 0) red[16 + warp] = s;
+    group_sync<4>(bar);
+    if (gw == 0 && lane == 0) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tot += red[16 + axis * 4 + q];
+      misc[axis] = mx + logf(tot);
+    }
+    group_topk<W, 4>(
+        gw, bar,
+        [&](auto f) {
+#pragma unroll
+          for (int j = 0; j < NPW; ++j) {
+            const int i = (j * 4 + gw) * 32 + lane;
+            if (i < n) f(v[j], static_cast<uint32_t>(i));
+          }
+        },
+        [&]() {  // the radix fallback reads values by index
+#pragma unroll
+          for (int j = 0; j < NPW; ++j) {
+            const int i = (j * 4 + gw) * 32 + lane;
+            if (i < n) vals[i] = v[j];
+          }
+        },
+        [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
+        hist, tbk, cnt);
+  }
+  __syncthreads();
+
+  // ---- k x k merge, all eight warps ----
+  const uint64_t* sr = reinterpret_cast<const uint64_t*>(smem + P.off_sel);
+  const uint64_t* sc = sr + 32 * W;
+  int32_t* roff = reinterpret_cast<int32_t*>(smem + P.off_roff);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + P.off_cand);
+  uint64_t* out = reinterpret_cast<uint64_t*>(smem + P.off_out);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + P.off_hist);
+  uint64_t* tbk = reinterpret_cast<uint64_t*>(smem + P.off_tbk);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + P.off_cnt);
+  if (warp == 0) {
+    // pairs of row a start at roff[a] (prefix of min(k, K/(a+1)))
+    int na = 0;
+    for (int a0 = 0; a0 < k; a0 += 32) {
+      const int a = a0 + lane;
+      int nb = 0;
+      if (a < k) {
+        nb = K / (a + 1);
+        if (nb > k) nb = k;
+      }
+      int incl = nb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t2;
+      }
+      if (a < k) roff[a] = na + incl - nb;
+      na += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  __syncthreads();
+  const int nc = P.cand;
+  float cmx = -INFINITY, cmn = INFINITY;
+  for (int c = threadIdx.x; c < nc; c += 256) {
+    int lo = 0, hi = k - 1;  // last row a with roff[a] <= c
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (roff[mid] <= c) lo = mid; else hi = mid - 1;
+    }
+    const uint64_t ra = sr[lo], cb = sc[c - roff[lo]];
+    const float sv = key_val(ra) + key_val(cb);
+    cand[c] = make_key(sv, key_id(ra) * static_cast<uint32_t>(Nc) + key_id(cb));
+    cmx = fmaxf(cmx, sv);
+    cmn = fminf(cmn, sv);
+  }
+  cmx = warp_max(cmx);
+  cmn = -warp_max(-cmn);
+  if (lane == 0) {
+    red[warp] = cmx;
+    red[8 + warp] = cmn;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    cmx = fmaxf(cmx, red[q]);
+    cmn = fminf(cmn, red[8 + q]);
+  }
+  group_topk<WK, 8>(
+      warp, 0,
+      [&](auto f) {
+        for (int c = threadIdx.x; c < nc; c += 256) {
+          const uint64_t kk = cand[c];
+          f(key_val(kk), key_id(kk));
+        }
+      },
+      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbk, cnt);
+  if (warp != 0) return;
+
+  // ---- gate = softmax of the K selected joint scores ----
+  const float s0 = key_val(out[0]);
+  float wsum = 0.0f;
+  for (int q = lane; q < K; q += 32) wsum += expf(key_val(out[q]) - s0);
+  wsum = warp_sum(wsum);
+  const float lse = misc[0] + misc[1];
+  for (int q = lane; q < K; q += 32) {
+    const uint64_t kk = out[q];
+    const float v = key_val(kk);
+    idx[t * K + q] = static_cast<int32_t>(key_id(kk));
+    gate[t * K + q] = expf(v - s0) / wsum;
+    if (score != nullptr) score[t * K + q] = v - lse;
+  }
+}
+
+template <int NPW, int W, int WK>
+cudaError_t launch_wide_t(const Dims& D, const float* Z, int parts, const float* br,
+                          const float* bc, int32_t* idx, float* gate, float* score,
+                          cudaStream_t s) {
+  const WidePlan P = make_wide_plan(D, W, WK);
+  cudaError_t err = cudaFuncSetAttribute(k_select_wide<NPW, W, WK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P.bytes);
+  if (err != cudaSuccess) return err;
+  k_select_wide<NPW, W, WK><<<static_cast<unsigned>(D.L), 256, P.bytes, s>>>(
+      Z, parts, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
+      static_cast<int>(D.K), br, bc, idx, gate, score, P);
+  return cudaGetLastError();
+}
+
+template <int NPW>
+cudaError_t launch_wide(const Dims& D, const float* Z, int parts, const float* br,
+                        const float* bc, int32_t* idx, float* gate, float* score, cudaStream_t s);
+
 int sort_width(int64_t m) {
   int w = 1;
   while (32 * w < m) w <<= 1;
@@ -493,7 +748,12 @@ template <int NPL, int W, int WK>
 cudaError_t launch_select_t(const Dims& D, const float* Z, const float* br, const float* bc,
                             int32_t* idx, float* gate, float* score, cudaStream_t s) {
   SelPlan P = make_plan(D, W, WK);
+  // up to four tokens per CTA, fewer when that leaves SMs idle (small batches)
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int pairs = 4;
+  while (pairs > 1 && (D.L + pairs - 1) / pairs < sms) pairs >>= 1;
   while (pairs > 1 && P.table_bytes + pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
   const size_t smem = static_cast<size_t>(P.table_bytes) + static_cast<size_t>(pairs) * P.pair_bytes;
   cudaError_t err =
@@ -519,17 +779,36 @@ cudaError_t launch_select_npl(const Dims& D, const float* Z, const float* br, co
   }
 }
 
+template <int NPW>
+cudaError_t launch_wide(const Dims& D, const float* Z, int parts, const float* br,
+                        const float* bc, int32_t* idx, float* gate, float* score, cudaStream_t s) {
+  switch (sort_width(D.k > D.K ? D.k : D.K)) {
+    case 1: return launch_wide_t<NPW, 1, 1>(D, Z, parts, br, bc, idx, gate, score, s);
+    case 2: return launch_wide_t<NPW, 2, 2>(D, Z, parts, br, bc, idx, gate, score, s);
+    case 4: return launch_wide_t<NPW, 4, 4>(D, Z, parts, br, bc, idx, gate, score, s);
+    default: return launch_wide_t<NPW, 8, 8>(D, Z, parts, br, bc, idx, gate, score, s);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
                           const float* bc, int32_t* idx, float* gate, float* score,
                           cudaStream_t s) {
   if (D.L == 0) return cudaSuccess;
+  const int64_t n = D.Nr > D.Nc ? D.Nr : D.Nc;
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (D.L <= sms) {  // too few tokens for two warps each to fill the GPU
+    if (n <= 256) return launch_wide<2>(D, Z, parts, br, bc, idx, gate, score, s);
+    if (n <= 1024) return launch_wide<8>(D, Z, parts, br, bc, idx, gate, score, s);
+    return launch_wide<32>(D, Z, parts, br, bc, idx, gate, score, s);
+  }
   if (parts > 1) {  // split-K partial logits: sum them first, in a fixed order
     cudaError_t e = launch_sum_partials(const_cast<float*>(Z), parts, D.L * (D.Nr + D.Nc), s);
     if (e != cudaSuccess) return e;
   }
-  const int64_t n = D.Nr > D.Nc ? D.Nr : D.Nc;
   if (n <= 256) return launch_select_npl<8>(D, Z, br, bc, idx, gate, score, s);
   if (n <= 1024) return launch_select_npl<32>(D, Z, br, bc, idx, gate, score, s);
   if (n <= 2048) return launch_select_npl<64>(D, Z, br, bc, idx, gate, score, s);

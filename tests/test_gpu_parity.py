@@ -338,9 +338,11 @@ def test_edge_shapes(cfg):
     assert rel_err(host_f64(yt), host_f64(y)) <= tol_y(cfg)
 
 
-def test_equal_logits_pick_smallest_ids():
-    """x = 0: every joint score ties; the K smallest ids of the k x k grid win."""
-    cfg = WL.Config("ties", L=8, d=64, Nr=16, Nc=24, k=4, K=6, B=4, dtype=WL.BF16, seed=3)
+@pytest.mark.parametrize("L", [8, 300], ids=["one-cta-per-token", "two-warps-per-token"])
+def test_equal_logits_pick_smallest_ids(L):
+    """x = 0: every joint score ties; the K smallest ids of the k x k grid win
+    (small batches take the 8-warp selection, larger ones the 2-warp one)."""
+    cfg = WL.Config("ties", L=L, d=64, Nr=16, Nc=24, k=4, K=6, B=4, dtype=WL.BF16, seed=3)
     h = WL.make_inputs(cfg)
     h["x"] = np.zeros_like(h["x"])
     d = {k: dev(v) for k, v in h.items()}
