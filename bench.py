@@ -62,6 +62,32 @@ def expert_stage_bytes(cfg, n_active):
     return 2 * cfg.d * n_active * e + 2 * cfg.L * cfg.d * e
 
 
+def rank_inputs(cfg, rank):
+    """Host inputs of one data-parallel rank: its own token batch x (seed +
+    1000*rank for ranks > 0) with the shared router weights and biases."""
+    host = WL.make_inputs(cfg, experts=False)
+    if rank > 0:
+        host["x"] = WL.make_inputs(cfg.with_(seed=cfg.seed + 1000 * rank), experts=False)["x"]
+    return host
+
+
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks: a job step takes as long as its
+    slowest rank (x itself with one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms):
+    """Whole-job tokens/s: every rank processes its own batch in ms (max over ranks)."""
+    return world * tokens_per_rank / (ms * 1e-3)
+
+
 def graph_kernel_nodes(g):
     """Kernel nodes of a captured CUDA graph (the forward's own launches; memset
     nodes excluded), or None when the graph cannot be inspected."""
@@ -230,11 +256,7 @@ def run_ours(args):
         return torch.from_numpy(a).to(device)
 
     cfg = {**WL.CONFIGS, **WL.EXTRA}[args.workload]
-    # every rank draws its own token batch (seed + rank); weights are shared
-    rcfg = cfg.with_(seed=cfg.seed)
-    host = WL.make_inputs(rcfg, experts=False)
-    if rank > 0:
-        host["x"] = WL.make_inputs(cfg.with_(seed=cfg.seed + 1000 * rank), experts=False)["x"]
+    host = rank_inputs(cfg, rank)  # own token batch per rank; weights are shared
     experts = WL.make_experts(cfg)
     d = {k: to_dev(v) for k, v in host.items()}
     d.update({k: to_dev(v) for k, v in experts.items()})
@@ -386,33 +408,23 @@ def run_ours(args):
         return ms, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
 
     ms, n_active, status, clocks, _, kernels = measure(cfg, d, args.steps, args.warmup)
-    ms_all = ms
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_all = float(t.item())
+    ms_all = max_over_ranks(ms, world, device)
     e2e_ms, h2d, d2h = measure_e2e(cfg, d, max(3, args.steps // 2), args.warmup)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
     st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
     stages = measure_stages(cfg, d, max(3, args.steps // 2))
 
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
         sc = SECONDARY
-        host2 = WL.make_inputs(sc.with_(seed=sc.seed + 1000 * rank), experts=False)
+        host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
         ms2, na2, st2, _, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
         stages2 = measure_stages(sc, d2, 10)
-        if world > 1:
-            t = torch.tensor([ms2], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms2 = float(t.item())
+        ms2 = max_over_ranks(ms2, world, device)
         f2, b2 = layer_work(sc, na2)
         extra[sc.name] = {
-            "value": world * sc.L / (ms2 * 1e-3), "unit": "tokens/s", "ms_per_step": ms2,
+            "value": job_throughput(world, sc.L, ms2), "unit": "tokens/s", "ms_per_step": ms2,
             "n_active": na2, "device_status": st2, "stages_ms": stages2,
             "layer_roofline": {"bound": "hbm" if b2 / (hbm * 1e9) > f2 / (tc * 1e12) else "tensor",
                                "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
@@ -437,7 +449,7 @@ def run_ours(args):
                          f"execution, fp64), {dt:.1f} s"}
     line = {
         "metric": METRIC,
-        "value": world * cfg.L / (ms_all * 1e-3),
+        "value": job_throughput(world, cfg.L, ms_all),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -462,7 +474,7 @@ def run_ours(args):
                      "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": eb,
                      "ms": st_ms, "peak_src": peak_src},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * cfg.L / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(world, cfg.L, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         # the library's kernels in the timed region: kernel nodes of the
         # captured forward (one replay per step)

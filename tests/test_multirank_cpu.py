@@ -1,0 +1,66 @@
+"""Host logic of the data-parallel bench (one rank per GPU, no collective on
+the data path) on two gloo ranks on the CPU: the step time is the slowest
+rank's, the job throughput counts every rank's batch, and each rank gets its
+own token batch with the shared weights."""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import workloads as WL
+
+CFG = WL.Config("ranks", L=16, d=64, Nr=8, Nc=8, k=2, K=2, B=4, dtype=WL.BF16, seed=5)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = bench.max_over_ranks(times[rank], world, "cpu")
+        x = bench.rank_inputs(CFG, rank)["x"]
+        np.save(os.path.join(out_dir, f"x{rank}.npy"), x)
+        with open(os.path.join(out_dir, f"ms{rank}.txt"), "w") as f:
+            f.write(repr(ms))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_two_ranks_reduce_to_the_slowest(tmp_path):
+    times = [1.25, 3.5]
+    mp.spawn(_rank_main, args=(2, _free_port(), times, str(tmp_path)), nprocs=2, join=True)
+    got = [float(open(tmp_path / f"ms{r}.txt").read()) for r in range(2)]
+    assert got == [max(times)] * 2
+    x0, x1 = np.load(tmp_path / "x0.npy"), np.load(tmp_path / "x1.npy")
+    assert x0.shape == x1.shape == (CFG.L, CFG.d)
+    assert not np.array_equal(x0, x1)  # each rank its own batch
+    # rank 0's batch is the workload's own; other ranks' are seeded apart
+    np.testing.assert_array_equal(x0, WL.make_inputs(CFG, experts=False)["x"])
+
+
+def test_rank_inputs_share_the_router_weights():
+    a, b = bench.rank_inputs(CFG, 0), bench.rank_inputs(CFG, 3)
+    for key in ("Wr", "Wc"):
+        np.testing.assert_array_equal(a[key], b[key])
+    assert not np.array_equal(a["x"], b["x"])
+    np.testing.assert_array_equal(b["x"], bench.rank_inputs(CFG, 3)["x"])  # deterministic
+
+
+def test_job_throughput_counts_every_rank():
+    assert bench.job_throughput(1, 16384, 2.0) == pytest.approx(8.192e6)
+    assert bench.job_throughput(4, 16384, 2.0) == pytest.approx(4 * 8.192e6)
+    assert bench.max_over_ranks(2.5, 1, "cpu") == 2.5
