@@ -62,6 +62,17 @@ def expert_stage_bytes(cfg, n_active):
     return 2 * cfg.d * n_active * e + 2 * cfg.L * cfg.d * e
 
 
+# DRAM bytes (read + write) of one expert-stage call, summed over its kernels,
+# from ncu. The full-size stage is too large for a full capture; these values
+# come from the proxy workload (profiles/expert_stage_bf16-prefill-proxy-N256K.md,
+# 1774.8 MB) scaled by the stage's algorithmic bytes (x3.90). Update them
+# whenever the stage's kernels change, else report None.
+STAGE_TRAFFIC = {
+    "bf16-prefill-N1M": (6.92e9, "ncu dram__bytes of bf16-prefill-proxy-N256K, scaled x3.90 "
+                                 "by algorithmic bytes"),
+}
+
+
 def rank_inputs(cfg, rank):
     """Host inputs of one data-parallel rank: its own token batch x (seed +
     1000*rank for ranks > 0) with the shared router weights and biases."""
@@ -471,7 +482,10 @@ def run_ours(args):
                            "flops": flops, "peak_src": peak_src},
         "roofline": {"kernel": "grouped expert-centric execution (omni_expert_forward)",
                      "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "algorithmic_bytes": eb,
+                     "frac": achieved / hbm,
+                     "traffic": STAGE_TRAFFIC.get(cfg.name, (None, None))[0],
+                     "traffic_src": STAGE_TRAFFIC.get(cfg.name, (None, None))[1],
+                     "algorithmic_bytes": eb,
                      "ms": st_ms, "peak_src": peak_src},
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(world, cfg.L, e2e_ms), "unit": "tokens/s",
