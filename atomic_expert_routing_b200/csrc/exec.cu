@@ -36,11 +36,27 @@ constexpr int kExpThreads = 128;  // 4 warps per CTA, each executing its own tas
 // Elements per 16-byte vector.
 template <typename T> constexpr int kEpv = 16 / sizeof(T);
 
-// Dot product contribution of one 16-byte vector pair, widened to fp32.
+// s0 += a.lo * b.lo, s1 += a.hi * b.hi for two bf16 pairs, with the
+// mixed-precision fma (bf16 operands, fp32 addend and result, one rounding):
+// the same value as widening both operands to fp32 and using fmaf.
+__device__ __forceinline__ void fma_bf16x2(float& s0, float& s1, uint32_t a, uint32_t b) {
+  asm("{\n .reg .b16 al, ah, bl, bh;\n"
+      " mov.b32 {al, ah}, %2;\n"
+      " mov.b32 {bl, bh}, %3;\n"
+      " fma.rn.f32.bf16 %0, al, bl, %0;\n"
+      " fma.rn.f32.bf16 %1, ah, bh, %1;\n}"
+      : "+f"(s0), "+f"(s1)
+      : "r"(a), "r"(b));
+}
+
+// Dot product contribution of one 16-byte vector pair, in fp32.
 __device__ __forceinline__ float dot_vec(uint4 a, uint4 b, __nv_bfloat16*) {
-  return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
-         bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
-         bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+  float s0 = 0.0f, s1 = 0.0f;
+  fma_bf16x2(s0, s1, a.x, b.x);
+  fma_bf16x2(s0, s1, a.y, b.y);
+  fma_bf16x2(s0, s1, a.z, b.z);
+  fma_bf16x2(s0, s1, a.w, b.w);
+  return s0 + s1;
 }
 __device__ __forceinline__ float dot_vec(uint4 a, uint4 b, float*) {
   return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
