@@ -219,6 +219,11 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -392,12 +397,14 @@ constexpr int kActWarps = 8;
 // c[dst[a]] = g[a] * SiLU(H[hidx[a]] . F[fidx[a]]) over a task list in which
 // tasks that share a held row H[h] are adjacent (a run).  Warp w takes slices
 // of S consecutive tasks; the run's held row sits in registers (the next
-// run's row is fetched while the current one is used; evict-first when
-// HOLD_ONCE), and every task's row of F streams through a ring of R
-// shared-memory slots per warp (cp.async, R - 1 rows in flight).  dst ==
+// run's row is fetched while the current one is used), and every task's row
+// of F streams through a ring of R shared-memory slots per warp (cp.async,
+// R - 1 rows in flight).  HOLD_KEEP: the held rows are re-read by later
+// tasks (x by token) -- keep them in L2 (evict-last) and read the F rows,
+// whose repeats come right after their first read, evict-first.  dst ==
 // nullptr writes c[a].  Indices are range-checked (OMNI_DEV_BAD_INDEX; the
 // task gets c = 0).
-template <typename T, int NV, int R, bool HOLD_ONCE>
+template <typename T, int NV, int R, bool HOLD_KEEP>
 __global__ void __launch_bounds__(kActWarps * 32, 2)
     k_act(const T* __restrict__ H, const int32_t* __restrict__ hidx, int64_t nh,
           const T* __restrict__ F, const int32_t* __restrict__ fidx, int64_t nf,
@@ -409,6 +416,7 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
   uint4* fring = ring + static_cast<size_t>(warp) * R * SLOT;
   const uint32_t fring_s = static_cast<uint32_t>(__cvta_generic_to_shared(fring));
   const uint64_t pol_once = policy_evict_first();
+  const uint64_t pol_keep = policy_evict_last();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kActWarps;
   for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kActWarps + warp; sl < nslices; sl += nw) {
     const int64_t a0 = sl * S;
@@ -436,8 +444,12 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
           const uint4* fr = reinterpret_cast<const uint4*>(F + f * d);
           const uint32_t base = fring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
 #pragma unroll
-          for (int v = 0; v < NV; ++v)
-            cp_async16_plain(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane);
+          for (int v = 0; v < NV; ++v) {
+            if (HOLD_KEEP)
+              cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane, pol_once);
+            else
+              cp_async16_plain(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane);
+          }
         }
       }
       cp_async_commit();
@@ -448,7 +460,7 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
     auto load_held = [&](int64_t h) {
       const uint4* hr = reinterpret_cast<const uint4*>(H + (h < 0 ? 0 : h) * d);
 #pragma unroll
-      for (int v = 0; v < NV; ++v) hn[v] = HOLD_ONCE ? ld_v4_hint(hr + v * 32 + lane, pol_once) : hr[v * 32 + lane];
+      for (int v = 0; v < NV; ++v) hn[v] = HOLD_KEEP ? ld_v4_hint(hr + v * 32 + lane, pol_keep) : hr[v * 32 + lane];
     };
     load_held(__shfl_sync(0xffffffffu, my_h, 0));
     for (int j = 0; j < n; ++j) {
@@ -665,7 +677,8 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
   static_assert(32 % D == 0, "the prefetch distance divides the slice");
   using QT = typename Quad<T>::type;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint64_t pol_stream = policy_evict_first();
+  // V rows of a window's repeated experts are re-read soon: normal priority
+  const uint64_t pol_stream = policy_evict_normal();
   const uint64_t pol_keep = policy_evict_last();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kAccWarps;
   int64_t sl = static_cast<int64_t>(blockIdx.x) * kAccWarps + warp;
@@ -1037,7 +1050,7 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
   constexpr int R = 3;
   constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
-  err = cudaFuncSetAttribute(k_act<T, NV, R, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  err = cudaFuncSetAttribute(k_act<T, NV, R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int64_t M = D.M();
@@ -1047,7 +1060,7 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   if (blocks > 2 * sm_count()) blocks = 2 * sm_count();
   // tasks by expert: x[t] held per run of one token, the W rows through the
   // ring (an expert's repeated row comes from L2 right after its first read)
-  k_act<T, NV, R, false><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
+  k_act<T, NV, R, true><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
       static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W), w.win.xe, D.N(),
       w.win.xg, w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status);
   err = cudaGetLastError();
