@@ -231,9 +231,9 @@ __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare
   const float scale = 256.0f / range;
   bool fast = want < n && range > 0.0f && isfinite(scale) && isfinite(range);
   if (fast) {
-    auto bin = [&](float v) -> int {
-      const float f = (v - lo) * scale;
-      return f >= 255.0f ? 255 : (f > 0.0f ? static_cast<int>(f) : 0);
+    const float off = -lo * scale;
+    auto bin = [&](float v) -> int {  // monotone in v: one fma, clamped to [0, 255]
+      return __float2int_rz(fminf(fmaxf(fmaf(v, scale, off), 0.0f), 255.0f));
     };
     for (int b = gt; b < 256; b += NW * 32) hist[b] = 0u;
     if (gt == 0) {
@@ -320,6 +320,7 @@ struct SelPlan {
       off_cnt;
   int pair_bytes;
   int table_bytes;                    // per CTA: the (a, b) pair table
+  int bias_bytes;                     // per CTA: cached row/column biases (0 without bias)
 };
 
 int merge_candidates(const Dims& D) {
@@ -347,19 +348,30 @@ SelPlan make_plan(const Dims& D, int W, int WK) {
   p.off_sc = off; off = al(off + 8 * 32 * W);
   p.off_cand = off; off = al(off + 8 * p.cand);
   p.off_out = off; off = al(off + 8 * 32 * WK);
-  p.off_misc = off; off = al(off + 16);
+  p.off_misc = off; off = al(off + 32);
   p.off_tr = off; off = al(off + 8 * kCandMax);
   p.off_tc = off; off = al(off + 8 * kCandMax);
   p.off_cnt = off; off = al(off + 16);
   p.pair_bytes = off;
   p.table_bytes = al(4 * p.cand);
+  p.bias_bytes = 0;
   return p;
 }
 
+__device__ __forceinline__ void cp_async4(float* dst, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
 // NPL: logits per lane and axis (n <= 32*NPL); W, WK: sorted lengths 32*W >=
-// k and 32*WK >= K.
+// k and 32*WK >= K.  Persistent: pair p of CTA b takes tokens b*pairs + p,
+// + gridDim.x*pairs, ...; while it merges one token, each warp's logits of
+// its next token land in shared memory (cp.async, each lane its own
+// elements), and the biases sit in shared memory for the whole CTA.
 template <int NPL, int W, int WK>
-__global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int64_t L, int Nr,
+__global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, int64_t L, int Nr,
                                                 int Nc, int k, int K,
                                                 const float* __restrict__ br,
                                                 const float* __restrict__ bc,
@@ -375,6 +387,7 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   // (a, b) pairs with (a+1)(b+1) <= K, row by row: pair c of row a sits at
   // roff(a) + b, roff the prefix sum of min(k, K/(a+1)); built once per CTA
   uint32_t* cab = reinterpret_cast<uint32_t*>(smem);
+  float* bias_s = reinterpret_cast<float*>(smem + P.table_bytes);  // [Nr + Nc] when biased
   if (threadIdx.x < 32) {
     int base = 0;
     for (int a0 = 0; a0 < k; a0 += 32) {
@@ -395,23 +408,42 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
+  if (P.bias_bytes > 0) {
+    for (int i = threadIdx.x; i < Nr + Nc; i += blockDim.x)
+      bias_s[i] = i < Nr ? (br != nullptr ? br[i] : 0.0f) : (bc != nullptr ? bc[i - Nr] : 0.0f);
+  }
   __syncthreads();
 
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * pairs + pair;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * pairs;
+  int64_t t = static_cast<int64_t>(blockIdx.x) * pairs + pair;
   if (t >= L) return;  // both warps of the pair leave together
-  uint8_t* base = smem + P.table_bytes + static_cast<size_t>(pair) * P.pair_bytes;
+  uint8_t* base = smem + P.table_bytes + P.bias_bytes + static_cast<size_t>(pair) * P.pair_bytes;
   float* misc = reinterpret_cast<float*>(base + P.off_misc);
+  const int n = role ? Nc : Nr;
+  const int zoff = role ? Nr : 0;
+  // this warp's logits of one token (raw, before bias); the radix fallback
+  // also reads values from here
+  float* vals = reinterpret_cast<float*>(base + (role ? P.off_vc : P.off_vr));
+  auto prefetch = [&](int64_t tt) {
+    const float* z = Z + tt * static_cast<int64_t>(Nr + Nc) + zoff;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      const int i = j * 32 + lane;
+      if (i < n) cp_async4(vals + i, z + i);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  prefetch(t);
 
+  for (; t < L; t += stride) {
   // ---- per-axis: log-sum-exp and top-k ----
   {
-    const int n = role ? Nc : Nr;
-    const float* z = Z + t * static_cast<int64_t>(Nr + Nc) + (role ? Nr : 0);
-    const float* bias = role ? bc : br;
-    float* vals = reinterpret_cast<float*>(base + (role ? P.off_vc : P.off_vr));
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + (role ? P.off_hc : P.off_hr));
     uint64_t* sel = reinterpret_cast<uint64_t*>(base + (role ? P.off_sc : P.off_sr));
     uint64_t* tbin = reinterpret_cast<uint64_t*>(base + (role ? P.off_tc : P.off_tr));
     uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt) + 2 * role;
+    const float* bias = P.bias_bytes > 0 ? bias_s + zoff : nullptr;
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies of token t
     float v[NPL];
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
@@ -419,7 +451,7 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
       const int i = j * 32 + lane;
       float x = 0.0f;
       if (i < n) {
-        x = z[i];
+        x = vals[i];
         if (bias != nullptr) x += bias[i];
         x = (x == 0.0f) ? 0.0f : x;  // one zero (no -0) so equal logits tie
         mx = fmaxf(mx, x);
@@ -432,7 +464,7 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
     float s = 0.0f;
 #pragma unroll
     for (int j = 0; j < NPL; ++j)
-      if (j * 32 + lane < n) s += expf(v[j] - mx);
+      if (j * 32 + lane < n) s += __expf(v[j] - mx);
     s = warp_sum(s);
     if (lane == 0) misc[role] = mx + logf(s);
     group_topk<W, 1>(
@@ -449,11 +481,13 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
         },
         [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
         hist, tbin, cnt);
+    __syncwarp();
+    if (t + stride < L) prefetch(t + stride);  // lands while the pair merges
   }
   asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
-  if (role != 0) return;
+  const float lse = misc[0] + misc[1];  // read before the next token rewrites them
 
-  // ---- k x k merge over the pairs that can reach the top-K ----
+  // ---- k x k merge over the pairs that can reach the top-K (both warps) ----
   const uint64_t* sr = reinterpret_cast<const uint64_t*>(base + P.off_sr);
   const uint64_t* sc = reinterpret_cast<const uint64_t*>(base + P.off_sc);
   uint64_t* cand = reinterpret_cast<uint64_t*>(base + P.off_cand);
@@ -462,8 +496,9 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   uint64_t* tbin = reinterpret_cast<uint64_t*>(base + P.off_tr);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt);
   const int nc = P.cand;
+  const int pt = role * 32 + lane;  // thread of the pair
   float cmx = -INFINITY, cmn = INFINITY;
-  for (int c = lane; c < nc; c += 32) {
+  for (int c = pt; c < nc; c += 64) {
     const uint32_t ab = cab[c];
     const uint64_t ra = sr[ab >> 16], cb = sc[ab & 0xffffu];
     const float sv = key_val(ra) + key_val(cb);
@@ -474,30 +509,40 @@ __global__ void __launch_bounds__(256) k_select(const float* __restrict__ Z, int
   }
   cmx = warp_max(cmx);
   cmn = -warp_max(-cmn);
-  __syncwarp();
-  group_topk<WK, 1>(
-      0, 0,
+  if (lane == 0) {
+    misc[2 + role] = cmx;
+    misc[4 + role] = cmn;
+  }
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
+  cmx = fmaxf(misc[2], misc[3]);
+  cmn = fminf(misc[4], misc[5]);
+  group_topk<WK, 2>(
+      role, 1 + pair,
       [&](auto f) {
-        for (int c = lane; c < nc; c += 32) {
+        for (int c = pt; c < nc; c += 64) {
           const uint64_t kk = cand[c];
           f(key_val(kk), key_id(kk));
         }
       },
       []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbin, cnt);
-
-  // ---- gate = softmax of the K selected joint scores ----
-  const float s0 = key_val(out[0]);
-  float wsum = 0.0f;
-  for (int q = lane; q < K; q += 32) wsum += expf(key_val(out[q]) - s0);
-  wsum = warp_sum(wsum);
-  const float lse = misc[0] + misc[1];
-  for (int q = lane; q < K; q += 32) {
-    const uint64_t kk = out[q];
-    const float v = key_val(kk);
-    idx[t * K + q] = static_cast<int32_t>(key_id(kk));
-    gate[t * K + q] = expf(v - s0) / wsum;
-    if (score != nullptr) score[t * K + q] = v - lse;
+  if (role == 0) {
+    // ---- gate = softmax of the K selected joint scores ----
+    const float s0 = key_val(out[0]);
+    float wsum = 0.0f;
+    for (int q = lane; q < K; q += 32) wsum += __expf(key_val(out[q]) - s0);
+    wsum = warp_sum(wsum);
+    for (int q = lane; q < K; q += 32) {
+      const uint64_t kk = out[q];
+      const float v = key_val(kk);
+      idx[t * K + q] = static_cast<int32_t>(key_id(kk));
+      gate[t * K + q] = __expf(v - s0) / wsum;
+      if (score != nullptr) score[t * K + q] = v - lse;
+    }
   }
+  // the next token's merge reuses out/cand/hist: both warps meet first
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // ---- small batches: one CTA of 8 warps per token ---------------------------
@@ -607,7 +652,7 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
     float s = 0.0f;
 #pragma unroll
     for (int j = 0; j < NPW; ++j)
-      if ((j * 4 + gw) * 32 + lane < n) s += expf(v[j] - mx);
+      if ((j * 4 + gw) * 32 + lane < n) s += __expf(v[j] - mx);
     s = warp_sum(s);
     if (lane == 0) red[16 + warp] = s;
     group_sync<4>(bar);
@@ -708,14 +753,14 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
   // ---- gate = softmax of the K selected joint scores ----
   const float s0 = key_val(out[0]);
   float wsum = 0.0f;
-  for (int q = lane; q < K; q += 32) wsum += expf(key_val(out[q]) - s0);
+  for (int q = lane; q < K; q += 32) wsum += __expf(key_val(out[q]) - s0);
   wsum = warp_sum(wsum);
   const float lse = misc[0] + misc[1];
   for (int q = lane; q < K; q += 32) {
     const uint64_t kk = out[q];
     const float v = key_val(kk);
     idx[t * K + q] = static_cast<int32_t>(key_id(kk));
-    gate[t * K + q] = expf(v - s0) / wsum;
+    gate[t * K + q] = __expf(v - s0) / wsum;
     if (score != nullptr) score[t * K + q] = v - lse;
   }
 }
@@ -748,19 +793,27 @@ template <int NPL, int W, int WK>
 cudaError_t launch_select_t(const Dims& D, const float* Z, const float* br, const float* bc,
                             int32_t* idx, float* gate, float* score, cudaStream_t s) {
   SelPlan P = make_plan(D, W, WK);
+  if (br != nullptr || bc != nullptr) P.bias_bytes = static_cast<int>((4 * (D.Nr + D.Nc) + 15) & ~15);
   // up to four tokens per CTA, fewer when that leaves SMs idle (small batches)
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int pairs = 4;
   while (pairs > 1 && (D.L + pairs - 1) / pairs < sms) pairs >>= 1;
-  while (pairs > 1 && P.table_bytes + pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
-  const size_t smem = static_cast<size_t>(P.table_bytes) + static_cast<size_t>(pairs) * P.pair_bytes;
+  while (pairs > 1 && P.table_bytes + P.bias_bytes + pairs * P.pair_bytes > 100 * 1024) pairs >>= 1;
+  const size_t smem = static_cast<size_t>(P.table_bytes) + P.bias_bytes +
+                      static_cast<size_t>(pairs) * P.pair_bytes;
   cudaError_t err =
       cudaFuncSetAttribute(k_select<NPL, W, WK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int64_t grid = (D.L + pairs - 1) / pairs;
+  int per_sm = 1;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_select<NPL, W, WK>, 64 * pairs,
+                                                      smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = (D.L + pairs - 1) / pairs;
+  if (grid > static_cast<int64_t>(sms) * per_sm) grid = static_cast<int64_t>(sms) * per_sm;
   k_select<NPL, W, WK><<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
       Z, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
       static_cast<int>(D.K), br, bc, idx, gate, score, P);
