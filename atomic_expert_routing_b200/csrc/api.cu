@@ -25,7 +25,8 @@ int check_dims(const omni_dims* in, Dims* D) {
   if (D->k > D->Nr || D->k > D->Nc || D->K > D->k * D->k) return OMNI_ERR_INVALID_ARG;
   if (D->Nr > OMNI_MAX_AXIS || D->Nc > OMNI_MAX_AXIS) return OMNI_ERR_UNSUPPORTED;
   if (D->k > OMNI_MAX_TOPK || D->K > OMNI_MAX_TOPK) return OMNI_ERR_UNSUPPORTED;
-  if (D->N() >= (int64_t(1) << 31) || D->M() >= (int64_t(1) << 31)) return OMNI_ERR_UNSUPPORTED;
+  // task counts travel in 30-bit fields of the scheduler's look-back words
+  if (D->N() >= (int64_t(1) << 31) || D->M() >= (int64_t(1) << 30)) return OMNI_ERR_UNSUPPORTED;
   if (D->d % 8 != 0 || D->d > (int64_t(1) << 16)) return OMNI_ERR_UNSUPPORTED;
   return OMNI_OK;
 }

@@ -15,8 +15,10 @@
 //             rank in U (sorted unique ids), U itself, |U| and the group
 //             count ceil(|U| / B);
 //  3. sort    stable LSD radix sort of the tasks by group = rank / B with
-//             8-bit digits (as many passes as the group-count bound needs);
-//             stability keeps (token, expert) order inside each group;
+//             8-bit digits (as many passes as the group-count bound needs),
+//             one kernel per pass (decoupled look-back over tiles) after one
+//             histogram kernel for all passes; stability keeps (token,
+//             expert) order inside each group;
 //  4. emit    gather the sorted tasks and mark each group's first task.
 #include "blocksort.cuh"
 #include "common.cuh"
@@ -154,84 +156,61 @@ struct KeySrc {
   }
 };
 
+// One-kernel radix pass (decoupled look-back).  A global histogram of every
+// pass's digits is taken once up front; then each pass is one kernel whose
+// CTAs take tiles in start order (an atomic tile counter), rank their keys
+// stably per warp, publish their per-digit counts, and find the counts of
+// all earlier tiles by walking back through the published words: a word
+// holds a 2-bit state (0 none, 1 this tile's count, 2 count of all tiles up
+// to and including this one) and a 30-bit count.  A tile only waits on tiles
+// that started before it; every wait is bounded (OMNI_DEV_TIMEOUT).
+constexpr uint32_t kLbAgg = 1u << 30, kLbIncl = 2u << 30, kLbCount = (1u << 30) - 1;
+
 __global__ void __launch_bounds__(kRsThreads)
-    k_rs_hist(KeySrc src, int64_t M, int shift, int ntiles, uint32_t* __restrict__ hist) {
-  __shared__ uint32_t h[256];
-  h[threadIdx.x] = 0;
+    k_rs_ghist(KeySrc src, int64_t M, int passes, uint32_t* __restrict__ dgh) {
+  __shared__ uint32_t h[4][256];
+  for (int j = threadIdx.x; j < 4 * 256; j += kRsThreads) (&h[0][0])[j] = 0u;
   __syncthreads();
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRsTile;
   for (int j = threadIdx.x; j < kRsTile; j += kRsThreads) {
     const int64_t i = t0 + j;
-    if (i < M) atomicAdd(&h[(src(i) >> shift) & 255u], 1u);
+    if (i < M) {
+      const uint32_t key = src(i);
+      for (int p = 0; p < passes; ++p) atomicAdd(&h[p][(key >> (8 * p)) & 255u], 1u);
+    }
   }
   __syncthreads();
-  hist[static_cast<int64_t>(threadIdx.x) * ntiles + blockIdx.x] = h[threadIdx.x];
-}
-
-// Device-wide exclusive scan of n words in place (digit-major radix table):
-// per-tile sums, one block scanning the tile sums, then each tile finishes.
-__global__ void __launch_bounds__(kScanThreads)
-    k_gscan_reduce(const uint32_t* __restrict__ v, int64_t n, int32_t* __restrict__ tile_sum) {
-  __shared__ int warp_tot[32];
-  __shared__ int total;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
-  int acc = 0;
-#pragma unroll
-  for (int j = 0; j < kScanItems; ++j)
-    if (base + j < n) acc += static_cast<int>(v[base + j]);
-  block_exclusive_scan(acc, warp_tot, &total);
-  if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
-}
-
-__global__ void __launch_bounds__(kScanThreads)
-    k_gscan_tiles(int32_t* __restrict__ tile_sum, int ntiles) {
-  __shared__ int warp_tot[32];
-  __shared__ int total;
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int c0 = 0; c0 < ntiles; c0 += kScanThreads) {
-    const int i = c0 + threadIdx.x;
-    const int v = i < ntiles ? tile_sum[i] : 0;
-    const int ex = block_exclusive_scan(v, warp_tot, &total);
-    if (i < ntiles) tile_sum[i] = carry + ex;
-    __syncthreads();
-    if (threadIdx.x == 0) carry += total;
-    __syncthreads();
+  for (int p = 0; p < passes; ++p) {
+    const uint32_t c = h[p][threadIdx.x];
+    if (c) atomicAdd(&dgh[p * 256 + threadIdx.x], c);
   }
 }
 
-__global__ void __launch_bounds__(kScanThreads)
-    k_gscan_finish(uint32_t* __restrict__ v, int64_t n, const int32_t* __restrict__ tile_off) {
-  __shared__ int warp_tot[32];
-  __shared__ int total;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
-  uint32_t f[kScanItems];
-  int acc = 0;
-#pragma unroll
-  for (int j = 0; j < kScanItems; ++j) {
-    f[j] = (base + j < n) ? v[base + j] : 0u;
-    acc += static_cast<int>(f[j]);
-  }
-  int r = block_exclusive_scan(acc, warp_tot, &total) + tile_off[blockIdx.x];
-#pragma unroll
-  for (int j = 0; j < kScanItems; ++j) {
-    if (base + j < n) v[base + j] = static_cast<uint32_t>(r);
-    r += static_cast<int>(f[j]);
-  }
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __global__ void __launch_bounds__(kRsThreads)
-    k_rs_scatter(KeySrc src, const uint32_t* __restrict__ vals_in, int64_t M, int shift,
-                 int ntiles, const uint32_t* __restrict__ hist, uint32_t* __restrict__ keys_out,
-                 uint32_t* __restrict__ vals_out) {
+    k_rs_onesweep(KeySrc src, const uint32_t* __restrict__ vals_in, int64_t M, int shift,
+                  const uint32_t* __restrict__ dgh, uint32_t* __restrict__ look,
+                  uint32_t* __restrict__ tile_ctr, uint32_t* __restrict__ keys_out,
+                  uint32_t* __restrict__ vals_out, int32_t* status) {
   __shared__ uint32_t wcount[kRsWarps][256];
-  __shared__ uint32_t dbase[256];
+  __shared__ uint32_t tbase[256];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int64_t tile_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int j = threadIdx.x; j < kRsWarps * 256; j += kRsThreads) (&wcount[0][0])[j] = 0;
-  dbase[threadIdx.x] = hist[static_cast<int64_t>(threadIdx.x) * ntiles + blockIdx.x];
+  if (threadIdx.x == 0) tile_s = atomicAdd(tile_ctr, 1u);
   __syncthreads();
-  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kRsTile + warp * kRsPerWarp;
+  const int64_t tile = tile_s;
+  const int64_t w0 = tile * kRsTile + warp * kRsPerWarp;
   constexpr int R = kRsPerWarp / 32;
   uint32_t key[R], rnk[R];
   // per-warp stable ranks, in element order
@@ -253,25 +232,53 @@ __global__ void __launch_bounds__(kRsThreads)
     __syncwarp();
   }
   __syncthreads();
-  // exclusive prefix of the per-warp counts, per digit
-  {
-    const int dgt = threadIdx.x;
-    uint32_t run = 0;
-    for (int w = 0; w < kRsWarps; ++w) {
-      const uint32_t c = wcount[w][dgt];
-      wcount[w][dgt] = run;
-      run += c;
-    }
+  const int d = threadIdx.x;  // one digit per thread
+  uint32_t local = 0;
+  for (int w = 0; w < kRsWarps; ++w) {
+    const uint32_t c = wcount[w][d];
+    wcount[w][d] = local;
+    local += c;
   }
+  uint32_t* mine = look + tile * 256 + d;
+  uint32_t excl = 0;
+  if (tile == 0) {
+    st_relaxed(mine, kLbIncl | local);
+  } else {
+    st_relaxed(mine, kLbAgg | local);
+    const uint64_t t0 = global_ns();
+    for (int64_t pt = tile - 1; pt >= 0;) {
+      const uint32_t v = ld_relaxed(look + pt * 256 + d);
+      const uint32_t state = v & ~kLbCount;
+      if (state == 0u) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          raise_status(status, OMNI_DEV_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+        continue;
+      }
+      excl += v & kLbCount;
+      if (state == kLbIncl) break;
+      --pt;
+    }
+    st_relaxed(mine, kLbIncl | (excl + local));
+  }
+  // global base of each digit: exclusive scan of the histogram
+  const int gex = block_exclusive_scan(static_cast<int>(dgh[d]), warp_tot, &total);
+  tbase[d] = static_cast<uint32_t>(gex) + excl;
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int64_t i = w0 + r * 32 + lane;
     if (i < M) {
       const uint32_t dig = (key[r] >> shift) & 255u;
-      const uint32_t pos = dbase[dig] + wcount[warp][dig] + rnk[r];
-      keys_out[pos] = key[r];
-      vals_out[pos] = vals_in ? vals_in[i] : static_cast<uint32_t>(i);
+      const uint32_t pos = tbase[dig] + wcount[warp][dig] + rnk[r];
+      if (pos < static_cast<uint64_t>(M)) {
+        keys_out[pos] = key[r];
+        vals_out[pos] = vals_in ? vals_in[i] : static_cast<uint32_t>(i);
+      } else {
+        raise_status(status, OMNI_DEV_TIMEOUT);  // only after a timed-out wait
+      }
     }
   }
 }
@@ -405,9 +412,10 @@ __global__ void __launch_bounds__(kSmallThreads)
 struct SchedWs {
   int32_t *flags, *rank, *tile_sum, *tmp_e;
   float* tmp_g;
-  uint32_t *ka, *va, *kb, *vb, *hist, *bits;
-  int32_t *hist_tiles, *wpre;
-  int64_t nscan, ntiles, nhscan;
+  uint32_t *ka, *va, *kb, *vb, *sweep;  // sweep: [passes][256] histogram, [passes] tile
+                                        // counters, [passes][ntiles][256] look-back words
+  size_t sweep_words;
+  int64_t nscan, ntiles;
   int passes;
 };
 
@@ -434,9 +442,8 @@ SchedWs carve(const Dims& D, void* base, size_t* bytes) {
     w.va = c.take<uint32_t>(M);
     w.kb = c.take<uint32_t>(M);
     w.vb = c.take<uint32_t>(M);
-    w.hist = c.take<uint32_t>(256 * w.ntiles);
-    w.nhscan = (256 * w.ntiles + kScanTile - 1) / kScanTile;
-    w.hist_tiles = c.take<int32_t>(w.nhscan + 1);
+    w.sweep_words = static_cast<size_t>(w.passes) * (256 + 1 + 256 * w.ntiles);
+    w.sweep = c.take<uint32_t>(w.sweep_words);
   }
   if (bytes) *bytes = c.off;
   return w;
@@ -498,22 +505,26 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
   const uint32_t* keys = nullptr;
   const uint32_t* vals = nullptr;
   uint32_t *ko = w.ka, *vo = w.va;
-  for (int p = 0; p < w.passes; ++p) {
-    KeySrc src{keys, w.tmp_e, w.rank, D.B};
-    k_rs_hist<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(src, M, 8 * p,
-                                                                      static_cast<int>(w.ntiles),
-                                                                      w.hist);
-    k_gscan_reduce<<<static_cast<unsigned>(w.nhscan), kScanThreads, 0, s>>>(
-        w.hist, 256 * w.ntiles, w.hist_tiles);
-    k_gscan_tiles<<<1, kScanThreads, 0, s>>>(w.hist_tiles, static_cast<int>(w.nhscan));
-    k_gscan_finish<<<static_cast<unsigned>(w.nhscan), kScanThreads, 0, s>>>(
-        w.hist, 256 * w.ntiles, w.hist_tiles);
-    k_rs_scatter<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(
-        src, vals, M, 8 * p, static_cast<int>(w.ntiles), w.hist, ko, vo);
-    keys = ko;
-    vals = vo;
-    ko = (ko == w.ka) ? w.kb : w.ka;
-    vo = (vo == w.va) ? w.vb : w.va;
+  if (w.passes > 0) {
+    uint32_t* dgh = w.sweep;
+    uint32_t* ctr = dgh + 256 * w.passes;
+    uint32_t* look = ctr + w.passes;
+    err = cudaMemsetAsync(w.sweep, 0, w.sweep_words * sizeof(uint32_t), s);
+    if (err != cudaSuccess) return err;
+    KeySrc src0{nullptr, w.tmp_e, w.rank, D.B};
+    k_rs_ghist<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(src0, M, w.passes, dgh);
+    for (int p = 0; p < w.passes; ++p) {
+      KeySrc src{keys, w.tmp_e, w.rank, D.B};
+      k_rs_onesweep<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(
+          src, vals, M, 8 * p, dgh + 256 * p, look + static_cast<size_t>(p) * 256 * w.ntiles,
+          ctr + p, ko, vo, status);
+      keys = ko;
+      vals = vo;
+      ko = (ko == w.ka) ? w.kb : w.ka;
+      vo = (vo == w.va) ? w.vb : w.va;
+    }
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
   }
   k_emit<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(
       keys, vals, M, static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate,

@@ -79,7 +79,7 @@ extern "C" {
 #define OMNI_MAX_TOPK 256       /* k, K */
 
 typedef struct omni_dims {
-  int64_t L;     /* tokens in the batch (>= 0) */
+  int64_t L;     /* tokens in the batch (>= 0; L*K < 2^30 tasks) */
   int64_t d;     /* model width (multiple of 8; of 4 for OMNI_F32) */
   int64_t Nr;    /* grid rows */
   int64_t Nc;    /* grid columns; N = Nr*Nc atomic experts (< 2^31) */
