@@ -383,6 +383,43 @@ def run_ours(args):
                 tot[i] += evs[i].elapsed_time(evs[i + 1])
         return {"route": tot[0] / steps, "schedule": tot[1] / steps, "expert": tot[2] / steps}
 
+    def measure_ablation(c, dd, steps):
+        """The pages' comparison on the same routing: expert-centric execution
+        (schedule + grouped execution) against token-centric execution, each
+        pass timed with events after an L2 flush."""
+        D = omni.LayerDims.of(c)
+        stream = torch.cuda.current_stream(device)
+        idx, gate, _ = omni.route(D, dd["x"], dd["Wr"], dd["Wc"], dd["bias_r"], dd["bias_c"],
+                                  with_score=False)
+        wsd, we = omni.Workspace(), omni.Workspace()
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        counts = omni.new_counts(device)
+
+        def ec():
+            s = omni.schedule(D, idx, gate, ws=wsd, counts=counts)
+            omni.expert_forward(D, dd["x"], dd["W"], dd["V"], s, y=y, ws=we)
+
+        def tc_():
+            omni.token_centric_forward(D, dd["x"], dd["W"], dd["V"], idx, gate, y=y,
+                                       counts=counts)
+
+        out = {}
+        for name, fn in (("expert_centric_ms", ec), ("token_centric_ms", tc_)):
+            fn()
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(steps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                tot += a.elapsed_time(b)
+            out[name] = tot / steps
+        out["token_over_expert"] = out["token_centric_ms"] / out["expert_centric_ms"]
+        return out
+
     def measure_e2e(c, dd, steps, warmup):
         """The public call with host buffers: pinned x -> device, forward, y -> pinned host."""
         D = omni.LayerDims.of(c)
@@ -425,21 +462,37 @@ def run_ours(args):
     st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
     stages = measure_stages(cfg, d, max(3, args.steps // 2))
 
+    ablation = measure_ablation(cfg, d, max(3, args.steps // 2))
+
+    def summary(sc, dd, steps, warmup, with_stages):
+        ms2, na2, st2, _, _, _ = measure(sc, dd, steps, warmup)
+        ms2 = max_over_ranks(ms2, world, device)
+        f2, b2 = layer_work(sc, na2)
+        rec = {"value": job_throughput(world, sc.L, ms2), "unit": "tokens/s", "ms_per_step": ms2,
+               "n_active": na2, "device_status": st2,
+               "layer_roofline": {"bound": "hbm" if b2 / (hbm * 1e9) > f2 / (tc * 1e12) else "tensor",
+                                  "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
+                                  "bytes": b2, "flops": f2}}
+        if with_stages:
+            rec["stages_ms"] = measure_stages(sc, dd, 10)
+            rec["ablation"] = measure_ablation(sc, dd, 10)
+        return rec
+
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
-        ms2, na2, st2, _, _, _ = measure(sc, d2, max(args.steps, 20), max(args.warmup, 5))
-        stages2 = measure_stages(sc, d2, 10)
-        ms2 = max_over_ranks(ms2, world, device)
-        f2, b2 = layer_work(sc, na2)
-        extra[sc.name] = {
-            "value": job_throughput(world, sc.L, ms2), "unit": "tokens/s", "ms_per_step": ms2,
-            "n_active": na2, "device_status": st2, "stages_ms": stages2,
-            "layer_roofline": {"bound": "hbm" if b2 / (hbm * 1e9) > f2 / (tc * 1e12) else "tensor",
-                               "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
-                               "bytes": b2, "flops": f2}}
+        extra[sc.name] = summary(sc, d2, max(args.steps, 20), max(args.warmup, 5), True)
+        del d2
+        # the other workloads (parity configurations), each with its own weights
+        for sc in (WL.TINY, WL.BF16_16K, WL.SKEWED):
+            hs = rank_inputs(sc, rank)
+            hs.update(WL.make_experts(sc))
+            ds = {k: to_dev(v) for k, v in hs.items()}
+            extra[sc.name] = summary(sc, ds, max(args.steps, 10), max(args.warmup, 3), False)
+            del ds, hs
+            torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:
@@ -477,6 +530,7 @@ def run_ours(args):
         "n_active": n_active,
         "device_status": status,
         "stages_ms": stages,
+        "ablation": ablation,
         "layer_roofline": {"bound": "hbm" if t_b >= t_f else "tensor",
                            "frac": max(t_f, t_b) / (ms_all * 1e-3), "bytes": bytes_,
                            "flops": flops, "peak_src": peak_src},
