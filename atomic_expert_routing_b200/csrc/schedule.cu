@@ -20,9 +20,13 @@
 //             histogram kernel for all passes; stability keeps (token,
 //             expert) order inside each group;
 //  4. emit    gather the sorted tasks and mark each group's first task.
+#include <cooperative_groups.h>
+
 #include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace omni {
 namespace {
@@ -301,112 +305,204 @@ __global__ void __launch_bounds__(256)
   if (i == M - 1) group_off[counts[1]] = static_cast<int32_t>(M);
 }
 
-// ---- small batches (M <= kSmallMax): the whole schedule in one CTA ----------
+// ---- small batches (M <= kSmallMax): the whole schedule in one cluster -------
+//
+// Eight CTAs of one thread-block cluster each own a contiguous eighth of the
+// tasks in shared memory.  Every stable LSD radix pass (8-bit digits) ranks
+// each CTA's keys per warp in element order, exchanges the per-CTA digit
+// totals through distributed shared memory, and scatters every key straight
+// into the shared memory of the CTA that owns its new position.  (1) Sort by
+// expert id; the "new id" flags, counted across the cluster, give U and the
+// rank of each task's expert.  (2) Stable sort of the expert-ordered tasks
+// by group * L + token: equal keys keep their expert order, so the tasks end
+// up ordered by (group, token, expert).  (3) Emit.  Every CTA takes the same
+// sequence of cluster barriers; none waits on a flag.
 constexpr int kSmallMax = kBlockSortMax;
-constexpr int kSmallThreads = kBlockSortThreads;
-constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallRounds = kSmallMax / kSmallThreads;  // rounds of 32 keys per warp
+constexpr int kClCtas = 8;
+constexpr int kClThreads = 512;
+constexpr int kClWarps = kClThreads / 32;
+constexpr int kClChunk = kSmallMax / kClCtas;      // keys per CTA at most
+constexpr int kClRounds = kClChunk / kClThreads;   // 32-key rounds per warp at most
 
-// Same outputs as the multi-kernel path.  (1) Radix-sort the tasks' expert
-// ids; a scan of the "new id" flags gives U and the rank of every task's
-// expert.  (2) Stable radix sort of the expert-ordered tasks by group * L +
-// token: equal keys keep their expert order, so the tasks end up ordered by
-// (group, token, expert).  (3) Emit.
-__global__ void __launch_bounds__(kSmallThreads)
-    k_sched_small(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L,
-                  int K, int64_t N, int64_t B, int epasses, int kpasses,
-                  int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
-                  float* __restrict__ task_gate, int32_t* __restrict__ uniq,
-                  int32_t* __restrict__ group_off, int32_t* counts) {
-  extern __shared__ uint32_t sm[];
-  uint32_t* keyA = sm;
-  uint32_t* keyB = keyA + kSmallMax;
-  uint16_t* valA = reinterpret_cast<uint16_t*>(keyB + kSmallMax);
-  uint16_t* valB = valA + kSmallMax;
-  uint16_t* rk = valB + kSmallMax;  // rank of each task's expert
-  uint32_t* wcount = reinterpret_cast<uint32_t*>(rk + kSmallMax);  // [kSmallWarps][256]
-  __shared__ int warp_tot[32];
-  __shared__ int total;
-  __shared__ uint32_t dbase[256];
+struct ClSmem {
+  uint32_t key[2][kClChunk];
+  uint16_t val[2][kClChunk];
+  uint32_t wcnt[kClWarps][256];
+  uint32_t tot[256];    // this CTA's digit totals, read by the other CTAs
+  uint32_t base[256];
+  int warp_tot[32];
+  int total;
+  int news;             // "new id" flags in this CTA, read by the other CTAs
+};
+
+// One stable radix pass over the cluster: keys move from buffer `in` to
+// buffer in ^ 1 (of whichever CTA owns their new position).
+__device__ void cl_radix_pass(cg::cluster_group& cl, ClSmem& S, int in, int n_local, int chunk,
+                              int shift) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = static_cast<int>(cl.block_rank());
+  const int rounds = (n_local + kClThreads - 1) / kClThreads;
+  for (int j = tid; j < kClWarps * 256; j += kClThreads) (&S.wcnt[0][0])[j] = 0u;
+  __syncthreads();
+  uint32_t dig[kClRounds], rnk[kClRounds];
+#pragma unroll
+  for (int r = 0; r < kClRounds; ++r) {
+    dig[r] = 0xffffffffu;
+    rnk[r] = 0u;
+    if (r < rounds) {  // block-uniform
+      const int j = (warp * rounds + r) * 32 + lane;
+      const bool valid = j < n_local;
+      dig[r] = valid ? ((S.key[in][j] >> shift) & 255u) : 0xffffffffu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dig[r]);
+      const int leader = __ffs(peers) - 1;
+      uint32_t old = 0;
+      if (valid && lane == leader) {
+        old = S.wcnt[warp][dig[r]];
+        S.wcnt[warp][dig[r]] = old + __popc(peers);
+      }
+      old = __shfl_sync(0xffffffffu, old, leader);
+      rnk[r] = old + __popc(peers & lanemask_lt());
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (tid < 256) {
+    uint32_t run = 0;
+    for (int w = 0; w < kClWarps; ++w) {
+      const uint32_t c = S.wcnt[w][tid];
+      S.wcnt[w][tid] = run;
+      run += c;
+    }
+    S.tot[tid] = run;
+  }
+  cl.sync();  // every CTA's digit totals are visible
+  int all = 0;
+  if (tid < 256) {
+    uint32_t before = 0, sum = 0;
+    for (int c = 0; c < kClCtas; ++c) {
+      const uint32_t v = cl.map_shared_rank(S.tot, c)[tid];
+      sum += v;
+      if (c < rank) before += v;
+    }
+    S.base[tid] = before;
+    all = static_cast<int>(sum);
+  }
+  const int ex = block_exclusive_scan(all, S.warp_tot, &S.total);
+  if (tid < 256) S.base[tid] += static_cast<uint32_t>(ex);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kClRounds; ++r) {
+    if (r < rounds) {
+      const int j = (warp * rounds + r) * 32 + lane;
+      if (j < n_local) {
+        const uint32_t pos = S.base[dig[r]] + S.wcnt[warp][dig[r]] + rnk[r];
+        const int dst = static_cast<int>(pos / static_cast<uint32_t>(chunk));
+        const int off = static_cast<int>(pos - static_cast<uint32_t>(dst) * chunk);
+        cl.map_shared_rank(&S.key[in ^ 1][0], dst)[off] = S.key[in][j];
+        cl.map_shared_rank(&S.val[in ^ 1][0], dst)[off] = S.val[in][j];
+      }
+    }
+  }
+  cl.sync();  // every key has landed in its new owner's buffer
+}
+
+__global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads)
+    k_sched_cluster(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L,
+                    int K, int64_t N, int64_t B, int epasses, int kpasses,
+                    int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
+                    float* __restrict__ task_gate, int32_t* __restrict__ uniq,
+                    int32_t* __restrict__ group_off, int32_t* counts) {
+  __shared__ ClSmem S;
+  cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x;
+  const int rank = static_cast<int>(cl.block_rank());
   const int M = static_cast<int>(L * K);
+  const int chunk = (M + kClCtas - 1) / kClCtas;
+  const int first = rank * chunk;
+  const int n_local = M - first < 0 ? 0 : (M - first < chunk ? M - first : chunk);
   int32_t* status = counts + 2;
-  // (1) sort by expert id
-  for (int i = tid; i < M; i += kSmallThreads) {
-    int64_t e = idx[i];
+  // (1) load this CTA's tasks: key = expert id, value = task index
+  for (int j = tid; j < n_local; j += kClThreads) {
+    int64_t e = idx[first + j];
     if (e < 0 || e >= N) {
       raise_status(status, OMNI_DEV_BAD_INDEX);
       e = 0;
     }
-    keyA[i] = static_cast<uint32_t>(e);
-    valA[i] = static_cast<uint16_t>(i);
+    S.key[0][j] = static_cast<uint32_t>(e);
+    S.val[0][j] = static_cast<uint16_t>(first + j);
   }
   __syncthreads();
-  uint32_t *kin = keyA, *kout = keyB;
-  uint16_t *vin = valA, *vout = valB;
+  int cur = 0;
   for (int p = 0; p < epasses; ++p) {
-    block_radix_pass(kin, vin, kout, vout, M, 8 * p, wcount, dbase, warp_tot, &total);
-    uint32_t* tk = kin; kin = kout; kout = tk;
-    uint16_t* tv = vin; vin = vout; vout = tv;
+    cl_radix_pass(cl, S, cur, n_local, chunk, 8 * p);
+    cur ^= 1;
   }
-  // ranks: each thread takes kSmallRounds consecutive sorted positions
-  const int b0 = tid * kSmallRounds;
+  // ranks: thread tid takes elements 2*tid, 2*tid + 1 of this CTA (position order)
+  const uint32_t prev_last =
+      (rank > 0 && n_local > 0) ? cl.map_shared_rank(&S.key[cur][0], rank - 1)[chunk - 1] : 0u;
   int nnew = 0;
+  bool isnew[kClChunk / kClThreads];
 #pragma unroll
-  for (int j = 0; j < kSmallRounds; ++j) {
-    const int q = b0 + j;
-    if (q < M && (q == 0 || kin[q] != kin[q - 1])) ++nnew;
-  }
-  int r = block_exclusive_scan(nnew, warp_tot, &total) - 1;
-  const int n_active = total;
-#pragma unroll
-  for (int j = 0; j < kSmallRounds; ++j) {
-    const int q = b0 + j;
-    if (q < M) {
-      if (q == 0 || kin[q] != kin[q - 1]) {
-        ++r;
-        uniq[r] = static_cast<int32_t>(kin[q]);
-      }
-      rk[vin[q]] = static_cast<uint16_t>(r);
+  for (int q = 0; q < kClChunk / kClThreads; ++q) {
+    const int j = tid * (kClChunk / kClThreads) + q;
+    isnew[q] = false;
+    if (j < n_local) {
+      const uint32_t prev = j > 0 ? S.key[cur][j - 1] : prev_last;
+      isnew[q] = (first + j == 0) || S.key[cur][j] != prev;
+      nnew += isnew[q];
     }
   }
+  const int ex = block_exclusive_scan(nnew, S.warp_tot, &S.total);
+  if (tid == 0) S.news = S.total;
+  cl.sync();
+  int before = 0, n_active = 0;
+  for (int c = 0; c < kClCtas; ++c) {
+    const int v = *cl.map_shared_rank(&S.news, c);
+    n_active += v;
+    if (c < rank) before += v;
+  }
   const int64_t G = (n_active + B - 1) / B;
-  if (tid == 0) {
+  if (rank == 0 && tid == 0) {
     counts[0] = n_active;
     counts[1] = static_cast<int32_t>(G);
   }
-  __syncthreads();
-  // (2) key g * L + t over the expert-sorted tasks; the stable passes keep
-  // expert order among equal keys, so the result is ordered by (g, t, e)
-  for (int q = tid; q < M; q += kSmallThreads) {
-    const int i = vin[q];
-    const uint32_t g = static_cast<uint32_t>(rk[i] / static_cast<uint64_t>(B));
-    kout[q] = g * static_cast<uint32_t>(L) + static_cast<uint32_t>(i / K);
-    vout[q] = static_cast<uint16_t>(i);
+  // (2) key g * L + t in place of the expert id (same positions, same CTA)
+  int r = before + ex - 1;
+#pragma unroll
+  for (int q = 0; q < kClChunk / kClThreads; ++q) {
+    const int j = tid * (kClChunk / kClThreads) + q;
+    if (j < n_local) {
+      if (isnew[q]) {
+        ++r;
+        uniq[r] = static_cast<int32_t>(S.key[cur][j]);
+      }
+      const uint32_t i = S.val[cur][j];
+      const uint32_t g = static_cast<uint32_t>(r / B);
+      S.key[cur][j] = g * static_cast<uint32_t>(L) + i / static_cast<uint32_t>(K);
+    }
   }
-  __syncthreads();
-  {
-    uint32_t* tk = kin; kin = kout; kout = tk;
-    uint16_t* tv = vin; vin = vout; vout = tv;
-  }
+  cl.sync();  // no CTA still reads a neighbour's last expert id
   for (int p = 0; p < kpasses; ++p) {
-    block_radix_pass(kin, vin, kout, vout, M, 8 * p, wcount, dbase, warp_tot, &total);
-    uint32_t* tk = kin; kin = kout; kout = tk;
-    uint16_t* tv = vin; vin = vout; vout = tv;
+    cl_radix_pass(cl, S, cur, n_local, chunk, 8 * p);
+    cur ^= 1;
   }
   // (3) emit
-  const uint32_t per_group = static_cast<uint32_t>(L);
-  for (int p = tid; p < M; p += kSmallThreads) {
-    const int i = vin[p];
-    const uint32_t g = kin[p] / per_group;
+  const uint32_t prev_key =
+      (rank > 0 && n_local > 0) ? cl.map_shared_rank(&S.key[cur][0], rank - 1)[chunk - 1] : 0u;
+  for (int j = tid; j < n_local; j += kClThreads) {
+    const int p = first + j;
+    const int i = S.val[cur][j];
+    const uint32_t g = S.key[cur][j] / static_cast<uint32_t>(L);
     task_token[p] = i / K;
     int32_t e = idx[i];
     if (e < 0 || e >= N) e = 0;
     task_expert[p] = e;
     task_gate[p] = gate[i];
-    if (p == 0 || kin[p - 1] / per_group != g) group_off[g] = p;
+    const uint32_t pk = j > 0 ? S.key[cur][j - 1] : prev_key;
+    if (p == 0 || pk / static_cast<uint32_t>(L) != g) group_off[g] = p;
     if (p == M - 1) group_off[G] = M;
   }
+  cl.sync();  // keep this CTA's shared memory alive until its neighbour has read it
 }
 
 struct SchedWs {
@@ -478,14 +574,9 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     // key g * L + t < gmax * L
     const int kpasses =
         (nbits(static_cast<uint64_t>(D.gmax()) * static_cast<uint64_t>(D.L)) + 7) / 8;
-    const size_t smem = static_cast<size_t>(kSmallMax) * (2 * sizeof(uint32_t) + 3 * sizeof(uint16_t)) +
-                        static_cast<size_t>(kSmallWarps) * 256 * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(k_sched_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    k_sched_small<<<1, kSmallThreads, smem, s>>>(idx, gate, D.L, static_cast<int>(D.K), N, D.B,
-                                                  epasses, kpasses, task_token, task_expert,
-                                                  task_gate, uniq, group_off, counts);
+    k_sched_cluster<<<kClCtas, kClThreads, 0, s>>>(idx, gate, D.L, static_cast<int>(D.K), N, D.B,
+                                                   epasses, kpasses, task_token, task_expert,
+                                                   task_gate, uniq, group_off, counts);
     return cudaGetLastError();
   }
   SchedWs w = carve(D, ws, nullptr);
