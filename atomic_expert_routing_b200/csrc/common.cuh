@@ -17,6 +17,19 @@ __device__ __forceinline__ void raise_status(int32_t* status, int bits) {
 }
 
 // Wall-clock bound for every device-side wait (nanoseconds of %globaltimer).
+// Programmatic dependent launch: every kernel of the library is launched
+// with programmatic stream serialisation.  pdl_wait() returns once the
+// previous kernel on the stream has completed and its memory is visible;
+// pdl_trigger() lets the next kernel be scheduled while this one runs (its
+// CTAs then wait in pdl_wait()).  Both are no-ops without a programmatic
+// dependency.  Short kernels trigger at their start; the long throughput
+// kernels (activations, accumulation sweeps, the persistent selection) do
+// not, since the waiting CTAs of their successors slowed them down.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
 __device__ __forceinline__ uint64_t global_ns() {

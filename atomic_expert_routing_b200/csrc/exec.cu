@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
                     const int32_t* __restrict__ task_expert,
                     const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
                     int S, float* __restrict__ yacc, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int EPV = kEpv<T>;
   const int lane = threadIdx.x & 31;
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -272,6 +274,8 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
                    const int32_t* __restrict__ task_expert,
                    const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
                    int S, int64_t nslices, float* __restrict__ yacc, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int EPV = kEpv<T>;
   constexpr int SLOT = 2 * NV * 32;  // uint4 per ring slot: W vectors, then V vectors
   extern __shared__ __align__(16) uint4 ring[];
@@ -410,6 +414,7 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
           const T* __restrict__ F, const int32_t* __restrict__ fidx, int64_t nf,
           const float* __restrict__ task_gate, const int32_t* __restrict__ dst, int64_t M, int d,
           int S, int64_t nslices, float* __restrict__ cbuf, int32_t* status) {
+  pdl_wait();
   constexpr int SLOT = NV * 32;  // uint4 per ring slot: one row of F
   extern __shared__ __align__(16) uint4 ring[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -522,6 +527,8 @@ __global__ void __launch_bounds__(kBlockSortThreads)
             const float* __restrict__ tg, const int32_t* __restrict__ group_off,
             const int32_t* __restrict__ counts, int64_t M, int64_t gmax, int T, int passes,
             WinOut o, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t wsm[];
   uint32_t* kA = reinterpret_cast<uint32_t*>(wsm);
   uint32_t* kB = kA + kBlockSortMax;
@@ -674,6 +681,7 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
     k_acc(const T* __restrict__ V, const int32_t* __restrict__ task_token,
           const int32_t* __restrict__ task_expert, const float* __restrict__ cbuf, int64_t M,
           int64_t L, int64_t N, int d, int col0, int64_t nslices, float* __restrict__ yacc) {
+  pdl_wait();
   static_assert(32 % D == 0, "the prefetch distance divides the slice");
   using QT = typename Quad<T>::type;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -768,6 +776,8 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
 // fp32 accumulator -> bf16 output (round to nearest even), 8 values per thread.
 __global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src,
                                               __nv_bfloat16* __restrict__ dst, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (i >= n) return;
   const float4 a = *reinterpret_cast<const float4*>(src + i);
@@ -786,6 +796,8 @@ __global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src,
 __global__ void __launch_bounds__(256)
     k_slice_finish(float* __restrict__ acc, __nv_bfloat16* __restrict__ y, int64_t L, int d,
                    int cast0, int zero0, int cols) {
+  pdl_wait();
+  pdl_trigger();
   const int per_row = cols / 8;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t row = i / per_row;
@@ -822,6 +834,8 @@ __global__ void __launch_bounds__(kTokThreads)
     k_token_centric(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
                     const int32_t* __restrict__ idx, const float* __restrict__ gate, int K, int d,
                     int64_t N, T* __restrict__ y, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int EPV = kEpv<T>;
   extern __shared__ __align__(16) uint8_t smem[];
   const int nvec = d / EPV;
@@ -938,9 +952,9 @@ cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const voi
   S = S < 1 ? 1 : (S > 32 ? 32 : S);
   const int64_t warps = (M + S - 1) / S;
   const int64_t blocks = (warps + kExpThreads / 32 - 1) / (kExpThreads / 32);
-  k_expert_slices<T, NV><<<static_cast<unsigned>(blocks), kExpThreads, 0, s>>>(
-      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
-      M, D.L, D.N(), static_cast<int>(D.d), S, acc, status);
+  OMNI_TRY(launch_k(k_expert_slices<T, NV>, static_cast<unsigned>(blocks), kExpThreads, 0, s,
+      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg, M,
+      D.L, D.N(), static_cast<int>(D.d), S, acc, status));
   return cudaGetLastError();
 }
 
@@ -963,9 +977,9 @@ cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void
   const int64_t nslices = (M + S - 1) / S;
   int64_t blocks = (nslices + kAsyncWarps - 1) / kAsyncWarps;
   if (blocks > sms) blocks = sms;  // persistent: one CTA per SM (shared-memory bound)
-  k_expert_async<T, NV, R><<<static_cast<unsigned>(blocks), kAsyncWarps * 32, smem, s>>>(
-      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg, M,
-      D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status);
+  OMNI_TRY(launch_k(k_expert_async<T, NV, R>, static_cast<unsigned>(blocks), kAsyncWarps * 32, smem,
+      s, static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
+      M, D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status));
   return cudaGetLastError();
 }
 
@@ -1006,8 +1020,8 @@ cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, co
   int bits = 0;
   while ((int64_t(1) << bits) < D.L) ++bits;
   const int passes = (bits + 7) / 8;
-  k_wsort<<<static_cast<unsigned>(nwin), kBlockSortThreads, smem, s>>>(
-      tt, te, tg, group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.win, status);
+  OMNI_TRY(launch_k(k_wsort, static_cast<unsigned>(nwin), kBlockSortThreads, smem, s, tt, te, tg,
+      group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.win, status));
   return cudaGetLastError();
 }
 
@@ -1024,9 +1038,9 @@ cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w
   int64_t blocks = (nslices + kAccWarps - 1) / kAccWarps;
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   if (blocks > cap) blocks = cap;
-  k_acc<T, NB, D><<<static_cast<unsigned>(blocks), kAccWarps * 32, 0, s>>>(
-      static_cast<const T*>(V), w.win.wt, w.win.we, w.cbuf, M, D_.L, D_.N(),
-      static_cast<int>(D_.d), col0, nslices, acc);
+  OMNI_TRY(launch_k(k_acc<T, NB, D>, static_cast<unsigned>(blocks), kAccWarps * 32, 0, s,
+      static_cast<const T*>(V), w.win.wt, w.win.we, w.cbuf, M, D_.L, D_.N(), static_cast<int>(D_.d),
+      col0, nslices, acc));
   return cudaGetLastError();
 }
 
@@ -1034,8 +1048,8 @@ cudaError_t launch_finish(const Dims& D, float* acc, __nv_bfloat16* y, int cast0
                           int cols, cudaStream_t s) {
   if (cast0 < 0 && zero0 < 0) return cudaSuccess;
   const int64_t threads = D.L * (cols / 8);
-  k_slice_finish<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-      acc, y, D.L, static_cast<int>(D.d), cast0, zero0, cols);
+  OMNI_TRY(launch_k(k_slice_finish, static_cast<unsigned>((threads + 255) / 256), 256, 0, s, acc, y,
+      D.L, static_cast<int>(D.d), cast0, zero0, cols));
   return cudaGetLastError();
 }
 
@@ -1060,9 +1074,9 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   if (blocks > 2 * sm_count()) blocks = 2 * sm_count();
   // tasks by expert: x[t] held per run of one token, the W rows through the
   // ring (an expert's repeated row comes from L2 right after its first read)
-  k_act<T, NV, R, true><<<static_cast<unsigned>(blocks), kActWarps * 32, smem, s>>>(
-      static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W), w.win.xe, D.N(),
-      w.win.xg, w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status);
+  OMNI_TRY(launch_k(k_act<T, NV, R, true>, static_cast<unsigned>(blocks), kActWarps * 32, smem, s,
+      static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W), w.win.xe, D.N(), w.win.xg,
+      w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status));
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int cols = static_cast<int>(D.d / Q);
@@ -1118,16 +1132,36 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                                               group_off, counts, w, acc, ycast, status, s);
   }
   const size_t ybytes = static_cast<size_t>(D.L) * D.d * sizeof(float);
-  cudaError_t err = cudaMemsetAsync(acc, 0, ybytes, s);
+  cudaError_t err = launch_zero(acc, ybytes / sizeof(float), s);
   if (err != cudaSuccess) return err;
   err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
             : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
                                              status, s);
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;
-  k_cast<<<static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s>>>(
-      acc, static_cast<__nv_bfloat16*>(y), n);
+  OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,
+      static_cast<__nv_bfloat16*>(y), n));
   return cudaGetLastError();
+}
+
+namespace {
+__global__ void __launch_bounds__(256) k_zero_words(uint32_t* __restrict__ p, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    *reinterpret_cast<uint4*>(p + i) = make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    for (int64_t j = i; j < n && j < i + 4; ++j) p[j] = 0u;
+  }
+}
+}  // namespace
+
+cudaError_t launch_zero(void* p, size_t n_words, cudaStream_t s) {
+  if (n_words == 0) return cudaSuccess;
+  const int64_t n = static_cast<int64_t>(n_words);
+  return launch_k(k_zero_words, static_cast<unsigned>((n / 4 + 256) / 256), 256, 0, s,
+                  static_cast<uint32_t*>(p), n);
 }
 
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
@@ -1143,18 +1177,18 @@ cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void
     err = cudaFuncSetAttribute(k_token_centric<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    k_token_centric<float><<<static_cast<unsigned>(D.L), kTokThreads, smem, s>>>(
+    OMNI_TRY(launch_k(k_token_centric<float>, static_cast<unsigned>(D.L), kTokThreads, smem, s,
         static_cast<const float*>(x), static_cast<const float*>(W), static_cast<const float*>(V),
         idx, gate, static_cast<int>(D.K), static_cast<int>(D.d), D.N(), static_cast<float*>(y),
-        status);
+        status));
   } else {
     err = cudaFuncSetAttribute(k_token_centric<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    k_token_centric<__nv_bfloat16><<<static_cast<unsigned>(D.L), kTokThreads, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W),
+    OMNI_TRY(launch_k(k_token_centric<__nv_bfloat16>, static_cast<unsigned>(D.L), kTokThreads, smem,
+        s, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W),
         static_cast<const __nv_bfloat16*>(V), idx, gate, static_cast<int>(D.K),
-        static_cast<int>(D.d), D.N(), static_cast<__nv_bfloat16*>(y), status);
+        static_cast<int>(D.d), D.N(), static_cast<__nv_bfloat16*>(y), status));
   }
   return cudaGetLastError();
 }

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace omni {
 
 struct Dims {
@@ -51,6 +53,35 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
                          cudaStream_t s);
+
+// Launch with programmatic stream serialisation (see pdl_wait/pdl_trigger):
+// the kernel may be scheduled while its predecessor on the stream finishes.
+// Arguments are converted to the kernel's parameter types.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Return the error of a CUDA call from the enclosing launch function.
+#define OMNI_TRY(expr)                              \
+  do {                                              \
+    const cudaError_t omni_try_e_ = (expr);         \
+    if (omni_try_e_ != cudaSuccess) return omni_try_e_; \
+  } while (0)
+
+// Zero n 32-bit words (a kernel, so that it joins the programmatic chain).
+cudaError_t launch_zero(void* p, size_t n_words, cudaStream_t s);
 
 // 256-byte aligned carving of a workspace (base == nullptr: size only)
 struct Carver {

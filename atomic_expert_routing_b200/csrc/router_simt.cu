@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(256) k_router_simt(const T* __restrict__ x,
                                                      const T* __restrict__ Wc,
                                                      float* __restrict__ Z, int64_t L, int Nr,
                                                      int Nc, int d, int tiles_r) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[TK][TM + 4];
   __shared__ float Bs[TK][TN + 4];
   const int tid = threadIdx.x;
@@ -77,15 +79,14 @@ cudaError_t launch_router_simt(const Dims& D, const void* x, const void* Wr, con
   const int tiles_c = static_cast<int>((D.Nc + TN - 1) / TN);
   dim3 grid(static_cast<unsigned>((D.L + TM - 1) / TM), tiles_r + tiles_c);
   if (D.dtype == OMNI_F32)
-    k_router_simt<float><<<grid, 256, 0, s>>>(
-        static_cast<const float*>(x), static_cast<const float*>(Wr),
-        static_cast<const float*>(Wc), Z, D.L, static_cast<int>(D.Nr),
-        static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r);
+    OMNI_TRY(launch_k(k_router_simt<float>, grid, 256, 0, s, static_cast<const float*>(x),
+        static_cast<const float*>(Wr), static_cast<const float*>(Wc), Z, D.L,
+        static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r));
   else
-    k_router_simt<__nv_bfloat16><<<grid, 256, 0, s>>>(
+    OMNI_TRY(launch_k(k_router_simt<__nv_bfloat16>, grid, 256, 0, s,
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
         static_cast<const __nv_bfloat16*>(Wc), Z, D.L, static_cast<int>(D.Nr),
-        static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r);
+        static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r));
   return cudaGetLastError();
 }
 

@@ -93,6 +93,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
                 const __grid_constant__ CUtensorMap tmBc, float* __restrict__ Z, int L, int Nr,
                 int Nc, int d, int tiles_r, int kper, int32_t* status) {
+  pdl_wait();
+  // let the selection launch early only for a single wave of tiles (small L):
+  // for many waves its waiting CTAs would sit beside the last tiles
+  if (gridDim.x * gridDim.y * gridDim.z <= 296u) pdl_trigger();
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
   constexpr uint32_t B_BYTES = BN * TC_BK * 2;
   extern __shared__ uint8_t smem_raw[];
@@ -261,9 +265,9 @@ cudaError_t launch_bn(const Dims& D, const CUtensorMap& a, const CUtensorMap& br
   const int ks = router_splits(D);
   const int kper = (nk + ks - 1) / ks;
   dim3 grid(static_cast<unsigned>(mt), tiles_r + tiles_c, ks);
-  k_router_tc<BN><<<grid, TC_THREADS, smem, s>>>(a, br, bc, Z, static_cast<int>(D.L),
-                                                 static_cast<int>(D.Nr), static_cast<int>(D.Nc),
-                                                 static_cast<int>(D.d), tiles_r, kper, status);
+  OMNI_TRY(launch_k(k_router_tc<BN>, grid, TC_THREADS, smem, s, a, br, bc, Z, static_cast<int>(D.L),
+      static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r, kper,
+      status));
   return cudaGetLastError();
 }
 
@@ -286,6 +290,8 @@ int router_splits(const Dims& D) {
 
 namespace {
 __global__ void __launch_bounds__(256) k_sum_partials(float* __restrict__ Z, int splits, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float acc = Z[i];
@@ -296,7 +302,8 @@ __global__ void __launch_bounds__(256) k_sum_partials(float* __restrict__ Z, int
 
 cudaError_t launch_sum_partials(float* Z, int splits, int64_t n, cudaStream_t s) {
   if (splits <= 1 || n == 0) return cudaSuccess;
-  k_sum_partials<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(Z, splits, n);
+  OMNI_TRY(launch_k(k_sum_partials, static_cast<unsigned>((n + 255) / 256), 256, 0, s, Z, splits,
+      n));
   return cudaGetLastError();
 }
 

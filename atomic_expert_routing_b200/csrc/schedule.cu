@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
     k_prep(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L, int K,
            int Kp, int64_t N, int32_t* __restrict__ flags, int32_t* __restrict__ tmp_e,
            float* __restrict__ tmp_g, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint64_t sbuf[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp;
@@ -89,6 +91,8 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
 // ---- 2. scan of the active flags ------------------------------------------
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_reduce(const int32_t* __restrict__ flags, int64_t N, int32_t* __restrict__ tile_sum) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
@@ -103,6 +107,8 @@ __global__ void __launch_bounds__(kScanThreads)
 // single block: exclusive scan of the tile sums; counts[0] = |U|, counts[1] = groups
 __global__ void __launch_bounds__(kScanThreads)
     k_scan_tiles(int32_t* __restrict__ tile_sum, int ntiles, int64_t B, int32_t* counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ int carry;
@@ -127,6 +133,8 @@ __global__ void __launch_bounds__(kScanThreads)
     k_scan_finish(const int32_t* __restrict__ flags, int64_t N,
                   const int32_t* __restrict__ tile_off, int32_t* __restrict__ rank,
                   int32_t* __restrict__ uniq) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
@@ -172,6 +180,8 @@ constexpr uint32_t kLbAgg = 1u << 30, kLbIncl = 2u << 30, kLbCount = (1u << 30) 
 
 __global__ void __launch_bounds__(kRsThreads)
     k_rs_ghist(KeySrc src, int64_t M, int passes, uint32_t* __restrict__ dgh) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint32_t h[4][256];
   for (int j = threadIdx.x; j < 4 * 256; j += kRsThreads) (&h[0][0])[j] = 0u;
   __syncthreads();
@@ -204,6 +214,8 @@ __global__ void __launch_bounds__(kRsThreads)
                   const uint32_t* __restrict__ dgh, uint32_t* __restrict__ look,
                   uint32_t* __restrict__ tile_ctr, uint32_t* __restrict__ keys_out,
                   uint32_t* __restrict__ vals_out, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint32_t wcount[kRsWarps][256];
   __shared__ uint32_t tbase[256];
   __shared__ int warp_tot[32];
@@ -294,6 +306,8 @@ __global__ void __launch_bounds__(256)
            int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
            float* __restrict__ task_gate, int32_t* __restrict__ group_off,
            const int32_t* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= M) return;
   const uint32_t pos = vals ? vals[i] : static_cast<uint32_t>(i);
@@ -412,6 +426,8 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads)
                     int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
                     float* __restrict__ task_gate, int32_t* __restrict__ uniq,
                     int32_t* __restrict__ group_off, int32_t* counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ ClSmem S;
   cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x;
@@ -574,23 +590,25 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     // key g * L + t < gmax * L
     const int kpasses =
         (nbits(static_cast<uint64_t>(D.gmax()) * static_cast<uint64_t>(D.L)) + 7) / 8;
-    k_sched_cluster<<<kClCtas, kClThreads, 0, s>>>(idx, gate, D.L, static_cast<int>(D.K), N, D.B,
-                                                   epasses, kpasses, task_token, task_expert,
-                                                   task_gate, uniq, group_off, counts);
+    OMNI_TRY(launch_k(k_sched_cluster, kClCtas, kClThreads, 0, s, idx, gate, D.L,
+        static_cast<int>(D.K), N, D.B, epasses, kpasses, task_token, task_expert, task_gate, uniq,
+        group_off, counts));
     return cudaGetLastError();
   }
   SchedWs w = carve(D, ws, nullptr);
-  cudaError_t err = cudaMemsetAsync(w.flags, 0, static_cast<size_t>(N) * sizeof(int32_t), s);
+  cudaError_t err = launch_zero(w.flags, static_cast<size_t>(N), s);
   if (err != cudaSuccess) return err;
   const int Kp = static_cast<int>(next_pow2(D.K));
   const size_t prep_smem = static_cast<size_t>(kPrepWarps) * Kp * sizeof(uint64_t);
-  k_prep<<<static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps), kPrepWarps * 32,
-           prep_smem, s>>>(idx, gate, D.L, static_cast<int>(D.K), Kp, N, w.flags, w.tmp_e,
-                           w.tmp_g, status);
-  k_scan_reduce<<<static_cast<unsigned>(w.nscan), kScanThreads, 0, s>>>(w.flags, N, w.tile_sum);
-  k_scan_tiles<<<1, kScanThreads, 0, s>>>(w.tile_sum, static_cast<int>(w.nscan), D.B, counts);
-  k_scan_finish<<<static_cast<unsigned>(w.nscan), kScanThreads, 0, s>>>(w.flags, N, w.tile_sum,
-                                                                       w.rank, uniq);
+  OMNI_TRY(launch_k(k_prep, static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps),
+      kPrepWarps * 32, prep_smem, s, idx, gate, D.L, static_cast<int>(D.K), Kp, N, w.flags, w.tmp_e,
+      w.tmp_g, status));
+  OMNI_TRY(launch_k(k_scan_reduce, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.flags, N,
+      w.tile_sum));
+  OMNI_TRY(launch_k(k_scan_tiles, 1, kScanThreads, 0, s, w.tile_sum, static_cast<int>(w.nscan), D.B,
+      counts));
+  OMNI_TRY(launch_k(k_scan_finish, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.flags, N,
+      w.tile_sum, w.rank, uniq));
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const uint32_t* keys = nullptr;
@@ -600,15 +618,16 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     uint32_t* dgh = w.sweep;
     uint32_t* ctr = dgh + 256 * w.passes;
     uint32_t* look = ctr + w.passes;
-    err = cudaMemsetAsync(w.sweep, 0, w.sweep_words * sizeof(uint32_t), s);
+    err = launch_zero(w.sweep, w.sweep_words, s);
     if (err != cudaSuccess) return err;
     KeySrc src0{nullptr, w.tmp_e, w.rank, D.B};
-    k_rs_ghist<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(src0, M, w.passes, dgh);
+    OMNI_TRY(launch_k(k_rs_ghist, static_cast<unsigned>(w.ntiles), kRsThreads, 0, s, src0, M,
+        w.passes, dgh));
     for (int p = 0; p < w.passes; ++p) {
       KeySrc src{keys, w.tmp_e, w.rank, D.B};
-      k_rs_onesweep<<<static_cast<unsigned>(w.ntiles), kRsThreads, 0, s>>>(
-          src, vals, M, 8 * p, dgh + 256 * p, look + static_cast<size_t>(p) * 256 * w.ntiles,
-          ctr + p, ko, vo, status);
+      OMNI_TRY(launch_k(k_rs_onesweep, static_cast<unsigned>(w.ntiles), kRsThreads, 0, s, src, vals,
+          M, 8 * p, dgh + 256 * p, look + static_cast<size_t>(p) * 256 * w.ntiles, ctr + p, ko, vo,
+          status));
       keys = ko;
       vals = vo;
       ko = (ko == w.ka) ? w.kb : w.ka;
@@ -617,9 +636,9 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  k_emit<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(
-      keys, vals, M, static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate,
-      group_off, counts);
+  OMNI_TRY(launch_k(k_emit, static_cast<unsigned>((M + 255) / 256), 256, 0, s, keys, vals, M,
+      static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate, group_off,
+      counts));
   return cudaGetLastError();
 }
 

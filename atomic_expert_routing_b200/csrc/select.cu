@@ -378,6 +378,7 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
                                                 int32_t* __restrict__ idx,
                                                 float* __restrict__ gate,
                                                 float* __restrict__ score, SelPlan P) {
+  pdl_wait();
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31;
   const int pair = threadIdx.x >> 6;
@@ -587,6 +588,8 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
                                                      int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
                                                      float* __restrict__ score, WidePlan P) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int axis = warp >> 2, gw = warp & 3;
@@ -773,9 +776,9 @@ cudaError_t launch_wide_t(const Dims& D, const float* Z, int parts, const float*
   cudaError_t err = cudaFuncSetAttribute(k_select_wide<NPW, W, WK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, P.bytes);
   if (err != cudaSuccess) return err;
-  k_select_wide<NPW, W, WK><<<static_cast<unsigned>(D.L), 256, P.bytes, s>>>(
-      Z, parts, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
-      static_cast<int>(D.K), br, bc, idx, gate, score, P);
+  OMNI_TRY(launch_k(k_select_wide<NPW, W, WK>, static_cast<unsigned>(D.L), 256, P.bytes, s, Z,
+      parts, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
+      static_cast<int>(D.K), br, bc, idx, gate, score, P));
   return cudaGetLastError();
 }
 
@@ -814,9 +817,9 @@ cudaError_t launch_select_t(const Dims& D, const float* Z, const float* br, cons
   if (per_sm < 1) per_sm = 1;
   int64_t grid = (D.L + pairs - 1) / pairs;
   if (grid > static_cast<int64_t>(sms) * per_sm) grid = static_cast<int64_t>(sms) * per_sm;
-  k_select<NPL, W, WK><<<static_cast<unsigned>(grid), 64 * pairs, smem, s>>>(
-      Z, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
-      static_cast<int>(D.K), br, bc, idx, gate, score, P);
+  OMNI_TRY(launch_k(k_select<NPL, W, WK>, static_cast<unsigned>(grid), 64 * pairs, smem, s, Z, D.L,
+      static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k), static_cast<int>(D.K),
+      br, bc, idx, gate, score, P));
   return cudaGetLastError();
 }
 
