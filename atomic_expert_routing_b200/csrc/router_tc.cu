@@ -5,13 +5,17 @@
 // This is the one dense contraction of the routed layer: 2*d*(Nr+Nc) flops
 // per token.
 //
-// One CTA computes a 128 x BN tile of Z.  Warp 4 (one elected lane) streams
-// 128 x 64 tiles of x and BN x 64 tiles of the axis keys into shared memory
-// with TMA (128-byte swizzle, no multicast), warp 5 (one lane) issues
-// tcgen05.mma (M=128, N=BN, K=16, bf16 -> fp32) into a TMEM accumulator and
-// releases each stage with tcgen05.commit; warps 0-3 drain TMEM with
-// tcgen05.ld (one accumulator row per thread) and store fp32 logits.
-// Every mbarrier wait is bounded; a time-out sets OMNI_DEV_TIMEOUT.
+// Persistent: CTA c computes the 128 x BN tiles c, c + gridDim.x, ... of Z
+// (N tile fastest, so the CTAs working at one time share their x rows in L2).
+// Warp 4 (one elected lane) streams 128 x 64 tiles of x and BN x 64 tiles of
+// the axis keys into a shared-memory ring with TMA (128-byte swizzle, no
+// multicast), without a break between tiles; warp 5 (one lane) issues
+// tcgen05.mma (M=128, N=BN, K=16, bf16 -> fp32) into one of two TMEM
+// accumulators and releases each stage with tcgen05.commit; warps 0-3 drain
+// the other accumulator with tcgen05.ld (one row per thread) and store fp32
+// logits, so a tile's epilogue overlaps the next tile's products.
+// Every mbarrier wait is bounded; a time-out sets OMNI_DEV_TIMEOUT and the
+// roles leave their loops.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -85,18 +89,31 @@ template <int BN>
 constexpr size_t tc_smem_bytes() {
   return 1024 /* alignment slack */ +
          static_cast<size_t>(TC_STAGES) * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) +
-         (2 * TC_STAGES + 1) * 8 + 16;
+         (2 * TC_STAGES + 4) * 8 + 16;
 }
+
+// Tile t of the grid of tiles: M block, N tile (rows then columns of the
+// grid of experts), K split.
+struct RouterTiles {
+  int mt, ntn, tiles_r, ks, kper, nk_all;
+  __device__ __forceinline__ void at(int t, int* m, int* n, int* z) const {
+    const int per = mt * ntn;
+    *z = t / per;
+    const int rem = t - *z * per;
+    *m = rem / ntn;
+    *n = rem - *m * ntn;
+  }
+};
 
 template <int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
                 const __grid_constant__ CUtensorMap tmBc, float* __restrict__ Z, int L, int Nr,
-                int Nc, int d, int tiles_r, int kper, int32_t* status) {
+                int Nc, RouterTiles T, int32_t* status) {
   pdl_wait();
   // let the selection launch early only for a single wave of tiles (small L):
   // for many waves its waiting CTAs would sit beside the last tiles
-  if (gridDim.x * gridDim.y * gridDim.z <= 296u) pdl_trigger();
+  if (T.mt * T.ntn * T.ks <= 296) pdl_trigger();
   constexpr uint32_t A_BYTES = TC_BM * TC_BK * 2;
   constexpr uint32_t B_BYTES = BN * TC_BK * 2;
   extern __shared__ uint8_t smem_raw[];
@@ -105,39 +122,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_STAGES * A_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 4);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + TC_STAGES);
-  const uint32_t accum = smem_u32(bars + 2 * TC_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * TC_STAGES);       // accumulator b ready
+  const uint32_t tempty0 = smem_u32(bars + 2 * TC_STAGES + 2);  // accumulator b drained
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * TC_BM;
-  const bool colax = static_cast<int>(blockIdx.y) >= tiles_r;
-  const CUtensorMap* tmB = colax ? &tmBc : &tmBr;
-  const int n0 = (colax ? static_cast<int>(blockIdx.y) - tiles_r : static_cast<int>(blockIdx.y)) * BN;
-  const int naxis = colax ? Nc : Nr;
   const int64_t ld = static_cast<int64_t>(Nr) + Nc;
-  const int zc0 = (colax ? Nr : 0) + n0;
-  // K range of this CTA; with a split K loop (gridDim.z > 1) every split
-  // writes its own partial logits, Z + blockIdx.z * L * (Nr + Nc)
-  const int nk_all = (d + TC_BK - 1) / TC_BK;
-  const int kb0 = static_cast<int>(blockIdx.z) * kper;
-  const int nk = (nk_all - kb0 < kper ? nk_all - kb0 : kper);
-  Z += static_cast<int64_t>(blockIdx.z) * L * (static_cast<int64_t>(Nr) + Nc);
+  const int ntiles = T.mt * T.ntn * T.ks;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 128);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(BN)
+                 "r"(2 * BN)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -147,63 +157,108 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4 && lane == 0) {
-    // producer: TMA loads of stage s
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % TC_STAGES;
-      const uint32_t ph = (kb / TC_STAGES) & 1;
-      if (!mbar_wait(empty0 + 8 * s, ph ^ 1, status)) break;
-      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES);
-      tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, full0 + 8 * s, (kb0 + kb) * TC_BK, m0);
-      tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, (kb0 + kb) * TC_BK, n0);
+    // producer: TMA loads, one ring of stages across all of this CTA's tiles
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      int m, n, z;
+      T.at(t, &m, &n, &z);
+      const bool colax = n >= T.tiles_r;
+      const CUtensorMap* tmB = colax ? &tmBc : &tmBr;
+      const int n0 = (colax ? n - T.tiles_r : n) * BN;
+      const int kb0 = z * T.kper;
+      const int nk = (T.nk_all - kb0 < T.kper ? T.nk_all - kb0 : T.kper);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % TC_STAGES;
+        const uint32_t ph = (it / TC_STAGES) & 1;
+        if (!mbar_wait(empty0 + 8 * s, ph ^ 1, status)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES);
+        tma_load_2d(smem_u32(sA + s * A_BYTES), &tmA, full0 + 8 * s, (kb0 + kb) * TC_BK,
+                    m * TC_BM);
+        tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, (kb0 + kb) * TC_BK, n0);
+      }
     }
   } else if (warp == 5 && lane == 0) {
-    // MMA issuer
+    // MMA issuer: tile j of this CTA accumulates in TMEM columns (j & 1) * BN
     constexpr uint32_t idesc = idesc_bf16<BN>();
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % TC_STAGES;
-      const uint32_t ph = (kb / TC_STAGES) & 1;
-      if (!mbar_wait(full0 + 8 * s, ph, status)) break;
+    uint32_t it = 0;
+    bool ok = true;
+    int j = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++j) {
+      int m, n, z;
+      T.at(t, &m, &n, &z);
+      const int kb0 = z * T.kper;
+      const int nk = (T.nk_all - kb0 < T.kper ? T.nk_all - kb0 : T.kper);
+      const int b = j & 1;
+      const uint32_t use = static_cast<uint32_t>(j >> 1);
+      if (!mbar_wait(tempty0 + 8 * b, (use & 1) ^ 1, status)) break;  // drained by the epilogue
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a0 = smem_u32(sA + s * A_BYTES);
-      const uint32_t b0 = smem_u32(sB + s * B_BYTES);
+      const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % TC_STAGES;
+        const uint32_t ph = (it / TC_STAGES) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph, status)) {
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t a0 = smem_u32(sA + s * A_BYTES);
+        const uint32_t b0 = smem_u32(sB + s * B_BYTES);
 #pragma unroll
-      for (int kk = 0; kk < TC_BK / 16; ++kk)
-        umma_bf16(tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
-                  (kb | kk) != 0 ? 1u : 0u);
-      umma_commit(empty0 + 8 * s);
+        for (int kk = 0; kk < TC_BK / 16; ++kk)
+          umma_bf16(acc, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                    (kb | kk) != 0 ? 1u : 0u);
+        umma_commit(empty0 + 8 * s);
+      }
+      umma_commit(tfull0 + 8 * b);
     }
-    umma_commit(accum);
   } else if (warp < 4) {
     // epilogue: TMEM lane (32*warp + lane) holds row m0 + 32*warp + lane
-    // the wait's outcome is made warp-uniform: tcgen05.ld below is .sync.aligned
-    if (__all_sync(0xffffffffu, mbar_wait(accum, 0, status))) {
+    int j = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++j) {
+      int m, n, z;
+      T.at(t, &m, &n, &z);
+      const int b = j & 1;
+      const uint32_t use = static_cast<uint32_t>(j >> 1);
+      // the wait's outcome is made warp-uniform: tcgen05.ld below is .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * b, use & 1, status))) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const int64_t grow = static_cast<int64_t>(m0) + warp * 32 + lane;
+      const bool colax = n >= T.tiles_r;
+      const int n0 = (colax ? n - T.tiles_r : n) * BN;
+      const int naxis = colax ? Nc : Nr;
+      const int zc0 = (colax ? Nr : 0) + n0;
+      float* Zs = Z + static_cast<int64_t>(z) * L * ld;  // split z writes its own partials
+      const int64_t grow = static_cast<int64_t>(m) * TC_BM + warp * 32 + lane;
       const bool vec_ok = (ld % 4 == 0) && (zc0 % 4 == 0);  // 16-byte aligned rows
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
+        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * BN + c, r);
         if (grow < L) {
-          float* zp = Z + grow * ld + zc0 + c;
+          float* zp = Zs + grow * ld + zc0 + c;
           if (n0 + c + 32 <= naxis && vec_ok) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(zp + j) =
-                  make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                              __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            for (int q = 0; q < 32; q += 4)
+              *reinterpret_cast<float4*>(zp + q) =
+                  make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                              __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
           } else {
-            for (int j = 0; j < 32; ++j)
-              if (n0 + c + j < naxis) zp[j] = __uint_as_float(r[j]);
+            for (int q = 0; q < 32; ++q)
+              if (n0 + c + q < naxis) zp[q] = __uint_as_float(r[q]);
           }
         }
       }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      mbar_arrive(tempty0 + 8 * b);
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN)
                  : "memory");
   }
 }
@@ -258,16 +313,20 @@ cudaError_t launch_bn(const Dims& D, const CUtensorMap& a, const CUtensorMap& br
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int tiles_r = static_cast<int>((D.Nr + BN - 1) / BN);
-  const int tiles_c = static_cast<int>((D.Nc + BN - 1) / BN);
-  const int64_t mt = (D.L + TC_BM - 1) / TC_BM;
-  const int nk = static_cast<int>((D.d + TC_BK - 1) / TC_BK);
-  const int ks = router_splits(D);
-  const int kper = (nk + ks - 1) / ks;
-  dim3 grid(static_cast<unsigned>(mt), tiles_r + tiles_c, ks);
-  OMNI_TRY(launch_k(k_router_tc<BN>, grid, TC_THREADS, smem, s, a, br, bc, Z, static_cast<int>(D.L),
-      static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.d), tiles_r, kper,
-      status));
+  RouterTiles T;
+  T.tiles_r = static_cast<int>((D.Nr + BN - 1) / BN);
+  T.ntn = T.tiles_r + static_cast<int>((D.Nc + BN - 1) / BN);
+  T.mt = static_cast<int>((D.L + TC_BM - 1) / TC_BM);
+  T.nk_all = static_cast<int>((D.d + TC_BK - 1) / TC_BK);
+  T.ks = router_splits(D);
+  T.kper = (T.nk_all + T.ks - 1) / T.ks;
+  const int64_t ntiles = static_cast<int64_t>(T.mt) * T.ntn * T.ks;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = ntiles < sms ? ntiles : sms;  // persistent: one CTA per SM
+  OMNI_TRY(launch_k(k_router_tc<BN>, static_cast<unsigned>(grid), TC_THREADS, smem, s, a, br, bc,
+      Z, static_cast<int>(D.L), static_cast<int>(D.Nr), static_cast<int>(D.Nc), T, status));
   return cudaGetLastError();
 }
 
