@@ -65,10 +65,10 @@ def expert_stage_bytes(cfg, n_active):
 # DRAM bytes (read + write) of one expert-stage call, summed over its kernels,
 # from ncu. The full-size stage is too large for a full capture; these values
 # come from the proxy workload (profiles/expert_stage_bf16-prefill-proxy-N256K.md,
-# 1774.8 MB) scaled by the stage's algorithmic bytes (x3.90). Update them
+# 1730.0 MB) scaled by the stage's algorithmic bytes (x3.90). Update them
 # whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
-    "bf16-prefill-N1M": (6.92e9, "ncu dram__bytes of bf16-prefill-proxy-N256K, scaled x3.90 "
+    "bf16-prefill-N1M": (6.75e9, "ncu dram__bytes of bf16-prefill-proxy-N256K, scaled x3.90 "
                                  "by algorithmic bytes"),
 }
 
