@@ -25,6 +25,7 @@
 #include "blocksort.cuh"
 #include "common.cuh"
 #include "internal.h"
+#include "warpsort.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -41,19 +42,24 @@ constexpr int kRsPerWarp = 512;  // consecutive tasks per warp in a tile
 constexpr int kRsTile = kRsWarps * kRsPerWarp;
 
 // ---- 1. per-token sort by expert id + active flags -----------------------
+// One warp per token: its K (expert, slot) keys sorted ascending in registers
+// (32*W >= K; a descending network over complemented keys), the experts
+// flagged as active.
+template <int W>
 __global__ void __launch_bounds__(kPrepWarps * 32)
     k_prep(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L, int K,
-           int Kp, int64_t N, int32_t* __restrict__ flags, int32_t* __restrict__ tmp_e,
+           int64_t N, int32_t* __restrict__ flags, int32_t* __restrict__ tmp_e,
            float* __restrict__ tmp_g, int32_t* status) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ uint64_t sbuf[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp;
-  if (t >= L) return;
-  uint64_t* s = sbuf + static_cast<size_t>(warp) * Kp;
-  for (int q = lane; q < Kp; q += 32) {
-    uint64_t key = ~0ull;
+  if (t >= L) return;  // warp-uniform
+  uint64_t key[W];
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int q = w * 32 + lane;
+    key[w] = 0ull;  // complement of the largest key: sorts last
     if (q < K) {
       int64_t e = idx[t * K + q];
       if (e < 0 || e >= N) {
@@ -61,30 +67,18 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
         e = 0;
       }
       flags[e] = 1;
-      key = (static_cast<uint64_t>(e) << 32) | static_cast<uint32_t>(q);
+      key[w] = ~((static_cast<uint64_t>(e) << 32) | static_cast<uint32_t>(q));
     }
-    s[q] = key;
   }
-  __syncwarp();
-  // bitonic sort, ascending
-  for (int size = 2; size <= Kp; size <<= 1)
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < Kp / 2; i += 32) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool asc = (lo & size) == 0;
-        const uint64_t a = s[lo], b = s[hi];
-        if ((a > b) == asc) {
-          s[lo] = b;
-          s[hi] = a;
-        }
-      }
-      __syncwarp();
+  reg_sort_desc<W>(key);
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int j = w * 32 + lane;
+    if (j < K) {
+      const uint64_t k = ~key[w];
+      tmp_e[t * K + j] = static_cast<int32_t>(k >> 32);
+      tmp_g[t * K + j] = gate[t * K + static_cast<uint32_t>(k)];
     }
-  for (int j = lane; j < K; j += 32) {
-    const uint64_t key = s[j];
-    tmp_e[t * K + j] = static_cast<int32_t>(key >> 32);
-    tmp_g[t * K + j] = gate[t * K + static_cast<uint32_t>(key)];
   }
 }
 
@@ -598,11 +592,13 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
   SchedWs w = carve(D, ws, nullptr);
   cudaError_t err = launch_zero(w.flags, static_cast<size_t>(N), s);
   if (err != cudaSuccess) return err;
-  const int Kp = static_cast<int>(next_pow2(D.K));
-  const size_t prep_smem = static_cast<size_t>(kPrepWarps) * Kp * sizeof(uint64_t);
-  OMNI_TRY(launch_k(k_prep, static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps),
-      kPrepWarps * 32, prep_smem, s, idx, gate, D.L, static_cast<int>(D.K), Kp, N, w.flags, w.tmp_e,
-      w.tmp_g, status));
+  const unsigned prep_blocks = static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps);
+  auto prep = [&](auto kern) {
+    return launch_k(kern, prep_blocks, kPrepWarps * 32, 0, s, idx, gate, D.L,
+                    static_cast<int>(D.K), N, w.flags, w.tmp_e, w.tmp_g, status);
+  };
+  OMNI_TRY(D.K <= 32 ? prep(k_prep<1>) : D.K <= 64 ? prep(k_prep<2>)
+           : D.K <= 128 ? prep(k_prep<4>) : prep(k_prep<8>));
   OMNI_TRY(launch_k(k_scan_reduce, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.flags, N,
       w.tile_sum));
   OMNI_TRY(launch_k(k_scan_tiles, 1, kScanThreads, 0, s, w.tile_sum, static_cast<int>(w.nscan), D.B,
