@@ -401,11 +401,11 @@ constexpr int kActWarps = 8;
 // c[dst[a]] = g[a] * SiLU(H[hidx[a]] . F[fidx[a]]) over a task list in which
 // tasks that share a held row H[h] are adjacent (a run).  Warp w takes slices
 // of S consecutive tasks; the run's held row sits in registers (the next
-// run's row is fetched while the current one is used), and every task's row
-// of F streams through a ring of R shared-memory slots per warp (cp.async,
-// R - 1 rows in flight).  HOLD_KEEP: the held rows are re-read by later
-// tasks (x by token) -- keep them in L2 (evict-last) and read the F rows,
-// whose repeats come right after their first read, evict-first.  dst ==
+// run's row is fetched while the current one is used), and the rows of F
+// stream through a ring of R shared-memory slots per warp (cp.async, R - 1
+// rows in flight), one per run of tasks that share it.  HOLD_KEEP: the held
+// rows are re-read by later tasks (x by token) -- keep them in L2
+// (evict-last) and read the F rows, each fetched once, evict-first.  dst ==
 // nullptr writes c[a].  Indices are range-checked (OMNI_DEV_BAD_INDEX; the
 // task gets c = 0).
 template <typename T, int NV, int R, bool HOLD_KEEP>
@@ -442,12 +442,20 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
     }
     const int64_t prev_h = __shfl_up_sync(0xffffffffu, my_h, 1);
     const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_h != my_h));
-    auto issue = [&](int j) {
-      if (j < n) {
+    const int64_t prev_f = __shfl_up_sync(0xffffffffu, my_f, 1);
+    const uint32_t fstarts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_f != my_f));
+    // the ring is filled run by run of F: a row repeated by adjacent tasks is
+    // fetched once.  Run r sits in slot r % R; every issue commits one group.
+    uint32_t pending = fstarts;
+    int issued = 0;
+    auto issue = [&]() {
+      if (pending != 0u) {
+        const int j = __ffs(pending) - 1;
+        pending &= pending - 1u;
         const int64_t f = __shfl_sync(0xffffffffu, my_f, j);
         if (f >= 0) {
           const uint4* fr = reinterpret_cast<const uint4*>(F + f * d);
-          const uint32_t base = fring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
+          const uint32_t base = fring_s + static_cast<uint32_t>((issued % R) * SLOT) * 16u;
 #pragma unroll
           for (int v = 0; v < NV; ++v) {
             if (HOLD_KEEP)
@@ -457,10 +465,11 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
           }
         }
       }
+      ++issued;
       cp_async_commit();
     };
 #pragma unroll
-    for (int j = 0; j < R - 1; ++j) issue(j);
+    for (int j = 0; j < R - 1; ++j) issue();
     uint4 hc[NV], hn[NV];
     auto load_held = [&](int64_t h) {
       const uint4* hr = reinterpret_cast<const uint4*>(H + (h < 0 ? 0 : h) * d);
@@ -468,19 +477,23 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
       for (int v = 0; v < NV; ++v) hn[v] = HOLD_KEEP ? ld_v4_hint(hr + v * 32 + lane, pol_keep) : hr[v * 32 + lane];
     };
     load_held(__shfl_sync(0xffffffffu, my_h, 0));
+    int run = -1;
     for (int j = 0; j < n; ++j) {
-      issue(j + R - 1);
+      if ((fstarts >> j) & 1u) {  // F run `run` is complete once R - 1 later ones are issued
+        ++run;
+        issue();
+        cp_async_wait<R - 1>();
+      }
       if ((starts >> j) & 1u) {
 #pragma unroll
         for (int v = 0; v < NV; ++v) hc[v] = hn[v];
         const uint32_t later = starts & ~((2u << j) - 1u);
         if (later) load_held(__shfl_sync(0xffffffffu, my_h, __ffs(later) - 1));
       }
-      cp_async_wait<R - 1>();
       const int64_t h = __shfl_sync(0xffffffffu, my_h, j);
       const float gj = __shfl_sync(0xffffffffu, my_g, j);
       if (h >= 0) {  // warp-uniform
-        const uint4* slot = fring + (j % R) * SLOT;
+        const uint4* slot = fring + (run % R) * SLOT;
         float sdot = 0.0f;
 #pragma unroll
         for (int v = 0; v < NV; ++v) sdot += dot_vec(hc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
