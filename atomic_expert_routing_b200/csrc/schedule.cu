@@ -515,6 +515,332 @@ __global__ void __cluster_dims__(kClCtas, 1, 1) __launch_bounds__(kClThreads)
   cl.sync();  // keep this CTA's shared memory alive until its neighbour has read it
 }
 
+// ---- small batches: a bitmap of the active ids across a cluster -----------
+//
+// One thread-block cluster of 8 CTAs.  CTA c holds tokens [c*Lc, (c+1)*Lc)
+// and the bitmap of ids [c*S, (c+1)*S); the CTAs reach each other's shared
+// memory directly.  Warps hold whole tokens, 32*W/P per pass (P = K rounded
+// up to a power of two).
+//  (A) Each token's K ids are sorted in registers and set their bits in the
+//      bitmap of the CTA that owns them.
+//  (B) Each CTA counts its bits in 8-word chunks and scans them; the CTA
+//      totals, summed across the cluster, give |U| and the first rank of each
+//      CTA's ids.  Each CTA writes its part of U.  The rank of any id is then
+//      its CTA's first rank plus its chunk's prefix plus the popcounts of the
+//      chunk's earlier words and of its own word below it.
+//  (C) Per token, the rank and group g = rank / B of every task.  A token's
+//      tasks of one group are consecutive in its sorted list, so a task's
+//      place among them is its distance to the first of them; the last one
+//      writes their count into the cell (g, token).  Each CTA sums its cells
+//      per group.
+//  (D) The group sums of all CTAs give the first position of every group and
+//      of every cell: groups in order, inside a group the tokens of CTA 0,
+//      then CTA 1, ..., each CTA's tokens in order.
+//  (E) Every task goes to its position: (group, token, expert) order, with
+//      equal ids of one token (only out-of-range ids, read as 0) in slot order.
+// The cluster takes the same five barriers on every path; no CTA waits on a
+// flag.  Batches beyond its limits take the radix cluster sort above.
+constexpr int kCbCtas = 8;
+constexpr int kCbThreads = 512;
+constexpr int kCbWarps = kCbThreads / 32;
+constexpr int kCbChunk = 8;             // bitmap words per chunk prefix
+constexpr int64_t kCbSlice = 1024;      // ids per CTA: a multiple of this
+constexpr int64_t kCbMaxWords = 16384;  // bitmap words per CTA: N <= 2^22
+constexpr int64_t kCbMaxTokens = 64;    // tokens per CTA
+constexpr int64_t kCbMaxCells = 8192;   // gmax * tokens per CTA
+constexpr int kCbMaxK = 256;
+constexpr int kCbSlotBits = 8;          // se = e << 8 | slot; info = g << 8 | place
+constexpr size_t kCbMaxSmem = 200 * 1024;
+
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int P>
+__global__ void __cluster_dims__(kCbCtas, 1, 1) __launch_bounds__(kCbThreads)
+    k_sched_bits(const int32_t* __restrict__ idx, const float* __restrict__ gate, int L, int K,
+                 int64_t N, int64_t B, uint32_t Bq, int S, int words, int Lc, int gmax,
+                 int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
+                 float* __restrict__ task_gate, int32_t* __restrict__ uniq,
+                 int32_t* __restrict__ group_off, int32_t* counts) {
+  constexpr int W = P > 32 ? P / 32 : 1;  // keys per lane: one token spans W rows
+  constexpr int TP = 32 * W / P;          // tokens per warp and pass
+  constexpr int WIDTH = P < 32 ? P : 32;  // lanes of one token in a row
+  constexpr uint32_t kSlotMask = (1u << kCbSlotBits) - 1u;
+  constexpr uint32_t kFull = 0xffffffffu;
+  extern __shared__ __align__(16) uint32_t csm[];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int tot_local;               // this CTA's active ids, read by the others
+  __shared__ int first_rank[kCbCtas + 1]; // first rank of each CTA's ids; [8] = |U|
+  cg::cluster_group cl = cg::this_cluster();
+  const int crank = static_cast<int>(cl.block_rank());
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int M = L * K;
+  const int t_lo = crank * Lc;
+  const int t_hi = L < t_lo + Lc ? L : t_lo + Lc;
+  const int Mc = t_hi > t_lo ? (t_hi - t_lo) * K : 0;
+  const int nchunks = words / kCbChunk;
+  uint32_t* bits = csm;                         // ids [crank*S, crank*S + S)
+  int* cpre = reinterpret_cast<int*>(bits + words);
+  int* cells = cpre + nchunks;                  // [gmax][Lc]
+  int* sg = cells + gmax * Lc;                  // [gmax] this CTA's tasks per group
+  int* gtot = sg + gmax;                        // [gmax] all CTAs' tasks per group
+  int* gbef = gtot + gmax;                      // [gmax] the earlier CTAs' tasks per group
+  uint32_t* se = reinterpret_cast<uint32_t*>(gbef + gmax);  // [Lc*K] e << 8 | slot
+  uint32_t* info = se + Lc * K;                 // [Lc*K] g << 8 | place
+  int32_t* status = counts + 2;
+  const int t_first = t_lo + warp * TP;
+  const int t_step = kCbWarps * TP;
+
+  // clearing the bitmaps and the cells needs nothing from the kernel before
+  // this one: it runs while that kernel finishes
+  for (int j = tid; j < words / 4; j += kCbThreads)
+    reinterpret_cast<uint4*>(bits)[j] = make_uint4(0u, 0u, 0u, 0u);
+  for (int j = tid; j < gmax * Lc; j += kCbThreads) cells[j] = 0;
+  cl.sync();  // (1) every bitmap is clear
+  pdl_wait();
+  pdl_trigger();
+  uint32_t key[W];
+  int eid[W];
+  auto load_keys = [&](int t0) {
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int i = w * 32 + lane;
+      const int t = t0 + i / P, q = i % P;
+      key[w] = 0u;  // complement of the largest key: sorts last
+      eid[w] = -1;
+      if (t < t_hi && q < K) {
+        int64_t e = idx[static_cast<int64_t>(t) * K + q];
+        if (e < 0 || e >= N) {
+          raise_status(status, OMNI_DEV_BAD_INDEX);
+          e = 0;
+        }
+        eid[w] = static_cast<int>(e);
+        key[w] = ~((static_cast<uint32_t>(e) << kCbSlotBits) | static_cast<uint32_t>(q));
+      }
+    }
+  };
+  // (A)
+  for (int t0 = t_first; t0 < t_hi; t0 += t_step) {
+    load_keys(t0);
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      if (eid[w] >= 0) {
+        const int o = eid[w] / S;
+        atomicOr(cl.map_shared_rank(bits, o) + ((eid[w] - o * S) >> 5), 1u << (eid[w] & 31));
+      }
+    }
+    reg_sort_desc<W, P>(key);
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int i = w * 32 + lane;
+      const int t = t0 + i / P, q = i % P;
+      if (t < t_hi && q < K) se[(t - t_lo) * K + q] = ~key[w];
+    }
+  }
+  cl.sync();  // (2) every bit is set
+  // (B) chunk popcounts (a warp reads 128 consecutive words a step), then their scan
+  for (int base = warp * 128; base < words; base += kCbWarps * 128) {
+    const int wd = base + lane * 4;
+    int c = 0;
+    if (wd < words) {
+      const uint4 v = *reinterpret_cast<const uint4*>(bits + wd);
+      c = __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+    }
+    c += __shfl_xor_sync(kFull, c, 1);
+    if (wd < words && (lane & 1) == 0) cpre[wd / kCbChunk] = c;
+  }
+  __syncthreads();
+  {
+    int4 v = make_int4(0, 0, 0, 0);
+    if (tid * 4 < nchunks) v = reinterpret_cast<const int4*>(cpre)[tid];
+    const int ex = block_exclusive_scan(v.x + v.y + v.z + v.w, warp_tot, &total);
+    if (tid * 4 < nchunks)
+      reinterpret_cast<int4*>(cpre)[tid] =
+          make_int4(ex, ex + v.x, ex + v.x + v.y, ex + v.x + v.y + v.z);
+    if (tid == 0) tot_local = total;
+  }
+  cl.sync();  // (3) every CTA's total is visible
+  if (warp == 0) {
+    const int v = lane < kCbCtas ? *cl.map_shared_rank(&tot_local, lane) : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < kCbCtas; o <<= 1) {
+      const int x = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane < kCbCtas) first_rank[lane] = incl - v;
+    if (lane == kCbCtas - 1) first_rank[kCbCtas] = incl;
+  }
+  __syncthreads();
+  const int n_active = first_rank[kCbCtas];
+  const int64_t G = (n_active + B - 1) / B;
+  if (crank == 0 && tid == 0) {
+    counts[0] = n_active;
+    counts[1] = static_cast<int32_t>(G);
+    group_off[G] = M;
+  }
+  // this CTA's part of U, a chunk per thread
+  for (int ch = tid; ch < nchunks; ch += kCbThreads) {
+    int r = first_rank[crank] + cpre[ch];
+    const uint4 lo = reinterpret_cast<const uint4*>(bits)[ch * 2];
+    const uint4 hi = reinterpret_cast<const uint4*>(bits)[ch * 2 + 1];
+    const uint32_t wv[kCbChunk] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int u = 0; u < kCbChunk; ++u) {
+      uint32_t v = wv[u];
+      while (v != 0u) {
+        const int b = __ffs(v) - 1;
+        v &= v - 1u;
+        uniq[r++] = crank * S + (ch * kCbChunk + u) * 32 + b;
+      }
+    }
+  }
+  // (C) per token: ranks, groups, places and cell counts
+  for (int t0 = t_first; t0 < t_hi; t0 += t_step) {
+    int g[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int i = w * 32 + lane;
+      const int t = t0 + i / P, q = i % P;
+      g[w] = -1;
+      if (t < t_hi && q < K) {
+        const uint32_t e = se[(t - t_lo) * K + q] >> kCbSlotBits;
+        const int o = static_cast<int>(e) / S;
+        const int wd = (static_cast<int>(e) - o * S) >> 5, c0 = wd & ~(kCbChunk - 1);
+        const uint4* rb = reinterpret_cast<const uint4*>(cl.map_shared_rank(bits, o) + c0);
+        const uint4 lo = rb[0], hi = rb[1];
+        const uint32_t wv[kCbChunk] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        int r = first_rank[o] + cl.map_shared_rank(cpre, o)[wd / kCbChunk];
+        const int jw = wd - c0;
+        const uint32_t below = (1u << (e & 31)) - 1u;
+#pragma unroll
+        for (int u = 0; u < kCbChunk; ++u)
+          r += __popc(wv[u] & (u < jw ? kFull : (u == jw ? below : 0u)));
+        g[w] = static_cast<int>(static_cast<uint32_t>(r) / Bq);
+      }
+    }
+    int carry = 0;  // first place of the run that reaches into this row
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int i = w * 32 + lane;
+      const int t = t0 + i / P, q = i % P;
+      const int row_prev = __shfl_sync(kFull, g[w > 0 ? w - 1 : 0], 31);
+      const int row_next = __shfl_sync(kFull, g[w + 1 < W ? w + 1 : W - 1], 0);
+      int gp = __shfl_up_sync(kFull, g[w], 1, WIDTH);
+      int gn = __shfl_down_sync(kFull, g[w], 1, WIDTH);
+      if (w > 0 && lane == 0) gp = row_prev;
+      if (w + 1 < W && lane == 31) gn = row_next;
+      int first = (q == 0 || gp != g[w]) ? q : 0;
+#pragma unroll
+      for (int o = 1; o < WIDTH; o <<= 1) {
+        const int f = __shfl_up_sync(kFull, first, o, WIDTH);
+        if ((lane % WIDTH) >= o) first = f > first ? f : first;
+      }
+      first = first > carry ? first : carry;
+      carry = __shfl_sync(kFull, first, 31);
+      if (t < t_hi && q < K) {
+        const int place = q - first;
+        info[(t - t_lo) * K + q] =
+            (static_cast<uint32_t>(g[w]) << kCbSlotBits) | static_cast<uint32_t>(place);
+        if (q == K - 1 || gn != g[w]) cells[g[w] * Lc + (t - t_lo)] = place + 1;
+      }
+    }
+  }
+  __syncthreads();
+  for (int g = tid; g < G; g += kCbThreads) {
+    int sum = 0;
+    for (int tl = 0; tl < Lc; ++tl) sum += cells[g * Lc + tl];
+    sg[g] = sum;
+  }
+  cl.sync();  // (4) every CTA's group sums are visible
+  // (D) group totals (thread k takes groups [k*per, k*per + per)), their scan, cell bases
+  const int per = static_cast<int>((G + kCbThreads - 1) / kCbThreads);
+  int mine = 0;
+  for (int g = tid * per; g < G && g < tid * per + per; ++g) {
+    int all = 0, before = 0;
+    for (int c = 0; c < kCbCtas; ++c) {
+      const int v = cl.map_shared_rank(sg, c)[g];
+      all += v;
+      if (c < crank) before += v;
+    }
+    gtot[g] = all;
+    gbef[g] = before;
+    mine += all;
+  }
+  cluster_arrive_release();  // this CTA reads no other CTA's shared memory from here on
+  {
+    int run = block_exclusive_scan(mine, warp_tot, &total);
+    for (int g = tid * per; g < G && g < tid * per + per; ++g) {
+      if (crank == 0) group_off[g] = run;
+      int pos = run + gbef[g];
+      for (int tl = 0; tl < Lc; ++tl) {
+        const int v = cells[g * Lc + tl];
+        cells[g * Lc + tl] = pos;
+        pos += v;
+      }
+      run += gtot[g];
+    }
+  }
+  __syncthreads();
+  // (E)
+  for (int j = tid; j < Mc; j += kCbThreads) {
+    const int tl = j / K;
+    const uint32_t a = se[j], b = info[j];
+    const int pos = cells[static_cast<int>(b >> kCbSlotBits) * Lc + tl] + static_cast<int>(b & kSlotMask);
+    if (pos < 0 || pos >= M) {  // unreachable for consistent inputs; never write outside
+      raise_status(status, OMNI_DEV_BAD_INDEX);
+      continue;
+    }
+    const int t = t_lo + tl;
+    task_token[pos] = t;
+    task_expert[pos] = static_cast<int32_t>(a >> kCbSlotBits);
+    task_gate[pos] = gate[static_cast<int64_t>(t) * K + (a & kSlotMask)];
+  }
+  cluster_wait_acquire();  // (5) no CTA still reads this CTA's shared memory
+}
+
+// The bitmap cluster scheduler's layout, or false when it does not apply.
+struct CbPlan {
+  int S, words, Lc, gmax;
+  size_t smem;
+};
+bool bits_plan(const Dims& D, CbPlan* p) {
+  const int64_t N = D.N(), M = D.M();
+  if (M > kSmallMax || D.K > kCbMaxK) return false;
+  const int64_t S = (N + kCbCtas * kCbSlice - 1) / (kCbCtas * kCbSlice) * kCbSlice;
+  const int64_t words = S / 32;
+  const int64_t Lc = (D.L + kCbCtas - 1) / kCbCtas;
+  const int64_t gmax = D.gmax();
+  if (words > kCbMaxWords || Lc > kCbMaxTokens || gmax * Lc > kCbMaxCells) return false;
+  const size_t smem = sizeof(uint32_t) *
+      static_cast<size_t>(words + words / kCbChunk + gmax * Lc + 3 * gmax + 2 * Lc * D.K);
+  if (smem > kCbMaxSmem) return false;
+  *p = CbPlan{static_cast<int>(S), static_cast<int>(words), static_cast<int>(Lc),
+              static_cast<int>(gmax), smem};
+  return true;
+}
+
+template <int P>
+cudaError_t launch_bits(const Dims& D, const CbPlan& p, const int32_t* idx, const float* gate,
+                        int32_t* task_token, int32_t* task_expert, float* task_gate,
+                        int32_t* uniq, int32_t* group_off, int32_t* counts, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(k_sched_bits<P>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(p.smem));
+  if (err != cudaSuccess) return err;
+  // ranks are below 2^22: any B beyond 2^30 puts every expert in group 0
+  const uint32_t Bq = static_cast<uint32_t>(D.B < (int64_t(1) << 30) ? D.B : (int64_t(1) << 30));
+  OMNI_TRY(launch_k(k_sched_bits<P>, kCbCtas, kCbThreads, p.smem, s, idx, gate,
+      static_cast<int>(D.L), static_cast<int>(D.K), D.N(), D.B, Bq, p.S, p.words, p.Lc, p.gmax,
+      task_token, task_expert, task_gate, uniq, group_off, counts));
+  return cudaGetLastError();
+}
+
 struct SchedWs {
   int32_t *flags, *rank, *tile_sum, *tmp_e;
   float* tmp_g;
@@ -573,6 +899,16 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     cudaError_t e = cudaMemsetAsync(counts, 0, 2 * sizeof(int32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(group_off, 0, sizeof(int32_t), s);
     return e;
+  }
+  CbPlan cp;
+  if (bits_plan(D, &cp)) {
+#define OMNI_BITS(P_) \
+  if (D.K <= P_)      \
+    return launch_bits<P_>(D, cp, idx, gate, task_token, task_expert, task_gate, uniq, group_off, \
+                           counts, s);
+    OMNI_BITS(1) OMNI_BITS(2) OMNI_BITS(4) OMNI_BITS(8) OMNI_BITS(16) OMNI_BITS(32) OMNI_BITS(64)
+    OMNI_BITS(128) OMNI_BITS(256)
+#undef OMNI_BITS
   }
   if (M <= kSmallMax) {
     auto nbits = [](uint64_t v) {

@@ -179,6 +179,41 @@ def test_schedule_group_size_extremes(B):
     np.testing.assert_array_equal(s["group_off"].cpu().numpy()[:cnt[1] + 1], ref["group_off"])
 
 
+SCHED = [
+    # one cluster over a bitmap of all ids; K rounded up to a power of two
+    # gives the segment each token's ids are sorted in
+    WL.Config("bits-K1", L=500, d=8, Nr=32, Nc=64, k=1, K=1, B=100, dtype=WL.F32),
+    WL.Config("bits-K3", L=37, d=8, Nr=12, Nc=20, k=3, K=3, B=2, dtype=WL.F32),
+    WL.Config("bits-K16", L=256, d=8, Nr=256, Nc=256, k=16, K=16, B=64, dtype=WL.F32),
+    WL.Config("bits-K32", L=100, d=8, Nr=512, Nc=512, k=32, K=32, B=50, dtype=WL.F32),
+    WL.Config("bits-K64-M8192", L=128, d=8, Nr=1024, Nc=1024, k=64, K=64, B=128, dtype=WL.F32),
+    WL.Config("bits-K100", L=20, d=8, Nr=64, Nc=64, k=64, K=100, B=7, dtype=WL.F32),
+    WL.Config("bits-K256", L=16, d=8, Nr=128, Nc=64, k=64, K=256, B=64, dtype=WL.F32),
+    WL.Config("bits-N4M", L=64, d=8, Nr=2048, Nc=2048, k=64, K=64, B=128, dtype=WL.F32),
+    # the radix cluster sort: more than 2^22 ids, or more than 512 tokens
+    WL.Config("cluster-N16M", L=64, d=8, Nr=4096, Nc=4096, k=64, K=64, B=128, dtype=WL.F32),
+    WL.Config("cluster-L1000", L=1000, d=8, Nr=64, Nc=64, k=8, K=8, B=1, dtype=WL.F32),
+    # the multi-kernel radix sort
+    WL.Config("radix-M16384", L=1024, d=8, Nr=128, Nc=128, k=16, K=16, B=64, dtype=WL.F32),
+]
+
+
+@pytest.mark.parametrize("cfg", SCHED, ids=[c.name for c in SCHED])
+def test_schedule_paths(cfg):
+    """Every scheduler variant against the oracle on a seeded routing whose
+    tokens share part of their experts."""
+    idx, gate = WL.random_routing(cfg)
+    ref = O.schedule(cfg, idx, gate.astype(np.float64))
+    s = omni.schedule(omni.LayerDims.of(cfg), dev(idx), dev(gate))
+    cnt = s["counts"].cpu().numpy()
+    assert cnt[0] == ref["n_active"] and cnt[1] == ref["n_groups"] and cnt[2] == 0
+    np.testing.assert_array_equal(s["task_token"].cpu().numpy(), ref["task_token"])
+    np.testing.assert_array_equal(s["task_expert"].cpu().numpy(), ref["task_expert"])
+    np.testing.assert_array_equal(s["task_gate"].cpu().numpy(), ref["task_gate"].astype(np.float32))
+    np.testing.assert_array_equal(s["uniq"].cpu().numpy()[:cnt[0]], ref["uniq"])
+    np.testing.assert_array_equal(s["group_off"].cpu().numpy()[:cnt[1] + 1], ref["group_off"])
+
+
 def test_schedule_bad_index_sets_status():
     cfg = WL.TINY
     h = host_inputs(cfg)

@@ -163,3 +163,21 @@ def sample_tokens(cfg: Config, n: int, seed: int = 1234) -> np.ndarray:
         return np.arange(cfg.L, dtype=np.int64)
     rng = np.random.default_rng(seed)
     return np.sort(rng.choice(cfg.L, size=n, replace=False)).astype(np.int64)
+
+
+def random_routing(cfg: Config, seed: int = 99, pool: int = 4096) -> tuple:
+    """A seeded routing decision for scheduler tests: idx [L, K] int32 with K
+    distinct ids per token, about half of them drawn from a shared pool of
+    ``pool`` ids (so groups hold several tokens and tokens share experts),
+    and gate [L, K] float32 uniform in (0, 1]."""
+    rng = np.random.default_rng(np.random.SeedSequence(entropy=seed, spawn_key=(cfg.L, cfg.K)))
+    hot = rng.choice(cfg.N, size=min(pool, cfg.N), replace=False)
+    idx = np.empty((cfg.L, cfg.K), np.int32)
+    for t in range(cfg.L):
+        n_hot = min(cfg.K // 2, len(hot))
+        picks = set(rng.choice(hot, size=n_hot, replace=False).tolist())
+        while len(picks) < cfg.K:
+            picks.update(rng.integers(0, cfg.N, size=cfg.K - len(picks)).tolist())
+        idx[t] = rng.permutation(np.fromiter(picks, np.int64, count=len(picks))[: cfg.K])
+    gate = (1.0 - rng.random((cfg.L, cfg.K))).astype(np.float32)
+    return idx, gate
