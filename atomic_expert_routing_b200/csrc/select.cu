@@ -421,12 +421,14 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
     }
     mx = warp_max(mx);
     mn = -warp_max(-mn);
-    float s = 0.0f;
+    if (score != nullptr) {  // the log-sum-exp moves only the scores, not ids or gates
+      float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < NPL; ++j)
-      if (j * 32 + lane < n) s += __expf(v[j] - mx);
-    s = warp_sum(s);
-    if (lane == 0) misc[role] = mx + logf(s);
+      for (int j = 0; j < NPL; ++j)
+        if (j * 32 + lane < n) s += __expf(v[j] - mx);
+      s = warp_sum(s);
+      if (lane == 0) misc[role] = mx + logf(s);
+    }
     group_topk<W, 1>(
         0, 0,
         [&](auto f) {
@@ -611,18 +613,20 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
       mx = fmaxf(mx, red[axis * 4 + q]);
       mn = fminf(mn, red[8 + axis * 4 + q]);
     }
-    float s = 0.0f;
+    if (score != nullptr) {  // the log-sum-exp moves only the scores, not ids or gates
+      float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < NPW; ++j)
-      if ((j * 4 + gw) * 32 + lane < n) s += __expf(v[j] - mx);
-    s = warp_sum(s);
-    if (lane == 0) red[16 + warp] = s;
-    group_sync<4>(bar);
-    if (gw == 0 && lane == 0) {
-      float tot = 0.0f;
+      for (int j = 0; j < NPW; ++j)
+        if ((j * 4 + gw) * 32 + lane < n) s += __expf(v[j] - mx);
+      s = warp_sum(s);
+      if (lane == 0) red[16 + warp] = s;
+      group_sync<4>(bar);
+      if (gw == 0 && lane == 0) {
+        float tot = 0.0f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tot += red[16 + axis * 4 + q];
-      misc[axis] = mx + logf(tot);
+        for (int q = 0; q < 4; ++q) tot += red[16 + axis * 4 + q];
+        misc[axis] = mx + logf(tot);
+      }
     }
     group_topk<W, 4>(
         gw, bar,

@@ -29,6 +29,9 @@ def _case(cfg):
 @pytest.mark.parametrize("cfg", [
     WL.Config("noalloc-bf16", L=96, d=256, Nr=32, Nc=48, k=8, K=8, B=16, dtype=WL.BF16, seed=21),
     WL.Config("noalloc-f32", L=40, d=64, Nr=16, Nc=16, k=4, K=6, B=8, dtype=WL.F32, seed=22),
+    # the largest batch the array takes: L * d = 4 Mi, with the per-token counts behind it
+    WL.Config("noalloc-largest", L=2048, d=2048, Nr=32, Nc=32, k=4, K=4, B=16, dtype=WL.BF16,
+              seed=23),
 ], ids=lambda c: c.name)
 def test_noalloc_matches_workspace_path_twice(cfg):
     D, d, sched = _case(cfg)
