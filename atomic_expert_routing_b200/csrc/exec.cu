@@ -681,8 +681,8 @@ __device__ __forceinline__ void fma_quad(float c, uint4 v, float* a) {
   a[2] = fmaf(c, __uint_as_float(v.z), a[2]); a[3] = fmaf(c, __uint_as_float(v.w), a[3]);
 }
 
-// One sweep over the window-ordered tasks: y[t, col0 : col0 + 128*NB] +=
-// c * V[e, same columns], summed over each run of one token's tasks in a
+// One sweep over the window-ordered tasks: yacc[t, 0 : 128*NB] (rows ld
+// floats apart) += c * V[e, col0 : col0 + 128*NB], summed over each run of one token's tasks in a
 // 32-task slice and added with one vector reduction per run and 128 columns.
 // Lane l owns columns col0 + 128*b + 4*l .. +3 of every block b, so each
 // reduction instruction covers 512 contiguous bytes of y (whole sectors).
@@ -693,7 +693,8 @@ template <typename T, int NB, int D>
 __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
     k_acc(const T* __restrict__ V, const int32_t* __restrict__ task_token,
           const int32_t* __restrict__ task_expert, const float* __restrict__ cbuf, int64_t M,
-          int64_t L, int64_t N, int d, int col0, int64_t nslices, float* __restrict__ yacc) {
+          int64_t L, int64_t N, int d, int col0, int64_t nslices, float* __restrict__ yacc,
+          int64_t ld) {
   pdl_wait();
   static_assert(32 % D == 0, "the prefetch distance divides the slice");
   using QT = typename Quad<T>::type;
@@ -767,7 +768,7 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
           if ((ends >> j) & 1u) {
             const int t = __shfl_sync(0xffffffffu, cur.t, j);
             if (t >= 0) {
-              float* yr = yacc + static_cast<int64_t>(t) * d + col0 + 4 * lane;
+              float* yr = yacc + static_cast<int64_t>(t) * ld + 4 * lane;
 #pragma unroll
               for (int bb = 0; bb < NB; ++bb)
                 red_add_v4_keep(yr + 128 * bb, acc[bb][0], acc[bb][1], acc[bb][2], acc[bb][3],
@@ -799,16 +800,18 @@ __global__ void __launch_bounds__(256) k_cast(const float* __restrict__ src,
   *reinterpret_cast<uint4*>(dst + i) = pack_vec(f, static_cast<__nv_bfloat16*>(nullptr));
 }
 
-// Bookkeeping between accumulation sweeps, on column slices of the fp32
-// accumulator (L rows of d floats), 8 columns per thread:
-//  - cast0 >= 0: columns [cast0, cast0 + cols) are final -- round them to
-//    bf16 into y and, the accumulator being scratch, drop its 128-byte lines
-//    from L2 without writing them back (discard.global.L2);
-//  - zero0 >= 0: zero columns [zero0, zero0 + cols) for the next sweep (the
-//    stores leave the slice in L2 for it).
+// Bookkeeping between accumulation sweeps on an fp32 slice of cols columns
+// of L rows, 8 columns per thread:
+//  - src != nullptr: the slice (rows src_ld floats apart) is final -- round
+//    it to bf16 into y (rows y_ld apart); with discard, the accumulator being
+//    scratch, drop its 128-byte lines from L2 without writing them back
+//    (discard.global.L2);
+//  - zdst != nullptr: zero the slice at zdst (rows z_ld apart) for the next
+//    sweep; the stores leave it in L2.  zdst may be src: each thread reads
+//    its eight values before it zeroes them.
 __global__ void __launch_bounds__(256)
-    k_slice_finish(float* __restrict__ acc, __nv_bfloat16* __restrict__ y, int64_t L, int d,
-                   int cast0, int zero0, int cols) {
+    k_slice_finish(const float* __restrict__ src, int64_t src_ld, __nv_bfloat16* __restrict__ y,
+                   int64_t y_ld, float* zdst, int64_t z_ld, int64_t L, int cols, int discard) {
   pdl_wait();
   pdl_trigger();
   const int per_row = cols / 8;
@@ -816,20 +819,22 @@ __global__ void __launch_bounds__(256)
   const int64_t row = i / per_row;
   const int c8 = static_cast<int>(i % per_row) * 8;
   const bool active = row < L;
-  if (cast0 >= 0) {
-    float* src = acc + row * d + cast0 + c8;
+  if (src != nullptr) {
+    const float* p = src + row * src_ld + c8;
     if (active) {
-      const float4 a = *reinterpret_cast<const float4*>(src);
-      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      const float4 a = *reinterpret_cast<const float4*>(p);
+      const float4 b = *reinterpret_cast<const float4*>(p + 4);
       const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      *reinterpret_cast<uint4*>(y + row * d + cast0 + c8) =
+      *reinterpret_cast<uint4*>(y + row * y_ld + c8) =
           pack_vec(f, static_cast<__nv_bfloat16*>(nullptr));
     }
-    __syncwarp();  // the four threads of a line have read it
-    if (active && (c8 & 31) == 0) asm volatile("discard.global.L2 [%0], 128;" ::"l"(src) : "memory");
+    if (discard) {
+      __syncwarp();  // the four threads of a line have read it
+      if (active && (c8 & 31) == 0) asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+    }
   }
-  if (zero0 >= 0 && active) {
-    float4* dst = reinterpret_cast<float4*>(acc + row * d + zero0 + c8);
+  if (zdst != nullptr && active) {
+    float4* dst = reinterpret_cast<float4*>(zdst + row * z_ld + c8);
     dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -929,7 +934,7 @@ size_t acc_bytes(const Dims& D) {
 
 SweepWs carve_sweeps(const Dims& D, void* ws, size_t* bytes) {
   Carver c(ws);
-  c.take<char>(acc_bytes(D));
+  c.take<char>(acc_bytes(D) / expert_sweeps(D));  // bf16: one fp32 slice of d / Q columns
   SweepWs w;
   const size_t M = static_cast<size_t>(D.M());
   w.cbuf = c.take<float>(M);
@@ -1040,7 +1045,7 @@ cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, co
 
 template <typename T, int NB, int D>
 cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w, float* acc,
-                       cudaStream_t s) {
+                       int64_t ld, cudaStream_t s) {
   int per_sm = 1;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_acc<T, NB, D>,
                                                                   kAccWarps * 32, 0);
@@ -1053,16 +1058,16 @@ cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w
   if (blocks > cap) blocks = cap;
   OMNI_TRY(launch_k(k_acc<T, NB, D>, static_cast<unsigned>(blocks), kAccWarps * 32, 0, s,
       static_cast<const T*>(V), w.win.wt, w.win.we, w.cbuf, M, D_.L, D_.N(), static_cast<int>(D_.d),
-      col0, nslices, acc));
+      col0, nslices, acc, ld));
   return cudaGetLastError();
 }
 
-cudaError_t launch_finish(const Dims& D, float* acc, __nv_bfloat16* y, int cast0, int zero0,
-                          int cols, cudaStream_t s) {
-  if (cast0 < 0 && zero0 < 0) return cudaSuccess;
+cudaError_t launch_finish(const Dims& D, const float* src, int64_t src_ld, __nv_bfloat16* y,
+                          float* zdst, int64_t z_ld, int cols, bool discard, cudaStream_t s) {
+  if (src == nullptr && zdst == nullptr) return cudaSuccess;
   const int64_t threads = D.L * (cols / 8);
-  OMNI_TRY(launch_k(k_slice_finish, static_cast<unsigned>((threads + 255) / 256), 256, 0, s, acc, y,
-      D.L, static_cast<int>(D.d), cast0, zero0, cols));
+  OMNI_TRY(launch_k(k_slice_finish, static_cast<unsigned>((threads + 255) / 256), 256, 0, s, src,
+      src_ld, y, static_cast<int64_t>(D.d), zdst, z_ld, D.L, cols, discard ? 1 : 0));
   return cudaGetLastError();
 }
 
@@ -1097,13 +1102,19 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   // of loads in flight per lane)
   constexpr int NB = NVQ * 32 * kEpv<T> / 128;
   constexpr int PD = 8 / NVQ;
-  // each sweep's slice is zeroed just before it and cast just after it
-  err = launch_finish(D, acc, ycast, -1, 0, cols, s);
+  // bf16: one compact fp32 slice [L x cols] serves every sweep -- zeroed
+  // before the first, then rounded into y's columns and zeroed in place
+  // (its lines stay in L2) between sweeps, and dropped after the last.
+  // fp32: the slices are y's own columns.
+  const int64_t ld = ycast ? cols : D.d;
+  auto slice = [&](int q) { return ycast ? acc : acc + static_cast<int64_t>(q) * cols; };
+  err = launch_finish(D, nullptr, 0, nullptr, slice(0), ld, cols, false, s);
   for (int q = 0; q < Q && err == cudaSuccess; ++q) {
-    err = launch_acc<T, NB, PD>(D, q * cols, V, w, acc, s);
-    if (err == cudaSuccess)
-      err = launch_finish(D, acc, ycast, ycast ? q * cols : -1, q + 1 < Q ? (q + 1) * cols : -1,
-                          cols, s);
+    err = launch_acc<T, NB, PD>(D, q * cols, V, w, slice(q), ld, s);
+    if (err != cudaSuccess) break;
+    const bool last = q + 1 == Q;
+    err = launch_finish(D, ycast ? acc : nullptr, ld, ycast ? ycast + static_cast<int64_t>(q) * cols : nullptr,
+                        last ? nullptr : slice(q + 1), ld, cols, last, s);
   }
   return err;
 }

@@ -68,8 +68,7 @@ def expert_stage_bytes(cfg, n_active):
 # 1730.0 MB) scaled by the stage's algorithmic bytes (x3.90). Update them
 # whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
-    "bf16-prefill-N1M": (6.74e9, "ncu dram__bytes of bf16-prefill-proxy-N256K, scaled x3.90 "
-                                 "by algorithmic bytes"),
+    # re-captured after every change to the stage's kernels; until then none
 }
 
 
