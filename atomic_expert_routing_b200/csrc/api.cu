@@ -48,6 +48,12 @@ struct FusedWs {
   void* sched;
   void* expert;
 };
+// A large bf16/fp32 batch on the sweep path: the fused forward goes from the
+// routing straight to the window order of the sweeps.
+bool fused_windows(const Dims& D) {
+  return omni::expert_sweeps(D) > 1 && omni::windows_supported(D);
+}
+
 FusedWs carve_fused(const Dims& D, Carver& c) {
   FusedWs w;
   w.route = carve_route(D, c);
@@ -59,7 +65,8 @@ FusedWs carve_fused(const Dims& D, Carver& c) {
   w.task_gate = c.take<float>(M);
   w.uniq = c.take<int32_t>(static_cast<size_t>(D.ucap() > 0 ? D.ucap() : 1));
   w.group_off = c.take<int32_t>(static_cast<size_t>(D.gmax()) + 1);
-  w.sched = c.take<char>(omni::schedule_ws_bytes(D));
+  w.sched = c.take<char>(fused_windows(D) ? omni::windows_ws_bytes(D)
+                                           : omni::schedule_ws_bytes(D));
   w.expert = c.take<char>(omni::expert_ws_bytes(D));
   return w;
 }
@@ -253,6 +260,12 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   float* gate = gate_out ? gate_out : w.gate;
   rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s);
   if (rc != OMNI_OK) return rc;
+  if (fused_windows(D)) {
+    rc = cuda_status(omni::launch_schedule_windows(D, idx, gate, w.uniq, w.group_off, counts,
+                                                   w.sched, omni::expert_windows(D, w.expert), s));
+    if (rc != OMNI_OK) return rc;
+    return cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s));
+  }
   rc = cuda_status(omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate,
                                          w.uniq, w.group_off, counts, w.sched, s));
   if (rc != OMNI_OK) return rc;

@@ -12,26 +12,28 @@ constexpr int kBlockSortThreads = 1024;  // threads of a CTA that sorts
 constexpr int kBlockSortWarps = kBlockSortThreads / 32;
 constexpr int kBlockSortRounds = kBlockSortMax / kBlockSortThreads;  // 32-key rounds per warp
 
-// Exclusive prefix sum of v over the threads of the block (any blockDim that
-// is a multiple of 32, up to 1024); *total receives the block's sum.
-// warp_tot: 32 ints of shared memory.  Every thread of the block must call it.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+// Exclusive prefix sum of v (int or a 64-bit unsigned) over the threads of
+// the block (any blockDim that is a multiple of 32, up to 1024); *total
+// receives the block's sum.  warp_tot: 32 values of shared memory.  Every
+// thread of the block must call it.
+template <typename V>
+__device__ __forceinline__ V block_exclusive_scan(V v, V* warp_tot, V* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+  V incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    const V u = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += u;
   }
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
     const int nw = blockDim.x >> 5;
-    int w = lane < nw ? warp_tot[lane] : 0;
-    int wi = w;
+    V w = lane < nw ? warp_tot[lane] : V(0);
+    V wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      const V u = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += u;
     }
     if (lane < nw) warp_tot[lane] = wi - w;

@@ -653,6 +653,75 @@ __global__ void __launch_bounds__(kBlockSortThreads)
   }
 }
 
+// The same window orders when the tasks already arrive in window token order
+// (wt/we/wg, windows [win_lo[w], win_lo[w+1])): only the stable sort by
+// expert is left.  Windows larger than the CTA sort keep token order.
+__global__ void __launch_bounds__(kBlockSortThreads)
+    k_wsort_x(const int32_t* __restrict__ win_lo, WinOut o) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) uint8_t wsm[];
+  uint32_t* kA = reinterpret_cast<uint32_t*>(wsm);
+  uint32_t* kB = kA + kBlockSortMax;
+  uint16_t* vA = reinterpret_cast<uint16_t*>(kB + kBlockSortMax);
+  uint16_t* vB = vA + kBlockSortMax;
+  uint32_t* wcount = reinterpret_cast<uint32_t*>(vB + 2 * kBlockSortMax);
+  __shared__ uint32_t dbase[256];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int emin, emax;
+  const int64_t a0 = win_lo[blockIdx.x];
+  const int64_t n = win_lo[blockIdx.x + 1] - a0;
+  if (n <= 0) return;
+  if (n > kBlockSortMax) {
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+      o.xt[a0 + i] = o.wt[a0 + i];
+      o.xe[a0 + i] = o.we[a0 + i];
+      o.xg[a0 + i] = o.wg[a0 + i];
+      o.xdst[a0 + i] = static_cast<int32_t>(a0 + i);
+    }
+    return;
+  }
+  if (threadIdx.x == 0) {
+    emin = INT_MAX;
+    emax = INT_MIN;
+  }
+  __syncthreads();
+  const int nn = static_cast<int>(n);
+  int lmin = INT_MAX, lmax = INT_MIN;
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const int e = o.we[a0 + i];
+    lmin = e < lmin ? e : lmin;
+    lmax = e > lmax ? e : lmax;
+  }
+  atomicMin(&emin, lmin);
+  atomicMax(&emax, lmax);
+  __syncthreads();
+  const int64_t span = static_cast<int64_t>(emax) - emin;
+  int ebits = 0;
+  while (ebits < 32 && (int64_t(1) << ebits) <= span) ++ebits;
+  const int epasses = (ebits + 7) / 8;
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    kA[i] = static_cast<uint32_t>(o.we[a0 + i] - emin);
+    vA[i] = static_cast<uint16_t>(i);
+  }
+  __syncthreads();
+  uint32_t* kin = kA; uint32_t* kout = kB;
+  uint16_t* vin = vA; uint16_t* vout = vB;
+  for (int p = 0; p < epasses; ++p) {
+    block_radix_pass(kin, vin, kout, vout, nn, 8 * p, wcount, dbase, warp_tot, &total);
+    uint32_t* tk = kin; kin = kout; kout = tk;
+    uint16_t* tv = vin; vin = vout; vout = tv;
+  }
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const int src = vin[i];
+    o.xt[a0 + i] = o.wt[a0 + src];
+    o.xe[a0 + i] = o.we[a0 + src];
+    o.xg[a0 + i] = o.wg[a0 + src];
+    o.xdst[a0 + i] = static_cast<int32_t>(a0 + src);
+  }
+}
+
 constexpr int kAccWarps = 4;
 
 // Four consecutive elements of T as one load: bf16 -> 8 bytes, fp32 -> 16 bytes.
@@ -926,6 +995,7 @@ int expert_sweeps(const Dims& D) {
 struct SweepWs {
   float* cbuf;
   WinOut win;
+  int32_t* win_lo;  // [nwin + 1] window starts, when the tasks come in window order
 };
 
 size_t acc_bytes(const Dims& D) {
@@ -945,6 +1015,8 @@ SweepWs carve_sweeps(const Dims& D, void* ws, size_t* bytes) {
   w.win.xe = c.take<int32_t>(M);
   w.win.xg = c.take<float>(M);
   w.win.xdst = c.take<int32_t>(M);
+  const int64_t T = window_tasks(D);
+  w.win_lo = c.take<int32_t>(static_cast<size_t>((D.M() + T - 1) / T) + 1);
   if (bytes) *bytes = c.off;
   return w;
 }
@@ -1022,19 +1094,35 @@ int sm_count() {
   return sms;
 }
 
+// about one window per SM, within what one CTA sorts
+int64_t window_tasks(const Dims& D) {
+  const int64_t T = (D.M() + sm_count() - 1) / sm_count();
+  return T < 1024 ? 1024 : (T > kWinTasks ? kWinTasks : T);
+}
+
+constexpr size_t kWsortSmem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 3 * 2) +
+                              static_cast<size_t>(kBlockSortWarps) * 256 * 4;
+
+// win_lo != nullptr: the tasks are in window token order already (wt/we/wg),
+// and only the expert order is left to make
 cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, const float* tg,
                          const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                         int32_t* status, cudaStream_t s) {
-  constexpr size_t smem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 3 * 2) +
-                          static_cast<size_t>(kBlockSortWarps) * 256 * 4;
+                         const int32_t* win_lo, int32_t* status, cudaStream_t s) {
+  const int64_t M = D.M();
+  const int64_t T = window_tasks(D);
+  const int64_t nwin = (M + T - 1) / T;
+  if (win_lo != nullptr) {
+    cudaError_t err = cudaFuncSetAttribute(k_wsort_x, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kWsortSmem));
+    if (err != cudaSuccess) return err;
+    OMNI_TRY(launch_k(k_wsort_x, static_cast<unsigned>(nwin), kBlockSortThreads, kWsortSmem, s,
+        win_lo, w.win));
+    return cudaGetLastError();
+  }
+  constexpr size_t smem = kWsortSmem;
   cudaError_t err = cudaFuncSetAttribute(k_wsort, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int64_t M = D.M();
-  // about one window per SM, within what one CTA sorts
-  int64_t T = (M + sm_count() - 1) / sm_count();
-  T = T < 1024 ? 1024 : (T > kWinTasks ? kWinTasks : T);
-  const int64_t nwin = (M + T - 1) / T;
   int bits = 0;
   while ((int64_t(1) << bits) < D.L) ++bits;
   const int passes = (bits + 7) / 8;
@@ -1076,8 +1164,9 @@ template <typename T, int NV, int NVQ>
 cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const void* V,
                       const int32_t* tt, const int32_t* te, const float* tg,
                       const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                      float* acc, __nv_bfloat16* ycast, int32_t* status, cudaStream_t s) {
-  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, status, s);
+                      const int32_t* win_lo, float* acc, __nv_bfloat16* ycast, int32_t* status,
+                      cudaStream_t s) {
+  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, win_lo, status, s);
   if (err != cudaSuccess) return err;
   // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
   constexpr int R = 3;
@@ -1123,15 +1212,16 @@ template <typename T>
 cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, const void* V,
                           const int32_t* tt, const int32_t* te, const float* tg,
                           const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                          float* acc, __nv_bfloat16* ycast, int32_t* status, cudaStream_t s) {
+                          const int32_t* win_lo, float* acc, __nv_bfloat16* ycast,
+                          int32_t* status, cudaStream_t s) {
   constexpr int row = 32 * kEpv<T>;
   const int64_t nv = D.d / row;             // vectors per lane for a whole row
   const int64_t nvq = (D.d / Q) / row;      // ... for one slice
   if (D.d % row != 0) return cudaErrorInvalidValue;
 #define OMNI_SWEEP(NV_, NVQ_)                                                               \
   if (nv == NV_ && nvq == NVQ_)                                                             \
-    return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, group_off, counts, w, acc,    \
-                                   ycast, status, s);
+    return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, group_off, counts, w, win_lo, \
+                                   acc, ycast, status, s);
   OMNI_SWEEP(8, 4) OMNI_SWEEP(8, 2) OMNI_SWEEP(8, 1) OMNI_SWEEP(4, 2) OMNI_SWEEP(4, 1)
   OMNI_SWEEP(2, 1)
 #undef OMNI_SWEEP
@@ -1151,9 +1241,10 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
     const SweepWs w = carve_sweeps(D, ws, nullptr);
     __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
     return f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate,
-                                      group_off, counts, w, acc, ycast, status, s)
+                                      group_off, counts, w, nullptr, acc, ycast, status, s)
                : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
-                                              group_off, counts, w, acc, ycast, status, s);
+                                              group_off, counts, w, nullptr, acc, ycast, status,
+                                              s);
   }
   const size_t ybytes = static_cast<size_t>(D.L) * D.d * sizeof(float);
   cudaError_t err = launch_zero(acc, ybytes / sizeof(float), s);
@@ -1166,6 +1257,26 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,
       static_cast<__nv_bfloat16*>(y), n));
   return cudaGetLastError();
+}
+
+WinTasks expert_windows(const Dims& D, void* ws) {
+  const SweepWs w = carve_sweeps(D, ws, nullptr);
+  return WinTasks{w.win.wt, w.win.we, w.win.wg, w.win_lo};
+}
+
+cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, const void* V,
+                                  int32_t* counts, void* y, void* ws, cudaStream_t s) {
+  const int Q = expert_sweeps(D);
+  if (D.L == 0 || Q <= 1) return cudaErrorInvalidValue;
+  const bool f32 = D.dtype == OMNI_F32;
+  float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
+  int32_t* status = counts + 2;
+  const SweepWs w = carve_sweeps(D, ws, nullptr);
+  __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
+  return f32 ? launch_sweeps<float>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr, counts, w,
+                                    w.win_lo, acc, ycast, status, s)
+             : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr,
+                                            counts, w, w.win_lo, acc, ycast, status, s);
 }
 
 namespace {

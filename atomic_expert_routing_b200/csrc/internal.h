@@ -37,8 +37,25 @@ cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float*
                           const float* bc, int32_t* idx, float* gate, float* score,
                           cudaStream_t s);
 
+// ---- windows of consecutive groups (the sweep path of the execution) ------
+// Window w holds the groups whose first task lies in [w*T, (w+1)*T).
+int64_t window_tasks(const Dims& D);  // T
+struct WinTasks {
+  int32_t *wt, *we;  // token and expert of every task, in window token order
+  float* wg;         // its gate
+  int32_t* win_lo;   // [nwin + 1] first task of every window
+};
+
 // ---- scheduling ----------------------------------------------------------
 size_t schedule_ws_bytes(const Dims& D);
+// The fused forward of a large batch: the schedule's ranks, U, counts and
+// group offsets, then every task straight into window token order (the
+// (group, token) order of omni_schedule is never formed).
+bool windows_supported(const Dims& D);
+size_t windows_ws_bytes(const Dims& D);
+cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const float* gate,
+                                    int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
+                                    const WinTasks& out, cudaStream_t s);
 cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate,
                             int32_t* task_token, int32_t* task_expert, float* task_gate,
                             int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
@@ -46,6 +63,11 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
 
 // ---- execution -----------------------------------------------------------
 size_t expert_ws_bytes(const Dims& D);
+int expert_sweeps(const Dims& D);                // slices of d (1: no sweeps)
+WinTasks expert_windows(const Dims& D, void* ws);  // the window buffers of an expert workspace
+// The sweeps from tasks already in window token order (expert_windows(ws)).
+cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, const void* V,
+                                  int32_t* counts, void* y, void* ws, cudaStream_t s);
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* group_off,

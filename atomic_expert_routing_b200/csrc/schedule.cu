@@ -9,17 +9,19 @@
 //
 // Steps (all on `stream`, data-dependent counts stay on the device):
 //  1. prep    one warp per token sorts its K (expert, gate) pairs by expert
-//             id, so the task list is in (token, expert) order, and flags
-//             every active expert in an N-long array;
-//  2. scan    exclusive prefix sum of the flags gives each active expert its
-//             rank in U (sorted unique ids), U itself, |U| and the group
-//             count ceil(|U| / B);
+//             id, so the task list is in (token, expert) order, and counts
+//             the tasks of every expert in an N-long array;
+//  2. scan    one exclusive prefix sum over the ids of (active, tasks) gives
+//             each active expert its rank in U (sorted unique ids), U itself,
+//             |U|, the group count ceil(|U| / B) and every group's first task;
 //  3. sort    stable LSD radix sort of the tasks by group = rank / B with
 //             8-bit digits (as many passes as the group-count bound needs),
 //             one kernel per pass (decoupled look-back over tiles) after one
 //             histogram kernel for all passes; stability keeps (token,
 //             expert) order inside each group;
-//  4. emit    gather the sorted tasks and mark each group's first task.
+//  4. emit    gather the sorted tasks.
+// The fused forward of a large batch replaces 3-4 by the window order its
+// expert stage consumes (launch_schedule_windows, at the end of this file).
 #include <cooperative_groups.h>
 
 #include "blocksort.cuh"
@@ -41,14 +43,14 @@ constexpr int kRsWarps = kRsThreads / 32;
 constexpr int kRsPerWarp = 512;  // consecutive tasks per warp in a tile
 constexpr int kRsTile = kRsWarps * kRsPerWarp;
 
-// ---- 1. per-token sort by expert id + active flags -----------------------
+// ---- 1. per-token sort by expert id + task counts ------------------------
 // One warp per token: its K (expert, slot) keys sorted ascending in registers
-// (32*W >= K; a descending network over complemented keys), the experts
-// flagged as active.
+// (32*W >= K; a descending network over complemented keys); mult[e] counts
+// the tasks of expert e (active: mult > 0).
 template <int W>
 __global__ void __launch_bounds__(kPrepWarps * 32)
     k_prep(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t L, int K,
-           int64_t N, int32_t* __restrict__ flags, int32_t* __restrict__ tmp_e,
+           int64_t N, int32_t* __restrict__ mult, int32_t* __restrict__ tmp_e,
            float* __restrict__ tmp_g, int32_t* status) {
   pdl_wait();
   pdl_trigger();
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
         raise_status(status, OMNI_DEV_BAD_INDEX);
         e = 0;
       }
-      flags[e] = 1;
+      atomicAdd(&mult[e], 1);
       key[w] = ~((static_cast<uint64_t>(e) << 32) | static_cast<uint32_t>(q));
     }
   }
@@ -82,72 +84,88 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
   }
 }
 
-// ---- 2. scan of the active flags ------------------------------------------
+// ---- 2. scan of the (active, task count) pairs over the ids ----------------
+// A 64-bit item packs (active ids) << 32 | (tasks): both sums stay below 2^31,
+// so one 64-bit scan carries both.  The rank of an id is the active ids
+// before it; the first task of group g is the task count before the id of
+// rank g * B.
+__device__ __forceinline__ uint64_t mult_item(int32_t m) {
+  return m > 0 ? ((uint64_t(1) << 32) | static_cast<uint32_t>(m)) : 0ull;
+}
+
 __global__ void __launch_bounds__(kScanThreads)
-    k_scan_reduce(const int32_t* __restrict__ flags, int64_t N, int32_t* __restrict__ tile_sum) {
+    k_scan_reduce(const int32_t* __restrict__ mult, int64_t N, uint64_t* __restrict__ tile_sum) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int warp_tot[32];
-  __shared__ int total;
+  __shared__ uint64_t warp_tot[32];
+  __shared__ uint64_t total;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
-  int v = 0;
+  uint64_t v = 0;
 #pragma unroll
   for (int j = 0; j < kScanItems; ++j)
-    if (base + j < N) v += flags[base + j];
+    if (base + j < N) v += mult_item(mult[base + j]);
   block_exclusive_scan(v, warp_tot, &total);
   if (threadIdx.x == 0) tile_sum[blockIdx.x] = total;
 }
 
 // single block: exclusive scan of the tile sums; counts[0] = |U|, counts[1] = groups
 __global__ void __launch_bounds__(kScanThreads)
-    k_scan_tiles(int32_t* __restrict__ tile_sum, int ntiles, int64_t B, int32_t* counts) {
+    k_scan_tiles(uint64_t* __restrict__ tile_sum, int ntiles, int64_t B, int32_t* counts) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int warp_tot[32];
-  __shared__ int total;
-  __shared__ int carry;
+  __shared__ uint64_t warp_tot[32];
+  __shared__ uint64_t total;
+  __shared__ uint64_t carry;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int c0 = 0; c0 < ntiles; c0 += kScanThreads) {
     const int i = c0 + threadIdx.x;
-    const int v = i < ntiles ? tile_sum[i] : 0;
-    const int ex = block_exclusive_scan(v, warp_tot, &total);
+    const uint64_t v = i < ntiles ? tile_sum[i] : 0ull;
+    const uint64_t ex = block_exclusive_scan(v, warp_tot, &total);
     if (i < ntiles) tile_sum[i] = carry + ex;
     __syncthreads();
     if (threadIdx.x == 0) carry += total;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    counts[0] = carry;
-    counts[1] = static_cast<int32_t>((carry + B - 1) / B);
+    const int64_t n_active = static_cast<int64_t>(carry >> 32);
+    counts[0] = static_cast<int32_t>(n_active);
+    counts[1] = static_cast<int32_t>((n_active + B - 1) / B);
   }
 }
 
+// rank[e], U, and group_off (every group start; group_off[G] = M)
 __global__ void __launch_bounds__(kScanThreads)
-    k_scan_finish(const int32_t* __restrict__ flags, int64_t N,
-                  const int32_t* __restrict__ tile_off, int32_t* __restrict__ rank,
-                  int32_t* __restrict__ uniq) {
+    k_scan_finish(const int32_t* __restrict__ mult, int64_t N,
+                  const uint64_t* __restrict__ tile_off, int64_t B, int64_t M,
+                  const int32_t* __restrict__ counts, int32_t* __restrict__ rank,
+                  int32_t* __restrict__ uniq, int32_t* __restrict__ group_off) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int warp_tot[32];
-  __shared__ int total;
+  __shared__ uint64_t warp_tot[32];
+  __shared__ uint64_t total;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kScanTile + threadIdx.x * kScanItems;
-  int f[kScanItems];
-  int v = 0;
+  uint64_t f[kScanItems];
+  uint64_t v = 0;
 #pragma unroll
   for (int j = 0; j < kScanItems; ++j) {
-    f[j] = (base + j < N) ? flags[base + j] : 0;
+    f[j] = (base + j < N) ? mult_item(mult[base + j]) : 0ull;
     v += f[j];
   }
-  int r = block_exclusive_scan(v, warp_tot, &total) + tile_off[blockIdx.x];
+  uint64_t r = block_exclusive_scan(v, warp_tot, &total) + tile_off[blockIdx.x];
 #pragma unroll
   for (int j = 0; j < kScanItems; ++j) {
     if (base + j < N) {
-      rank[base + j] = r;
-      if (f[j]) uniq[r] = static_cast<int32_t>(base + j);
+      const int64_t rk = static_cast<int64_t>(r >> 32);
+      rank[base + j] = static_cast<int32_t>(rk);
+      if (f[j] != 0ull) {
+        uniq[rk] = static_cast<int32_t>(base + j);
+        if (rk % B == 0) group_off[rk / B] = static_cast<int32_t>(r & 0xffffffffull);
+      }
     }
     r += f[j];
   }
+  if (blockIdx.x == 0 && threadIdx.x == 0) group_off[counts[1]] = static_cast<int32_t>(M);
 }
 
 // ---- 3. stable radix sort by group id ---------------------------------------
@@ -295,22 +313,18 @@ __global__ void __launch_bounds__(kRsThreads)
 
 // ---- 4. emit ---------------------------------------------------------------
 __global__ void __launch_bounds__(256)
-    k_emit(const uint32_t* __restrict__ keys, const uint32_t* __restrict__ vals, int64_t M, int K,
+    k_emit(const uint32_t* __restrict__ vals, int64_t M, int K,
            const int32_t* __restrict__ tmp_e, const float* __restrict__ tmp_g,
            int32_t* __restrict__ task_token, int32_t* __restrict__ task_expert,
-           float* __restrict__ task_gate, int32_t* __restrict__ group_off,
-           const int32_t* __restrict__ counts) {
+           float* __restrict__ task_gate) {
   pdl_wait();
   pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= M) return;
   const uint32_t pos = vals ? vals[i] : static_cast<uint32_t>(i);
-  const uint32_t g = keys ? keys[i] : 0u;
   task_token[i] = static_cast<int32_t>(pos / static_cast<uint32_t>(K));
   task_expert[i] = tmp_e[pos];
   task_gate[i] = tmp_g[pos];
-  if (i == 0 || (keys ? keys[i - 1] : 0u) != g) group_off[g] = static_cast<int32_t>(i);
-  if (i == M - 1) group_off[counts[1]] = static_cast<int32_t>(M);
 }
 
 // ---- small batches (M <= kSmallMax): the whole schedule in one cluster -------
@@ -842,8 +856,10 @@ cudaError_t launch_bits(const Dims& D, const CbPlan& p, const int32_t* idx, cons
 }
 
 struct SchedWs {
-  int32_t *flags, *rank, *tile_sum, *tmp_e;
+  int32_t *mult, *rank, *tmp_e;
+  uint64_t* tile_sum;
   float* tmp_g;
+  int32_t* cnt;  // windows: [nwin][L] tasks per (window, token)
   uint32_t *ka, *va, *kb, *vb, *sweep;  // sweep: [passes][256] histogram, [passes] tile
                                         // counters, [passes][ntiles][256] look-back words
   size_t sweep_words;
@@ -851,11 +867,13 @@ struct SchedWs {
   int passes;
 };
 
-SchedWs carve(const Dims& D, void* base, size_t* bytes) {
+// windows: the scratch of launch_schedule_windows (no radix buffers; the
+// (window, token) counts instead)
+SchedWs carve(const Dims& D, void* base, size_t* bytes, bool windows = false) {
   Carver c(base);
   SchedWs w{};
   const int64_t N = D.N(), M = D.M();
-  if (M <= kSmallMax) {  // the single-CTA path works in shared memory only
+  if (M <= kSmallMax && !windows) {  // the cluster paths work in shared memory only
     if (bytes) *bytes = 0;
     return w;
   }
@@ -864,12 +882,15 @@ SchedWs carve(const Dims& D, void* base, size_t* bytes) {
   int bits = 0;
   while ((int64_t(1) << bits) < D.gmax()) ++bits;
   w.passes = (bits + 7) / 8;
-  w.flags = c.take<int32_t>(N);
+  w.mult = c.take<int32_t>(N);
   w.rank = c.take<int32_t>(N);
-  w.tile_sum = c.take<int32_t>(w.nscan + 1);
+  w.tile_sum = c.take<uint64_t>(w.nscan + 1);
   w.tmp_e = c.take<int32_t>(M);
   w.tmp_g = c.take<float>(M);
-  if (w.passes > 0) {
+  if (windows) {
+    const int64_t T = window_tasks(D);
+    w.cnt = c.take<int32_t>(static_cast<size_t>((M + T - 1) / T) * D.L);
+  } else if (w.passes > 0) {
     w.ka = c.take<uint32_t>(M);
     w.va = c.take<uint32_t>(M);
     w.kb = c.take<uint32_t>(M);
@@ -879,6 +900,183 @@ SchedWs carve(const Dims& D, void* base, size_t* bytes) {
   }
   if (bytes) *bytes = c.off;
   return w;
+}
+
+// zero the task counts, sort every token's tasks, scan the counts: ranks,
+// U, |U|, G and the group offsets
+cudaError_t prep_and_scan(const Dims& D, const int32_t* idx, const float* gate, int32_t* uniq,
+                          int32_t* group_off, int32_t* counts, const SchedWs& w, cudaStream_t s) {
+  const int64_t N = D.N();
+  int32_t* status = counts + 2;
+  cudaError_t err = launch_zero(w.mult, static_cast<size_t>(N), s);
+  if (err != cudaSuccess) return err;
+  const unsigned prep_blocks = static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps);
+  auto prep = [&](auto kern) {
+    return launch_k(kern, prep_blocks, kPrepWarps * 32, 0, s, idx, gate, D.L,
+                    static_cast<int>(D.K), N, w.mult, w.tmp_e, w.tmp_g, status);
+  };
+  OMNI_TRY(D.K <= 32 ? prep(k_prep<1>) : D.K <= 64 ? prep(k_prep<2>)
+           : D.K <= 128 ? prep(k_prep<4>) : prep(k_prep<8>));
+  OMNI_TRY(launch_k(k_scan_reduce, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.mult, N,
+      w.tile_sum));
+  OMNI_TRY(launch_k(k_scan_tiles, 1, kScanThreads, 0, s, w.tile_sum, static_cast<int>(w.nscan), D.B,
+      counts));
+  OMNI_TRY(launch_k(k_scan_finish, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.mult, N,
+      w.tile_sum, D.B, D.M(), static_cast<const int32_t*>(counts), w.rank, uniq, group_off));
+  return cudaGetLastError();
+}
+
+// ---- the fused forward's windows: the tasks in window token order --------
+//
+// Window w holds the groups whose first task lies in [w*T, (w+1)*T); the
+// expert stage wants its tasks by token, a token's tasks by expert.  A
+// token's tasks, sorted by expert, visit the windows in order, so the tasks
+// of one (window, token) pair are consecutive in its list.  cnt[w][t] counts
+// them; scanned along t it gives the pair's first position inside the
+// window, whose own first position is its first group's.  The order equals
+// that of a stable sort by token of the window's tasks in schedule order.
+constexpr int64_t kWinCellsMax = int64_t(1) << 23;  // nwin * L
+
+// win_lo[w] = first task of window w (M when it has no group); win_lo[nwin] = M
+__global__ void __launch_bounds__(256)
+    k_winbase(const int32_t* __restrict__ group_off, const int32_t* __restrict__ counts, int64_t M,
+              int64_t T, int nwin, int32_t* __restrict__ win_lo) {
+  pdl_wait();
+  pdl_trigger();
+  const int w = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (w > nwin) return;
+  if (w == nwin) {
+    win_lo[w] = static_cast<int32_t>(M);
+    return;
+  }
+  const int64_t G = counts[1];
+  const int64_t v = static_cast<int64_t>(w) * T;
+  int64_t lo = 0, hi = G;  // first group starting at or after v
+  while (lo < hi) {
+    const int64_t m = (lo + hi) >> 1;
+    if (group_off[m] >= v) hi = m; else lo = m + 1;
+  }
+  win_lo[w] = lo < G ? group_off[lo] : static_cast<int32_t>(M);
+}
+
+// Token t's task j (sorted by expert): its window, and the index of the first
+// task of its (window, token) run.  One warp per token, element j = w*32 + lane.
+template <int W>
+__device__ __forceinline__ void token_windows(const int32_t* __restrict__ tmp_e,
+                                              const int32_t* __restrict__ rank,
+                                              const int32_t* __restrict__ group_off, int64_t t,
+                                              int K, int64_t B, int64_t T, int (&win)[W],
+                                              int (&first)[W], uint32_t (&last)[W]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int j = w * 32 + lane;
+    win[w] = -1;
+    if (j < K) {
+      const int32_t e = tmp_e[t * K + j];
+      const int64_t g = rank[e] / B;
+      win[w] = static_cast<int>(group_off[g] / T);
+    }
+  }
+  int carry = 0;
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int j = w * 32 + lane;
+    const int row_prev = __shfl_sync(0xffffffffu, win[w > 0 ? w - 1 : 0], 31);
+    const int row_next = __shfl_sync(0xffffffffu, win[w + 1 < W ? w + 1 : W - 1], 0);
+    int wp = __shfl_up_sync(0xffffffffu, win[w], 1);
+    int wn = __shfl_down_sync(0xffffffffu, win[w], 1);
+    if (w > 0 && lane == 0) wp = row_prev;
+    if (w + 1 < W && lane == 31) wn = row_next;
+    int f = (j == 0 || wp != win[w]) ? j : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, f, o);
+      if (lane >= o) f = x > f ? x : f;
+    }
+    f = f > carry ? f : carry;
+    carry = __shfl_sync(0xffffffffu, f, 31);
+    first[w] = f;
+    last[w] = (j < K && (j == K - 1 || wn != win[w])) ? 1u : 0u;
+  }
+}
+
+template <int W>
+__global__ void __launch_bounds__(kPrepWarps * 32)
+    k_wincount(const int32_t* __restrict__ tmp_e, const int32_t* __restrict__ rank,
+               const int32_t* __restrict__ group_off, int64_t L, int K, int64_t B, int64_t T,
+               int32_t* __restrict__ cnt) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp;
+  if (t >= L) return;  // warp-uniform
+  int win[W], first[W];
+  uint32_t last[W];
+  token_windows<W>(tmp_e, rank, group_off, t, K, B, T, win, first, last);
+#pragma unroll
+  for (int w = 0; w < W; ++w)
+    if (last[w]) cnt[static_cast<int64_t>(win[w]) * L + t] = w * 32 + lane - first[w] + 1;
+}
+
+// one CTA per window: exclusive scan of its row of L counts, in place
+__global__ void __launch_bounds__(kScanThreads) k_rowscan(int32_t* __restrict__ cnt, int64_t L) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  int32_t* row = cnt + static_cast<int64_t>(blockIdx.x) * L;
+  int carry = 0;
+  for (int64_t b0 = 0; b0 < L; b0 += kScanTile) {
+    const int64_t base = b0 + threadIdx.x * kScanItems;
+    int v[kScanItems];
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < kScanItems; ++j) {
+      v[j] = base + j < L ? row[base + j] : 0;
+      sum += v[j];
+    }
+    int run = carry + block_exclusive_scan(sum, warp_tot, &total);
+#pragma unroll
+    for (int j = 0; j < kScanItems; ++j) {
+      if (base + j < L) row[base + j] = run;
+      run += v[j];
+    }
+    carry += total;
+    __syncthreads();  // total is rewritten by the next chunk's scan
+  }
+}
+
+template <int W>
+__global__ void __launch_bounds__(kPrepWarps * 32)
+    k_winscatter(const int32_t* __restrict__ tmp_e, const float* __restrict__ tmp_g,
+                 const int32_t* __restrict__ rank, const int32_t* __restrict__ group_off,
+                 const int32_t* __restrict__ win_lo, const int32_t* __restrict__ cnt, int64_t L,
+                 int K, int64_t B, int64_t T, int64_t M, int32_t* __restrict__ wt,
+                 int32_t* __restrict__ we, float* __restrict__ wg, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kPrepWarps + warp;
+  if (t >= L) return;  // warp-uniform
+  int win[W], first[W];
+  uint32_t last[W];
+  token_windows<W>(tmp_e, rank, group_off, t, K, B, T, win, first, last);
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    const int j = w * 32 + lane;
+    if (j < K) {
+      const int64_t pos = static_cast<int64_t>(win_lo[win[w]]) +
+                          cnt[static_cast<int64_t>(win[w]) * L + t] + (j - first[w]);
+      if (pos < 0 || pos >= M) {  // unreachable for consistent counts; never write outside
+        raise_status(status, OMNI_DEV_BAD_INDEX);
+        continue;
+      }
+      wt[pos] = static_cast<int32_t>(t);
+      we[pos] = tmp_e[t * K + j];
+      wg[pos] = tmp_g[t * K + j];
+    }
+  }
 }
 
 }  // namespace
@@ -926,22 +1124,7 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     return cudaGetLastError();
   }
   SchedWs w = carve(D, ws, nullptr);
-  cudaError_t err = launch_zero(w.flags, static_cast<size_t>(N), s);
-  if (err != cudaSuccess) return err;
-  const unsigned prep_blocks = static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps);
-  auto prep = [&](auto kern) {
-    return launch_k(kern, prep_blocks, kPrepWarps * 32, 0, s, idx, gate, D.L,
-                    static_cast<int>(D.K), N, w.flags, w.tmp_e, w.tmp_g, status);
-  };
-  OMNI_TRY(D.K <= 32 ? prep(k_prep<1>) : D.K <= 64 ? prep(k_prep<2>)
-           : D.K <= 128 ? prep(k_prep<4>) : prep(k_prep<8>));
-  OMNI_TRY(launch_k(k_scan_reduce, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.flags, N,
-      w.tile_sum));
-  OMNI_TRY(launch_k(k_scan_tiles, 1, kScanThreads, 0, s, w.tile_sum, static_cast<int>(w.nscan), D.B,
-      counts));
-  OMNI_TRY(launch_k(k_scan_finish, static_cast<unsigned>(w.nscan), kScanThreads, 0, s, w.flags, N,
-      w.tile_sum, w.rank, uniq));
-  err = cudaGetLastError();
+  cudaError_t err = prep_and_scan(D, idx, gate, uniq, group_off, counts, w, s);
   if (err != cudaSuccess) return err;
   const uint32_t* keys = nullptr;
   const uint32_t* vals = nullptr;
@@ -968,9 +1151,52 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  OMNI_TRY(launch_k(k_emit, static_cast<unsigned>((M + 255) / 256), 256, 0, s, keys, vals, M,
-      static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate, group_off,
-      counts));
+  OMNI_TRY(launch_k(k_emit, static_cast<unsigned>((M + 255) / 256), 256, 0, s, vals, M,
+      static_cast<int>(D.K), w.tmp_e, w.tmp_g, task_token, task_expert, task_gate));
+  return cudaGetLastError();
+}
+
+size_t windows_ws_bytes(const Dims& D) {
+  size_t b = 0;
+  carve(D, nullptr, &b, true);
+  return b;
+}
+
+bool windows_supported(const Dims& D) {
+  const int64_t T = window_tasks(D);
+  const int64_t nwin = (D.M() + T - 1) / T;
+  return D.M() > 0 && nwin * D.L <= kWinCellsMax && D.K <= 256;
+}
+
+cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const float* gate,
+                                    int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
+                                    const WinTasks& out, cudaStream_t s) {
+  const int64_t M = D.M();
+  const int64_t T = window_tasks(D);
+  const int nwin = static_cast<int>((M + T - 1) / T);
+  SchedWs w = carve(D, ws, nullptr, true);
+  cudaError_t err = prep_and_scan(D, idx, gate, uniq, group_off, counts, w, s);
+  if (err != cudaSuccess) return err;
+  err = launch_zero(w.cnt, static_cast<size_t>(nwin) * D.L, s);
+  if (err != cudaSuccess) return err;
+  OMNI_TRY(launch_k(k_winbase, static_cast<unsigned>((nwin + 1 + 255) / 256), 256, 0, s, group_off,
+      counts, M, T, nwin, out.win_lo));
+  const unsigned blocks = static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps);
+  const int K = static_cast<int>(D.K);
+  auto count = [&](auto kern) {
+    return launch_k(kern, blocks, kPrepWarps * 32, 0, s, w.tmp_e, w.rank, group_off, D.L, K, D.B,
+                    T, w.cnt);
+  };
+  OMNI_TRY(K <= 32 ? count(k_wincount<1>) : K <= 64 ? count(k_wincount<2>)
+           : K <= 128 ? count(k_wincount<4>) : count(k_wincount<8>));
+  OMNI_TRY(launch_k(k_rowscan, static_cast<unsigned>(nwin), kScanThreads, 0, s, w.cnt, D.L));
+  auto scatter = [&](auto kern) {
+    return launch_k(kern, blocks, kPrepWarps * 32, 0, s, w.tmp_e, w.tmp_g, w.rank, group_off,
+                    static_cast<const int32_t*>(out.win_lo), static_cast<const int32_t*>(w.cnt),
+                    D.L, K, D.B, T, M, out.wt, out.we, out.wg, counts + 2);
+  };
+  OMNI_TRY(K <= 32 ? scatter(k_winscatter<1>) : K <= 64 ? scatter(k_winscatter<2>)
+           : K <= 128 ? scatter(k_winscatter<4>) : scatter(k_winscatter<8>));
   return cudaGetLastError();
 }
 

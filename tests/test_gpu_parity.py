@@ -429,6 +429,27 @@ def test_expert_sweeps_path(cfg):
     assert int(counts[2].item()) == 0
 
 
+@pytest.mark.parametrize("cfg", SWEEP, ids=[c.name for c in SWEEP])
+def test_fused_sweeps_path(cfg):
+    """The fused forward of a sweep-sized batch goes from the routing straight
+    to the window order of the sweeps: same y as the oracle's expert-centric
+    execution of the routing it chose, same |U| and group count."""
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    D = omni.LayerDims.of(cfg)
+    idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
+    counts = omni.new_counts("cuda")
+    y = omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"],
+                         counts=counts, idx=idx, gate=gate)
+    gi = idx.cpu().numpy()
+    ref_s = O.schedule(cfg, gi, gate.cpu().numpy().astype(np.float64))
+    y_ref, _ = O.forward_expert(cfg, h, ref_s)
+    c = counts.cpu().numpy()
+    assert c[0] == ref_s["n_active"] and c[1] == ref_s["n_groups"] and c[2] == 0
+    assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
+
+
 def test_expert_sweeps_bad_group_count():
     """A group count on the device above its bound: the executor flags it
     (OMNI_DEV_BAD_INDEX) and still executes every task once, in schedule order."""
