@@ -165,8 +165,7 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 // Top `want` (<= 32*W) of the n keys make_key(value, id) held by a group of
 // NW warps (gw: this warp's index in the group, bar_id: the group's named
 // barrier), by (value desc, id asc), written sorted to out[0 .. 32*W)
-// (padded with 0) by the group's warp 0 -- the other warps must synchronise
-// with it before reading out.
+// (padded with 0); out is complete for every warp of the group on return.
 //
 // for_each(f) calls f(value, id) for every element of the calling thread (in
 // any order; elements are split over the group's threads), key_at(i) gives
@@ -175,11 +174,13 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 // value: bin(v) = floor((v - lo) * 256 / (hi - lo)) is monotone in v, so
 // every key in a bin above the threshold bin is selected and equal values
 // share a bin.  A 256-bin histogram (shared-memory atomics) finds the
-// threshold bin; keys above it are compacted through an atomic counter
-// (about want of n), the threshold bin's keys (at most kCandMax) are sorted
-// in registers for the remainder, and the want keys are sorted in registers.
-// A threshold bin that is too full, or a non-finite range, falls back to the
-// radix select.  hist: 256 words; tbk: kCandMax keys; cnt: 2 words.
+// threshold bin; the histogram, scanned from the top bin down, gives every
+// bin at or above it its first output position, and each of those keys
+// (about want of n, the threshold bin at most kCandMax) is placed at its
+// bin's position plus the number of larger keys of its bin: the output is
+// sorted without a sorting network.  A threshold bin that is too full, or a
+// non-finite range, falls back to the radix select.  hist: 256 words; tbk:
+// kCandMax keys; cnt: 2 words.
 template <int W, int NW, typename ForEach, typename Prepare, typename KeyAt>
 __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare, KeyAt key_at,
                            int n, int want, float lo, float hi, uint64_t* out, uint32_t* hist,
@@ -239,38 +240,62 @@ __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare
     at = __shfl_sync(0xffffffffu, at, src);
     fast = at <= static_cast<uint32_t>(kCandMax);
     if (fast) {
-      // keys above the threshold bin -> out (unordered), its own keys -> tbk
+      // the keys of bins >= tb in bin order: bin b starts after the keys of
+      // the bins above it (warp 0 turns the histogram into those offsets)
+      group_sync<NW>(bar_id);  // every warp has read the histogram
+      if (gw == 0) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int b = 255 - 8 * lane - j;
+          if (b >= tb) hist[b] = run;
+          run += c[j];
+        }
+      }
+      group_sync<NW>(bar_id);
+      // slots [0, above) live in out, [above, above + at) in tbk
+      auto slot = [&](uint32_t q) -> uint64_t& { return q < above ? out[q] : tbk[q - above]; };
       for_each([&](float v, uint32_t id) {
         const int b = bin(v);
-        if (b > tb) out[atomicAdd(&cnt[0], 1u)] = make_key(v, id);
-        else if (b == tb) tbk[atomicAdd(&cnt[1], 1u)] = make_key(v, id);
+        if (b >= tb) slot(atomicAdd(&hist[b], 1u)) = make_key(v, id);
       });
       group_sync<NW>(bar_id);
-      if (gw == 0) {
-        const int need = want - static_cast<int>(above);
-        if (at <= 32u) {
-          uint64_t key[1];
-          key[0] = lane < static_cast<int>(at) ? tbk[lane] : 0ull;
-          reg_sort_desc<1>(key);
-          if (lane < need) out[above + lane] = key[0];
-        } else {
-          uint64_t key[2];
-          key[0] = tbk[lane];
-          key[1] = 32 + lane < static_cast<int>(at) ? tbk[32 + lane] : 0ull;
-          reg_sort_desc<2>(key);
-          if (lane < need) out[above + lane] = key[0];
-          if (32 + lane < need) out[above + 32 + lane] = key[1];
+      // hist[b] now ends bin b, so bin b spans [hist[b + 1], hist[b]) (255: from 0);
+      // a key's rank is its bin's start plus the larger keys of its bin
+      constexpr int PER = (32 * W + kCandMax + NW * 32 - 1) / (NW * 32);
+      const uint32_t staged = above + at;
+      uint64_t kk[PER];
+      int rk[PER];
+#pragma unroll
+      for (int q = 0; q < PER; ++q) {
+        const uint32_t s0 = static_cast<uint32_t>(gt + q * NW * 32);
+        rk[q] = -1;
+        kk[q] = 0ull;
+        if (s0 < staged) {
+          kk[q] = slot(s0);
+          const int b = bin(key_val(kk[q]));
+          const uint32_t lo_s = b == 255 ? 0u : hist[b + 1], hi_s = hist[b];
+          uint32_t r = lo_s;
+          for (uint32_t s1 = lo_s; s1 < hi_s; ++s1) r += slot(s1) > kk[q] ? 1u : 0u;
+          rk[q] = static_cast<int>(r);
         }
-        __syncwarp();
       }
+      group_sync<NW>(bar_id);  // every staged key is read before out is rewritten
+#pragma unroll
+      for (int q = 0; q < PER; ++q)
+        if (rk[q] >= 0 && rk[q] < want) out[rk[q]] = kk[q];
+      for (int p = want + gt; p < 32 * W; p += NW * 32) out[p] = 0ull;
     }
   }
   if (!fast) {
     prepare();
     group_sync<NW>(bar_id);
-    if (gw == 0) warp_select_top(key_at, n, want, out, hist);
+    if (gw == 0) {
+      warp_select_top(key_at, n, want, out, hist);
+      sort_out<W>(out, want < n ? want : n);
+    }
   }
-  if (gw == 0) sort_out<W>(out, want < n ? want : n);
+  group_sync<NW>(bar_id);  // out is complete for every warp of the group
 }
 
 struct SelPlan {
