@@ -101,7 +101,8 @@ int cuda_status(cudaError_t e) {
 
 int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, const float* br,
                const float* bc, int32_t* idx, float* gate, float* score, int32_t* status,
-               float* Z, cudaStream_t s) {
+               float* Z, cudaStream_t s, float* zero = nullptr, int64_t zero_words = 0,
+               bool* zeroed = nullptr) {
   cudaError_t e;
   int parts = 1;
   if (omni::router_tc_supported(D, x, Wr, Wc)) {
@@ -111,7 +112,8 @@ int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, con
     e = omni::launch_router_simt(D, x, Wr, Wc, Z, s);
   }
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(omni::launch_select(D, Z, parts, br, bc, idx, gate, score, s));
+  return cuda_status(
+      omni::launch_select(D, Z, parts, br, bc, idx, gate, score, s, zero, zero_words, zeroed));
 }
 
 bool tensors_ok(const void* const* p16, int n16) {
@@ -258,7 +260,14 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   FusedWs w = carve_fused(D, c);
   int32_t* idx = idx_out ? idx_out : w.idx;
   float* gate = gate_out ? gate_out : w.gate;
-  rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s);
+  // a batch without sweeps accumulates into a buffer the selection can clear
+  // while the router runs (y itself for fp32, else the expert workspace)
+  const int64_t acc_words = omni::expert_acc_words(D);
+  float* acc = acc_words == 0 ? nullptr
+               : static_cast<float*>(D.dtype == OMNI_F32 ? y : w.expert);
+  bool acc_zeroed = false;
+  rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s, acc,
+                  acc_words, &acc_zeroed);
   if (rc != OMNI_OK) return rc;
   if (fused_windows(D)) {
     rc = cuda_status(omni::launch_schedule_windows(D, idx, gate, w.uniq, w.group_off, counts,
@@ -270,7 +279,7 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
                                          w.uniq, w.group_off, counts, w.sched, s));
   if (rc != OMNI_OK) return rc;
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
-                                         w.group_off, counts, y, w.expert, s));
+                                         w.group_off, counts, y, w.expert, s, acc_zeroed));
 }
 
 int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,

@@ -1231,7 +1231,8 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* group_off,
-                          const int32_t* counts, void* y, void* ws, cudaStream_t s) {
+                          const int32_t* counts, void* y, void* ws, cudaStream_t s,
+                          bool acc_zeroed) {
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
   float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
@@ -1246,8 +1247,8 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                                               group_off, counts, w, nullptr, acc, ycast, status,
                                               s);
   }
-  const size_t ybytes = static_cast<size_t>(D.L) * D.d * sizeof(float);
-  cudaError_t err = launch_zero(acc, ybytes / sizeof(float), s);
+  cudaError_t err = acc_zeroed ? cudaSuccess
+                               : launch_zero(acc, static_cast<size_t>(expert_acc_words(D)), s);
   if (err != cudaSuccess) return err;
   err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
             : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
@@ -1257,6 +1258,10 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,
       static_cast<__nv_bfloat16*>(y), n));
   return cudaGetLastError();
+}
+
+int64_t expert_acc_words(const Dims& D) {
+  return expert_sweeps(D) > 1 ? 0 : D.L * D.d;
 }
 
 WinTasks expert_windows(const Dims& D, void* ws) {

@@ -33,9 +33,12 @@ cudaError_t launch_sum_partials(float* Z, int splits, int64_t n, cudaStream_t s)
 
 // ---- selection: per-axis top-k, k x k merge, top-K, gate ----------------
 // Z holds `parts` consecutive partial logit arrays, summed in order on load.
+// zero (nullable, zero_words floats): a buffer the small-batch kernel clears
+// before it waits on the kernel ahead of it; *zeroed says whether it did.
 cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
                           const float* bc, int32_t* idx, float* gate, float* score,
-                          cudaStream_t s);
+                          cudaStream_t s, float* zero = nullptr, int64_t zero_words = 0,
+                          bool* zeroed = nullptr);
 
 // ---- windows of consecutive groups (the sweep path of the execution) ------
 // Window w holds the groups whose first task lies in [w*T, (w+1)*T).
@@ -71,7 +74,12 @@ cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, c
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* group_off,
-                          const int32_t* counts, void* y, void* ws, cudaStream_t s);
+                          const int32_t* counts, void* y, void* ws, cudaStream_t s,
+                          bool acc_zeroed = false);
+// The accumulator launch_expert clears before a batch without sweeps (its fp32
+// partial sums: y itself for fp32, else the head of ws), in floats; 0 for
+// batches with sweeps.
+int64_t expert_acc_words(const Dims& D);
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
                          cudaStream_t s);

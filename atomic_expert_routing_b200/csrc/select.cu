@@ -573,7 +573,20 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
                                                      const float* __restrict__ bc,
                                                      int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
-                                                     float* __restrict__ score, WidePlan P) {
+                                                     float* __restrict__ score, WidePlan P,
+                                                     float* __restrict__ zero, int64_t zero_words) {
+  // the caller's buffer to clear needs nothing from the kernel ahead of this one
+  if (zero != nullptr) {
+    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    if ((reinterpret_cast<uintptr_t>(zero) & 15) == 0) {
+      for (int64_t i = i0; i < zero_words / 4; i += stride)
+        reinterpret_cast<float4*>(zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t i = (zero_words / 4) * 4 + i0; i < zero_words; i += stride) zero[i] = 0.0f;
+    } else {
+      for (int64_t i = i0; i < zero_words; i += stride) zero[i] = 0.0f;
+    }
+  }
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem[];
@@ -759,14 +772,14 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
 template <int NPW, int W, int WK>
 cudaError_t launch_wide_t(const Dims& D, const float* Z, int parts, const float* br,
                           const float* bc, int32_t* idx, float* gate, float* score,
-                          cudaStream_t s) {
+                          float* zero, int64_t zero_words, cudaStream_t s) {
   const WidePlan P = make_wide_plan(D, W, WK);
   cudaError_t err = cudaFuncSetAttribute(k_select_wide<NPW, W, WK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, P.bytes);
   if (err != cudaSuccess) return err;
   OMNI_TRY(launch_k(k_select_wide<NPW, W, WK>, static_cast<unsigned>(D.L), 256, P.bytes, s, Z,
       parts, D.L, static_cast<int>(D.Nr), static_cast<int>(D.Nc), static_cast<int>(D.k),
-      static_cast<int>(D.K), br, bc, idx, gate, score, P));
+      static_cast<int>(D.K), br, bc, idx, gate, score, P, zero, zero_words));
   return cudaGetLastError();
 }
 
@@ -825,12 +838,13 @@ cudaError_t launch_select_npl(const Dims& D, const float* Z, const float* br, co
 
 template <int NPW>
 cudaError_t launch_wide(const Dims& D, const float* Z, int parts, const float* br,
-                        const float* bc, int32_t* idx, float* gate, float* score, cudaStream_t s) {
+                        const float* bc, int32_t* idx, float* gate, float* score, float* zero,
+                        int64_t zero_words, cudaStream_t s) {
   switch (sort_width(D.k > D.K ? D.k : D.K)) {
-    case 1: return launch_wide_t<NPW, 1, 1>(D, Z, parts, br, bc, idx, gate, score, s);
-    case 2: return launch_wide_t<NPW, 2, 2>(D, Z, parts, br, bc, idx, gate, score, s);
-    case 4: return launch_wide_t<NPW, 4, 4>(D, Z, parts, br, bc, idx, gate, score, s);
-    default: return launch_wide_t<NPW, 8, 8>(D, Z, parts, br, bc, idx, gate, score, s);
+    case 1: return launch_wide_t<NPW, 1, 1>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
+    case 2: return launch_wide_t<NPW, 2, 2>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
+    case 4: return launch_wide_t<NPW, 4, 4>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
+    default: return launch_wide_t<NPW, 8, 8>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
   }
 }
 
@@ -838,16 +852,18 @@ cudaError_t launch_wide(const Dims& D, const float* Z, int parts, const float* b
 
 cudaError_t launch_select(const Dims& D, const float* Z, int parts, const float* br,
                           const float* bc, int32_t* idx, float* gate, float* score,
-                          cudaStream_t s) {
+                          cudaStream_t s, float* zero, int64_t zero_words, bool* zeroed) {
+  if (zeroed != nullptr) *zeroed = false;
   if (D.L == 0) return cudaSuccess;
   const int64_t n = D.Nr > D.Nc ? D.Nr : D.Nc;
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (D.L <= sms) {  // too few tokens for two warps each to fill the GPU
-    if (n <= 256) return launch_wide<2>(D, Z, parts, br, bc, idx, gate, score, s);
-    if (n <= 1024) return launch_wide<8>(D, Z, parts, br, bc, idx, gate, score, s);
-    return launch_wide<32>(D, Z, parts, br, bc, idx, gate, score, s);
+    if (zeroed != nullptr) *zeroed = zero != nullptr;
+    if (n <= 256) return launch_wide<2>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
+    if (n <= 1024) return launch_wide<8>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
+    return launch_wide<32>(D, Z, parts, br, bc, idx, gate, score, zero, zero_words, s);
   }
   if (parts > 1) {  // split-K partial logits: sum them first, in a fixed order
     cudaError_t e = launch_sum_partials(const_cast<float*>(Z), parts, D.L * (D.Nr + D.Nc), s);
