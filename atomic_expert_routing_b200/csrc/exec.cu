@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
 // unit -- its rows are read while its window is in flight -- and every task
 // exactly once.
 constexpr int kWinTasks = 7168;
+constexpr int kWinCountBins = 2 * kBlockSortMax;  // counters of the counting expert order
 
 // Window w takes the groups whose first task lies in [w*T, (w+1)*T).  Two
 // orders of its tasks are written: by token (wt/we/wg, for the accumulation
@@ -654,8 +655,13 @@ __global__ void __launch_bounds__(kBlockSortThreads)
 }
 
 // The same window orders when the tasks already arrive in window token order
-// (wt/we/wg, windows [win_lo[w], win_lo[w+1])): only the stable sort by
-// expert is left.  Windows larger than the CTA sort keep token order.
+// (wt/we/wg, windows [win_lo[w], win_lo[w+1])): only the expert order is
+// left.  The activation pass needs an expert's tasks adjacent, not in any
+// order among themselves (each task's activation is its own dot product), so
+// a window whose ids span at most kWinCountBins is ordered by one counting
+// pass (shared-memory counters, then placement by atomic cursors); a wider
+// one by the stable radix sort.  Windows larger than the CTA sort keep token
+// order.
 __global__ void __launch_bounds__(kBlockSortThreads)
     k_wsort_x(const int32_t* __restrict__ win_lo, WinOut o) {
   pdl_wait();
@@ -698,6 +704,33 @@ __global__ void __launch_bounds__(kBlockSortThreads)
   atomicMax(&emax, lmax);
   __syncthreads();
   const int64_t span = static_cast<int64_t>(emax) - emin;
+  if (span < kWinCountBins) {
+    int* cnt = reinterpret_cast<int*>(kA);  // kA and kB: kWinCountBins counters
+    const int bins = static_cast<int>(span) + 1;
+    for (int b = threadIdx.x; b < bins; b += blockDim.x) cnt[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nn; i += blockDim.x) atomicAdd(&cnt[o.we[a0 + i] - emin], 1);
+    __syncthreads();
+    // exclusive scan of the counters: thread k takes bins [k*per, k*per + per)
+    const int per = (bins + kBlockSortThreads - 1) / kBlockSortThreads;
+    int mine = 0;
+    for (int b = threadIdx.x * per; b < bins && b < threadIdx.x * per + per; ++b) mine += cnt[b];
+    int run = block_exclusive_scan(mine, warp_tot, &total);
+    for (int b = threadIdx.x * per; b < bins && b < threadIdx.x * per + per; ++b) {
+      const int c = cnt[b];
+      cnt[b] = run;
+      run += c;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+      const int pos = atomicAdd(&cnt[o.we[a0 + i] - emin], 1);
+      o.xt[a0 + pos] = o.wt[a0 + i];
+      o.xe[a0 + pos] = o.we[a0 + i];
+      o.xg[a0 + pos] = o.wg[a0 + i];
+      o.xdst[a0 + pos] = static_cast<int32_t>(a0 + i);
+    }
+    return;
+  }
   int ebits = 0;
   while (ebits < 32 && (int64_t(1) << ebits) <= span) ++ebits;
   const int epasses = (ebits + 7) / 8;

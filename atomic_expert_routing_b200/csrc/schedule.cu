@@ -937,28 +937,6 @@ cudaError_t prep_and_scan(const Dims& D, const int32_t* idx, const float* gate, 
 // that of a stable sort by token of the window's tasks in schedule order.
 constexpr int64_t kWinCellsMax = int64_t(1) << 23;  // nwin * L
 
-// win_lo[w] = first task of window w (M when it has no group); win_lo[nwin] = M
-__global__ void __launch_bounds__(256)
-    k_winbase(const int32_t* __restrict__ group_off, const int32_t* __restrict__ counts, int64_t M,
-              int64_t T, int nwin, int32_t* __restrict__ win_lo) {
-  pdl_wait();
-  pdl_trigger();
-  const int w = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
-  if (w > nwin) return;
-  if (w == nwin) {
-    win_lo[w] = static_cast<int32_t>(M);
-    return;
-  }
-  const int64_t G = counts[1];
-  const int64_t v = static_cast<int64_t>(w) * T;
-  int64_t lo = 0, hi = G;  // first group starting at or after v
-  while (lo < hi) {
-    const int64_t m = (lo + hi) >> 1;
-    if (group_off[m] >= v) hi = m; else lo = m + 1;
-  }
-  win_lo[w] = lo < G ? group_off[lo] : static_cast<int32_t>(M);
-}
-
 // Token t's task j (sorted by expert): its window, and the index of the first
 // task of its (window, token) run.  One warp per token, element j = w*32 + lane.
 template <int W>
@@ -1019,12 +997,28 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
     if (last[w]) cnt[static_cast<int64_t>(win[w]) * L + t] = w * 32 + lane - first[w] + 1;
 }
 
-// one CTA per window: exclusive scan of its row of L counts, in place
-__global__ void __launch_bounds__(kScanThreads) k_rowscan(int32_t* __restrict__ cnt, int64_t L) {
+// One CTA per window: the exclusive scan of its row of L counts, in place,
+// and win_lo[w], the window's first task (that of the first group starting at
+// or after w*T; M when none does), with win_lo[nwin] = M.
+__global__ void __launch_bounds__(kScanThreads)
+    k_rowscan(int32_t* __restrict__ cnt, int64_t L, const int32_t* __restrict__ group_off,
+              const int32_t* __restrict__ counts, int64_t M, int64_t T,
+              int32_t* __restrict__ win_lo) {
   pdl_wait();
   pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int total;
+  if (threadIdx.x == 0) {
+    const int64_t G = counts[1];
+    const int64_t v = static_cast<int64_t>(blockIdx.x) * T;
+    int64_t lo = 0, hi = G;
+    while (lo < hi) {
+      const int64_t m = (lo + hi) >> 1;
+      if (group_off[m] >= v) hi = m; else lo = m + 1;
+    }
+    win_lo[blockIdx.x] = lo < G ? group_off[lo] : static_cast<int32_t>(M);
+    if (blockIdx.x == gridDim.x - 1) win_lo[gridDim.x] = static_cast<int32_t>(M);
+  }
   int32_t* row = cnt + static_cast<int64_t>(blockIdx.x) * L;
   int carry = 0;
   for (int64_t b0 = 0; b0 < L; b0 += kScanTile) {
@@ -1179,8 +1173,6 @@ cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const flo
   if (err != cudaSuccess) return err;
   err = launch_zero(w.cnt, static_cast<size_t>(nwin) * D.L, s);
   if (err != cudaSuccess) return err;
-  OMNI_TRY(launch_k(k_winbase, static_cast<unsigned>((nwin + 1 + 255) / 256), 256, 0, s, group_off,
-      counts, M, T, nwin, out.win_lo));
   const unsigned blocks = static_cast<unsigned>((D.L + kPrepWarps - 1) / kPrepWarps);
   const int K = static_cast<int>(D.K);
   auto count = [&](auto kern) {
@@ -1189,7 +1181,9 @@ cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const flo
   };
   OMNI_TRY(K <= 32 ? count(k_wincount<1>) : K <= 64 ? count(k_wincount<2>)
            : K <= 128 ? count(k_wincount<4>) : count(k_wincount<8>));
-  OMNI_TRY(launch_k(k_rowscan, static_cast<unsigned>(nwin), kScanThreads, 0, s, w.cnt, D.L));
+  OMNI_TRY(launch_k(k_rowscan, static_cast<unsigned>(nwin), kScanThreads, 0, s, w.cnt, D.L,
+      static_cast<const int32_t*>(group_off), static_cast<const int32_t*>(counts), M, T,
+      out.win_lo));
   auto scatter = [&](auto kern) {
     return launch_k(kern, blocks, kPrepWarps * 32, 0, s, w.tmp_e, w.tmp_g, w.rank, group_off,
                     static_cast<const int32_t*>(out.win_lo), static_cast<const int32_t*>(w.cnt),
