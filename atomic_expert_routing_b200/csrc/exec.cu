@@ -694,11 +694,22 @@ __global__ void __launch_bounds__(kBlockSortThreads)
   }
   __syncthreads();
   const int nn = static_cast<int>(n);
+  // this thread's tasks i = threadIdx.x + q * blockDim.x, read once
+  constexpr int kPer = kBlockSortMax / kBlockSortThreads;
+  int te_r[kPer], tt_r[kPer];
+  float tg_r[kPer];
   int lmin = INT_MAX, lmax = INT_MIN;
-  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
-    const int e = o.we[a0 + i];
-    lmin = e < lmin ? e : lmin;
-    lmax = e > lmax ? e : lmax;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int i = threadIdx.x + q * kBlockSortThreads;
+    te_r[q] = 0;
+    if (i < nn) {
+      te_r[q] = o.we[a0 + i];
+      tt_r[q] = o.wt[a0 + i];
+      tg_r[q] = o.wg[a0 + i];
+      lmin = te_r[q] < lmin ? te_r[q] : lmin;
+      lmax = te_r[q] > lmax ? te_r[q] : lmax;
+    }
   }
   atomicMin(&emin, lmin);
   atomicMax(&emax, lmax);
@@ -709,7 +720,9 @@ __global__ void __launch_bounds__(kBlockSortThreads)
     const int bins = static_cast<int>(span) + 1;
     for (int b = threadIdx.x; b < bins; b += blockDim.x) cnt[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < nn; i += blockDim.x) atomicAdd(&cnt[o.we[a0 + i] - emin], 1);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (threadIdx.x + q * kBlockSortThreads < nn) atomicAdd(&cnt[te_r[q] - emin], 1);
     __syncthreads();
     // exclusive scan of the counters: thread k takes bins [k*per, k*per + per)
     const int per = (bins + kBlockSortThreads - 1) / kBlockSortThreads;
@@ -722,12 +735,16 @@ __global__ void __launch_bounds__(kBlockSortThreads)
       run += c;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < nn; i += blockDim.x) {
-      const int pos = atomicAdd(&cnt[o.we[a0 + i] - emin], 1);
-      o.xt[a0 + pos] = o.wt[a0 + i];
-      o.xe[a0 + pos] = o.we[a0 + i];
-      o.xg[a0 + pos] = o.wg[a0 + i];
-      o.xdst[a0 + pos] = static_cast<int32_t>(a0 + i);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int i = threadIdx.x + q * kBlockSortThreads;
+      if (i < nn) {
+        const int pos = atomicAdd(&cnt[te_r[q] - emin], 1);
+        o.xt[a0 + pos] = tt_r[q];
+        o.xe[a0 + pos] = te_r[q];
+        o.xg[a0 + pos] = tg_r[q];
+        o.xdst[a0 + pos] = static_cast<int32_t>(a0 + i);
+      }
     }
     return;
   }

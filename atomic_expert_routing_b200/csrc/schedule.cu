@@ -1008,16 +1008,28 @@ __global__ void __launch_bounds__(kScanThreads)
   pdl_trigger();
   __shared__ int warp_tot[32];
   __shared__ int total;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {  // warp 0: a 32-way search for the first group starting at >= w*T
+    const int lane = threadIdx.x;
     const int64_t G = counts[1];
     const int64_t v = static_cast<int64_t>(blockIdx.x) * T;
-    int64_t lo = 0, hi = G;
+    int64_t lo = 0, hi = G;  // the answer lies in [lo, hi]; G: no such group
     while (lo < hi) {
-      const int64_t m = (lo + hi) >> 1;
-      if (group_off[m] >= v) hi = m; else lo = m + 1;
+      const int64_t step = (hi - lo + 31) / 32;
+      const int64_t pos = lo + lane * step;
+      const uint32_t ge = __ballot_sync(0xffffffffu, pos < hi && group_off[pos] >= v);
+      const uint32_t in = __ballot_sync(0xffffffffu, pos < hi);
+      if (ge != 0u) {
+        const int f = __ffs(ge) - 1;
+        hi = lo + f * step;
+        lo = f > 0 ? lo + (f - 1) * step + 1 : hi;
+      } else {
+        lo = lo + (31 - __clz(in)) * step + 1;
+      }
     }
-    win_lo[blockIdx.x] = lo < G ? group_off[lo] : static_cast<int32_t>(M);
-    if (blockIdx.x == gridDim.x - 1) win_lo[gridDim.x] = static_cast<int32_t>(M);
+    if (lane == 0) {
+      win_lo[blockIdx.x] = lo < G ? group_off[lo] : static_cast<int32_t>(M);
+      if (blockIdx.x == gridDim.x - 1) win_lo[gridDim.x] = static_cast<int32_t>(M);
+    }
   }
   int32_t* row = cnt + static_cast<int64_t>(blockIdx.x) * L;
   int carry = 0;
