@@ -182,13 +182,15 @@ class Clocks:
 # --------------------------------------------------------------------------- CPU oracle arm
 
 
-def oracle_timing(cfg, target_s=10.0, max_tokens=None):
+def oracle_timing(cfg, target_s=10.0, max_tokens=None, h=None):
     """Time the fp64 oracle (route -> schedule -> expert-centric execution) on a
     bounded token sample sized for about target_s of CPU work.  Returns
-    (tokens/s, sample tokens, seconds, threads)."""
+    (tokens/s, sample tokens, seconds, threads, inputs); h: the inputs, when
+    already drawn."""
     import oracle as O
 
-    h = WL.make_inputs(cfg)
+    if h is None:
+        h = WL.make_inputs(cfg)
     n = 64
     while True:
         tok = WL.sample_tokens(cfg, n)
@@ -508,10 +510,20 @@ def run_ours(args):
     achieved = eb / (st_ms * 1e-3) / 1e9
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rate, n, dt, threads, _ = oracle_timing(cfg, target_s=args.cpu_seconds)
+        rate, n, dt, threads, h_cpu = oracle_timing(cfg, target_s=args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} of {cfg.L} tokens of {cfg.name} (route+schedule+expert-centric "
                          f"execution, fp64), {dt:.1f} s"}
+        # the same oracle on one thread, over a smaller sample
+        import oracle as O
+        try:
+            O.set_num_threads(1)
+            rate1, n1, dt1, _, _ = oracle_timing(cfg, target_s=min(2.0, args.cpu_seconds),
+                                                 max_tokens=max(64, n // 8), h=h_cpu)
+        finally:
+            O.set_num_threads(threads)
+        cpu["value_1_thread"] = rate1
+        cpu["sample_1_thread"] = f"{n1} tokens, {dt1:.1f} s"
     line = {
         "metric": METRIC,
         "value": job_throughput(world, cfg.L, ms_all),

@@ -54,6 +54,11 @@ def num_threads() -> int:
     return int(lib().oracle_num_threads())
 
 
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's later OpenMP regions (timing only)."""
+    lib().oracle_set_num_threads(C.c_int(int(n)))
+
+
 def _tokens(cfg, tokens):
     if tokens is None:
         return np.arange(cfg.L, dtype=np.int64)

@@ -499,3 +499,13 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Sets the threads of later OpenMP regions (n >= 1); timing only, the results
+   do not depend on it. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

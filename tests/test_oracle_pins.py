@@ -333,3 +333,20 @@ def test_execution_closed_forms():
     np.testing.assert_allclose(y2, -2 * y, rtol=0, atol=1e-15)
     yt, _ = O.forward_token(cfg, inp, idx, gate)
     np.testing.assert_allclose(yt, ref, rtol=0, atol=1e-15)
+
+
+def test_thread_count_does_not_change_results():
+    """The oracle's OpenMP loops split independent tokens (and ids): one thread
+    and all threads give bit-identical routing and y."""
+    cfg = WL.TINY
+    h = WL.make_inputs(cfg)
+    a = O.moe_forward(cfg, h)
+    n = O.num_threads()
+    try:
+        O.set_num_threads(1)
+        assert O.num_threads() == 1
+        b = O.moe_forward(cfg, h)
+    finally:
+        O.set_num_threads(n)
+    for k in ("idx", "gate", "score", "y"):
+        np.testing.assert_array_equal(np.asarray(a[k]), np.asarray(b[k]))
