@@ -180,11 +180,11 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 // bin's position plus the number of larger keys of its bin: the output is
 // sorted without a sorting network.  A threshold bin that is too full, or a
 // non-finite range, falls back to the radix select.  hist: 256 words; tbk:
-// kCandMax keys; cnt: 2 words.
+// kCandMax keys.
 template <int W, int NW, typename ForEach, typename Prepare, typename KeyAt>
 __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare, KeyAt key_at,
                            int n, int want, float lo, float hi, uint64_t* out, uint32_t* hist,
-                           uint64_t* tbk, uint32_t* cnt) {
+                           uint64_t* tbk) {
   const int lane = threadIdx.x & 31;
   const int gt = gw * 32 + lane;
   const float range = hi - lo;
@@ -196,10 +196,6 @@ __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare
       return __float2int_rz(fminf(fmaxf(fmaf(v, scale, off), 0.0f), 255.0f));
     };
     for (int b = gt; b < 256; b += NW * 32) hist[b] = 0u;
-    if (gt == 0) {
-      cnt[0] = 0u;
-      cnt[1] = 0u;
-    }
     group_sync<NW>(bar_id);
     for_each([&](float v, uint32_t) { atomicAdd(&hist[bin(v)], 1u); });
     group_sync<NW>(bar_id);
@@ -300,8 +296,7 @@ __device__ void group_topk(int gw, int bar_id, ForEach for_each, Prepare prepare
 
 struct SelPlan {
   int cand;                           // (a, b) candidate pairs of the k x k merge
-  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc,
-      off_cnt;
+  int off_vr, off_vc, off_hr, off_hc, off_sr, off_sc, off_cand, off_out, off_misc, off_tr, off_tc;
   int pair_bytes;
   int table_bytes;                    // per CTA: the (a, b) pair table
   int bias_bytes;                     // per CTA: cached row/column biases (0 without bias)
@@ -335,7 +330,6 @@ SelPlan make_plan(const Dims& D, int W, int WK) {
   p.off_misc = off; off = al(off + 32);
   p.off_tr = off; off = al(off + 8 * kCandMax);
   p.off_tc = off; off = al(off + 8 * kCandMax);
-  p.off_cnt = off; off = al(off + 16);
   p.pair_bytes = off;
   p.table_bytes = al(4 * p.cand);
   p.bias_bytes = 0;
@@ -426,7 +420,6 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + (role ? P.off_hc : P.off_hr));
     uint64_t* sel = reinterpret_cast<uint64_t*>(base + (role ? P.off_sc : P.off_sr));
     uint64_t* tbin = reinterpret_cast<uint64_t*>(base + (role ? P.off_tc : P.off_tr));
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt) + 2 * role;
     const float* bias = P.bias_bytes > 0 ? bias_s + zoff : nullptr;
     asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies of token t
     float v[NPL];
@@ -467,7 +460,7 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
             if (j * 32 + lane < n) vals[j * 32 + lane] = v[j];
         },
         [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
-        hist, tbin, cnt);
+        hist, tbin);
     __syncwarp();
     if (t + stride < L) prefetch(t + stride);  // lands while the pair merges
   }
@@ -481,7 +474,6 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
   uint64_t* out = reinterpret_cast<uint64_t*>(base + P.off_out);
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + P.off_hr);
   uint64_t* tbin = reinterpret_cast<uint64_t*>(base + P.off_tr);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(base + P.off_cnt);
   const int nc = P.cand;
   const int pt = role * 32 + lane;  // thread of the pair
   float cmx = -INFINITY, cmn = INFINITY;
@@ -511,7 +503,7 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
           f(key_val(kk), key_id(kk));
         }
       },
-      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbin, cnt);
+      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbin);
   if (role == 0) {
     // ---- gate = softmax of the K selected joint scores ----
     const float s0 = key_val(out[0]);
@@ -542,7 +534,7 @@ __global__ void __launch_bounds__(256, 3) k_select(const float* __restrict__ Z, 
 // of one warp, as in k_select.
 struct WidePlan {
   int cand;
-  int off_vals, off_hist, off_sel, off_tbk, off_cnt, off_red, off_roff, off_cand, off_out, off_misc;
+  int off_vals, off_hist, off_sel, off_tbk, off_red, off_roff, off_cand, off_out, off_misc;
   int bytes;
 };
 
@@ -556,7 +548,6 @@ WidePlan make_wide_plan(const Dims& D, int W, int WK) {
   p.off_hist = off; off = al(off + 2 * 4 * 256);
   p.off_sel = off; off = al(off + 2 * 8 * 32 * W);
   p.off_tbk = off; off = al(off + 2 * 8 * kCandMax);
-  p.off_cnt = off; off = al(off + 16);
   p.off_red = off; off = al(off + 4 * 3 * 8);
   p.off_roff = off; off = al(off + 4 * static_cast<int>(D.k));
   p.off_cand = off; off = al(off + 8 * p.cand);
@@ -607,7 +598,6 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + P.off_hist) + axis * 256;
     uint64_t* sel = reinterpret_cast<uint64_t*>(smem + P.off_sel) + axis * 32 * W;
     uint64_t* tbk = reinterpret_cast<uint64_t*>(smem + P.off_tbk) + axis * kCandMax;
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + P.off_cnt) + 2 * axis;
     const int bar = 1 + axis;
     // split-K partial logits (parts > 1) are summed here, in order
     const int64_t zs = L * static_cast<int64_t>(Nr + Nc);
@@ -683,7 +673,7 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
           }
         },
         [&](int i) { return make_key(vals[i], static_cast<uint32_t>(i)); }, n, k, mn, mx, sel,
-        hist, tbk, cnt);
+        hist, tbk);
   }
   __syncthreads();
 
@@ -695,7 +685,6 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
   uint64_t* out = reinterpret_cast<uint64_t*>(smem + P.off_out);
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + P.off_hist);
   uint64_t* tbk = reinterpret_cast<uint64_t*>(smem + P.off_tbk);
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + P.off_cnt);
   if (warp == 0) {
     // pairs of row a start at roff[a] (prefix of min(k, K/(a+1)))
     int na = 0;
@@ -751,7 +740,7 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
           f(key_val(kk), key_id(kk));
         }
       },
-      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbk, cnt);
+      []() {}, [&](int i) { return cand[i]; }, nc, K, cmn, cmx, out, hist, tbk);
   if (warp != 0) return;
 
   // ---- gate = softmax of the K selected joint scores ----
