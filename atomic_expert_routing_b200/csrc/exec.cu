@@ -663,7 +663,18 @@ __global__ void __launch_bounds__(kBlockSortThreads)
 // one by the stable radix sort.  Windows larger than the CTA sort keep token
 // order.
 __global__ void __launch_bounds__(kBlockSortThreads)
-    k_wsort_x(const int32_t* __restrict__ win_lo, WinOut o) {
+    k_wsort_x(const int32_t* __restrict__ win_lo, WinOut o, float* __restrict__ zslice,
+              int64_t zrows, int zcols, int64_t zld) {
+  // the first sweep's slice (zrows x zcols floats, rows zld apart) is cleared
+  // before the wait: no kernel still in flight ahead of this one touches it
+  if (zslice != nullptr) {
+    const int per_row = zcols / 4;
+    const int64_t n = zrows * per_row;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+      reinterpret_cast<float4*>(zslice + (i / per_row) * zld)[i % per_row] =
+          make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t wsm[];
@@ -1157,7 +1168,8 @@ constexpr size_t kWsortSmem = static_cast<size_t>(kBlockSortMax) * (2 * 4 + 3 * 
 // and only the expert order is left to make
 cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, const float* tg,
                          const int32_t* group_off, const int32_t* counts, const SweepWs& w,
-                         const int32_t* win_lo, int32_t* status, cudaStream_t s) {
+                         const int32_t* win_lo, float* zslice, int zcols, int64_t zld,
+                         int32_t* status, cudaStream_t s) {
   const int64_t M = D.M();
   const int64_t T = window_tasks(D);
   const int64_t nwin = (M + T - 1) / T;
@@ -1166,7 +1178,7 @@ cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, co
                                            static_cast<int>(kWsortSmem));
     if (err != cudaSuccess) return err;
     OMNI_TRY(launch_k(k_wsort_x, static_cast<unsigned>(nwin), kBlockSortThreads, kWsortSmem, s,
-        win_lo, w.win));
+        win_lo, w.win, zslice, D.L, zcols, zld));
     return cudaGetLastError();
   }
   constexpr size_t smem = kWsortSmem;
@@ -1216,7 +1228,16 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
                       const int32_t* group_off, const int32_t* counts, const SweepWs& w,
                       const int32_t* win_lo, float* acc, __nv_bfloat16* ycast, int32_t* status,
                       cudaStream_t s) {
-  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, win_lo, status, s);
+  const int cols = static_cast<int>(D.d / Q);
+  // bf16: one compact fp32 slice [L x cols] serves every sweep -- zeroed
+  // before the first, then rounded into y's columns and zeroed in place
+  // (its lines stay in L2) between sweeps, and dropped after the last.
+  // fp32: the slices are y's own columns.  On the window path the window
+  // sort clears the first slice.
+  const int64_t ld = ycast ? cols : D.d;
+  auto slice = [&](int q) { return ycast ? acc : acc + static_cast<int64_t>(q) * cols; };
+  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, win_lo,
+                                 win_lo != nullptr ? slice(0) : nullptr, cols, ld, status, s);
   if (err != cudaSuccess) return err;
   // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
   constexpr int R = 3;
@@ -1236,18 +1257,11 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
       w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status));
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int cols = static_cast<int>(D.d / Q);
   // 128-column blocks per slice and the prefetch distance (about 16 vectors
   // of loads in flight per lane)
   constexpr int NB = NVQ * 32 * kEpv<T> / 128;
   constexpr int PD = 8 / NVQ;
-  // bf16: one compact fp32 slice [L x cols] serves every sweep -- zeroed
-  // before the first, then rounded into y's columns and zeroed in place
-  // (its lines stay in L2) between sweeps, and dropped after the last.
-  // fp32: the slices are y's own columns.
-  const int64_t ld = ycast ? cols : D.d;
-  auto slice = [&](int q) { return ycast ? acc : acc + static_cast<int64_t>(q) * cols; };
-  err = launch_finish(D, nullptr, 0, nullptr, slice(0), ld, cols, false, s);
+  if (win_lo == nullptr) err = launch_finish(D, nullptr, 0, nullptr, slice(0), ld, cols, false, s);
   for (int q = 0; q < Q && err == cudaSuccess; ++q) {
     err = launch_acc<T, NB, PD>(D, q * cols, V, w, slice(q), ld, s);
     if (err != cudaSuccess) break;

@@ -468,3 +468,25 @@ def test_expert_sweeps_bad_group_count():
     y = omni.expert_forward(D, d["x"], d["W"], d["V"], sched)
     assert int(counts[2].item()) & omni._lib.OMNI_DEV_BAD_INDEX
     assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
+
+
+@pytest.mark.parametrize("cfg", [
+    SWEEP[0],  # the window path of the fused forward
+    # one CTA per token selects and clears the expert accumulator
+    WL.Config("reuse-small", L=64, d=256, Nr=64, Nc=64, k=8, K=8, B=16, dtype=WL.BF16, seed=41),
+], ids=lambda c: c.name)
+def test_fused_workspace_reuse(cfg):
+    """One workspace, filled with 0xFF before first use, serves two fused
+    forwards of different batches: each equals a forward on a fresh workspace
+    (nothing carries over from the workspace's earlier contents)."""
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    D = omni.LayerDims.of(cfg)
+    ws = omni.Workspace()
+    ws.get(omni.workspace_size(D, omni._lib.OMNI_WS_FUSED), torch.device("cuda")).fill_(255)
+    x2 = torch.roll(d["x"], shifts=7, dims=0).contiguous()
+    ys = [omni.moe_forward(D, x, d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"], ws=ws)
+          for x in (d["x"], x2)]
+    for x, y in zip((d["x"], x2), ys):
+        y_fresh = omni.moe_forward(D, x, d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"])
+        assert rel_err(host_f64(y), host_f64(y_fresh)) <= tol_y(cfg)
