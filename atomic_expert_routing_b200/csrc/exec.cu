@@ -519,6 +519,18 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
 constexpr int kWinTasks = 7168;
 constexpr int kWinCountBins = 2 * kBlockSortMax;  // counters of the counting expert order
 
+// The first sweep's fp32 slice (zrows x zcols floats, rows zld apart;
+// nullptr: nothing) is cleared by the window sort.
+__device__ __forceinline__ void clear_slice(float* zslice, int64_t zrows, int zcols, int64_t zld) {
+  if (zslice == nullptr) return;
+  const int per_row = zcols / 4;
+  const int64_t n = zrows * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(zslice + (i / per_row) * zld)[i % per_row] =
+        make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // Window w takes the groups whose first task lies in [w*T, (w+1)*T).  Two
 // orders of its tasks are written: by token (wt/we/wg, for the accumulation
 // sweeps) and by expert (xt/xe/xg, for the activations, so that the tasks of
@@ -540,9 +552,11 @@ __global__ void __launch_bounds__(kBlockSortThreads)
     k_wsort(const int32_t* __restrict__ tt, const int32_t* __restrict__ te,
             const float* __restrict__ tg, const int32_t* __restrict__ group_off,
             const int32_t* __restrict__ counts, int64_t M, int64_t gmax, int T, int passes,
-            WinOut o, int32_t* status) {
-  pdl_wait();
+            WinOut o, int32_t* status, float* __restrict__ zslice, int64_t zrows, int zcols,
+            int64_t zld) {
+  pdl_wait();  // the kernel ahead may be a previous call's last use of the slice
   pdl_trigger();
+  clear_slice(zslice, zrows, zcols, zld);
   extern __shared__ __align__(16) uint8_t wsm[];
   uint32_t* kA = reinterpret_cast<uint32_t*>(wsm);
   uint32_t* kB = kA + kBlockSortMax;
@@ -665,16 +679,9 @@ __global__ void __launch_bounds__(kBlockSortThreads)
 __global__ void __launch_bounds__(kBlockSortThreads)
     k_wsort_x(const int32_t* __restrict__ win_lo, WinOut o, float* __restrict__ zslice,
               int64_t zrows, int zcols, int64_t zld) {
-  // the first sweep's slice (zrows x zcols floats, rows zld apart) is cleared
-  // before the wait: no kernel still in flight ahead of this one touches it
-  if (zslice != nullptr) {
-    const int per_row = zcols / 4;
-    const int64_t n = zrows * per_row;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-      reinterpret_cast<float4*>(zslice + (i / per_row) * zld)[i % per_row] =
-          make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  // the kernel ahead is the window scatter of the same forward, which does
+  // not touch the slice: clear it before the wait
+  clear_slice(zslice, zrows, zcols, zld);
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t wsm[];
@@ -1189,7 +1196,8 @@ cudaError_t launch_wsort(const Dims& D, const int32_t* tt, const int32_t* te, co
   while ((int64_t(1) << bits) < D.L) ++bits;
   const int passes = (bits + 7) / 8;
   OMNI_TRY(launch_k(k_wsort, static_cast<unsigned>(nwin), kBlockSortThreads, smem, s, tt, te, tg,
-      group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.win, status));
+      group_off, counts, M, D.gmax(), static_cast<int>(T), passes, w.win, status, zslice, D.L,
+      zcols, zld));
   return cudaGetLastError();
 }
 
@@ -1232,12 +1240,12 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   // bf16: one compact fp32 slice [L x cols] serves every sweep -- zeroed
   // before the first, then rounded into y's columns and zeroed in place
   // (its lines stay in L2) between sweeps, and dropped after the last.
-  // fp32: the slices are y's own columns.  On the window path the window
-  // sort clears the first slice.
+  // fp32: the slices are y's own columns.  The window sort clears the first
+  // slice.
   const int64_t ld = ycast ? cols : D.d;
   auto slice = [&](int q) { return ycast ? acc : acc + static_cast<int64_t>(q) * cols; };
-  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, win_lo,
-                                 win_lo != nullptr ? slice(0) : nullptr, cols, ld, status, s);
+  cudaError_t err = launch_wsort(D, tt, te, tg, group_off, counts, w, win_lo, slice(0), cols, ld,
+                                 status, s);
   if (err != cudaSuccess) return err;
   // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
   constexpr int R = 3;
@@ -1261,7 +1269,6 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
   // of loads in flight per lane)
   constexpr int NB = NVQ * 32 * kEpv<T> / 128;
   constexpr int PD = 8 / NVQ;
-  if (win_lo == nullptr) err = launch_finish(D, nullptr, 0, nullptr, slice(0), ld, cols, false, s);
   for (int q = 0; q < Q && err == cudaSuccess; ++q) {
     err = launch_acc<T, NB, PD>(D, q * cols, V, w, slice(q), ld, s);
     if (err != cudaSuccess) break;

@@ -566,7 +566,10 @@ __global__ void __launch_bounds__(256) k_select_wide(const float* __restrict__ Z
                                                      float* __restrict__ gate,
                                                      float* __restrict__ score, WidePlan P,
                                                      float* __restrict__ zero, int64_t zero_words) {
-  // the caller's buffer to clear needs nothing from the kernel ahead of this one
+  // The buffer to clear (passed by the fused forward only) is cleared before
+  // the wait.  The kernel ahead is that forward's router, which lets this
+  // one start only after its own wait, so every earlier user of the buffer
+  // has finished.
   if (zero != nullptr) {
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
