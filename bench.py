@@ -69,8 +69,6 @@ def expert_stage_bytes(cfg, n_active):
 # whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
     # re-captured after every change to the stage's kernels; until then none
-    "bf16-prefill-N1M": (6.69e9, "ncu dram__bytes of bf16-prefill-proxy-N256K (window sort, k_act, "
-                                 "2 x k_acc, 3 x k_slice_finish), scaled x3.90 by algorithmic bytes"),
 }
 
 

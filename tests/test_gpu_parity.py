@@ -490,3 +490,32 @@ def test_fused_workspace_reuse(cfg):
     for x, y in zip((d["x"], x2), ys):
         y_fresh = omni.moe_forward(D, x, d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"])
         assert rel_err(host_f64(y), host_f64(y_fresh)) <= tol_y(cfg)
+
+
+def test_expert_sweeps_back_to_back():
+    """Two grouped executions in a row on one workspace and stream, the second
+    on other gates: the second's first clear of the accumulator slice must wait
+    for the first call's last read of it."""
+    cfg = SWEEP[0]
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    oi, og, _ = O.route(cfg, h)
+    D = omni.LayerDims.of(cfg)
+    ws = omni.Workspace()
+    scheds, refs = [], []
+    for scale in (1.0, -0.5):
+        g32 = (og * scale).astype(np.float32)
+        ref_s = O.schedule(cfg, oi, g32.astype(np.float64))
+        refs.append(O.forward_expert(cfg, h, ref_s)[0])
+        counts = torch.tensor([ref_s["n_active"], ref_s["n_groups"], 0, 0], dtype=torch.int32,
+                              device="cuda")
+        scheds.append({"task_token": dev(ref_s["task_token"]),
+                       "task_expert": dev(ref_s["task_expert"]),
+                       "task_gate": dev(ref_s["task_gate"].astype(np.float32)),
+                       "uniq": dev(ref_s["uniq"]), "group_off": dev(ref_s["group_off"]),
+                       "counts": counts})
+    torch.cuda.synchronize()
+    ys = [omni.expert_forward(D, d["x"], d["W"], d["V"], sc, ws=ws) for sc in scheds]
+    torch.cuda.synchronize()
+    for y, y_ref in zip(ys, refs):
+        assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
