@@ -69,6 +69,9 @@ def expert_stage_bytes(cfg, n_active):
 # whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
     # re-captured after every change to the stage's kernels; until then none
+    "bf16-prefill-N1M": (6.69e9, "ncu dram__bytes of bf16-prefill-proxy-N256K (k_act, 2 x k_acc, "
+                                 "2 x k_slice_finish; k_wsort's 3.2 MB from a capture before it "
+                                 "took the first slice's clear), scaled x3.90 by algorithmic bytes"),
 }
 
 
