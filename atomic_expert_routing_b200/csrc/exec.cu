@@ -1162,9 +1162,12 @@ int sm_count() {
   return sms;
 }
 
-// about one window per SM, within what one CTA sorts
+// About one window per SM of a B200 (148), within what one CTA sorts.  A
+// function of the batch alone, not of the device queried: workspace sizes
+// computed before a launch hold for it on any device.
 int64_t window_tasks(const Dims& D) {
-  const int64_t T = (D.M() + sm_count() - 1) / sm_count();
+  constexpr int64_t kWindowsPerBatch = 148;
+  const int64_t T = (D.M() + kWindowsPerBatch - 1) / kWindowsPerBatch;
   return T < 1024 ? 1024 : (T > kWinTasks ? kWinTasks : T);
 }
 
