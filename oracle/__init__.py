@@ -27,9 +27,12 @@ class _Dims(C.Structure):
 
 
 def lib():
+    """The oracle's shared library.  ``OMNI_ORACLE_LIB`` names another build of
+    ``oracle.c`` instead: the mutation tests run the pins against copies with
+    one planted mistake each, loaded this way in a child process."""
     global _lib
     if _lib is None:
-        _lib = C.CDLL(_build.build())
+        _lib = C.CDLL(os.environ.get("OMNI_ORACLE_LIB") or _build.build())
         _lib.oracle_num_threads.restype = C.c_int
     return _lib
 

@@ -13,13 +13,20 @@ SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+FLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+
+def compile_source(src: str, out: str, quiet: bool = False) -> None:
+    """gcc ``src`` into the shared library ``out`` with the oracle's flags."""
+    subprocess.run(["gcc", *FLAGS, "-o", out, src, "-lm"], check=True,
+                   capture_output=quiet)
+
+
 def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
-           "-o", tmp, SRC, "-lm"]
-    subprocess.run(cmd, check=True)
+    compile_source(SRC, tmp)
     os.replace(tmp, LIB)
     return LIB
 

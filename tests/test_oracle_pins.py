@@ -13,6 +13,7 @@ import os
 import numpy as np
 import pytest
 from scipy.special import expit, logsumexp, softmax
+from scipy.special import log_softmax as scipy_log_softmax
 
 import oracle as O
 import workloads as WL
@@ -50,6 +51,39 @@ def test_kxk_path_equals_bruteforce(name, inputs_cache):
     np.testing.assert_allclose(score, bs, rtol=0, atol=0)
     # the K-th score beats the (K+1)-th (strict order by (S desc, e asc))
     assert np.all(bs[:, -1] >= nxt)
+
+
+def test_row_log_softmax_matches_scipy():
+    """The oracle's row-wise log-softmax (applied to logits the caller brings)
+    against scipy's, on rows of different scales, and against the log-softmax
+    the oracle's own routing applies to its axis logits."""
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((7, 33)) * np.array([1e-3, 1, 3, 10, 50, 200, 700])[:, None]
+    np.testing.assert_allclose(O.log_softmax(z), scipy_log_softmax(z, axis=1), rtol=1e-14,
+                               atol=1e-12)
+    cfg = _small(L=12)
+    inp = WL.make_inputs(cfg, experts=False)
+    zr, zc = O.axis_logits(cfg, inp)
+    lr, lc = O.axis_logprobs(cfg, inp)
+    np.testing.assert_array_equal(O.log_softmax(zr), lr)
+    np.testing.assert_array_equal(O.log_softmax(zc), lc)
+
+
+def test_bruteforce_matches_numpy_sort():
+    """The brute force against numpy on all N joint scores S = lr[i] + lc[j]
+    (e = i*Nc + j): its K ids are np.lexsort's first K by (S desc, e asc), its
+    scores are theirs, and its near-tie reference is the (K+1)-th best score."""
+    for cfg in (_small(L=16), _small(L=16, k=4, K=7), WL.TINY.with_(L=16)):
+        inp = WL.make_inputs(cfg, experts=False)
+        lr, lc = O.axis_logprobs(cfg, inp)
+        idx, _, score, nxt = O.select_bruteforce(cfg, lr, lc)
+        S = (lr[:, :, None] + lc[:, None, :]).reshape(cfg.L, cfg.N)
+        ids = np.arange(cfg.N)
+        for t in range(cfg.L):
+            order = np.lexsort((ids, -S[t]))
+            np.testing.assert_array_equal(idx[t], order[:cfg.K])
+            np.testing.assert_array_equal(score[t], S[t, order[:cfg.K]])
+            assert nxt[t] == S[t, order[cfg.K]]
 
 
 @pytest.mark.parametrize("name", ["tiny-fp32", "bf16-N16K", "bf16-skewed-N256K",
@@ -145,6 +179,62 @@ def test_hand_worked_example():
     np.testing.assert_allclose(y[0], [2 / 3 * 0.75 * ln3, 1 / 3 * (-2 / (1 + math.e ** 2))],
                                atol=1e-7)
     assert rows == (2, 2)
+
+
+# bf16 bit patterns and their values, decoded by hand from the format (1 sign
+# bit, 8 exponent bits with bias 127, 7 mantissa bits)
+_BF16_HAND = [
+    (0x3F80, 1.0),
+    (0xC000, -2.0),
+    (0x4049, 3.140625),                     # 2 * (1 + 73/128)
+    (0x3F81, 1.0078125),                    # 1 + 2^-7
+    (0xBE80, -0.25),                        # exponent 125
+    (0x0001, 2.0 ** -133),                  # smallest subnormal: 2^-7 * 2^-126
+    (0x7F7F, 2.0 ** 127 * 255 / 128),       # largest finite
+    (0x8000, -0.0),
+]
+
+
+def test_bf16_widening_and_rounding_of_the_input_generator():
+    """The shared input generator's bf16 helpers against hand-decoded values:
+    exact widening, and round-to-nearest with ties to even."""
+    bits = np.array([b for b, _ in _BF16_HAND], np.uint16)
+    vals = WL.bf16_bits_to_f32(bits).astype(np.float64)
+    for (b, want), got in zip(_BF16_HAND, vals):
+        assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), hex(b)
+    np.testing.assert_array_equal(WL.f32_to_bf16_bits(vals.astype(np.float32)), bits)
+    f = np.array([1.0 + 2.0 ** -8,                # half-way, 0x3F80 is even
+                  1.0 + 3 * 2.0 ** -8,            # half-way, 0x3F82 is even
+                  1.0 + 2.0 ** -8 + 2.0 ** -20,   # just above half-way
+                  -(1.0 + 2.0 ** -8 - 2.0 ** -20),  # just below half-way, negative
+                  float(np.float32(math.pi))], np.float32)
+    np.testing.assert_array_equal(WL.f32_to_bf16_bits(f),
+                                  np.array([0x3F80, 0x3F82, 0x3F81, 0xBF80, 0x4049], np.uint16))
+
+
+def test_bf16_storage_is_read_exactly():
+    """bf16-stored operands enter the oracle at their exact values: with x = 1
+    (d = 1) each raw row logit is the hand-decoded value of one stored key."""
+    cfg = WL.Config("bits", L=1, d=1, Nr=len(_BF16_HAND), Nc=2, k=1, K=1, B=1, dtype=WL.BF16)
+    inp = {
+        "x": np.array([[0x3F80]], np.uint16),
+        "Wr": np.array([[b] for b, _ in _BF16_HAND], np.uint16),
+        "Wc": np.array([[0x3F80], [0xC000]], np.uint16),
+    }
+    zr, zc = O.axis_logits(cfg, inp)
+    np.testing.assert_array_equal(zr[0], [v for _, v in _BF16_HAND])
+    np.testing.assert_array_equal(zc[0], [1.0, -2.0])
+
+
+def test_bf16_router_logits_match_numpy():
+    """Raw router logits of a bf16 workload against numpy's x @ Wr^T on the
+    widened operands (Nr != Nc, so a transposed router matrix fails too)."""
+    cfg = _small(dtype=WL.BF16, d=96, L=40)
+    inp = WL.make_inputs(cfg, experts=False)
+    x, Wr, Wc = (_f64(inp[n], cfg) for n in ("x", "Wr", "Wc"))
+    zr, zc = O.axis_logits(cfg, inp)
+    np.testing.assert_allclose(zr, x @ Wr.T, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(zc, x @ Wc.T, rtol=1e-13, atol=1e-13)
 
 
 def test_equal_logits_break_ties_by_smaller_id():
