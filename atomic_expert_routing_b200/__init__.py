@@ -22,7 +22,7 @@ from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_WS_EXPERT, O
                    OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
 
 __all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",
-           "token_centric_forward", "new_counts", "OmniError", "workspace_size"]
+           "token_centric_forward", "new_counts", "OmniError", "workspace_size", "wait_selftest"]
 
 
 @dataclass(frozen=True)
@@ -237,3 +237,11 @@ def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, y=None, counts=No
         C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(idx), _ptr(gate), _ptr(y), _ptr(counts),
         None, 0, _stream(stream)))
     return y
+
+
+def wait_selftest(counts, *, stream=None):
+    """Makes one bounded device wait run out (about 1 s): afterwards counts[2]
+    holds OMNI_DEV_TIMEOUT.  A check of the failure reporting, not a layer op."""
+    _device(counts)
+    _lib.check("omni_wait_selftest", _lib.load().omni_wait_selftest(_ptr(counts),
+                                                                    _stream(stream)))

@@ -43,6 +43,7 @@ SIGNATURES = {
     "omni_expert_forward_noalloc": ([_P] * 12, C.c_int),
     "omni_moe_forward": ([_P] * 13 + [C.c_size_t, _P], C.c_int),
     "omni_token_centric_forward": ([_P] * 9 + [C.c_size_t, _P], C.c_int),
+    "omni_wait_selftest": ([_P, _P], C.c_int),
 }
 
 

@@ -116,6 +116,18 @@ int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, con
       omni::launch_select(D, Z, parts, br, bc, idx, gate, score, s, zero, zero_words, zeroed));
 }
 
+// Diagnostic: one thread waits on a shared-memory barrier that expects one
+// arrival nobody makes.  The library's bounded wait gives up, ORs
+// OMNI_DEV_TIMEOUT into *status and the kernel returns.
+__global__ void k_wait_selftest(int32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  omni::pdl_wait();  // the caller's writes to *status come first
+  if (threadIdx.x != 0) return;
+  const uint32_t b = omni::smem_u32(&bar);
+  omni::mbar_init(b, 1);
+  omni::mbar_wait(b, 0, status);
+}
+
 bool tensors_ok(const void* const* p16, int n16) {
   for (int i = 0; i < n16; ++i)
     if (p16[i] == nullptr || !al(p16[i], 16)) return false;
@@ -127,6 +139,12 @@ bool tensors_ok(const void* const* p16, int n16) {
 extern "C" {
 
 int omni_abi_version(void) { return OMNI_ABI_VERSION; }
+
+int omni_wait_selftest(int32_t* counts, void* stream) {
+  if (counts == nullptr || !al(counts, 4)) return OMNI_ERR_INVALID_ARG;
+  return cuda_status(omni::launch_k(k_wait_selftest, 1, 32, 0,
+                                    static_cast<cudaStream_t>(stream), counts + 2));
+}
 
 const char* omni_last_cuda_error_name(void) { return cudaGetErrorName(g_last_cuda); }
 

@@ -30,7 +30,12 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Every spin wait of the library ends by time (kWaitLimitNs on the global
+// timer) and, independently of the timer, by a count of failed polls: a poll
+// takes at least tens of nanoseconds, so kWaitMaxPolls polls last about a
+// second or more.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+constexpr uint32_t kWaitMaxPolls = 1u << 26;
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -139,13 +144,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity; gives up after kWaitLimitNs,
-// raising OMNI_DEV_TIMEOUT.  Returns false on time-out.
+// Wait for the phase with the given parity; gives up after kWaitLimitNs or
+// kWaitMaxPolls failed polls, whichever comes first, raising
+// OMNI_DEV_TIMEOUT.  Returns false on time-out.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
+  for (uint32_t polls = 1; !mbar_try_wait(bar, parity); ++polls) {
+    if (polls >= kWaitMaxPolls || global_ns() - t0 > kWaitLimitNs) {
       raise_status(status, OMNI_DEV_TIMEOUT);
       return false;
     }

@@ -89,7 +89,7 @@ template <int BN>
 constexpr size_t tc_smem_bytes() {
   return 1024 /* alignment slack */ +
          static_cast<size_t>(TC_STAGES) * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) +
-         (2 * TC_STAGES + 4) * 8 + 16;
+         (2 * TC_STAGES + 5) * 8 + 16;
 }
 
 // Tile t of the grid of tiles: M block, N tile (rows then columns of the
@@ -122,11 +122,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_STAGES * A_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 5);
+  uint32_t* aborted = tmem_slot + 1;  // a wait of this CTA timed out
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + TC_STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * TC_STAGES);       // accumulator b ready
   const uint32_t tempty0 = smem_u32(bars + 2 * TC_STAGES + 2);  // accumulator b drained
+  const uint32_t drain = smem_u32(bars + 2 * TC_STAGES + 4);    // MMAs in flight, after a time-out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ld = static_cast<int64_t>(Nr) + Nc;
@@ -141,6 +143,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 128);
     }
+    mbar_init(drain, 1);
+    *aborted = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -156,6 +160,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
+  bool timed_out = false;
+  uint32_t issued = 0;  // producer: TMA stages loaded
   if (warp == 4 && lane == 0) {
     // producer: TMA loads, one ring of stages across all of this CTA's tiles
     uint32_t it = 0;
@@ -181,6 +187,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tma_load_2d(smem_u32(sB + s * B_BYTES), tmB, full0 + 8 * s, (kb0 + kb) * TC_BK, n0);
       }
     }
+    timed_out = !ok;
+    issued = it;
   } else if (warp == 5 && lane == 0) {
     // MMA issuer: tile j of this CTA accumulates in TMEM columns (j & 1) * BN
     constexpr uint32_t idesc = idesc_bf16<BN>();
@@ -194,7 +202,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int nk = (T.nk_all - kb0 < T.kper ? T.nk_all - kb0 : T.kper);
       const int b = j & 1;
       const uint32_t use = static_cast<uint32_t>(j >> 1);
-      if (!mbar_wait(tempty0 + 8 * b, (use & 1) ^ 1, status)) break;  // drained by the epilogue
+      if (!mbar_wait(tempty0 + 8 * b, (use & 1) ^ 1, status)) {  // drained by the epilogue
+        ok = false;
+        break;
+      }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
       for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -215,6 +226,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       umma_commit(tfull0 + 8 * b);
     }
+    timed_out = !ok;
   } else if (warp < 4) {
     // epilogue: TMEM lane (32*warp + lane) holds row m0 + 32*warp + lane
     int j = 0;
@@ -224,7 +236,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int b = j & 1;
       const uint32_t use = static_cast<uint32_t>(j >> 1);
       // the wait's outcome is made warp-uniform: tcgen05.ld below is .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * b, use & 1, status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * b, use & 1, status))) {
+        timed_out = true;
+        break;
+      }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const bool colax = n >= T.tiles_r;
       const int n0 = (colax ? n - T.tiles_r : n) * BN;
@@ -254,8 +269,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_arrive(tempty0 + 8 * b);
     }
   }
+  if (timed_out) *aborted = 1u;
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
+  if (*aborted != 0u) {
+    // a wait timed out: this CTA's own TMA loads and MMAs still in flight
+    // land (each wait bounded again) before TMEM is freed and the CTA exits.
+    // The last TC_STAGES loads went to distinct stages, each in its latest
+    // phase; one commit tracks every MMA the issuing thread started.
+    if (warp == 4 && lane == 0) {
+      const uint32_t first = issued > TC_STAGES ? issued - TC_STAGES : 0u;
+      for (uint32_t i = first; i < issued; ++i)
+        mbar_wait(full0 + 8 * (i % TC_STAGES), (i / TC_STAGES) & 1, status);
+    } else if (warp == 5 && lane == 0) {
+      umma_commit(drain);
+      mbar_wait(drain, 0, status);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+  }
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN)

@@ -274,11 +274,12 @@ __global__ void __launch_bounds__(kRsThreads)
   } else {
     st_relaxed(mine, kLbAgg | local);
     const uint64_t t0 = global_ns();
+    uint32_t polls = 0;
     for (int64_t pt = tile - 1; pt >= 0;) {
       const uint32_t v = ld_relaxed(look + pt * 256 + d);
       const uint32_t state = v & ~kLbCount;
       if (state == 0u) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (++polls >= kWaitMaxPolls || global_ns() - t0 > kWaitLimitNs) {
           raise_status(status, OMNI_DEV_TIMEOUT);
           break;
         }

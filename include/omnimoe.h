@@ -218,6 +218,18 @@ const char* omni_last_cuda_error_name(void);
 /* OMNI_ABI_VERSION of the loaded library. */
 int omni_abi_version(void);
 
+/* Diagnostic of the library's failure reporting, not an operation of the
+ * layer.  Every spin wait inside the kernels is bounded: after about 1 s (or
+ * a fixed number of failed polls) it gives up, ORs OMNI_DEV_TIMEOUT into
+ * counts[2] and its kernel returns, so that the context stays usable.  This
+ * call makes one such wait run out: one thread waits on a shared-memory
+ * barrier that nothing completes.
+ * counts: device int32[4], 4-byte aligned, caller-owned; only counts[2] is
+ * written (OR).  Asynchronous on the stream; the wait takes about 1 s of one
+ * thread.  Returns OMNI_ERR_INVALID_ARG for a null or misaligned counts,
+ * OMNI_ERR_CUDA if the launch fails. */
+int omni_wait_selftest(int32_t* counts, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -100,6 +100,9 @@ def test_host_checks_reject_before_any_launch(lib):
     # the fused call needs counts
     assert lib.omni_moe_forward(C.byref(D), *([fake] * 10), None, fake, 1 << 30,
                                 None) == _lib.OMNI_ERR_INVALID_ARG
+    # the wait diagnostic needs an aligned counts
+    assert lib.omni_wait_selftest(None, None) == _lib.OMNI_ERR_INVALID_ARG
+    assert lib.omni_wait_selftest(C.c_void_p(4096 + 2), None) == _lib.OMNI_ERR_INVALID_ARG
 
 
 def test_empty_batch_is_a_no_op(lib):
