@@ -425,44 +425,95 @@ def run_ours(args):
         return out
 
     def measure_e2e(c, dd, steps, warmup):
-        """The public call with host buffers: pinned x -> device, forward, y -> pinned host."""
+        """The public call with host buffers: every step copies its x from pinned
+        host memory to the device, runs the forward and copies its y back to
+        pinned host memory.  Returns (serial ms, pipelined ms, H2D bytes, D2H
+        bytes) per step.
+
+        Serial: copy in, forward, copy out on one stream, one step at a time.
+        Pipelined (double buffers, three streams): the copy-in of step i+1 and
+        the copy-out of step i-1 run while step i computes, as a serving loop
+        would; the L2 flush of each step runs on the compute stream inside the
+        timed region, and one pair of events spans all the steps, from the
+        first copy in to the last copy out."""
         D = omni.LayerDims.of(c)
         xh = torch.empty((c.L, c.d), dtype=D.torch_dtype).pin_memory()
         xh.copy_(dd["x"].cpu())
-        yh = torch.empty((c.L, c.d), dtype=D.torch_dtype).pin_memory()
-        xd = torch.empty_like(dd["x"])
-        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        yh = [torch.empty((c.L, c.d), dtype=D.torch_dtype).pin_memory() for _ in range(2)]
+        xd = [torch.empty_like(dd["x"]) for _ in range(2)]
+        y = [torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device) for _ in range(2)]
         counts = omni.new_counts(device)
         ws = omni.Workspace()
-        stream = torch.cuda.Stream(device)
+        comp, h2d, d2h = (torch.cuda.Stream(device) for _ in range(3))
 
-        def step():
-            xd.copy_(xh, non_blocking=True)
-            omni.moe_forward(D, xd, dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
-                             dd["bias_c"], y=y, counts=counts, ws=ws, stream=stream)
-            yh.copy_(y, non_blocking=True)
+        def fwd(j):
+            omni.moe_forward(D, xd[j], dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                             dd["bias_c"], y=y[j], counts=counts, ws=ws, stream=comp)
 
-        with torch.cuda.stream(stream):
+        def serial_step():
+            xd[0].copy_(xh, non_blocking=True)
+            fwd(0)
+            yh[0].copy_(y[0], non_blocking=True)
+
+        with torch.cuda.stream(comp):
             for _ in range(warmup):
                 flush.zero_()
-                step()
+                serial_step()
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
-        with torch.cuda.stream(stream):
+        with torch.cuda.stream(comp):
             for a, b in ev:
                 flush.zero_()
-                a.record(stream)
-                step()
-                b.record(stream)
+                a.record(comp)
+                serial_step()
+                b.record(comp)
         torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
-        return ms, xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+        serial_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+
+        x_ready = [torch.cuda.Event() for _ in range(2)]
+        x_free = [torch.cuda.Event() for _ in range(2)]
+        y_ready = [torch.cuda.Event() for _ in range(2)]
+        y_free = [torch.cuda.Event() for _ in range(2)]
+
+        def pipeline(n):
+            for i in range(n):
+                j = i & 1
+                if i >= 2:  # buffer j: step i-2 has read its x and its y has left
+                    h2d.wait_event(x_free[j])
+                    comp.wait_event(y_free[j])
+                with torch.cuda.stream(h2d):
+                    xd[j].copy_(xh, non_blocking=True)
+                x_ready[j].record(h2d)
+                comp.wait_event(x_ready[j])
+                with torch.cuda.stream(comp):
+                    flush.zero_()
+                    fwd(j)
+                x_free[j].record(comp)
+                y_ready[j].record(comp)
+                d2h.wait_event(y_ready[j])
+                with torch.cuda.stream(d2h):
+                    yh[j].copy_(y[j], non_blocking=True)
+                y_free[j].record(d2h)
+
+        pipeline(max(warmup, 2))
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(h2d)
+        comp.wait_event(t0)
+        d2h.wait_event(t0)
+        pipeline(steps)
+        t1.record(d2h)  # the last copy out follows every other operation of the steps
+        torch.cuda.synchronize()
+        pipe_ms = t0.elapsed_time(t1) / steps
+        return serial_ms, pipe_ms, xh.numel() * xh.element_size(), yh[0].numel() * yh[0].element_size()
 
     ms, n_active, status, clocks, _, kernels = measure(cfg, d, args.steps, args.warmup)
     ms_all = max_over_ranks(ms, world, device)
-    e2e_ms, h2d, d2h = measure_e2e(cfg, d, max(3, args.steps // 2), args.warmup)
+    e2e_steps = max(8, args.steps)
+    e2e_serial_ms, e2e_ms, h2d, d2h = measure_e2e(cfg, d, e2e_steps, args.warmup)
     e2e_ms = max_over_ranks(e2e_ms, world, device)
+    e2e_serial_ms = max_over_ranks(e2e_serial_ms, world, device)
     st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
     stages = measure_stages(cfg, d, max(3, args.steps // 2))
 
@@ -557,7 +608,12 @@ def run_ours(args):
                      "ms": st_ms, "peak_src": peak_src},
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(world, cfg.L, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": e2e_steps,
+                "mode": "pipelined: double buffers on three streams; the copy in of step i+1 "
+                        "and the copy out of step i-1 overlap step i; L2 flush inside",
+                "serial": {"value": job_throughput(world, cfg.L, e2e_serial_ms),
+                           "ms_per_step": e2e_serial_ms}},
         # the library's kernels in the timed region: kernel nodes of the
         # captured forward (one replay per step)
         "gpu_launches": kernels * args.steps if kernels is not None else None,
