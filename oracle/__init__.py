@@ -137,12 +137,6 @@ def route(cfg, inp, tokens=None):
     return select(cfg, lr, lc)
 
 
-def near_ties(score, nxt, rel=1e-4):
-    """Boolean per token: K-th and (K+1)-th best joint scores differ by < rel * |S_K|."""
-    sk = score[:, -1]
-    return np.abs(sk - nxt) < rel * np.abs(sk)
-
-
 def schedule(cfg, idx, gate, tokens=None):
     """Expert-centric schedule of the tasks of the listed tokens (dict of arrays)."""
     tok = _tokens(cfg, tokens)
