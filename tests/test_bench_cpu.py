@@ -1,6 +1,7 @@
-"""The benchmark's reference arm (the fp64 oracle on the host cores) on the CPU:
-its JSON line carries the contract's keys, at least 3 warm-up steps run, and
-ranks other than 0 do no work."""
+"""The benchmark on the CPU.  Its reference arm (the fp64 oracle on the host
+cores): the JSON line carries the contract's keys, at least 3 warm-up steps
+run, and ranks other than 0 do no work.  Its roofline arithmetic, worked by
+hand."""
 import json
 import os
 import subprocess
@@ -40,3 +41,39 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = _run({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def _golden_traffic():
+    rows = {}
+    with open(os.path.join(ROOT, "tests", "golden", "traffic_model.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()
+                rows[k] = v
+    return rows
+
+
+def test_roofline_arithmetic():
+    """The bench's algorithmic work, worked by hand at the prefill and decode
+    sizes: F = 2d(Nr+Nc)L + 4dLK, layer bytes = x + Wr + Wc + 2d|E|esize + y,
+    the expert stage's bytes = 2d|E|esize + x + y, and its parameter bytes are
+    the pages' expert-centric traffic 2d|E_active| elements (golden file)."""
+    import bench
+    import workloads as WL
+
+    p, n_act = WL.PREFILL, 652642
+    f, b = bench.layer_work(p, n_act)
+    assert f == 137_438_953_472 + 8_589_934_592 == 146_028_888_064
+    x = y = 16384 * 2048 * 2                     # 64 MiB each, bf16
+    keys = 2 * 1024 * 2048 * 2                   # Wr and Wc
+    rows = 2 * 2048 * n_act * 2                  # W and V rows of the active experts
+    assert b == x + keys + rows + y == 5_489_049_600
+    assert bench.expert_stage_bytes(p, n_act) == rows + x + y == 5_480_660_992
+    g = _golden_traffic()
+    env = {"d": p.d, "L": p.L, "K": p.K, "n_active": n_act}
+    assert eval(g["expert_centric"], {}, env) * p.esize == rows
+    assert eval(g["token_centric"], {}, env) * p.esize == 2 * 2048 * 16384 * 64 * 2
+    f, _ = bench.layer_work(WL.DECODE, 4082)
+    assert f == 536_870_912 + 33_554_432 == 570_425_344
+    assert bench.job_throughput(1, 16384, 1.6) == 16384 / 1.6e-3
+    assert bench.job_throughput(4, 16384, 1.6) == 4 * 16384 / 1.6e-3
