@@ -189,9 +189,17 @@ int omni_expert_forward_noalloc(const omni_dims* dims, const void* x, const void
                                 void* y, void* stream);
 
 /*
- * The whole routed branch: omni_route -> omni_schedule -> omni_expert_forward
- * on one stream, intermediates in ws.  idx_out / gate_out (nullable, [L x K])
- * receive the routing decisions.  y as in omni_expert_forward.
+ * The whole routed branch on one stream, intermediates in ws: omni_route,
+ * then scheduling, then grouped execution.  idx_out / gate_out (nullable,
+ * [L x K]) receive the routing decisions; counts[0], counts[1] are written as
+ * by omni_schedule; y as in omni_expert_forward.
+ * Small batches run omni_schedule's order.  Batches whose fp32 accumulator is
+ * executed in column-slice sweeps (L*d*4 above about 40 MiB) go from the
+ * routing straight to the executor's order.  That order is the same groups,
+ * in windows of consecutive groups, with each window's tasks ordered by
+ * token; the (group, token, expert) order itself is not formed.  Every task
+ * is still executed once, so y differs from the staged calls only in the
+ * order of its fp32 additions.
  */
 int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                      const float* bias_r, const float* bias_c, const void* W, const void* V,
