@@ -141,6 +141,7 @@ extern "C" {
 int omni_abi_version(void) { return OMNI_ABI_VERSION; }
 
 int omni_wait_selftest(int32_t* counts, void* stream) {
+  omni::CallRange range("omni_wait_selftest");
   if (counts == nullptr || !al(counts, 4)) return OMNI_ERR_INVALID_ARG;
   return cuda_status(omni::launch_k(k_wait_selftest, 1, 32, 0,
                                     static_cast<cudaStream_t>(stream), counts + 2));
@@ -171,6 +172,7 @@ int omni_workspace_size(const omni_dims* dims, int which, size_t* bytes) {
 int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                const float* bias_r, const float* bias_c, int32_t* idx, float* gate, float* score,
                int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_route");
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -186,6 +188,7 @@ int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void*
 
 int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                        float* logits, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_router_logits");
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -213,6 +216,7 @@ int omni_router_logits(const omni_dims* dims, const void* x, const void* Wr, con
 int omni_route_select(const omni_dims* dims, const float* logits, const float* bias_r,
                       const float* bias_c, int32_t* idx, float* gate, float* score,
                       int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_route_select");
   (void)counts;
   (void)ws;
   (void)ws_bytes;
@@ -229,6 +233,7 @@ int omni_route_select(const omni_dims* dims, const float* logits, const float* b
 int omni_schedule(const omni_dims* dims, const int32_t* idx, const float* gate,
                   int32_t* task_token, int32_t* task_expert, float* task_gate, int32_t* uniq,
                   int32_t* group_off, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_schedule");
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -246,6 +251,7 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
                         const int32_t* task_token, const int32_t* task_expert,
                         const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                         int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_expert_forward");
   (void)uniq;
   Dims D;
   int rc = check_dims(dims, &D);
@@ -265,6 +271,7 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
                      const float* bias_r, const float* bias_c, const void* W, const void* V,
                      void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
                      size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_forward");
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -284,18 +291,30 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   float* acc = acc_words == 0 ? nullptr
                : static_cast<float*>(D.dtype == OMNI_F32 ? y : w.expert);
   bool acc_zeroed = false;
-  rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s, acc,
-                  acc_words, &acc_zeroed);
+  {
+    omni::CallRange stage("route");
+    rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s,
+                    acc, acc_words, &acc_zeroed);
+  }
   if (rc != OMNI_OK) return rc;
   if (fused_windows(D)) {
-    rc = cuda_status(omni::launch_schedule_windows(D, idx, gate, w.uniq, w.group_off, counts,
-                                                   w.sched, omni::expert_windows(D, w.expert), s));
+    {
+      omni::CallRange stage("schedule");
+      rc = cuda_status(omni::launch_schedule_windows(D, idx, gate, w.uniq, w.group_off, counts,
+                                                     w.sched, omni::expert_windows(D, w.expert),
+                                                     s));
+    }
     if (rc != OMNI_OK) return rc;
+    omni::CallRange stage("expert");
     return cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s));
   }
-  rc = cuda_status(omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate,
-                                         w.uniq, w.group_off, counts, w.sched, s));
+  {
+    omni::CallRange stage("schedule");
+    rc = cuda_status(omni::launch_schedule(D, idx, gate, w.task_token, w.task_expert, w.task_gate,
+                                           w.uniq, w.group_off, counts, w.sched, s));
+  }
   if (rc != OMNI_OK) return rc;
+  omni::CallRange stage("expert");
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
                                          w.group_off, counts, y, w.expert, s, acc_zeroed));
 }
@@ -303,6 +322,7 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
 int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,
                                const void* V, const int32_t* idx, const float* gate, void* y,
                                int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_token_centric_forward");
   (void)ws;
   (void)ws_bytes;
   Dims D;

@@ -7,7 +7,19 @@
 
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace omni {
+
+// NVTX range over one ABI call or one stage of it, on the host: it spans the
+// launches the call enqueues, so a profiler can select a stage's kernels by
+// range.  A no-op unless a profiling tool is attached.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 struct Dims {
   int64_t L, d, Nr, Nc, k, K, B;

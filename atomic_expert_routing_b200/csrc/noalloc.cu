@@ -49,6 +49,7 @@ extern "C" int omni_expert_forward_noalloc(const omni_dims* dims, const void* x,
                                            const int32_t* task_expert, const float* task_gate,
                                            const int32_t* uniq, const int32_t* group_off,
                                            int32_t* counts, void* y, void* stream) {
+  omni::CallRange range("omni_expert_forward_noalloc");
   (void)uniq;
   if (dims == nullptr) return OMNI_ERR_INVALID_ARG;
   size_t need = 0;

@@ -55,6 +55,18 @@ def layer_work(cfg, n_active):
     return flops, bytes_
 
 
+def traffic_model(cfg, n_active):
+    """The pages' parameter-traffic model of the two execution orders for one
+    batch: token-centric D = 2d*L*K, expert-centric D = 2d*|E_active| (in
+    bytes of the storage type), and the expert usage |E_active| / N."""
+    e = cfg.esize
+    d_tok = 2 * cfg.d * cfg.L * cfg.K * e
+    d_exp = 2 * cfg.d * n_active * e
+    return {"expert_usage": n_active / cfg.N, "tasks_per_active_expert": cfg.L * cfg.K / n_active
+            if n_active else None, "d_token_centric_bytes": d_tok,
+            "d_expert_centric_bytes": d_exp, "saving": d_tok / d_exp if d_exp else None}
+
+
 def expert_stage_bytes(cfg, n_active):
     """Algorithmic bytes of the grouped execution: active rows of W and V once,
     x read, y written."""
@@ -593,6 +605,7 @@ def run_ours(args):
                    "N": cfg.N, "k": cfg.k, "K": cfg.K, "B": cfg.B, "l2": "flushed before each step",
                    "graph": True, "parallelism": f"dp{world} (independent token batches)"},
         "n_active": n_active,
+        "traffic_model": traffic_model(cfg, n_active),
         "device_status": status,
         "stages_ms": stages,
         "ablation": ablation,

@@ -77,3 +77,21 @@ def test_roofline_arithmetic():
     assert f == 536_870_912 + 33_554_432 == 570_425_344
     assert bench.job_throughput(1, 16384, 1.6) == 16384 / 1.6e-3
     assert bench.job_throughput(4, 16384, 1.6) == 4 * 16384 / 1.6e-3
+
+
+def test_traffic_model_of_the_pages():
+    """Token-centric 2d*L*K against expert-centric 2d*|E_active| parameter
+    traffic (golden formulas), in bytes, with the expert usage |E|/N."""
+    import bench
+    import workloads as WL
+
+    p, n_act = WL.PREFILL, 652642
+    t = bench.traffic_model(p, n_act)
+    g = _golden_traffic()
+    env = {"d": p.d, "L": p.L, "K": p.K, "n_active": n_act}
+    assert t["d_token_centric_bytes"] == eval(g["token_centric"], {}, env) * 2 == 8_589_934_592
+    assert t["d_expert_centric_bytes"] == eval(g["expert_centric"], {}, env) * 2 == 5_346_443_264
+    assert abs(t["saving"] - 8_589_934_592 / 5_346_443_264) < 1e-12
+    assert abs(t["expert_usage"] - n_act / 2 ** 20) < 1e-15
+    assert abs(t["tasks_per_active_expert"] - 16384 * 64 / n_act) < 1e-12
+    assert bench.traffic_model(WL.TINY, 0)["saving"] is None
