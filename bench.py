@@ -67,6 +67,19 @@ def traffic_model(cfg, n_active):
             "d_expert_centric_bytes": d_exp, "saving": d_tok / d_exp if d_exp else None}
 
 
+def group_stats(group_off, B, n_active):
+    """Tasks per group of a schedule, from its group offsets (int array of
+    n_groups + 1 entries): count, min / median / mean / max, and the number of
+    experts in the last group (the others hold B)."""
+    go = np.asarray(group_off, dtype=np.int64)
+    per = np.diff(go)
+    if per.size == 0:
+        return {"groups": 0}
+    return {"groups": int(per.size), "tasks_min": int(per.min()),
+            "tasks_median": float(np.median(per)), "tasks_mean": float(per.mean()),
+            "tasks_max": int(per.max()), "experts_in_last_group": int(n_active - B * (per.size - 1))}
+
+
 def expert_stage_bytes(cfg, n_active):
     """Algorithmic bytes of the grouped execution: active rows of W and V once,
     x read, y written."""
@@ -386,18 +399,25 @@ def run_ours(args):
             omni.expert_forward(D, dd["x"], dd["W"], dd["V"], s, y=y, ws=we)
             if evs:
                 evs[3].record(stream)
+            return s
 
-        one()
+        s = one()
         torch.cuda.synchronize()
         tot = [0.0, 0.0, 0.0]
         for _ in range(steps):
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             flush.zero_()
-            one(evs)
+            s = one(evs)
             torch.cuda.synchronize()
             for i in range(3):
                 tot[i] += evs[i].elapsed_time(evs[i + 1])
-        return {"route": tot[0] / steps, "schedule": tot[1] / steps, "expert": tot[2] / steps}
+        out = {"route": tot[0] / steps, "schedule": tot[1] / steps, "expert": tot[2] / steps}
+        try:  # a diagnostic: it may not cost the line
+            na, ng = (int(v) for v in counts[:2].cpu().tolist())
+            out["groups"] = group_stats(s["group_off"][: ng + 1].cpu().numpy(), c.B, na)
+        except Exception as exc:  # noqa: BLE001
+            out["groups"] = {"error": repr(exc)[:200]}
+        return out
 
     def measure_ablation(c, dd, steps):
         """The pages' comparison on the same routing: expert-centric execution
@@ -528,6 +548,7 @@ def run_ours(args):
     e2e_serial_ms = max_over_ranks(e2e_serial_ms, world, device)
     st_ms, n_act2 = measure_expert_stage(cfg, d, max(3, args.steps // 2))
     stages = measure_stages(cfg, d, max(3, args.steps // 2))
+    sched_groups = stages.pop("groups", None)
 
     ablation = measure_ablation(cfg, d, max(3, args.steps // 2))
 
@@ -541,7 +562,9 @@ def run_ours(args):
                                   "frac": max(f2 / (tc * 1e12), b2 / (hbm * 1e9)) / (ms2 * 1e-3),
                                   "bytes": b2, "flops": f2}}
         if with_stages:
-            rec["stages_ms"] = measure_stages(sc, dd, 10)
+            st2 = measure_stages(sc, dd, 10)
+            rec["schedule_groups"] = st2.pop("groups", None)
+            rec["stages_ms"] = st2
             rec["ablation"] = measure_ablation(sc, dd, 10)
         return rec
 
@@ -608,6 +631,7 @@ def run_ours(args):
         "traffic_model": traffic_model(cfg, n_active),
         "device_status": status,
         "stages_ms": stages,
+        "schedule_groups": sched_groups,
         "ablation": ablation,
         "layer_roofline": {"bound": "hbm" if t_b >= t_f else "tensor",
                            "frac": max(t_f, t_b) / (ms_all * 1e-3), "bytes": bytes_,

@@ -95,3 +95,13 @@ def test_traffic_model_of_the_pages():
     assert abs(t["expert_usage"] - n_act / 2 ** 20) < 1e-15
     assert abs(t["tasks_per_active_expert"] - 16384 * 64 / n_act) < 1e-12
     assert bench.traffic_model(WL.TINY, 0)["saving"] is None
+
+
+def test_group_stats():
+    """Tasks per group from group offsets, worked by hand."""
+    import bench
+
+    g = bench.group_stats([0, 5, 7, 16, 18], B=4, n_active=14)
+    assert g == {"groups": 4, "tasks_min": 2, "tasks_median": 3.5, "tasks_mean": 4.5,
+                 "tasks_max": 9, "experts_in_last_group": 2}
+    assert bench.group_stats([0], B=4, n_active=0) == {"groups": 0}
