@@ -3,6 +3,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -27,6 +28,15 @@ def _headers() -> list[str]:
 
 def _obj(src: str) -> str:
     return os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+
+
+def report(src: str) -> str:
+    """ptxas resource report (registers, spills, shared memory per kernel) of
+    the last compile of ``src``."""
+    return os.path.join(OBJ, os.path.basename(src)[:-3] + ".ptxas.txt")
+
+
+_RESOURCE_LINE = re.compile(r"^(ptxas info\s*:|\s+\d+ bytes stack frame)")
 
 
 def _stale_obj(src: str, newest_header: float) -> bool:
@@ -60,10 +70,16 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         o = _obj(src)
         tmp = o + f".tmp{os.getpid()}"
         cmd = [nvcc, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
-               "-I", INCLUDE, "-c", "-o", tmp, src]
-        if verbose_ptxas:
-            cmd.insert(1, "-Xptxas=-v")
-        subprocess.run(cmd, check=True)
+               "-Xptxas=-v", "-I", INCLUDE, "-c", "-o", tmp, src]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        # the resource lines go to the report; anything else (warnings,
+        # errors) is shown as the compiler printed it
+        other = "".join(ln for ln in r.stderr.splitlines(True) if not _RESOURCE_LINE.match(ln))
+        sys.stderr.write(r.stdout + (r.stderr if verbose_ptxas else other))
+        if r.returncode != 0:
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+        with open(report(src), "w") as fh:
+            fh.write(r.stderr)
         os.replace(tmp, o)
 
     with ThreadPoolExecutor(max_workers=max(1, min(len(todo), os.cpu_count() or 1))) as ex:
