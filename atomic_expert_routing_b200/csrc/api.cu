@@ -22,11 +22,17 @@ int check_dims(const omni_dims* in, Dims* D) {
     return OMNI_ERR_INVALID_ARG;
   if (D->dtype != OMNI_F32 && D->dtype != OMNI_BF16) return OMNI_ERR_INVALID_ARG;
   if ((D->flags & ~OMNI_FLAG_ROUTER_SIMT) != 0) return OMNI_ERR_INVALID_ARG;
-  if (D->k > D->Nr || D->k > D->Nc || D->K > D->k * D->k) return OMNI_ERR_INVALID_ARG;
+  // k*k in 128 bits: k is only bounded by the axes here
+  if (D->k > D->Nr || D->k > D->Nc ||
+      static_cast<__int128>(D->K) > static_cast<__int128>(D->k) * D->k)
+    return OMNI_ERR_INVALID_ARG;
   if (D->Nr > OMNI_MAX_AXIS || D->Nc > OMNI_MAX_AXIS) return OMNI_ERR_UNSUPPORTED;
   if (D->k > OMNI_MAX_TOPK || D->K > OMNI_MAX_TOPK) return OMNI_ERR_UNSUPPORTED;
   // task counts travel in 30-bit fields of the scheduler's look-back words
-  if (D->N() >= (int64_t(1) << 31) || D->M() >= (int64_t(1) << 30)) return OMNI_ERR_UNSUPPORTED;
+  // (L is bounded first, so L*K cannot overflow)
+  if (D->N() >= (int64_t(1) << 31) || D->L >= (int64_t(1) << 30) ||
+      D->M() >= (int64_t(1) << 30))
+    return OMNI_ERR_UNSUPPORTED;
   if (D->d % 8 != 0 || D->d > (int64_t(1) << 16)) return OMNI_ERR_UNSUPPORTED;
   return OMNI_OK;
 }

@@ -78,9 +78,18 @@ extern "C" {
 #define OMNI_MAX_AXIS 4096      /* Nr, Nc */
 #define OMNI_MAX_TOPK 256       /* k, K */
 
+/* Host checks of omni_dims, made by every call that takes dims.
+ * A field outside its range returns OMNI_ERR_INVALID_ARG:
+ *   L < 0; d, Nr, Nc, k, K or B < 1; k > min(Nr, Nc); K > k*k;
+ *   an unknown dtype or flag.
+ * A valid field beyond this build's limits returns OMNI_ERR_UNSUPPORTED:
+ *   Nr or Nc > OMNI_MAX_AXIS; k or K > OMNI_MAX_TOPK; N >= 2^31;
+ *   L*K >= 2^30; d not a multiple of 8, or d > 65536.
+ * When both apply, OMNI_ERR_INVALID_ARG is returned. */
+
 typedef struct omni_dims {
   int64_t L;     /* tokens in the batch (>= 0; L*K < 2^30 tasks) */
-  int64_t d;     /* model width (multiple of 8; of 4 for OMNI_F32) */
+  int64_t d;     /* model width (a multiple of 8, at most 65536) */
   int64_t Nr;    /* grid rows */
   int64_t Nc;    /* grid columns; N = Nr*Nc atomic experts (< 2^31) */
   int64_t k;     /* per-axis top-k, 1 <= k <= min(Nr, Nc) */

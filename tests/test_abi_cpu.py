@@ -113,3 +113,49 @@ def test_empty_batch_is_a_no_op(lib):
     assert lib.omni_expert_forward(C.byref(D), *([fake] * 10), None, 0, None) == _lib.OMNI_OK
     assert lib.omni_token_centric_forward(C.byref(D), *([fake] * 7), None, 0,
                                           None) == _lib.OMNI_OK
+
+
+def _documented_code(L, d, Nr, Nc, k, K, B, dtype, flags):
+    """The host checks as the header states them (invalid before unsupported)."""
+    if (L < 0 or min(d, Nr, Nc, k, K, B) < 1 or dtype not in (_lib.OMNI_F32, _lib.OMNI_BF16)
+            or flags & ~_lib.OMNI_FLAG_ROUTER_SIMT or k > min(Nr, Nc) or K > k * k):
+        return _lib.OMNI_ERR_INVALID_ARG
+    if (max(Nr, Nc) > 4096 or max(k, K) > 256 or Nr * Nc >= 2 ** 31 or L * K >= 2 ** 30
+            or d % 8 or d > 65536):
+        return _lib.OMNI_ERR_UNSUPPORTED
+    return _lib.OMNI_OK
+
+
+_I64 = 2 ** 63 - 1
+
+
+def test_dims_checks_follow_the_header(lib):
+    """Randomised dims, from ordinary to absurd (up to the int64 range): the
+    library returns the code the header documents, and a positive workspace
+    size of every kind for every accepted dims."""
+    from hypothesis import HealthCheck, example, given, settings, strategies as st
+
+    small = st.integers(-2, 5000)
+    anyint = st.one_of(small, st.integers(-_I64 - 1, _I64), st.sampled_from(
+        [2 ** 30, 2 ** 31, 2 ** 32 + 1, 2 ** 62, _I64]))
+    field = st.one_of(small, small, anyint)
+
+    @settings(max_examples=3000, deadline=None, database=None,
+              suppress_health_check=list(HealthCheck))
+    @given(L=field, d=st.one_of(st.sampled_from([8, 16, 40, 64, 2048, 65536, 65544]), field),
+           Nr=field, Nc=field, k=st.one_of(st.integers(1, 300), field),
+           K=st.one_of(st.integers(1, 300), field), B=field,
+           dtype=st.sampled_from([0, 1, 2, -1]), flags=st.sampled_from([0, 1, 2, 3]))
+    # L*K that wraps around int64; k*k that does
+    @example(L=2 ** 62, d=64, Nr=64, Nc=64, k=2, K=4, B=1, dtype=1, flags=0)
+    @example(L=16, d=64, Nr=2 ** 33, Nc=2 ** 33, k=2 ** 32, K=1, B=1, dtype=1, flags=0)
+    def check(L, d, Nr, Nc, k, K, B, dtype, flags):
+        D = _lib.Dims(L=L, d=d, Nr=Nr, Nc=Nc, k=k, K=K, B=B, dtype=dtype, flags=flags)
+        want = _documented_code(L, d, Nr, Nc, k, K, B, dtype, flags)
+        for which in range(6):
+            rc, n = _wsz(lib, D, which)
+            assert rc == want, (L, d, Nr, Nc, k, K, B, dtype, flags, which)
+            if rc == _lib.OMNI_OK and which in (_lib.OMNI_WS_ROUTE, _lib.OMNI_WS_FUSED) and L > 0:
+                assert n > 0
+
+    check()
