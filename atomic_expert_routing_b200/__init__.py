@@ -2,8 +2,9 @@
 
 Thin binding over the C ABI of ``libomnimoe.so`` (include/omnimoe.h).  Every
 step of the layer runs in the library's CUDA kernels; this module only checks
-tensor placement, allocates outputs and workspace with PyTorch, and passes raw
-pointers and the current CUDA stream.  There is no CPU path: calls need a CUDA
+each tensor's placement, dtype and element count against the dims, allocates
+outputs and workspace with PyTorch, and passes raw pointers and the current
+CUDA stream.  There is no CPU path: calls need a CUDA
 device and the built library and raise otherwise.
 
 Names follow the layer: ``route`` (Cartesian Product Router), ``schedule``
@@ -82,6 +83,51 @@ def _device(*ts):
     raise ValueError("no tensor given")
 
 
+def _expect(name, t, n, dtype, *, optional=False):
+    """Refuse a tensor whose dtype differs from the one the call reads, or
+    that holds fewer than the n elements the call touches.  The C ABI sees
+    only pointers, so this is the one place a too-small buffer becomes an
+    error instead of an out-of-bounds device access."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, the call reads {dtype}")
+    if t.numel() < n:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {n}")
+
+
+def _expect_io(D, **ts):
+    """Checks by argument name: storage-type tensors (x, W, V, Wr, Wc, y),
+    fp32 biases and logits, int32 counts."""
+    f32, i32 = torch.float32, torch.int32
+    spec = {
+        "x": (D.L * D.d, D.torch_dtype), "y": (D.L * D.d, D.torch_dtype),
+        "Wr": (D.Nr * D.d, D.torch_dtype), "Wc": (D.Nc * D.d, D.torch_dtype),
+        "W": (D.N * D.d, D.torch_dtype), "V": (D.N * D.d, D.torch_dtype),
+        "bias_r": (D.Nr, f32), "bias_c": (D.Nc, f32),
+        "logits": (D.L * (D.Nr + D.Nc), f32), "counts": (4, i32),
+        "idx": (D.M, i32), "gate": (D.M, f32),
+    }
+    optional = {"bias_r", "bias_c", "counts", "y", "idx", "gate"}
+    for name, t in ts.items():
+        n, dt = spec[name]
+        _expect(name, t, n, dt, optional=name in optional)
+
+
+def _expect_sched(D, sched):
+    ucap = max(1, min(D.N, D.M))
+    gmax = (ucap + D.B - 1) // D.B
+    i32 = torch.int32
+    for name, n, dt in (("task_token", D.M, i32), ("task_expert", D.M, i32),
+                        ("task_gate", D.M, torch.float32), ("uniq", ucap, i32),
+                        ("group_off", gmax + 1, i32), ("counts", 4, i32)):
+        if name not in sched:
+            raise ValueError(f"schedule entry {name} is missing")
+        _expect(name, sched[name], n, dt)
+
+
 def workspace_size(D: LayerDims, which: int) -> int:
     n = C.c_size_t(0)
     dd = D.c()
@@ -120,6 +166,7 @@ def new_counts(device) -> torch.Tensor:
 def route(D: LayerDims, x, Wr, Wc, bias_r=None, bias_c=None, *, counts=None, ws=None,
           stream=None, with_score=True):
     """Cartesian Product Router: (idx int32 [L,K], gate f32 [L,K], score f32 [L,K] or None)."""
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, bias_r=bias_r, bias_c=bias_c, counts=counts)
     dev = _device(x)
     idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
     gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
@@ -134,6 +181,7 @@ def route(D: LayerDims, x, Wr, Wc, bias_r=None, bias_c=None, *, counts=None, ws=
 
 def router_logits(D: LayerDims, x, Wr, Wc, *, counts=None, ws=None, stream=None):
     """Router projections: float32 [L, Nr + Nc] (row logits, then column logits)."""
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, counts=counts)
     dev = _device(x)
     z = torch.empty((D.L, D.Nr + D.Nc), dtype=torch.float32, device=dev)
     wsp, n = _ws(D, OMNI_WS_ROUTE, dev, ws)
@@ -146,6 +194,7 @@ def router_logits(D: LayerDims, x, Wr, Wc, *, counts=None, ws=None, stream=None)
 
 def route_select(D: LayerDims, logits, bias_r=None, bias_c=None, *, counts=None, stream=None):
     """Selection from axis logits [L, Nr + Nc] (float32)."""
+    _expect_io(D, logits=logits, bias_r=bias_r, bias_c=bias_c, counts=counts)
     dev = _device(logits)
     idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
     gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
@@ -159,6 +208,9 @@ def route_select(D: LayerDims, logits, bias_r=None, bias_c=None, *, counts=None,
 
 def schedule(D: LayerDims, idx, gate, *, counts=None, ws=None, stream=None) -> dict:
     """Expert-Centric Scheduling of the L*K routing decisions (device tensors)."""
+    _expect_io(D, idx=idx, gate=gate, counts=counts)
+    _expect("idx", idx, D.M, torch.int32)
+    _expect("gate", gate, D.M, torch.float32)
     dev = _device(idx)
     M = D.M
     ucap = max(1, min(D.N, M))
@@ -182,6 +234,8 @@ def schedule(D: LayerDims, idx, gate, *, counts=None, ws=None, stream=None) -> d
 
 def expert_forward(D: LayerDims, x, W, V, sched: dict, *, y=None, ws=None, stream=None):
     """Grouped (expert-centric) execution of a schedule; returns y [L, d]."""
+    _expect_io(D, x=x, W=W, V=V, y=y)
+    _expect_sched(D, sched)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
@@ -199,20 +253,27 @@ def expert_forward_noalloc(D: LayerDims, x, W, V, sched: dict, *, y=None, stream
     device memory when the layer runs (the accumulator is a fixed array inside
     the library; L*d <= 4194304; calls must not overlap on the GPU).  Pass y to
     keep the call itself free of allocations."""
+    _expect_io(D, x=x, W=W, V=V, y=y)
+    _expect_sched(D, sched)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
     dd = D.c()
-    _lib.check("omni_expert_forward_noalloc", _lib.load().omni_expert_forward_noalloc(
-        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(sched["task_token"]),
-        _ptr(sched["task_expert"]), _ptr(sched["task_gate"]), _ptr(sched["uniq"]),
-        _ptr(sched["group_off"]), _ptr(sched["counts"]), _ptr(y), _stream(stream)))
+    args = (_ptr(x), _ptr(W), _ptr(V), _ptr(sched["task_token"]), _ptr(sched["task_expert"]),
+            _ptr(sched["task_gate"]), _ptr(sched["uniq"]), _ptr(sched["group_off"]),
+            _ptr(sched["counts"]), _ptr(y))
+    # the library uses the fixed array of the current device
+    with torch.cuda.device(dev):
+        _lib.check("omni_expert_forward_noalloc", _lib.load().omni_expert_forward_noalloc(
+            C.byref(dd), *args, _stream(stream)))
     return y
 
 
 def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=None,
                 counts=None, idx=None, gate=None, ws=None, stream=None):
     """Route -> schedule -> grouped execution in one call; returns y [L, d]."""
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, V=V, bias_r=bias_r, bias_c=bias_c, y=y,
+               counts=counts, idx=idx, gate=gate)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
@@ -229,6 +290,9 @@ def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=No
 def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, y=None, counts=None,
                           stream=None):
     """Token-centric execution (ablation): every token gathers its own experts."""
+    _expect_io(D, x=x, W=W, V=V, y=y, counts=counts)
+    _expect("idx", idx, D.M, torch.int32)
+    _expect("gate", gate, D.M, torch.float32)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
@@ -242,6 +306,7 @@ def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, y=None, counts=No
 def wait_selftest(counts, *, stream=None):
     """Makes one bounded device wait run out (about 1 s): afterwards counts[2]
     holds OMNI_DEV_TIMEOUT.  A check of the failure reporting, not a layer op."""
+    _expect("counts", counts, 4, torch.int32)
     _device(counts)
     _lib.check("omni_wait_selftest", _lib.load().omni_wait_selftest(_ptr(counts),
                                                                     _stream(stream)))

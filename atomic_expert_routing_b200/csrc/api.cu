@@ -8,7 +8,19 @@
 #include "internal.h"
 
 using omni::Carver;
+using omni::cuda_status;
 using omni::Dims;
+
+namespace {
+// last failing CUDA call of this host thread (diagnostics only)
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+}  // namespace
+
+int omni::cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return OMNI_OK;
+  g_last_cuda = e;
+  return OMNI_ERR_CUDA;
+}
 
 namespace {
 
@@ -35,6 +47,16 @@ int check_dims(const omni_dims* in, Dims* D) {
     return OMNI_ERR_UNSUPPORTED;
   if (D->d % 8 != 0 || D->d > (int64_t(1) << 16)) return OMNI_ERR_UNSUPPORTED;
   return OMNI_OK;
+}
+
+// The calls that select experts take the top-K of the k x k candidate pairs.
+// That equals the top-K over all N joint scores only when k >= K (a row
+// outside the top-k is beaten by at least k >= K others), so they refuse
+// K > k.  Scheduling and execution do not use k and take any K <= k*k.
+int check_route_dims(const omni_dims* in, Dims* D) {
+  const int rc = check_dims(in, D);
+  if (rc != OMNI_OK) return rc;
+  return D->K > D->k ? OMNI_ERR_UNSUPPORTED : OMNI_OK;
 }
 
 // workspace layouts
@@ -96,14 +118,6 @@ int ws_ok(const Dims& D, int which, const void* ws, size_t ws_bytes) {
   return OMNI_OK;
 }
 
-// last failing CUDA call of this host thread (diagnostics only)
-thread_local cudaError_t g_last_cuda = cudaSuccess;
-
-int cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return OMNI_OK;
-  g_last_cuda = e;
-  return OMNI_ERR_CUDA;
-}
 
 int route_impl(const Dims& D, const void* x, const void* Wr, const void* Wc, const float* br,
                const float* bc, int32_t* idx, float* gate, float* score, int32_t* status,
@@ -180,7 +194,7 @@ int omni_route(const omni_dims* dims, const void* x, const void* Wr, const void*
                int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
   omni::CallRange range("omni_route");
   Dims D;
-  int rc = check_dims(dims, &D);
+  int rc = check_route_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
   if (D.L == 0) return OMNI_OK;
   const void* t16[] = {x, Wr, Wc};
@@ -227,7 +241,7 @@ int omni_route_select(const omni_dims* dims, const float* logits, const float* b
   (void)ws;
   (void)ws_bytes;
   Dims D;
-  int rc = check_dims(dims, &D);
+  int rc = check_route_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
   if (D.L == 0) return OMNI_OK;
   if (logits == nullptr || !al(logits, 16) || idx == nullptr || gate == nullptr)
@@ -279,7 +293,7 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
                      size_t ws_bytes, void* stream) {
   omni::CallRange range("omni_moe_forward");
   Dims D;
-  int rc = check_dims(dims, &D);
+  int rc = check_route_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
   if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
   if (D.L == 0) return OMNI_OK;

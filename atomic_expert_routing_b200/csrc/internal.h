@@ -21,6 +21,10 @@ struct CallRange {
   CallRange& operator=(const CallRange&) = delete;
 };
 
+// OMNI_OK for cudaSuccess; otherwise records e as this host thread's last
+// CUDA error (omni_last_cuda_error_name) and returns OMNI_ERR_CUDA.
+int cuda_status(cudaError_t e);
+
 struct Dims {
   int64_t L, d, Nr, Nc, k, K, B;
   int dtype;

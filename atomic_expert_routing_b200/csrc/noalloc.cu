@@ -25,7 +25,8 @@ std::mutex g_mu;
 float* g_acc_addr[kMaxDevices] = {};  // device address of g_noalloc_acc, per device
 
 // Device address of the accumulator on the current device, looked up once per
-// device (the host-side name of the array is not a device address).
+// device (the host-side name of the array is not a device address).  The
+// cached address is not refreshed after a cudaDeviceReset of that device.
 cudaError_t acc_address(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -67,11 +68,14 @@ extern "C" int omni_expert_forward_noalloc(const omni_dims* dims, const void* x,
   D.L = dims->L; D.d = dims->d; D.Nr = dims->Nr; D.Nc = dims->Nc;
   D.k = dims->k; D.K = dims->K; D.B = dims->B; D.dtype = dims->dtype; D.flags = dims->flags;
   float* acc = nullptr;
-  if (need > 0 && acc_address(&acc) != cudaSuccess) return OMNI_ERR_CUDA;
+  if (need > 0) {
+    const cudaError_t e = acc_address(&acc);
+    if (e != cudaSuccess) return omni::cuda_status(e);
+  }
   // launch_expert zeroes the accumulator before use (it keeps the previous
   // call's contents otherwise)
   const cudaError_t e = omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate,
                                             group_off, counts, y, acc,
                                             static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? OMNI_OK : OMNI_ERR_CUDA;
+  return omni::cuda_status(e);
 }

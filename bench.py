@@ -89,8 +89,8 @@ def expert_stage_bytes(cfg, n_active):
 
 # DRAM bytes (read + write) of one expert-stage call, summed over its kernels,
 # from ncu. The full-size stage is too large for a full capture; these values
-# come from the proxy workload (profiles/expert_stage_bf16-prefill-proxy-N256K.md,
-# 1730.0 MB) scaled by the stage's algorithmic bytes (x3.90). Update them
+# come from a capture of the bf16-prefill-proxy-N256K workload (1716.4 MB per
+# stage call) scaled by the stage's algorithmic bytes (x3.90). Update them
 # whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
     # re-captured after every change to the stage's kernels; until then none

@@ -85,7 +85,13 @@ extern "C" {
  * A valid field beyond this build's limits returns OMNI_ERR_UNSUPPORTED:
  *   Nr or Nc > OMNI_MAX_AXIS; k or K > OMNI_MAX_TOPK; N >= 2^31;
  *   L*K >= 2^30; d not a multiple of 8, or d > 65536.
- * When both apply, OMNI_ERR_INVALID_ARG is returned. */
+ * When both apply, OMNI_ERR_INVALID_ARG is returned.
+ * The calls that select experts (omni_route, omni_route_select and
+ * omni_moe_forward) also return OMNI_ERR_UNSUPPORTED for K > k: the top-K of the k x k
+ * candidate pairs is the top-K over all N joint scores only when k >= K
+ * (a grid row outside the per-axis top-k is beaten by at least k others, so
+ * none of its pairs can reach the top K).  The other calls, and
+ * omni_workspace_size, do not use k and take any K <= k*k. */
 
 typedef struct omni_dims {
   int64_t L;     /* tokens in the batch (>= 0; L*K < 2^30 tasks) */
@@ -93,7 +99,7 @@ typedef struct omni_dims {
   int64_t Nr;    /* grid rows */
   int64_t Nc;    /* grid columns; N = Nr*Nc atomic experts (< 2^31) */
   int64_t k;     /* per-axis top-k, 1 <= k <= min(Nr, Nc) */
-  int64_t K;     /* experts per token, 1 <= K <= k*k */
+  int64_t K;     /* experts per token, 1 <= K <= k*k; K <= k where experts are selected */
   int64_t B;     /* active experts per scheduling group, >= 1 */
   int32_t dtype; /* OMNI_F32 or OMNI_BF16 */
   int32_t flags; /* OMNI_FLAG_* */
@@ -187,8 +193,11 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
  * so L*d must not exceed 4194304 (OMNI_ERR_UNSUPPORTED otherwise).  The array
  * is shared by every call and zeroed by each call before use: calls that can
  * overlap on the GPU (different streams, or several host threads) race on it
- * and must be serialised by the caller.  The first call on a device looks up
- * the array's device address; make that first call before any stream capture.
+ * and must be serialised by the caller.  The array used is the one on the
+ * current device, which must be the device of `stream` and of every pointer.
+ * The first call on a device looks up the array's device address and keeps
+ * it for the life of the process (it is not looked up again after a
+ * cudaDeviceReset); make that first call before any stream capture.
  * Allocates nothing.
  */
 int omni_expert_forward_noalloc(const omni_dims* dims, const void* x, const void* W,

@@ -42,7 +42,14 @@ def check_selection(cfg, gpu_idx, gpu_gate, gpu_score, ora_idx, ora_gate, ora_sc
     (score desc, id asc) in each side's own arithmetic, so it is unique only where
     the scores are separated: the GPU order must agree with the oracle's wherever
     the oracle's scores differ by more than order_tol.  Near-tie tokens must hold a
-    valid top-K within the tie band.  Returns (exact tokens, near-tie tokens)."""
+    valid top-K within the tie band.  Returns (exact tokens, near-tie tokens).
+
+    The band compares the oracle's K-th score with the (K+1)-th over all N
+    joint scores (nxt).  That is the right pair only when k >= K: then the
+    k x k candidates hold the true top-K, and a near-tie at the per-axis k-th
+    place shows up as one at the K-th joint place.  The library refuses K > k
+    where it selects, so a K > k configuration is a mistake in the test."""
+    assert cfg.K <= cfg.k, "selection parity is defined for K <= k only"
     near = np.abs(ora_score[:, -1] - nxt) < rel * np.abs(ora_score[:, -1])
     exact = ~near
     gs = np.sort(gpu_idx, axis=1)

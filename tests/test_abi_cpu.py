@@ -159,3 +159,50 @@ def test_dims_checks_follow_the_header(lib):
                 assert n > 0
 
     check()
+
+
+def test_selecting_calls_refuse_K_above_k(lib):
+    """The top-K of the k x k candidate pairs is the top-K of all N joint
+    scores only when k >= K.  The calls that select experts refuse K > k
+    before any other check; scheduling and execution do not use k and pass
+    the dims check (they then stop at a null pointer, not at the dims)."""
+    D = _dims(k=4, K=6)
+    fake = C.c_void_p(4096)
+    U = _lib.OMNI_ERR_UNSUPPORTED
+    assert lib.omni_route(C.byref(D), fake, fake, fake, None, None, fake, fake, None, fake,
+                          fake, 1 << 30, None) == U
+    assert lib.omni_route_select(C.byref(D), fake, None, None, fake, fake, None, fake, None, 0,
+                                 None) == U
+    assert lib.omni_moe_forward(C.byref(D), *([fake] * 11), fake, 1 << 30, None) == U
+    assert lib.omni_schedule(C.byref(D), fake, fake, fake, fake, fake, fake, fake, None, fake,
+                             1 << 30, None) == _lib.OMNI_ERR_INVALID_ARG
+    assert lib.omni_expert_forward(C.byref(D), *([fake] * 8), None, fake, fake, 1 << 30,
+                                   None) == _lib.OMNI_ERR_INVALID_ARG
+    for which in range(6):
+        assert _wsz(lib, D, which)[0] == _lib.OMNI_OK
+    # K == k is accepted (the same null-pointer stop as above)
+    D = _dims(k=6, K=6)
+    assert lib.omni_moe_forward(C.byref(D), *([fake] * 10), None, fake, 1 << 30,
+                                None) == _lib.OMNI_ERR_INVALID_ARG
+
+
+NOALLOC_MAX = 1 << 22  # floats in the library's fixed accumulator
+
+
+@pytest.mark.parametrize("L,d,code", [
+    # exactly at the limit: past the size check, stopped by the null y
+    (NOALLOC_MAX // 2048, 2048, _lib.OMNI_ERR_INVALID_ARG),
+    (NOALLOC_MAX // 8, 8, _lib.OMNI_ERR_INVALID_ARG),
+    # one row past it, and far past it
+    (NOALLOC_MAX // 8 + 1, 8, _lib.OMNI_ERR_UNSUPPORTED),
+    (NOALLOC_MAX // 2048 + 1, 2048, _lib.OMNI_ERR_UNSUPPORTED),
+    (4096, 2048, _lib.OMNI_ERR_UNSUPPORTED),
+])
+def test_noalloc_size_limit(lib, L, d, code):
+    """omni_expert_forward_noalloc takes batches up to L*d = 4194304 (its
+    fixed accumulator) and refuses larger ones before touching the GPU."""
+    D = _dims(L=L, d=d, Nr=32, Nc=32, k=4, K=4, B=16, dtype=_lib.OMNI_BF16)
+    fake = C.c_void_p(4096)
+    args = [fake] * 10
+    args[9] = None  # y
+    assert lib.omni_expert_forward_noalloc(C.byref(D), *args, None) == code

@@ -342,11 +342,11 @@ def test_full_size_fused_and_staged(cfg):
 # --------------------------------------------------------------------------- edge cases
 
 EDGE = [
-    WL.Config("ragged-bf16", L=130, d=72, Nr=48, Nc=80, k=5, K=7, B=4, dtype=WL.BF16, seed=11),
-    WL.Config("ragged-f32", L=37, d=40, Nr=12, Nc=20, k=3, K=9, B=2, dtype=WL.F32, seed=12),
+    WL.Config("ragged-bf16", L=130, d=72, Nr=48, Nc=80, k=7, K=5, B=4, dtype=WL.BF16, seed=11),
+    WL.Config("ragged-f32", L=37, d=40, Nr=12, Nc=20, k=9, K=9, B=2, dtype=WL.F32, seed=12),
     WL.Config("single-token", L=1, d=64, Nr=16, Nc=16, k=4, K=4, B=3, dtype=WL.BF16, seed=13),
     WL.Config("k1", L=200, d=128, Nr=32, Nc=64, k=1, K=1, B=5, dtype=WL.BF16, seed=14),
-    WL.Config("max-topk", L=64, d=64, Nr=4096, Nc=16, k=16, K=256, B=64, dtype=WL.BF16, seed=15),
+    WL.Config("max-topk", L=64, d=64, Nr=4096, Nc=256, k=256, K=256, B=64, dtype=WL.BF16, seed=15),
     WL.Config("wide-k", L=96, d=256, Nr=256, Nc=256, k=128, K=100, B=128, dtype=WL.BF16, seed=16),
 ]
 
@@ -377,7 +377,7 @@ def test_edge_shapes(cfg):
 def test_equal_logits_pick_smallest_ids(L):
     """x = 0: every joint score ties; the K smallest ids of the k x k grid win
     (small batches take the 8-warp selection, larger ones the 2-warp one)."""
-    cfg = WL.Config("ties", L=L, d=64, Nr=16, Nc=24, k=4, K=6, B=4, dtype=WL.BF16, seed=3)
+    cfg = WL.Config("ties", L=L, d=64, Nr=16, Nc=24, k=6, K=6, B=4, dtype=WL.BF16, seed=3)
     h = WL.make_inputs(cfg)
     h["x"] = np.zeros_like(h["x"])
     d = {k: dev(v) for k, v in h.items()}

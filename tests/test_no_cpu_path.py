@@ -74,3 +74,54 @@ def test_the_product_never_imports_the_oracle():
             elif isinstance(node, ast.ImportFrom):
                 names = [node.module or ""]
             assert not any(n == "oracle" or n.startswith("oracle.") for n in names), path
+
+
+def _shrunk_calls():
+    """Each compute entry with one argument a row too short or of the wrong
+    dtype: (call name, argument name, call)."""
+    c = CFG
+    D = omni.LayerDims.of(c)
+    M = c.L * c.K
+    x, Wr, Wc = _t(c.L, c.d), _t(c.Nr, c.d), _t(c.Nc, c.d)
+    W, V = _t(c.N, c.d), _t(c.N, c.d)
+    idx = torch.zeros((c.L, c.K), dtype=torch.int32)
+    gate = _t(c.L, c.K)
+    sched = {"task_token": torch.zeros(M, dtype=torch.int32),
+             "task_expert": torch.zeros(M, dtype=torch.int32), "task_gate": _t(M),
+             "uniq": torch.zeros(M, dtype=torch.int32),
+             "group_off": torch.zeros(M + 1, dtype=torch.int32),
+             "counts": torch.zeros(4, dtype=torch.int32)}
+    short = dict(sched, task_expert=torch.zeros(M - 1, dtype=torch.int32))
+    return [
+        ("route", "x", lambda: omni.route(D, x[:-1], Wr, Wc)),
+        ("route", "Wc", lambda: omni.route(D, x, Wr, Wc.to(torch.float64))),
+        ("route", "bias_r", lambda: omni.route(D, x, Wr, Wc, bias_r=_t(c.Nr - 1))),
+        ("router_logits", "Wr", lambda: omni.router_logits(D, x, Wr[:-1], Wc)),
+        ("route_select", "logits", lambda: omni.route_select(D, _t(c.L - 1, c.Nr + c.Nc))),
+        ("schedule", "idx", lambda: omni.schedule(D, idx.long(), gate)),
+        ("schedule", "gate", lambda: omni.schedule(D, idx, gate[:-1])),
+        ("expert_forward", "W", lambda: omni.expert_forward(D, x, W[:-1], V, sched)),
+        ("expert_forward", "task_expert", lambda: omni.expert_forward(D, x, W, V, short)),
+        ("expert_forward", "y", lambda: omni.expert_forward(D, x, W, V, sched, y=_t(1))),
+        ("expert_forward_noalloc", "V",
+         lambda: omni.expert_forward_noalloc(D, x, W, V.half(), sched)),
+        ("moe_forward", "V", lambda: omni.moe_forward(D, x, Wr, Wc, W, V[:-1])),
+        ("moe_forward", "counts",
+         lambda: omni.moe_forward(D, x, Wr, Wc, W, V, counts=torch.zeros(3, dtype=torch.int32))),
+        ("token_centric_forward", "gate",
+         lambda: omni.token_centric_forward(D, x, W, V, idx, gate.double())),
+        ("wait_selftest", "counts", lambda: omni.wait_selftest(torch.zeros(4))),
+    ]
+
+
+@pytest.mark.parametrize("case", _shrunk_calls(), ids=lambda c: f"{c[0]}-{c[1]}")
+def test_sizes_and_dtypes_are_checked_before_the_library(case, monkeypatch):
+    """A tensor too small for the dims, or of another dtype, raises in the
+    binding; the library is never loaded or called."""
+    def no_library(*a, **k):
+        raise AssertionError("the library was reached")
+
+    monkeypatch.setattr(_lib, "load", no_library)
+    _, arg, call = case
+    with pytest.raises(ValueError, match=rf"^{arg}\b"):
+        call()

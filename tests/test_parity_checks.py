@@ -138,3 +138,13 @@ def test_bf16_round_trip_of_the_data_movers():
     assert t.dtype == torch.bfloat16
     np.testing.assert_array_equal(host_f64(t), WL.bf16_bits_to_f32(bits).astype(np.float64))
     assert dev(None) is None
+
+
+def test_selection_check_refuses_K_above_k(routed):
+    """The near-tie band compares the K-th and (K+1)-th joint scores over all
+    N, which is only the selection's own margin when k >= K."""
+    idx, gate, score, nxt, lr, lc = routed
+    bad = CFG.with_(K=CFG.k + 1)
+    with pytest.raises(AssertionError, match="K <= k"):
+        check_selection(bad, idx, gate.astype(np.float32), score.astype(np.float32), idx, gate,
+                        score, nxt, lr, lc)
