@@ -117,12 +117,14 @@ def _expect_io(D, **ts):
 
 
 def _expect_sched(D, sched):
-    ucap = max(1, min(D.N, D.M))
-    gmax = (ucap + D.B - 1) // D.B
+    """A schedule passed to the grouped execution.  The execution does not
+    read uniq, and reads group_off only up to the group count held on the
+    device (counts[1] + 1 entries), so an exactly sized schedule is valid and
+    only the task arrays' lengths are known on the host."""
     i32 = torch.int32
     for name, n, dt in (("task_token", D.M, i32), ("task_expert", D.M, i32),
-                        ("task_gate", D.M, torch.float32), ("uniq", ucap, i32),
-                        ("group_off", gmax + 1, i32), ("counts", 4, i32)):
+                        ("task_gate", D.M, torch.float32), ("uniq", 0, i32),
+                        ("group_off", 1, i32), ("counts", 4, i32)):
         if name not in sched:
             raise ValueError(f"schedule entry {name} is missing")
         _expect(name, sched[name], n, dt)
