@@ -19,7 +19,8 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_WS_EXPERT, OMNI_WS_FUSED,
+from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_FLAG_STAGED_SMALL,
+                   OMNI_WS_EXPERT, OMNI_WS_FUSED,
                    OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
 
 __all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",

@@ -33,7 +33,8 @@ int check_dims(const omni_dims* in, Dims* D) {
   if (D->L < 0 || D->d < 1 || D->Nr < 1 || D->Nc < 1 || D->k < 1 || D->K < 1 || D->B < 1)
     return OMNI_ERR_INVALID_ARG;
   if (D->dtype != OMNI_F32 && D->dtype != OMNI_BF16) return OMNI_ERR_INVALID_ARG;
-  if ((D->flags & ~OMNI_FLAG_ROUTER_SIMT) != 0) return OMNI_ERR_INVALID_ARG;
+  if ((D->flags & ~(OMNI_FLAG_ROUTER_SIMT | OMNI_FLAG_STAGED_SMALL)) != 0)
+    return OMNI_ERR_INVALID_ARG;
   // k*k in 128 bits: k is only bounded by the axes here
   if (D->k > D->Nr || D->k > D->Nc ||
       static_cast<__int128>(D->K) > static_cast<__int128>(D->k) * D->k)
@@ -95,7 +96,11 @@ FusedWs carve_fused(const Dims& D, Carver& c) {
   w.group_off = c.take<int32_t>(static_cast<size_t>(D.gmax()) + 1);
   w.sched = c.take<char>(fused_windows(D) ? omni::windows_ws_bytes(D)
                                            : omni::schedule_ws_bytes(D));
-  w.expert = c.take<char>(omni::expert_ws_bytes(D));
+  // the small-batch tail (activations by expert tile, value gather) uses the
+  // expert workspace for its counters and activations
+  const size_t tail = omni::sched_exec_supported(D) ? omni::sched_exec_ws_words(D) * 4 : 0;
+  const size_t ex = omni::expert_ws_bytes(D);
+  w.expert = c.take<char>(ex > tail ? ex : tail);
   return w;
 }
 
@@ -310,13 +315,26 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   const int64_t acc_words = omni::expert_acc_words(D);
   float* acc = acc_words == 0 ? nullptr
                : static_cast<float*>(D.dtype == OMNI_F32 ? y : w.expert);
+  // a small batch runs the two-kernel tail; its two counters are cleared
+  // by the selection kernel in place of the accumulator
+  const bool tail = omni::sched_exec_supported(D);
+  float* zero = tail ? static_cast<float*>(w.expert) : acc;
+  const int64_t zero_words = tail ? 2 : acc_words;
   bool acc_zeroed = false;
   {
     omni::CallRange stage("route");
     rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s,
-                    acc, acc_words, &acc_zeroed);
+                    zero, zero_words, &acc_zeroed);
   }
   if (rc != OMNI_OK) return rc;
+  if (tail) {
+    omni::CallRange stage("schedule+expert");
+    if (!acc_zeroed &&
+        (rc = cuda_status(omni::launch_zero(zero, static_cast<size_t>(zero_words), s))) != OMNI_OK)
+      return rc;
+    return cuda_status(omni::launch_sched_exec(D, x, W, V, idx, gate, y,
+                                               static_cast<uint32_t*>(w.expert), counts, s));
+  }
   if (fused_windows(D)) {
     {
       omni::CallRange stage("schedule");

@@ -73,6 +73,10 @@ extern "C" {
 
 /* dims.flags bits */
 #define OMNI_FLAG_ROUTER_SIMT 1 /* diagnostic: router logits on CUDA cores for bf16 too */
+#define OMNI_FLAG_STAGED_SMALL 2 /* diagnostic: omni_moe_forward of a small batch runs the
+                                    scheduling and grouped-execution kernels of
+                                    omni_schedule and omni_expert_forward instead of its
+                                    two-kernel small-batch tail */
 
 /* Limits of this build (host checks return OMNI_ERR_UNSUPPORTED beyond them). */
 #define OMNI_MAX_AXIS 4096      /* Nr, Nc */
@@ -211,7 +215,15 @@ int omni_expert_forward_noalloc(const omni_dims* dims, const void* x, const void
  * then scheduling, then grouped execution.  idx_out / gate_out (nullable,
  * [L x K]) receive the routing decisions; counts[0], counts[1] are written as
  * by omni_schedule; y as in omni_expert_forward.
- * Small batches run omni_schedule's order.  Batches whose fp32 accumulator is
+ * Small batches run omni_schedule's order.  A batch of at most 8192 tasks with
+ * N <= 2^20 (and a row width of 256, 512, 1024 or 2048 bf16 / 128 .. 1024
+ * fp32 elements) runs scheduling and execution as two kernels: the first
+ * splits the ids into tiles of consecutive ids, sorts each tile's tasks by
+ * expert and computes their activations gate * SiLU(x[t] . W[e]) (an
+ * expert's W row read once for all its tokens), and counts |U| and the
+ * groups; the second forms y[t] = sum of activation * V[e] over the token's
+ * tasks and writes it once.  No schedule arrays are written (counts[0],
+ * counts[1] are).  Batches whose fp32 accumulator is
  * executed in column-slice sweeps (L*d*4 above about 40 MiB) go from the
  * routing straight to the executor's order.  That order is the same groups,
  * in windows of consecutive groups, with each window's tasks ordered by

@@ -519,3 +519,48 @@ def test_expert_sweeps_back_to_back():
     torch.cuda.synchronize()
     for y, y_ref in zip(ys, refs):
         assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
+
+
+# ------------------------------- small batches: the two-kernel tail of the fused forward
+
+SMALL_TAIL = [
+    WL.Config("one-bf16-d256-L1", L=1, d=256, Nr=16, Nc=16, k=4, K=4, B=200, dtype=WL.BF16,
+              seed=51),
+    WL.Config("one-bf16-d512", L=37, d=512, Nr=40, Nc=30, k=16, K=16, B=7, dtype=WL.BF16, seed=52),
+    WL.Config("one-bf16-d1024-skew", L=100, d=1024, Nr=64, Nc=64, k=8, K=8, B=64, dtype=WL.BF16,
+              seed=53, zipf_s=1.1),
+    WL.Config("one-f32-d128", L=50, d=128, Nr=32, Nc=32, k=6, K=6, B=16, dtype=WL.F32, seed=54),
+    WL.Config("one-f32-d512", L=20, d=512, Nr=16, Nc=16, k=4, K=4, B=5, dtype=WL.F32, seed=55),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_TAIL + [WL.DECODE], ids=lambda c: c.name)
+def test_small_batch_tail(cfg):
+    """The fused forward of a small batch ends in two kernels (activations of
+    expert-id tiles, then a per-token gather of the value rows): y against the
+    oracle's expert-centric y of the same routing, |U| and the group count
+    exactly, and y against the staged scheduling and execution kernels
+    (OMNI_FLAG_STAGED_SMALL) on the same routing."""
+    h = host_inputs(cfg) if cfg is WL.DECODE else WL.make_inputs(cfg)
+    d = dev_inputs(cfg) if cfg is WL.DECODE else {k: dev(v) for k, v in h.items()}
+    outs = {}
+    for flags in (0, omni.OMNI_FLAG_STAGED_SMALL):
+        D = omni.LayerDims.of(cfg, flags=flags)
+        idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
+        gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
+        counts = omni.new_counts("cuda")
+        y = omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"],
+                             d["bias_c"], counts=counts, idx=idx, gate=gate)
+        torch.cuda.synchronize()
+        outs[flags] = (y.clone(), idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy())
+    y1, i1, g1, c1 = outs[0]
+    y2, i2, g2, c2 = outs[omni.OMNI_FLAG_STAGED_SMALL]
+    assert np.array_equal(i1, i2) and np.array_equal(g1, g2)
+    assert c1[2] == 0 and c2[2] == 0
+    assert c1[0] == c2[0] and c1[1] == c2[1]
+    assert rel_err(host_f64(y1), host_f64(y2)) <= tol_y(cfg)
+    # against the oracle: its schedule of the GPU's routing, and y of that routing
+    ref_s = O.schedule(cfg, i1, g1.astype(np.float64))
+    assert c1[0] == ref_s["n_active"] and c1[1] == ref_s["n_groups"]
+    y_ref, _ = O.forward_expert(cfg, h, ref_s)
+    assert rel_err(host_f64(y1), y_ref) <= tol_y(cfg)
