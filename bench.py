@@ -80,6 +80,34 @@ def group_stats(group_off, B, n_active):
             "tasks_max": int(per.max()), "experts_in_last_group": int(n_active - B * (per.size - 1))}
 
 
+def group_density(task_token, group_off, B, n_active, block=128):
+    """How dense each group's token x expert tile is: tasks_g / (T_g * B_g)
+    with T_g the group's distinct tokens and B_g its experts (B, fewer in the
+    last group), and the tasks per touched tile of `block` consecutive
+    tokens by the group's B experts -- the fill of the tiles a dense
+    (tensor-core) formulation of the grouped contraction would compute.
+    task_token: the schedule's task tokens (sorted by token inside a group)."""
+    tt = np.asarray(task_token, dtype=np.int64)
+    go = np.asarray(group_off, dtype=np.int64)
+    G = go.size - 1
+    if G < 1:
+        return {}
+    dens, per_tile = [], []
+    for g in range(G):
+        t = tt[go[g]:go[g + 1]]
+        if t.size == 0:
+            continue
+        bg = B if g < G - 1 else int(n_active - B * (G - 1))
+        tokens = 1 + int(np.count_nonzero(np.diff(t)))
+        tiles = 1 + int(np.count_nonzero(np.diff(t // block)))
+        dens.append(t.size / (tokens * bg))
+        per_tile.append(t.size / tiles)
+    dens, per_tile = np.array(dens), np.array(per_tile)
+    return {"density_median": float(np.median(dens)), "density_max": float(dens.max()),
+            "tasks_per_tile_median": float(np.median(per_tile)),
+            "tasks_per_tile_max": float(per_tile.max()), "tile_tokens": block}
+
+
 def expert_stage_bytes(cfg, n_active):
     """Algorithmic bytes of the grouped execution: active rows of W and V once,
     x read, y written."""
@@ -414,7 +442,9 @@ def run_ours(args):
         out = {"route": tot[0] / steps, "schedule": tot[1] / steps, "expert": tot[2] / steps}
         try:  # a diagnostic: it may not cost the line
             na, ng = (int(v) for v in counts[:2].cpu().tolist())
-            out["groups"] = group_stats(s["group_off"][: ng + 1].cpu().numpy(), c.B, na)
+            go = s["group_off"][: ng + 1].cpu().numpy()
+            out["groups"] = group_stats(go, c.B, na)
+            out["groups"].update(group_density(s["task_token"].cpu().numpy(), go, c.B, na))
         except Exception as exc:  # noqa: BLE001
             out["groups"] = {"error": repr(exc)[:200]}
         return out
@@ -580,7 +610,7 @@ def run_ours(args):
             hs = rank_inputs(sc, rank)
             hs.update(WL.make_experts(sc))
             ds = {k: to_dev(v) for k, v in hs.items()}
-            extra[sc.name] = summary(sc, ds, max(args.steps, 10), max(args.warmup, 3), False)
+            extra[sc.name] = summary(sc, ds, max(args.steps, 10), max(args.warmup, 3), True)
             del ds, hs
             torch.cuda.empty_cache()
 

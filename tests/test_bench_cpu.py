@@ -105,3 +105,17 @@ def test_group_stats():
     assert g == {"groups": 4, "tasks_min": 2, "tasks_median": 3.5, "tasks_mean": 4.5,
                  "tasks_max": 9, "experts_in_last_group": 2}
     assert bench.group_stats([0], B=4, n_active=0) == {"groups": 0}
+
+
+def test_group_density_by_hand():
+    """Two groups of B = 4 experts (n_active = 6: the last group has 2).
+    Group 0: tokens 0, 0, 1, 200 (3 tokens; tiles of 128 tokens: 0 and 1) ->
+    density 4 / (3 * 4), 4 / 2 tasks per touched tile.  Group 1: tokens 5, 5
+    (1 token, 2 experts) -> density 2 / (1 * 2), 2 tasks in one tile."""
+    import bench
+
+    d = bench.group_density([0, 0, 1, 200, 5, 5], [0, 4, 6], B=4, n_active=6)
+    assert abs(d["density_median"] - (4 / 12 + 1.0) / 2) < 1e-12
+    assert d["density_max"] == 1.0
+    assert d["tasks_per_tile_median"] == 2.0 and d["tasks_per_tile_max"] == 2.0
+    assert bench.group_density([], [0], B=4, n_active=0) == {}
