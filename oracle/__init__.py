@@ -204,3 +204,18 @@ def moe_forward(cfg, inp, tokens=None):
     sched = schedule(cfg, idx, gate, tokens)
     y, rows = forward_expert(cfg, inp, sched, tokens)
     return {"idx": idx, "gate": gate, "score": score, "sched": sched, "y": y, "rows": rows}
+
+
+def shared_mlp(cfg, inp, W1, W2, tokens=None):
+    """The shared dense MLP branch: SiLU(x W1^T) W2^T, fp64 [nt, d].  W1 [F, d]
+    and W2 [d, F] in the storage layout of ``workloads`` (bf16 as uint16)."""
+    tok = _tokens(cfg, tokens)
+    W1 = np.ascontiguousarray(W1)
+    W2 = np.ascontiguousarray(W2)
+    F = W1.shape[0]
+    assert W1.shape == (F, cfg.d) and W2.shape == (cfg.d, F)
+    y = np.empty((len(tok), cfg.d), np.float64)
+    D = dims(cfg)
+    _check(lib().oracle_shared_mlp(C.byref(D), C.c_int64(F), _p(inp["x"]), _p(W1), _p(W2),
+                                   _p(tok), C.c_int64(len(tok)), _p(y)), "shared_mlp")
+    return y

@@ -491,6 +491,46 @@ int oracle_forward_token(const or_dims* D, const void* x, const void* W, const v
   return 0;
 }
 
+/*
+ * Shared dense MLP branch [NL 2.1]: an always-on dense MLP beside the routed
+ * experts, y = MLP(x) + routed(x) (the explainer's ablation table removes it
+ * as "w/o shared MLP").  The pages give neither its width nor its
+ * activation; the reading taken is one hidden layer of F units with the same
+ * scalar SiLU as the atomic experts:
+ *   h[f] = SiLU(x[t] . W1[f]),  f < F;   mlp[t, j] = h . W2[j],  j < d,
+ * with W1 [F x d] and W2 [d x F] in the storage type (row j of W2 holds the
+ * F weights of output j).  Row r of y (fp64, d values) is token tok[r].
+ */
+int oracle_shared_mlp(const or_dims* D, int64_t F, const void* x, const void* W1, const void* W2,
+                      const int64_t* tok, int64_t nt, double* y) {
+  const int64_t d = D->d;
+  if (F < 1) return 1;
+#pragma omp parallel
+  {
+    double* xt = (double*)malloc(sizeof(double) * d);
+    double* h = (double*)malloc(sizeof(double) * F);
+    double* w1 = (double*)malloc(sizeof(double) * d);
+    double* w2 = (double*)malloc(sizeof(double) * F);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nt; ++r) {
+      load_row(x, D->dtype, tok[r], d, xt);
+      for (int64_t f = 0; f < F; ++f) {
+        load_row(W1, D->dtype, f, d, w1);
+        h[f] = silu(dot(xt, w1, d));
+      }
+      for (int64_t j = 0; j < d; ++j) {
+        load_row(W2, D->dtype, j, F, w2);
+        y[r * d + j] = dot(h, w2, F);
+      }
+    }
+    free(xt);
+    free(h);
+    free(w1);
+    free(w2);
+  }
+  return 0;
+}
+
 /* Threads an OpenMP region of this library uses (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

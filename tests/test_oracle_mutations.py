@@ -25,6 +25,16 @@ PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 
 # (name, text of oracle.c, its replacement); each text occurs exactly once
 MUTANTS = [
+    # shared dense MLP branch
+    ("mlp-silu-on-the-output", "y[r * d + j] = dot(h, w2, F);",
+     "y[r * d + j] = silu(dot(h, w2, F));"),
+    ("mlp-w2-transposed", "load_row(W2, D->dtype, j, F, w2);",
+     "for (int64_t f = 0; f < F; ++f) w2[f] = elem(W2, D->dtype, f * d + j);"),
+    ("mlp-drops-last-hidden-unit", "h[f] = silu(dot(xt, w1, d));",
+     "h[f] = f + 1 < F ? silu(dot(xt, w1, d)) : 0.0;"),
+    ("mlp-linear-hidden", "h[f] = silu(dot(xt, w1, d));", "h[f] = dot(xt, w1, d);"),
+    ("mlp-x-of-row-not-token", "load_row(x, D->dtype, tok[r], d, xt);",
+     "load_row(x, D->dtype, r, d, xt);"),
     # atomic expert: sigma, dot product, operand rows
     ("silu-sign", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
     ("dot-drops-last-term", "for (int64_t m = 0; m < n; ++m) s += a[m] * b[m];",

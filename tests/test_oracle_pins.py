@@ -440,3 +440,65 @@ def test_thread_count_does_not_change_results():
         O.set_num_threads(n)
     for k in ("idx", "gate", "score", "y"):
         np.testing.assert_array_equal(np.asarray(a[k]), np.asarray(b[k]))
+
+
+# ------------------------------------------------------------ shared dense MLP branch
+
+def _mlp_cfg(L, d, dtype=WL.F32):
+    return WL.Config("mlp", L=L, d=d, Nr=2, Nc=2, k=1, K=1, B=1, dtype=dtype, seed=0)
+
+
+def test_shared_mlp_hand_worked():
+    """d = 2, F = 3, two tokens; the numbers are worked by hand.
+    Token 0, x = (1, -2): x W1^T = (1, -2, -1), SiLU of those
+    = (sigmoid(1), -2 sigmoid(-2), -sigmoid(-1)) = (0.7310585786, -0.2384058440,
+    -0.2689414214); with W2 rows (1, -1, 2) and (0, 3, 0.5) the outputs are
+    (0.4315815799, -0.8496882428).  Token 1, x = (0.5, 0): x W1^T = (0.5, 0,
+    0.5), SiLU = (0.3112296656, 0, 0.3112296656), outputs (0.9336889968,
+    0.1556148328)."""
+    cfg = _mlp_cfg(2, 2)
+    x = np.array([[1.0, -2.0], [0.5, 0.0]], np.float32)
+    W1 = np.array([[1, 0], [0, 1], [1, 1]], np.float32)
+    W2 = np.array([[1, -1, 2], [0, 3, 0.5]], np.float32)
+    y = O.shared_mlp(cfg, {"x": x}, W1, W2)
+    ref = np.array([[0.4315815799, -0.8496882428], [0.9336889968, 0.1556148328]])
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("dtype", [WL.F32, WL.BF16], ids=["f32", "bf16"])
+def test_shared_mlp_identity_output_is_silu_of_the_projection(dtype):
+    """With F = d and W2 = I the branch is SiLU(x W1^T), element by element:
+    numpy's matmul and scipy's expit in fp64 on the exact stored values."""
+    cfg = _mlp_cfg(7, 24, dtype)
+    rng = np.random.default_rng(5)
+    x32 = rng.standard_normal((7, 24)).astype(np.float32)
+    W132 = (rng.standard_normal((24, 24)) / 5).astype(np.float32)
+    if dtype == WL.BF16:
+        x, W1 = WL.f32_to_bf16_bits(x32), WL.f32_to_bf16_bits(W132)
+        W2 = WL.f32_to_bf16_bits(np.eye(24, dtype=np.float32))
+        xf, W1f = WL.bf16_bits_to_f32(x), WL.bf16_bits_to_f32(W1)
+    else:
+        x, W1, W2, xf, W1f = x32, W132, np.eye(24, dtype=np.float32), x32, W132
+    y = O.shared_mlp(cfg, {"x": x}, W1, W2)
+    z = xf.astype(np.float64) @ W1f.astype(np.float64).T
+    np.testing.assert_allclose(y, z * expit(z), rtol=1e-12, atol=1e-14)
+
+
+def test_shared_mlp_linearity_rows_and_zero():
+    """Linear in W2; every token depends on its own row of x only (a token
+    subset gives those rows); x = 0 gives 0 (SiLU(0) = 0)."""
+    cfg = _mlp_cfg(9, 16)
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((9, 16)).astype(np.float32)
+    x[4] = 0.0
+    W1 = (rng.standard_normal((40, 16)) / 4).astype(np.float32)
+    # dyadic weights: 2 W2a - 3 W2b is exact in fp32
+    W2a = (rng.integers(-8, 9, (16, 40)) / 64).astype(np.float32)
+    W2b = (rng.integers(-8, 9, (16, 40)) / 64).astype(np.float32)
+    ya = O.shared_mlp(cfg, {"x": x}, W1, W2a)
+    yb = O.shared_mlp(cfg, {"x": x}, W1, W2b)
+    yab = O.shared_mlp(cfg, {"x": x}, W1, (2 * W2a - 3 * W2b).astype(np.float32))
+    np.testing.assert_allclose(yab, 2 * ya - 3 * yb, rtol=1e-12, atol=1e-12)
+    assert np.all(ya[4] == 0.0)
+    tok = np.array([1, 4, 8], np.int64)
+    np.testing.assert_array_equal(O.shared_mlp(cfg, {"x": x}, W1, W2a, tokens=tok), ya[tok])
