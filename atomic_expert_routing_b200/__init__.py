@@ -24,7 +24,8 @@ from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_FLAG_STAGED_
                    OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
 
 __all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",
-           "token_centric_forward", "new_counts", "OmniError", "workspace_size", "wait_selftest"]
+           "token_centric_forward", "new_counts", "OmniError", "workspace_size", "wait_selftest",
+           "shared_mlp", "moe_mlp_forward", "mlp_workspace_size"]
 
 
 @dataclass(frozen=True)
@@ -287,6 +288,61 @@ def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=No
     _lib.check("omni_moe_forward", _lib.load().omni_moe_forward(
         C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c), _ptr(W), _ptr(V),
         _ptr(y), _ptr(idx), _ptr(gate), _ptr(counts), wsp, n, _stream(stream)))
+    return y
+
+
+def mlp_workspace_size(D: LayerDims, F: int, with_routed: bool) -> int:
+    n = C.c_size_t(0)
+    dd = D.c()
+    _lib.check("omni_mlp_workspace_size", _lib.load().omni_mlp_workspace_size(
+        C.byref(dd), C.c_int64(F), 1 if with_routed else 0, C.byref(n)))
+    return int(n.value)
+
+
+def _expect_mlp(D, F, W1, W2):
+    _expect("W1", W1, F * D.d, D.torch_dtype)
+    _expect("W2", W2, D.d * F, D.torch_dtype)
+
+
+def shared_mlp(D: LayerDims, x, W1, W2, *, y=None, accumulate=False, counts=None, ws=None,
+               stream=None):
+    """Shared dense MLP branch: y (+)= SiLU(x W1^T) W2^T (W1 [F, d], W2 [d, F], bf16)."""
+    F = int(W1.shape[0])
+    _expect_io(D, x=x, y=y, counts=counts)
+    _expect_mlp(D, F, W1, W2)
+    if accumulate and y is None:
+        raise ValueError("y is required to accumulate into")
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    n = mlp_workspace_size(D, F, False)
+    buf = (Workspace() if ws is None else ws).get(n, dev)
+    dd = D.c()
+    _lib.check("omni_shared_mlp", _lib.load().omni_shared_mlp(
+        C.byref(dd), C.c_int64(F), _ptr(x), _ptr(W1), _ptr(W2), _ptr(y), 1 if accumulate else 0,
+        _ptr(counts), _ptr(buf) if buf is not None else None, n, _stream(stream)))
+    return y
+
+
+def moe_mlp_forward(D: LayerDims, x, Wr, Wc, W, V, W1, W2, bias_r=None, bias_c=None, *, y=None,
+                    counts=None, idx=None, gate=None, ws=None, stream=None):
+    """The layer output routed(x) + MLP(x) in one call; returns y [L, d]."""
+    F = int(W1.shape[0])
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, V=V, bias_r=bias_r, bias_c=bias_c, y=y,
+               counts=counts, idx=idx, gate=gate)
+    _expect_mlp(D, F, W1, W2)
+    dev = _device(x)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
+    if counts is None:
+        counts = new_counts(dev)
+    n = mlp_workspace_size(D, F, True)
+    buf = (Workspace() if ws is None else ws).get(n, dev)
+    dd = D.c()
+    _lib.check("omni_moe_mlp_forward", _lib.load().omni_moe_mlp_forward(
+        C.byref(dd), C.c_int64(F), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c),
+        _ptr(W), _ptr(V), _ptr(W1), _ptr(W2), _ptr(y), _ptr(idx), _ptr(gate), _ptr(counts),
+        _ptr(buf) if buf is not None else None, n, _stream(stream)))
     return y
 
 

@@ -45,6 +45,9 @@ SIGNATURES = {
     "omni_moe_forward": ([_P] * 13 + [C.c_size_t, _P], C.c_int),
     "omni_token_centric_forward": ([_P] * 9 + [C.c_size_t, _P], C.c_int),
     "omni_wait_selftest": ([_P, _P], C.c_int),
+    "omni_shared_mlp": ([_P, _I64, _P, _P, _P, _P, C.c_int, _P, _P, C.c_size_t, _P], C.c_int),
+    "omni_moe_mlp_forward": ([_P, _I64] + [_P] * 14 + [C.c_size_t, _P], C.c_int),
+    "omni_mlp_workspace_size": ([_P, _I64, C.c_int, C.POINTER(C.c_size_t)], C.c_int),
 }
 
 

@@ -292,20 +292,16 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
                                          static_cast<cudaStream_t>(stream)));
 }
 
-int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+}  // extern "C"
+
+namespace {
+
+// The fused routed branch; dims, pointers and workspace already checked.
+int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* Wc,
                      const float* bias_r, const float* bias_c, const void* W, const void* V,
                      void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
-                     size_t ws_bytes, void* stream) {
-  omni::CallRange range("omni_moe_forward");
-  Dims D;
-  int rc = check_route_dims(dims, &D);
-  if (rc != OMNI_OK) return rc;
-  if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
-  if (D.L == 0) return OMNI_OK;
-  const void* t16[] = {x, Wr, Wc, W, V, y};
-  if (!tensors_ok(t16, 6)) return OMNI_ERR_INVALID_ARG;
-  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+                     cudaStream_t s) {
+  int rc = OMNI_OK;
   Carver c(ws);
   FusedWs w = carve_fused(D, c);
   int32_t* idx = idx_out ? idx_out : w.idx;
@@ -355,6 +351,94 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
   omni::CallRange stage("expert");
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
                                          w.group_off, counts, y, w.expert, s, acc_zeroed));
+}
+
+// The checks of the shared MLP's width: F >= 1; a multiple of 8 (16-byte
+// rows of H and W2) and at most 65536, else unsupported; bf16 storage only.
+int check_mlp(const Dims& D, int64_t F) {
+  if (F < 1) return OMNI_ERR_INVALID_ARG;
+  if (F % 8 != 0 || F > 65536 || D.dtype != OMNI_BF16) return OMNI_ERR_UNSUPPORTED;
+  return OMNI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                     const float* bias_r, const float* bias_c, const void* W, const void* V,
+                     void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
+                     size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_forward");
+  Dims D;
+  int rc = check_route_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, W, V, y};
+  if (!tensors_ok(t16, 6)) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
+  return moe_forward_impl(D, x, Wr, Wc, bias_r, bias_c, W, V, y, idx_out, gate_out, counts, ws,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int omni_mlp_workspace_size(const omni_dims* dims, int64_t F, int with_routed, size_t* bytes) {
+  Dims D;
+  int rc = with_routed ? check_route_dims(dims, &D) : check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if ((rc = check_mlp(D, F)) != OMNI_OK) return rc;
+  if (bytes == nullptr) return OMNI_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  if (with_routed) c.take<char>(ws_size(D, OMNI_WS_FUSED));
+  c.take<char>(omni::mlp_ws_bytes(D, F));
+  *bytes = c.off;
+  return OMNI_OK;
+}
+
+int omni_shared_mlp(const omni_dims* dims, int64_t F, const void* x, const void* W1,
+                    const void* W2, void* y, int accumulate, int32_t* counts, void* ws,
+                    size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_shared_mlp");
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if ((rc = check_mlp(D, F)) != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W1, W2, y};
+  if (!tensors_ok(t16, 4)) return OMNI_ERR_INVALID_ARG;
+  if (ws == nullptr || !al(ws, 256) || ws_bytes < omni::mlp_ws_bytes(D, F))
+    return OMNI_ERR_WORKSPACE;
+  return cuda_status(omni::launch_shared_mlp(D, F, x, W1, W2, y, accumulate != 0, ws,
+                                             counts ? counts + 2 : nullptr,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int omni_moe_mlp_forward(const omni_dims* dims, int64_t F, const void* x, const void* Wr,
+                         const void* Wc, const float* bias_r, const float* bias_c, const void* W,
+                         const void* V, const void* W1, const void* W2, void* y,
+                         int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
+                         size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_mlp_forward");
+  Dims D;
+  int rc = check_route_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if ((rc = check_mlp(D, F)) != OMNI_OK) return rc;
+  if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, W, V, W1, W2, y};
+  if (!tensors_ok(t16, 8)) return OMNI_ERR_INVALID_ARG;
+  size_t need = 0;
+  omni_mlp_workspace_size(dims, F, 1, &need);
+  if (ws == nullptr || !al(ws, 256) || ws_bytes < need) return OMNI_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carver c(ws);
+  void* ws_routed = c.take<char>(ws_size(D, OMNI_WS_FUSED));
+  void* ws_mlp = c.take<char>(omni::mlp_ws_bytes(D, F));
+  if ((rc = moe_forward_impl(D, x, Wr, Wc, bias_r, bias_c, W, V, y, idx_out, gate_out, counts,
+                             ws_routed, s)) != OMNI_OK)
+    return rc;
+  omni::CallRange stage("shared_mlp");
+  return cuda_status(omni::launch_shared_mlp(D, F, x, W1, W2, y, true, ws_mlp, counts + 2, s));
 }
 
 int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,

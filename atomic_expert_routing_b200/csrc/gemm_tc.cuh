@@ -22,6 +22,7 @@
 // columns c .. c + 31 (0 <= c < BN).
 #pragma once
 
+#include "internal.h"
 #include "tc_common.cuh"
 
 namespace omni {

@@ -113,6 +113,13 @@ cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
                          cudaStream_t s);
 
+// ---- shared dense MLP: y (+)= SiLU(x W1^T) W2^T on the tensor cores ---------
+// bf16 storage only; ws holds the hidden activations H [L x F] (bf16).
+size_t mlp_ws_bytes(const Dims& D, int64_t F);
+cudaError_t launch_shared_mlp(const Dims& D, int64_t F, const void* x, const void* W1,
+                              const void* W2, void* y, bool accumulate, void* ws, int32_t* status,
+                              cudaStream_t s);
+
 // Launch with programmatic stream serialisation (see pdl_wait/pdl_trigger):
 // the kernel may be scheduled while its predecessor on the stream finishes.
 // Arguments are converted to the kernel's parameter types.

@@ -598,8 +598,39 @@ def run_ours(args):
             rec["ablation"] = measure_ablation(sc, dd, 10)
         return rec
 
+    def measure_mlp(c, dd, F, steps):
+        """The shared dense MLP branch (omni_shared_mlp: two tcgen05 GEMMs) of
+        width F on this batch, timed alone with events after an L2 flush;
+        2 * 2 * L * d * F flops against the measured bf16 peak (burst)."""
+        D = omni.LayerDims.of(c)
+        w = {k: to_dev(v) for k, v in WL.make_mlp(c, F).items()}
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        ws = omni.Workspace()
+        stream = torch.cuda.current_stream(device)
+        for _ in range(3):
+            omni.shared_mlp(D, dd["x"], w["W1"], w["W2"], y=y, ws=ws)
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            omni.shared_mlp(D, dd["x"], w["W1"], w["W2"], y=y, ws=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        ms = tot / steps
+        flops = 4.0 * c.L * c.d * F
+        ach = flops / (ms * 1e-3) / 1e12
+        return {"F": F, "ms": ms, "kernel": "two tcgen05 GEMMs (SiLU epilogue to bf16 H; add into y)",
+                "roofline": {"bound": "tensor", "achieved": ach, "peak": tc, "unit": "TFLOP/s",
+                             "frac": ach / tc, "flops": flops, "peak_src": peak_src}}
+
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
+        # the shared dense MLP of the same batch, width F = d
+        extra["shared_mlp"] = measure_mlp(cfg, d, cfg.d, max(3, args.steps // 2))
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)

@@ -237,6 +237,42 @@ int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const
                      size_t ws_bytes, void* stream);
 
 /*
+ * The shared dense MLP branch [NL 2.1] (an always-on dense MLP beside the
+ * routed experts; the pages give neither its width nor its activation, and
+ * this library takes one hidden layer of F units with the experts' scalar
+ * SiLU):  y (+)= SiLU(x W1^T) W2^T.
+ *   W1 [F x d], W2 [d x F]: bf16, row-major, 16-byte aligned.
+ *   y  [L x d] bf16: overwritten (accumulate == 0) or added to (accumulate
+ *      != 0: y = bf16(y + MLP(x)), one rounding of the sum).
+ * Both products run on the tensor cores; the hidden activations are stored
+ * in bf16 in ws (omni_mlp_workspace_size with with_routed = 0).
+ * F < 1 returns OMNI_ERR_INVALID_ARG; F not a multiple of 8, F > 65536 or
+ * fp32 storage return OMNI_ERR_UNSUPPORTED.  counts (nullable) receives
+ * device status bits in counts[2].
+ */
+int omni_shared_mlp(const omni_dims* dims, int64_t F, const void* x, const void* W1,
+                    const void* W2, void* y, int accumulate, int32_t* counts, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * The whole OmniMoE layer output of [NL 2.1], y = routed(x) + MLP(x): the
+ * routed branch as omni_moe_forward (same arguments and outputs), then the
+ * shared MLP of omni_shared_mlp added into y on the same stream.  The routed
+ * part is rounded to bf16 in y before the MLP's sum is added and rounded
+ * again.  ws: omni_mlp_workspace_size with with_routed = 1.
+ */
+int omni_moe_mlp_forward(const omni_dims* dims, int64_t F, const void* x, const void* Wr,
+                         const void* Wc, const float* bias_r, const float* bias_c, const void* W,
+                         const void* V, const void* W1, const void* W2, void* y,
+                         int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Bytes of workspace of omni_shared_mlp (with_routed == 0) or of
+ * omni_moe_mlp_forward (with_routed != 0) for these dims and width F; the
+ * same dims and F checks as those calls. */
+int omni_mlp_workspace_size(const omni_dims* dims, int64_t F, int with_routed, size_t* bytes);
+
+/*
  * Token-centric execution, the order Expert-Centric Scheduling replaces
  * [NL 2.2], [MS sched]: every token gathers the rows of its own K experts,
  * y[t] = sum_k gate[t,k] * SiLU(x[t] . W[idx[t,k]]) * V[idx[t,k]].

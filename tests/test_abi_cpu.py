@@ -207,3 +207,28 @@ def test_noalloc_size_limit(lib, L, d, code):
     args = [fake] * 10
     args[9] = None  # y
     assert lib.omni_expert_forward_noalloc(C.byref(D), *args, None) == code
+
+
+@pytest.mark.parametrize("F,dtype,code", [
+    (0, _lib.OMNI_BF16, _lib.OMNI_ERR_INVALID_ARG),
+    (-8, _lib.OMNI_BF16, _lib.OMNI_ERR_INVALID_ARG),
+    (12, _lib.OMNI_BF16, _lib.OMNI_ERR_UNSUPPORTED),      # not a multiple of 8
+    (65544, _lib.OMNI_BF16, _lib.OMNI_ERR_UNSUPPORTED),
+    (64, _lib.OMNI_F32, _lib.OMNI_ERR_UNSUPPORTED),       # tensor cores: bf16 only
+    (64, _lib.OMNI_BF16, _lib.OMNI_OK),
+])
+def test_shared_mlp_host_checks(lib, F, dtype, code):
+    """The MLP width and storage checks, before any launch (null tensors
+    stop the accepted case)."""
+    D = _dims(dtype=dtype)
+    n = C.c_size_t(0)
+    assert lib.omni_mlp_workspace_size(C.byref(D), F, 0, C.byref(n)) == code
+    if code == _lib.OMNI_OK:
+        assert n.value == 128 * 64 * 2  # the bf16 hidden activations
+        assert lib.omni_mlp_workspace_size(C.byref(D), F, 1, C.byref(n)) == _lib.OMNI_OK
+        assert n.value >= 128 * 64 * 2 + _wsz(lib, D, _lib.OMNI_WS_FUSED)[1]
+    fake = C.c_void_p(4096)
+    rc = lib.omni_shared_mlp(C.byref(D), F, None, fake, fake, fake, 0, None, fake, 1 << 30, None)
+    assert rc == (code if code != _lib.OMNI_OK else _lib.OMNI_ERR_INVALID_ARG)
+    rc = lib.omni_moe_mlp_forward(C.byref(D), F, *([fake] * 12), None, fake, 1 << 30, None)
+    assert rc == (code if code != _lib.OMNI_OK else _lib.OMNI_ERR_INVALID_ARG)

@@ -48,10 +48,24 @@ def _calls():
     }
 
 
-@pytest.mark.parametrize("name", list(_calls()))
+def _mlp_calls():
+    c = CFG.with_(dtype=WL.BF16)
+    D = omni.LayerDims.of(c)
+    b = torch.bfloat16
+    x, Wr, Wc = _t(c.L, c.d, dtype=b), _t(c.Nr, c.d, dtype=b), _t(c.Nc, c.d, dtype=b)
+    W, V = _t(c.N, c.d, dtype=b), _t(c.N, c.d, dtype=b)
+    W1, W2 = _t(16, c.d, dtype=b), _t(c.d, 16, dtype=b)
+    return {
+        "shared_mlp": lambda: omni.shared_mlp(D, x, W1, W2),
+        "moe_mlp_forward": lambda: omni.moe_mlp_forward(D, x, Wr, Wc, W, V, W1, W2),
+    }
+
+
+@pytest.mark.parametrize("name", list(_calls()) + list(_mlp_calls()))
 def test_host_tensors_are_refused(name):
+    calls = dict(_calls(), **_mlp_calls())
     with pytest.raises(ValueError, match="CUDA device"):
-        _calls()[name]()
+        calls[name]()
 
 
 def test_a_missing_library_is_an_error(tmp_path):

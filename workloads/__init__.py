@@ -32,6 +32,7 @@ CHUNK = 1 << 22  # elements per independent random stream
 
 # fixed per-tensor stream offsets
 _T_X, _T_WR, _T_WC, _T_W, _T_V, _T_PERM_R, _T_PERM_C = 0, 1, 2, 3, 4, 5, 6
+_T_W1, _T_W2 = 7, 8  # the shared dense MLP
 
 F32 = 0
 BF16 = 1
@@ -155,6 +156,13 @@ def make_experts(cfg: Config) -> dict:
     sc = 1.0 / np.sqrt(cfg.d)
     return {"W": _normal(cfg.seed, _T_W, (cfg.N, cfg.d), sc, cfg.dtype),
             "V": _normal(cfg.seed, _T_V, (cfg.N, cfg.d), sc, cfg.dtype)}
+
+
+def make_mlp(cfg: Config, F: int) -> dict:
+    """Weights of a shared dense MLP of width F: W1 [F x d] ~ N(0, 1/d),
+    W2 [d x F] ~ N(0, 1/F) (so both products keep unit scale)."""
+    return {"W1": _normal(cfg.seed, _T_W1, (F, cfg.d), 1.0 / np.sqrt(cfg.d), cfg.dtype),
+            "W2": _normal(cfg.seed, _T_W2, (cfg.d, F), 1.0 / np.sqrt(F), cfg.dtype)}
 
 
 def sample_tokens(cfg: Config, n: int, seed: int = 1234) -> np.ndarray:
