@@ -19,7 +19,8 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_ROUTER_SIMT, OMNI_FLAG_STAGED_SMALL,
+from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_DENSE_TENSOR_CORES, OMNI_FLAG_ROUTER_SIMT,
+                   OMNI_FLAG_STAGED_SMALL,
                    OMNI_WS_EXPERT, OMNI_WS_FUSED,
                    OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
 

@@ -20,6 +20,7 @@ OMNI_F32 = 0
 OMNI_BF16 = 1
 OMNI_FLAG_ROUTER_SIMT = 1
 OMNI_FLAG_STAGED_SMALL = 2
+OMNI_FLAG_DENSE_TENSOR_CORES = 4
 
 OMNI_WS_ROUTE = 0
 OMNI_WS_SCHEDULE = 1

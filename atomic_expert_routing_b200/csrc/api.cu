@@ -33,7 +33,7 @@ int check_dims(const omni_dims* in, Dims* D) {
   if (D->L < 0 || D->d < 1 || D->Nr < 1 || D->Nc < 1 || D->k < 1 || D->K < 1 || D->B < 1)
     return OMNI_ERR_INVALID_ARG;
   if (D->dtype != OMNI_F32 && D->dtype != OMNI_BF16) return OMNI_ERR_INVALID_ARG;
-  if ((D->flags & ~(OMNI_FLAG_ROUTER_SIMT | OMNI_FLAG_STAGED_SMALL)) != 0)
+  if ((D->flags & ~(OMNI_FLAG_ROUTER_SIMT | OMNI_FLAG_STAGED_SMALL | OMNI_FLAG_DENSE_TENSOR_CORES)) != 0)
     return OMNI_ERR_INVALID_ARG;
   // k*k in 128 bits: k is only bounded by the axes here
   if (D->k > D->Nr || D->k > D->Nc ||
@@ -277,7 +277,6 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
                         const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                         int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream) {
   omni::CallRange range("omni_expert_forward");
-  (void)uniq;
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
@@ -287,7 +286,7 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
       task_gate == nullptr || group_off == nullptr || counts == nullptr)
     return OMNI_ERR_INVALID_ARG;
   if ((rc = ws_ok(D, OMNI_WS_EXPERT, ws, ws_bytes)) != OMNI_OK) return rc;
-  return cuda_status(omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate,
+  return cuda_status(omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate, uniq,
                                          group_off, counts, y, ws,
                                          static_cast<cudaStream_t>(stream)));
 }
@@ -350,7 +349,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   if (rc != OMNI_OK) return rc;
   omni::CallRange stage("expert");
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
-                                         w.group_off, counts, y, w.expert, s, acc_zeroed));
+                                         w.uniq, w.group_off, counts, y, w.expert, s, acc_zeroed));
 }
 
 // The checks of the shared MLP's width: F >= 1; a multiple of 8 (16-byte

@@ -266,14 +266,17 @@ constexpr int kAsyncWarps = 8;
 // vectors, so no cross-lane synchronisation is needed), prefetches x of the
 // next piece into registers one task ahead, and computes the current task
 // from shared memory.  Warps run a grid-stride loop over task slices; the
-// pipeline restarts at every slice.
+// pipeline restarts at every slice.  With dense != nullptr, a task with
+// dense[a] set takes its activation c from cpre[a] (formed on the tensor
+// cores) and fetches only its V row.
 template <typename T, int NV, int R>
 __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
     k_expert_async(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
                    const int32_t* __restrict__ task_token,
                    const int32_t* __restrict__ task_expert,
                    const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
-                   int S, int64_t nslices, float* __restrict__ yacc, int32_t* status) {
+                   int S, int64_t nslices, float* __restrict__ yacc, int32_t* status,
+                   const uint8_t* __restrict__ dense, const float* __restrict__ cpre) {
   pdl_wait();
   pdl_trigger();
   constexpr int EPV = kEpv<T>;
@@ -289,33 +292,43 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
     const int64_t a0 = sl * S;
     const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
     int64_t my_t = -1, my_e = -1;
-    float my_g = 0.0f;
+    float my_g = 0.0f, my_cp = 0.0f;
+    bool my_dense = false;
     if (lane < n) {
       my_t = task_token[a0 + lane];
       my_e = task_expert[a0 + lane];
       my_g = task_gate[a0 + lane];
+      if (dense != nullptr && dense[a0 + lane] != 0) {
+        my_dense = true;
+        my_cp = cpre[a0 + lane];
+      }
       if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
         raise_status(status, OMNI_DEV_BAD_INDEX);
         my_e = -1;
         my_t = -1;
       }
     }
+    const uint32_t dmask = __ballot_sync(0xffffffffu, my_dense);
     const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
     const int64_t next_t = __shfl_down_sync(0xffffffffu, my_t, 1);
     const uint32_t starts = __ballot_sync(0xffffffffu, lane < n && (lane == 0 || prev_t != my_t));
     const uint32_t ends = __ballot_sync(0xffffffffu, lane < n && (lane == n - 1 || next_t != my_t));
 
-    // issue the row copies of task j into slot j % R (one commit group per task)
+    // issue the row copies of task j into slot j % R (one commit group per
+    // task; a dense task needs only its V row)
     auto issue = [&](int j) {
       if (j < n) {
         const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
         if (e >= 0) {
+          const bool need_w = !((dmask >> j) & 1u);
           const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
           const uint4* vr = reinterpret_cast<const uint4*>(V + e * d);
           const uint32_t base = wring_s + static_cast<uint32_t>((j % R) * SLOT) * 16u;
 #pragma unroll
           for (int v = 0; v < NV; ++v) {
-            cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, wr + v * 32 + lane, pol_stream);
+            if (need_w)
+              cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, wr + v * 32 + lane,
+                         pol_stream);
             cp_async16(base + static_cast<uint32_t>((NV + v) * 32 + lane) * 16u, vr + v * 32 + lane,
                        pol_stream);
           }
@@ -358,11 +371,17 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
       const int64_t t = __shfl_sync(0xffffffffu, my_t, j);
       if (e >= 0) {  // warp-uniform
         const uint4* slot = wring + (j % R) * SLOT;
-        float sdot = 0.0f;
+        float c;
+        if ((dmask >> j) & 1u) {  // warp-uniform
+          c = __shfl_sync(0xffffffffu, my_cp, j);
+        } else {
+          float sdot = 0.0f;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
-        sdot = warp_sum(sdot);
-        const float c = gj * silu(sdot);
+          for (int v = 0; v < NV; ++v)
+            sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
+          sdot = warp_sum(sdot);
+          c = gj * silu(sdot);
+        }
 #pragma unroll
         for (int v = 0; v < NV; ++v)
           axpy_vec(c, slot[(NV + v) * 32 + lane], acc + v * EPV, static_cast<T*>(nullptr));
@@ -1089,8 +1108,18 @@ SweepWs carve_sweeps(const Dims& D, void* ws, size_t* bytes) {
   return w;
 }
 
+// bf16 batches without sweeps whose row width has a k_expert_async instance
+// run the activations of dense groups on the tensor cores first.
+bool dense_path(const Dims& D) {
+  if (!dense_supported(D) || expert_sweeps(D) > 1) return false;
+  return D.d == 256 || D.d == 512 || D.d == 1024 || D.d == 2048;
+}
+
+size_t dense_ws_offset(const Dims& D) { return (acc_bytes(D) + 255) & ~size_t(255); }
+
 size_t expert_ws_bytes(const Dims& D) {
-  if (expert_sweeps(D) <= 1) return acc_bytes(D);
+  if (expert_sweeps(D) <= 1)
+    return dense_path(D) ? dense_ws_offset(D) + dense_ws_bytes(D) : acc_bytes(D);
   size_t b = 0;
   carve_sweeps(D, nullptr, &b);
   return b;
@@ -1119,7 +1148,7 @@ cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const voi
 template <typename T, int NV, int R>
 cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* tt, const int32_t* te, const float* tg, float* acc,
-                         int32_t* status, cudaStream_t s) {
+                         int32_t* status, cudaStream_t s, const DenseFlags& df) {
   constexpr size_t smem = static_cast<size_t>(kAsyncWarps) * R * 2 * NV * 32 * 16;
   cudaError_t err = cudaFuncSetAttribute(k_expert_async<T, NV, R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1137,20 +1166,23 @@ cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void
   if (blocks > sms) blocks = sms;  // persistent: one CTA per SM (shared-memory bound)
   OMNI_TRY(launch_k(k_expert_async<T, NV, R>, static_cast<unsigned>(blocks), kAsyncWarps * 32, smem,
       s, static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
-      M, D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status));
+      M, D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status, df.flag, df.cbuf));
   return cudaGetLastError();
 }
 
+// df: the dense-group activations (flag == nullptr: none).  Row widths
+// without a k_expert_async instance take k_expert_slices, which forms every
+// activation itself; the dense path is only run for widths that have one.
 template <typename T>
 cudaError_t dispatch_slices(const Dims& D, const void* x, const void* W, const void* V,
                             const int32_t* tt, const int32_t* te, const float* tg, float* acc,
-                            int32_t* status, cudaStream_t s) {
+                            int32_t* status, cudaStream_t s, const DenseFlags& df) {
   constexpr int row = 32 * kEpv<T>;  // elements covered by one vector per lane
   switch (D.d == row * 8 ? 8 : D.d == row * 4 ? 4 : D.d == row * 2 ? 2 : D.d == row ? 1 : 0) {
-    case 8: return launch_async<T, 8, 3>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 4: return launch_async<T, 4, 4>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 2: return launch_async<T, 2, 4>(D, x, W, V, tt, te, tg, acc, status, s);
-    case 1: return launch_async<T, 1, 4>(D, x, W, V, tt, te, tg, acc, status, s);
+    case 8: return launch_async<T, 8, 3>(D, x, W, V, tt, te, tg, acc, status, s, df);
+    case 4: return launch_async<T, 4, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
+    case 2: return launch_async<T, 2, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
+    case 1: return launch_async<T, 1, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
     default: return launch_slices<T, 0>(D, x, W, V, tt, te, tg, acc, status, s);
   }
 }
@@ -1304,9 +1336,9 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
 
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
-                          const float* task_gate, const int32_t* group_off,
+                          const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                           const int32_t* counts, void* y, void* ws, cudaStream_t s,
-                          bool acc_zeroed) {
+                          bool acc_zeroed, bool allow_dense) {
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
   float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
@@ -1324,9 +1356,17 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
   cudaError_t err = acc_zeroed ? cudaSuccess
                                : launch_zero(acc, static_cast<size_t>(expert_acc_words(D)), s);
   if (err != cudaSuccess) return err;
-  err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status, s)
+  DenseFlags df{nullptr, nullptr};
+  if (allow_dense && uniq != nullptr && dense_path(D)) {
+    void* dws = static_cast<char*>(ws) + dense_ws_offset(D);
+    OMNI_TRY(launch_dense_activations(D, x, W, task_token, task_expert, task_gate, uniq,
+                                      group_off, const_cast<int32_t*>(counts), dws, s));
+    df = dense_flags(D, dws);
+  }
+  err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status,
+                                     s, df)
             : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
-                                             status, s);
+                                             status, s, df);
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;
   OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,

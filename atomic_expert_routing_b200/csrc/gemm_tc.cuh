@@ -17,9 +17,13 @@
 //
 // Tile source: int count() (tiles, read after the kernel ahead finished) and
 // void at(int t, int* a_row0, int* b_row0) (first rows of tile t).
-// Epilogue: void operator()(int t, int a_row0, int b_row0, int r, int c,
-// const uint32_t* v) -- row r (0..127) of tile t, fp32 bit patterns of its
-// columns c .. c + 31 (0 <= c < BN).
+// Epilogue: static constexpr size_t kStageBytes (shared memory it may use,
+// 0 for none); void operator()(int t, int a_row0, int b_row0, int r, int c,
+// const uint32_t* v, float* stage) -- row r (0..127) of tile t, fp32 bit
+// patterns of its columns c .. c + 31 (0 <= c < BN); and, when kStageBytes
+// > 0, void tile_end(int t, int a_row0, int b_row0, int i, float* stage),
+// called by the 128 epilogue threads (i = 0..127) once every row of the tile
+// has been handed over (the stage is theirs until the next tile's rows).
 #pragma once
 
 #include "internal.h"
@@ -33,6 +37,11 @@ constexpr size_t gemm_smem_bytes() {
   return 1024 /* alignment slack */ +
          static_cast<size_t>(TC_STAGES) * (TC_BM * TC_BK * 2 + BN * TC_BK * 2) +
          (2 * TC_STAGES + 5) * 8 + 16;
+}
+
+// named barrier of the four epilogue warps (barrier 0 is __syncthreads)
+__device__ __forceinline__ void epilogue_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 template <int BN, class Tiles, class Epi>
@@ -50,6 +59,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * B_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * TC_STAGES + 5);
   uint32_t* aborted = tmem_slot + 1;  // a wait of this CTA timed out
+  float* stage = reinterpret_cast<float*>(aborted + 3);  // Epi::kStageBytes (4-byte aligned)
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + TC_STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * TC_STAGES);       // accumulator b ready
@@ -157,10 +167,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + b * BN + c, r);
-        epi(t, a0, b0, warp * 32 + lane, c, r);
+        epi(t, a0, b0, warp * 32 + lane, c, r, stage);
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      mbar_arrive(tempty0 + 8 * b);
+      mbar_arrive(tempty0 + 8 * b);  // TMEM is free once every row is read
+      if constexpr (Epi::kStageBytes > 0) {
+        epilogue_sync();  // every row is in the stage
+        epi.tile_end(t, a0, b0, warp * 32 + lane, stage);
+        epilogue_sync();  // the stage is free for the next tile
+      }
     }
   }
   if (timed_out) *aborted = 1u;
@@ -205,7 +220,7 @@ struct DenseTiles {
 template <int BN, class Tiles, class Epi>
 cudaError_t launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int nk, const Tiles& T,
                            int64_t tiles_hint, const Epi& epi, int32_t* status, cudaStream_t s) {
-  const size_t smem = gemm_smem_bytes<BN>();
+  const size_t smem = gemm_smem_bytes<BN>() + Epi::kStageBytes;
   cudaError_t err = cudaFuncSetAttribute(k_gemm_tc<BN, Tiles, Epi>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

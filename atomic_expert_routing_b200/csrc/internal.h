@@ -93,6 +93,23 @@ cudaError_t launch_sched_exec(const Dims& D, const void* x, const void* W, const
                               const int32_t* idx, const float* gate, void* y, uint32_t* ws,
                               int32_t* counts, cudaStream_t s);
 
+// ---- activations of dense groups on the tensor cores ----------------------
+// bf16, d a multiple of 64, B <= 256.  The planner flags the tasks of dense
+// groups and the tensor-core pass writes their activations c (both in the
+// dense workspace); counts[3] receives the number of dense groups.
+bool dense_supported(const Dims& D);
+size_t dense_ws_bytes(const Dims& D);
+struct DenseFlags {
+  const uint8_t* flag;  // [M] task of a dense group (its c is in cbuf)
+  const float* cbuf;    // [M]
+};
+DenseFlags dense_flags(const Dims& D, void* ws);
+cudaError_t launch_dense_activations(const Dims& D, const void* x, const void* W,
+                                     const int32_t* task_token, const int32_t* task_expert,
+                                     const float* task_gate, const int32_t* uniq,
+                                     const int32_t* group_off, int32_t* counts, void* ws,
+                                     cudaStream_t s);
+
 // ---- execution -----------------------------------------------------------
 size_t expert_ws_bytes(const Dims& D);
 int expert_sweeps(const Dims& D);                // slices of d (1: no sweeps)
@@ -100,11 +117,14 @@ WinTasks expert_windows(const Dims& D, void* ws);  // the window buffers of an e
 // The sweeps from tasks already in window token order (expert_windows(ws)).
 cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, const void* V,
                                   int32_t* counts, void* y, void* ws, cudaStream_t s);
+// uniq: the schedule's U (the dense-group path reads it); allow_dense: run
+// the activations of dense groups on the tensor cores when the workspace is
+// the full OMNI_WS_EXPERT size (false: ws holds only the accumulator).
 cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* task_token, const int32_t* task_expert,
-                          const float* task_gate, const int32_t* group_off,
+                          const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                           const int32_t* counts, void* y, void* ws, cudaStream_t s,
-                          bool acc_zeroed = false);
+                          bool acc_zeroed = false, bool allow_dense = true);
 // The accumulator launch_expert clears before a batch without sweeps (its fp32
 // partial sums: y itself for fp32, else the head of ws), in floats; 0 for
 // batches with sweeps.

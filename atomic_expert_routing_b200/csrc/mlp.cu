@@ -33,11 +33,12 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* f) {
 // First GEMM: H[row, col] = bf16(SiLU(acc)).  Rows of H are ld elements apart
 // (ld a multiple of 8, so 32-column chunks are 16-byte aligned).
 struct SiluToHidden {
+  static constexpr size_t kStageBytes = 0;
   __nv_bfloat16* H;
   int64_t ld;
   int rows, cols;
   __device__ __forceinline__ void operator()(int, int a0, int b0, int r, int c,
-                                             const uint32_t* v) const {
+                                             const uint32_t* v, float*) const {
     const int row = a0 + r;
     if (row >= rows) return;
     const int col = b0 + c;
@@ -60,11 +61,12 @@ struct SiluToHidden {
 
 // Second GEMM: y[row, col] = bf16(acc + (accumulate ? y[row, col] : 0)).
 struct AddToOutput {
+  static constexpr size_t kStageBytes = 0;
   __nv_bfloat16* Y;
   int64_t ld;
   int rows, cols, accumulate;
   __device__ __forceinline__ void operator()(int, int a0, int b0, int r, int c,
-                                             const uint32_t* v) const {
+                                             const uint32_t* v, float*) const {
     const int row = a0 + r;
     if (row >= rows) return;
     const int col = b0 + c;

@@ -51,14 +51,12 @@ extern "C" int omni_expert_forward_noalloc(const omni_dims* dims, const void* x,
                                            const int32_t* uniq, const int32_t* group_off,
                                            int32_t* counts, void* y, void* stream) {
   omni::CallRange range("omni_expert_forward_noalloc");
-  (void)uniq;
   if (dims == nullptr) return OMNI_ERR_INVALID_ARG;
   size_t need = 0;
-  int rc = omni_workspace_size(dims, OMNI_WS_EXPERT, &need);  // also validates dims
+  int rc = omni_workspace_size(dims, OMNI_WS_EXPERT, &need);  // validates dims
   if (rc != OMNI_OK) return rc;
   if (dims->L == 0) return OMNI_OK;
-  if (static_cast<size_t>(dims->L) * static_cast<size_t>(dims->d) > kNoAllocMaxElems ||
-      need > sizeof(g_noalloc_acc))
+  if (static_cast<size_t>(dims->L) * static_cast<size_t>(dims->d) > kNoAllocMaxElems)
     return OMNI_ERR_UNSUPPORTED;  // batch too large for the fixed scratch
   auto al16 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(x) || !al16(W) || !al16(V) || !al16(y) || task_token == nullptr ||
@@ -67,15 +65,18 @@ extern "C" int omni_expert_forward_noalloc(const omni_dims* dims, const void* x,
   omni::Dims D;
   D.L = dims->L; D.d = dims->d; D.Nr = dims->Nr; D.Nc = dims->Nc;
   D.k = dims->k; D.K = dims->K; D.B = dims->B; D.dtype = dims->dtype; D.flags = dims->flags;
+  // the array holds the accumulator only: the sweep path and the dense-group
+  // path need more scratch than that
+  if (omni::expert_sweeps(D) > 1) return OMNI_ERR_UNSUPPORTED;
   float* acc = nullptr;
-  if (need > 0) {
+  if (omni::expert_acc_words(D) > 0) {
     const cudaError_t e = acc_address(&acc);
     if (e != cudaSuccess) return omni::cuda_status(e);
   }
   // launch_expert zeroes the accumulator before use (it keeps the previous
   // call's contents otherwise)
   const cudaError_t e = omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate,
-                                            group_off, counts, y, acc,
-                                            static_cast<cudaStream_t>(stream));
+                                            uniq, group_off, counts, y, acc,
+                                            static_cast<cudaStream_t>(stream), false, false);
   return omni::cuda_status(e);
 }

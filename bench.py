@@ -108,6 +108,12 @@ def group_density(task_token, group_off, B, n_active, block=128):
             "tasks_per_tile_max": float(per_tile.max()), "tile_tokens": block}
 
 
+# A synthetic batch whose groups are dense: 8192 tokens routed to 256
+# experts (two groups of 128), for the timing of the tensor-core activations.
+DENSE_SYNTH = WL.Config("bf16-dense-groups-N256", L=8192, d=1024, Nr=16, Nc=16, k=8, K=8, B=128,
+                        dtype=WL.BF16, seed=0)
+
+
 def expert_stage_bytes(cfg, n_active):
     """Algorithmic bytes of the grouped execution: active rows of W and V once,
     x read, y written."""
@@ -627,10 +633,49 @@ def run_ours(args):
                 "roofline": {"bound": "tensor", "achieved": ach, "peak": tc, "unit": "TFLOP/s",
                              "frac": ach / tc, "flops": flops, "peak_src": peak_src}}
 
+    def measure_dense_paths(steps):
+        """A batch routed to 256 experts by 8192 tokens (two groups, 512 tasks
+        per touched 128-token tile): its grouped execution with the dense
+        groups' activations on the tensor cores (OMNI_FLAG_DENSE_TENSOR_CORES)
+        and with every activation on the CUDA cores (the default), each after
+        an L2 flush."""
+        dc = DENSE_SYNTH
+        hs = WL.make_inputs(dc)
+        ds = {k: to_dev(v) for k, v in hs.items()}
+        out = {"workload": dc.name}
+        for name, flags in (("tensor_cores", omni.OMNI_FLAG_DENSE_TENSOR_CORES), ("cuda_cores", 0)):
+            D = omni.LayerDims.of(dc, flags=flags)
+            idx, gate, _ = omni.route(D, ds["x"], ds["Wr"], ds["Wc"], with_score=False)
+            counts = omni.new_counts(device)
+            counts[3] = -1
+            sch = omni.schedule(D, idx, gate, counts=counts)
+            y = torch.empty((dc.L, dc.d), dtype=D.torch_dtype, device=device)
+            ws = omni.Workspace()
+            stream = torch.cuda.current_stream(device)
+            for _ in range(3):
+                omni.expert_forward(D, ds["x"], ds["W"], ds["V"], sch, y=y, ws=ws)
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                omni.expert_forward(D, ds["x"], ds["W"], ds["V"], sch, y=y, ws=ws)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1)
+            out[name] = {"expert_ms": tot / steps, "dense_groups": int(counts[3].item()),
+                         "groups": int(counts[1].item())}
+        del ds
+        torch.cuda.empty_cache()
+        return out
+
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
         # the shared dense MLP of the same batch, width F = d
         extra["shared_mlp"] = measure_mlp(cfg, d, cfg.d, max(3, args.steps // 2))
+        extra["dense_groups"] = measure_dense_paths(max(3, args.steps // 2))
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)

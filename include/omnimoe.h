@@ -77,6 +77,11 @@ extern "C" {
                                     scheduling and grouped-execution kernels of
                                     omni_schedule and omni_expert_forward instead of its
                                     two-kernel small-batch tail */
+#define OMNI_FLAG_DENSE_TENSOR_CORES 4 /* grouped execution of bf16 batches without
+                                          column sweeps: the activations of dense groups
+                                          (>= 384 tasks per 128-token tile of a group's
+                                          B <= 128 experts) are formed on the tensor cores;
+                                          counts[3] receives how many groups were */
 
 /* Limits of this build (host checks return OMNI_ERR_UNSUPPORTED beyond them). */
 #define OMNI_MAX_AXIS 4096      /* Nr, Nc */

@@ -118,7 +118,8 @@ def test_empty_batch_is_a_no_op(lib):
 def _documented_code(L, d, Nr, Nc, k, K, B, dtype, flags):
     """The host checks as the header states them (invalid before unsupported)."""
     if (L < 0 or min(d, Nr, Nc, k, K, B) < 1 or dtype not in (_lib.OMNI_F32, _lib.OMNI_BF16)
-            or flags & ~(_lib.OMNI_FLAG_ROUTER_SIMT | _lib.OMNI_FLAG_STAGED_SMALL)
+            or flags & ~(_lib.OMNI_FLAG_ROUTER_SIMT | _lib.OMNI_FLAG_STAGED_SMALL
+                         | _lib.OMNI_FLAG_DENSE_TENSOR_CORES)
             or k > min(Nr, Nc) or K > k * k):
         return _lib.OMNI_ERR_INVALID_ARG
     if (max(Nr, Nc) > 4096 or max(k, K) > 256 or Nr * Nc >= 2 ** 31 or L * K >= 2 ** 30
@@ -146,7 +147,7 @@ def test_dims_checks_follow_the_header(lib):
     @given(L=field, d=st.one_of(st.sampled_from([8, 16, 40, 64, 2048, 65536, 65544]), field),
            Nr=field, Nc=field, k=st.one_of(st.integers(1, 300), field),
            K=st.one_of(st.integers(1, 300), field), B=field,
-           dtype=st.sampled_from([0, 1, 2, -1]), flags=st.sampled_from([0, 1, 2, 3, 4, 7]))
+           dtype=st.sampled_from([0, 1, 2, -1]), flags=st.sampled_from([0, 1, 2, 3, 4, 7, 8, 15]))
     # L*K that wraps around int64; k*k that does
     @example(L=2 ** 62, d=64, Nr=64, Nc=64, k=2, K=4, B=1, dtype=1, flags=0)
     @example(L=16, d=64, Nr=2 ** 33, Nc=2 ** 33, k=2 ** 32, K=1, B=1, dtype=1, flags=0)
