@@ -166,7 +166,8 @@ def schedule(cfg, idx, gate, tokens=None):
 
 
 def forward_expert(cfg, inp, sched, tokens=None):
-    """Expert-centric execution; returns (y [nt, d] float64, rows_loaded (W, V))."""
+    """Expert-centric execution; returns (y [nt, d] float64, rows_loaded (W, V)).
+    With inp["U"] the experts are gated: h = SiLU(x.W[e]) * (x.U[e])."""
     tok = _tokens(cfg, tokens)
     out_row = np.full(cfg.L, -1, np.int64)
     out_row[tok] = np.arange(len(tok))
@@ -175,7 +176,7 @@ def forward_expert(cfg, inp, sched, tokens=None):
     D = dims(cfg)
     go = np.ascontiguousarray(sched["group_off"], np.int32)
     _check(lib().oracle_forward_expert(
-        C.byref(D), _p(inp["x"]), _p(inp["W"]), _p(inp["V"]),
+        C.byref(D), _p(inp["x"]), _p(inp["W"]), _p(inp.get("U")), _p(inp["V"]),
         _p(np.ascontiguousarray(sched["task_token"], np.int32)),
         _p(np.ascontiguousarray(sched["task_expert"], np.int32)),
         _p(np.ascontiguousarray(sched["task_gate"], np.float64)),
@@ -186,13 +187,15 @@ def forward_expert(cfg, inp, sched, tokens=None):
 
 
 def forward_token(cfg, inp, idx, gate, tokens=None):
-    """Token-centric execution; returns (y [nt, d] float64, rows_loaded (W, V))."""
+    """Token-centric execution; returns (y [nt, d] float64, rows_loaded (W, V)).
+    With inp["U"] the experts are gated, as in forward_expert."""
     tok = _tokens(cfg, tokens)
     y = np.empty((len(tok), cfg.d), np.float64)
     rows = np.zeros(2, np.int64)
     D = dims(cfg)
     _check(lib().oracle_forward_token(
-        C.byref(D), _p(inp["x"]), _p(inp["W"]), _p(inp["V"]), _p(tok), C.c_int64(len(tok)),
+        C.byref(D), _p(inp["x"]), _p(inp["W"]), _p(inp.get("U")), _p(inp["V"]), _p(tok),
+        C.c_int64(len(tok)),
         _p(np.ascontiguousarray(idx, np.int32)), _p(np.ascontiguousarray(gate, np.float64)),
         _p(y), _p(rows)), "forward_token")
     return y, (int(rows[0]), int(rows[1]))

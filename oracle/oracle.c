@@ -381,7 +381,11 @@ static int64_t slot_of(const int32_t* uniq, int64_t u0, int64_t nb, int32_t e) {
  * Expert-centric order [MS sched]: group by group, the rows W[e], V[e] of the
  * group's experts uniq[g*B .. min((g+1)*B, n_active)) are loaded once; then
  * every task (t, e, gate) of the group, in (token, expert) order, adds
- * gate * SiLU(x[t] . W[e]) * V[e] to y[t]   [NL 2.1], [NL 2.2].
+ * gate * h * V[e] to y[t]   [NL 2.1], [NL 2.2], with h = SiLU(x[t] . W[e]).
+ * With U != NULL the expert is gated (SwiGLU, named by the OmniMoE explainer's
+ * Atomic Expert section; the pages give only the pair (w_in, w_out), and the
+ * gated form taken here adds a third global matrix U [N x d]):
+ * h = SiLU(x[t] . W[e]) * (x[t] . U[e]).
  * y rows are indexed by out_row[t] (the caller's row of token t).
  * rows_loaded[0] / [1] count rows of W / V brought in (|E_active| each).
  *
@@ -390,8 +394,8 @@ static int64_t slot_of(const int32_t* uniq, int64_t u0, int64_t nb, int32_t e) {
  * the accumulation y[t] += c * V[e] (output columns split across threads, so
  * each y element receives its terms in the single-threaded order).
  */
-int oracle_forward_expert(const or_dims* D, const void* x, const void* W, const void* V,
-                          const int32_t* task_token, const int32_t* task_expert,
+int oracle_forward_expert(const or_dims* D, const void* x, const void* W, const void* U,
+                          const void* V, const int32_t* task_token, const int32_t* task_expert,
                           const double* task_gate, const int32_t* uniq,
                           const int32_t* group_off, int64_t n_active, int64_t n_groups,
                           const int64_t* out_row, double* y, int64_t y_rows,
@@ -404,19 +408,24 @@ int oracle_forward_expert(const or_dims* D, const void* x, const void* W, const 
 #pragma omp parallel reduction(+ : wloaded)
   {
     double* wg = (double*)malloc(sizeof(double) * B * d);
+    double* ug = (double*)malloc(sizeof(double) * B * d);
     double* xrow = (double*)malloc(sizeof(double) * d);
 #pragma omp for schedule(dynamic, 1)
     for (int64_t g = 0; g < n_groups; ++g) {
       const int64_t u0 = g * B, nb = (n_active - u0 < B) ? n_active - u0 : B;
       for (int64_t j = 0; j < nb; ++j) load_row(W, D->dtype, uniq[u0 + j], d, wg + j * d);
+      if (U)
+        for (int64_t j = 0; j < nb; ++j) load_row(U, D->dtype, uniq[u0 + j], d, ug + j * d);
       wloaded += nb;
       for (int64_t q = group_off[g]; q < group_off[g + 1]; ++q) {
         const int64_t j = slot_of(uniq, u0, nb, task_expert[q]);
         load_row(x, D->dtype, task_token[q], d, xrow);
         c[q] = task_gate[q] * silu(dot(xrow, wg + j * d, d));
+        if (U) c[q] *= dot(xrow, ug + j * d, d);
       }
     }
     free(wg);
+    free(ug);
     free(xrow);
   }
   int nth_used = 1;
@@ -454,11 +463,13 @@ int oracle_forward_expert(const or_dims* D, const void* x, const void* W, const 
 /*
  * Token-centric order (the execution the scheduling replaces) [NL 2.2],
  * [MS sched]: every token fetches the rows of each of its K experts itself,
- * y[t] = sum_k gate[t,k] * SiLU(x[t] . W[e_k]) * V[e_k].
+ * y[t] = sum_k gate[t,k] * SiLU(x[t] . W[e_k]) * V[e_k], times
+ * (x[t] . U[e_k]) for the gated expert (U != NULL, as oracle_forward_expert).
  * Row r of idx/gate belongs to token tok[r]; y row r is written.
  * rows_loaded[0] / [1] count rows of W / V fetched (L*K each).
  */
-int oracle_forward_token(const or_dims* D, const void* x, const void* W, const void* V,
+int oracle_forward_token(const or_dims* D, const void* x, const void* W, const void* U,
+                         const void* V,
                          const int64_t* tok, int64_t nt, const int32_t* idx, const double* gate,
                          double* y, int64_t* rows_loaded) {
   const int64_t d = D->d, K = D->K;
@@ -468,6 +479,7 @@ int oracle_forward_token(const or_dims* D, const void* x, const void* W, const v
     double* xrow = (double*)malloc(sizeof(double) * d);
     double* wrow = (double*)malloc(sizeof(double) * d);
     double* vrow = (double*)malloc(sizeof(double) * d);
+    double* urow = (double*)malloc(sizeof(double) * d);
 #pragma omp for schedule(dynamic, 4)
     for (int64_t r = 0; r < nt; ++r) {
       double* yr = y + r * d;
@@ -478,13 +490,18 @@ int oracle_forward_token(const or_dims* D, const void* x, const void* W, const v
         load_row(W, D->dtype, e, d, wrow);
         load_row(V, D->dtype, e, d, vrow);
         fetched += 1;
-        const double cq = gate[r * K + q] * silu(dot(xrow, wrow, d));
+        double cq = gate[r * K + q] * silu(dot(xrow, wrow, d));
+        if (U) {
+          load_row(U, D->dtype, e, d, urow);
+          cq *= dot(xrow, urow, d);
+        }
         for (int64_t m = 0; m < d; ++m) yr[m] += cq * vrow[m];
       }
     }
     free(xrow);
     free(wrow);
     free(vrow);
+    free(urow);
   }
   rows_loaded[0] = fetched;
   rows_loaded[1] = fetched;

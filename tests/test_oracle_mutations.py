@@ -88,13 +88,19 @@ MUTANTS = [
     # execution
     ("expert-order-drops-gate", "c[q] = task_gate[q] * silu(dot(xrow, wg + j * d, d));",
      "c[q] = silu(dot(xrow, wg + j * d, d));"),
-    ("token-order-drops-gate", "const double cq = gate[r * K + q] * silu(dot(xrow, wrow, d));",
-     "const double cq = silu(dot(xrow, wrow, d));"),
+    ("token-order-drops-gate", "double cq = gate[r * K + q] * silu(dot(xrow, wrow, d));",
+     "double cq = silu(dot(xrow, wrow, d));"),
     ("slot-search-off-by-one", "if (uniq[u0 + mid] < e)", "if (uniq[u0 + mid] <= e)"),
     ("expert-order-V-row-of-first-expert", "elem(V, D->dtype, (int64_t)uniq[u0 + j] * d + m)",
      "elem(V, D->dtype, (int64_t)uniq[u0] * d + m)"),
     ("expert-order-overwrites-y", "yr[m] += c[q] * vg[j * w + (m - c0)];",
      "yr[m] = c[q] * vg[j * w + (m - c0)];"),
+    # gated (SwiGLU) expert
+    ("glu-drops-the-gate-factor", "if (U) c[q] *= dot(xrow, ug + j * d, d);", "if (U) c[q] *= 1.0;"),
+    ("glu-gate-row-of-W", "if (U) c[q] *= dot(xrow, ug + j * d, d);",
+     "if (U) c[q] *= dot(xrow, wg + j * d, d);"),
+    ("glu-token-order-gate-of-first-expert", "load_row(U, D->dtype, e, d, urow);",
+     "load_row(U, D->dtype, idx[r * K], d, urow);"),
     ("token-order-swaps-W-and-V",
      "load_row(W, D->dtype, e, d, wrow);\n        load_row(V, D->dtype, e, d, vrow);",
      "load_row(V, D->dtype, e, d, wrow);\n        load_row(W, D->dtype, e, d, vrow);"),

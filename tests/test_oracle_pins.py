@@ -502,3 +502,70 @@ def test_shared_mlp_linearity_rows_and_zero():
     assert np.all(ya[4] == 0.0)
     tok = np.array([1, 4, 8], np.int64)
     np.testing.assert_array_equal(O.shared_mlp(cfg, {"x": x}, W1, W2a, tokens=tok), ya[tok])
+
+
+# ------------------------------------------------------------ gated (SwiGLU) atomic expert
+
+def test_gated_expert_hand_worked():
+    """The closed-form tasks above with a gate matrix: U[e] = b_e * e_7 and
+    x[t, 7] = (2, 1, 5), so x . U[e] = x7_t b_e and h = SiLU(s_t a_e) x7_t b_e.
+    Worked by hand: token 0 -> expert 1 (a = -2, b = 0.5) and expert 5 (a = 3,
+    b = -0.5); token 1 -> expert 0 (a = 2, b = 1) and expert 4 (a = -0.25,
+    b = 4); token 2 has s = 0, so SiLU(0) = 0 and its row stays 0."""
+    cfg = WL.Config("closed-glu", L=3, d=8, Nr=2, Nc=3, k=2, K=2, B=2, dtype=WL.F32)
+    x = np.zeros((3, 8), np.float32)
+    x[:, 0] = [1.0, -1.5, 0.0]
+    x[:, 7] = [2.0, 1.0, 5.0]
+    W = np.zeros((6, 8), np.float32)
+    W[:, 0] = [2.0, -2.0, 0.5, 1.0, -0.25, 3.0]
+    U = np.zeros((6, 8), np.float32)
+    U[:, 7] = [1.0, 0.5, -1.0, 2.0, 4.0, -0.5]
+    V = np.zeros((6, 8), np.float32)
+    V[np.arange(6), [1, 2, 3, 4, 5, 6]] = [1.0, 2.0, -1.0, 0.5, 4.0, -3.0]
+    inp = {"x": x, "W": W, "U": U, "V": V}
+    idx = np.array([[1, 5], [0, 4], [2, 3]], np.int32)
+    gate = np.array([[0.75, 0.25], [0.5, 0.5], [0.9, 0.1]])
+    sched = _manual_schedule(cfg, idx, gate)
+    y, _ = O.forward_expert(cfg, inp, sched)
+    ref = np.zeros((3, 8))
+    ref[0, 2] = -0.3576087661   # 0.75 * SiLU(-2) * (2 * 0.5) * 2
+    ref[0, 6] = 2.1432917854    # 0.25 * SiLU(3) * (2 * -0.5) * -3
+    ref[1, 1] = -0.0711388098   # 0.5 * SiLU(-3) * (1 * 1) * 1
+    ref[1, 5] = 1.7779997999    # 0.5 * SiLU(0.375) * (1 * 4) * 4
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-9)
+    yt, _ = O.forward_token(cfg, inp, idx, gate)
+    np.testing.assert_allclose(yt, ref, rtol=0, atol=1e-9)
+
+
+def test_gated_expert_with_a_unit_gate_is_the_plain_expert():
+    """A constant feature x[:, 0] = 1 and U[e] = e_0 make x . U[e] = 1 for every
+    task: the gated expert reduces to the plain one (both orders)."""
+    cfg = WL.TINY.with_(L=40)
+    h = WL.make_inputs(cfg)
+    x = WL.bf16_bits_to_f32(h["x"]) if cfg.dtype == WL.BF16 else h["x"].copy()
+    x[:, 0] = 1.0
+    U = np.zeros((cfg.N, cfg.d), np.float32)
+    U[:, 0] = 1.0
+    inp = dict(h, x=x.astype(np.float32))
+    idx, gate, _ = O.route(cfg, inp)
+    sched = O.schedule(cfg, idx, gate)
+    y_plain, _ = O.forward_expert(cfg, inp, sched)
+    y_glu, _ = O.forward_expert(cfg, dict(inp, U=U), sched)
+    np.testing.assert_allclose(y_glu, y_plain, rtol=1e-12, atol=1e-14)
+    yt, _ = O.forward_token(cfg, dict(inp, U=U), idx, gate)
+    np.testing.assert_allclose(yt, y_plain, rtol=1e-12, atol=1e-14)
+
+
+def test_gated_expert_linear_in_U_and_orders_agree():
+    cfg = WL.TINY.with_(L=48)
+    h = WL.make_inputs(cfg)
+    rng = np.random.default_rng(8)
+    U = (rng.integers(-8, 9, (cfg.N, cfg.d)) / 64).astype(np.float32)  # dyadic: 3U exact
+    idx, gate, _ = O.route(cfg, h)
+    sched = O.schedule(cfg, idx, gate)
+    y1, _ = O.forward_expert(cfg, dict(h, U=U), sched)
+    y3, _ = O.forward_expert(cfg, dict(h, U=(3 * U).astype(np.float32)), sched)
+    np.testing.assert_allclose(y3, 3 * y1, rtol=1e-12, atol=1e-13)
+    yt, _ = O.forward_token(cfg, dict(h, U=U), idx, gate)
+    np.testing.assert_allclose(yt, y1, rtol=1e-12, atol=1e-13)
+    assert np.abs(y1).max() > 0
