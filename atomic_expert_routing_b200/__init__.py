@@ -102,18 +102,19 @@ def _expect(name, t, n, dtype, *, optional=False):
 
 
 def _expect_io(D, **ts):
-    """Checks by argument name: storage-type tensors (x, W, V, Wr, Wc, y),
+    """Checks by argument name: storage-type tensors (x, W, U, V, Wr, Wc, y),
     fp32 biases and logits, int32 counts."""
     f32, i32 = torch.float32, torch.int32
     spec = {
         "x": (D.L * D.d, D.torch_dtype), "y": (D.L * D.d, D.torch_dtype),
         "Wr": (D.Nr * D.d, D.torch_dtype), "Wc": (D.Nc * D.d, D.torch_dtype),
         "W": (D.N * D.d, D.torch_dtype), "V": (D.N * D.d, D.torch_dtype),
+        "U": (D.N * D.d, D.torch_dtype),
         "bias_r": (D.Nr, f32), "bias_c": (D.Nc, f32),
         "logits": (D.L * (D.Nr + D.Nc), f32), "counts": (4, i32),
         "idx": (D.M, i32), "gate": (D.M, f32),
     }
-    optional = {"bias_r", "bias_c", "counts", "y", "idx", "gate"}
+    optional = {"bias_r", "bias_c", "counts", "y", "idx", "gate", "U"}
     for name, t in ts.items():
         n, dt = spec[name]
         _expect(name, t, n, dt, optional=name in optional)
@@ -237,17 +238,28 @@ def schedule(D: LayerDims, idx, gate, *, counts=None, ws=None, stream=None) -> d
     return out
 
 
-def expert_forward(D: LayerDims, x, W, V, sched: dict, *, y=None, ws=None, stream=None):
-    """Grouped (expert-centric) execution of a schedule; returns y [L, d]."""
-    _expect_io(D, x=x, W=W, V=V, y=y)
+def _weights(fn, W, U, V):
+    """The entry point and the expert-weight pointers: the plain expert
+    (W, V), or with U the gated one, h = SiLU(x.W[e]) * (x.U[e])."""
+    if U is None:
+        return fn, (_ptr(W), _ptr(V))
+    return fn + "_glu", (_ptr(W), _ptr(U), _ptr(V))
+
+
+def expert_forward(D: LayerDims, x, W, V, sched: dict, *, U=None, y=None, ws=None,
+                   stream=None):
+    """Grouped (expert-centric) execution of a schedule; returns y [L, d].
+    U [N, d] (optional): the gate matrix of gated (SwiGLU) experts."""
+    _expect_io(D, x=x, W=W, U=U, V=V, y=y)
     _expect_sched(D, sched)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
     wsp, n = _ws(D, OMNI_WS_EXPERT, dev, ws)
     dd = D.c()
-    _lib.check("omni_expert_forward", _lib.load().omni_expert_forward(
-        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(sched["task_token"]),
+    fn, wts = _weights("omni_expert_forward", W, U, V)
+    _lib.check(fn, getattr(_lib.load(), fn)(
+        C.byref(dd), _ptr(x), *wts, _ptr(sched["task_token"]),
         _ptr(sched["task_expert"]), _ptr(sched["task_gate"]), _ptr(sched["uniq"]),
         _ptr(sched["group_off"]), _ptr(sched["counts"]), _ptr(y), wsp, n, _stream(stream)))
     return y
@@ -274,10 +286,11 @@ def expert_forward_noalloc(D: LayerDims, x, W, V, sched: dict, *, y=None, stream
     return y
 
 
-def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=None,
+def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, U=None, y=None,
                 counts=None, idx=None, gate=None, ws=None, stream=None):
-    """Route -> schedule -> grouped execution in one call; returns y [L, d]."""
-    _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, V=V, bias_r=bias_r, bias_c=bias_c, y=y,
+    """Route -> schedule -> grouped execution in one call; returns y [L, d].
+    U [N, d] (optional): the gate matrix of gated (SwiGLU) experts."""
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, U=U, V=V, bias_r=bias_r, bias_c=bias_c, y=y,
                counts=counts, idx=idx, gate=gate)
     dev = _device(x)
     if y is None:
@@ -286,8 +299,9 @@ def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, y=No
         counts = new_counts(dev)
     wsp, n = _ws(D, OMNI_WS_FUSED, dev, ws)
     dd = D.c()
-    _lib.check("omni_moe_forward", _lib.load().omni_moe_forward(
-        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c), _ptr(W), _ptr(V),
+    fn, wts = _weights("omni_moe_forward", W, U, V)
+    _lib.check(fn, getattr(_lib.load(), fn)(
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c), *wts,
         _ptr(y), _ptr(idx), _ptr(gate), _ptr(counts), wsp, n, _stream(stream)))
     return y
 
@@ -347,18 +361,20 @@ def moe_mlp_forward(D: LayerDims, x, Wr, Wc, W, V, W1, W2, bias_r=None, bias_c=N
     return y
 
 
-def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, y=None, counts=None,
+def token_centric_forward(D: LayerDims, x, W, V, idx, gate, *, U=None, y=None, counts=None,
                           stream=None):
-    """Token-centric execution (ablation): every token gathers its own experts."""
-    _expect_io(D, x=x, W=W, V=V, y=y, counts=counts)
+    """Token-centric execution (ablation): every token gathers its own experts.
+    U [N, d] (optional): the gate matrix of gated (SwiGLU) experts."""
+    _expect_io(D, x=x, W=W, U=U, V=V, y=y, counts=counts)
     _expect("idx", idx, D.M, torch.int32)
     _expect("gate", gate, D.M, torch.float32)
     dev = _device(x)
     if y is None:
         y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=dev)
     dd = D.c()
-    _lib.check("omni_token_centric_forward", _lib.load().omni_token_centric_forward(
-        C.byref(dd), _ptr(x), _ptr(W), _ptr(V), _ptr(idx), _ptr(gate), _ptr(y), _ptr(counts),
+    fn, wts = _weights("omni_token_centric_forward", W, U, V)
+    _lib.check(fn, getattr(_lib.load(), fn)(
+        C.byref(dd), _ptr(x), *wts, _ptr(idx), _ptr(gate), _ptr(y), _ptr(counts),
         None, 0, _stream(stream)))
     return y
 

@@ -159,6 +159,43 @@ bool tensors_ok(const void* const* p16, int n16) {
   return true;
 }
 
+// The staged grouped execution, plain or gated (then U is checked like the
+// other tensors).
+int expert_forward_impl(const omni_dims* dims, bool gated, const void* x, const void* W,
+                        const void* U, const void* V, const int32_t* task_token,
+                        const int32_t* task_expert, const float* task_gate, const int32_t* uniq,
+                        const int32_t* group_off, int32_t* counts, void* y, void* ws,
+                        size_t ws_bytes, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W, V, y, gated ? U : x};
+  if (!tensors_ok(t16, 5) || task_token == nullptr || task_expert == nullptr ||
+      task_gate == nullptr || group_off == nullptr || counts == nullptr)
+    return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_EXPERT, ws, ws_bytes)) != OMNI_OK) return rc;
+  return cuda_status(omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate, uniq,
+                                         group_off, counts, y, ws,
+                                         static_cast<cudaStream_t>(stream), false, true,
+                                         gated ? U : nullptr));
+}
+
+// The token-centric ablation, plain or gated.
+int token_forward_impl(const omni_dims* dims, bool gated, const void* x, const void* W,
+                       const void* U, const void* V, const int32_t* idx, const float* gate,
+                       void* y, int32_t* counts, void* stream) {
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W, V, y, gated ? U : x};
+  if (!tensors_ok(t16, 5) || idx == nullptr || gate == nullptr) return OMNI_ERR_INVALID_ARG;
+  return cuda_status(omni::launch_token(D, x, W, V, idx, gate, y, counts ? counts + 2 : nullptr,
+                                        static_cast<cudaStream_t>(stream),
+                                        gated ? U : nullptr));
+}
+
 }  // namespace
 
 extern "C" {
@@ -277,18 +314,17 @@ int omni_expert_forward(const omni_dims* dims, const void* x, const void* W, con
                         const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                         int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream) {
   omni::CallRange range("omni_expert_forward");
-  Dims D;
-  int rc = check_dims(dims, &D);
-  if (rc != OMNI_OK) return rc;
-  if (D.L == 0) return OMNI_OK;
-  const void* t16[] = {x, W, V, y};
-  if (!tensors_ok(t16, 4) || task_token == nullptr || task_expert == nullptr ||
-      task_gate == nullptr || group_off == nullptr || counts == nullptr)
-    return OMNI_ERR_INVALID_ARG;
-  if ((rc = ws_ok(D, OMNI_WS_EXPERT, ws, ws_bytes)) != OMNI_OK) return rc;
-  return cuda_status(omni::launch_expert(D, x, W, V, task_token, task_expert, task_gate, uniq,
-                                         group_off, counts, y, ws,
-                                         static_cast<cudaStream_t>(stream)));
+  return expert_forward_impl(dims, false, x, W, nullptr, V, task_token, task_expert, task_gate, uniq,
+                             group_off, counts, y, ws, ws_bytes, stream);
+}
+
+int omni_expert_forward_glu(const omni_dims* dims, const void* x, const void* W, const void* U,
+                            const void* V, const int32_t* task_token, const int32_t* task_expert,
+                            const float* task_gate, const int32_t* uniq, const int32_t* group_off,
+                            int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_expert_forward_glu");
+  return expert_forward_impl(dims, true, x, W, U, V, task_token, task_expert, task_gate, uniq,
+                             group_off, counts, y, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -299,7 +335,7 @@ namespace {
 int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* Wc,
                      const float* bias_r, const float* bias_c, const void* W, const void* V,
                      void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
-                     cudaStream_t s) {
+                     cudaStream_t s, const void* U = nullptr) {
   int rc = OMNI_OK;
   Carver c(ws);
   FusedWs w = carve_fused(D, c);
@@ -328,7 +364,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
         (rc = cuda_status(omni::launch_zero(zero, static_cast<size_t>(zero_words), s))) != OMNI_OK)
       return rc;
     return cuda_status(omni::launch_sched_exec(D, x, W, V, idx, gate, y,
-                                               static_cast<uint32_t*>(w.expert), counts, s));
+                                               static_cast<uint32_t*>(w.expert), counts, s, U));
   }
   if (fused_windows(D)) {
     {
@@ -339,7 +375,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
     }
     if (rc != OMNI_OK) return rc;
     omni::CallRange stage("expert");
-    return cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s));
+    return cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s, U));
   }
   {
     omni::CallRange stage("schedule");
@@ -349,7 +385,8 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   if (rc != OMNI_OK) return rc;
   omni::CallRange stage("expert");
   return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
-                                         w.uniq, w.group_off, counts, y, w.expert, s, acc_zeroed));
+                                         w.uniq, w.group_off, counts, y, w.expert, s, acc_zeroed,
+                                         true, U));
 }
 
 // The checks of the shared MLP's width: F >= 1; a multiple of 8 (16-byte
@@ -446,14 +483,34 @@ int omni_token_centric_forward(const omni_dims* dims, const void* x, const void*
   omni::CallRange range("omni_token_centric_forward");
   (void)ws;
   (void)ws_bytes;
+  return token_forward_impl(dims, false, x, W, nullptr, V, idx, gate, y, counts, stream);
+}
+
+int omni_token_centric_forward_glu(const omni_dims* dims, const void* x, const void* W,
+                                   const void* U, const void* V, const int32_t* idx,
+                                   const float* gate, void* y, int32_t* counts, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_token_centric_forward_glu");
+  (void)ws;
+  (void)ws_bytes;
+  return token_forward_impl(dims, true, x, W, U, V, idx, gate, y, counts, stream);
+}
+
+int omni_moe_forward_glu(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                         const float* bias_r, const float* bias_c, const void* W, const void* U,
+                         const void* V, void* y, int32_t* idx_out, float* gate_out,
+                         int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_forward_glu");
   Dims D;
-  int rc = check_dims(dims, &D);
+  int rc = check_route_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
+  if (counts == nullptr) return OMNI_ERR_INVALID_ARG;
   if (D.L == 0) return OMNI_OK;
-  const void* t16[] = {x, W, V, y};
-  if (!tensors_ok(t16, 4) || idx == nullptr || gate == nullptr) return OMNI_ERR_INVALID_ARG;
-  return cuda_status(omni::launch_token(D, x, W, V, idx, gate, y, counts ? counts + 2 : nullptr,
-                                        static_cast<cudaStream_t>(stream)));
+  const void* t16[] = {x, Wr, Wc, W, U, V, y};
+  if (!tensors_ok(t16, 7)) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
+  return moe_forward_impl(D, x, Wr, Wc, bias_r, bias_c, W, V, y, idx_out, gate_out, counts, ws,
+                          static_cast<cudaStream_t>(stream), U);
 }
 
 }  // extern "C"

@@ -104,8 +104,8 @@ __device__ __forceinline__ uint4 pack_vec(const float* a, float*) {
 // warp-uniform points.
 template <typename T, int NV>
 __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
-    k_expert_slices(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
-                    const int32_t* __restrict__ task_token,
+    k_expert_slices(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
+                    const T* __restrict__ V, const int32_t* __restrict__ task_token,
                     const int32_t* __restrict__ task_expert,
                     const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
                     int S, float* __restrict__ yacc, int32_t* status) {
@@ -163,7 +163,14 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
 #pragma unroll
         for (int v = 0; v < NV; ++v) s += dot_vec(xv[v], wv[v], static_cast<T*>(nullptr));
         s = warp_sum(s);
-        const float c = gj * silu(s);
+        float c = gj * silu(s);
+        if (U != nullptr) {  // gated expert: times x[t] . U[e]
+          const uint4* ur = reinterpret_cast<const uint4*>(U + e * d);
+          float su = 0.0f;
+#pragma unroll
+          for (int v = 0; v < NV; ++v) su += dot_vec(xv[v], ur[v * 32 + lane], static_cast<T*>(nullptr));
+          c *= warp_sum(su);
+        }
 #pragma unroll
         for (int v = 0; v < NV; ++v) axpy_vec(c, vv[v], acc + v * EPV, static_cast<T*>(nullptr));
       }
@@ -182,14 +189,19 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
       float my_c = 0.0f;
       for (int j = p; j < q; ++j) {
         const int64_t e = __shfl_sync(0xffffffffu, my_e, j);
-        float sacc = 0.0f;
+        float sacc = 0.0f, uacc = 0.0f;
         if (e >= 0) {  // warp-uniform; no shuffle inside
           const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
           for (int v = lane; v < nvec; v += 32) sacc += dot_vec(xr[v], wr[v], static_cast<T*>(nullptr));
+          if (U != nullptr) {
+            const uint4* ur = reinterpret_cast<const uint4*>(U + e * d);
+            for (int v = lane; v < nvec; v += 32) uacc += dot_vec(xr[v], ur[v], static_cast<T*>(nullptr));
+          }
         }
         sacc = warp_sum(sacc);
+        uacc = warp_sum(uacc);
         const float gj = __shfl_sync(0xffffffffu, my_g, j);
-        if (lane == j) my_c = (e >= 0) ? gj * silu(sacc) : 0.0f;
+        if (lane == j) my_c = (e >= 0) ? gj * silu(sacc) * (U != nullptr ? uacc : 1.0f) : 0.0f;
       }
       for (int v0 = 0; v0 < nvec; v0 += 32) {
         const int v = v0 + lane;
@@ -268,10 +280,12 @@ constexpr int kAsyncWarps = 8;
 // from shared memory.  Warps run a grid-stride loop over task slices; the
 // pipeline restarts at every slice.  With dense != nullptr, a task with
 // dense[a] set takes its activation c from cpre[a] (formed on the tensor
-// cores) and fetches only its V row.
-template <typename T, int NV, int R>
+// cores) and fetches only its V row.  GLU: gated experts, c also times
+// x[t] . U[e]; a ring slot then holds the U row after the W and V rows.
+template <typename T, int NV, int R, bool GLU>
 __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
-    k_expert_async(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
+    k_expert_async(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
+                   const T* __restrict__ V,
                    const int32_t* __restrict__ task_token,
                    const int32_t* __restrict__ task_expert,
                    const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
@@ -280,7 +294,7 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
   pdl_wait();
   pdl_trigger();
   constexpr int EPV = kEpv<T>;
-  constexpr int SLOT = 2 * NV * 32;  // uint4 per ring slot: W vectors, then V vectors
+  constexpr int SLOT = (GLU ? 3 : 2) * NV * 32;  // uint4 per ring slot: W, V (, U) vectors
   extern __shared__ __align__(16) uint4 ring[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint4* wring = ring + static_cast<size_t>(warp) * R * SLOT;
@@ -331,6 +345,9 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
                          pol_stream);
             cp_async16(base + static_cast<uint32_t>((NV + v) * 32 + lane) * 16u, vr + v * 32 + lane,
                        pol_stream);
+            if constexpr (GLU)
+              cp_async16(base + static_cast<uint32_t>((2 * NV + v) * 32 + lane) * 16u,
+                         reinterpret_cast<const uint4*>(U + e * d) + v * 32 + lane, pol_stream);
           }
         }
       }
@@ -381,6 +398,13 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
             sdot += dot_vec(xc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
           sdot = warp_sum(sdot);
           c = gj * silu(sdot);
+          if constexpr (GLU) {
+            float su = 0.0f;
+#pragma unroll
+            for (int v = 0; v < NV; ++v)
+              su += dot_vec(xc[v], slot[(2 * NV + v) * 32 + lane], static_cast<T*>(nullptr));
+            c *= warp_sum(su);
+          }
         }
 #pragma unroll
         for (int v = 0; v < NV; ++v)
@@ -426,15 +450,16 @@ constexpr int kActWarps = 8;
 // rows are re-read by later tasks (x by token) -- keep them in L2
 // (evict-last) and read the F rows, each fetched once, evict-first.  dst ==
 // nullptr writes c[a].  Indices are range-checked (OMNI_DEV_BAD_INDEX; the
-// task gets c = 0).
-template <typename T, int NV, int R, bool HOLD_KEEP>
-__global__ void __launch_bounds__(kActWarps * 32, 2)
+// task gets c = 0).  GLU: gated experts, c also times H[h] . G[f]; a ring
+// slot then holds the row of G after the row of F (one CTA per SM).
+template <typename T, int NV, int R, bool HOLD_KEEP, bool GLU>
+__global__ void __launch_bounds__(kActWarps * 32, GLU ? 1 : 2)
     k_act(const T* __restrict__ H, const int32_t* __restrict__ hidx, int64_t nh,
-          const T* __restrict__ F, const int32_t* __restrict__ fidx, int64_t nf,
-          const float* __restrict__ task_gate, const int32_t* __restrict__ dst, int64_t M, int d,
-          int S, int64_t nslices, float* __restrict__ cbuf, int32_t* status) {
+          const T* __restrict__ F, const T* __restrict__ G, const int32_t* __restrict__ fidx,
+          int64_t nf, const float* __restrict__ task_gate, const int32_t* __restrict__ dst,
+          int64_t M, int d, int S, int64_t nslices, float* __restrict__ cbuf, int32_t* status) {
   pdl_wait();
-  constexpr int SLOT = NV * 32;  // uint4 per ring slot: one row of F
+  constexpr int SLOT = (GLU ? 2 : 1) * NV * 32;  // uint4 per ring slot: a row of F (and of G)
   extern __shared__ __align__(16) uint4 ring[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint4* fring = ring + static_cast<size_t>(warp) * R * SLOT;
@@ -481,6 +506,9 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
               cp_async16(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane, pol_once);
             else
               cp_async16_plain(base + static_cast<uint32_t>(v * 32 + lane) * 16u, fr + v * 32 + lane);
+            if constexpr (GLU)
+              cp_async16(base + static_cast<uint32_t>((NV + v) * 32 + lane) * 16u,
+                         reinterpret_cast<const uint4*>(G + f * d) + v * 32 + lane, pol_once);
           }
         }
       }
@@ -517,7 +545,15 @@ __global__ void __launch_bounds__(kActWarps * 32, 2)
 #pragma unroll
         for (int v = 0; v < NV; ++v) sdot += dot_vec(hc[v], slot[v * 32 + lane], static_cast<T*>(nullptr));
         sdot = warp_sum(sdot);
-        if (lane == j) my_c = gj * silu(sdot);
+        float cj = gj * silu(sdot);
+        if constexpr (GLU) {
+          float su = 0.0f;
+#pragma unroll
+          for (int v = 0; v < NV; ++v)
+            su += dot_vec(hc[v], slot[(NV + v) * 32 + lane], static_cast<T*>(nullptr));
+          cj *= warp_sum(su);
+        }
+        if (lane == j) my_c = cj;
       }
     }
     cp_async_wait<0>();
@@ -1005,7 +1041,8 @@ constexpr int kTokThreads = 128;
 // c_q * V[e_q] over the K tasks.  No reductions across CTAs.
 template <typename T>
 __global__ void __launch_bounds__(kTokThreads)
-    k_token_centric(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ V,
+    k_token_centric(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
+                    const T* __restrict__ V,
                     const int32_t* __restrict__ idx, const float* __restrict__ gate, int K, int d,
                     int64_t N, T* __restrict__ y, int32_t* status) {
   pdl_wait();
@@ -1031,13 +1068,19 @@ __global__ void __launch_bounds__(kTokThreads)
   __syncthreads();
   for (int q = warp; q < K; q += kTokThreads / 32) {
     const int64_t e = es[q];
-    float s = 0.0f;
+    float s = 0.0f, su = 0.0f;
     if (e >= 0) {
       const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
       for (int v = lane; v < nvec; v += 32) s += dot_vec(xs[v], wr[v], static_cast<T*>(nullptr));
+      if (U != nullptr) {  // gated expert: times x[t] . U[e]
+        const uint4* ur = reinterpret_cast<const uint4*>(U + e * d);
+        for (int v = lane; v < nvec; v += 32) su += dot_vec(xs[v], ur[v], static_cast<T*>(nullptr));
+      }
     }
     s = warp_sum(s);
-    if (lane == 0) cq[q] = (e >= 0) ? gate[t * K + q] * silu(s) : 0.0f;
+    su = warp_sum(su);
+    if (lane == 0)
+      cq[q] = (e >= 0) ? gate[t * K + q] * silu(s) * (U != nullptr ? su : 1.0f) : 0.0f;
   }
   __syncthreads();
   uint4* yr = reinterpret_cast<uint4*>(y + t * d);
@@ -1128,7 +1171,7 @@ size_t expert_ws_bytes(const Dims& D) {
 template <typename T, int NV>
 cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const void* V,
                           const int32_t* tt, const int32_t* te, const float* tg, float* acc,
-                          int32_t* status, cudaStream_t s) {
+                          int32_t* status, cudaStream_t s, const void* U) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1140,17 +1183,18 @@ cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const voi
   const int64_t warps = (M + S - 1) / S;
   const int64_t blocks = (warps + kExpThreads / 32 - 1) / (kExpThreads / 32);
   OMNI_TRY(launch_k(k_expert_slices<T, NV>, static_cast<unsigned>(blocks), kExpThreads, 0, s,
-      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg, M,
+      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U),
+      static_cast<const T*>(V), tt, te, tg, M,
       D.L, D.N(), static_cast<int>(D.d), S, acc, status));
   return cudaGetLastError();
 }
 
-template <typename T, int NV, int R>
+template <typename T, int NV, int R, bool GLU>
 cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* tt, const int32_t* te, const float* tg, float* acc,
-                         int32_t* status, cudaStream_t s, const DenseFlags& df) {
-  constexpr size_t smem = static_cast<size_t>(kAsyncWarps) * R * 2 * NV * 32 * 16;
-  cudaError_t err = cudaFuncSetAttribute(k_expert_async<T, NV, R>,
+                         int32_t* status, cudaStream_t s, const DenseFlags& df, const void* U) {
+  constexpr size_t smem = static_cast<size_t>(kAsyncWarps) * R * (GLU ? 3 : 2) * NV * 32 * 16;
+  cudaError_t err = cudaFuncSetAttribute(k_expert_async<T, NV, R, GLU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -1164,8 +1208,9 @@ cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void
   const int64_t nslices = (M + S - 1) / S;
   int64_t blocks = (nslices + kAsyncWarps - 1) / kAsyncWarps;
   if (blocks > sms) blocks = sms;  // persistent: one CTA per SM (shared-memory bound)
-  OMNI_TRY(launch_k(k_expert_async<T, NV, R>, static_cast<unsigned>(blocks), kAsyncWarps * 32, smem,
-      s, static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(V), tt, te, tg,
+  OMNI_TRY(launch_k(k_expert_async<T, NV, R, GLU>, static_cast<unsigned>(blocks), kAsyncWarps * 32,
+      smem, s, static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U),
+      static_cast<const T*>(V), tt, te, tg,
       M, D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status, df.flag, df.cbuf));
   return cudaGetLastError();
 }
@@ -1173,17 +1218,30 @@ cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void
 // df: the dense-group activations (flag == nullptr: none).  Row widths
 // without a k_expert_async instance take k_expert_slices, which forms every
 // activation itself; the dense path is only run for widths that have one.
+// U != nullptr: gated experts (a third row per task; fewer ring slots at the
+// widest rows so that the ring still fits the shared memory).
 template <typename T>
 cudaError_t dispatch_slices(const Dims& D, const void* x, const void* W, const void* V,
                             const int32_t* tt, const int32_t* te, const float* tg, float* acc,
-                            int32_t* status, cudaStream_t s, const DenseFlags& df) {
+                            int32_t* status, cudaStream_t s, const DenseFlags& df,
+                            const void* U) {
   constexpr int row = 32 * kEpv<T>;  // elements covered by one vector per lane
-  switch (D.d == row * 8 ? 8 : D.d == row * 4 ? 4 : D.d == row * 2 ? 2 : D.d == row ? 1 : 0) {
-    case 8: return launch_async<T, 8, 3>(D, x, W, V, tt, te, tg, acc, status, s, df);
-    case 4: return launch_async<T, 4, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
-    case 2: return launch_async<T, 2, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
-    case 1: return launch_async<T, 1, 4>(D, x, W, V, tt, te, tg, acc, status, s, df);
-    default: return launch_slices<T, 0>(D, x, W, V, tt, te, tg, acc, status, s);
+  const int nv = D.d == row * 8 ? 8 : D.d == row * 4 ? 4 : D.d == row * 2 ? 2 : D.d == row ? 1 : 0;
+  if (U != nullptr) {
+    switch (nv) {
+      case 8: return launch_async<T, 8, 2, true>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+      case 4: return launch_async<T, 4, 3, true>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+      case 2: return launch_async<T, 2, 4, true>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+      case 1: return launch_async<T, 1, 4, true>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+      default: return launch_slices<T, 0>(D, x, W, V, tt, te, tg, acc, status, s, U);
+    }
+  }
+  switch (nv) {
+    case 8: return launch_async<T, 8, 3, false>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+    case 4: return launch_async<T, 4, 4, false>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+    case 2: return launch_async<T, 2, 4, false>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+    case 1: return launch_async<T, 1, 4, false>(D, x, W, V, tt, te, tg, acc, status, s, df, U);
+    default: return launch_slices<T, 0>(D, x, W, V, tt, te, tg, acc, status, s, U);
   }
 }
 
@@ -1270,7 +1328,7 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
                       const int32_t* tt, const int32_t* te, const float* tg,
                       const int32_t* group_off, const int32_t* counts, const SweepWs& w,
                       const int32_t* win_lo, float* acc, __nv_bfloat16* ycast, int32_t* status,
-                      cudaStream_t s) {
+                      cudaStream_t s, const void* U) {
   const int cols = static_cast<int>(D.d / Q);
   // bf16: one compact fp32 slice [L x cols] serves every sweep -- zeroed
   // before the first, then rounded into y's columns and zeroed in place
@@ -1283,22 +1341,28 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
                                  status, s);
   if (err != cudaSuccess) return err;
   // three ring slots per warp: two rows in flight, two CTAs (16 warps) per SM
+  // (gated experts: a W and a U row per slot, one CTA per SM)
   constexpr int R = 3;
-  constexpr size_t smem = static_cast<size_t>(kActWarps) * R * NV * 32 * 16;
-  err = cudaFuncSetAttribute(k_act<T, NV, R, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
   const int64_t M = D.M();
   const int S = 32;
   const int64_t nslices = (M + S - 1) / S;
   int64_t blocks = (nslices + kActWarps - 1) / kActWarps;
-  if (blocks > 2 * sm_count()) blocks = 2 * sm_count();
   // tasks by expert: x[t] held per run of one token, the W rows through the
   // ring (an expert's repeated row comes from L2 right after its first read)
-  OMNI_TRY(launch_k(k_act<T, NV, R, true>, static_cast<unsigned>(blocks), kActWarps * 32, smem, s,
-      static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W), w.win.xe, D.N(), w.win.xg,
-      w.win.xdst, M, static_cast<int>(D.d), S, nslices, w.cbuf, status));
-  err = cudaGetLastError();
+  auto act = [&](auto kernel, int per_sm, size_t smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int64_t b = blocks > per_sm * sm_count() ? per_sm * sm_count() : blocks;
+    OMNI_TRY(launch_k(kernel, static_cast<unsigned>(b), kActWarps * 32, smem, s,
+        static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W),
+        static_cast<const T*>(U), w.win.xe, D.N(), w.win.xg, w.win.xdst, M,
+        static_cast<int>(D.d), S, nslices, w.cbuf, status));
+    return cudaGetLastError();
+  };
+  err = U != nullptr
+            ? act(k_act<T, NV, R, true, true>, 1, static_cast<size_t>(kActWarps) * R * 2 * NV * 32 * 16)
+            : act(k_act<T, NV, R, true, false>, 2, static_cast<size_t>(kActWarps) * R * NV * 32 * 16);
   if (err != cudaSuccess) return err;
   // 128-column blocks per slice and the prefetch distance (about 16 vectors
   // of loads in flight per lane)
@@ -1319,7 +1383,7 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
                           const int32_t* tt, const int32_t* te, const float* tg,
                           const int32_t* group_off, const int32_t* counts, const SweepWs& w,
                           const int32_t* win_lo, float* acc, __nv_bfloat16* ycast,
-                          int32_t* status, cudaStream_t s) {
+                          int32_t* status, cudaStream_t s, const void* U) {
   constexpr int row = 32 * kEpv<T>;
   const int64_t nv = D.d / row;             // vectors per lane for a whole row
   const int64_t nvq = (D.d / Q) / row;      // ... for one slice
@@ -1327,7 +1391,7 @@ cudaError_t launch_sweeps(const Dims& D, int Q, const void* x, const void* W, co
 #define OMNI_SWEEP(NV_, NVQ_)                                                               \
   if (nv == NV_ && nvq == NVQ_)                                                             \
     return sweeps_nv<T, NV_, NVQ_>(D, Q, x, W, V, tt, te, tg, group_off, counts, w, win_lo, \
-                                   acc, ycast, status, s);
+                                   acc, ycast, status, s, U);
   OMNI_SWEEP(8, 4) OMNI_SWEEP(8, 2) OMNI_SWEEP(8, 1) OMNI_SWEEP(4, 2) OMNI_SWEEP(4, 1)
   OMNI_SWEEP(2, 1)
 #undef OMNI_SWEEP
@@ -1338,7 +1402,7 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                           const int32_t* counts, void* y, void* ws, cudaStream_t s,
-                          bool acc_zeroed, bool allow_dense) {
+                          bool acc_zeroed, bool allow_dense, const void* U) {
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
   float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
@@ -1348,25 +1412,25 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
     const SweepWs w = carve_sweeps(D, ws, nullptr);
     __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
     return f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate,
-                                      group_off, counts, w, nullptr, acc, ycast, status, s)
+                                      group_off, counts, w, nullptr, acc, ycast, status, s, U)
                : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
                                               group_off, counts, w, nullptr, acc, ycast, status,
-                                              s);
+                                              s, U);
   }
   cudaError_t err = acc_zeroed ? cudaSuccess
                                : launch_zero(acc, static_cast<size_t>(expert_acc_words(D)), s);
   if (err != cudaSuccess) return err;
   DenseFlags df{nullptr, nullptr};
-  if (allow_dense && uniq != nullptr && dense_path(D)) {
+  if (allow_dense && U == nullptr && uniq != nullptr && dense_path(D)) {
     void* dws = static_cast<char*>(ws) + dense_ws_offset(D);
     OMNI_TRY(launch_dense_activations(D, x, W, task_token, task_expert, task_gate, uniq,
                                       group_off, const_cast<int32_t*>(counts), dws, s));
     df = dense_flags(D, dws);
   }
   err = f32 ? dispatch_slices<float>(D, x, W, V, task_token, task_expert, task_gate, acc, status,
-                                     s, df)
+                                     s, df, U)
             : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
-                                             status, s, df);
+                                             status, s, df, U);
   if (err != cudaSuccess || f32) return err;
   const int64_t n = D.L * D.d;
   OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,
@@ -1384,7 +1448,8 @@ WinTasks expert_windows(const Dims& D, void* ws) {
 }
 
 cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, const void* V,
-                                  int32_t* counts, void* y, void* ws, cudaStream_t s) {
+                                  int32_t* counts, void* y, void* ws, cudaStream_t s,
+                                  const void* U) {
   const int Q = expert_sweeps(D);
   if (D.L == 0 || Q <= 1) return cudaErrorInvalidValue;
   const bool f32 = D.dtype == OMNI_F32;
@@ -1393,9 +1458,9 @@ cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, c
   const SweepWs w = carve_sweeps(D, ws, nullptr);
   __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
   return f32 ? launch_sweeps<float>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr, counts, w,
-                                    w.win_lo, acc, ycast, status, s)
+                                    w.win_lo, acc, ycast, status, s, U)
              : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr,
-                                            counts, w, w.win_lo, acc, ycast, status, s);
+                                            counts, w, w.win_lo, acc, ycast, status, s, U);
 }
 
 namespace {
@@ -1420,7 +1485,7 @@ cudaError_t launch_zero(void* p, size_t n_words, cudaStream_t s) {
 
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
-                         cudaStream_t s) {
+                         cudaStream_t s, const void* U) {
   if (D.L == 0) return cudaSuccess;
   const size_t esz = D.dtype == OMNI_F32 ? 4 : 2;
   const size_t smem = static_cast<size_t>(D.d) * esz +
@@ -1432,16 +1497,17 @@ cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     OMNI_TRY(launch_k(k_token_centric<float>, static_cast<unsigned>(D.L), kTokThreads, smem, s,
-        static_cast<const float*>(x), static_cast<const float*>(W), static_cast<const float*>(V),
-        idx, gate, static_cast<int>(D.K), static_cast<int>(D.d), D.N(), static_cast<float*>(y),
-        status));
+        static_cast<const float*>(x), static_cast<const float*>(W), static_cast<const float*>(U),
+        static_cast<const float*>(V), idx, gate, static_cast<int>(D.K), static_cast<int>(D.d),
+        D.N(), static_cast<float*>(y), status));
   } else {
     err = cudaFuncSetAttribute(k_token_centric<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     OMNI_TRY(launch_k(k_token_centric<__nv_bfloat16>, static_cast<unsigned>(D.L), kTokThreads, smem,
         s, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W),
-        static_cast<const __nv_bfloat16*>(V), idx, gate, static_cast<int>(D.K),
+        static_cast<const __nv_bfloat16*>(U), static_cast<const __nv_bfloat16*>(V), idx, gate,
+        static_cast<int>(D.K),
         static_cast<int>(D.d), D.N(), static_cast<__nv_bfloat16*>(y), status));
   }
   return cudaGetLastError();

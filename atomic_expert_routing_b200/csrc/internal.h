@@ -91,7 +91,7 @@ size_t sched_exec_ws_words(const Dims& D);
 // Writes y [L x d] completely, and counts[0], [1].
 cudaError_t launch_sched_exec(const Dims& D, const void* x, const void* W, const void* V,
                               const int32_t* idx, const float* gate, void* y, uint32_t* ws,
-                              int32_t* counts, cudaStream_t s);
+                              int32_t* counts, cudaStream_t s, const void* U = nullptr);
 
 // ---- activations of dense groups on the tensor cores ----------------------
 // bf16, d a multiple of 64, B <= 256.  The planner flags the tasks of dense
@@ -115,8 +115,10 @@ size_t expert_ws_bytes(const Dims& D);
 int expert_sweeps(const Dims& D);                // slices of d (1: no sweeps)
 WinTasks expert_windows(const Dims& D, void* ws);  // the window buffers of an expert workspace
 // The sweeps from tasks already in window token order (expert_windows(ws)).
+// U (nullable): the gate matrix of gated experts, h = SiLU(x.W[e]) * (x.U[e]).
 cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, const void* V,
-                                  int32_t* counts, void* y, void* ws, cudaStream_t s);
+                                  int32_t* counts, void* y, void* ws, cudaStream_t s,
+                                  const void* U = nullptr);
 // uniq: the schedule's U (the dense-group path reads it); allow_dense: run
 // the activations of dense groups on the tensor cores when the workspace is
 // the full OMNI_WS_EXPERT size (false: ws holds only the accumulator).
@@ -124,14 +126,15 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                           const int32_t* task_token, const int32_t* task_expert,
                           const float* task_gate, const int32_t* uniq, const int32_t* group_off,
                           const int32_t* counts, void* y, void* ws, cudaStream_t s,
-                          bool acc_zeroed = false, bool allow_dense = true);
+                          bool acc_zeroed = false, bool allow_dense = true,
+                          const void* U = nullptr);
 // The accumulator launch_expert clears before a batch without sweeps (its fp32
 // partial sums: y itself for fp32, else the head of ws), in floats; 0 for
 // batches with sweeps.
 int64_t expert_acc_words(const Dims& D);
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
-                         cudaStream_t s);
+                         cudaStream_t s, const void* U = nullptr);
 
 // ---- shared dense MLP: y (+)= SiLU(x W1^T) W2^T on the tensor cores ---------
 // bf16 storage only; ws holds the hidden activations H [L x F] (bf16).

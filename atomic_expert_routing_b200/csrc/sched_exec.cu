@@ -8,7 +8,8 @@
 // scatter-adding every task's d-vector into the few rows of y piles fp32
 // reductions onto the same lines.  Here:
 //
-// k_sched_act -- scheduling and the activations, split by expert id:
+// k_sched_act -- scheduling and the activations, split by expert id (gated
+// experts, with a gate matrix U: c also times x[t] . U[e]):
 //  1. The ids are cut into kSeTiles tiles of consecutive ids; kSeParts CTAs
 //     share a tile.  Every CTA of a tile reads the whole routing (L*K ids)
 //     and keeps the tasks whose expert lies in its tile; the tile's CTAs ask
@@ -103,10 +104,12 @@ struct SePlan {
 };
 
 // d = NV * 32 * (16 / sizeof(T)): every lane holds NV 16-byte vectors of a row.
-// Every phase issues its global loads before it uses any of them.
-template <typename T, int NV>
+// Every phase issues its global loads before it uses any of them.  GLU: gated
+// experts, c also times x[t] . U[e].
+template <typename T, int NV, bool GLU>
 __global__ void __launch_bounds__(kSeThreads, 1)
-    k_sched_act(const T* __restrict__ x, const T* __restrict__ W, const int32_t* __restrict__ idx,
+    k_sched_act(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
+                const int32_t* __restrict__ idx,
                 const float* __restrict__ gate, int L, int K, int64_t N, int B, SePlan P,
                 float* __restrict__ cbuf, SeScratch sc, int32_t* __restrict__ counts) {
   constexpr int EPV = 16 / sizeof(T);
@@ -244,9 +247,10 @@ __global__ void __launch_bounds__(kSeThreads, 1)
   // (4) activations; warp w takes positions b0 + w, b0 + w + 16, ..., PAIR at
   // a time (their x and W rows loaded together; one at d = 256 vectors, which
   // fill the registers)
-  constexpr int PAIR = NV >= 8 ? 1 : 2;
+  constexpr int PAIR = (NV >= 8 || (GLU && NV >= 4)) ? 1 : 2;
+  constexpr int NU = GLU ? NV : 1;  // vectors of the U row held per lane
   for (int p0 = b0 + warp; p0 < b1; p0 += PAIR * kSeWarps) {
-    uint4 xv[PAIR][NV], wv[PAIR][NV];
+    uint4 xv[PAIR][NV], wv[PAIR][NV], uv[PAIR][NU];
     int ii[PAIR];
 #pragma unroll
     for (int r = 0; r < PAIR; ++r) {
@@ -263,6 +267,11 @@ __global__ void __launch_bounds__(kSeThreads, 1)
         xv[r][q] = xr[q * 32 + lane];
         wv[r][q] = wr[q * 32 + lane];
       }
+      if constexpr (GLU) {
+        const uint4* ur = reinterpret_cast<const uint4*>(U + e * d);
+#pragma unroll
+        for (int q = 0; q < NV; ++q) uv[r][q] = ur[q * 32 + lane];
+      }
     }
 #pragma unroll
     for (int r = 0; r < PAIR; ++r) {
@@ -271,7 +280,14 @@ __global__ void __launch_bounds__(kSeThreads, 1)
 #pragma unroll
       for (int q = 0; q < NV; ++q) sdot += dot16(xv[r][q], wv[r][q], static_cast<const T*>(nullptr));
       sdot = warp_sum(sdot);
-      if (lane == 0) cbuf[ii[r]] = gate[ii[r]] * silu(sdot);
+      float c = gate[ii[r]] * silu(sdot);
+      if constexpr (GLU) {
+        float su = 0.0f;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) su += dot16(xv[r][q], uv[r][q], static_cast<const T*>(nullptr));
+        c *= warp_sum(su);
+      }
+      if (lane == 0) cbuf[ii[r]] = c;
     }
   }
 }
@@ -365,11 +381,11 @@ bool se_plan(const Dims& D, SePlan* P) {
 // c [M] floats from the next 256-byte boundary
 constexpr size_t kSeCbufOff = 64;
 
-template <typename T, int NV>
+template <typename T, int NV, bool GLU>
 cudaError_t launch_se_t(const Dims& D, const SePlan& P, const void* x, const void* W,
                         const void* V, const int32_t* idx, const float* gate, void* y,
-                        uint32_t* ws, int32_t* counts, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_sched_act<T, NV>,
+                        uint32_t* ws, int32_t* counts, cudaStream_t s, const void* U) {
+  cudaError_t err = cudaFuncSetAttribute(k_sched_act<T, NV, GLU>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(P.smem));
   if (err != cudaSuccess) return err;
@@ -377,8 +393,9 @@ cudaError_t launch_se_t(const Dims& D, const SePlan& P, const void* x, const voi
   sc.uacc = ws;
   sc.tiles_done = ws + 1;
   float* cbuf = reinterpret_cast<float*>(ws + kSeCbufOff);
-  OMNI_TRY(launch_k(k_sched_act<T, NV>, kSeTiles * kSeParts, kSeThreads, P.smem, s,
-      static_cast<const T*>(x), static_cast<const T*>(W), idx, gate, static_cast<int>(D.L),
+  OMNI_TRY(launch_k(k_sched_act<T, NV, GLU>, kSeTiles * kSeParts, kSeThreads, P.smem, s,
+      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U), idx, gate,
+      static_cast<int>(D.L),
       static_cast<int>(D.K), D.N(), static_cast<int>(D.B), P, cbuf, sc, counts));
   // value rows: NS vectors per lane and CTA, 2 when the row has them
   constexpr int NS = NV < 2 ? NV : 2;
@@ -402,23 +419,28 @@ size_t sched_exec_ws_words(const Dims& D) { return kSeCbufOff + static_cast<size
 
 cudaError_t launch_sched_exec(const Dims& D, const void* x, const void* W, const void* V,
                               const int32_t* idx, const float* gate, void* y, uint32_t* ws,
-                              int32_t* counts, cudaStream_t s) {
+                              int32_t* counts, cudaStream_t s, const void* U) {
   SePlan P;
   if (!se_plan(D, &P)) return cudaErrorInvalidValue;
+#define OMNI_SE(T_, NV_)                                                                  \
+  return U != nullptr                                                                     \
+             ? launch_se_t<T_, NV_, true>(D, P, x, W, V, idx, gate, y, ws, counts, s, U)  \
+             : launch_se_t<T_, NV_, false>(D, P, x, W, V, idx, gate, y, ws, counts, s, U);
   if (D.dtype == OMNI_F32) {
     switch (se_nv(D)) {
-      case 1: return launch_se_t<float, 1>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-      case 2: return launch_se_t<float, 2>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-      case 4: return launch_se_t<float, 4>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-      default: return launch_se_t<float, 8>(D, P, x, W, V, idx, gate, y, ws, counts, s);
+      case 1: OMNI_SE(float, 1)
+      case 2: OMNI_SE(float, 2)
+      case 4: OMNI_SE(float, 4)
+      default: OMNI_SE(float, 8)
     }
   }
   switch (se_nv(D)) {
-    case 1: return launch_se_t<__nv_bfloat16, 1>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-    case 2: return launch_se_t<__nv_bfloat16, 2>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-    case 4: return launch_se_t<__nv_bfloat16, 4>(D, P, x, W, V, idx, gate, y, ws, counts, s);
-    default: return launch_se_t<__nv_bfloat16, 8>(D, P, x, W, V, idx, gate, y, ws, counts, s);
+    case 1: OMNI_SE(__nv_bfloat16, 1)
+    case 2: OMNI_SE(__nv_bfloat16, 2)
+    case 4: OMNI_SE(__nv_bfloat16, 4)
+    default: OMNI_SE(__nv_bfloat16, 8)
   }
+#undef OMNI_SE
 }
 
 }  // namespace omni

@@ -17,6 +17,8 @@
  *             no N-wide score vector.
  *   [MS sched]  same page, Expert-Centric Scheduling steps and the traffic
  *             model D = 2d*L*K (token-centric) vs 2d*|E_active|.
+ *   [MS expert] same page, Atomic Expert section: the expert's activation is
+ *             named as SwiGLU.
  *
  * Conventions for every call
  *   - All pointers are DEVICE pointers owned by the caller (except `dims`,
@@ -286,6 +288,32 @@ int omni_mlp_workspace_size(const omni_dims* dims, int64_t F, int with_routed, s
 int omni_token_centric_forward(const omni_dims* dims, const void* x, const void* W,
                                const void* V, const int32_t* idx, const float* gate, void* y,
                                int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Gated atomic experts (SwiGLU, named by [MS expert]; the pages give only the
+ * pair (w_in, w_out), and the gated form taken here adds a third global
+ * matrix U [N x d], row e the gate vector of expert e):
+ *   h = SiLU(x[t] . W[e]) * (x[t] . U[e]),  y[t] = sum gate * h * V[e].
+ * Each of the three calls below is its plain counterpart (same arguments,
+ * workspace, outputs, orders and error codes) with U added: U is a DEVICE
+ * pointer, the dtype of x, row-major [N x d], 16-byte aligned, checked like
+ * W and V (OMNI_ERR_INVALID_ARG if NULL or misaligned in a non-empty
+ * batch).  Expert-centric order
+ * loads each active expert's three rows once; the tensor-core activations of
+ * dense groups (OMNI_FLAG_DENSE_TENSOR_CORES) are not used for gated experts.
+ */
+int omni_moe_forward_glu(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                         const float* bias_r, const float* bias_c, const void* W, const void* U,
+                         const void* V, void* y, int32_t* idx_out, float* gate_out,
+                         int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+int omni_expert_forward_glu(const omni_dims* dims, const void* x, const void* W, const void* U,
+                            const void* V, const int32_t* task_token, const int32_t* task_expert,
+                            const float* task_gate, const int32_t* uniq, const int32_t* group_off,
+                            int32_t* counts, void* y, void* ws, size_t ws_bytes, void* stream);
+int omni_token_centric_forward_glu(const omni_dims* dims, const void* x, const void* W,
+                                   const void* U, const void* V, const int32_t* idx,
+                                   const float* gate, void* y, int32_t* counts, void* ws,
+                                   size_t ws_bytes, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* omni_status_string(int status);

@@ -233,3 +233,37 @@ def test_shared_mlp_host_checks(lib, F, dtype, code):
     assert rc == (code if code != _lib.OMNI_OK else _lib.OMNI_ERR_INVALID_ARG)
     rc = lib.omni_moe_mlp_forward(C.byref(D), F, *([fake] * 12), None, fake, 1 << 30, None)
     assert rc == (code if code != _lib.OMNI_OK else _lib.OMNI_ERR_INVALID_ARG)
+
+
+def test_gated_entries_check_U_like_the_other_tensors(lib):
+    """The gated (SwiGLU) calls take the plain calls' checks plus U: a null or
+    misaligned U is an invalid argument in a non-empty batch, an empty batch
+    is a no-op, and the selecting call refuses K > k first."""
+    D = _dims()
+    fake = C.c_void_p(4096)
+    odd = C.c_void_p(4096 + 4)
+    bad = _lib.OMNI_ERR_INVALID_ARG
+    for U in (None, odd):
+        # x, Wr, Wc, bias_r, bias_c, W, U, V, y, idx, gate, counts
+        args = [fake, fake, fake, None, None, fake, U, fake, fake, None, None, fake]
+        assert lib.omni_moe_forward_glu(C.byref(D), *args, fake, 1 << 30, None) == bad
+        # x, W, U, V, task_token, task_expert, task_gate, uniq, group_off, counts, y
+        args = [fake, fake, U] + [fake] * 8
+        assert lib.omni_expert_forward_glu(C.byref(D), *args, fake, 1 << 30, None) == bad
+        # x, W, U, V, idx, gate, y, counts
+        args = [fake, fake, U] + [fake] * 5
+        assert lib.omni_token_centric_forward_glu(C.byref(D), *args, None, 0, None) == bad
+    # a good U: the same stop as the plain calls (a null counts / task array)
+    assert lib.omni_moe_forward_glu(C.byref(D), *([fake] * 11), None, fake, 1 << 30,
+                                    None) == bad
+    assert lib.omni_expert_forward_glu(C.byref(D), *([fake] * 9), None, fake, fake, 1 << 30,
+                                       None) == bad
+    E = _dims(L=0)
+    assert lib.omni_expert_forward_glu(C.byref(E), *([None] * 11), None, 0, None) == _lib.OMNI_OK
+    assert lib.omni_token_centric_forward_glu(C.byref(E), *([None] * 8), None, 0,
+                                              None) == _lib.OMNI_OK
+    assert lib.omni_moe_forward_glu(C.byref(E), *([None] * 11), fake, None, 0,
+                                    None) == _lib.OMNI_OK
+    K6 = _dims(k=4, K=6)
+    assert lib.omni_moe_forward_glu(C.byref(K6), *([fake] * 12), fake, 1 << 30,
+                                    None) == _lib.OMNI_ERR_UNSUPPORTED

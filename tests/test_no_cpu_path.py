@@ -44,6 +44,10 @@ def _calls():
         "expert_forward_noalloc": lambda: omni.expert_forward_noalloc(D, x, W, V, sched),
         "moe_forward": lambda: omni.moe_forward(D, x, Wr, Wc, W, V),
         "token_centric_forward": lambda: omni.token_centric_forward(D, x, W, V, idx, gate),
+        "moe_forward-glu": lambda: omni.moe_forward(D, x, Wr, Wc, W, V, U=W),
+        "expert_forward-glu": lambda: omni.expert_forward(D, x, W, V, sched, U=W),
+        "token_centric_forward-glu":
+            lambda: omni.token_centric_forward(D, x, W, V, idx, gate, U=W),
         "wait_selftest": lambda: omni.wait_selftest(torch.zeros(4, dtype=torch.int32)),
     }
 
@@ -124,6 +128,10 @@ def _shrunk_calls():
          lambda: omni.moe_forward(D, x, Wr, Wc, W, V, counts=torch.zeros(3, dtype=torch.int32))),
         ("token_centric_forward", "gate",
          lambda: omni.token_centric_forward(D, x, W, V, idx, gate.double())),
+        ("moe_forward", "U", lambda: omni.moe_forward(D, x, Wr, Wc, W, V, U=W[:-1])),
+        ("expert_forward", "U", lambda: omni.expert_forward(D, x, W, V, sched, U=W.half())),
+        ("token_centric_forward", "U",
+         lambda: omni.token_centric_forward(D, x, W, V, idx, gate, U=W[:-1])),
         ("wait_selftest", "counts", lambda: omni.wait_selftest(torch.zeros(4))),
     ]
 

@@ -33,6 +33,7 @@ CHUNK = 1 << 22  # elements per independent random stream
 # fixed per-tensor stream offsets
 _T_X, _T_WR, _T_WC, _T_W, _T_V, _T_PERM_R, _T_PERM_C = 0, 1, 2, 3, 4, 5, 6
 _T_W1, _T_W2 = 7, 8  # the shared dense MLP
+_T_U = 9  # the gate matrix of gated (SwiGLU) experts
 
 F32 = 0
 BF16 = 1
@@ -156,6 +157,12 @@ def make_experts(cfg: Config) -> dict:
     sc = 1.0 / np.sqrt(cfg.d)
     return {"W": _normal(cfg.seed, _T_W, (cfg.N, cfg.d), sc, cfg.dtype),
             "V": _normal(cfg.seed, _T_V, (cfg.N, cfg.d), sc, cfg.dtype)}
+
+
+def make_gate(cfg: Config) -> dict:
+    """The gate matrix U [N x d] of gated (SwiGLU) experts, drawn like W
+    (N(0, 1/d), so x.U[e] has unit scale)."""
+    return {"U": _normal(cfg.seed, _T_U, (cfg.N, cfg.d), 1.0 / np.sqrt(cfg.d), cfg.dtype)}
 
 
 def make_mlp(cfg: Config, F: int) -> dict:
