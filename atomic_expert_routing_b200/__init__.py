@@ -306,6 +306,48 @@ def moe_forward(D: LayerDims, x, Wr, Wc, W, V, bias_r=None, bias_c=None, *, U=No
     return y
 
 
+def moe_forward_shard(D: LayerDims, x, Wr, Wc, W, V, e_lo: int, e_hi: int, bias_r=None,
+                      bias_c=None, *, U=None, y_part=None, counts=None, idx=None, gate=None,
+                      ws=None, stream=None):
+    """This process' share of an expert-sharded forward: routing over all N
+    ids, execution of the tasks whose expert lies in [e_lo, e_hi) only, with
+    W, V (and U) the shard's rows [(e_hi - e_lo), d].  Returns y_part [L, d]
+    fp32, the shard's partial sum (add the shards' partials, then
+    cast_output)."""
+    if not 0 <= e_lo < e_hi <= D.N:
+        raise ValueError(f"shard ids [{e_lo}, {e_hi}) outside [0, {D.N})")
+    rows = (e_hi - e_lo) * D.d
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, bias_r=bias_r, bias_c=bias_c, counts=counts, idx=idx,
+               gate=gate)
+    for name, t in (("W", W), ("V", V), ("U", U)):
+        _expect(name, t, rows, D.torch_dtype, optional=name == "U")
+    _expect("y_part", y_part, D.L * D.d, torch.float32, optional=True)
+    dev = _device(x)
+    if y_part is None:
+        y_part = torch.empty((D.L, D.d), dtype=torch.float32, device=dev)
+    if counts is None:
+        counts = new_counts(dev)
+    wsp, n = _ws(D, OMNI_WS_FUSED, dev, ws)
+    dd = D.c()
+    _lib.check("omni_moe_forward_shard", _lib.load().omni_moe_forward_shard(
+        C.byref(dd), e_lo, e_hi, _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c),
+        _ptr(W), _ptr(U), _ptr(V), _ptr(y_part), _ptr(idx), _ptr(gate), _ptr(counts), wsp, n,
+        _stream(stream)))
+    return y_part
+
+
+def cast_output(D: LayerDims, src, *, y=None, stream=None):
+    """y [L, d] in the storage type from an fp32 [L, d] sum (bf16: nearest even)."""
+    _expect("src", src, D.L * D.d, torch.float32)
+    _expect_io(D, y=y)
+    if y is None:
+        y = torch.empty((D.L, D.d), dtype=D.torch_dtype, device=_device(src))
+    dd = D.c()
+    _lib.check("omni_cast_output", _lib.load().omni_cast_output(
+        C.byref(dd), _ptr(src), _ptr(y), _stream(stream)))
+    return y
+
+
 def mlp_workspace_size(D: LayerDims, F: int, with_routed: bool) -> int:
     n = C.c_size_t(0)
     dd = D.c()

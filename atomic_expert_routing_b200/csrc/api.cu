@@ -345,7 +345,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   // while the router runs (y itself for fp32, else the expert workspace)
   const int64_t acc_words = omni::expert_acc_words(D);
   float* acc = acc_words == 0 ? nullptr
-               : static_cast<float*>(D.dtype == OMNI_F32 ? y : w.expert);
+               : static_cast<float*>(D.dtype == OMNI_F32 || D.sharded() ? y : w.expert);
   // a small batch runs the two-kernel tail; its two counters are cleared
   // by the selection kernel in place of the accumulator
   const bool tail = omni::sched_exec_supported(D);
@@ -375,7 +375,10 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
     }
     if (rc != OMNI_OK) return rc;
     omni::CallRange stage("expert");
-    return cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s, U));
+    if ((rc = cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s, U))) !=
+        OMNI_OK)
+      return rc;
+    return D.sharded() ? cuda_status(omni::launch_shard_counts(D, w.uniq, counts, s)) : OMNI_OK;
   }
   {
     omni::CallRange stage("schedule");
@@ -384,9 +387,11 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   }
   if (rc != OMNI_OK) return rc;
   omni::CallRange stage("expert");
-  return cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
-                                         w.uniq, w.group_off, counts, y, w.expert, s, acc_zeroed,
-                                         true, U));
+  if ((rc = cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
+                                            w.uniq, w.group_off, counts, y, w.expert, s,
+                                            acc_zeroed, true, U))) != OMNI_OK)
+    return rc;
+  return D.sharded() ? cuda_status(omni::launch_shard_counts(D, w.uniq, counts, s)) : OMNI_OK;
 }
 
 // The checks of the shared MLP's width: F >= 1; a multiple of 8 (16-byte
@@ -511,6 +516,38 @@ int omni_moe_forward_glu(const omni_dims* dims, const void* x, const void* Wr, c
   if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
   return moe_forward_impl(D, x, Wr, Wc, bias_r, bias_c, W, V, y, idx_out, gate_out, counts, ws,
                           static_cast<cudaStream_t>(stream), U);
+}
+
+int omni_moe_forward_shard(const omni_dims* dims, int64_t e_lo, int64_t e_hi, const void* x,
+                           const void* Wr, const void* Wc, const float* bias_r,
+                           const float* bias_c, const void* W, const void* U, const void* V,
+                           float* y_part, int32_t* idx_out, float* gate_out, int32_t* counts,
+                           void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_forward_shard");
+  Dims D;
+  int rc = check_route_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (e_lo < 0 || e_hi <= e_lo || e_hi > D.N() || counts == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, W, V, y_part, U != nullptr ? U : x};
+  if (!tensors_ok(t16, 7)) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
+  D.e_lo = e_lo;
+  D.e_hi = e_hi;
+  return moe_forward_impl(D, x, Wr, Wc, bias_r, bias_c, W, V, y_part, idx_out, gate_out, counts,
+                          ws, static_cast<cudaStream_t>(stream), U);
+}
+
+int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* stream) {
+  omni::CallRange range("omni_cast_output");
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {src, y};
+  if (!tensors_ok(t16, 2)) return OMNI_ERR_INVALID_ARG;
+  if (D.dtype == OMNI_BF16 && static_cast<const void*>(src) == y) return OMNI_ERR_INVALID_ARG;
+  return cuda_status(omni::launch_cast_output(D, src, y, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

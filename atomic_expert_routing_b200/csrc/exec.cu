@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
                     const T* __restrict__ V, const int32_t* __restrict__ task_token,
                     const int32_t* __restrict__ task_expert,
                     const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
-                    int S, float* __restrict__ yacc, int32_t* status) {
+                    int S, ShardIds sh, float* __restrict__ yacc, int32_t* status) {
   pdl_wait();
   pdl_trigger();
   constexpr int EPV = kEpv<T>;
@@ -128,6 +128,11 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
     if (my_t < 0 || my_t >= L || my_e < 0 || my_e >= N) {
       raise_status(status, OMNI_DEV_BAD_INDEX);
       my_e = -1;
+    } else if (!sh.has(my_e)) {  // another shard's task: nothing to add
+      my_e = -1;
+      my_t = -1;
+    } else {
+      my_e -= sh.lo;
     }
   }
   const int64_t prev_t = __shfl_up_sync(0xffffffffu, my_t, 1);
@@ -289,8 +294,9 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
                    const int32_t* __restrict__ task_token,
                    const int32_t* __restrict__ task_expert,
                    const float* __restrict__ task_gate, int64_t M, int64_t L, int64_t N, int d,
-                   int S, int64_t nslices, float* __restrict__ yacc, int32_t* status,
-                   const uint8_t* __restrict__ dense, const float* __restrict__ cpre) {
+                   int S, int64_t nslices, ShardIds sh, float* __restrict__ yacc,
+                   int32_t* status, const uint8_t* __restrict__ dense,
+                   const float* __restrict__ cpre) {
   pdl_wait();
   pdl_trigger();
   constexpr int EPV = kEpv<T>;
@@ -320,6 +326,11 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
         raise_status(status, OMNI_DEV_BAD_INDEX);
         my_e = -1;
         my_t = -1;
+      } else if (!sh.has(my_e)) {  // another shard's task: nothing to add
+        my_e = -1;
+        my_t = -1;
+      } else {
+        my_e -= sh.lo;
       }
     }
     const uint32_t dmask = __ballot_sync(0xffffffffu, my_dense);
@@ -456,8 +467,9 @@ template <typename T, int NV, int R, bool HOLD_KEEP, bool GLU>
 __global__ void __launch_bounds__(kActWarps * 32, GLU ? 1 : 2)
     k_act(const T* __restrict__ H, const int32_t* __restrict__ hidx, int64_t nh,
           const T* __restrict__ F, const T* __restrict__ G, const int32_t* __restrict__ fidx,
-          int64_t nf, const float* __restrict__ task_gate, const int32_t* __restrict__ dst,
-          int64_t M, int d, int S, int64_t nslices, float* __restrict__ cbuf, int32_t* status) {
+          int64_t nf, ShardIds fs, const float* __restrict__ task_gate,
+          const int32_t* __restrict__ dst, int64_t M, int d, int S, int64_t nslices,
+          float* __restrict__ cbuf, int32_t* status) {
   pdl_wait();
   constexpr int SLOT = (GLU ? 2 : 1) * NV * 32;  // uint4 per ring slot: a row of F (and of G)
   extern __shared__ __align__(16) uint4 ring[];
@@ -482,6 +494,11 @@ __global__ void __launch_bounds__(kActWarps * 32, GLU ? 1 : 2)
         my_h = -1;
         my_f = -1;
         if (my_d < 0 || my_d >= M) my_d = -1;
+      } else if (!fs.has(my_f)) {  // a row of another shard: c = 0
+        my_h = -1;
+        my_f = -1;
+      } else {
+        my_f -= fs.lo;
       }
     }
     const int64_t prev_h = __shfl_up_sync(0xffffffffu, my_h, 1);
@@ -885,8 +902,8 @@ template <typename T, int NB, int D>
 __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
     k_acc(const T* __restrict__ V, const int32_t* __restrict__ task_token,
           const int32_t* __restrict__ task_expert, const float* __restrict__ cbuf, int64_t M,
-          int64_t L, int64_t N, int d, int col0, int64_t nslices, float* __restrict__ yacc,
-          int64_t ld) {
+          int64_t L, int64_t N, int d, int col0, int64_t nslices, ShardIds sh,
+          float* __restrict__ yacc, int64_t ld) {
   pdl_wait();
   static_assert(32 % D == 0, "the prefetch distance divides the slice");
   using QT = typename Quad<T>::type;
@@ -909,9 +926,10 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
       if (lane < m.n) {
         const int64_t t = task_token[a0 + lane];
         const int64_t e = task_expert[a0 + lane];
-        if (t >= 0 && t < L && e >= 0 && e < N) {
+        // (other shards' tasks are skipped like bad indices, silently)
+        if (t >= 0 && t < L && e >= 0 && e < N && sh.has(e)) {
           m.t = static_cast<int>(t);
-          m.e = static_cast<int>(e);
+          m.e = static_cast<int>(e - sh.lo);
           m.c = cbuf[a0 + lane];
         }
       }
@@ -1185,7 +1203,7 @@ cudaError_t launch_slices(const Dims& D, const void* x, const void* W, const voi
   OMNI_TRY(launch_k(k_expert_slices<T, NV>, static_cast<unsigned>(blocks), kExpThreads, 0, s,
       static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U),
       static_cast<const T*>(V), tt, te, tg, M,
-      D.L, D.N(), static_cast<int>(D.d), S, acc, status));
+      D.L, D.N(), static_cast<int>(D.d), S, shard_ids(D), acc, status));
   return cudaGetLastError();
 }
 
@@ -1211,7 +1229,8 @@ cudaError_t launch_async(const Dims& D, const void* x, const void* W, const void
   OMNI_TRY(launch_k(k_expert_async<T, NV, R, GLU>, static_cast<unsigned>(blocks), kAsyncWarps * 32,
       smem, s, static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U),
       static_cast<const T*>(V), tt, te, tg,
-      M, D.L, D.N(), static_cast<int>(D.d), S, nslices, acc, status, df.flag, df.cbuf));
+      M, D.L, D.N(), static_cast<int>(D.d), S, nslices, shard_ids(D), acc, status, df.flag,
+      df.cbuf));
   return cudaGetLastError();
 }
 
@@ -1309,7 +1328,7 @@ cudaError_t launch_acc(const Dims& D_, int col0, const void* V, const SweepWs& w
   if (blocks > cap) blocks = cap;
   OMNI_TRY(launch_k(k_acc<T, NB, D>, static_cast<unsigned>(blocks), kAccWarps * 32, 0, s,
       static_cast<const T*>(V), w.win.wt, w.win.we, w.cbuf, M, D_.L, D_.N(), static_cast<int>(D_.d),
-      col0, nslices, acc, ld));
+      col0, nslices, shard_ids(D_), acc, ld));
   return cudaGetLastError();
 }
 
@@ -1356,7 +1375,7 @@ cudaError_t sweeps_nv(const Dims& D, int Q, const void* x, const void* W, const 
     const int64_t b = blocks > per_sm * sm_count() ? per_sm * sm_count() : blocks;
     OMNI_TRY(launch_k(kernel, static_cast<unsigned>(b), kActWarps * 32, smem, s,
         static_cast<const T*>(x), w.win.xt, D.L, static_cast<const T*>(W),
-        static_cast<const T*>(U), w.win.xe, D.N(), w.win.xg, w.win.xdst, M,
+        static_cast<const T*>(U), w.win.xe, D.N(), shard_ids(D), w.win.xg, w.win.xdst, M,
         static_cast<int>(D.d), S, nslices, w.cbuf, status));
     return cudaGetLastError();
   };
@@ -1405,12 +1424,14 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                           bool acc_zeroed, bool allow_dense, const void* U) {
   if (D.L == 0) return cudaSuccess;
   const bool f32 = D.dtype == OMNI_F32;
-  float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
+  // fp32 storage and a shard's partial sum accumulate in y itself
+  const bool out32 = f32 || D.sharded();
+  float* acc = out32 ? static_cast<float*>(y) : static_cast<float*>(ws);
   int32_t* status = const_cast<int32_t*>(counts) + 2;
   const int Q = expert_sweeps(D);
   if (Q > 1) {  // the sweeps zero, accumulate and cast slice by slice
     const SweepWs w = carve_sweeps(D, ws, nullptr);
-    __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
+    __nv_bfloat16* ycast = out32 ? nullptr : static_cast<__nv_bfloat16*>(y);
     return f32 ? launch_sweeps<float>(D, Q, x, W, V, task_token, task_expert, task_gate,
                                       group_off, counts, w, nullptr, acc, ycast, status, s, U)
                : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, task_token, task_expert, task_gate,
@@ -1421,7 +1442,7 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                                : launch_zero(acc, static_cast<size_t>(expert_acc_words(D)), s);
   if (err != cudaSuccess) return err;
   DenseFlags df{nullptr, nullptr};
-  if (allow_dense && U == nullptr && uniq != nullptr && dense_path(D)) {
+  if (allow_dense && U == nullptr && !D.sharded() && uniq != nullptr && dense_path(D)) {
     void* dws = static_cast<char*>(ws) + dense_ws_offset(D);
     OMNI_TRY(launch_dense_activations(D, x, W, task_token, task_expert, task_gate, uniq,
                                       group_off, const_cast<int32_t*>(counts), dws, s));
@@ -1431,7 +1452,7 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
                                      s, df, U)
             : dispatch_slices<__nv_bfloat16>(D, x, W, V, task_token, task_expert, task_gate, acc,
                                              status, s, df, U);
-  if (err != cudaSuccess || f32) return err;
+  if (err != cudaSuccess || out32) return err;
   const int64_t n = D.L * D.d;
   OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, acc,
       static_cast<__nv_bfloat16*>(y), n));
@@ -1453,10 +1474,11 @@ cudaError_t launch_expert_windows(const Dims& D, const void* x, const void* W, c
   const int Q = expert_sweeps(D);
   if (D.L == 0 || Q <= 1) return cudaErrorInvalidValue;
   const bool f32 = D.dtype == OMNI_F32;
-  float* acc = f32 ? static_cast<float*>(y) : static_cast<float*>(ws);
+  const bool out32 = f32 || D.sharded();  // the accumulator is y itself
+  float* acc = out32 ? static_cast<float*>(y) : static_cast<float*>(ws);
   int32_t* status = counts + 2;
   const SweepWs w = carve_sweeps(D, ws, nullptr);
-  __nv_bfloat16* ycast = f32 ? nullptr : static_cast<__nv_bfloat16*>(y);
+  __nv_bfloat16* ycast = out32 ? nullptr : static_cast<__nv_bfloat16*>(y);
   return f32 ? launch_sweeps<float>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr, counts, w,
                                     w.win_lo, acc, ycast, status, s, U)
              : launch_sweeps<__nv_bfloat16>(D, Q, x, W, V, nullptr, nullptr, nullptr, nullptr,
@@ -1481,6 +1503,19 @@ cudaError_t launch_zero(void* p, size_t n_words, cudaStream_t s) {
   const int64_t n = static_cast<int64_t>(n_words);
   return launch_k(k_zero_words, static_cast<unsigned>((n / 4 + 256) / 256), 256, 0, s,
                   static_cast<uint32_t*>(p), n);
+}
+
+cudaError_t launch_cast_output(const Dims& D, const float* src, void* y, cudaStream_t s) {
+  const int64_t n = D.L * D.d;
+  if (n == 0) return cudaSuccess;
+  if (D.dtype == OMNI_F32) {
+    if (src == y) return cudaSuccess;
+    return cudaMemcpyAsync(y, src, static_cast<size_t>(n) * sizeof(float),
+                           cudaMemcpyDeviceToDevice, s);
+  }
+  OMNI_TRY(launch_k(k_cast, static_cast<unsigned>((n / 8 + 255) / 256), 256, 0, s, src,
+      static_cast<__nv_bfloat16*>(y), n));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,

@@ -29,11 +29,28 @@ struct Dims {
   int64_t L, d, Nr, Nc, k, K, B;
   int dtype;
   int flags;
+  // Expert shard: this process holds the W/V (and U) rows of ids
+  // [e_lo, e_hi), id e in row e - e_lo.  A sharded execution skips the tasks
+  // of other ids (silently: they are not bad indices) and leaves its partial
+  // sum in fp32, whatever the storage type.  e_hi < 0: not sharded.
+  int64_t e_lo = 0, e_hi = -1;
+  bool sharded() const { return e_hi >= 0; }
+  int64_t shard_lo() const { return sharded() ? e_lo : 0; }
+  int64_t shard_hi() const { return sharded() ? e_hi : N(); }
   int64_t N() const { return Nr * Nc; }
   int64_t M() const { return L * K; }
   int64_t ucap() const { return N() < M() ? N() : M(); }       // bound on |U|
   int64_t gmax() const { return (ucap() + B - 1) / B; }        // bound on #groups
 };
+
+// The ids whose rows this process holds, as the kernels see them: a task of
+// id e outside [lo, hi) belongs to another shard and is skipped; row e - lo
+// otherwise.  Unsharded: [0, N).
+struct ShardIds {
+  int64_t lo, hi;
+  __host__ __device__ bool has(int64_t e) const { return e >= lo && e < hi; }
+};
+inline ShardIds shard_ids(const Dims& D) { return ShardIds{D.shard_lo(), D.shard_hi()}; }
 
 // ---- router logits: Z [L x (Nr + Nc)] fp32 -------------------------------
 cudaError_t launch_router_simt(const Dims& D, const void* x, const void* Wr, const void* Wc,
@@ -132,6 +149,13 @@ cudaError_t launch_expert(const Dims& D, const void* x, const void* W, const voi
 // partial sums: y itself for fp32, else the head of ws), in floats; 0 for
 // batches with sweeps.
 int64_t expert_acc_words(const Dims& D);
+// y [L x d] in the storage type <- src fp32 (bf16: nearest even; fp32: a
+// copy unless src == y).
+cudaError_t launch_cast_output(const Dims& D, const float* src, void* y, cudaStream_t s);
+// After a sharded execution of a schedule: counts[0], counts[1] replaced by
+// the shard's active ids in uniq and their group count.
+cudaError_t launch_shard_counts(const Dims& D, const int32_t* uniq, int32_t* counts,
+                                cudaStream_t s);
 cudaError_t launch_token(const Dims& D, const void* x, const void* W, const void* V,
                          const int32_t* idx, const float* gate, void* y, int32_t* status,
                          cudaStream_t s, const void* U = nullptr);

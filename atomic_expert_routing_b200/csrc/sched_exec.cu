@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(kSeThreads, 1)
     k_sched_act(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
                 const int32_t* __restrict__ idx,
                 const float* __restrict__ gate, int L, int K, int64_t N, int B, SePlan P,
-                float* __restrict__ cbuf, SeScratch sc, int32_t* __restrict__ counts) {
+                ShardIds sh, float* __restrict__ cbuf, SeScratch sc,
+                int32_t* __restrict__ counts) {
   constexpr int EPV = 16 / sizeof(T);
   constexpr int kPer = kSeMaxM / kSeThreads;  // routing ids per thread
   constexpr uint32_t kIdxMask = (1u << 13) - 1u;
@@ -119,8 +120,10 @@ __global__ void __launch_bounds__(kSeThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int M = L * K;
   const int tile = blockIdx.x / kSeParts, part = blockIdx.x % kSeParts;
-  const int64_t lo = static_cast<int64_t>(tile) * P.span;
-  const int64_t hi = lo + P.span < N ? lo + P.span : N;
+  // the tile's ids [lo, hi) within this process' ids [sh.lo, sh.hi); the
+  // row of id e is e - sh.lo
+  const int64_t lo = sh.lo + static_cast<int64_t>(tile) * P.span;
+  const int64_t hi = lo + P.span < sh.hi ? lo + P.span : sh.hi;
   extern __shared__ __align__(16) uint8_t sm[];
   uint32_t* own = reinterpret_cast<uint32_t*>(sm);   // [M] (e - lo) << 13 | task index
   uint32_t* sorted = own + M;                        // [M] the same, by expert
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(kSeThreads, 1)
   // r asks L2 for those of own tasks r, r + parts, ... while the tile is
   // sorted
   for (int q = part + kSeParts * tid; q < n; q += kSeParts * kSeThreads)
-    prefetch_l2(W + (lo + (own[q] >> 13)) * d, static_cast<uint32_t>(d * sizeof(T)));
+    prefetch_l2(W + (lo - sh.lo + (own[q] >> 13)) * d, static_cast<uint32_t>(d * sizeof(T)));
 
   // (2) rank of every active id of the tile (popcount prefix of the bitmap)
   {
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(kSeThreads, 1)
       if (pos >= b1) continue;
       const uint32_t v = sorted[pos];  // warp-uniform
       ii[r] = static_cast<int>(v & kIdxMask);
-      const int64_t e = lo + (v >> 13);
+      const int64_t e = lo - sh.lo + (v >> 13);  // the row
       const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(ii[r] / K) * d);
       const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
 #pragma unroll
@@ -296,11 +299,11 @@ __global__ void __launch_bounds__(kSeThreads, 1)
 // columns], cols = NS * 32 * (16 / sizeof(T)).  Warp w sums tasks w, w + 16,
 // ... in registers; the warps' partial rows are added in shared memory in a
 // fixed order (the result does not depend on timing).
-template <typename T, int NS>
+template <typename T, int NS, typename O>
 __global__ void __launch_bounds__(kSeThreads)
     k_gather_v(const T* __restrict__ V, const int32_t* __restrict__ idx,
-               const float* __restrict__ cbuf, int K, int64_t N, int d, T* __restrict__ y,
-               int32_t* __restrict__ status) {
+               const float* __restrict__ cbuf, int K, int64_t N, int d, ShardIds sh,
+               O* __restrict__ y, int32_t* __restrict__ status) {
   constexpr int EPV = 16 / sizeof(T);
   constexpr int COLS = NS * 32 * EPV;
   __shared__ __align__(16) float part[kSeWarps][COLS];
@@ -317,24 +320,28 @@ __global__ void __launch_bounds__(kSeThreads)
   for (int k0 = warp; k0 < K; k0 += 2 * kSeWarps) {
     uint4 vv[2][NS];
     float cc[2];
+    bool live[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int k = k0 + r * kSeWarps;
       cc[r] = 0.0f;
+      live[r] = false;
       if (k >= K) continue;
       int64_t e = idx[t * K + k];
       if (e < 0 || e >= N) {
         if (lane == 0) raise_status(status, OMNI_DEV_BAD_INDEX);
         e = 0;
       }
+      if (!sh.has(e)) continue;  // another shard's task
+      live[r] = true;
       cc[r] = cbuf[t * K + k];
-      const uint4* vr = reinterpret_cast<const uint4*>(V + e * d + col0);
+      const uint4* vr = reinterpret_cast<const uint4*>(V + (e - sh.lo) * d + col0);
 #pragma unroll
       for (int q = 0; q < NS; ++q) vv[r][q] = vr[q * 32 + lane];
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      if (k0 + r * kSeWarps >= K) continue;
+      if (!live[r]) continue;
 #pragma unroll
       for (int q = 0; q < NS; ++q) axpy16(cc[r], vv[r][q], a[q], static_cast<const T*>(nullptr));
     }
@@ -371,7 +378,8 @@ bool se_plan(const Dims& D, SePlan* P) {
   const int64_t M = D.M();
   if (D.L < 1 || M > kSeMaxM || D.N() > kSeMaxN || se_nv(D) == 0) return false;
   if (D.B > (int64_t(1) << 30)) return false;
-  P->span = (D.N() + kSeTiles - 1) / kSeTiles;
+  const int64_t ids = D.shard_hi() - D.shard_lo();  // this process' ids
+  P->span = (ids + kSeTiles - 1) / kSeTiles;
   P->words = static_cast<int>((P->span + 31) / 32);
   P->smem = static_cast<size_t>(M) * 16 + static_cast<size_t>(P->words) * 8;
   return P->smem <= 200 * 1024;
@@ -396,14 +404,21 @@ cudaError_t launch_se_t(const Dims& D, const SePlan& P, const void* x, const voi
   OMNI_TRY(launch_k(k_sched_act<T, NV, GLU>, kSeTiles * kSeParts, kSeThreads, P.smem, s,
       static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U), idx, gate,
       static_cast<int>(D.L),
-      static_cast<int>(D.K), D.N(), static_cast<int>(D.B), P, cbuf, sc, counts));
+      static_cast<int>(D.K), D.N(), static_cast<int>(D.B), P, shard_ids(D), cbuf, sc, counts));
   // value rows: NS vectors per lane and CTA, 2 when the row has them
   constexpr int NS = NV < 2 ? NV : 2;
   constexpr int COLS = NS * 32 * (16 / sizeof(T));
   const dim3 grid(static_cast<unsigned>(D.L), static_cast<unsigned>(D.d / COLS));
-  OMNI_TRY(launch_k(k_gather_v<T, NS>, grid, kSeThreads, 0, s, static_cast<const T*>(V), idx,
-      static_cast<const float*>(cbuf), static_cast<int>(D.K), D.N(), static_cast<int>(D.d),
-      static_cast<T*>(y), counts + 2));
+  // a shard's partial sum stays in fp32
+  if (D.sharded()) {
+    OMNI_TRY(launch_k(k_gather_v<T, NS, float>, grid, kSeThreads, 0, s, static_cast<const T*>(V),
+        idx, static_cast<const float*>(cbuf), static_cast<int>(D.K), D.N(),
+        static_cast<int>(D.d), shard_ids(D), static_cast<float*>(y), counts + 2));
+  } else {
+    OMNI_TRY(launch_k(k_gather_v<T, NS, T>, grid, kSeThreads, 0, s, static_cast<const T*>(V), idx,
+        static_cast<const float*>(cbuf), static_cast<int>(D.K), D.N(), static_cast<int>(D.d),
+        shard_ids(D), static_cast<T*>(y), counts + 2));
+  }
   return cudaGetLastError();
 }
 

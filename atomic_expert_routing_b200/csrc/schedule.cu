@@ -1207,4 +1207,36 @@ cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const flo
   return cudaGetLastError();
 }
 
+namespace {
+// counts[0] (|U| of the whole batch) and counts[1] replaced by those of the
+// shard's ids [lo, hi): the active ids in U (sorted) between the two bounds.
+__global__ void k_shard_counts(const int32_t* __restrict__ uniq, int32_t* __restrict__ counts,
+                               int64_t lo, int64_t hi, int64_t ucap, int64_t B) {
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x != 0) return;
+  int64_t n = counts[0];
+  if (n < 0) n = 0;
+  if (n > ucap) n = ucap;
+  auto lower = [&](int64_t v) {  // first position of U holding an id >= v
+    int64_t l = 0, h = n;
+    while (l < h) {
+      const int64_t m = (l + h) >> 1;
+      if (uniq[m] < v) l = m + 1; else h = m;
+    }
+    return l;
+  };
+  const int64_t u = lower(hi) - lower(lo);
+  counts[0] = static_cast<int32_t>(u);
+  counts[1] = static_cast<int32_t>((u + B - 1) / B);
+}
+}  // namespace
+
+cudaError_t launch_shard_counts(const Dims& D, const int32_t* uniq, int32_t* counts,
+                                cudaStream_t s) {
+  OMNI_TRY(launch_k(k_shard_counts, 1, 32, 0, s, uniq, counts, D.shard_lo(), D.shard_hi(),
+      D.ucap(), D.B));
+  return cudaGetLastError();
+}
+
 }  // namespace omni

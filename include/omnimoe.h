@@ -315,6 +315,43 @@ int omni_token_centric_forward_glu(const omni_dims* dims, const void* x, const v
                                    const float* gate, void* y, int32_t* counts, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/*
+ * Expert-sharded forward, one call per process (GPU) of a group that splits
+ * the N experts by contiguous id ranges.  The pages describe no distribution;
+ * this follows the natural split of the expert-centric order: routing and
+ * scheduling are replicated (Wr, Wc are small), each process executes only
+ * the tasks whose expert lies in its ids [e_lo, e_hi), and the partial
+ * outputs are summed across processes by the caller (one all-reduce).
+ *   W, V (and U, nullable: gated experts as in omni_moe_forward_glu): the
+ *      shard's rows only, [(e_hi - e_lo) x d], id e in row e - e_lo.
+ *   y_part [L x d] fp32, overwritten with this shard's partial sum
+ *      sum over the tasks (t, e, g) with e in [e_lo, e_hi) of g * h * V[e]
+ *      (tokens without such a task get 0).  The sum over a partition of
+ *      [0, N) of the y_part is y of omni_moe_forward up to the order of fp32
+ *      additions; omni_cast_output rounds it to the storage type.
+ *   idx_out / gate_out (nullable): the whole batch's routing, as
+ *      omni_moe_forward (every process computes the same).
+ *   counts[0], counts[1]: the number of active ids in [e_lo, e_hi) and
+ *      their group count ceil(counts[0] / B); counts[2] status bits.
+ *   ws: omni_workspace_size(dims, OMNI_WS_FUSED).
+ * dims describe the whole layer (N = Nr * Nc ids); 0 <= e_lo < e_hi <= N
+ * else OMNI_ERR_INVALID_ARG; the other checks as omni_moe_forward.  The
+ * tensor-core activations of dense groups are not used.
+ */
+int omni_moe_forward_shard(const omni_dims* dims, int64_t e_lo, int64_t e_hi, const void* x,
+                           const void* Wr, const void* Wc, const float* bias_r,
+                           const float* bias_c, const void* W, const void* U, const void* V,
+                           float* y_part, int32_t* idx_out, float* gate_out, int32_t* counts,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * y [L x d] in the storage type of dims <- src [L x d] fp32 (bf16: rounded
+ * to nearest even; fp32: copied unless src == y).  The last step of a
+ * sharded forward, after the partial sums are added.  src == y with bf16
+ * storage is OMNI_ERR_INVALID_ARG.
+ */
+int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* omni_status_string(int status);
 

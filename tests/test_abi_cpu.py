@@ -267,3 +267,43 @@ def test_gated_entries_check_U_like_the_other_tensors(lib):
     K6 = _dims(k=4, K=6)
     assert lib.omni_moe_forward_glu(C.byref(K6), *([fake] * 12), fake, 1 << 30,
                                     None) == _lib.OMNI_ERR_UNSUPPORTED
+
+
+def test_shard_entry_host_checks(lib):
+    """omni_moe_forward_shard: the shard's id range must be a non-empty part
+    of [0, N), y_part and the (optional) U 16-byte aligned; an empty batch
+    is a no-op; K > k is refused as in the unsharded call."""
+    D = _dims(Nr=8, Nc=8)  # N = 64
+    fake = C.c_void_p(4096)
+    odd = C.c_void_p(4096 + 4)
+    bad = _lib.OMNI_ERR_INVALID_ARG
+
+    def call(dims, lo, hi, U=None, y_part=fake, counts=fake):
+        # x, Wr, Wc, bias_r, bias_c, W, U, V, y_part, idx, gate, counts
+        args = [fake, fake, fake, None, None, fake, U, fake, y_part, None, None, counts]
+        return lib.omni_moe_forward_shard(C.byref(dims), lo, hi, *args, None, 0, None)
+
+    for lo, hi in ((-1, 4), (4, 4), (5, 4), (0, 65), (64, 65)):
+        assert call(D, lo, hi) == bad, (lo, hi)
+    assert call(D, 0, 64, counts=None) == bad
+    assert call(D, 0, 64, y_part=odd) == bad
+    assert call(D, 0, 64, U=odd) == bad
+    # a valid call stops at the workspace (none given)
+    assert call(D, 0, 64) == _lib.OMNI_ERR_WORKSPACE
+    assert call(D, 63, 64, U=fake) == _lib.OMNI_ERR_WORKSPACE
+    assert call(_dims(L=0, Nr=8, Nc=8), 3, 9) == _lib.OMNI_OK
+    assert call(_dims(Nr=8, Nc=8, k=2, K=3), 0, 64) == _lib.OMNI_ERR_UNSUPPORTED
+
+
+def test_cast_output_host_checks(lib):
+    fake, other = C.c_void_p(4096), C.c_void_p(8192)
+    D = _dims(dtype=_lib.OMNI_BF16)
+    assert lib.omni_cast_output(C.byref(D), None, fake, None) == _lib.OMNI_ERR_INVALID_ARG
+    assert lib.omni_cast_output(C.byref(D), fake, C.c_void_p(4100), None) == \
+        _lib.OMNI_ERR_INVALID_ARG
+    # in place is a bf16 error (the fp32 sum would be overwritten as it is read)
+    assert lib.omni_cast_output(C.byref(D), fake, fake, None) == _lib.OMNI_ERR_INVALID_ARG
+    assert lib.omni_cast_output(C.byref(_dims(L=0)), fake, other, None) == _lib.OMNI_OK
+    # fp32 in place: nothing to do, no launch
+    F = _dims(dtype=_lib.OMNI_F32)
+    assert lib.omni_cast_output(C.byref(F), fake, fake, None) == _lib.OMNI_OK

@@ -32,7 +32,8 @@ HOT = {
     "omni::(anonymous namespace)::k_router_tc<64>": 0,
     "omni::(anonymous namespace)::k_select_wide<8, 2, 2>": 16,
     "omni::(anonymous namespace)::k_sched_act<__nv_bfloat16, 8, false>": 0,
-    "omni::(anonymous namespace)::k_gather_v<__nv_bfloat16, 2>": 0,
+    "omni::(anonymous namespace)::k_gather_v<__nv_bfloat16, 2, __nv_bfloat16>": 0,
+    "omni::(anonymous namespace)::k_gather_v<__nv_bfloat16, 2, float>": 0,
     # decode stages timed separately (omni_schedule + omni_expert_forward)
     "omni::(anonymous namespace)::k_sched_bits<64>": 0,
     "omni::(anonymous namespace)::k_expert_async<__nv_bfloat16, 8, 3, false>": 0,

@@ -64,3 +64,66 @@ def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(1, 16384, 2.0) == pytest.approx(8.192e6)
     assert bench.job_throughput(4, 16384, 2.0) == pytest.approx(4 * 8.192e6)
     assert bench.max_over_ranks(2.5, 1, "cpu") == 2.5
+
+
+# ------------------------------------------------- expert-sharded forward (host logic)
+
+SHARD_CFG = WL.Config("shards", L=24, d=64, Nr=8, Nc=8, k=4, K=4, B=3, dtype=WL.F32, seed=9)
+
+
+def _shard_main(rank, world, port, out_dir):
+    """One process of an expert-sharded forward with the oracle in place of
+    the kernels: the whole batch's routing, this rank's experts only (other
+    rows replaced by garbage that must not leak), the partials summed by
+    sharded.combine over gloo."""
+    import torch
+    import oracle as O
+    from atomic_expert_routing_b200 import sharded
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = SHARD_CFG
+        h = WL.make_inputs(cfg)
+        idx, gate, _ = O.route(cfg, h)
+        lo, hi = sharded.shard_ranges(cfg.N, world)[rank]
+        local = dict(h)
+        for key in ("W", "V"):
+            rows = np.full_like(h[key], 1e6)
+            rows[lo:hi] = h[key][lo:hi]
+            local[key] = rows
+        inside = (idx >= lo) & (idx < hi)
+        y_part, _ = O.forward_token(cfg, local, idx, np.where(inside, gate, 0.0))
+        y = sharded.combine(torch.from_numpy(y_part.astype(np.float32)))
+        np.save(os.path.join(out_dir, f"y{rank}.npy"), y.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_shards_sum_to_the_layer(tmp_path, world):
+    import oracle as O
+    mp.spawn(_shard_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    h = WL.make_inputs(SHARD_CFG)
+    idx, gate, _ = O.route(SHARD_CFG, h)
+    y_ref, _ = O.forward_token(SHARD_CFG, h, idx, gate)
+    for r in range(world):
+        y = np.load(tmp_path / f"y{r}.npy")
+        np.testing.assert_allclose(y, y_ref, rtol=1e-5, atol=1e-6 * np.abs(y_ref).max())
+
+
+def test_shard_ranges_partition_the_ids():
+    from atomic_expert_routing_b200 import sharded
+    for N, G in ((1, 1), (7, 3), (64, 8), (1 << 20, 7), (10, 10)):
+        r = sharded.shard_ranges(N, G)
+        assert len(r) == G and r[0][0] == 0 and r[-1][1] == N
+        assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+        sizes = [hi - lo for lo, hi in r]
+        assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1
+    for N, G in ((3, 4), (5, 0)):
+        with pytest.raises(ValueError):
+            sharded.shard_ranges(N, G)

@@ -48,6 +48,8 @@ def _calls():
         "expert_forward-glu": lambda: omni.expert_forward(D, x, W, V, sched, U=W),
         "token_centric_forward-glu":
             lambda: omni.token_centric_forward(D, x, W, V, idx, gate, U=W),
+        "moe_forward_shard": lambda: omni.moe_forward_shard(D, x, Wr, Wc, W[:2], V[:2], 0, 2),
+        "cast_output": lambda: omni.cast_output(D, _t(c.L, c.d)),
         "wait_selftest": lambda: omni.wait_selftest(torch.zeros(4, dtype=torch.int32)),
     }
 
@@ -132,6 +134,12 @@ def _shrunk_calls():
         ("expert_forward", "U", lambda: omni.expert_forward(D, x, W, V, sched, U=W.half())),
         ("token_centric_forward", "U",
          lambda: omni.token_centric_forward(D, x, W, V, idx, gate, U=W[:-1])),
+        ("moe_forward_shard", "W",
+         lambda: omni.moe_forward_shard(D, x, Wr, Wc, W[:1], V[:2], 0, 2)),
+        ("moe_forward_shard", "y_part",
+         lambda: omni.moe_forward_shard(D, x, Wr, Wc, W[:2], V[:2], 0, 2, y_part=x.half())),
+        ("cast_output", "src", lambda: omni.cast_output(D, x.double())),
+        ("cast_output", "y", lambda: omni.cast_output(D, x, y=x[:-1])),
         ("wait_selftest", "counts", lambda: omni.wait_selftest(torch.zeros(4))),
     ]
 
