@@ -74,6 +74,7 @@ struct FusedWs {
   RouteWs route;
   int32_t *idx, *task_token, *task_expert, *uniq, *group_off;
   float *gate, *task_gate;
+  int64_t* shard_range;  // [2]: the task range a sharded execution visits
   void* sched;
   void* expert;
 };
@@ -101,6 +102,7 @@ FusedWs carve_fused(const Dims& D, Carver& c) {
   const size_t tail = omni::sched_exec_supported(D) ? omni::sched_exec_ws_words(D) * 4 : 0;
   const size_t ex = omni::expert_ws_bytes(D);
   w.expert = c.take<char>(ex > tail ? ex : tail);
+  w.shard_range = c.take<int64_t>(2);
   return w;
 }
 
@@ -375,7 +377,15 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
     }
     if (rc != OMNI_OK) return rc;
     omni::CallRange stage("expert");
-    if ((rc = cuda_status(omni::launch_expert_windows(D, x, W, V, counts, y, w.expert, s, U))) !=
+    Dims De = D;
+    if (D.sharded()) {
+      if ((rc = cuda_status(omni::launch_shard_range(D, w.uniq, w.group_off, counts,
+                                                     omni::window_tasks(D), w.shard_range, s))) !=
+          OMNI_OK)
+        return rc;
+      De.shard_range = w.shard_range;
+    }
+    if ((rc = cuda_status(omni::launch_expert_windows(De, x, W, V, counts, y, w.expert, s, U))) !=
         OMNI_OK)
       return rc;
     return D.sharded() ? cuda_status(omni::launch_shard_counts(D, w.uniq, counts, s)) : OMNI_OK;
@@ -387,9 +397,18 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   }
   if (rc != OMNI_OK) return rc;
   omni::CallRange stage("expert");
-  if ((rc = cuda_status(omni::launch_expert(D, x, W, V, w.task_token, w.task_expert, w.task_gate,
-                                            w.uniq, w.group_off, counts, y, w.expert, s,
-                                            acc_zeroed, true, U))) != OMNI_OK)
+  Dims De = D;
+  if (D.sharded()) {
+    // the sweeps (if any) visit whole windows of the schedule's order
+    const int64_t T = omni::expert_sweeps(D) > 1 ? omni::window_tasks(D) : 0;
+    if ((rc = cuda_status(omni::launch_shard_range(D, w.uniq, w.group_off, counts, T,
+                                                   w.shard_range, s))) != OMNI_OK)
+      return rc;
+    De.shard_range = w.shard_range;
+  }
+  if ((rc = cuda_status(omni::launch_expert(De, x, W, V, w.task_token, w.task_expert,
+                                            w.task_gate, w.uniq, w.group_off, counts, y, w.expert,
+                                            s, acc_zeroed, true, U))) != OMNI_OK)
     return rc;
   return D.sharded() ? cuda_status(omni::launch_shard_counts(D, w.uniq, counts, s)) : OMNI_OK;
 }

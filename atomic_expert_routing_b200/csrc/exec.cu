@@ -116,6 +116,11 @@ __global__ void __launch_bounds__(kExpThreads, (NV >= 8 ? 3 : 4))
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t a0 = wid * S;
   if (a0 >= M) return;  // whole warp
+  {
+    int64_t s0, s1;  // a shard's slices (all of them unsharded)
+    sh.slices(S, (M + S - 1) / S, &s0, &s1);
+    if (wid < s0 || wid >= s1) return;
+  }
   const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
   const int nvec = d / EPV;
   // one task per lane (S <= 32): token, expert, gate
@@ -308,7 +313,9 @@ __global__ void __launch_bounds__(kAsyncWarps * 32, 1)
   const uint64_t pol_stream = policy_evict_first();
   const uint64_t pol_keep = policy_evict_last();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kAsyncWarps;
-  for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kAsyncWarps + warp; sl < nslices; sl += nw) {
+  int64_t s0, s1;  // a shard's slices (all of them unsharded)
+  sh.slices(S, nslices, &s0, &s1);
+  for (int64_t sl = s0 + static_cast<int64_t>(blockIdx.x) * kAsyncWarps + warp; sl < s1; sl += nw) {
     const int64_t a0 = sl * S;
     const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
     int64_t my_t = -1, my_e = -1;
@@ -479,7 +486,9 @@ __global__ void __launch_bounds__(kActWarps * 32, GLU ? 1 : 2)
   const uint64_t pol_once = policy_evict_first();
   const uint64_t pol_keep = policy_evict_last();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kActWarps;
-  for (int64_t sl = static_cast<int64_t>(blockIdx.x) * kActWarps + warp; sl < nslices; sl += nw) {
+  int64_t s0, s1;  // a shard's slices (all of them unsharded)
+  fs.slices(S, nslices, &s0, &s1);
+  for (int64_t sl = s0 + static_cast<int64_t>(blockIdx.x) * kActWarps + warp; sl < s1; sl += nw) {
     const int64_t a0 = sl * S;
     const int n = static_cast<int>(M - a0 < S ? M - a0 : S);
     int64_t my_h = -1, my_f = -1, my_d = -1;
@@ -912,15 +921,17 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
   const uint64_t pol_stream = policy_evict_normal();
   const uint64_t pol_keep = policy_evict_last();
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kAccWarps;
-  int64_t sl = static_cast<int64_t>(blockIdx.x) * kAccWarps + warp;
-  if (sl >= nslices) return;
+  int64_t s0, s1;  // a shard's slices (all of them unsharded)
+  sh.slices(32, nslices, &s0, &s1);
+  int64_t sl = s0 + static_cast<int64_t>(blockIdx.x) * kAccWarps + warp;
+  if (sl >= s1) return;
   struct Meta {
     int n, t, e;
     float c;
   };
   auto load_meta = [&](int64_t s) {
     Meta m{0, -1, -1, 0.0f};
-    if (s < nslices) {
+    if (s < s1) {
       const int64_t a0 = s * 32;
       m.n = static_cast<int>(M - a0 < 32 ? M - a0 : 32);
       if (lane < m.n) {
@@ -991,7 +1002,7 @@ __global__ void __launch_bounds__(kAccWarps * 32, (NB >= 8 ? 4 : 5))
       }
     }
     sl += nw;
-    if (sl >= nslices) break;
+    if (sl >= s1) break;
     cur = nxt;
     nxt = load_meta(sl + nw);
   }

@@ -34,6 +34,9 @@ struct Dims {
   // of other ids (silently: they are not bad indices) and leaves its partial
   // sum in fp32, whatever the storage type.  e_hi < 0: not sharded.
   int64_t e_lo = 0, e_hi = -1;
+  // device [2] (nullable): the task positions the execution visits for the
+  // shard (launch_shard_range); nullptr: every task
+  const int64_t* shard_range = nullptr;
   bool sharded() const { return e_hi >= 0; }
   int64_t shard_lo() const { return sharded() ? e_lo : 0; }
   int64_t shard_hi() const { return sharded() ? e_hi : N(); }
@@ -46,11 +49,30 @@ struct Dims {
 // The ids whose rows this process holds, as the kernels see them: a task of
 // id e outside [lo, hi) belongs to another shard and is skipped; row e - lo
 // otherwise.  Unsharded: [0, N).
+// arange (device, nullable): the task positions [arange[0], arange[1]) of
+// the execution order that can hold the shard's tasks (launch_shard_range);
+// execution kernels visit only the slices that overlap it.
 struct ShardIds {
   int64_t lo, hi;
+  const int64_t* arange;
   __host__ __device__ bool has(int64_t e) const { return e >= lo && e < hi; }
+  // the slices [*s0, *s1) of S tasks (of nslices) to visit; read on the
+  // device after the kernel's dependency wait
+  __device__ void slices(int S, int64_t nslices, int64_t* s0, int64_t* s1) const {
+    *s0 = 0;
+    *s1 = nslices;
+    if (arange == nullptr) return;
+    const int64_t a0 = arange[0], a1 = arange[1];
+    const int64_t b0 = a0 < 0 ? 0 : a0 / S;
+    const int64_t b1 = a1 <= 0 ? 0 : (a1 + S - 1) / S;
+    *s0 = b0 < nslices ? b0 : nslices;
+    *s1 = b1 < nslices ? b1 : nslices;
+    if (*s1 < *s0) *s1 = *s0;
+  }
 };
-inline ShardIds shard_ids(const Dims& D) { return ShardIds{D.shard_lo(), D.shard_hi()}; }
+inline ShardIds shard_ids(const Dims& D) {
+  return ShardIds{D.shard_lo(), D.shard_hi(), D.sharded() ? D.shard_range : nullptr};
+}
 
 // ---- router logits: Z [L x (Nr + Nc)] fp32 -------------------------------
 cudaError_t launch_router_simt(const Dims& D, const void* x, const void* Wr, const void* Wc,
@@ -152,6 +174,15 @@ int64_t expert_acc_words(const Dims& D);
 // y [L x d] in the storage type <- src fp32 (bf16: nearest even; fp32: a
 // copy unless src == y).
 cudaError_t launch_cast_output(const Dims& D, const float* src, void* y, cudaStream_t s);
+// Before a sharded execution: the range of task positions that can hold the
+// shard's tasks, arange[0..1], from the schedule (U sorted, group_off) --
+// the groups from the one holding the shard's first active id to the one
+// holding its last -- and, for the window order of the sweeps (T =
+// window_tasks(D); 0 for the schedule's own order), widened to whole
+// windows.  Empty ([0, 0)) when the shard has no active id.
+cudaError_t launch_shard_range(const Dims& D, const int32_t* uniq, const int32_t* group_off,
+                               const int32_t* counts, int64_t T, int64_t* arange,
+                               cudaStream_t s);
 // After a sharded execution of a schedule: counts[0], counts[1] replaced by
 // the shard's active ids in uniq and their group count.
 cudaError_t launch_shard_counts(const Dims& D, const int32_t* uniq, int32_t* counts,

@@ -378,11 +378,17 @@ bool se_plan(const Dims& D, SePlan* P) {
   const int64_t M = D.M();
   if (D.L < 1 || M > kSeMaxM || D.N() > kSeMaxN || se_nv(D) == 0) return false;
   if (D.B > (int64_t(1) << 30)) return false;
-  const int64_t ids = D.shard_hi() - D.shard_lo();  // this process' ids
-  P->span = (ids + kSeTiles - 1) / kSeTiles;
-  P->words = static_cast<int>((P->span + 31) / 32);
-  P->smem = static_cast<size_t>(M) * 16 + static_cast<size_t>(P->words) * 8;
-  return P->smem <= 200 * 1024;
+  // supported or not by the whole layer's ids (a shard's tiles are no
+  // larger), so that the decision and the workspace do not depend on the
+  // shard; the tiles then split this process' ids
+  auto plan = [&](int64_t ids) {
+    P->span = (ids + kSeTiles - 1) / kSeTiles;
+    P->words = static_cast<int>((P->span + 31) / 32);
+    P->smem = static_cast<size_t>(M) * 16 + static_cast<size_t>(P->words) * 8;
+    return P->smem <= 200 * 1024;
+  };
+  if (!plan(D.N())) return false;
+  return plan(D.shard_hi() - D.shard_lo());
 }
 
 // workspace words: the two scratch counters (cleared before the call), then

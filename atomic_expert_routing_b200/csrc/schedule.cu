@@ -1208,6 +1208,59 @@ cudaError_t launch_schedule_windows(const Dims& D, const int32_t* idx, const flo
 }
 
 namespace {
+// First position of the sorted ids uniq[0, n) holding an id >= v.
+__device__ __forceinline__ int64_t lower_id(const int32_t* uniq, int64_t n, int64_t v) {
+  int64_t l = 0, h = n;
+  while (l < h) {
+    const int64_t m = (l + h) >> 1;
+    if (uniq[m] < v) l = m + 1; else h = m;
+  }
+  return l;
+}
+
+// T > 0: the window order (window w holds the groups whose first task lies
+// in [w*T, (w+1)*T) and starts at the first of them); the range is widened
+// to whole windows.
+__global__ void k_shard_range(const int32_t* __restrict__ uniq,
+                              const int32_t* __restrict__ group_off,
+                              const int32_t* __restrict__ counts, int64_t T, int64_t lo,
+                              int64_t hi, int64_t ucap, int64_t gmax, int64_t B, int64_t M,
+                              int64_t* __restrict__ arange) {
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x != 0) return;
+  int64_t n = counts[0], G = counts[1];
+  n = n < 0 ? 0 : (n > ucap ? ucap : n);
+  G = G < 0 ? 0 : (G > gmax ? gmax : G);
+  const int64_t r0 = lower_id(uniq, n, lo), r1 = lower_id(uniq, n, hi);
+  int64_t a0 = 0, a1 = 0;
+  if (r1 > r0) {
+    const int64_t g0 = r0 / B, g1 = (r1 - 1) / B;  // first and last group of the shard
+    a0 = group_off[g0];
+    a1 = g1 + 1 < G ? group_off[g1 + 1] : M;
+    if (T > 0) {
+      // first task of the window holding task position v: that of the first
+      // group starting at or after the window's start (M if none)
+      auto window_start = [&](int64_t v) {
+        const int64_t w0 = (v / T) * T;
+        int64_t l = 0, h = G;
+        while (l < h) {
+          const int64_t m = (l + h) >> 1;
+          if (group_off[m] >= w0) h = m; else l = m + 1;
+        }
+        return l < G ? static_cast<int64_t>(group_off[l]) : M;
+      };
+      a0 = window_start(a0);
+      // the end of the window holding the last group: the start of the next
+      const int64_t last = group_off[g1];
+      const int64_t next = (last / T + 1) * T;
+      a1 = next >= M ? M : window_start(next);
+    }
+  }
+  arange[0] = a0;
+  arange[1] = a1;
+}
+
 // counts[0] (|U| of the whole batch) and counts[1] replaced by those of the
 // shard's ids [lo, hi): the active ids in U (sorted) between the two bounds.
 __global__ void k_shard_counts(const int32_t* __restrict__ uniq, int32_t* __restrict__ counts,
@@ -1218,19 +1271,19 @@ __global__ void k_shard_counts(const int32_t* __restrict__ uniq, int32_t* __rest
   int64_t n = counts[0];
   if (n < 0) n = 0;
   if (n > ucap) n = ucap;
-  auto lower = [&](int64_t v) {  // first position of U holding an id >= v
-    int64_t l = 0, h = n;
-    while (l < h) {
-      const int64_t m = (l + h) >> 1;
-      if (uniq[m] < v) l = m + 1; else h = m;
-    }
-    return l;
-  };
-  const int64_t u = lower(hi) - lower(lo);
+  const int64_t u = lower_id(uniq, n, hi) - lower_id(uniq, n, lo);
   counts[0] = static_cast<int32_t>(u);
   counts[1] = static_cast<int32_t>((u + B - 1) / B);
 }
 }  // namespace
+
+cudaError_t launch_shard_range(const Dims& D, const int32_t* uniq, const int32_t* group_off,
+                               const int32_t* counts, int64_t T, int64_t* arange,
+                               cudaStream_t s) {
+  OMNI_TRY(launch_k(k_shard_range, 1, 32, 0, s, uniq, group_off, counts, T, D.shard_lo(),
+      D.shard_hi(), D.ucap(), D.gmax(), D.B, D.M(), arange));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_shard_counts(const Dims& D, const int32_t* uniq, int32_t* counts,
                                 cudaStream_t s) {

@@ -309,6 +309,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     import atomic_expert_routing_b200 as omni
+    import atomic_expert_routing_b200.sharded as omni_sharded
     from atomic_expert_routing_b200 import build as libbuild
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -671,11 +672,103 @@ def run_ours(args):
         torch.cuda.empty_cache()
         return out
 
+    def timed_graph(fn, steps, warmup=2):
+        """Mean CUDA-event time of fn captured in a graph, L2 flushed before
+        each replay."""
+        stream = torch.cuda.Stream(device)
+        with torch.cuda.stream(stream):
+            fn(stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                flush.zero_()
+                g.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        del g
+        return ms
+
+    def measure_shards(c, dd, steps):
+        """Expert-sharded forward on this batch, one G-way split at a time:
+        every shard's per-process work (routing, schedule, its own experts'
+        execution into an fp32 partial, the cast) timed alone on this GPU.
+        The job's step is the slowest shard plus one all-reduce of the
+        L x d fp32 partials, which one GPU cannot time: it is estimated from
+        the measured 8-GPU all-reduce bus bandwidth, 725 GB/s."""
+        D = omni.LayerDims.of(c)
+        out = {"workload": c.name, "allreduce_busbw_gbs": 725.0,
+               "note": "per-shard times measured; the all-reduce time is an estimate"}
+        part_bytes = c.L * c.d * 4
+        for G in (2, 4, 8):
+            shard_ms, active = [], []
+            for lo, hi in omni_sharded.shard_ranges(c.N, G):
+                ws = omni.Workspace()
+                counts = omni.new_counts(device)
+                yp = torch.empty((c.L, c.d), dtype=torch.float32, device=device)
+                y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+                Wl, Vl = dd["W"][lo:hi], dd["V"][lo:hi]
+
+                def fwd(stream):
+                    omni.moe_forward_shard(D, dd["x"], dd["Wr"], dd["Wc"], Wl, Vl, lo, hi,
+                                           dd["bias_r"], dd["bias_c"], y_part=yp, counts=counts,
+                                           ws=ws, stream=stream)
+                    omni.cast_output(D, yp, y=y, stream=stream)
+
+                shard_ms.append(timed_graph(fwd, steps))
+                active.append(int(counts[0].item()))
+                del ws, yp, y
+            ar = part_bytes * 2 * (G - 1) / G / (725.0e9) * 1e3
+            out[str(G)] = {"shard_ms": shard_ms, "max_shard_ms": max(shard_ms),
+                           "active_per_shard": active, "allreduce_ms_estimate": ar,
+                           "step_ms_estimate": max(shard_ms) + ar,
+                           "expert_bytes_per_gpu": 2 * c.d * max(active) * c.esize}
+        torch.cuda.empty_cache()
+        return out
+
+    def measure_glu(c, dd, steps):
+        """The gated (SwiGLU) forward of this batch: a third expert matrix U,
+        drawn on the device (timing only), read once per active expert."""
+        D = omni.LayerDims.of(c)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(c.seed + 77)
+        U = (torch.randn((c.N, c.d), generator=gen, device=device, dtype=torch.float32)
+             / np.sqrt(c.d)).to(D.torch_dtype)
+        ws = omni.Workspace()
+        counts = omni.new_counts(device)
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+
+        def fwd(stream):
+            omni.moe_forward(D, dd["x"], dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                             dd["bias_c"], U=U, y=y, counts=counts, ws=ws, stream=stream)
+
+        ms = timed_graph(fwd, steps)
+        na = int(counts[0].item())
+        flops, bytes_ = layer_work(c, na)
+        bytes_ += c.d * na * c.esize  # the U rows
+        del U, ws
+        torch.cuda.empty_cache()
+        return {"ms_per_step": ms, "value": c.L / (ms * 1e-3), "unit": "tokens/s", "n_active": na,
+                "layer_roofline": {"bound": "hbm", "frac": bytes_ / (hbm * 1e9) / (ms * 1e-3),
+                                   "bytes": bytes_}}
+
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
         # the shared dense MLP of the same batch, width F = d
         extra["shared_mlp"] = measure_mlp(cfg, d, cfg.d, max(3, args.steps // 2))
         extra["dense_groups"] = measure_dense_paths(max(3, args.steps // 2))
+        extra["expert_shards"] = measure_shards(cfg, d, 3)
+        extra["glu"] = measure_glu(cfg, d, max(3, args.steps // 2))
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
