@@ -123,14 +123,13 @@ def expert_stage_bytes(cfg, n_active):
 
 # DRAM bytes (read + write) of one expert-stage call, summed over its kernels,
 # from ncu. The full-size stage is too large for a full capture; these values
-# come from a capture of the bf16-prefill-proxy-N256K workload (1716.4 MB per
-# stage call) scaled by the stage's algorithmic bytes (x3.90). Update them
-# whenever the stage's kernels change, else report None.
+# come from one capture per kernel of the bf16-prefill-proxy-N256K workload
+# (1721.3 MB per stage call) scaled by the stage's algorithmic bytes (x3.90).
+# Update them whenever the stage's kernels change, else report None.
 STAGE_TRAFFIC = {
-    # re-captured after every change to the stage's kernels; until then none
-    "bf16-prefill-N1M": (6.69e9, "ncu dram__bytes of bf16-prefill-proxy-N256K (k_act, 2 x k_acc, "
-                                 "2 x k_slice_finish; k_wsort's 3.2 MB from a capture before it "
-                                 "took the first slice's clear), scaled x3.90 by algorithmic bytes"),
+    "bf16-prefill-N1M": (6.713e9, "ncu dram__bytes of bf16-prefill-proxy-N256K, one capture per "
+                                  "kernel (k_wsort_x, k_act, 2 x k_acc, 2 x k_slice_finish), "
+                                  "scaled x3.90 by algorithmic bytes"),
 }
 
 
