@@ -209,6 +209,31 @@ def moe_forward(cfg, inp, tokens=None):
     return {"idx": idx, "gate": gate, "score": score, "sched": sched, "y": y, "rows": rows}
 
 
+def backward(cfg, inp, idx, gate, dy, tokens=None):
+    """Gradients of the routed branch for the loss sum(dy * y), with the
+    forward's routing (idx, gate) fixed; dy [nt, d] float64.  Returns a dict
+    of float64 arrays: dx [nt, d], dW, dV [N, d], dWr [Nr, d], dWc [Nc, d],
+    dbias_r [Nr], dbias_c [Nc] (the parameter gradients of these tokens
+    alone)."""
+    tok = _tokens(cfg, tokens)
+    nt = len(tok)
+    out = {"dx": np.empty((nt, cfg.d), np.float64),
+           "dW": np.zeros((cfg.N, cfg.d), np.float64), "dV": np.zeros((cfg.N, cfg.d), np.float64),
+           "dWr": np.zeros((cfg.Nr, cfg.d), np.float64),
+           "dWc": np.zeros((cfg.Nc, cfg.d), np.float64),
+           "dbias_r": np.zeros(cfg.Nr, np.float64), "dbias_c": np.zeros(cfg.Nc, np.float64)}
+    D = dims(cfg)
+    br = None if inp.get("bias_r") is None else np.ascontiguousarray(inp["bias_r"], np.float32)
+    bc = None if inp.get("bias_c") is None else np.ascontiguousarray(inp["bias_c"], np.float32)
+    _check(lib().oracle_backward(
+        C.byref(D), _p(inp["x"]), _p(inp["Wr"]), _p(inp["Wc"]), _p(br), _p(bc), _p(inp["W"]),
+        _p(inp["V"]), _p(tok), C.c_int64(nt),
+        _p(np.ascontiguousarray(idx, np.int32)), _p(np.ascontiguousarray(gate, np.float64)),
+        _p(np.ascontiguousarray(dy, np.float64)), _p(out["dx"]), _p(out["dW"]), _p(out["dV"]),
+        _p(out["dWr"]), _p(out["dWc"]), _p(out["dbias_r"]), _p(out["dbias_c"])), "backward")
+    return out
+
+
 def shared_mlp(cfg, inp, W1, W2, tokens=None):
     """The shared dense MLP branch: SiLU(x W1^T) W2^T, fp64 [nt, d].  W1 [F, d]
     and W2 [d, F] in the storage layout of ``workloads`` (bf16 as uint16)."""

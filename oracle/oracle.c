@@ -548,6 +548,149 @@ int oracle_shared_mlp(const or_dims* D, int64_t F, const void* x, const void* W1
   return 0;
 }
 
+/* ------------------------------------------------------------------------- */
+/* Backward of the routed branch                                             */
+/* ------------------------------------------------------------------------- */
+
+/* d SiLU / dz = sig(z) * (1 + z * (1 - sig(z))), sig the logistic function. */
+static double silu_grad(double z) {
+  const double sg = 1.0 / (1.0 + exp(-z));
+  return sg * (1.0 + z * (1.0 - sg));
+}
+
+/*
+ * Gradients of the routed branch (the pages train the model [NL 4]; this is
+ * the forward differentiated by the chain rule).  With the forward's routing
+ * fixed (idx: the K experts chosen for each token, gate: the softmax of their
+ * joint scores) and the loss l = sum over t of dy[t] . y[t]:
+ *
+ *   forward, per token t and selected expert e_k = idx[t,k] (i_k = e_k / Nc,
+ *   j_k = e_k % Nc):
+ *     zr = x[t] . Wr^T + br,  zc = x[t] . Wc^T + bc          [NL 2.2]
+ *     lr = zr - LSE(zr),      lc = zc - LSE(zc)              (per-axis log-softmax)
+ *     S_k = lr[i_k] + lc[j_k],  gate_k = exp(S_k) / sum_q exp(S_q)
+ *     a_k = x[t] . W[e_k],  h_k = SiLU(a_k),  y[t] = sum_k gate_k h_k V[e_k]
+ *
+ *   backward, in the reverse order:
+ *     s_k = dy[t] . V[e_k]
+ *     dV[e_k]  += gate_k h_k dy[t]
+ *     dgate_k   = h_k s_k
+ *     da_k      = gate_k s_k SiLU'(a_k)
+ *     dW[e_k]  += da_k x[t],   dx[t] += da_k W[e_k]
+ *     dS_k      = gate_k (dgate_k - sum_q gate_q dgate_q)     (softmax)
+ *     dlr[i_k] += dS_k,        dlc[j_k] += dS_k
+ *     dzr = dlr - softmax(zr) sum_i dlr[i]                     (log-softmax; same for c)
+ *     dWr[i] += dzr[i] x[t],   dbr[i] += dzr[i],   dx[t] += dzr[i] Wr[i]   (same for c)
+ *
+ * The choice of the top-k rows, columns and pairs is piecewise constant in
+ * the inputs: no gradient flows through it.
+ * Row r of idx/gate/dy/dx belongs to token tok[r].  dx [nt x d] is
+ * overwritten; dW, dV [N x d], dWr [Nr x d], dWc [Nc x d], dbr [Nr], dbc [Nc]
+ * are added to.  Parameter gradients are summed token by token in order
+ * (each output column by one thread), so they do not depend on the thread
+ * count.
+ */
+int oracle_backward(const or_dims* D, const void* x, const void* Wr, const void* Wc,
+                    const float* br, const float* bc, const void* W, const void* V,
+                    const int64_t* tok, int64_t nt, const int32_t* idx, const double* gate,
+                    const double* dy, double* dx, double* dW, double* dV, double* dWr,
+                    double* dWc, double* dbr, double* dbc) {
+  const int64_t d = D->d, K = D->K, Nr = D->Nr, Nc = D->Nc;
+  const int64_t M = nt * K;
+  double* h = (double*)malloc(sizeof(double) * (size_t)M);
+  double* da = (double*)malloc(sizeof(double) * (size_t)M);
+  double* dzr = (double*)calloc((size_t)(nt * Nr), sizeof(double));
+  double* dzc = (double*)calloc((size_t)(nt * Nc), sizeof(double));
+  if (!h || !da || !dzr || !dzc) {
+    free(h); free(da); free(dzr); free(dzc);
+    return 1;
+  }
+  /* per token: the scalars of its tasks, the logit gradients, dx */
+#pragma omp parallel
+  {
+    double* xrow = (double*)malloc(sizeof(double) * d);
+    double* wrow = (double*)malloc(sizeof(double) * d);
+    double* vrow = (double*)malloc(sizeof(double) * d);
+    double* zr = (double*)malloc(sizeof(double) * Nr);
+    double* zc = (double*)malloc(sizeof(double) * Nc);
+    double* dg = (double*)malloc(sizeof(double) * K);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nt; ++r) {
+      const int64_t t = tok[r];
+      const double* dyr = dy + r * d;
+      double* dxr = dx + r * d;
+      for (int64_t m = 0; m < d; ++m) dxr[m] = 0.0;
+      load_row(x, D->dtype, t, d, xrow);
+      /* experts */
+      for (int64_t q = 0; q < K; ++q) {
+        const int64_t e = idx[r * K + q];
+        load_row(V, D->dtype, e, d, vrow);
+        load_row(W, D->dtype, e, d, wrow);
+        const double sk = dot(dyr, vrow, d);
+        const double a = dot(xrow, wrow, d);
+        h[r * K + q] = silu(a);
+        dg[q] = h[r * K + q] * sk;
+        da[r * K + q] = gate[r * K + q] * sk * silu_grad(a);
+        for (int64_t m = 0; m < d; ++m) dxr[m] += da[r * K + q] * wrow[m];
+      }
+      /* gate = softmax of the selected joint scores */
+      double gdg = 0.0;
+      for (int64_t q = 0; q < K; ++q) gdg += gate[r * K + q] * dg[q];
+      double* dlr = dzr + r * Nr;
+      double* dlc = dzc + r * Nc;
+      for (int64_t q = 0; q < K; ++q) {
+        const int64_t e = idx[r * K + q];
+        const double dS = gate[r * K + q] * (dg[q] - gdg);
+        dlr[e / Nc] += dS;
+        dlc[e % Nc] += dS;
+      }
+      /* per-axis log-softmax, then the projections */
+      axis_logits(x, Wr, br, D->dtype, t, d, Nr, xrow, wrow, zr);
+      axis_logits(x, Wc, bc, D->dtype, t, d, Nc, xrow, wrow, zc);
+      log_softmax(zr, Nr);
+      log_softmax(zc, Nc);
+      double sr = 0.0, sc = 0.0;
+      for (int64_t i = 0; i < Nr; ++i) sr += dlr[i];
+      for (int64_t j = 0; j < Nc; ++j) sc += dlc[j];
+      for (int64_t i = 0; i < Nr; ++i) dlr[i] -= exp(zr[i]) * sr;
+      for (int64_t j = 0; j < Nc; ++j) dlc[j] -= exp(zc[j]) * sc;
+      load_row(x, D->dtype, t, d, xrow);
+      for (int64_t i = 0; i < Nr; ++i) {
+        load_row(Wr, D->dtype, i, d, wrow);
+        for (int64_t m = 0; m < d; ++m) dxr[m] += dlr[i] * wrow[m];
+      }
+      for (int64_t j = 0; j < Nc; ++j) {
+        load_row(Wc, D->dtype, j, d, wrow);
+        for (int64_t m = 0; m < d; ++m) dxr[m] += dlc[j] * wrow[m];
+      }
+    }
+    free(xrow); free(wrow); free(vrow); free(zr); free(zc); free(dg);
+  }
+  /* parameter gradients, token by token in order; one thread per column */
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < d; ++m) {
+    for (int64_t r = 0; r < nt; ++r) {
+      const double xm = elem(x, D->dtype, tok[r] * d + m);
+      const double dym = dy[r * d + m];
+      for (int64_t q = 0; q < K; ++q) {
+        const int64_t e = idx[r * K + q];
+        dV[e * d + m] += gate[r * K + q] * h[r * K + q] * dym;
+        dW[e * d + m] += da[r * K + q] * xm;
+      }
+      for (int64_t i = 0; i < Nr; ++i) dWr[i * d + m] += dzr[r * Nr + i] * xm;
+      for (int64_t j = 0; j < Nc; ++j) dWc[j * d + m] += dzc[r * Nc + j] * xm;
+    }
+  }
+  for (int64_t r = 0; r < nt; ++r) {
+    if (dbr)
+      for (int64_t i = 0; i < Nr; ++i) dbr[i] += dzr[r * Nr + i];
+    if (dbc)
+      for (int64_t j = 0; j < Nc; ++j) dbc[j] += dzc[r * Nc + j];
+  }
+  free(h); free(da); free(dzr); free(dzc);
+  return 0;
+}
+
 /* Threads an OpenMP region of this library uses (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

@@ -25,6 +25,24 @@ PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 
 # (name, text of oracle.c, its replacement); each text occurs exactly once
 MUTANTS = [
+    # backward
+    ("bwd-silu-grad-first-factor-only", "return sg * (1.0 + z * (1.0 - sg));", "return sg;"),
+    ("bwd-softmax-drops-mean", "const double dS = gate[r * K + q] * (dg[q] - gdg);",
+     "const double dS = gate[r * K + q] * dg[q];"),
+    ("bwd-dV-without-gate", "dV[e * d + m] += gate[r * K + q] * h[r * K + q] * dym;",
+     "dV[e * d + m] += h[r * K + q] * dym;"),
+    ("bwd-da-without-gate", "da[r * K + q] = gate[r * K + q] * sk * silu_grad(a);",
+     "da[r * K + q] = sk * silu_grad(a);"),
+    ("bwd-dx-through-V", "for (int64_t m = 0; m < d; ++m) dxr[m] += da[r * K + q] * wrow[m];",
+     "for (int64_t m = 0; m < d; ++m) dxr[m] += da[r * K + q] * vrow[m];"),
+    ("bwd-column-of-row-index", "dlc[e % Nc] += dS;", "dlc[e / Nr % Nc] += dS;"),
+    ("bwd-dWr-times-dy", "for (int64_t i = 0; i < Nr; ++i) dWr[i * d + m] += dzr[r * Nr + i] * xm;",
+     "for (int64_t i = 0; i < Nr; ++i) dWr[i * d + m] += dzr[r * Nr + i] * dym;"),
+    ("bwd-router-dx-dropped",
+     "for (int64_t m = 0; m < d; ++m) dxr[m] += dlc[j] * wrow[m];",
+     "for (int64_t m = 0; m < d; ++m) dxr[m] += 0.0 * wrow[m];"),
+    ("bwd-bias-c-from-row-axis", "for (int64_t j = 0; j < Nc; ++j) dbc[j] += dzc[r * Nc + j];",
+     "for (int64_t j = 0; j < Nc; ++j) dbc[j] += dzr[r * Nr + j % Nr];"),
     # shared dense MLP branch
     ("mlp-silu-on-the-output", "y[r * d + j] = dot(h, w2, F);",
      "y[r * d + j] = silu(dot(h, w2, F));"),

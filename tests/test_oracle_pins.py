@@ -569,3 +569,106 @@ def test_gated_expert_linear_in_U_and_orders_agree():
     yt, _ = O.forward_token(cfg, dict(h, U=U), idx, gate)
     np.testing.assert_allclose(yt, y1, rtol=1e-12, atol=1e-13)
     assert np.abs(y1).max() > 0
+
+
+# ------------------------------------------------------------------ backward
+#
+# The gradients are pinned to the oracle's forward, not to a second copy of
+# their formulas: for the loss l = sum(dy * y), the central difference of l
+# along a direction v of one input, (l(p + e v) - l(p - e v)), must equal
+# <grad, p+ - p-> up to terms of third order in e, where p+- are the stored
+# (fp32) perturbed inputs.  The selected sets must not change between the
+# two evaluations (the selection is piecewise constant); the test asserts it.
+
+BWD_CFGS = [
+    WL.Config("bwd-tiny", L=4, d=8, Nr=5, Nc=4, k=3, K=3, B=2, dtype=WL.F32, seed=3),
+    WL.Config("bwd-small", L=12, d=24, Nr=9, Nc=7, k=4, K=4, B=3, dtype=WL.F32, seed=4),
+]
+
+
+def _loss(cfg, h, dy):
+    res = O.moe_forward(cfg, h)
+    return float(np.sum(dy * res["y"])), res["idx"]
+
+
+def _bias_inputs(cfg):
+    h = WL.make_inputs(cfg)
+    rng = np.random.default_rng(cfg.seed)
+    h["bias_r"] = (0.3 * rng.standard_normal(cfg.Nr)).astype(np.float32)
+    h["bias_c"] = (0.3 * rng.standard_normal(cfg.Nc)).astype(np.float32)
+    return h
+
+
+@pytest.mark.parametrize("cfg", BWD_CFGS, ids=lambda c: c.name)
+@pytest.mark.parametrize("name,grad", [("x", "dx"), ("W", "dW"), ("V", "dV"), ("Wr", "dWr"),
+                                       ("Wc", "dWc"), ("bias_r", "dbias_r"),
+                                       ("bias_c", "dbias_c")])
+def test_backward_matches_central_differences_of_the_forward(cfg, name, grad):
+    h = _bias_inputs(cfg)
+    rng = np.random.default_rng(100 + len(name))
+    dy = rng.standard_normal((cfg.L, cfg.d))
+    idx, gate, _ = O.route(cfg, h)
+    g = O.backward(cfg, h, idx, gate, dy)[grad]
+    base = h[name].astype(np.float64)
+    for trial in range(3):
+        v = rng.standard_normal(base.shape)
+        eps = 1e-4 * max(1.0, float(np.abs(base).max()))
+        hp, hm = dict(h), dict(h)
+        hp[name] = (base + eps * v).astype(np.float32)
+        hm[name] = (base - eps * v).astype(np.float32)
+        lp, ip = _loss(cfg, hp, dy)
+        lm, im = _loss(cfg, hm, dy)
+        # the same selected sets (their order may swap where scores are close;
+        # y does not depend on it)
+        same = np.sort(idx, axis=1)
+        assert np.array_equal(np.sort(ip, axis=1), same), "routing moved"
+        assert np.array_equal(np.sort(im, axis=1), same), "routing moved"
+        step = hp[name].astype(np.float64) - hm[name].astype(np.float64)
+        pred = float(np.sum(g * step))
+        fd = lp - lm
+        scale = float(np.sum(np.abs(g * step))) + 1e-30
+        assert abs(fd - pred) <= 2e-5 * scale, (name, trial, fd, pred)
+
+
+def test_backward_of_a_single_token_and_expert_in_closed_form():
+    """K = 1: the gate is 1 and its gradient vanishes, so the router receives
+    nothing; y = SiLU(a) V[e] with a = x.W[e], hence dV[e] = SiLU(a) dy,
+    dW[e] = (dy.V[e]) SiLU'(a) x, dx = (dy.V[e]) SiLU'(a) W[e], with
+    SiLU'(a) = s(a)(1 + a(1 - s(a))) for the logistic s (scipy's expit)."""
+    cfg = WL.Config("bwd-k1", L=1, d=6, Nr=3, Nc=2, k=1, K=1, B=1, dtype=WL.F32, seed=5)
+    h = WL.make_inputs(cfg)
+    idx, gate, _ = O.route(cfg, h)
+    e = int(idx[0, 0])
+    dy = np.arange(1.0, cfg.d + 1.0)[None, :] / 7.0
+    r = O.backward(cfg, h, idx, gate, dy)
+    x = h["x"][0].astype(np.float64)
+    w = h["W"][e].astype(np.float64)
+    v = h["V"][e].astype(np.float64)
+    a = float(x @ w)
+    sig = float(expit(a))
+    s1 = sig * (1.0 + a * (1.0 - sig))
+    sv = float(dy[0] @ v)
+    np.testing.assert_allclose(r["dV"][e], a * sig * dy[0], rtol=1e-12)
+    np.testing.assert_allclose(r["dW"][e], sv * s1 * x, rtol=1e-12)
+    np.testing.assert_allclose(r["dx"][0], sv * s1 * w, rtol=1e-12, atol=1e-15)
+    assert not np.delete(r["dW"], e, axis=0).any() and not np.delete(r["dV"], e, axis=0).any()
+    assert np.all(np.abs(r["dWr"]) < 1e-15) and np.all(np.abs(r["dWc"]) < 1e-15)
+
+
+def test_backward_invariants():
+    """Softmax shift invariance: the bias gradients of each axis sum to zero;
+    rows of experts no token chose get no gradient; the gradients are linear
+    in dy."""
+    cfg = BWD_CFGS[1]
+    h = _bias_inputs(cfg)
+    idx, gate, _ = O.route(cfg, h)
+    rng = np.random.default_rng(7)
+    dy1, dy2 = rng.standard_normal((2, cfg.L, cfg.d))
+    r1 = O.backward(cfg, h, idx, gate, dy1)
+    r2 = O.backward(cfg, h, idx, gate, dy2)
+    r12 = O.backward(cfg, h, idx, gate, dy1 + 2.0 * dy2)
+    for key in r1:
+        np.testing.assert_allclose(r12[key], r1[key] + 2.0 * r2[key], rtol=1e-10, atol=1e-12)
+    assert abs(r1["dbias_r"].sum()) < 1e-12 and abs(r1["dbias_c"].sum()) < 1e-12
+    idle = np.setdiff1d(np.arange(cfg.N), idx)
+    assert not r1["dW"][idle].any() and not r1["dV"][idle].any()
