@@ -21,12 +21,13 @@ import torch
 from . import _lib
 from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_DENSE_TENSOR_CORES, OMNI_FLAG_ROUTER_SIMT,
                    OMNI_FLAG_STAGED_SMALL,
-                   OMNI_WS_EXPERT, OMNI_WS_FUSED,
+                   OMNI_WS_BACKWARD, OMNI_WS_EXPERT, OMNI_WS_FUSED,
                    OMNI_WS_ROUTE, OMNI_WS_SCHEDULE, OmniError)
 
 __all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",
            "token_centric_forward", "new_counts", "OmniError", "workspace_size", "wait_selftest",
-           "shared_mlp", "moe_mlp_forward", "mlp_workspace_size"]
+           "shared_mlp", "moe_mlp_forward", "mlp_workspace_size", "expert_forward_noalloc",
+           "moe_forward_shard", "cast_output", "moe_backward"]
 
 
 @dataclass(frozen=True)
@@ -346,6 +347,42 @@ def cast_output(D: LayerDims, src, *, y=None, stream=None):
     _lib.check("omni_cast_output", _lib.load().omni_cast_output(
         C.byref(dd), _ptr(src), _ptr(y), _stream(stream)))
     return y
+
+
+def moe_backward(D: LayerDims, x, Wr, Wc, W, V, idx, gate, dy, *, grads=None, bias=True,
+                 counts=None, ws=None, stream=None):
+    """Gradients of the loss sum(dy * y) with the forward's routing (idx,
+    gate) fixed.  grads (optional): a dict of fp32 tensors to add the
+    parameter gradients to -- dW, dV [N, d], dWr [Nr, d], dWc [Nc, d],
+    dbias_r [Nr], dbias_c [Nc] (missing ones are created as zeros; with
+    bias=False the bias gradients are skipped) -- and dx [L, d] (fp32,
+    overwritten).  Returns the dict."""
+    f32 = torch.float32
+    _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, V=V, idx=idx, gate=gate, counts=counts)
+    _expect("dy", dy, D.L * D.d, D.torch_dtype)
+    dev = _device(x)
+    shapes = {"dx": (D.L, D.d), "dW": (D.N, D.d), "dV": (D.N, D.d), "dWr": (D.Nr, D.d),
+              "dWc": (D.Nc, D.d), "dbias_r": (D.Nr,), "dbias_c": (D.Nc,)}
+    g = dict(grads or {})
+    for name, shape in shapes.items():
+        if name.startswith("dbias") and not bias:
+            g.pop(name, None)
+            continue
+        if name not in g:
+            g[name] = (torch.empty if name == "dx" else torch.zeros)(shape, dtype=f32, device=dev)
+        n = 1
+        for v in shape:
+            n *= v
+        _expect(name, g[name], n, f32)
+    if counts is None:
+        counts = new_counts(dev)
+    wsp, n = _ws(D, OMNI_WS_BACKWARD, dev, ws)
+    dd = D.c()
+    _lib.check("omni_moe_backward", _lib.load().omni_moe_backward(
+        C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(W), _ptr(V), _ptr(idx), _ptr(gate),
+        _ptr(dy), _ptr(g["dx"]), _ptr(g["dW"]), _ptr(g["dV"]), _ptr(g["dWr"]), _ptr(g["dWc"]),
+        _ptr(g.get("dbias_r")), _ptr(g.get("dbias_c")), _ptr(counts), wsp, n, _stream(stream)))
+    return g
 
 
 def mlp_workspace_size(D: LayerDims, F: int, with_routed: bool) -> int:

@@ -113,6 +113,12 @@ size_t ws_size(const Dims& D, int which) {
     case OMNI_WS_SCHEDULE: c.take<char>(omni::schedule_ws_bytes(D)); break;
     case OMNI_WS_EXPERT: c.take<char>(omni::expert_ws_bytes(D)); break;
     case OMNI_WS_FUSED: carve_fused(D, c); break;
+    case OMNI_WS_BACKWARD: {
+      size_t b = 0;
+      omni::carve_backward(D, nullptr, &b);
+      c.take<char>(b);
+      break;
+    }
     default: break;
   }
   return c.off;
@@ -228,7 +234,7 @@ int omni_workspace_size(const omni_dims* dims, int which, size_t* bytes) {
   Dims D;
   int rc = check_dims(dims, &D);
   if (rc != OMNI_OK) return rc;
-  if (bytes == nullptr || which < OMNI_WS_ROUTE || which > OMNI_WS_SELECT) return OMNI_ERR_INVALID_ARG;
+  if (bytes == nullptr || which < OMNI_WS_ROUTE || which > OMNI_WS_BACKWARD) return OMNI_ERR_INVALID_ARG;
   *bytes = ws_size(D, which);
   return OMNI_OK;
 }
@@ -567,6 +573,27 @@ int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* str
   if (!tensors_ok(t16, 2)) return OMNI_ERR_INVALID_ARG;
   if (D.dtype == OMNI_BF16 && static_cast<const void*>(src) == y) return OMNI_ERR_INVALID_ARG;
   return cuda_status(omni::launch_cast_output(D, src, y, static_cast<cudaStream_t>(stream)));
+}
+
+int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                      const void* W, const void* V, const int32_t* idx, const float* gate,
+                      const void* dy, float* dx, float* dW, float* dV, float* dWr, float* dWc,
+                      float* dbias_r, float* dbias_c, int32_t* counts, void* ws, size_t ws_bytes,
+                      void* stream) {
+  omni::CallRange range("omni_moe_backward");
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (D.dtype != OMNI_BF16) return OMNI_ERR_UNSUPPORTED;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, Wr, Wc, W, V, dy, dx, dW, dV, dWr, dWc};
+  if (!tensors_ok(t16, 11) || idx == nullptr || gate == nullptr || counts == nullptr ||
+      !al(dbias_r, 4) || !al(dbias_c, 4))
+    return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_BACKWARD, ws, ws_bytes)) != OMNI_OK) return rc;
+  return cuda_status(omni::launch_backward(D, x, Wr, Wc, W, V, idx, gate, dy, dx, dW, dV, dWr,
+                                           dWc, dbias_r, dbias_c, counts, ws,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -235,5 +235,28 @@ cudaError_t launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int nk, c
   return cudaGetLastError();
 }
 
+// One GEMM D = A B^T (A [rows x K], B [cols x K], bf16, K-major, rows of K
+// elements 16-byte aligned) with epilogue epi: 256-wide B tiles when they
+// still give every SM a tile, else 128-wide.
+template <class Epi>
+cudaError_t gemm_bf16(const void* A, const void* Bm, int64_t rows, int64_t cols, int64_t K,
+                      const Epi& epi, int32_t* status, cudaStream_t s) {
+  const int64_t mt = (rows + TC_BM - 1) / TC_BM;
+  const int nk = static_cast<int>((K + TC_BK - 1) / TC_BK);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  CUtensorMap a, b;
+  if (!make_map(&a, A, rows, K, TC_BM)) return cudaErrorInvalidValue;
+  if (mt * ((cols + 255) / 256) >= sms) {
+    if (!make_map(&b, Bm, cols, K, 256)) return cudaErrorInvalidValue;
+    DenseTiles<256> T{static_cast<int>(mt), static_cast<int>((cols + 255) / 256)};
+    return launch_gemm_tc<256>(a, b, nk, T, mt * T.nt, epi, status, s);
+  }
+  if (!make_map(&b, Bm, cols, K, 128)) return cudaErrorInvalidValue;
+  DenseTiles<128> T{static_cast<int>(mt), static_cast<int>((cols + 127) / 128)};
+  return launch_gemm_tc<128>(a, b, nk, T, mt * T.nt, epi, status, s);
+}
+
 }  // namespace tc
 }  // namespace omni

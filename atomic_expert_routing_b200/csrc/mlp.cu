@@ -98,32 +98,6 @@ struct AddToOutput {
   }
 };
 
-int sm_count_mlp() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
-
-// One GEMM D = A B^T (A [rows x K], B [cols x K]) with epilogue epi: 256-wide
-// B tiles when they still give every SM a tile, else 128-wide.
-template <class Epi>
-cudaError_t gemm(const void* A, const void* Bm, int64_t rows, int64_t cols, int64_t K,
-                 const Epi& epi, int32_t* status, cudaStream_t s) {
-  const int64_t mt = (rows + TC_BM - 1) / TC_BM;
-  const int nk = static_cast<int>((K + TC_BK - 1) / TC_BK);
-  CUtensorMap a, b;
-  if (!make_map(&a, A, rows, K, TC_BM)) return cudaErrorInvalidValue;
-  if (mt * ((cols + 255) / 256) >= sm_count_mlp()) {
-    if (!make_map(&b, Bm, cols, K, 256)) return cudaErrorInvalidValue;
-    DenseTiles<256> T{static_cast<int>(mt), static_cast<int>((cols + 255) / 256)};
-    return launch_gemm_tc<256>(a, b, nk, T, mt * T.nt, epi, status, s);
-  }
-  if (!make_map(&b, Bm, cols, K, 128)) return cudaErrorInvalidValue;
-  DenseTiles<128> T{static_cast<int>(mt), static_cast<int>((cols + 127) / 128)};
-  return launch_gemm_tc<128>(a, b, nk, T, mt * T.nt, epi, status, s);
-}
-
 }  // namespace
 
 size_t mlp_ws_bytes(const Dims& D, int64_t F) {
@@ -136,9 +110,9 @@ cudaError_t launch_shared_mlp(const Dims& D, int64_t F, const void* x, const voi
   if (D.L == 0) return cudaSuccess;
   if (D.dtype != OMNI_BF16 || encode_fn() == nullptr) return cudaErrorNotSupported;
   __nv_bfloat16* H = static_cast<__nv_bfloat16*>(ws);
-  OMNI_TRY(gemm(x, W1, D.L, F, D.d, SiluToHidden{H, F, static_cast<int>(D.L), static_cast<int>(F)},
-                status, s));
-  return gemm(H, W2, D.L, D.d, F,
+  OMNI_TRY(gemm_bf16(x, W1, D.L, F, D.d,
+                     SiluToHidden{H, F, static_cast<int>(D.L), static_cast<int>(F)}, status, s));
+  return gemm_bf16(H, W2, D.L, D.d, F,
               AddToOutput{static_cast<__nv_bfloat16*>(y), D.d, static_cast<int>(D.L),
                           static_cast<int>(D.d), accumulate ? 1 : 0},
               status, s);

@@ -123,6 +123,7 @@ typedef struct omni_dims {
 #define OMNI_WS_FUSED 3
 #define OMNI_WS_TOKEN 4
 #define OMNI_WS_SELECT 5
+#define OMNI_WS_BACKWARD 6
 
 /* Bytes of workspace the call `which` needs for `dims` (0 is possible). */
 int omni_workspace_size(const omni_dims* dims, int which, size_t* bytes);
@@ -351,6 +352,39 @@ int omni_moe_forward_shard(const omni_dims* dims, int64_t e_lo, int64_t e_hi, co
  * storage is OMNI_ERR_INVALID_ARG.
  */
 int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* stream);
+
+/*
+ * Backward of the routed branch: the gradients of the loss sum(dy * y) with
+ * the forward's routing fixed (the pages train the model [NL 4]; this is the
+ * forward differentiated by the chain rule).  Per task (t, k), e = idx[t,k],
+ * a = x[t] . W[e], h = SiLU(a), s = dy[t] . V[e]:
+ *   dV[e] += gate h dy[t];  dW[e] += da x[t];  dx[t] += da W[e],
+ *   with da = gate s SiLU'(a);
+ * through gate = softmax of the selected joint scores S_k = lr[i_k] + lc[j_k]
+ * and the per-axis log-softmax: dS_k = gate_k (h_k s_k - sum_q gate_q h_q s_q)
+ * added to row logit i_k and column logit j_k; then
+ *   dx += dZ [Wr; Wc],  [dWr; dWc] += dZ^T x,  dbias += column sums of dZ.
+ * The selection of the experts is piecewise constant: no gradient flows
+ * through it.
+ *   x, Wr, Wc, W, V: the forward's inputs; idx, gate: its routing outputs
+ *     ([L x K], as omni_moe_forward's idx_out / gate_out); dy [L x d] in the
+ *     storage type.
+ *   dx [L x d] fp32: overwritten.
+ *   dW, dV [N x d], dWr [Nr x d], dWc [Nc x d], dbias_r [Nr], dbias_c [Nc]
+ *     (the two biases nullable) fp32: added to (rows of experts no token
+ *     chose are not touched), so that gradients accumulate across calls.
+ *   counts[0], counts[1]: the active experts; counts[2]: status bits.
+ *   ws: omni_workspace_size(dims, OMNI_WS_BACKWARD).
+ * All arrays 16-byte aligned.  Router gradients go through tensor-core
+ * products of bf16 operands (dZ rounded to bf16, fp32 accumulation); the
+ * experts' gradients are fp32 throughout.  bf16 storage only (fp32 storage
+ * returns OMNI_ERR_UNSUPPORTED); the other checks as omni_expert_forward.
+ */
+int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
+                      const void* W, const void* V, const int32_t* idx, const float* gate,
+                      const void* dy, float* dx, float* dW, float* dV, float* dWr, float* dWc,
+                      float* dbias_r, float* dbias_c, int32_t* counts, void* ws, size_t ws_bytes,
+                      void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* omni_status_string(int status);

@@ -307,3 +307,32 @@ def test_cast_output_host_checks(lib):
     # fp32 in place: nothing to do, no launch
     F = _dims(dtype=_lib.OMNI_F32)
     assert lib.omni_cast_output(C.byref(F), fake, fake, None) == _lib.OMNI_OK
+
+
+def test_backward_host_checks(lib):
+    """omni_moe_backward: bf16 storage only; null or misaligned arrays are
+    invalid; the workspace is checked; an empty batch is a no-op."""
+    fake = C.c_void_p(4096)
+    odd = C.c_void_p(4096 + 4)
+    B16 = _dims(dtype=_lib.OMNI_BF16)
+
+    def call(dims, **over):
+        names = ["x", "Wr", "Wc", "W", "V", "idx", "gate", "dy", "dx", "dW", "dV", "dWr", "dWc",
+                 "dbias_r", "dbias_c", "counts"]
+        args = {n: fake for n in names}
+        args["dbias_r"] = args["dbias_c"] = None
+        args.update(over)
+        ws = over.pop("ws", None)
+        return lib.omni_moe_backward(C.byref(dims), *[args[n] for n in names], ws,
+                                     1 << 30 if ws is not None else 0, None)
+
+    assert call(_dims(dtype=_lib.OMNI_F32)) == _lib.OMNI_ERR_UNSUPPORTED
+    assert call(B16, dy=None) == _lib.OMNI_ERR_INVALID_ARG
+    assert call(B16, dW=odd) == _lib.OMNI_ERR_INVALID_ARG
+    assert call(B16, counts=None) == _lib.OMNI_ERR_INVALID_ARG
+    assert call(B16, dbias_r=C.c_void_p(4096 + 2)) == _lib.OMNI_ERR_INVALID_ARG
+    assert call(B16) == _lib.OMNI_ERR_WORKSPACE
+    assert call(_dims(L=0, dtype=_lib.OMNI_BF16), x=None) == _lib.OMNI_OK
+    n = C.c_size_t(0)
+    assert lib.omni_workspace_size(C.byref(B16), _lib.OMNI_WS_BACKWARD, C.byref(n)) == 0
+    assert n.value > 0
