@@ -350,13 +350,14 @@ def cast_output(D: LayerDims, src, *, y=None, stream=None):
 
 
 def moe_backward(D: LayerDims, x, Wr, Wc, W, V, idx, gate, dy, *, grads=None, bias=True,
-                 counts=None, ws=None, stream=None):
+                 accumulate=True, counts=None, ws=None, stream=None):
     """Gradients of the loss sum(dy * y) with the forward's routing (idx,
-    gate) fixed.  grads (optional): a dict of fp32 tensors to add the
-    parameter gradients to -- dW, dV [N, d], dWr [Nr, d], dWc [Nc, d],
-    dbias_r [Nr], dbias_c [Nc] (missing ones are created as zeros; with
-    bias=False the bias gradients are skipped) -- and dx [L, d] (fp32,
-    overwritten).  Returns the dict."""
+    gate) fixed.  grads (optional): a dict of fp32 tensors for the parameter
+    gradients -- dW, dV [N, d], dWr [Nr, d], dWc [Nc, d], dbias_r [Nr],
+    dbias_c [Nc] (missing ones are created as zeros; with bias=False the bias
+    gradients are skipped), added to (accumulate) or overwritten (rows of
+    dW, dV of experts no token chose untouched either way) -- and dx [L, d]
+    (fp32, overwritten).  Returns the dict."""
     f32 = torch.float32
     _expect_io(D, x=x, Wr=Wr, Wc=Wc, W=W, V=V, idx=idx, gate=gate, counts=counts)
     _expect("dy", dy, D.L * D.d, D.torch_dtype)
@@ -381,7 +382,8 @@ def moe_backward(D: LayerDims, x, Wr, Wc, W, V, idx, gate, dy, *, grads=None, bi
     _lib.check("omni_moe_backward", _lib.load().omni_moe_backward(
         C.byref(dd), _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(W), _ptr(V), _ptr(idx), _ptr(gate),
         _ptr(dy), _ptr(g["dx"]), _ptr(g["dW"]), _ptr(g["dV"]), _ptr(g["dWr"]), _ptr(g["dWc"]),
-        _ptr(g.get("dbias_r")), _ptr(g.get("dbias_c")), _ptr(counts), wsp, n, _stream(stream)))
+        _ptr(g.get("dbias_r")), _ptr(g.get("dbias_c")), 1 if accumulate else 0, _ptr(counts),
+        wsp, n, _stream(stream)))
     return g
 
 

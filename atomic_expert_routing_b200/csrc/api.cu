@@ -578,8 +578,8 @@ int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* str
 int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                       const void* W, const void* V, const int32_t* idx, const float* gate,
                       const void* dy, float* dx, float* dW, float* dV, float* dWr, float* dWc,
-                      float* dbias_r, float* dbias_c, int32_t* counts, void* ws, size_t ws_bytes,
-                      void* stream) {
+                      float* dbias_r, float* dbias_c, int accumulate, int32_t* counts, void* ws,
+                      size_t ws_bytes, void* stream) {
   omni::CallRange range("omni_moe_backward");
   Dims D;
   int rc = check_dims(dims, &D);
@@ -592,7 +592,7 @@ int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, cons
     return OMNI_ERR_INVALID_ARG;
   if ((rc = ws_ok(D, OMNI_WS_BACKWARD, ws, ws_bytes)) != OMNI_OK) return rc;
   return cuda_status(omni::launch_backward(D, x, Wr, Wc, W, V, idx, gate, dy, dx, dW, dV, dWr,
-                                           dWc, dbias_r, dbias_c, counts, ws,
+                                           dWc, dbias_r, dbias_c, accumulate != 0, counts, ws,
                                            static_cast<cudaStream_t>(stream)));
 }
 

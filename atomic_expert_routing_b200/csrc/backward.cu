@@ -64,12 +64,17 @@ __device__ __forceinline__ void axpy8(float c, uint4 v, float* acc) {
   }
 }
 
-// o[0..8) += acc (fp32, 32-byte aligned)
-__device__ __forceinline__ void add8(float* o, const float* acc) {
+// o[0..8) += acc, or = acc without reading o (add == false); fp32,
+// 32-byte aligned
+__device__ __forceinline__ void put8(float* o, const float* acc, bool add) {
   float4* p = reinterpret_cast<float4*>(o);
-  float4 u = p[0], w = p[1];
-  u.x += acc[0]; u.y += acc[1]; u.z += acc[2]; u.w += acc[3];
-  w.x += acc[4]; w.y += acc[5]; w.z += acc[6]; w.w += acc[7];
+  float4 u = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  float4 w = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  if (add) {
+    const float4 a = p[0], b = p[1];
+    u.x += a.x; u.y += a.y; u.z += a.z; u.w += a.w;
+    w.x += b.x; w.y += b.y; w.z += b.z; w.w += b.w;
+  }
   p[0] = u;
   p[1] = w;
 }
@@ -82,7 +87,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
                  const int32_t* __restrict__ task_token, const int32_t* __restrict__ task_expert,
                  const float* __restrict__ task_gate, const int32_t* __restrict__ group_off,
                  const int32_t* __restrict__ counts, const int32_t* __restrict__ idx, int64_t L,
-                 int K, int64_t N, int d, int64_t gmax, float* __restrict__ dW,
+                 int K, int64_t N, int d, int64_t gmax, int accumulate, float* __restrict__ dW,
                  float* __restrict__ dV, float* __restrict__ da_slot,
                  float* __restrict__ dg_slot, int32_t* status) {
   pdl_wait();
@@ -173,8 +178,11 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
           axpy8(cvj, reinterpret_cast<const uint4*>(dy + t * d)[v], av);
         }
         if (v < nvec) {
-          add8(dW + e * d + static_cast<int64_t>(v) * 8, aw);
-          add8(dV + e * d + static_cast<int64_t>(v) * 8, av);
+          // the expert's first 32 tasks overwrite its rows unless the call
+          // accumulates; later ones add to what the first wrote
+          const bool add = accumulate != 0 || c0 > a0;
+          put8(dW + e * d + static_cast<int64_t>(v) * 8, aw, add);
+          put8(dV + e * d + static_cast<int64_t>(v) * 8, av, add);
         }
       }
     }
@@ -275,14 +283,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// GEMM epilogues: D[row, col] += acc (fp32; rows of ld floats), rows below
-// `split` in D0 and the others in D1 (row - split).
+// GEMM epilogue: D[row, col] += acc (accumulate != 0) or = acc (fp32; rows
+// of ld floats), rows below `split` in D0 and the others in D1 (row - split).
 struct AddF32Split {
   static constexpr size_t kStageBytes = 0;
   float* D0;
   float* D1;
   int64_t split, ld;
-  int rows, cols;
+  int rows, cols, accumulate;
   __device__ __forceinline__ void operator()(int, int a0, int b0, int r, int c,
                                              const uint32_t* v, float*) const {
     const int row = a0 + r;
@@ -293,17 +301,18 @@ struct AddF32Split {
     if (col + 32 <= cols) {
 #pragma unroll
       for (int q = 0; q < 32; q += 4) {
-        float4 u = *reinterpret_cast<float4*>(o + q);
-        u.x += __uint_as_float(v[q]);
-        u.y += __uint_as_float(v[q + 1]);
-        u.z += __uint_as_float(v[q + 2]);
-        u.w += __uint_as_float(v[q + 3]);
+        float4 u = make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+                               __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+        if (accumulate) {
+          const float4 a = *reinterpret_cast<const float4*>(o + q);
+          u.x += a.x; u.y += a.y; u.z += a.z; u.w += a.w;
+        }
         *reinterpret_cast<float4*>(o + q) = u;
       }
     } else {
 #pragma unroll
       for (int q = 0; q < 32; ++q)
-        if (col + q < cols) o[q] += __uint_as_float(v[q]);
+        if (col + q < cols) o[q] = __uint_as_float(v[q]) + (accumulate ? o[q] : 0.0f);
     }
   }
 };
@@ -340,8 +349,8 @@ BwdWs carve_backward(const Dims& D, void* base, size_t* bytes) {
 cudaError_t launch_backward(const Dims& D, const void* x, const void* Wr, const void* Wc,
                             const void* W, const void* V, const int32_t* idx, const float* gate,
                             const void* dy, float* dx, float* dW, float* dV, float* dWr,
-                            float* dWc, float* dbr, float* dbc, int32_t* counts, void* ws,
-                            cudaStream_t s) {
+                            float* dWc, float* dbr, float* dbc, bool accumulate,
+                            int32_t* counts, void* ws, cudaStream_t s) {
   if (D.L == 0) return cudaSuccess;
   if (D.dtype != OMNI_BF16 || encode_fn() == nullptr) return cudaErrorNotSupported;
   const BwdWs w = carve_backward(D, ws, nullptr);
@@ -366,10 +375,14 @@ cudaError_t launch_backward(const Dims& D, const void* x, const void* Wr, const 
         static_cast<const bf16*>(W), static_cast<const bf16*>(V), static_cast<const bf16*>(dy),
         static_cast<const int32_t*>(w.task_token), static_cast<const int32_t*>(w.task_expert),
         static_cast<const float*>(w.task_gate), static_cast<const int32_t*>(w.group_off),
-        static_cast<const int32_t*>(counts), idx, D.L, K, D.N(), d, D1.gmax(), dW, dV, w.da, w.dg,
-        status));
+        static_cast<const int32_t*>(counts), idx, D.L, K, D.N(), d, D1.gmax(), accumulate ? 1 : 0,
+        dW, dV, w.da, w.dg, status));
   }
   // 3. per token: dS, the dZ row, the bias gradients, dx (experts)
+  if (!accumulate) {  // the bias gradients are sums of atomic adds
+    if (dbr != nullptr) OMNI_TRY(launch_zero(dbr, static_cast<size_t>(D.Nr), s));
+    if (dbc != nullptr) OMNI_TRY(launch_zero(dbc, static_cast<size_t>(D.Nc), s));
+  }
   {
     const size_t smem = static_cast<size_t>(D.Nr + D.Nc) * sizeof(float);
     cudaError_t err = cudaFuncSetAttribute(k_bwd_token, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -395,10 +408,12 @@ cudaError_t launch_backward(const Dims& D, const void* x, const void* Wr, const 
   OMNI_TRY(transpose(x, D.L, D.d, D.d, w.xT, Lp, Lp));
   // dx [L x d] += dZ [L x Kp] . WrcT [d x Kp]^T
   OMNI_TRY(gemm_bf16(w.dzb, w.WrcT, D.L, D.d, Kp,
-                     AddF32Split{dx, dx, D.L, D.d, static_cast<int>(D.L), d}, status, s));
+                     AddF32Split{dx, dx, D.L, D.d, static_cast<int>(D.L), d, 1}, status, s));
   // [dWr; dWc] [(Nr + Nc) x d] += dZ^T [(Nr + Nc) x Lp] . xT [d x Lp]^T
   return gemm_bf16(w.dzT, w.xT, D.Nr + D.Nc, D.d, Lp,
-                   AddF32Split{dWr, dWc, D.Nr, D.d, static_cast<int>(D.Nr + D.Nc), d}, status, s);
+                   AddF32Split{dWr, dWc, D.Nr, D.d, static_cast<int>(D.Nr + D.Nc), d,
+                               accumulate ? 1 : 0},
+                   status, s);
 }
 
 }  // namespace omni

@@ -200,14 +200,15 @@ struct BwdWs {
 };
 // The workspace's buffers (base == nullptr: sizes only, total in *bytes).
 BwdWs carve_backward(const Dims& D, void* base, size_t* bytes);
-// dx [L x d] fp32 overwritten; dW, dV [N x d], dWr [Nr x d], dWc [Nc x d],
-// dbr [Nr], dbc [Nc] (nullable) fp32 added to.  counts[0], [1]: the active
-// experts (twice: groups of one); counts[2] status bits.
+// dx [L x d] fp32 overwritten; dW, dV [N x d] (active rows), dWr [Nr x d],
+// dWc [Nc x d], dbr [Nr], dbc [Nc] (nullable) fp32 added to (accumulate) or
+// overwritten.  counts[0], [1]: the active experts (twice: groups of one);
+// counts[2] status bits.
 cudaError_t launch_backward(const Dims& D, const void* x, const void* Wr, const void* Wc,
                             const void* W, const void* V, const int32_t* idx, const float* gate,
                             const void* dy, float* dx, float* dW, float* dV, float* dWr,
-                            float* dWc, float* dbr, float* dbc, int32_t* counts, void* ws,
-                            cudaStream_t s);
+                            float* dWc, float* dbr, float* dbc, bool accumulate,
+                            int32_t* counts, void* ws, cudaStream_t s);
 
 // ---- shared dense MLP: y (+)= SiLU(x W1^T) W2^T on the tensor cores ---------
 // bf16 storage only; ws holds the hidden activations H [L x F] (bf16).

@@ -576,6 +576,94 @@ def run_ours(args):
         pipe_ms = t0.elapsed_time(t1) / steps
         return serial_ms, pipe_ms, xh.numel() * xh.element_size(), yh[0].numel() * yh[0].element_size()
 
+    def timed_graph(fn, steps, warmup=2):
+        """Mean CUDA-event time of fn captured in a graph, L2 flushed before
+        each replay."""
+        stream = torch.cuda.Stream(device)
+        with torch.cuda.stream(stream):
+            fn(stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                flush.zero_()
+                g.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        del g
+        return ms
+
+    def measure_backward(c, dd, steps):
+        """The backward of this batch (omni_moe_backward) on the forward's
+        routing, gradients accumulated into fp32 arrays, timed alone after an
+        L2 flush.  Algorithmic bytes: x and dy read; the active rows of W and
+        V read and of dW and dV read and written in fp32; dx written in fp32;
+        the router weights read and their fp32 gradients read and written;
+        the routing read."""
+        D = omni.LayerDims.of(c)
+        idx = torch.empty((c.L, c.K), dtype=torch.int32, device=device)
+        gate = torch.empty((c.L, c.K), dtype=torch.float32, device=device)
+        counts = omni.new_counts(device)
+        omni.moe_forward(D, dd["x"], dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                         dd["bias_c"], idx=idx, gate=gate, counts=counts)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(c.seed + 91)
+        dy = torch.randn((c.L, c.d), generator=gen, device=device).to(D.torch_dtype)
+        f32 = torch.float32
+        grads = {"dx": torch.empty((c.L, c.d), dtype=f32, device=device),
+                 "dW": torch.zeros((c.N, c.d), dtype=f32, device=device),
+                 "dV": torch.zeros((c.N, c.d), dtype=f32, device=device),
+                 "dWr": torch.zeros((c.Nr, c.d), dtype=f32, device=device),
+                 "dWc": torch.zeros((c.Nc, c.d), dtype=f32, device=device),
+                 "dbias_r": torch.zeros(c.Nr, dtype=f32, device=device),
+                 "dbias_c": torch.zeros(c.Nc, dtype=f32, device=device)}
+        ws = omni.Workspace()
+
+        def run(accumulate):
+            def fwd(stream):
+                omni.moe_backward(D, dd["x"], dd["Wr"], dd["Wc"], dd["W"], dd["V"], idx, gate,
+                                  dy, grads=grads, accumulate=accumulate, counts=counts, ws=ws,
+                                  stream=stream)
+            return timed_graph(fwd, steps)
+
+        ms = run(True)
+        ms_over = run(False)
+        na = int(counts[0].item())
+        e = c.esize
+        bytes_ = (2 * c.L * c.d * e + 2 * c.d * na * e + 2 * 2 * c.d * na * 4 + c.L * c.d * 4
+                  + (c.Nr + c.Nc) * c.d * e + 2 * (c.Nr + c.Nc) * c.d * 4 + 8 * c.L * c.K)
+        flops = 4 * c.L * (c.Nr + c.Nc) * c.d + 8 * c.L * c.K * c.d
+        del grads, ws, dy
+        torch.cuda.empty_cache()
+        # overwriting skips the reads of the old gradient rows
+        bytes_over = bytes_ - 2 * c.d * na * 4 - (c.Nr + c.Nc) * c.d * 4
+        return {"ms": ms, "n_active": na, "tokens_per_s": c.L / (ms * 1e-3),
+                "roofline": {"bound": "hbm", "bytes": bytes_, "flops": flops,
+                             "achieved": bytes_ / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                             "frac": bytes_ / (hbm * 1e9) / (ms * 1e-3), "peak_src": peak_src},
+                "overwrite": {"ms": ms_over, "bytes": bytes_over,
+                              "frac": bytes_over / (hbm * 1e9) / (ms_over * 1e-3)},
+                "note": "gradients accumulated into fp32 arrays (accumulate); overwrite: the "
+                        "first micro-batch, old gradient rows not read"}
+
+    if args.backward_only:
+        # profiling entry: the backward of this workload alone (no JSON line)
+        rec = measure_backward(cfg, d, args.steps)
+        if rank == 0:
+            print(f"backward {cfg.name}: {rec['ms']:.4f} ms, {rec['roofline']['frac']:.3f} of "
+                  f"HBM; overwriting: {rec['overwrite']['ms']:.4f} ms, "
+                  f"{rec['overwrite']['frac']:.3f}", flush=True)
+        return 0
     ms, n_active, status, clocks, _, kernels = measure(cfg, d, args.steps, args.warmup)
     ms_all = max_over_ranks(ms, world, device)
     e2e_steps = max(8, args.steps)
@@ -671,33 +759,6 @@ def run_ours(args):
         torch.cuda.empty_cache()
         return out
 
-    def timed_graph(fn, steps, warmup=2):
-        """Mean CUDA-event time of fn captured in a graph, L2 flushed before
-        each replay."""
-        stream = torch.cuda.Stream(device)
-        with torch.cuda.stream(stream):
-            fn(stream)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            fn(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(warmup):
-                flush.zero_()
-                g.replay()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(steps)]
-        with torch.cuda.stream(stream):
-            for a, b in ev:
-                flush.zero_()
-                a.record(stream)
-                g.replay()
-                b.record(stream)
-        torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
-        del g
-        return ms
-
     def measure_shards(c, dd, steps):
         """Expert-sharded forward on this batch, one G-way split at a time:
         every shard's per-process work (routing, schedule, its own experts'
@@ -768,6 +829,7 @@ def run_ours(args):
         extra["dense_groups"] = measure_dense_paths(max(3, args.steps // 2))
         extra["expert_shards"] = measure_shards(cfg, d, 3)
         extra["glu"] = measure_glu(cfg, d, max(3, args.steps // 2))
+        extra["backward"] = measure_backward(cfg, d, max(3, args.steps // 2))
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
@@ -874,6 +936,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward of the workload (profiling; no JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

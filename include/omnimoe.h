@@ -371,8 +371,10 @@ int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* str
  *     storage type.
  *   dx [L x d] fp32: overwritten.
  *   dW, dV [N x d], dWr [Nr x d], dWc [Nc x d], dbias_r [Nr], dbias_c [Nc]
- *     (the two biases nullable) fp32: added to (rows of experts no token
- *     chose are not touched), so that gradients accumulate across calls.
+ *     (the two biases nullable) fp32: added to when accumulate != 0, so that
+ *     gradients accumulate across calls; overwritten when accumulate == 0
+ *     (without reading them: the first micro-batch).  Either way the rows
+ *     of dW and dV of experts no token chose are not touched.
  *   counts[0], counts[1]: the active experts; counts[2]: status bits.
  *   ws: omni_workspace_size(dims, OMNI_WS_BACKWARD).
  * All arrays 16-byte aligned.  Router gradients go through tensor-core
@@ -383,8 +385,8 @@ int omni_cast_output(const omni_dims* dims, const float* src, void* y, void* str
 int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                       const void* W, const void* V, const int32_t* idx, const float* gate,
                       const void* dy, float* dx, float* dW, float* dV, float* dWr, float* dWc,
-                      float* dbias_r, float* dbias_c, int32_t* counts, void* ws, size_t ws_bytes,
-                      void* stream);
+                      float* dbias_r, float* dbias_c, int accumulate, int32_t* counts, void* ws,
+                      size_t ws_bytes, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* omni_status_string(int status);

@@ -323,8 +323,8 @@ def test_backward_host_checks(lib):
         args["dbias_r"] = args["dbias_c"] = None
         args.update(over)
         ws = over.pop("ws", None)
-        return lib.omni_moe_backward(C.byref(dims), *[args[n] for n in names], ws,
-                                     1 << 30 if ws is not None else 0, None)
+        return lib.omni_moe_backward(C.byref(dims), *[args[n] for n in names[:-1]], 1,
+                                     args["counts"], ws, 1 << 30 if ws is not None else 0, None)
 
     assert call(_dims(dtype=_lib.OMNI_F32)) == _lib.OMNI_ERR_UNSUPPORTED
     assert call(B16, dy=None) == _lib.OMNI_ERR_INVALID_ARG

@@ -110,3 +110,37 @@ def test_backward_without_bias_gradients():
     ref = O.backward(cfg, h, idx.cpu().numpy(), gate.cpu().numpy().astype(np.float64),
                      _bf16_dy(cfg).float().numpy().astype(np.float64))
     assert rel_err(g["dWr"].cpu().numpy().astype(np.float64), ref["dWr"]) <= TOL["dWr"]
+
+
+def test_backward_overwrites_without_reading():
+    """accumulate=False: the active rows of dW, dV and the whole router and
+    bias gradients are overwritten (what was there before does not matter,
+    even NaN); rows of experts no token chose keep their values."""
+    cfg = CONFIGS[4]
+    init = {name: torch.full(shape, float("nan"), device="cuda")
+            for name, shape in (("dW", (cfg.N, cfg.d)), ("dV", (cfg.N, cfg.d)),
+                                ("dWr", (cfg.Nr, cfg.d)), ("dWc", (cfg.Nc, cfg.d)),
+                                ("dbias_r", (cfg.Nr,)), ("dbias_c", (cfg.Nc,)))}
+    h = WL.make_inputs(cfg)
+    d = {k: dev(v) for k, v in h.items()}
+    D = omni.LayerDims.of(cfg)
+    idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
+    omni.moe_forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], d["bias_r"], d["bias_c"],
+                     idx=idx, gate=gate)
+    dy = _bf16_dy(cfg)
+    g = omni.moe_backward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], idx, gate, dy.cuda(),
+                          grads={k: v.clone() for k, v in init.items()}, accumulate=False)
+    torch.cuda.synchronize()
+    gi = idx.cpu().numpy()
+    ref = O.backward(cfg, h, gi, gate.cpu().numpy().astype(np.float64),
+                     dy.float().numpy().astype(np.float64))
+    act = np.unique(gi)
+    idle = np.setdiff1d(np.arange(cfg.N), act)
+    for key in ("dW", "dV"):
+        got = g[key].cpu().numpy()
+        assert np.isnan(got[idle]).all()
+        assert rel_err(got[act].astype(np.float64), ref[key][act]) <= TOL[key]
+    for key in ("dWr", "dWc", "dbias_r", "dbias_c", "dx"):
+        got = g[key].cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all() and rel_err(got, ref[key]) <= TOL[key], key
