@@ -354,11 +354,12 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   const int64_t acc_words = omni::expert_acc_words(D);
   float* acc = acc_words == 0 ? nullptr
                : static_cast<float*>(D.dtype == OMNI_F32 || D.sharded() ? y : w.expert);
-  // a small batch runs the two-kernel tail; its two counters are cleared
-  // by the selection kernel in place of the accumulator
+  // a small batch runs the two-kernel tail; its counters and id bitmap are
+  // cleared by the selection kernel in place of the accumulator
   const bool tail = omni::sched_exec_supported(D);
   float* zero = tail ? static_cast<float*>(w.expert) : acc;
-  const int64_t zero_words = tail ? 2 : acc_words;
+  const int64_t zero_words =
+      tail ? static_cast<int64_t>(omni::sched_exec_zero_words(D)) : acc_words;
   bool acc_zeroed = false;
   {
     omni::CallRange stage("route");

@@ -119,14 +119,16 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
                             int32_t* uniq, int32_t* group_off, int32_t* counts, void* ws,
                             cudaStream_t s);
 
-// ---- scheduling and execution of a small batch: two kernels ---------------
-// Supported: M <= 8192 tasks, N <= 2^20, d of 256/512/1024/2048 bf16 or
-// 128/256/512/1024 fp32 elements; not with OMNI_FLAG_STAGED_SMALL.  A
-// function of the dims alone.
+// ---- execution of a small batch straight from the routing: two kernels -----
+// Supported: M <= 8192 tasks, N <= 2^20, 1 <= L <= 65535, d of
+// 256/512/1024/2048 bf16 or 128/256/512/1024 fp32 elements; not with
+// OMNI_FLAG_STAGED_SMALL.  A function of the dims alone.
 bool sched_exec_supported(const Dims& D);
 // 32-bit words of workspace (256-byte aligned) the two kernels need; the
-// first two words must be zero at the call (the rest is scratch).
+// first sched_exec_zero_words(D) words must be zero at the call (the rest is
+// scratch).
 size_t sched_exec_ws_words(const Dims& D);
+size_t sched_exec_zero_words(const Dims& D);
 // Writes y [L x d] completely, and counts[0], [1].
 cudaError_t launch_sched_exec(const Dims& D, const void* x, const void* W, const void* V,
                               const int32_t* idx, const float* gate, void* y, uint32_t* ws,

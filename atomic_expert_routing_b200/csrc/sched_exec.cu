@@ -1,32 +1,21 @@
-// Expert-Centric Scheduling and grouped execution of a small batch in two
-// kernels ("OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at
+// Grouped execution of a small batch in two kernels, straight from the
+// routing ("OmniMoE: An Efficient MoE by Orchestrating Atomic Experts at
 // Scale" (gist.science), Technisch Overzicht section 2.2; the OmniMoE
 // explainer on manus.space, Expert-Centric Scheduling steps 1-4).
 //
-// For a decode-sized batch (a few thousand tasks) the separate scheduling and
-// execution kernels are each bound by their own latency, not by bytes, and
-// scatter-adding every task's d-vector into the few rows of y piles fp32
-// reductions onto the same lines.  Here:
+// Expert-Centric Scheduling orders the tasks by expert so that each active
+// expert's W and V rows leave HBM once for all its tokens.  A batch of at
+// most 8192 tasks touches at most 8192 rows of each matrix (32 MiB at
+// d = 2048 in bf16), which the 126 MB L2 of a B200 holds: in any task order
+// a row leaves HBM once and later reads of it are L2 hits.  So here the tasks
+// are not sorted; the schedule's counts (|U| and the group count) are still
+// formed, from a bitmap of the active ids:
 //
-// k_sched_act -- scheduling and the activations, split by expert id (gated
-// experts, with a gate matrix U: c also times x[t] . U[e]):
-//  1. The ids are cut into kSeTiles tiles of consecutive ids; kSeParts CTAs
-//     share a tile.  Every CTA of a tile reads the whole routing (L*K ids)
-//     and keeps the tasks whose expert lies in its tile; the tile's CTAs ask
-//     L2 to prefetch an eighth of its W rows each.
-//  2. It sorts them by expert: a bitmap over the tile's ids and its popcount
-//     prefix give every task's expert its rank among the tile's active ids
-//     (so the tile's count of active ids), per-rank counts and their scan
-//     give every expert its first position.  Tasks of one expert (each for a
-//     different token) are placed in any order: that changes no result.
-//  3. Part r of the tile computes c = gate * SiLU(x[t] . W[e]) for a
-//     contiguous share of that list, cut at expert boundaries, so an
-//     expert's W row is read once for all its tokens; c goes to the task's
-//     slot t*K + k.  A group of B consecutive active ids is thus executed
-//     expert by expert by the CTAs its ids fall to; no CTA needs the global
-//     ranks for its part.
-//  4. |U| is the sum of the tiles' counts of active ids (atomic adds); the
-//     tile that finishes last writes it and the group count ceil(|U| / B).
+// k_task_act -- one warp per task (t, k) in routing order: marks its id in
+//   the bitmap (the first task to set a bit counts the id), then
+//   c = gate * SiLU(x[t] . W[e]) (gated experts, with a gate matrix U: c also
+//   times x[t] . U[e]) into the task's slot t*K + k.  The CTA that finishes
+//   last writes |U| and ceil(|U| / B).
 //
 // k_gather_v -- the value rows: CTA (t, s) forms columns s of
 //  y[t] = sum over k of c[t, k] * V[idx[t, k]] in registers (each warp a
@@ -34,27 +23,20 @@
 //  stores them in the storage type (bf16: nearest even).  Each output
 //  element is written once: no reductions into y, no accumulator to clear.
 //
-// Tiles have a fixed count, so the split of the ids does not depend on the
-// device; no CTA waits on another.  Ids outside [0, N) raise
-// OMNI_DEV_BAD_INDEX and are executed as expert 0, as omni_schedule treats
-// them.
+// No CTA waits on another.  Ids outside [0, N) raise OMNI_DEV_BAD_INDEX and
+// are executed as expert 0, as omni_schedule treats them.
 #include "common.cuh"
-#include "blocksort.cuh"
 #include "internal.h"
 
 namespace omni {
 namespace {
 
-constexpr int kSeThreads = 512;
+constexpr int kSeThreads = 512;  // k_gather_v
 constexpr int kSeWarps = kSeThreads / 32;
-constexpr int kSeTiles = 18;              // tiles of consecutive ids
-constexpr int kSeParts = 8;               // CTAs per tile
-constexpr int64_t kSeMaxM = 8192;         // tasks (13 bits of a packed task)
-constexpr int64_t kSeMaxN = int64_t(1) << 20;  // tile spans below 2^16 ids
-
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
+constexpr int kTaThreads = 256;  // k_task_act: a task per warp
+constexpr int kTaWarps = kTaThreads / 32;
+constexpr int64_t kSeMaxM = 8192;              // tasks: their rows stay in L2
+constexpr int64_t kSeMaxN = int64_t(1) << 20;  // ids: a bitmap of at most 128 KiB
 
 __device__ __forceinline__ float dot16(uint4 a, uint4 b, const __nv_bfloat16*) {
   float s0 = 0.0f, s1 = 0.0f;
@@ -90,207 +72,85 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 }
 __device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
-// Global scratch of one call, zeroed before the kernel: the sum of the
-// tiles' active ids, finished tiles.
+// Global scratch of one call, zeroed before the kernel (the zero words of
+// sched_exec_zero_words): the active ids counted, finished CTAs, and the
+// bitmap of this process' ids.
 struct SeScratch {
   uint32_t* uacc;
-  uint32_t* tiles_done;
+  uint32_t* ctas_done;
+  uint32_t* bits;
 };
 
-struct SePlan {
-  int64_t span;   // ids per tile
-  int words;      // bitmap words of a tile
-  size_t smem;
-};
-
-// d = NV * 32 * (16 / sizeof(T)): every lane holds NV 16-byte vectors of a row.
-// Every phase issues its global loads before it uses any of them.  GLU: gated
-// experts, c also times x[t] . U[e].
+// d = NV * 32 * (16 / sizeof(T)): every lane holds NV 16-byte vectors of a
+// row, all loaded before the first is used.  GLU: gated experts, c also
+// times x[t] . U[e].
 template <typename T, int NV, bool GLU>
-__global__ void __launch_bounds__(kSeThreads, 1)
-    k_sched_act(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
-                const int32_t* __restrict__ idx,
-                const float* __restrict__ gate, int L, int K, int64_t N, int B, SePlan P,
-                ShardIds sh, float* __restrict__ cbuf, SeScratch sc,
-                int32_t* __restrict__ counts) {
+__global__ void __launch_bounds__(kTaThreads)
+    k_task_act(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
+               const int32_t* __restrict__ idx, const float* __restrict__ gate, int L, int K,
+               int64_t N, int B, ShardIds sh, float* __restrict__ cbuf, SeScratch sc,
+               int32_t* __restrict__ counts) {
   constexpr int EPV = 16 / sizeof(T);
-  constexpr int kPer = kSeMaxM / kSeThreads;  // routing ids per thread
-  constexpr uint32_t kIdxMask = (1u << 13) - 1u;
   const int d = NV * 32 * EPV;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int M = L * K;
-  const int tile = blockIdx.x / kSeParts, part = blockIdx.x % kSeParts;
-  // the tile's ids [lo, hi) within this process' ids [sh.lo, sh.hi); the
-  // row of id e is e - sh.lo
-  const int64_t lo = sh.lo + static_cast<int64_t>(tile) * P.span;
-  const int64_t hi = lo + P.span < sh.hi ? lo + P.span : sh.hi;
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint32_t* own = reinterpret_cast<uint32_t*>(sm);   // [M] (e - lo) << 13 | task index
-  uint32_t* sorted = own + M;                        // [M] the same, by expert
-  int* ecnt = reinterpret_cast<int*>(sorted + M);    // [M] tasks per expert rank, then first position
-  int* ecur = ecnt + M;                              // [M] placement cursors
-  uint32_t* lbits = reinterpret_cast<uint32_t*>(ecur + M);  // [words] the tile's active ids
-  int* lpre = reinterpret_cast<int*>(lbits + P.words);      // [words] rank before each word
-  __shared__ int warp_tot[32];
-  __shared__ int total, nown;
-  int32_t* status = counts + 2;
-
-  for (int j = tid; j < P.words; j += kSeThreads) lbits[j] = 0u;
-  if (tid == 0) nown = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ uint32_t cta_new;
+  if (threadIdx.x == 0) cta_new = 0u;
   pdl_wait();
   pdl_trigger();
   __syncthreads();
-
-  // (1) the tile's tasks: every routing id of this thread loaded first
-  {
-    int ev[kPer];
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      const int i = tid + q * kSeThreads;
-      ev[q] = i < M ? idx[i] : 0;
+  const int64_t M = static_cast<int64_t>(L) * K;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kTaWarps + warp;  // the task's slot
+  if (i < M) {
+    int64_t e = idx[i];
+    if (e < 0 || e >= N) {
+      if (lane == 0) raise_status(counts + 2, OMNI_DEV_BAD_INDEX);
+      e = 0;
     }
+    if (sh.has(e)) {  // warp-uniform
+      const int64_t row = e - sh.lo;
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (i / K) * d);
+      const uint4* wr = reinterpret_cast<const uint4*>(W + row * d);
+      constexpr int NU = GLU ? NV : 1;
+      uint4 xv[NV], wv[NV], uv[NU];
 #pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      const int i = tid + q * kSeThreads;
-      if (i < M) {
-        int64_t e = ev[q];
-        if (e < 0 || e >= N) {
-          if (blockIdx.x == 0) raise_status(status, OMNI_DEV_BAD_INDEX);
-          e = 0;
-        }
-        if (e >= lo && e < hi) {
-          const uint32_t el = static_cast<uint32_t>(e - lo);
-          own[atomicAdd(&nown, 1)] = (el << 13) | static_cast<uint32_t>(i);
-          atomicOr(&lbits[el >> 5], 1u << (el & 31));
-        }
+      for (int q = 0; q < NV; ++q) {
+        xv[q] = xr[q * 32 + lane];
+        wv[q] = wr[q * 32 + lane];
       }
+      if constexpr (GLU) {
+        const uint4* ur = reinterpret_cast<const uint4*>(U + row * d);
+#pragma unroll
+        for (int q = 0; q < NV; ++q) uv[q] = ur[q * 32 + lane];
+      }
+      if (lane == 0) {  // the first task to set the id's bit counts the id
+        const uint32_t m = 1u << (row & 31);
+        if ((atomicOr(&sc.bits[row >> 5], m) & m) == 0u) atomicAdd(&cta_new, 1u);
+      }
+      float sdot = 0.0f;
+#pragma unroll
+      for (int q = 0; q < NV; ++q) sdot += dot16(xv[q], wv[q], static_cast<const T*>(nullptr));
+      sdot = warp_sum(sdot);
+      float c = gate[i] * silu(sdot);
+      if constexpr (GLU) {
+        float su = 0.0f;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) su += dot16(xv[q], uv[q], static_cast<const T*>(nullptr));
+        c *= warp_sum(su);
+      }
+      if (lane == 0) cbuf[i] = c;
     }
   }
-  __syncthreads();
-  const int n = nown;
-  // the tile's W rows, whole (d * sizeof(T) bytes, 16-byte multiples): part
-  // r asks L2 for those of own tasks r, r + parts, ... while the tile is
-  // sorted
-  for (int q = part + kSeParts * tid; q < n; q += kSeParts * kSeThreads)
-    prefetch_l2(W + (lo - sh.lo + (own[q] >> 13)) * d, static_cast<uint32_t>(d * sizeof(T)));
-
-  // (2) rank of every active id of the tile (popcount prefix of the bitmap)
-  {
-    const int per = (P.words + kSeThreads - 1) / kSeThreads;
-    const int w0 = tid * per;
-    const int w1 = w0 + per < P.words ? w0 + per : P.words;
-    int mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(lbits[w]);
-    int run = block_exclusive_scan(mine, warp_tot, &total);
-    for (int w = w0; w < w1; ++w) {
-      lpre[w] = run;
-      run += __popc(lbits[w]);
-    }
-  }
-  __syncthreads();
-  const int u_tile = total;
-  auto rank_of = [&](uint32_t el) {
-    return lpre[el >> 5] + __popc(lbits[el >> 5] & ((1u << (el & 31)) - 1u));
-  };
-  for (int r = tid; r < u_tile; r += kSeThreads) {
-    ecnt[r] = 0;
-    ecur[r] = 0;
-  }
-  __syncthreads();
-  for (int j = tid; j < n; j += kSeThreads) atomicAdd(&ecnt[rank_of(own[j] >> 13)], 1);
-  __syncthreads();
-  // first position of every expert (exclusive scan of the counts, in place)
-  {
-    const int per = (u_tile + kSeThreads - 1) / kSeThreads;
-    const int r0 = tid * per;
-    const int r1 = r0 + per < u_tile ? r0 + per : u_tile;
-    int mine = 0;
-    for (int r = r0; r < r1; ++r) mine += ecnt[r];
-    int run = block_exclusive_scan(mine, warp_tot, &total);
-    for (int r = r0; r < r1; ++r) {
-      const int c = ecnt[r];
-      ecnt[r] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  for (int j = tid; j < n; j += kSeThreads) {
-    const uint32_t v = own[j];
-    const int r = rank_of(v >> 13);
-    sorted[ecnt[r] + atomicAdd(&ecur[r], 1)] = v;
-  }
-  // |U| and the group count: part 0 of every tile adds its count; the tile
+  // |U| and the group count: every CTA adds its newly counted ids; the CTA
   // that finishes last writes both
-  if (part == 0 && tid == 0) {
-    atomicAdd(sc.uacc, static_cast<uint32_t>(u_tile));
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicAdd(sc.uacc, cta_new);
     __threadfence();
-    if (atomicAdd(sc.tiles_done, 1u) == kSeTiles - 1) {
+    if (atomicAdd(sc.ctas_done, 1u) == gridDim.x - 1) {
       __threadfence();
       const uint32_t u = atomicAdd(sc.uacc, 0u);
       counts[0] = static_cast<int32_t>(u);
       counts[1] = static_cast<int32_t>((static_cast<int64_t>(u) + B - 1) / B);
-    }
-  }
-  __syncthreads();
-
-  // (3) this part's share [b0, b1) of the expert-sorted list, cut where an
-  // expert starts (the first expert starting at or after part * n / parts)
-  auto cut = [&](int q) {
-    if (q >= kSeParts) return n;
-    const int want = static_cast<int>((static_cast<int64_t>(q) * n + kSeParts - 1) / kSeParts);
-    int l = 0, h = u_tile;  // first rank whose start is >= want
-    while (l < h) {
-      const int m = (l + h) >> 1;
-      if (ecnt[m] >= want) h = m; else l = m + 1;
-    }
-    return l < u_tile ? ecnt[l] : n;
-  };
-  const int b0 = cut(part), b1 = cut(part + 1);
-
-  // (4) activations; warp w takes positions b0 + w, b0 + w + 16, ..., PAIR at
-  // a time (their x and W rows loaded together; one at d = 256 vectors, which
-  // fill the registers)
-  constexpr int PAIR = (NV >= 8 || (GLU && NV >= 4)) ? 1 : 2;
-  constexpr int NU = GLU ? NV : 1;  // vectors of the U row held per lane
-  for (int p0 = b0 + warp; p0 < b1; p0 += PAIR * kSeWarps) {
-    uint4 xv[PAIR][NV], wv[PAIR][NV], uv[PAIR][NU];
-    int ii[PAIR];
-#pragma unroll
-    for (int r = 0; r < PAIR; ++r) {
-      const int pos = p0 + r * kSeWarps;
-      ii[r] = -1;
-      if (pos >= b1) continue;
-      const uint32_t v = sorted[pos];  // warp-uniform
-      ii[r] = static_cast<int>(v & kIdxMask);
-      const int64_t e = lo - sh.lo + (v >> 13);  // the row
-      const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(ii[r] / K) * d);
-      const uint4* wr = reinterpret_cast<const uint4*>(W + e * d);
-#pragma unroll
-      for (int q = 0; q < NV; ++q) {
-        xv[r][q] = xr[q * 32 + lane];
-        wv[r][q] = wr[q * 32 + lane];
-      }
-      if constexpr (GLU) {
-        const uint4* ur = reinterpret_cast<const uint4*>(U + e * d);
-#pragma unroll
-        for (int q = 0; q < NV; ++q) uv[r][q] = ur[q * 32 + lane];
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < PAIR; ++r) {
-      if (ii[r] < 0) continue;
-      float sdot = 0.0f;
-#pragma unroll
-      for (int q = 0; q < NV; ++q) sdot += dot16(xv[r][q], wv[r][q], static_cast<const T*>(nullptr));
-      sdot = warp_sum(sdot);
-      float c = gate[ii[r]] * silu(sdot);
-      if constexpr (GLU) {
-        float su = 0.0f;
-#pragma unroll
-        for (int q = 0; q < NV; ++q) su += dot16(xv[r][q], uv[r][q], static_cast<const T*>(nullptr));
-        c *= warp_sum(su);
-      }
-      if (lane == 0) cbuf[ii[r]] = c;
     }
   }
 }
@@ -374,43 +234,30 @@ int se_nv(const Dims& D) {
 
 // A function of the dims alone (not of the device), so that the workspace
 // sized from it holds for a launch on any device.
-bool se_plan(const Dims& D, SePlan* P) {
-  const int64_t M = D.M();
-  if (D.L < 1 || M > kSeMaxM || D.N() > kSeMaxN || se_nv(D) == 0) return false;
-  if (D.B > (int64_t(1) << 30)) return false;
-  // supported or not by the whole layer's ids (a shard's tiles are no
-  // larger), so that the decision and the workspace do not depend on the
-  // shard; the tiles then split this process' ids
-  auto plan = [&](int64_t ids) {
-    P->span = (ids + kSeTiles - 1) / kSeTiles;
-    P->words = static_cast<int>((P->span + 31) / 32);
-    P->smem = static_cast<size_t>(M) * 16 + static_cast<size_t>(P->words) * 8;
-    return P->smem <= 200 * 1024;
-  };
-  if (!plan(D.N())) return false;
-  return plan(D.shard_hi() - D.shard_lo());
+bool se_ok(const Dims& D) {
+  return D.L >= 1 && D.L <= 65535 && D.M() <= kSeMaxM && D.N() <= kSeMaxN && se_nv(D) != 0 &&
+         D.B <= (int64_t(1) << 30);
 }
 
-// workspace words: the two scratch counters (cleared before the call), then
-// c [M] floats from the next 256-byte boundary
-constexpr size_t kSeCbufOff = 64;
+// workspace words: the two counters, the bitmap of the ids (all zeroed
+// before the call), then c [M] floats, each part on a 256-byte boundary
+constexpr size_t kSeBitsOff = 64;
+size_t se_bits_words(const Dims& D) { return (static_cast<size_t>(D.N()) + 31) / 32; }
+size_t se_cbuf_off(const Dims& D) { return (kSeBitsOff + se_bits_words(D) + 63) / 64 * 64; }
 
 template <typename T, int NV, bool GLU>
-cudaError_t launch_se_t(const Dims& D, const SePlan& P, const void* x, const void* W,
-                        const void* V, const int32_t* idx, const float* gate, void* y,
-                        uint32_t* ws, int32_t* counts, cudaStream_t s, const void* U) {
-  cudaError_t err = cudaFuncSetAttribute(k_sched_act<T, NV, GLU>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(P.smem));
-  if (err != cudaSuccess) return err;
+cudaError_t launch_se_t(const Dims& D, const void* x, const void* W, const void* V,
+                        const int32_t* idx, const float* gate, void* y, uint32_t* ws,
+                        int32_t* counts, cudaStream_t s, const void* U) {
   SeScratch sc;
   sc.uacc = ws;
-  sc.tiles_done = ws + 1;
-  float* cbuf = reinterpret_cast<float*>(ws + kSeCbufOff);
-  OMNI_TRY(launch_k(k_sched_act<T, NV, GLU>, kSeTiles * kSeParts, kSeThreads, P.smem, s,
-      static_cast<const T*>(x), static_cast<const T*>(W), static_cast<const T*>(U), idx, gate,
-      static_cast<int>(D.L),
-      static_cast<int>(D.K), D.N(), static_cast<int>(D.B), P, shard_ids(D), cbuf, sc, counts));
+  sc.ctas_done = ws + 1;
+  sc.bits = ws + kSeBitsOff;
+  float* cbuf = reinterpret_cast<float*>(ws + se_cbuf_off(D));
+  const unsigned blocks = static_cast<unsigned>((D.M() + kTaWarps - 1) / kTaWarps);
+  OMNI_TRY(launch_k(k_task_act<T, NV, GLU>, blocks, kTaThreads, 0, s, static_cast<const T*>(x),
+      static_cast<const T*>(W), static_cast<const T*>(U), idx, gate, static_cast<int>(D.L),
+      static_cast<int>(D.K), D.N(), static_cast<int>(D.B), shard_ids(D), cbuf, sc, counts));
   // value rows: NS vectors per lane and CTA, 2 when the row has them
   constexpr int NS = NV < 2 ? NV : 2;
   constexpr int COLS = NS * 32 * (16 / sizeof(T));
@@ -431,22 +278,21 @@ cudaError_t launch_se_t(const Dims& D, const SePlan& P, const void* x, const voi
 }  // namespace
 
 bool sched_exec_supported(const Dims& D) {
-  if (D.flags & OMNI_FLAG_STAGED_SMALL) return false;
-  SePlan P;
-  return se_plan(D, &P) && D.L <= 65535;
+  return (D.flags & OMNI_FLAG_STAGED_SMALL) == 0 && se_ok(D);
 }
 
-size_t sched_exec_ws_words(const Dims& D) { return kSeCbufOff + static_cast<size_t>(D.M()); }
+size_t sched_exec_ws_words(const Dims& D) { return se_cbuf_off(D) + static_cast<size_t>(D.M()); }
+
+size_t sched_exec_zero_words(const Dims& D) { return kSeBitsOff + se_bits_words(D); }
 
 cudaError_t launch_sched_exec(const Dims& D, const void* x, const void* W, const void* V,
                               const int32_t* idx, const float* gate, void* y, uint32_t* ws,
                               int32_t* counts, cudaStream_t s, const void* U) {
-  SePlan P;
-  if (!se_plan(D, &P)) return cudaErrorInvalidValue;
-#define OMNI_SE(T_, NV_)                                                                  \
-  return U != nullptr                                                                     \
-             ? launch_se_t<T_, NV_, true>(D, P, x, W, V, idx, gate, y, ws, counts, s, U)  \
-             : launch_se_t<T_, NV_, false>(D, P, x, W, V, idx, gate, y, ws, counts, s, U);
+  if (!se_ok(D)) return cudaErrorInvalidValue;
+#define OMNI_SE(T_, NV_)                                                               \
+  return U != nullptr                                                                  \
+             ? launch_se_t<T_, NV_, true>(D, x, W, V, idx, gate, y, ws, counts, s, U)  \
+             : launch_se_t<T_, NV_, false>(D, x, W, V, idx, gate, y, ws, counts, s, U);
   if (D.dtype == OMNI_F32) {
     switch (se_nv(D)) {
       case 1: OMNI_SE(float, 1)

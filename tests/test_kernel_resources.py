@@ -31,7 +31,7 @@ HOT = {
     # decode forward
     "omni::(anonymous namespace)::k_router_tc<64>": 0,
     "omni::(anonymous namespace)::k_select_wide<8, 2, 2>": 16,
-    "omni::(anonymous namespace)::k_sched_act<__nv_bfloat16, 8, false>": 0,
+    "omni::(anonymous namespace)::k_task_act<__nv_bfloat16, 8, false>": 0,
     "omni::(anonymous namespace)::k_gather_v<__nv_bfloat16, 2, __nv_bfloat16>": 0,
     "omni::(anonymous namespace)::k_gather_v<__nv_bfloat16, 2, float>": 0,
     # decode stages timed separately (omni_schedule + omni_expert_forward)
@@ -39,7 +39,7 @@ HOT = {
     "omni::(anonymous namespace)::k_expert_async<__nv_bfloat16, 8, 3, false>": 0,
     "omni::(anonymous namespace)::k_cast": 0,
     # gated experts (SwiGLU) on the same paths
-    "omni::(anonymous namespace)::k_sched_act<__nv_bfloat16, 8, true>": 0,
+    "omni::(anonymous namespace)::k_task_act<__nv_bfloat16, 8, true>": 0,
     "omni::(anonymous namespace)::k_act<__nv_bfloat16, 8, 3, true, true>": 0,
     "omni::(anonymous namespace)::k_expert_async<__nv_bfloat16, 8, 2, true>": 0,
 }
