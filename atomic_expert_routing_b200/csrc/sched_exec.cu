@@ -4,12 +4,13 @@
 // explainer on manus.space, Expert-Centric Scheduling steps 1-4).
 //
 // Expert-Centric Scheduling orders the tasks by expert so that each active
-// expert's W and V rows leave HBM once for all its tokens.  A batch of at
-// most 8192 tasks touches at most 8192 rows of each matrix (32 MiB at
-// d = 2048 in bf16), which the 126 MB L2 of a B200 holds: in any task order
-// a row leaves HBM once and later reads of it are L2 hits.  So here the tasks
-// are not sorted; the schedule's counts (|U| and the group count) are still
-// formed, from a bitmap of the active ids:
+// expert's W and V rows leave HBM once for all its tokens.  A batch touches
+// at most min(N, L*K) rows of each matrix; when those fit in 64 MiB (decode:
+// 4096 rows of 4 KiB each at d = 2048 in bf16), the 126 MB L2 of a B200 holds
+// them, so in any task order a row leaves HBM once and later reads of it are
+// L2 hits.  For such a batch the tasks are not sorted; the schedule's counts
+// (|U| and the group count) are still formed, from a bitmap of the active
+// ids:
 //
 // k_task_act -- one warp per task (t, k) in routing order: marks its id in
 //   the bitmap (the first task to set a bit counts the id), then
@@ -35,7 +36,9 @@ constexpr int kSeThreads = 512;  // k_gather_v
 constexpr int kSeWarps = kSeThreads / 32;
 constexpr int kTaThreads = 256;  // k_task_act: a task per warp
 constexpr int kTaWarps = kTaThreads / 32;
-constexpr int64_t kSeMaxM = 8192;              // tasks: their rows stay in L2
+// The bytes of W and V rows a batch can touch (min(N, L*K) rows each) that
+// L2 is trusted to hold while the batch runs.
+constexpr int64_t kSeRowBudget = int64_t(64) << 20;
 constexpr int64_t kSeMaxN = int64_t(1) << 20;  // ids: a bitmap of at most 128 KiB
 
 __device__ __forceinline__ float dot16(uint4 a, uint4 b, const __nv_bfloat16*) {
@@ -235,8 +238,11 @@ int se_nv(const Dims& D) {
 // A function of the dims alone (not of the device), so that the workspace
 // sized from it holds for a launch on any device.
 bool se_ok(const Dims& D) {
-  return D.L >= 1 && D.L <= 65535 && D.M() <= kSeMaxM && D.N() <= kSeMaxN && se_nv(D) != 0 &&
-         D.B <= (int64_t(1) << 30);
+  if (D.L < 1 || D.L > 65535 || D.N() > kSeMaxN || se_nv(D) == 0 || D.B > (int64_t(1) << 30))
+    return false;
+  const int64_t rows = D.N() < D.M() ? D.N() : D.M();  // distinct ids a batch can use
+  const int64_t esize = D.dtype == OMNI_F32 ? 4 : 2;
+  return rows * D.d * esize * 2 <= kSeRowBudget;
 }
 
 // workspace words: the two counters, the bitmap of the ids (all zeroed
