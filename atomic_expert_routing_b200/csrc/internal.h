@@ -120,8 +120,8 @@ cudaError_t launch_schedule(const Dims& D, const int32_t* idx, const float* gate
                             cudaStream_t s);
 
 // ---- execution of a small batch straight from the routing: two kernels -----
-// Supported: min(N, L*K) rows of W and V within 64 MiB (they stay in L2),
-// N <= 2^20, 1 <= L <= 65535, d of 256/512/1024/2048 bf16 or
+// Supported: min(N, L*K) rows of W and V within 64 MiB (they stay in L2) or
+// L*K rows within 1 GiB, N <= 2^20, 1 <= L <= 65535, d of 256/512/1024/2048 bf16 or
 // 128/256/512/1024 fp32 elements; not with OMNI_FLAG_STAGED_SMALL.  A
 // function of the dims alone.
 bool sched_exec_supported(const Dims& D);

@@ -8,9 +8,12 @@
 // at most min(N, L*K) rows of each matrix; when those fit in 64 MiB (decode:
 // 4096 rows of 4 KiB each at d = 2048 in bf16), the 126 MB L2 of a B200 holds
 // them, so in any task order a row leaves HBM once and later reads of it are
-// L2 hits.  For such a batch the tasks are not sorted; the schedule's counts
-// (|U| and the group count) are still formed, from a bitmap of the active
-// ids:
+// L2 hits.  A batch whose tasks read at most 1 GiB of rows even without any
+// reuse (L*K rows of each matrix) takes the same path: its worst case, about
+// 0.16 ms of HBM traffic, is below the cost of sorting its tasks, and the
+// rows it shares come from L2.  For such a batch the tasks are not sorted;
+// the schedule's counts (|U| and the group count) are still formed, from a
+// bitmap of the active ids:
 //
 // k_task_act -- one warp per task (t, k) in routing order: marks its id in
 //   the bitmap (the first task to set a bit counts the id), then
@@ -37,8 +40,10 @@ constexpr int kSeWarps = kSeThreads / 32;
 constexpr int kTaThreads = 256;  // k_task_act: a task per warp
 constexpr int kTaWarps = kTaThreads / 32;
 // The bytes of W and V rows a batch can touch (min(N, L*K) rows each) that
-// L2 is trusted to hold while the batch runs.
+// L2 is trusted to hold while the batch runs; and the most row bytes a batch
+// may read from HBM if no row of it were reused from L2 (a row per task).
 constexpr int64_t kSeRowBudget = int64_t(64) << 20;
+constexpr int64_t kSeTaskBudget = int64_t(1) << 30;
 constexpr int64_t kSeMaxN = int64_t(1) << 20;  // ids: a bitmap of at most 128 KiB
 
 __device__ __forceinline__ float dot16(uint4 a, uint4 b, const __nv_bfloat16*) {
@@ -242,7 +247,7 @@ bool se_ok(const Dims& D) {
     return false;
   const int64_t rows = D.N() < D.M() ? D.N() : D.M();  // distinct ids a batch can use
   const int64_t esize = D.dtype == OMNI_F32 ? 4 : 2;
-  return rows * D.d * esize * 2 <= kSeRowBudget;
+  return rows * D.d * esize * 2 <= kSeRowBudget || D.M() * D.d * esize * 2 <= kSeTaskBudget;
 }
 
 // workspace words: the two counters, the bitmap of the ids (all zeroed

@@ -146,8 +146,11 @@ def test_gated_sweeps(cfg):
     y_ref, _ = O.forward_expert(cfg, h, ref_s)
     y = omni.expert_forward(omni.LayerDims.of(cfg), d["x"], d["W"], d["V"], sched, U=d["U"])
     assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
-    y, gi, gg, c = _fused(cfg, d)
-    _check_fused(cfg, h, y, gi, gg, c)
+    # the fused forward on the window path (the default takes the tail: the
+    # batch's rows fit in L2) and by default
+    for flags in (omni.OMNI_FLAG_STAGED_SMALL, 0):
+        y, gi, gg, c = _fused(cfg, d, flags)
+        _check_fused(cfg, h, y, gi, gg, c)
 
 
 def test_gated_ignores_the_dense_tensor_core_flag():

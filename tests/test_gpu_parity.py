@@ -429,14 +429,17 @@ def test_expert_sweeps_path(cfg):
     assert int(counts[2].item()) == 0
 
 
+@pytest.mark.parametrize("flags", [omni.OMNI_FLAG_STAGED_SMALL, 0], ids=["windows", "default"])
 @pytest.mark.parametrize("cfg", SWEEP, ids=[c.name for c in SWEEP])
-def test_fused_sweeps_path(cfg):
+def test_fused_sweeps_path(cfg, flags):
     """The fused forward of a sweep-sized batch goes from the routing straight
-    to the window order of the sweeps: same y as the oracle's expert-centric
-    execution of the routing it chose, same |U| and group count."""
+    to the window order of the sweeps (these batches' rows also fit in L2, so
+    by default they take the routing-order tail; OMNI_FLAG_STAGED_SMALL keeps
+    them on the window path): same y as the oracle's expert-centric execution
+    of the routing it chose, same |U| and group count."""
     h = WL.make_inputs(cfg)
     d = {k: dev(v) for k, v in h.items()}
-    D = omni.LayerDims.of(cfg)
+    D = omni.LayerDims.of(cfg, flags=flags)
     idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
     gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
     counts = omni.new_counts("cuda")

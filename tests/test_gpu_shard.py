@@ -62,9 +62,9 @@ def _unsharded(cfg, d, U=None):
     return y, idx.cpu().numpy(), gate.cpu().numpy()
 
 
-def _run_shards(cfg, h, d, G, gated=False):
+def _run_shards(cfg, h, d, G, gated=False, flags=0):
     """Every shard of the G-way split in turn; returns the summed partials."""
-    D = omni.LayerDims.of(cfg)
+    D = omni.LayerDims.of(cfg, flags=flags)
     U = d.get("U") if gated else None
     y_full, i_ref, g_ref = _unsharded(cfg, d, U)
     total = torch.zeros((cfg.L, cfg.d), dtype=torch.float32, device="cuda")
@@ -104,6 +104,15 @@ def _run_shards(cfg, h, d, G, gated=False):
 def test_shards_partition_the_layer(cfg, G):
     h, d = _inputs(cfg)
     _run_shards(cfg, h, d, G)
+
+
+@pytest.mark.parametrize("cfg", CONFIGS[2:], ids=lambda c: c.name)
+def test_shards_on_the_scheduled_paths(cfg):
+    """OMNI_FLAG_STAGED_SMALL keeps batches whose rows fit in L2 on the
+    schedule-based paths (grouped kernels, or the window order of the
+    sweeps), which the shard's task range bounds."""
+    h, d = _inputs(cfg)
+    _run_shards(cfg, h, d, 3, flags=omni.OMNI_FLAG_STAGED_SMALL)
 
 
 @pytest.mark.parametrize("cfg", [CONFIGS[0], CONFIGS[2], CONFIGS[4]], ids=lambda c: c.name)
