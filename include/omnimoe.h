@@ -75,10 +75,11 @@ extern "C" {
 
 /* dims.flags bits */
 #define OMNI_FLAG_ROUTER_SIMT 1 /* diagnostic: router logits on CUDA cores for bf16 too */
-#define OMNI_FLAG_STAGED_SMALL 2 /* diagnostic: omni_moe_forward of a small batch runs the
-                                    scheduling and grouped-execution kernels of
-                                    omni_schedule and omni_expert_forward instead of its
-                                    two-kernel small-batch tail */
+#define OMNI_FLAG_STAGED_SMALL 2 /* diagnostic: omni_moe_forward of a batch whose rows
+                                    fit in L2 runs the scheduled order (the kernels of
+                                    omni_schedule and omni_expert_forward, or the window
+                                    order of the sweeps) instead of its two-kernel
+                                    routing-order tail */
 #define OMNI_FLAG_DENSE_TENSOR_CORES 4 /* grouped execution of bf16 batches without
                                           column sweeps: the activations of dense groups
                                           (>= 384 tasks per 128-token tile of a group's
@@ -223,21 +224,26 @@ int omni_expert_forward_noalloc(const omni_dims* dims, const void* x, const void
  * then scheduling, then grouped execution.  idx_out / gate_out (nullable,
  * [L x K]) receive the routing decisions; counts[0], counts[1] are written as
  * by omni_schedule; y as in omni_expert_forward.
- * Small batches run omni_schedule's order.  A batch of at most 8192 tasks with
- * N <= 2^20 (and a row width of 256, 512, 1024 or 2048 bf16 / 128 .. 1024
- * fp32 elements) runs scheduling and execution as two kernels: the first
- * splits the ids into tiles of consecutive ids, sorts each tile's tasks by
- * expert and computes their activations gate * SiLU(x[t] . W[e]) (an
- * expert's W row read once for all its tokens), and counts |U| and the
- * groups; the second forms y[t] = sum of activation * V[e] over the token's
- * tasks and writes it once.  No schedule arrays are written (counts[0],
- * counts[1] are).  Batches whose fp32 accumulator is
- * executed in column-slice sweeps (L*d*4 above about 40 MiB) go from the
- * routing straight to the executor's order.  That order is the same groups,
- * in windows of consecutive groups, with each window's tasks ordered by
- * token; the (group, token, expert) order itself is not formed.  Every task
- * is still executed once, so y differs from the staged calls only in the
- * order of its fp32 additions.
+ * The execution order depends on the batch's shape (never on its data):
+ *  - A batch whose rows fit in L2 runs as two kernels straight from the
+ *    routing.  That means at most 64 MiB of the W and V rows it can touch
+ *    (min(N, L*K) of each), or at most 1 GiB of rows even if no row were
+ *    reused (L*K of each); it also needs N <= 2^20, L <= 65535 and a row
+ *    width of 256, 512, 1024 or 2048 bf16 / 128 .. 1024 fp32 elements.
+ *    The first kernel computes every task's activation
+ *    gate * SiLU(x[t] . W[e]) in routing order, and counts |U| and the
+ *    groups from a bitmap of the active ids.  The second forms
+ *    y[t] = sum of activation * V[e] over the token's tasks and writes it
+ *    once.  The rows stay in L2, so each leaves HBM about once without
+ *    sorting the tasks by expert.  No schedule arrays are written
+ *    (counts[0], counts[1] are).  OMNI_FLAG_STAGED_SMALL turns this path off.
+ *  - Other batches run omni_schedule's order.  If their fp32 accumulator is
+ *    executed in column-slice sweeps (L*d*4 above about 40 MiB), they go
+ *    from the routing straight to the executor's order: the same groups, in
+ *    windows of consecutive groups, each window's tasks ordered by token.
+ *    The (group, token, expert) order itself is not formed.
+ * Every task is executed once, so y differs from the staged calls only in
+ * the order of its fp32 additions.
  */
 int omni_moe_forward(const omni_dims* dims, const void* x, const void* Wr, const void* Wc,
                      const float* bias_r, const float* bias_c, const void* W, const void* V,

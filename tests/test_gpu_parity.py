@@ -539,10 +539,11 @@ SMALL_TAIL = [
 
 @pytest.mark.parametrize("cfg", SMALL_TAIL + [WL.DECODE], ids=lambda c: c.name)
 def test_small_batch_tail(cfg):
-    """The fused forward of a small batch ends in two kernels (activations of
-    expert-id tiles, then a per-token gather of the value rows): y against the
-    oracle's expert-centric y of the same routing, |U| and the group count
-    exactly, and y against the staged scheduling and execution kernels
+    """The fused forward of a batch whose rows fit in L2 ends in two kernels
+    (activations in routing order with a bitmap count of the active ids, then
+    a per-token gather of the value rows): y against the oracle's
+    expert-centric y of the same routing, |U| and the group count exactly,
+    and y against the scheduling and execution kernels
     (OMNI_FLAG_STAGED_SMALL) on the same routing."""
     h = host_inputs(cfg) if cfg is WL.DECODE else WL.make_inputs(cfg)
     d = dev_inputs(cfg) if cfg is WL.DECODE else {k: dev(v) for k, v in h.items()}
