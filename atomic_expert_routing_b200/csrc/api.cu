@@ -97,7 +97,7 @@ FusedWs carve_fused(const Dims& D, Carver& c) {
   w.group_off = c.take<int32_t>(static_cast<size_t>(D.gmax()) + 1);
   w.sched = c.take<char>(fused_windows(D) ? omni::windows_ws_bytes(D)
                                            : omni::schedule_ws_bytes(D));
-  // the small-batch tail (activations by expert tile, value gather) uses the
+  // the routing-order tail (activations per task, value gather) uses the
   // expert workspace for its counters and activations
   const size_t tail = omni::sched_exec_supported(D) ? omni::sched_exec_ws_words(D) * 4 : 0;
   const size_t ex = omni::expert_ws_bytes(D);
@@ -354,7 +354,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   const int64_t acc_words = omni::expert_acc_words(D);
   float* acc = acc_words == 0 ? nullptr
                : static_cast<float*>(D.dtype == OMNI_F32 || D.sharded() ? y : w.expert);
-  // a small batch runs the two-kernel tail; its counters and id bitmap are
+  // a batch whose rows fit in L2 runs the two-kernel tail; its counters and id bitmap are
   // cleared by the selection kernel in place of the accumulator
   const bool tail = omni::sched_exec_supported(D);
   float* zero = tail ? static_cast<float*>(w.expert) : acc;

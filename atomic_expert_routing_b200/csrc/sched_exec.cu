@@ -90,10 +90,9 @@ struct SeScratch {
 };
 
 // d = NV * 32 * (16 / sizeof(T)): every lane holds NV 16-byte vectors of a
-// row, all loaded before the first is used.  GLU: gated experts, c also
-// times x[t] . U[e].
+// row.  GLU: gated experts, c also times x[t] . U[e].
 template <typename T, int NV, bool GLU>
-__global__ void __launch_bounds__(kTaThreads)
+__global__ void __launch_bounds__(kTaThreads, GLU ? 2 : 4)
     k_task_act(const T* __restrict__ x, const T* __restrict__ W, const T* __restrict__ U,
                const int32_t* __restrict__ idx, const float* __restrict__ gate, int L, int K,
                int64_t N, int B, ShardIds sh, float* __restrict__ cbuf, SeScratch sc,
@@ -118,33 +117,33 @@ __global__ void __launch_bounds__(kTaThreads)
       const int64_t row = e - sh.lo;
       const uint4* xr = reinterpret_cast<const uint4*>(x + (i / K) * d);
       const uint4* wr = reinterpret_cast<const uint4*>(W + row * d);
-      constexpr int NU = GLU ? NV : 1;
-      uint4 xv[NV], wv[NV], uv[NU];
-#pragma unroll
-      for (int q = 0; q < NV; ++q) {
-        xv[q] = xr[q * 32 + lane];
-        wv[q] = wr[q * 32 + lane];
-      }
-      if constexpr (GLU) {
-        const uint4* ur = reinterpret_cast<const uint4*>(U + row * d);
-#pragma unroll
-        for (int q = 0; q < NV; ++q) uv[q] = ur[q * 32 + lane];
-      }
+      const uint4* ur = GLU ? reinterpret_cast<const uint4*>(U + row * d) : nullptr;
       if (lane == 0) {  // the first task to set the id's bit counts the id
         const uint32_t m = 1u << (row & 31);
         if ((atomicOr(&sc.bits[row >> 5], m) & m) == 0u) atomicAdd(&cta_new, 1u);
       }
-      float sdot = 0.0f;
+      // the row in chunks of CH vectors per lane, each chunk's loads issued
+      // together (registers for every task of the batch to be resident)
+      constexpr int CH = NV > 4 ? 4 : NV;
+      float sdot = 0.0f, su = 0.0f;
 #pragma unroll
-      for (int q = 0; q < NV; ++q) sdot += dot16(xv[q], wv[q], static_cast<const T*>(nullptr));
+      for (int q0 = 0; q0 < NV; q0 += CH) {
+        uint4 xv[CH], wv[CH], uv[GLU ? CH : 1];
+#pragma unroll
+        for (int q = 0; q < CH; ++q) {
+          xv[q] = xr[(q0 + q) * 32 + lane];
+          wv[q] = wr[(q0 + q) * 32 + lane];
+          if constexpr (GLU) uv[q] = ur[(q0 + q) * 32 + lane];
+        }
+#pragma unroll
+        for (int q = 0; q < CH; ++q) {
+          sdot += dot16(xv[q], wv[q], static_cast<const T*>(nullptr));
+          if constexpr (GLU) su += dot16(xv[q], uv[q], static_cast<const T*>(nullptr));
+        }
+      }
       sdot = warp_sum(sdot);
       float c = gate[i] * silu(sdot);
-      if constexpr (GLU) {
-        float su = 0.0f;
-#pragma unroll
-        for (int q = 0; q < NV; ++q) su += dot16(xv[q], uv[q], static_cast<const T*>(nullptr));
-        c *= warp_sum(su);
-      }
+      if constexpr (GLU) c *= warp_sum(su);
       if (lane == 0) cbuf[i] = c;
     }
   }

@@ -18,7 +18,7 @@ from helpers import dev, host_f64, rel_err, tol_y
 
 pytestmark = pytest.mark.gpu
 
-# the small-batch tail (one config per row width it compiles for, both
+# the routing-order tail (one config per row width it compiles for, both
 # storage types, a ragged batch and a skewed one)
 TAIL = [
     WL.Config("glu-tail-bf16-d256", L=1, d=256, Nr=16, Nc=16, k=4, K=4, B=200, dtype=WL.BF16,
@@ -97,7 +97,7 @@ def _oracle_schedule(cfg, h):
 
 @pytest.mark.parametrize("cfg", TAIL, ids=lambda c: c.name)
 def test_gated_small_batch_tail(cfg):
-    """The two-kernel tail with U, and the staged kernels it replaces
+    """The two-kernel tail with U, and the scheduled kernels
     (OMNI_FLAG_STAGED_SMALL) on the same routing."""
     h, d = _inputs(cfg)
     y1, i1, g1, c1 = _fused(cfg, d)

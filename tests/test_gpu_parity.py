@@ -524,7 +524,7 @@ def test_expert_sweeps_back_to_back():
         assert rel_err(host_f64(y), y_ref) <= tol_y(cfg)
 
 
-# ------------------------------- small batches: the two-kernel tail of the fused forward
+# --------------------- batches whose rows fit in L2: the two-kernel tail of the fused forward
 
 SMALL_TAIL = [
     WL.Config("one-bf16-d256-L1", L=1, d=256, Nr=16, Nc=16, k=4, K=4, B=200, dtype=WL.BF16,

@@ -26,7 +26,7 @@ from helpers import dev, host_f64, rel_err, tol_y
 pytestmark = pytest.mark.gpu
 
 CONFIGS = [
-    # the small-batch tail (decode shape)
+    # the routing-order tail (decode shape)
     WL.Config("shard-tail-bf16-d2048", L=64, d=2048, Nr=128, Nc=128, k=64, K=64, B=128,
               dtype=WL.BF16, seed=81),
     WL.Config("shard-tail-f32-d256", L=40, d=256, Nr=32, Nc=48, k=8, K=8, B=16, dtype=WL.F32,
