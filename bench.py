@@ -822,6 +822,50 @@ def run_ours(args):
                 "layer_roofline": {"bound": "hbm", "frac": bytes_ / (hbm * 1e9) / (ms * 1e-3),
                                    "bytes": bytes_}}
 
+    def measure_rotating_x(c, dd, steps, nbatch=8):
+        """The forward of the workload with x rotated among nbatch seeded
+        token batches (one graph per batch, replayed in turn), L2 flushed
+        before each step as in the headline: a step never finds its x, or
+        rows its tokens share with the previous batch, in L2."""
+        D = omni.LayerDims.of(c)
+        ws = omni.Workspace()
+        counts = omni.new_counts(device)
+        y = torch.empty((c.L, c.d), dtype=D.torch_dtype, device=device)
+        xs = [dd["x"]] + [to_dev(rank_inputs(c.with_(seed=c.seed + 7919 * (b + 1)), rank)["x"])
+                          for b in range(nbatch - 1)]
+        stream = torch.cuda.Stream(device)
+        graphs = []
+        for xb in xs:
+            def fwd(xb=xb):
+                omni.moe_forward(D, xb, dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                                 dd["bias_c"], y=y, counts=counts, ws=ws, stream=stream)
+            with torch.cuda.stream(stream):
+                fwd()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fwd()
+            graphs.append(g)
+        with torch.cuda.stream(stream):
+            for g in graphs:
+                flush.zero_()
+                g.replay()
+        n = max(steps, nbatch)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for j, (a, b) in enumerate(ev):
+                flush.zero_()
+                a.record(stream)
+                graphs[j % nbatch].replay()
+                b.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / n
+        del graphs, xs, ws
+        torch.cuda.empty_cache()
+        return {"ms_per_step": ms, "batches": nbatch, "steps": n,
+                "value": job_throughput(world, c.L, ms), "unit": "tokens/s"}
+
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
         # the shared dense MLP of the same batch, width F = d
@@ -830,10 +874,18 @@ def run_ours(args):
         extra["expert_shards"] = measure_shards(cfg, d, 3)
         extra["glu"] = measure_glu(cfg, d, max(3, args.steps // 2))
         extra["backward"] = measure_backward(cfg, d, max(3, args.steps // 2))
+        extra["rotating_x"] = measure_rotating_x(cfg, d, args.steps)
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
         extra[sc.name] = summary(sc, d2, max(args.steps, 20), max(args.warmup, 5), True)
+        # the decode batch through the public call with host buffers
+        es, ep, eh, eo = measure_e2e(sc, d2, max(args.steps, 20), max(args.warmup, 5))
+        extra[sc.name]["e2e"] = {"value": job_throughput(world, sc.L, ep), "unit": "tokens/s",
+                                 "ms_per_step": ep, "h2d_bytes_per_step": eh,
+                                 "d2h_bytes_per_step": eo,
+                                 "serial": {"value": job_throughput(world, sc.L, es),
+                                            "ms_per_step": es}}
         del d2
         # the other workloads (parity configurations), each with its own weights
         for sc in (WL.TINY, WL.BF16_16K, WL.SKEWED):
