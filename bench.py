@@ -879,13 +879,17 @@ def run_ours(args):
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
         extra[sc.name] = summary(sc, d2, max(args.steps, 20), max(args.warmup, 5), True)
-        # the decode batch through the public call with host buffers
+        # the decode batch through the public call with host buffers.  Its
+        # copies are 256 KiB each way, so one step at a time (the L2 flush
+        # outside the events) is the figure; the pipelined loop times its
+        # 256 MiB flush inside every step, which is most of a decode step
         es, ep, eh, eo = measure_e2e(sc, d2, max(args.steps, 20), max(args.warmup, 5))
-        extra[sc.name]["e2e"] = {"value": job_throughput(world, sc.L, ep), "unit": "tokens/s",
-                                 "ms_per_step": ep, "h2d_bytes_per_step": eh,
+        extra[sc.name]["e2e"] = {"value": job_throughput(world, sc.L, es), "unit": "tokens/s",
+                                 "ms_per_step": es, "h2d_bytes_per_step": eh,
                                  "d2h_bytes_per_step": eo,
-                                 "serial": {"value": job_throughput(world, sc.L, es),
-                                            "ms_per_step": es}}
+                                 "mode": "serial: copy in, forward, copy out on one stream",
+                                 "pipelined_with_flush": {"value": job_throughput(world, sc.L, ep),
+                                                          "ms_per_step": ep}}
         del d2
         # the other workloads (parity configurations), each with its own weights
         for sc in (WL.TINY, WL.BF16_16K, WL.SKEWED):
