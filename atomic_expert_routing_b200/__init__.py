@@ -27,7 +27,7 @@ from ._lib import (OMNI_BF16, OMNI_F32, OMNI_FLAG_DENSE_TENSOR_CORES, OMNI_FLAG_
 __all__ = ["LayerDims", "route", "router_logits", "route_select", "schedule", "expert_forward", "moe_forward",
            "token_centric_forward", "new_counts", "OmniError", "workspace_size", "wait_selftest",
            "shared_mlp", "moe_mlp_forward", "mlp_workspace_size", "expert_forward_noalloc",
-           "moe_forward_shard", "cast_output", "moe_backward"]
+           "moe_forward_shard", "moe_forward_shard_routed", "cast_output", "moe_backward"]
 
 
 @dataclass(frozen=True)
@@ -171,12 +171,17 @@ def new_counts(device) -> torch.Tensor:
 
 
 def route(D: LayerDims, x, Wr, Wc, bias_r=None, bias_c=None, *, counts=None, ws=None,
-          stream=None, with_score=True):
-    """Cartesian Product Router: (idx int32 [L,K], gate f32 [L,K], score f32 [L,K] or None)."""
+          stream=None, with_score=True, out=None):
+    """Cartesian Product Router: (idx int32 [L,K], gate f32 [L,K], score f32 [L,K] or None).
+    out (optional): (idx, gate) tensors to write."""
     _expect_io(D, x=x, Wr=Wr, Wc=Wc, bias_r=bias_r, bias_c=bias_c, counts=counts)
     dev = _device(x)
-    idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
-    gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
+    if out is not None:
+        idx, gate = out
+        _expect_io(D, idx=idx, gate=gate)
+    else:
+        idx = torch.empty((D.L, D.K), dtype=torch.int32, device=dev)
+        gate = torch.empty((D.L, D.K), dtype=torch.float32, device=dev)
     score = torch.empty((D.L, D.K), dtype=torch.float32, device=dev) if with_score else None
     wsp, n = _ws(D, OMNI_WS_ROUTE, dev, ws)
     dd = D.c()
@@ -334,6 +339,32 @@ def moe_forward_shard(D: LayerDims, x, Wr, Wc, W, V, e_lo: int, e_hi: int, bias_
         C.byref(dd), e_lo, e_hi, _ptr(x), _ptr(Wr), _ptr(Wc), _ptr(bias_r), _ptr(bias_c),
         _ptr(W), _ptr(U), _ptr(V), _ptr(y_part), _ptr(idx), _ptr(gate), _ptr(counts), wsp, n,
         _stream(stream)))
+    return y_part
+
+
+def moe_forward_shard_routed(D: LayerDims, x, W, V, e_lo: int, e_hi: int, idx, gate, *,
+                             U=None, y_part=None, counts=None, ws=None, stream=None):
+    """moe_forward_shard from a given routing (idx, gate [L, K] of all L
+    tokens), which is read and not computed.  Returns y_part [L, d] fp32."""
+    if not 0 <= e_lo < e_hi <= D.N:
+        raise ValueError(f"shard ids [{e_lo}, {e_hi}) outside [0, {D.N})")
+    rows = (e_hi - e_lo) * D.d
+    _expect_io(D, x=x, counts=counts)
+    _expect("idx", idx, D.M, torch.int32)
+    _expect("gate", gate, D.M, torch.float32)
+    for name, t in (("W", W), ("V", V), ("U", U)):
+        _expect(name, t, rows, D.torch_dtype, optional=name == "U")
+    _expect("y_part", y_part, D.L * D.d, torch.float32, optional=True)
+    dev = _device(x)
+    if y_part is None:
+        y_part = torch.empty((D.L, D.d), dtype=torch.float32, device=dev)
+    if counts is None:
+        counts = new_counts(dev)
+    wsp, n = _ws(D, OMNI_WS_FUSED, dev, ws)
+    dd = D.c()
+    _lib.check("omni_moe_forward_shard_routed", _lib.load().omni_moe_forward_shard_routed(
+        C.byref(dd), e_lo, e_hi, _ptr(x), _ptr(W), _ptr(U), _ptr(V), _ptr(idx), _ptr(gate),
+        _ptr(y_part), _ptr(counts), wsp, n, _stream(stream)))
     return y_part
 
 

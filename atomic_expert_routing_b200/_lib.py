@@ -51,6 +51,7 @@ SIGNATURES = {
     "omni_token_centric_forward_glu": ([_P] * 10 + [C.c_size_t, _P], C.c_int),
     "omni_moe_forward_shard": ([_P, _I64, _I64] + [_P] * 13 + [C.c_size_t, _P], C.c_int),
     "omni_cast_output": ([_P] * 4, C.c_int),
+    "omni_moe_forward_shard_routed": ([_P, _I64, _I64] + [_P] * 9 + [C.c_size_t, _P], C.c_int),
     "omni_moe_backward": ([_P] * 16 + [C.c_int, _P, _P, C.c_size_t, _P], C.c_int),
     "omni_wait_selftest": ([_P, _P], C.c_int),
     "omni_shared_mlp": ([_P, _I64, _P, _P, _P, _P, C.c_int, _P, _P, C.c_size_t, _P], C.c_int),

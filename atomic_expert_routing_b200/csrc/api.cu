@@ -340,10 +340,12 @@ int omni_expert_forward_glu(const omni_dims* dims, const void* x, const void* W,
 namespace {
 
 // The fused routed branch; dims, pointers and workspace already checked.
+// routed: idx_out / gate_out hold the batch's routing already (the route is
+// skipped and they are only read).
 int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* Wc,
                      const float* bias_r, const float* bias_c, const void* W, const void* V,
                      void* y, int32_t* idx_out, float* gate_out, int32_t* counts, void* ws,
-                     cudaStream_t s, const void* U = nullptr) {
+                     cudaStream_t s, const void* U = nullptr, bool routed = false) {
   int rc = OMNI_OK;
   Carver c(ws);
   FusedWs w = carve_fused(D, c);
@@ -361,7 +363,7 @@ int moe_forward_impl(const Dims& D, const void* x, const void* Wr, const void* W
   const int64_t zero_words =
       tail ? static_cast<int64_t>(omni::sched_exec_zero_words(D)) : acc_words;
   bool acc_zeroed = false;
-  {
+  if (!routed) {
     omni::CallRange stage("route");
     rc = route_impl(D, x, Wr, Wc, bias_r, bias_c, idx, gate, nullptr, counts + 2, w.route.Z, s,
                     zero, zero_words, &acc_zeroed);
@@ -595,6 +597,26 @@ int omni_moe_backward(const omni_dims* dims, const void* x, const void* Wr, cons
   return cuda_status(omni::launch_backward(D, x, Wr, Wc, W, V, idx, gate, dy, dx, dW, dV, dWr,
                                            dWc, dbias_r, dbias_c, accumulate != 0, counts, ws,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int omni_moe_forward_shard_routed(const omni_dims* dims, int64_t e_lo, int64_t e_hi,
+                                  const void* x, const void* W, const void* U, const void* V,
+                                  const int32_t* idx, const float* gate, float* y_part,
+                                  int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  omni::CallRange range("omni_moe_forward_shard_routed");
+  Dims D;
+  int rc = check_dims(dims, &D);
+  if (rc != OMNI_OK) return rc;
+  if (e_lo < 0 || e_hi <= e_lo || e_hi > D.N() || counts == nullptr) return OMNI_ERR_INVALID_ARG;
+  if (D.L == 0) return OMNI_OK;
+  const void* t16[] = {x, W, V, y_part, U != nullptr ? U : x};
+  if (!tensors_ok(t16, 5) || idx == nullptr || gate == nullptr) return OMNI_ERR_INVALID_ARG;
+  if ((rc = ws_ok(D, OMNI_WS_FUSED, ws, ws_bytes)) != OMNI_OK) return rc;
+  D.e_lo = e_lo;
+  D.e_hi = e_hi;
+  return moe_forward_impl(D, x, nullptr, nullptr, nullptr, nullptr, W, V, y_part,
+                          const_cast<int32_t*>(idx), const_cast<float*>(gate), counts, ws,
+                          static_cast<cudaStream_t>(stream), U, true);
 }
 
 }  // extern "C"

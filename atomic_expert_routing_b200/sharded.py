@@ -22,7 +22,7 @@ import contextlib
 
 import torch
 
-from . import LayerDims, cast_output, moe_forward_shard
+from . import LayerDims, cast_output, moe_forward_shard, moe_forward_shard_routed, route
 
 
 def shard_ranges(N: int, G: int) -> list[tuple[int, int]]:
@@ -37,6 +37,35 @@ def shard_ranges(N: int, G: int) -> list[tuple[int, int]]:
         out.append((lo, hi))
         lo = hi
     return out
+
+
+def token_ranges(L: int, G: int) -> list[tuple[int, int]]:
+    """Process g routes tokens [g*T, min((g+1)*T, L)), T = ceil(L / G)
+    (the last ranges may be short or empty)."""
+    if G < 1:
+        raise ValueError("a group has at least one process")
+    T = -(-L // G)
+    return [(min(g * T, L), min((g + 1) * T, L)) for g in range(G)]
+
+
+def gather_routing(idx_part: torch.Tensor, gate_part: torch.Tensor, L: int, group=None):
+    """The whole batch's routing from every process's share (token_ranges):
+    one all-gather of the ids and one of the gates, each share padded to
+    ceil(L / G) rows.  Returns (idx [L, K], gate [L, K])."""
+    import torch.distributed as dist
+    G = dist.get_world_size(group) if dist.is_initialized() else 1
+    if G == 1:
+        return idx_part, gate_part
+    K = idx_part.shape[1]
+    T = -(-L // G)
+    outs = []
+    for part in (idx_part, gate_part):
+        padded = torch.zeros((T, K), dtype=part.dtype, device=part.device)
+        padded[: part.shape[0]] = part
+        full = torch.empty((G * T, K), dtype=part.dtype, device=part.device)
+        dist.all_gather_into_tensor(full, padded, group=group)
+        outs.append(full[:L].contiguous())
+    return outs[0], outs[1]
 
 
 def combine(y_part: torch.Tensor, group=None) -> torch.Tensor:
@@ -59,5 +88,35 @@ def forward(D: LayerDims, x, Wr, Wc, W_shard, V_shard, e_lo: int, e_hi: int, bia
                                ws=ws, stream=stream)
     # the collective is ordered after the shard's kernels on their stream
     with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+        combine(y_part, group)
+    return cast_output(D, y_part, y=y, stream=stream)
+
+
+def forward_split_routing(D: LayerDims, x, Wr, Wc, W_shard, V_shard, e_lo: int, e_hi: int,
+                          bias_r=None, bias_c=None, *, U_shard=None, group=None, y=None,
+                          y_part=None, counts=None, ws=None, stream=None):
+    """forward() with the routing split as well: process g routes only its
+    tokens (token_ranges), the shares are all-gathered, and each process
+    then schedules and executes its experts from the whole routing.  The
+    route is computed once per token in the group instead of once per
+    process."""
+    import torch.distributed as dist
+    G = dist.get_world_size(group) if dist.is_initialized() else 1
+    g = dist.get_rank(group) if dist.is_initialized() else 0
+    t0, t1 = token_ranges(D.L, G)[g]
+    Dg = LayerDims(t1 - t0, D.d, D.Nr, D.Nc, D.k, D.K, D.B, D.dtype, D.flags)
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    if t1 > t0:
+        idx_part, gate_part, _ = route(Dg, x[t0:t1], Wr, Wc, bias_r, bias_c, with_score=False,
+                                       stream=stream)
+    else:
+        idx_part = torch.empty((0, D.K), dtype=torch.int32, device=x.device)
+        gate_part = torch.empty((0, D.K), dtype=torch.float32, device=x.device)
+    with ctx:
+        idx, gate = gather_routing(idx_part, gate_part, D.L, group)
+    y_part = moe_forward_shard_routed(D, x, W_shard, V_shard, e_lo, e_hi, idx, gate,
+                                      U=U_shard, y_part=y_part, counts=counts, ws=ws,
+                                      stream=stream)
+    with ctx:
         combine(y_part, group)
     return cast_output(D, y_part, y=y, stream=stream)

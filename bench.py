@@ -768,10 +768,18 @@ def run_ours(args):
         the measured 8-GPU all-reduce bus bandwidth, 725 GB/s."""
         D = omni.LayerDims.of(c)
         out = {"workload": c.name, "allreduce_busbw_gbs": 725.0,
-               "note": "per-shard times measured; the all-reduce time is an estimate"}
+               "note": "per-shard times measured; the all-reduce and all-gather times are "
+                       "estimates; split_routing: each process routes L/G tokens and the "
+                       "routing is all-gathered (sharded.forward_split_routing)"}
         part_bytes = c.L * c.d * 4
+        # the batch's routing, for the shards that take it as input
+        r_idx = torch.empty((c.L, c.K), dtype=torch.int32, device=device)
+        r_gate = torch.empty((c.L, c.K), dtype=torch.float32, device=device)
+        omni.moe_forward(D, dd["x"], dd["Wr"], dd["Wc"], dd["W"], dd["V"], dd["bias_r"],
+                         dd["bias_c"], idx=r_idx, gate=r_gate)
         for G in (2, 4, 8):
-            shard_ms, active = [], []
+            shard_ms, active, split_ms = [], [], []
+            tok = omni_sharded.token_ranges(c.L, G)
             for lo, hi in omni_sharded.shard_ranges(c.N, G):
                 ws = omni.Workspace()
                 counts = omni.new_counts(device)
@@ -787,11 +795,36 @@ def run_ours(args):
 
                 shard_ms.append(timed_graph(fwd, steps))
                 active.append(int(counts[0].item()))
-                del ws, yp, y
+                # split routing: this process's L/G tokens routed, then its
+                # experts executed from the whole routing
+                g = len(split_ms)
+                t0, t1 = tok[g]
+                Dg = omni.LayerDims(t1 - t0, c.d, c.Nr, c.Nc, c.k, c.K, c.B, c.dtype, 0)
+                ws_r = omni.Workspace()
+                xg = dd["x"][t0:t1]
+                i_g = torch.empty((t1 - t0, c.K), dtype=torch.int32, device=device)
+                g_g = torch.empty((t1 - t0, c.K), dtype=torch.float32, device=device)
+                c_g = omni.new_counts(device)
+
+                def fwd_split(stream):
+                    if t1 > t0:
+                        omni.route(Dg, xg, dd["Wr"], dd["Wc"], dd["bias_r"], dd["bias_c"],
+                                   counts=c_g, ws=ws_r, stream=stream, with_score=False,
+                                   out=(i_g, g_g))
+                    omni.moe_forward_shard_routed(D, dd["x"], Wl, Vl, lo, hi, r_idx, r_gate,
+                                                  y_part=yp, counts=counts, ws=ws, stream=stream)
+                    omni.cast_output(D, yp, y=y, stream=stream)
+
+                split_ms.append(timed_graph(fwd_split, steps))
+                del ws, yp, y, ws_r
             ar = part_bytes * 2 * (G - 1) / G / (725.0e9) * 1e3
+            ag = c.L * c.K * 8 * (G - 1) / G / (725.0e9) * 1e3
             out[str(G)] = {"shard_ms": shard_ms, "max_shard_ms": max(shard_ms),
                            "active_per_shard": active, "allreduce_ms_estimate": ar,
                            "step_ms_estimate": max(shard_ms) + ar,
+                           "split_routing_shard_ms": split_ms,
+                           "allgather_ms_estimate": ag,
+                           "split_routing_step_ms_estimate": max(split_ms) + ag + ar,
                            "expert_bytes_per_gpu": 2 * c.d * max(active) * c.esize}
         torch.cuda.empty_cache()
         return out

@@ -352,6 +352,20 @@ int omni_moe_forward_shard(const omni_dims* dims, int64_t e_lo, int64_t e_hi, co
                            void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * omni_moe_forward_shard from a routing computed elsewhere: idx, gate [L x K]
+ * (as omni_route writes them, for all L tokens) are read, not computed, so
+ * that the processes of a group can each route a share of the tokens and
+ * exchange the routing instead of every process routing the whole batch.
+ * The other arguments and the results are those of omni_moe_forward_shard;
+ * the dims checks are those of omni_schedule (k is not used).  Ids outside
+ * [0, N) set OMNI_DEV_BAD_INDEX in counts[2].
+ */
+int omni_moe_forward_shard_routed(const omni_dims* dims, int64_t e_lo, int64_t e_hi,
+                                  const void* x, const void* W, const void* U, const void* V,
+                                  const int32_t* idx, const float* gate, float* y_part,
+                                  int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * y [L x d] in the storage type of dims <- src [L x d] fp32 (bf16: rounded
  * to nearest even; fp32: copied unless src == y).  The last step of a
  * sharded forward, after the partial sums are added.  src == y with bf16

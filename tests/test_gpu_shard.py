@@ -62,21 +62,32 @@ def _unsharded(cfg, d, U=None):
     return y, idx.cpu().numpy(), gate.cpu().numpy()
 
 
-def _run_shards(cfg, h, d, G, gated=False, flags=0):
-    """Every shard of the G-way split in turn; returns the summed partials."""
+def _run_shards(cfg, h, d, G, gated=False, flags=0, routed=False):
+    """Every shard of the G-way split in turn; returns the summed partials.
+    routed: the shards take the unsharded call's routing as input
+    (omni_moe_forward_shard_routed) instead of routing the batch."""
     D = omni.LayerDims.of(cfg, flags=flags)
     U = d.get("U") if gated else None
     y_full, i_ref, g_ref = _unsharded(cfg, d, U)
+    i_dev, g_dev = torch.from_numpy(i_ref).cuda(), torch.from_numpy(g_ref).cuda()
     total = torch.zeros((cfg.L, cfg.d), dtype=torch.float32, device="cuda")
     active = np.unique(i_ref)
     for lo, hi in sharded.shard_ranges(cfg.N, G):
         idx = torch.empty((cfg.L, cfg.K), dtype=torch.int32, device="cuda")
         gate = torch.empty((cfg.L, cfg.K), dtype=torch.float32, device="cuda")
         counts = omni.new_counts("cuda")
-        yp = omni.moe_forward_shard(D, d["x"], d["Wr"], d["Wc"], d["W"][lo:hi], d["V"][lo:hi],
-                                    lo, hi, d["bias_r"], d["bias_c"],
-                                    U=U[lo:hi] if U is not None else None, counts=counts,
-                                    idx=idx, gate=gate)
+        if routed:
+            yp = omni.moe_forward_shard_routed(D, d["x"], d["W"][lo:hi], d["V"][lo:hi], lo, hi,
+                                               i_dev, g_dev,
+                                               U=U[lo:hi] if U is not None else None,
+                                               counts=counts)
+            idx.copy_(i_dev)
+            gate.copy_(g_dev)
+        else:
+            yp = omni.moe_forward_shard(D, d["x"], d["Wr"], d["Wc"], d["W"][lo:hi],
+                                        d["V"][lo:hi], lo, hi, d["bias_r"], d["bias_c"],
+                                        U=U[lo:hi] if U is not None else None, counts=counts,
+                                        idx=idx, gate=gate)
         torch.cuda.synchronize()
         gi, gg, c = idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy()
         assert np.array_equal(gi, i_ref) and np.array_equal(gg, g_ref)
@@ -115,6 +126,16 @@ def test_shards_on_the_scheduled_paths(cfg):
     _run_shards(cfg, h, d, 3, flags=omni.OMNI_FLAG_STAGED_SMALL)
 
 
+@pytest.mark.parametrize("flags", [0, omni.OMNI_FLAG_STAGED_SMALL], ids=["default", "scheduled"])
+@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: c.name)
+def test_shards_from_a_given_routing(cfg, flags):
+    """omni_moe_forward_shard_routed: the shards take the batch's routing as
+    input (as the processes of a group do after exchanging their shares of
+    it) and give the same partials."""
+    h, d = _inputs(cfg)
+    _run_shards(cfg, h, d, 3, flags=flags, routed=True)
+
+
 @pytest.mark.parametrize("cfg", [CONFIGS[0], CONFIGS[2], CONFIGS[4]], ids=lambda c: c.name)
 def test_gated_shards(cfg):
     h, d = _inputs(cfg, gated=True)
@@ -146,10 +167,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_sharded_forward_over_a_one_process_nccl_group():
-    """sharded.forward end to end, its all-reduce on NCCL, in a group of one
-    process holding every id: y as the unsharded forward's, within the
-    storage bar of the oracle."""
+@pytest.mark.parametrize("split_routing", [False, True], ids=["replicated", "split-routing"])
+def test_sharded_forward_over_a_one_process_nccl_group(split_routing):
+    """sharded.forward (and forward_split_routing, whose all-gathers are then
+    trivial) end to end, the all-reduce on NCCL, in a group of one process
+    holding every id: y as the unsharded forward's, within the storage bar
+    of the oracle."""
     import torch.distributed as dist
     cfg = CONFIGS[2]
     h, d = _inputs(cfg)
@@ -160,8 +183,8 @@ def test_sharded_forward_over_a_one_process_nccl_group():
                             device_id=torch.device("cuda", torch.cuda.current_device()))
     try:
         D = omni.LayerDims.of(cfg)
-        y = sharded.forward(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], 0, cfg.N,
-                            d["bias_r"], d["bias_c"])
+        fwd = sharded.forward_split_routing if split_routing else sharded.forward
+        y = fwd(D, d["x"], d["Wr"], d["Wc"], d["W"], d["V"], 0, cfg.N, d["bias_r"], d["bias_c"])
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

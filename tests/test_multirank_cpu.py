@@ -127,3 +127,48 @@ def test_shard_ranges_partition_the_ids():
     for N, G in ((3, 4), (5, 0)):
         with pytest.raises(ValueError):
             sharded.shard_ranges(N, G)
+
+
+def _gather_main(rank, world, port, L, K, out_dir):
+    """Each rank holds the routing of its token_ranges share (ids and gates
+    that encode the token and slot); gather_routing assembles the batch."""
+    import torch
+    from atomic_expert_routing_b200 import sharded
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        t0, t1 = sharded.token_ranges(L, world)[rank]
+        tok = torch.arange(t0, t1, dtype=torch.int32)[:, None]
+        slot = torch.arange(K, dtype=torch.int32)[None, :]
+        idx = (tok * 1000 + slot).contiguous()
+        gate = (tok.float() + slot.float() / 100.0).contiguous()
+        gi, gg = sharded.gather_routing(idx, gate, L)
+        np.save(os.path.join(out_dir, f"gi{rank}.npy"), gi.numpy())
+        np.save(os.path.join(out_dir, f"gg{rank}.npy"), gg.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+@pytest.mark.parametrize("world,L", [(2, 10), (3, 7), (3, 2)])
+def test_routing_shares_gather_to_the_batch(tmp_path, world, L):
+    K = 4
+    mp.spawn(_gather_main, args=(world, _free_port(), L, K, str(tmp_path)), nprocs=world,
+             join=True)
+    want_i = np.arange(L)[:, None] * 1000 + np.arange(K)[None, :]
+    want_g = (np.arange(L)[:, None] + np.arange(K)[None, :] / 100.0).astype(np.float32)
+    for r in range(world):
+        np.testing.assert_array_equal(np.load(tmp_path / f"gi{r}.npy"), want_i)
+        np.testing.assert_array_equal(np.load(tmp_path / f"gg{r}.npy"), want_g)
+
+
+def test_token_ranges_cover_the_batch():
+    from atomic_expert_routing_b200 import sharded
+    for L, G in ((10, 3), (7, 7), (2, 3), (0, 2), (16384, 8)):
+        r = sharded.token_ranges(L, G)
+        assert len(r) == G and r[0][0] == 0 and r[-1][1] == L
+        assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
