@@ -42,6 +42,12 @@ HOT = {
     "omni::(anonymous namespace)::k_task_act<__nv_bfloat16, 8, true>": 0,
     "omni::(anonymous namespace)::k_act<__nv_bfloat16, 8, 3, true, true>": 0,
     "omni::(anonymous namespace)::k_expert_async<__nv_bfloat16, 8, 2, true>": 0,
+    # backward
+    "omni::(anonymous namespace)::k_bwd_expert": 0,
+    "omni::(anonymous namespace)::k_bwd_token": 0,
+    "omni::(anonymous namespace)::k_transpose16": 0,
+    # shards
+    "omni::(anonymous namespace)::k_shard_range": 0,
 }
 
 
