@@ -901,13 +901,17 @@ def run_ours(args):
 
     extra = {}
     if args.workload == PRIMARY.name and not args.no_secondary:
-        # the shared dense MLP of the same batch, width F = d
-        extra["shared_mlp"] = measure_mlp(cfg, d, cfg.d, max(3, args.steps // 2))
-        extra["dense_groups"] = measure_dense_paths(max(3, args.steps // 2))
-        extra["expert_shards"] = measure_shards(cfg, d, 3)
-        extra["glu"] = measure_glu(cfg, d, max(3, args.steps // 2))
-        extra["backward"] = measure_backward(cfg, d, max(3, args.steps // 2))
-        extra["rotating_x"] = measure_rotating_x(cfg, d, args.steps)
+        if world == 1:
+            # single-process extras (each rank of a group would repeat them):
+            # the shared dense MLP of the same batch (width F = d), the
+            # tensor-core dense groups, expert shards, gated experts, the
+            # backward and the rotating-batch check
+            extra["shared_mlp"] = measure_mlp(cfg, d, cfg.d, max(3, args.steps // 2))
+            extra["dense_groups"] = measure_dense_paths(max(3, args.steps // 2))
+            extra["expert_shards"] = measure_shards(cfg, d, 3)
+            extra["glu"] = measure_glu(cfg, d, max(3, args.steps // 2))
+            extra["backward"] = measure_backward(cfg, d, max(3, args.steps // 2))
+            extra["rotating_x"] = measure_rotating_x(cfg, d, args.steps)
         sc = SECONDARY
         host2 = rank_inputs(sc, rank)
         d2 = dict(d, x=to_dev(host2["x"]), bias_r=None, bias_c=None)
