@@ -19,12 +19,15 @@
 //  2. k_bwd_expert: a warp per expert reads its W and V rows, computes every
 //     task's scalars (a, s, da, dgate), writes da and dgate to the task's
 //     slot t*K + k, and adds its row gradients dW[e], dV[e] (fp32) once per
-//     32 tasks -- no atomics, an expert belongs to one warp;
+//     32 tasks -- no atomics, an expert belongs to one warp.  A call that
+//     does not accumulate writes the rows with the first 32 tasks instead of
+//     adding to them, without reading them;
 //  3. k_bwd_token: a CTA per token forms dS, its dZ row (bf16, the GEMM
 //     operand; fp32 atomics into the bias gradients) and dx[t] = sum_k da_k
 //     W[e_k] (fp32);
 //  4. transposes to K-major bf16 operands, then two tcgen05 GEMMs with fp32
-//     accumulation: dx += dZ [Wr; Wc] and [dWr; dWc] += dZ^T x.
+//     accumulation: dx += dZ [Wr; Wc] and [dWr; dWc] += dZ^T x (= when the
+//     call does not accumulate; the bias gradients are then cleared first).
 // bf16 storage only (the GEMM operands; dZ is rounded to bf16 for them).
 #include "common.cuh"
 #include "gemm_tc.cuh"
