@@ -30,6 +30,13 @@ CONFIGS = [
               dtype=WL.BF16, seed=94),
     WL.Config("bwd-skewed", L=512, d=256, Nr=32, Nc=32, k=8, K=8, B=32, dtype=WL.BF16, seed=95,
               zipf_s=1.1),
+    # edges: one expert per token (the gate is 1, the router gets nothing);
+    # the largest top-K (256 ids per token to search for each task's slot);
+    # a single token
+    WL.Config("bwd-k1", L=200, d=128, Nr=32, Nc=64, k=1, K=1, B=5, dtype=WL.BF16, seed=96),
+    WL.Config("bwd-max-topk", L=64, d=64, Nr=4096, Nc=256, k=256, K=256, B=64, dtype=WL.BF16,
+              seed=97),
+    WL.Config("bwd-one-token", L=1, d=256, Nr=16, Nc=16, k=4, K=4, B=3, dtype=WL.BF16, seed=98),
 ]
 TOL = {"dW": 1e-4, "dV": 1e-4, "dbias_r": 1e-3, "dbias_c": 1e-3, "dx": 2e-2, "dWr": 2e-2,
        "dWc": 2e-2}
@@ -67,6 +74,9 @@ def test_backward_matches_the_oracle(cfg):
     assert c[0] == len(np.unique(gi))
     for key, tol in TOL.items():
         got = g[key].cpu().numpy().astype(np.float64)
+        if not np.abs(ref[key]).max() > 0:  # K = 1: the router gets nothing
+            assert np.abs(got).max() <= 1e-6, key
+            continue
         err = rel_err(got, ref[key])
         assert err <= tol, (key, err)
     idle = np.setdiff1d(np.arange(cfg.N), gi)
