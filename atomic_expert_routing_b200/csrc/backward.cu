@@ -41,6 +41,7 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kBwdWarps = 8;
 constexpr int kTokThreadsB = 256;
+static_assert(kTokThreadsB >= OMNI_MAX_TOPK, "k_bwd_token: a thread per task of a token");
 
 __device__ __forceinline__ float silu_grad(float z) {
   const float sg = 1.0f / (1.0f + expf(-z));
